@@ -1,0 +1,254 @@
+/*
+ * moe_oracle.c -- the CPU oracle of the fused MoE FFN layer forward.
+ *
+ * TEST INFRASTRUCTURE ONLY. The tests, the smoke check and the benchmark's CPU-baseline leg
+ * are the only code that may load this library; the product path (the CUDA library and its
+ * Python binding) never links, imports or calls it, and shares no code with it.
+ *
+ * Plain, slow and direct: every floating-point step is carried out in IEEE double on inputs
+ * that are bf16 values (passed as their raw 16-bit patterns and widened exactly). No step is
+ * blocked, fused or reordered beyond what the definitions below state. The only parallelism
+ * is an OpenMP loop over independent tokens.
+ *
+ * Sources (page title, then the section or figure):
+ *  - Layer equation and SwiGLU: Mixture-of-Kittens blog, section "Overlapping compute and
+ *    communication in MoE":  x' = W_shared(x) + sum_{e in top-k} w_e W_down^e SwiGLU(W_up^e x,
+ *    W_gate^e x),  SwiGLU(u, g) = SiLU(u) (.) g  -- SiLU sits on the *up* projection.
+ *  - Router projection and top-k: Weave blog, section 1.1 (a router picks top-k experts per
+ *    token); vLLM MoE execution analysis, table "Per-decode-step kernel launches"
+ *    (topk_softmax); FlashMoE review, "core formulas" (gate affinities G_phi).
+ *  - Align: vLLM PR #53280 summary, "implementation breakdown" items 1-2 and the reviewer's
+ *    all-blocks alternative (per-expert counts, exclusive cumsum, token ids written into
+ *    per-expert segments padded to a multiple of the block size, one block id per block);
+ *    vLLM MoE execution analysis, moe_align_block_size and BLOCK_SIZE_M.
+ *  - Capacity: FlashMoE review, "core formulas" (routing table T_phi with capacity C per
+ *    expert) and the FlashMoE experimental setup (capacity factor 1.0).
+ *
+ * Readings taken where the pages are silent (each is listed in the design notes):
+ *  - top-k ties: the lower expert index wins; selection compares logits, not rounded
+ *    probabilities.
+ *  - gating weights: softmax over all E experts, then the k selected probabilities are
+ *    renormalised to sum to 1.
+ *  - align order inside an expert segment: ascending slot id s = t*k + j (stable).
+ *  - padding sentinel: S = T*k; unused expert_ids entries: -1.
+ *  - capacity C = ceil(cf * S / E); a slot whose stable rank inside its expert is >= C is
+ *    dropped (contributes nothing) and the other weights are not renormalised again.
+ *  - a router bias, when given, is added to the logits before softmax and selection.
+ *  - the shared expert is an ungated SwiGLU FFN with weight 1.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_API __attribute__((visibility("default")))
+
+static double bf16_to_double(uint16_t b)
+{
+    uint32_t u = ((uint32_t)b) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* Router projection: logits[t][e] = sum_h x[t][h] * W_router[e][h] (+ bias[e]), summed in
+ * ascending h.  absdot[t][e] = sum_h |x[t][h] * W_router[e][h]| (nullable): the quantity
+ * that bounds the rounding error of any fp32 evaluation of the same dot product. */
+ORACLE_API void moe_oracle_router_logits(const uint16_t *x, const uint16_t *w_router,
+                                         const float *bias, int64_t T, int64_t H, int64_t E,
+                                         double *logits, double *absdot)
+{
+    double *wr = (double *)malloc(sizeof(double) * (size_t)(E * H));
+    for (int64_t i = 0; i < E * H; ++i) wr[i] = bf16_to_double(w_router[i]);
+#pragma omp parallel
+    {
+        double *xt = (double *)malloc(sizeof(double) * (size_t)H);
+#pragma omp for schedule(static)
+        for (int64_t t = 0; t < T; ++t) {
+            for (int64_t h = 0; h < H; ++h) xt[h] = bf16_to_double(x[t * H + h]);
+            for (int64_t e = 0; e < E; ++e) {
+                const double *w = wr + e * H;
+                double s = 0.0, a = 0.0;
+                for (int64_t h = 0; h < H; ++h) {
+                    s += xt[h] * w[h];
+                    a += fabs(xt[h] * w[h]);
+                }
+                if (bias) s += (double)bias[e];
+                logits[t * E + e] = s;
+                if (absdot) absdot[t * E + e] = a;
+            }
+        }
+        free(xt);
+    }
+    free(wr);
+}
+
+/* Top-k selection and renormalised softmax for each token.
+ * Selection: k rounds, each taking the largest remaining logit (ties to the lower index).
+ * Weights: p = softmax(logits[t]) over all E experts; w_j = p_{ids_j} / sum_i p_{ids_i}.
+ * ids are written in selection order (descending logit). */
+ORACLE_API void moe_oracle_topk_softmax(const double *logits, int64_t T, int64_t E, int64_t k,
+                                        int32_t *topk_ids, double *topk_w)
+{
+#pragma omp parallel
+    {
+        unsigned char *taken = (unsigned char *)malloc((size_t)E);
+        double *p = (double *)malloc(sizeof(double) * (size_t)E);
+#pragma omp for schedule(static)
+        for (int64_t t = 0; t < T; ++t) {
+            const double *v = logits + t * E;
+            memset(taken, 0, (size_t)E);
+            for (int64_t j = 0; j < k; ++j) {
+                int64_t best = -1;
+                for (int64_t e = 0; e < E; ++e) {
+                    if (taken[e]) continue;
+                    if (best < 0 || v[e] > v[best]) best = e; /* equal value: keep lower index */
+                }
+                taken[best] = 1;
+                topk_ids[t * k + j] = (int32_t)best;
+            }
+            /* softmax over all experts (shifted by the max for range, which cancels) */
+            double m = v[0];
+            for (int64_t e = 1; e < E; ++e) if (v[e] > m) m = v[e];
+            double z = 0.0;
+            for (int64_t e = 0; e < E; ++e) { p[e] = exp(v[e] - m); z += p[e]; }
+            for (int64_t e = 0; e < E; ++e) p[e] /= z;
+            double s = 0.0;
+            for (int64_t j = 0; j < k; ++j) s += p[topk_ids[t * k + j]];
+            for (int64_t j = 0; j < k; ++j) topk_w[t * k + j] = p[topk_ids[t * k + j]] / s;
+        }
+        free(p);
+        free(taken);
+    }
+}
+
+/* Align (moe_align_block_size semantics).
+ * Inputs: topk_ids [T*k] (slot s = t*k + j), E experts, block size block_m, capacity
+ * (<= 0 means dropless).
+ * Outputs:
+ *   kept[s]          1 if slot s survives the capacity limit
+ *   sorted_ids[i]    slot ids grouped by expert in ascending slot order, each expert's
+ *                    segment padded with the sentinel S up to a multiple of block_m; every
+ *                    entry from P to sorted_len-1 is the sentinel too
+ *   expert_ids[b]    expert owning block b (b < P/block_m); -1 for b >= P/block_m
+ *   *num_post_padded P = sum_e ceil(kept_e / block_m) * block_m
+ * Returns P, or -1 if sorted_len or blocks_len is too small. */
+ORACLE_API int64_t moe_oracle_align(const int32_t *topk_ids, int64_t T, int64_t k, int64_t E,
+                                    int64_t block_m, int64_t capacity, int32_t *sorted_ids,
+                                    int64_t sorted_len, int32_t *expert_ids, int64_t blocks_len,
+                                    int32_t *num_post_padded, uint8_t *kept)
+{
+    const int64_t S = T * k;
+    int64_t *count = (int64_t *)calloc((size_t)E, sizeof(int64_t));
+    int64_t *kept_n = (int64_t *)calloc((size_t)E, sizeof(int64_t));
+    int64_t *offset = (int64_t *)calloc((size_t)E + 1, sizeof(int64_t));
+    int64_t *fill = (int64_t *)calloc((size_t)E, sizeof(int64_t));
+
+    /* per-expert histogram, with the capacity decision taken by stable rank */
+    for (int64_t s = 0; s < S; ++s) {
+        int64_t e = topk_ids[s];
+        int64_t rank = count[e]++;
+        int keep = (capacity <= 0) || (rank < capacity);
+        kept[s] = (uint8_t)keep;
+        if (keep) kept_n[e]++;
+    }
+    /* exclusive scan of the padded segment lengths */
+    for (int64_t e = 0; e < E; ++e) {
+        int64_t padded = (kept_n[e] + block_m - 1) / block_m * block_m;
+        offset[e + 1] = offset[e] + padded;
+    }
+    const int64_t P = offset[E];
+    if (P > sorted_len || P / block_m > blocks_len) {
+        free(count); free(kept_n); free(offset); free(fill);
+        return -1;
+    }
+    for (int64_t i = 0; i < sorted_len; ++i) sorted_ids[i] = (int32_t)S;
+    for (int64_t s = 0; s < S; ++s) {
+        if (!kept[s]) continue;
+        int64_t e = topk_ids[s];
+        sorted_ids[offset[e] + fill[e]++] = (int32_t)s;
+    }
+    for (int64_t b = 0; b < blocks_len; ++b) expert_ids[b] = -1;
+    for (int64_t e = 0; e < E; ++e)
+        for (int64_t i = offset[e]; i < offset[e + 1]; i += block_m) expert_ids[i / block_m] = (int32_t)e;
+    *num_post_padded = (int32_t)P;
+    free(count); free(kept_n); free(offset); free(fill);
+    return P;
+}
+
+/* One expert FFN on one token: y = W_down . SwiGLU(W_up x, W_gate x), SiLU(u) = u/(1+e^-u).
+ * w_up, w_gate: [D][H]; w_down: [H][D]; a: scratch [D]. */
+static void expert_ffn(const double *x, const uint16_t *w_up, const uint16_t *w_gate,
+                       const uint16_t *w_down, int64_t H, int64_t D, double *a, double *y)
+{
+    for (int64_t d = 0; d < D; ++d) {
+        const uint16_t *ru = w_up + d * H, *rg = w_gate + d * H;
+        double u = 0.0, g = 0.0;
+        for (int64_t h = 0; h < H; ++h) {
+            u += bf16_to_double(ru[h]) * x[h];
+            g += bf16_to_double(rg[h]) * x[h];
+        }
+        a[d] = (u / (1.0 + exp(-u))) * g;
+    }
+    for (int64_t h = 0; h < H; ++h) {
+        const uint16_t *rd = w_down + h * D;
+        double s = 0.0;
+        for (int64_t d = 0; d < D; ++d) s += bf16_to_double(rd[d]) * a[d];
+        y[h] = s;
+    }
+}
+
+/* The layer output for a list of tokens:
+ *   out[i] = W_shared(x_t) + sum_{j: kept} w[t*k+j] * W_down^e SwiGLU(W_up^e x_t, W_gate^e x_t)
+ * with t = tokens[i], e = topk_ids[t*k+j]; the shared term first, then j ascending.
+ * W_up, W_gate: [E][D][H]; W_down: [E][H][D]; shared weights [Ds][H], [Ds][H], [H][Ds]
+ * (ignored when Ds == 0). out: [n_tokens][H]. */
+ORACLE_API void moe_oracle_layer(const uint16_t *x, int64_t T, int64_t H, int64_t D, int64_t E,
+                                 int64_t k, const int32_t *topk_ids, const double *topk_w,
+                                 const uint8_t *kept, const uint16_t *w_up,
+                                 const uint16_t *w_gate, const uint16_t *w_down, int64_t Ds,
+                                 const uint16_t *ws_up, const uint16_t *ws_gate,
+                                 const uint16_t *ws_down, const int64_t *tokens,
+                                 int64_t n_tokens, double *out)
+{
+    (void)T; (void)E;
+    const int64_t Dmax = Ds > D ? Ds : D;
+#pragma omp parallel
+    {
+        double *xt = (double *)malloc(sizeof(double) * (size_t)H);
+        double *a = (double *)malloc(sizeof(double) * (size_t)Dmax);
+        double *y = (double *)malloc(sizeof(double) * (size_t)H);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t i = 0; i < n_tokens; ++i) {
+            const int64_t t = tokens[i];
+            double *o = out + i * H;
+            for (int64_t h = 0; h < H; ++h) xt[h] = bf16_to_double(x[t * H + h]);
+            for (int64_t h = 0; h < H; ++h) o[h] = 0.0;
+            if (Ds > 0) {
+                expert_ffn(xt, ws_up, ws_gate, ws_down, H, Ds, a, y);
+                for (int64_t h = 0; h < H; ++h) o[h] += y[h];
+            }
+            for (int64_t j = 0; j < k; ++j) {
+                const int64_t s = t * k + j;
+                if (!kept[s]) continue;
+                const int64_t e = topk_ids[s];
+                expert_ffn(xt, w_up + e * D * H, w_gate + e * D * H, w_down + e * H * D, H, D, a, y);
+                for (int64_t h = 0; h < H; ++h) o[h] += topk_w[s] * y[h];
+            }
+        }
+        free(y);
+        free(a);
+        free(xt);
+    }
+}
+
+/* Threads the OpenMP loops above use (1 when built without OpenMP). */
+ORACLE_API int moe_oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    extern int omp_get_max_threads(void);
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

@@ -1,0 +1,71 @@
+"""Planted mistakes in the oracle must fail its pins.
+
+Each mutant is a copy of moe_oracle.c with one plausible mistake (a swapped operand, a
+dropped term, an off-by-one, a wrong tie rule ...), compiled on the CPU into a temporary
+library. The pins of test_oracle_pins.py run against it, and at least one must fail.
+"""
+import os
+import subprocess
+
+import pytest
+
+from oracle import oracle
+import test_oracle_pins as pins  # noqa: E402
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "moe_oracle.c")
+
+MUTANTS = {
+    "silu_on_gate": ("a[d] = (u / (1.0 + exp(-u))) * g;", "a[d] = (g / (1.0 + exp(-g))) * u;"),
+    "no_shared_term": ("for (int64_t h = 0; h < H; ++h) o[h] += y[h];",
+                       "for (int64_t h = 0; h < H; ++h) o[h] += 0.0 * y[h];"),
+    "unweighted_combine": ("o[h] += topk_w[s] * y[h];", "o[h] += y[h];"),
+    "tie_to_higher_index": ("v[e] > v[best]) best = e;", "v[e] >= v[best]) best = e;"),
+    "no_renormalise": ("topk_w[t * k + j] = p[topk_ids[t * k + j]] / s;",
+                       "topk_w[t * k + j] = p[topk_ids[t * k + j]];"),
+    "capacity_off_by_one": ("(rank < capacity)", "(rank <= capacity)"),
+    "bias_sign": ("if (bias) s += (double)bias[e];", "if (bias) s -= (double)bias[e];"),
+    "down_transposed": ("s += bf16_to_double(rd[d]) * a[d];",
+                        "s += bf16_to_double(w_down[d * H + h]) * a[d];"),
+    "segment_not_padded": ("int64_t padded = (kept_n[e] + block_m - 1) / block_m * block_m;",
+                           "int64_t padded = kept_n[e];"),
+    "unstable_segment_order": ("sorted_ids[offset[e] + fill[e]++] = (int32_t)s;",
+                               "sorted_ids[offset[e] + kept_n[e] - 1 - fill[e]++] = (int32_t)s;"),
+    "router_row_index": ("const double *w = wr + e * H;", "const double *w = wr + (E - 1 - e) * H;"),
+}
+
+PIN_TESTS = [
+    lambda: pins.test_hand_worked_golden("hand_worked_layer.json"),
+    lambda: pins.test_hand_worked_golden("hand_worked_capacity.json"),
+    lambda: pins.test_router_logits_match_matmul(),
+    lambda: pins.test_topk_softmax_matches_sort_definition(64, 2, True),
+    lambda: pins.test_topk_exact_ties_prefer_lower_index(),
+    lambda: pins.test_align_matches_argsort_definition("random", 48, 1.0),
+    lambda: pins.test_capacity_keeps_first_slots_in_token_order(),
+    lambda: pins.test_brute_force_tiny_workload(),
+    lambda: pins.test_brute_force_with_capacity_and_shared(),
+    lambda: pins.test_brute_force_with_bias(),
+    lambda: pins.test_top_k_equals_E_is_dense_softmax_mixture(),
+]
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_mistake_fails_a_pin(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation anchor not unique: {old}"
+    mut = tmp_path / "mut.c"
+    mut.write_text(src.replace(old, new))
+    so = tmp_path / "libmut.so"
+    subprocess.check_call(["gcc", "-O1", "-std=c99", "-fPIC", "-shared", "-fopenmp", str(mut),
+                           "-o", str(so), "-lm"])
+    failed = 0
+    oracle.use_library(str(so))
+    try:
+        for pin in PIN_TESTS:
+            try:
+                pin()
+            except AssertionError:
+                failed += 1
+    finally:
+        oracle.use_library(None)
+    assert failed > 0, f"mutant {name} passed every pin"
