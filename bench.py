@@ -1,0 +1,343 @@
+"""Benchmark of the fused MoE layer forward on B200: MoE-layer tokens/s and TFLOP/s, with the
+dominant kernel's fraction of the HBM (or tensor) roofline.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mine|reference]
+                  [--workload flashmoe_prefill] [--no-cpu-baseline] [--e2e-steps M]
+
+One step = one whole layer forward (router projection, gating, align, expert GEMMs with the
+fused SwiGLU and weighted combine) over one batch of seeded synthetic input already resident
+in HBM. The default workload is the FlashMoE-shaped prefill layer (T=4096, H=2048, D=2048,
+E=64, top-2, capacity factor 1.0); its 1.6 GB of expert weights exceed the 126 MB L2, so no
+L2 flush is needed between steps. With N > 1 (torchrun) every rank runs an independent
+replica on its own GPU (no collective on the data path; weak scaling); rank 0 prints one
+JSON line. `--impl reference` times the CPU oracle instead, on a bounded sample of the same
+workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from mixture_experts_layer_block_b200 import configs, inputs as gen  # noqa: E402
+
+METRIC = "MoE layer tokens/s and TFLOP/s on 1 B200; % of bf16/HBM roofline"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------------------------------
+# workload arithmetic (reporting only)
+# ------------------------------------------------------------------------------------------
+
+def algorithmic_bytes_gemm(w, hit_experts: int) -> float:
+    """Bytes the expert-GEMM kernel must move at least once: the bf16 weights of the experts
+    that receive tokens, the shared expert's weights, x (bf16) and out (fp32)."""
+    b = 3.0 * hit_experts * w.D * w.H * 2
+    b += 3.0 * w.D_shared * w.H * 2
+    b += w.T * w.H * 2 + w.T * w.H * 4
+    return b
+
+
+def routing_stats(layer, w, dev):
+    dbg = layer.debug_outputs(w.T, w.top_k, dev)
+    torch.cuda.synchronize()
+    S = w.T * w.top_k
+    P = int(dbg["num_post_padded"].item())
+    body = dbg["sorted_ids"][:P]
+    kept_ids = dbg["topk_ids"].reshape(-1)[body[body < S].long()]
+    counts = torch.bincount(kept_ids, minlength=w.E).cpu().numpy()
+    return {"kept_slots": int(counts.sum()), "hit_experts": int((counts > 0).sum()),
+            "max_over_mean_load": float(counts.max() / max(counts.mean(), 1e-9)),
+            "empty_experts_frac": float((counts == 0).mean())}
+
+
+# ------------------------------------------------------------------------------------------
+# clocks during the timed region
+# ------------------------------------------------------------------------------------------
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.15)
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        loaded = [s for s in sm if s > 0.5 * max(sm)]
+        return {"sm_mhz": float(np.median(loaded)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------------
+# CPU oracle timing (the reported baseline, and the reference arm)
+# ------------------------------------------------------------------------------------------
+
+def oracle_sample_time(w, wts_host, x_host, n_tokens):
+    from oracle import oracle
+    sub = w.replace(T=n_tokens)
+    inp = dict(wts_host, x=x_host[:n_tokens])
+    t0 = time.perf_counter()
+    oracle.forward(inp, sub.top_k, sub.block_m, sub.capacity_factor)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(w, wts_dev, x_dev, budget_s=12.0):
+    """Time the oracle, as it stands, on the first n tokens of the batch (a smaller batch of
+    the same layer), n sized for about `budget_s` of CPU work."""
+    from oracle import oracle
+    wts_host = {k: (v.cpu() if v is not None else None) for k, v in wts_dev.items()}
+    x_host = x_dev.cpu()
+    n = min(w.T, 16)
+    dt = oracle_sample_time(w, wts_host, x_host, n)
+    n2 = int(min(w.T, max(n, n * budget_s / max(dt, 1e-3))))
+    if n2 > n:
+        n = n2
+        dt = oracle_sample_time(w, wts_host, x_host, n)
+    return {"value": n / dt, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"oracle forward (fp64 C, OpenMP) on the first {n} tokens of the {w.name} batch "
+                      f"as a batch of its own ({dt:.1f} s)"}
+
+
+# ------------------------------------------------------------------------------------------
+# main
+# ------------------------------------------------------------------------------------------
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def max_over_ranks(value: float, world: int) -> float:
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    w = configs.WORKLOADS[args.workload]
+    wts = gen.make_weights(w, "cpu")
+    x = gen.make_x(w, "cpu")
+    from oracle import oracle
+    n = min(w.T, args.ref_tokens)
+    for _ in range(max(0, min(args.warmup, 1))):
+        oracle_sample_time(w, wts, x, min(n, 8))
+    times = [oracle_sample_time(w, wts, x, n) for _ in range(args.steps)]
+    per_tok = float(np.mean(times)) / n
+    value = 1.0 / per_tok
+    ms_step = per_tok * w.T * 1e3
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": w.name, **w.describe()},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+                             "sample": f"each step: oracle forward on the first {n} tokens of the batch"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["mine", "reference"], default="mine")
+    ap.add_argument("--workload", default="flashmoe_prefill", choices=sorted(configs.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--ref-tokens", type=int, default=256)
+    ap.add_argument("--traffic-bytes", type=float, default=None,
+                    help="ncu dram bytes per launch of the expert-GEMM kernel, if captured")
+    args = ap.parse_args()
+    world, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            return run_reference(args, world, rank)
+        return run_mine(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+def run_mine(args, world, rank, local):
+    from mixture_experts_layer_block_b200.native import (MOE_FLAG_HOST_STAGING, MOE_FLAG_STAGE_TIMING,
+                                                         MoELayer)
+    w = configs.WORKLOADS[args.workload]
+    dev = torch.device("cuda", local)
+    wts = gen.make_weights(w, dev)
+    x = gen.make_x(w.replace(seed=w.seed + 1000 * rank) if rank else w, dev)  # each replica its own tokens
+    out = torch.empty((w.T, w.H), dtype=torch.float32, device=dev)
+    layer = MoELayer.for_workload(w, flags=MOE_FLAG_STAGE_TIMING | MOE_FLAG_HOST_STAGING)
+    stream = torch.cuda.current_stream(dev)
+
+    for _ in range(args.warmup):
+        layer.forward(x, wts, out)
+    torch.cuda.synchronize()
+    rc, st = layer.status()
+    assert rc == 0 and st == 0, (rc, st)
+    stats = routing_stats(layer, w, dev)
+    layer.stage_times()  # drop the warm-up window
+
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            layer.forward(x, wts, out)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms = e0.elapsed_time(e1) / args.steps
+    ms = max_over_ranks(ms, world)
+    stage_ms = layer.stage_times()  # mean per kernel over the first 256 timed forwards
+    rc, st = layer.status()
+    assert rc == 0 and st == 0, (rc, st)
+
+    tokens_per_s = world * w.T / (ms * 1e-3)
+    flops = configs.useful_flops(w, stats["kept_slots"])
+    tflops = flops / (ms * 1e-3) / 1e12
+
+    # end to end through the C ABI with host buffers: H2D of x, forward, D2H of out, per step
+    x_pin = x.cpu().pin_memory()
+    out_pin = torch.empty((w.T, w.H), dtype=torch.float32).pin_memory()
+    for _ in range(3):
+        layer.forward_host(x_pin, wts, out_pin)
+    barrier(world)
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(args.e2e_steps):
+        layer.forward_host(x_pin, wts, out_pin)
+    f1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1) / args.e2e_steps, world)
+    layer.stage_times()
+
+    peaks, peak_src = load_peaks()
+    gemm_ms = stage_ms[3]
+    gbytes = algorithmic_bytes_gemm(w, stats["hit_experts"])
+    gemm_flops = flops - 2.0 * w.T * w.H * w.E
+    hbm_t = gbytes / (peaks["hbm_gbs"] * 1e9)
+    tc_t = gemm_flops / (peaks["bf16_tflops"] * 1e12)
+    if hbm_t >= tc_t:
+        achieved = gbytes / (gemm_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"]}
+    else:
+        achieved = gemm_flops / (gemm_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"]}
+    roof.update({"traffic": args.traffic_bytes, "kernel": "moe_gemm_kernel",
+                 "algorithmic_bytes": gbytes, "kernel_ms": gemm_ms, "peak_source": peak_src})
+
+    line = {"metric": METRIC, "value": tokens_per_s, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "T": w.T, "H": w.H, "D": w.D, "E": w.E, "top_k": w.top_k,
+                       "block_m": w.block_m, "D_shared": w.D_shared, "capacity_factor": w.capacity_factor,
+                       "parallelism": f"replicas{world}",
+                       "l2": "inputs larger than L2 (expert weights read each step exceed 126 MB)"},
+            "tflops": tflops, "tflops_frac_of_bf16_peak": tflops / peaks["bf16_tflops"],
+            "stage_ms": {"router": stage_ms[0], "gating": stage_ms[1], "align_scatter": stage_ms[2],
+                         "expert_gemm": stage_ms[3]},
+            "routing": stats, "roofline": roof,
+            "e2e": {"value": world * w.T / (e2e_ms * 1e-3), "unit": UNIT,
+                    "h2d_bytes_per_step": w.T * w.H * 2, "d2h_bytes_per_step": w.T * w.H * 4},
+            "gpu_launches": 4 * args.steps,
+            "clocks": clk.summary()}
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, wts, x)
+    layer.close()
+    if rank == 0:
+        print(json.dumps(line))
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

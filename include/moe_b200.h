@@ -1,0 +1,207 @@
+/*
+ * moe_b200.h -- C ABI of the fused MoE FFN layer forward for NVIDIA B200 (sm_100a).
+ *
+ * The layer (Mixture-of-Kittens blog, section "Overlapping compute and communication in
+ * MoE", layer equation):
+ *
+ *     x' = W_shared(x) + sum_{e in top-k(x)} w_e * W_down^e * SwiGLU(W_up^e x, W_gate^e x),
+ *     SwiGLU(u, g) = SiLU(u) (.) g.
+ *
+ * It runs as four stream-ordered kernels with no host synchronisation and no allocation:
+ *   1. router projection  logits = x W_router^T (+ bias)     tcgen05 GEMM, fp32 out
+ *   2. gating             warp-level top-k + renormalised softmax, per-chunk expert
+ *                         histogram, and (last CTA) the expert/block/tile scans
+ *   3. align scatter      grid-wide writes of sorted_ids / expert_ids (+ zeroing of out)
+ *   4. expert GEMMs       one persistent kernel; its CTAs claim (expert, m-tile, n-tile)
+ *                         tasks from an atomic counter (Weave blog, sections 2.1-2.2):
+ *                         up/gate GEMM with SwiGLU in the epilogue, then down GEMM with
+ *                         the router-weighted combine in the epilogue.
+ *
+ * Conventions for every entry point below
+ *  - Tensors are dense, row-major and contiguous. "bf16" buffers hold IEEE bfloat16 values
+ *    as raw 16-bit patterns. Device pointers are CUDA global-memory addresses on the
+ *    handle's device; they must be 16-byte aligned (the kernels read them with TMA).
+ *  - The caller owns every pointer it passes; the library keeps none of them past the call
+ *    (tensor-map descriptors built from weight pointers are cached by address, so a weight
+ *    buffer may be reused but not freed and re-allocated at the same address with a
+ *    different shape while a handle is alive).
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream). Launches are
+ *    asynchronous; a non-zero return means nothing was launched unless stated otherwise.
+ *  - Errors: every function returns MOE_OK (0) or a negative MOE_ERR_* code. Device-side
+ *    failures (a bounded wait that ran out) are reported by moe_get_status().
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------------------- */
+#define MOE_OK                  0
+#define MOE_ERR_INVALID_ARG    -1  /* null pointer, bad size, top_k > E, T > max_tokens ... */
+#define MOE_ERR_UNSUPPORTED    -2  /* a shape this build cannot run (see moe_init) */
+#define MOE_ERR_CUDA           -3  /* a CUDA runtime/driver call failed */
+#define MOE_ERR_OUT_OF_MEMORY  -4  /* workspace allocation failed in moe_init */
+#define MOE_ERR_MISALIGNED     -5  /* a device pointer is not 16-byte aligned */
+#define MOE_ERR_DEVICE_TIMEOUT -6  /* a device-side wait exceeded moe_config.timeout_ns */
+#define MOE_ERR_NOT_READY      -7  /* the requested data does not exist yet */
+
+/* ---- moe_config.flags --------------------------------------------------------------- */
+#define MOE_FLAG_STAGE_TIMING  1u  /* record CUDA events around each kernel (moe_stage_times) */
+#define MOE_FLAG_HOST_STAGING  2u  /* allocate device staging buffers for moe_forward_host */
+#define MOE_FLAG_TRACE         4u  /* record per-task claim/finish times (moe_trace_read) */
+
+typedef struct moe_config {
+    int32_t hidden;           /* H: model dimension; multiple of 8 */
+    int32_t inter;            /* D: routed-expert intermediate dimension; multiple of 8 */
+    int32_t inter_shared;     /* D_shared: shared-expert intermediate dimension, 0 = none */
+    int32_t num_experts;      /* E: routed experts, 1..1024 */
+    int32_t top_k;            /* largest top_k moe_forward will be called with, 1..min(E,32) */
+    int32_t block_m;          /* align block size (segment padding), 1..1024 */
+    float capacity_factor;    /* 0 = dropless; else C = ceil(cf * T * top_k / E) slots/expert */
+    int32_t max_tokens;       /* largest T moe_forward will be called with, >= 1 */
+    uint32_t flags;           /* MOE_FLAG_* */
+    int32_t device;           /* CUDA device ordinal; -1 = the calling thread's current device */
+    int64_t timeout_ns;       /* limit of every device-side wait; <= 0 = 2e9 (2 s) */
+} moe_config;
+
+typedef struct moe_handle moe_handle;
+
+/* Shared-expert weights (device, bf16): up [D_shared][H], gate [D_shared][H],
+ * down [H][D_shared]. */
+typedef struct moe_shared_w {
+    const void *up;
+    const void *gate;
+    const void *down;
+} moe_shared_w;
+
+/* Create a handle: validates `cfg`, selects the device, allocates and owns the whole
+ * workspace (router logits, top-k ids/weights, histograms, sorted_ids, expert_ids, tile and
+ * task tables, the bf16 intermediate SwiGLU activations h, counters and status word; plus the
+ * staging buffers when MOE_FLAG_HOST_STAGING is set), and queries the SM count.
+ * Intermediate-cache pre-allocation follows the vLLM execution analysis ("Memory allocation
+ * per step": allocate once, reuse across calls); moe_forward never allocates.
+ * On success *out receives the handle. Returns MOE_ERR_INVALID_ARG for a bad cfg,
+ * MOE_ERR_OUT_OF_MEMORY / MOE_ERR_CUDA for allocation or device failures. */
+MOE_API int moe_init(const moe_config *cfg, moe_handle **out);
+
+/* Release the workspace and the handle (synchronises the handle's device first). NULL is
+ * allowed. */
+MOE_API void moe_destroy(moe_handle *h);
+
+/* One layer forward (Mixture-of-Kittens layer equation; top-k softmax gating renormalised
+ * over the selected experts; moe_align_block_size-style sort padded to cfg.block_m;
+ * dropless unless cfg.capacity_factor > 0, in which case a slot whose rank inside its
+ * expert, in ascending slot order s = t*top_k + j, is >= C is dropped and contributes 0).
+ *   x           device bf16 [T][H]
+ *   T           0..cfg.max_tokens
+ *   w_router    device bf16 [E][H]
+ *   router_bias device fp32 [E], added to the logits before selection and softmax; nullable
+ *   w_up,w_gate device bf16 [E][D][H]
+ *   w_down      device bf16 [E][H][D]
+ *   w_shared    nullable; required (all three non-null) iff cfg.inter_shared > 0
+ *   top_k       1..cfg.top_k
+ *   out         device fp32 [T][H]; fully overwritten with x'
+ * Asynchronous on `stream`; no host synchronisation, so it may be captured in a CUDA graph
+ * once the handle's tensor-map cache holds the weight pointers. */
+MOE_API int moe_forward(moe_handle *h, const void *x, int32_t T, const void *w_router,
+                const float *router_bias, const void *w_up, const void *w_gate,
+                const void *w_down, const moe_shared_w *w_shared, int32_t top_k, float *out,
+                void *stream);
+
+/* moe_forward with HOST activations: copies x_host (bf16 [T][H], pinned host memory for
+ * full speed) to a device staging buffer, runs the forward, copies the result to out_host
+ * (fp32 [T][H]) and synchronises `stream`. Weights stay device pointers. Needs
+ * MOE_FLAG_HOST_STAGING at moe_init (else MOE_ERR_NOT_READY). */
+MOE_API int moe_forward_host(moe_handle *h, const void *x_host, int32_t T, const void *w_router,
+                     const float *router_bias, const void *w_up, const void *w_gate,
+                     const void *w_down, const moe_shared_w *w_shared, int32_t top_k,
+                     float *out_host, void *stream);
+
+/* Synchronise the handle's last stream and report the device status word:
+ * *device_status = 0 when every kernel since the last call finished normally, else a
+ * device error code (bit 30 set, low bits naming the wait that ran out). The word is
+ * cleared by this call. Returns MOE_ERR_DEVICE_TIMEOUT if a wait ran out, MOE_ERR_CUDA if
+ * the stream reported a CUDA error, else MOE_OK. */
+MOE_API int moe_get_status(moe_handle *h, int32_t *device_status);
+
+/* Stage entry points (each is one step of moe_forward, callable on its own).
+ *
+ * moe_router_logits: logits (device fp32 [T][E]) = x W_router^T (+ bias). */
+MOE_API int moe_router_logits(moe_handle *h, const void *x, int32_t T, const void *w_router,
+                      const float *router_bias, float *logits, void *stream);
+
+/* moe_gate_topk: per token, the top_k largest logits (ties to the lower expert index) in
+ * descending order, and weights softmax(logits)[id] renormalised over the selected set.
+ * logits device fp32 [T][E]; topk_ids device int32 [T][top_k]; topk_w device fp32
+ * [T][top_k]. (Weave blog section 1.1; vLLM execution analysis, topk_softmax.) */
+MOE_API int moe_gate_topk(moe_handle *h, const float *logits, int32_t T, int32_t top_k,
+                  int32_t *topk_ids, float *topk_w, void *stream);
+
+/* moe_align_block_size: from topk_ids (device int32 [T][top_k]) write
+ *   sorted_ids      device int32 [moe_sorted_len(h, T, top_k)]: slot ids s = t*top_k + j
+ *                   grouped by expert, ascending s inside an expert, each expert segment
+ *                   padded with the sentinel T*top_k to a multiple of cfg.block_m; entries
+ *                   from num_post_padded on are the sentinel
+ *   expert_ids      device int32 [moe_blocks_len(h, T, top_k)]: expert of each block,
+ *                   -1 past the last block
+ *   num_post_padded device int32 [1]: total padded length P
+ * with cfg.capacity_factor applied as in moe_forward. Expert ids outside [0, E) are
+ * invalid input. (vLLM PR #53280 summary, implementation breakdown; all-blocks variant.) */
+MOE_API int moe_align_block_size(moe_handle *h, const int32_t *topk_ids, int32_t T, int32_t top_k,
+                         int32_t *sorted_ids, int32_t *expert_ids, int32_t *num_post_padded,
+                         void *stream);
+
+/* Buffer lengths of moe_align_block_size: T*top_k + E*(block_m-1) and
+ * ceil(that / block_m). Return -1 for a NULL handle or negative sizes. */
+MOE_API int64_t moe_sorted_len(const moe_handle *h, int32_t T, int32_t top_k);
+MOE_API int64_t moe_blocks_len(const moe_handle *h, int32_t T, int32_t top_k);
+
+/* Copy the intermediates of the most recent moe_forward on `stream` into caller device
+ * buffers (each nullable): logits fp32 [T][E], topk_ids int32 [T][k], topk_w fp32 [T][k],
+ * sorted_ids int32 [moe_sorted_len], expert_ids int32 [moe_blocks_len], num_post_padded
+ * int32 [1]. Returns MOE_ERR_NOT_READY before the first forward. */
+MOE_API int moe_debug_outputs(moe_handle *h, float *logits, int32_t *topk_ids, float *topk_w,
+                      int32_t *sorted_ids, int32_t *expert_ids, int32_t *num_post_padded,
+                      void *stream);
+
+/* Mean durations in milliseconds of the kernels of the forwards recorded since the previous
+ * call (the first 256 of them; needs MOE_FLAG_STAGE_TIMING; synchronises, then starts a new
+ * recording window): ms[0] router, ms[1] gating, ms[2] align scatter, ms[3] expert GEMMs.
+ * n = entries of ms (up to 4). Each duration is measured with CUDA events recorded on the
+ * forward's stream around the kernel. MOE_ERR_NOT_READY when nothing was recorded. */
+MOE_API int moe_stage_times(moe_handle *h, float *ms, int32_t n);
+
+/* Handle facts: which = 0 SM count, 1 persistent-kernel CTAs, 2 workspace bytes,
+ * 3 tasks of the last forward (synchronises), 4 m-tiles of the last forward (synchronises),
+ * 5 dependency lag (units) of the last forward. */
+MOE_API int moe_query(const moe_handle *h, int32_t which, int64_t *value);
+
+/* Per-task trace of the last forward (needs MOE_FLAG_TRACE; synchronises). Fills up to
+ * `cap` records of 4 int64 each: {cta, task, t_claim_ns, t_done_ns} (device globaltimer),
+ * sets *n to the records written. */
+MOE_API int moe_trace_read(moe_handle *h, int64_t *records, int64_t cap, int64_t *n);
+
+/* Testing hook: when `extra` > 0, the down-projection tasks of the next moe_forward wait
+ * for `extra` more up-projection completions than can ever arrive, so their bounded wait
+ * runs out after cfg.timeout_ns and the forward reports MOE_ERR_DEVICE_TIMEOUT through
+ * moe_get_status. The hook clears itself after one forward. */
+MOE_API int moe_debug_inject_stall(moe_handle *h, int32_t extra);
+
+/* Human-readable name of a MOE_* status code. */
+MOE_API const char *moe_status_string(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

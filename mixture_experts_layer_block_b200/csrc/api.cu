@@ -1,0 +1,574 @@
+// api.cu -- the C ABI declared in include/moe_b200.h: argument checks, the workspace,
+// tensor-map encoding (cached per weight pointer), kernel launches and status readback.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "launch.h"
+#include "moe_b200.h"
+
+namespace moe {
+cudaError_t configure_gate_kernels(size_t gate_smem);
+cudaError_t configure_router_kernel();
+cudaError_t configure_gemm_kernel();
+}  // namespace moe
+
+using namespace moe;
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+struct MapKey {
+  const void* ptr;
+  uint64_t inner, outer, stride;
+  uint32_t box0, box1;
+  bool operator==(const MapKey& o) const {
+    return ptr == o.ptr && inner == o.inner && outer == o.outer && stride == o.stride &&
+           box0 == o.box0 && box1 == o.box1;
+  }
+};
+
+struct MapEntry {
+  MapKey key;
+  CUtensorMap map;
+};
+
+constexpr int64_t kDefaultTimeoutNs = 2000000000LL;
+constexpr size_t kMapCacheMax = 64;
+constexpr int kTimingRing = 256;  // forwards whose kernel durations moe_stage_times averages
+
+// Dynamic shared memory limit already granted to the gating kernels (shared by all handles).
+size_t g_gate_smem_granted = 0;
+
+}  // namespace
+
+struct moe_handle {
+  moe_config cfg{};
+  int device = 0;
+  int num_sms = 0;
+  char* ws_mem = nullptr;
+  size_t ws_bytes = 0;
+  Workspace ws{};
+  int max_tiles = 0, max_lag = 0, max_units = 0;
+  int64_t sorted_len_max = 0, blocks_len_max = 0;
+  size_t gate_smem = 0;
+  EncodeTiledFn encode = nullptr;
+  std::vector<MapEntry> cache;
+  CUtensorMap h_routed{}, h_shared{};
+  std::vector<cudaEvent_t> ev;  // kTimingRing x 5 events (router, gate, scatter, gemm, end)
+  int timed = 0;                // forwards recorded since the last moe_stage_times
+  bool timing = false;
+  cudaStream_t last_stream = nullptr;
+  bool have_forward = false;
+  int last_T = 0, last_k = 0, last_lag = 0;
+  void* x_stage = nullptr;
+  float* out_stage = nullptr;
+  int dep_extra_next = 0;
+  int64_t timeout_ns = kDefaultTimeoutNs;
+};
+
+namespace {
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int encode_map(moe_handle* h, CUtensorMap* out, const void* ptr, uint64_t inner, uint64_t outer,
+               uint64_t stride_bytes, uint32_t box0, uint32_t box1) {
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {stride_bytes};
+  cuuint32_t box[2] = {box0, box1};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = h->encode(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims,
+                         strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// Weight maps are cached by (pointer, shape, box): encoding is cheap, but caching keeps the
+// per-call host work to a lookup.
+int cached_map(moe_handle* h, CUtensorMap* out, const void* ptr, uint64_t inner, uint64_t outer,
+               uint64_t stride_bytes, uint32_t box0, uint32_t box1) {
+  const MapKey key{ptr, inner, outer, stride_bytes, box0, box1};
+  for (const MapEntry& e : h->cache)
+    if (e.key == key) {
+      *out = e.map;
+      return MOE_OK;
+    }
+  MapEntry e{key, {}};
+  const int rc = encode_map(h, &e.map, ptr, inner, outer, stride_bytes, box0, box1);
+  if (rc != MOE_OK) return rc;
+  if (h->cache.size() >= kMapCacheMax) h->cache.erase(h->cache.begin());
+  h->cache.push_back(e);
+  *out = e.map;
+  return MOE_OK;
+}
+
+int capacity_of(const moe_config& c, int T, int k) {
+  if (!(c.capacity_factor > 0.f)) return 0;
+  const double v = std::ceil((double)c.capacity_factor * (double)T * (double)k / (double)c.num_experts);
+  return (int)std::min<double>(v, (double)T * k);
+}
+
+Shape make_shape(const moe_handle* h, int T, int k) {
+  const moe_config& c = h->cfg;
+  Shape sh{};
+  sh.T = T;
+  sh.H = c.hidden;
+  sh.D = c.inter;
+  sh.Ds = c.inter_shared;
+  sh.E = c.num_experts;
+  sh.k = k;
+  sh.block_m = c.block_m;
+  sh.capacity = capacity_of(c, T, k);
+  sh.chunk_tokens = std::max(kMinChunkTokens, ceil_div(std::max(T, 1), kMaxChunks));
+  sh.num_chunks = std::max(1, ceil_div(T, sh.chunk_tokens));
+  sh.sorted_len = T * k + c.num_experts * (c.block_m - 1);
+  sh.blocks_len = ceil_div(sh.sorted_len, c.block_m);
+  const int n1 = ceil_div(c.inter, kBN1), n2 = ceil_div(c.hidden, kBN2);
+  sh.lag = std::max(1, std::min(h->max_lag, ceil_div(2 * h->num_sms, n1 + n2)));
+  sh.dep_extra = 0;
+  sh.timeout_ns = h->timeout_ns;
+  return sh;
+}
+
+int check_cuda(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+int router_bn(int E) { return E <= 16 ? 16 : (E <= 32 ? 32 : kRouterMaxN); }
+
+int select_device(moe_handle* h) { return check_cuda(cudaSetDevice(h->device)); }
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(int code) {
+  switch (code) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported shape";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_OUT_OF_MEMORY: return "out of device memory";
+    case MOE_ERR_MISALIGNED: return "device pointer not 16-byte aligned";
+    case MOE_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case MOE_ERR_NOT_READY: return "not ready";
+    default: return "unknown status";
+  }
+}
+
+int moe_init(const moe_config* cfg, moe_handle** out) {
+  if (!cfg || !out) return MOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  const moe_config c = *cfg;
+  // ---- argument checks (no CUDA call before these pass) ----
+  if (c.hidden < 8 || c.hidden % 8 != 0) return MOE_ERR_INVALID_ARG;
+  if (c.inter < 8 || c.inter % 8 != 0) return MOE_ERR_INVALID_ARG;
+  if (c.inter_shared < 0 || c.inter_shared % 8 != 0) return MOE_ERR_INVALID_ARG;
+  if (c.num_experts < 1 || c.num_experts > kMaxExperts) return MOE_ERR_INVALID_ARG;
+  if (c.top_k < 1 || c.top_k > std::min(c.num_experts, 32)) return MOE_ERR_INVALID_ARG;
+  if (c.block_m < 1 || c.block_m > 4096) return MOE_ERR_INVALID_ARG;
+  if (!(c.capacity_factor >= 0.f) || std::isinf(c.capacity_factor)) return MOE_ERR_INVALID_ARG;
+  if (c.max_tokens < 1) return MOE_ERR_INVALID_ARG;
+  const int64_t S_max = (int64_t)c.max_tokens * c.top_k;
+  const int64_t sorted_len_max = S_max + (int64_t)c.num_experts * (c.block_m - 1);
+  if (sorted_len_max > (int64_t)INT32_MAX / 2) return MOE_ERR_UNSUPPORTED;
+  if ((int64_t)c.num_experts * std::max(c.inter, c.hidden) > (int64_t)INT32_MAX / 2) return MOE_ERR_UNSUPPORTED;
+  if ((int64_t)c.max_tokens * c.hidden > ((int64_t)1 << 40)) return MOE_ERR_UNSUPPORTED;
+
+  moe_handle* h = new (std::nothrow) moe_handle();
+  if (!h) return MOE_ERR_OUT_OF_MEMORY;
+  h->cfg = c;
+  h->timeout_ns = c.timeout_ns > 0 ? c.timeout_ns : kDefaultTimeoutNs;
+  h->timing = (c.flags & MOE_FLAG_STAGE_TIMING) != 0;
+  int rc = MOE_OK;
+  auto fail = [&](int code) {
+    moe_destroy(h);
+    return code;
+  };
+
+  if (c.device >= 0) {
+    if (cudaSetDevice(c.device) != cudaSuccess) return fail(MOE_ERR_CUDA);
+  }
+  if (cudaGetDevice(&h->device) != cudaSuccess) return fail(MOE_ERR_CUDA);
+  int major = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, h->device) != cudaSuccess)
+    return fail(MOE_ERR_CUDA);
+  if (major != 10) return fail(MOE_ERR_UNSUPPORTED);
+  if (cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess)
+    return fail(MOE_ERR_CUDA);
+
+  // driver entry point for tensor-map encoding (no link-time dependency on libcuda)
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q{};
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || !fn)
+    return fail(MOE_ERR_CUDA);
+  h->encode = reinterpret_cast<EncodeTiledFn>(fn);
+
+  // ---- sizes ----
+  const int E = c.num_experts;
+  h->sorted_len_max = sorted_len_max;
+  h->blocks_len_max = ceil_div((int)sorted_len_max, c.block_m);
+  h->max_tiles = (int)(ceil_div((int)S_max, kBM) + E + (c.inter_shared > 0 ? ceil_div(c.max_tokens, kBM) : 0));
+  h->max_lag = 2 * h->num_sms;
+  h->max_units = h->max_tiles + h->max_lag;
+  const int ldh = std::max(c.inter, c.inter_shared);
+  const int n_task_max = ceil_div(ldh, kBN1) + ceil_div(c.hidden, kBN2);
+  const int trace_cap = (c.flags & MOE_FLAG_TRACE) ? h->max_tiles * n_task_max : 0;
+
+  struct Piece {
+    void** dst;
+    size_t bytes;
+  };
+  Workspace& w = h->ws;
+  const size_t T_ = (size_t)c.max_tokens, K_ = (size_t)c.top_k, E_ = (size_t)E;
+  std::vector<Piece> pieces = {
+      {(void**)&w.meta, sizeof(DeviceMeta)},
+      {(void**)&w.logits, T_ * E_ * 4},
+      {(void**)&w.topk_ids, T_ * K_ * 4},
+      {(void**)&w.topk_w, T_ * K_ * 4},
+      {(void**)&w.chunk_hist, (size_t)kMaxChunks * E_ * 4},
+      {(void**)&w.chunk_base, (size_t)kMaxChunks * E_ * 4},
+      {(void**)&w.expert_off, (E_ + 1) * 4},
+      {(void**)&w.expert_kept, E_ * 4},
+      {(void**)&w.sorted_ids, (size_t)sorted_len_max * 4},
+      {(void**)&w.expert_ids, (size_t)h->blocks_len_max * 4},
+      {(void**)&w.tile_expert, (size_t)h->max_tiles * 4},
+      {(void**)&w.tile_row0, (size_t)h->max_tiles * 4},
+      {(void**)&w.tile_nrows, (size_t)h->max_tiles * 4},
+      {(void**)&w.unit_start, (size_t)(h->max_units + 1) * 4},
+      {(void**)&w.done1, (size_t)h->max_tiles * 4},
+      {(void**)&w.h, (size_t)h->max_tiles * kBM * ldh * 2},
+      {(void**)&w.trace, (size_t)trace_cap * 4 * 8},
+      {(void**)&h->x_stage, (c.flags & MOE_FLAG_HOST_STAGING) ? T_ * c.hidden * 2 : 0},
+      {(void**)&h->out_stage, (c.flags & MOE_FLAG_HOST_STAGING) ? T_ * c.hidden * 4 : 0},
+  };
+  size_t total = 0;
+  for (const Piece& p : pieces) total += (p.bytes + 255) & ~size_t(255);
+  if (cudaMalloc(&h->ws_mem, total) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(MOE_ERR_OUT_OF_MEMORY);
+  }
+  h->ws_bytes = total;
+  size_t off = 0;
+  for (const Piece& p : pieces) {
+    *p.dst = p.bytes ? h->ws_mem + off : nullptr;
+    off += (p.bytes + 255) & ~size_t(255);
+  }
+  w.trace_cap = trace_cap;
+  w.ldh = ldh;
+  if (cudaMemset(h->ws_mem, 0, total) != cudaSuccess) return fail(MOE_ERR_CUDA);
+
+  // h tensor maps (fixed for the handle's lifetime)
+  const uint64_t h_rows = (uint64_t)h->max_tiles * kBM;
+  if ((rc = encode_map(h, &h->h_routed, w.h, c.inter, h_rows, (uint64_t)ldh * 2, kBK, kBM))) return fail(rc);
+  if (c.inter_shared > 0) {
+    if ((rc = encode_map(h, &h->h_shared, w.h, c.inter_shared, h_rows, (uint64_t)ldh * 2, kBK, kBM)))
+      return fail(rc);
+  } else {
+    h->h_shared = h->h_routed;
+  }
+
+  // kernel attributes
+  Shape sh = make_shape(h, c.max_tokens, c.top_k);
+  h->gate_smem = gate_smem_bytes(sh, h->max_units);
+  if (h->gate_smem > g_gate_smem_granted) {
+    if (check_cuda(configure_gate_kernels(h->gate_smem))) return fail(MOE_ERR_CUDA);
+    g_gate_smem_granted = h->gate_smem;
+  }
+  if (check_cuda(configure_router_kernel()) || check_cuda(configure_gemm_kernel())) return fail(MOE_ERR_CUDA);
+  if (h->timing) {
+    h->ev.assign((size_t)kTimingRing * 5, nullptr);
+    for (auto& e : h->ev)
+      if (cudaEventCreate(&e) != cudaSuccess) return fail(MOE_ERR_CUDA);
+  }
+  *out = h;
+  return MOE_OK;
+}
+
+void moe_destroy(moe_handle* h) {
+  if (!h) return;
+  if (h->ws_mem || !h->ev.empty()) {
+    cudaSetDevice(h->device);
+    cudaDeviceSynchronize();
+  }
+  for (auto& e : h->ev)
+    if (e) cudaEventDestroy(e);
+  if (h->ws_mem) cudaFree(h->ws_mem);
+  delete h;
+}
+
+int64_t moe_sorted_len(const moe_handle* h, int32_t T, int32_t top_k) {
+  if (!h || T < 0 || top_k < 0) return -1;
+  return (int64_t)T * top_k + (int64_t)h->cfg.num_experts * (h->cfg.block_m - 1);
+}
+
+int64_t moe_blocks_len(const moe_handle* h, int32_t T, int32_t top_k) {
+  const int64_t n = moe_sorted_len(h, T, top_k);
+  if (n < 0) return -1;
+  return (n + h->cfg.block_m - 1) / h->cfg.block_m;
+}
+
+static int check_tokens(const moe_handle* h, int32_t T, int32_t top_k) {
+  if (T < 0 || T > h->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
+  if (top_k < 1 || top_k > h->cfg.top_k) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+static int forward_impl(moe_handle* h, const void* x, int32_t T, const void* w_router,
+                        const float* router_bias, const void* w_up, const void* w_gate,
+                        const void* w_down, const moe_shared_w* w_shared, int32_t top_k,
+                        float* out, cudaStream_t st) {
+  const moe_config& c = h->cfg;
+  int rc;
+  if ((rc = check_tokens(h, T, top_k))) return rc;
+  if (!x || !w_router || !w_up || !w_gate || !w_down || !out) return MOE_ERR_INVALID_ARG;
+  const bool has_shared = c.inter_shared > 0;
+  if (has_shared && (!w_shared || !w_shared->up || !w_shared->gate || !w_shared->down))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_router) || !aligned16(w_up) || !aligned16(w_gate) ||
+      !aligned16(w_down) || !aligned16(out) || (router_bias && !aligned16(router_bias)))
+    return MOE_ERR_MISALIGNED;
+  if (has_shared && (!aligned16(w_shared->up) || !aligned16(w_shared->gate) || !aligned16(w_shared->down)))
+    return MOE_ERR_MISALIGNED;
+  if ((rc = select_device(h))) return rc;
+  h->last_stream = st;
+  h->last_T = T;
+  h->last_k = top_k;
+  h->have_forward = true;
+  if (T == 0) return MOE_OK;
+
+  const int E = c.num_experts, H = c.hidden, D = c.inter, Ds = c.inter_shared;
+  Shape sh = make_shape(h, T, top_k);
+  sh.dep_extra = h->dep_extra_next;
+  h->dep_extra_next = 0;
+  h->last_lag = sh.lag;
+  const Workspace& w = h->ws;
+
+  // tensor maps
+  CUtensorMap x_router, wr_map;
+  GemmMaps maps;
+  const int bn = router_bn(E);
+  if ((rc = encode_map(h, &x_router, x, H, T, (uint64_t)H * 2, kBK, kBM))) return rc;
+  if ((rc = encode_map(h, &maps.x_gather, x, H, T, (uint64_t)H * 2, kBK, 1))) return rc;
+  if ((rc = cached_map(h, &wr_map, w_router, H, E, (uint64_t)H * 2, kBK, bn))) return rc;
+  if ((rc = cached_map(h, &maps.w_up, w_up, H, (uint64_t)E * D, (uint64_t)H * 2, kBK, kBN1))) return rc;
+  if ((rc = cached_map(h, &maps.w_gate, w_gate, H, (uint64_t)E * D, (uint64_t)H * 2, kBK, kBN1))) return rc;
+  if ((rc = cached_map(h, &maps.w_down, w_down, D, (uint64_t)E * H, (uint64_t)D * 2, kBK, kBN2))) return rc;
+  maps.h_routed = h->h_routed;
+  if (has_shared) {
+    if ((rc = cached_map(h, &maps.ws_up, w_shared->up, H, Ds, (uint64_t)H * 2, kBK, kBN1))) return rc;
+    if ((rc = cached_map(h, &maps.ws_gate, w_shared->gate, H, Ds, (uint64_t)H * 2, kBK, kBN1))) return rc;
+    if ((rc = cached_map(h, &maps.ws_down, w_shared->down, Ds, H, (uint64_t)Ds * 2, kBK, kBN2))) return rc;
+    maps.h_shared = h->h_shared;
+  } else {
+    maps.ws_up = maps.w_up;
+    maps.ws_gate = maps.w_gate;
+    maps.ws_down = maps.w_down;
+    maps.h_shared = h->h_routed;
+  }
+
+  cudaEvent_t* ev = nullptr;
+  if (h->timing && h->timed < kTimingRing) ev = &h->ev[(size_t)h->timed++ * 5];
+  if (ev && cudaEventRecord(ev[0], st) != cudaSuccess) return MOE_ERR_CUDA;
+  if ((rc = check_cuda(launch_router(x_router, wr_map, router_bias, w.logits, T, E, H, bn, w.meta,
+                                     h->timeout_ns, st))))
+    return rc;
+  if (ev && cudaEventRecord(ev[1], st) != cudaSuccess) return MOE_ERR_CUDA;
+  if ((rc = check_cuda(launch_gate(w.logits, w.topk_ids, w.topk_w, w, sh, true, true, h->gate_smem, st))))
+    return rc;
+  if (ev && cudaEventRecord(ev[2], st) != cudaSuccess) return MOE_ERR_CUDA;
+  if ((rc = check_cuda(launch_scatter(w.topk_ids, w.sorted_ids, w.expert_ids, nullptr, out,
+                                      (int64_t)T * H / 4, w, sh, 2 * h->num_sms, st))))
+    return rc;
+  if (ev && cudaEventRecord(ev[3], st) != cudaSuccess) return MOE_ERR_CUDA;
+  if ((rc = check_cuda(launch_moe_gemm(maps, w, sh, out, h->num_sms, st)))) return rc;
+  if (ev && cudaEventRecord(ev[4], st) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+int moe_forward(moe_handle* h, const void* x, int32_t T, const void* w_router,
+                const float* router_bias, const void* w_up, const void* w_gate, const void* w_down,
+                const moe_shared_w* w_shared, int32_t top_k, float* out, void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  return forward_impl(h, x, T, w_router, router_bias, w_up, w_gate, w_down, w_shared, top_k, out,
+                      static_cast<cudaStream_t>(stream));
+}
+
+int moe_forward_host(moe_handle* h, const void* x_host, int32_t T, const void* w_router,
+                     const float* router_bias, const void* w_up, const void* w_gate,
+                     const void* w_down, const moe_shared_w* w_shared, int32_t top_k,
+                     float* out_host, void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  if (!h->x_stage || !h->out_stage) return MOE_ERR_NOT_READY;
+  int rc;
+  if ((rc = check_tokens(h, T, top_k))) return rc;
+  if (!x_host || !out_host) return MOE_ERR_INVALID_ARG;
+  if ((rc = select_device(h))) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t xb = (size_t)T * h->cfg.hidden * 2, ob = (size_t)T * h->cfg.hidden * 4;
+  if (T > 0 && cudaMemcpyAsync(h->x_stage, x_host, xb, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if ((rc = forward_impl(h, h->x_stage, T, w_router, router_bias, w_up, w_gate, w_down, w_shared,
+                         top_k, h->out_stage, st)))
+    return rc;
+  if (T > 0 && cudaMemcpyAsync(out_host, h->out_stage, ob, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return check_cuda(cudaStreamSynchronize(st));
+}
+
+int moe_get_status(moe_handle* h, int32_t* device_status) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  int rc;
+  if ((rc = select_device(h))) return rc;
+  if (cudaStreamSynchronize(h->last_stream) != cudaSuccess) {
+    if (device_status) *device_status = 0;
+    return MOE_ERR_CUDA;
+  }
+  int32_t st = 0;
+  if (cudaMemcpy(&st, &h->ws.meta->status, sizeof st, cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  const int32_t zero = 0;
+  if (cudaMemcpy(&h->ws.meta->status, &zero, sizeof zero, cudaMemcpyHostToDevice) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (device_status) *device_status = st;
+  if (st & kStatusTimeout) return MOE_ERR_DEVICE_TIMEOUT;
+  return MOE_OK;
+}
+
+int moe_router_logits(moe_handle* h, const void* x, int32_t T, const void* w_router,
+                      const float* router_bias, float* logits, void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  if (T < 0 || T > h->cfg.max_tokens || !x || !w_router || !logits) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_router) || !aligned16(logits)) return MOE_ERR_MISALIGNED;
+  int rc;
+  if ((rc = select_device(h))) return rc;
+  if (T == 0) return MOE_OK;
+  const int E = h->cfg.num_experts, H = h->cfg.hidden, bn = router_bn(E);
+  CUtensorMap xm, wm;
+  if ((rc = encode_map(h, &xm, x, H, T, (uint64_t)H * 2, kBK, kBM))) return rc;
+  if ((rc = cached_map(h, &wm, w_router, H, E, (uint64_t)H * 2, kBK, bn))) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  h->last_stream = st;
+  return check_cuda(launch_router(xm, wm, router_bias, logits, T, E, H, bn, h->ws.meta, h->timeout_ns, st));
+}
+
+int moe_gate_topk(moe_handle* h, const float* logits, int32_t T, int32_t top_k, int32_t* topk_ids,
+                  float* topk_w, void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  int rc;
+  if ((rc = check_tokens(h, T, top_k))) return rc;
+  if (!logits || !topk_ids || !topk_w) return MOE_ERR_INVALID_ARG;
+  if ((rc = select_device(h))) return rc;
+  if (T == 0) return MOE_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  h->last_stream = st;
+  const Shape sh = make_shape(h, T, top_k);
+  return check_cuda(launch_gate(logits, topk_ids, topk_w, h->ws, sh, false, false, 0, st));
+}
+
+int moe_align_block_size(moe_handle* h, const int32_t* topk_ids, int32_t T, int32_t top_k,
+                         int32_t* sorted_ids, int32_t* expert_ids, int32_t* num_post_padded,
+                         void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  int rc;
+  if ((rc = check_tokens(h, T, top_k))) return rc;
+  if ((T > 0 && !topk_ids) || !sorted_ids || !expert_ids || !num_post_padded) return MOE_ERR_INVALID_ARG;
+  if ((rc = select_device(h))) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  h->last_stream = st;
+  const Shape sh = make_shape(h, T, top_k);
+  if ((rc = check_cuda(launch_hist(topk_ids, h->ws, sh, h->gate_smem, st)))) return rc;
+  return check_cuda(launch_scatter(topk_ids, sorted_ids, expert_ids, num_post_padded, nullptr, 0,
+                                   h->ws, sh, 2 * h->num_sms, st));
+}
+
+int moe_debug_outputs(moe_handle* h, float* logits, int32_t* topk_ids, float* topk_w,
+                      int32_t* sorted_ids, int32_t* expert_ids, int32_t* num_post_padded,
+                      void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  if (!h->have_forward) return MOE_ERR_NOT_READY;
+  int rc;
+  if ((rc = select_device(h))) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t T = h->last_T, k = h->last_k, E = h->cfg.num_experts;
+  const Workspace& w = h->ws;
+  auto cp = [&](void* dst, const void* src, size_t bytes) {
+    if (!dst || bytes == 0) return MOE_OK;
+    return check_cuda(cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, st));
+  };
+  if ((rc = cp(logits, w.logits, T * E * 4))) return rc;
+  if ((rc = cp(topk_ids, w.topk_ids, T * k * 4))) return rc;
+  if ((rc = cp(topk_w, w.topk_w, T * k * 4))) return rc;
+  if ((rc = cp(sorted_ids, w.sorted_ids, (size_t)moe_sorted_len(h, (int)T, (int)k) * 4))) return rc;
+  if ((rc = cp(expert_ids, w.expert_ids, (size_t)moe_blocks_len(h, (int)T, (int)k) * 4))) return rc;
+  if ((rc = cp(num_post_padded, &w.meta->P, 4))) return rc;
+  return MOE_OK;
+}
+
+int moe_stage_times(moe_handle* h, float* ms, int32_t n) {
+  if (!h || !ms || n < 1) return MOE_ERR_INVALID_ARG;
+  if (!h->timing || h->timed == 0) return MOE_ERR_NOT_READY;
+  const int m = h->timed;
+  h->timed = 0;
+  for (int i = 0; i < std::min(n, 4); ++i) ms[i] = 0.f;
+  if (cudaEventSynchronize(h->ev[(size_t)(m - 1) * 5 + 4]) != cudaSuccess) return MOE_ERR_CUDA;
+  for (int f = 0; f < m; ++f)
+    for (int i = 0; i < std::min(n, 4); ++i) {
+      float t = 0.f;
+      if (cudaEventElapsedTime(&t, h->ev[(size_t)f * 5 + i], h->ev[(size_t)f * 5 + i + 1]) != cudaSuccess)
+        return MOE_ERR_CUDA;
+      ms[i] += t / m;
+    }
+  return MOE_OK;
+}
+
+int moe_query(const moe_handle* h, int32_t which, int64_t* value) {
+  if (!h || !value) return MOE_ERR_INVALID_ARG;
+  switch (which) {
+    case 0: *value = h->num_sms; return MOE_OK;
+    case 1: *value = h->num_sms; return MOE_OK;
+    case 2: *value = (int64_t)h->ws_bytes; return MOE_OK;
+    case 3:
+    case 4: {
+      if (!h->have_forward) return MOE_ERR_NOT_READY;
+      if (cudaSetDevice(h->device) != cudaSuccess) return MOE_ERR_CUDA;
+      if (cudaStreamSynchronize(h->last_stream) != cudaSuccess) return MOE_ERR_CUDA;
+      DeviceMeta m{};
+      if (cudaMemcpy(&m, h->ws.meta, sizeof m, cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+      *value = (which == 3) ? m.total_tasks : m.num_tiles;
+      return MOE_OK;
+    }
+    case 5: *value = h->last_lag; return MOE_OK;
+    default: return MOE_ERR_INVALID_ARG;
+  }
+}
+
+int moe_trace_read(moe_handle* h, int64_t* records, int64_t cap, int64_t* n) {
+  if (!h || !records || !n || cap < 0) return MOE_ERR_INVALID_ARG;
+  if (h->ws.trace_cap == 0) return MOE_ERR_NOT_READY;
+  int64_t total = 0;
+  int rc;
+  if ((rc = moe_query(h, 3, &total))) return rc;
+  const int64_t m = std::min<int64_t>(std::min<int64_t>(total, h->ws.trace_cap), cap);
+  if (m > 0 && cudaMemcpy(records, h->ws.trace, (size_t)m * 4 * 8, cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  *n = m;
+  return MOE_OK;
+}
+
+int moe_debug_inject_stall(moe_handle* h, int32_t extra) {
+  if (!h || extra < 0) return MOE_ERR_INVALID_ARG;
+  h->dep_extra_next = extra;
+  return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,174 @@
+// common.cuh -- definitions shared by the kernels and the host API: tile sizes, workspace
+// layout, device status codes, task encoding and bounded waits.
+#pragma once
+
+#include <cstdint>
+
+#include "ptx.cuh"
+
+namespace moe {
+
+// ---- tile geometry of the expert GEMMs ---------------------------------------------------
+constexpr int kBM = 128;        // rows (token slots) per m-tile = UMMA M
+constexpr int kBK = 64;         // K elements per pipeline stage = one 128-byte swizzle row
+constexpr int kUK = 16;         // K per tcgen05.mma (bf16)
+constexpr int kBN1 = 128;       // D columns per up/gate task; MMA N = 2*kBN1 (up | gate)
+constexpr int kBN2 = 256;       // H columns per down task; MMA N = kBN2
+constexpr int kUmmaN = 256;     // N of every expert-GEMM MMA
+constexpr int kStages = 4;      // smem pipeline depth
+constexpr int kABytes = kBM * kBK * 2;       // 16 KB
+constexpr int kBBytes = kUmmaN * kBK * 2;    // 32 KB
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kTaskSlots = 4;   // depth of the producer -> MMA/epilogue task ring
+constexpr int kAccCols = 256;   // TMEM columns per accumulator buffer (2 buffers)
+constexpr int kGemmThreads = 192;  // warp 0 producer, warp 1 MMA, warps 2-5 epilogue
+
+// ---- router GEMM -------------------------------------------------------------------------
+constexpr int kRouterStages = 4;
+constexpr int kRouterMaxN = 64;
+
+// ---- gating / align ------------------------------------------------------------------------
+constexpr int kGateThreads = 256;
+constexpr int kMaxChunks = 128;    // token chunks of the histogram (chunk = ceil(T/128) >= 64)
+constexpr int kMinChunkTokens = 64;
+constexpr int kMaxExperts = 1024;
+
+// ---- device status word --------------------------------------------------------------------
+constexpr int kStatusTimeout = 1 << 30;     // | where-code
+enum WaitSite : int {
+  kSiteProducerEmpty = 1,
+  kSiteProducerTask = 2,
+  kSiteDependency = 3,
+  kSiteMmaTask = 4,
+  kSiteMmaAcc = 5,
+  kSiteMmaFull = 6,
+  kSiteEpiTask = 7,
+  kSiteEpiAcc = 8,
+  kSiteDrain = 9,
+  kSiteRouter = 10,
+};
+
+// Counters and scalars that live in device memory (one int each).
+struct DeviceMeta {
+  int task_counter;   // atomic work queue head
+  int abort;          // set by any wait that gave up; every CTA then drains and exits
+  int status;         // first device error code (0 = ok)
+  int hist_done;      // CTAs of the histogram kernel that finished (last one scans)
+  int num_tiles;      // m-tiles of this forward (routed + shared)
+  int total_tasks;    // tasks of this forward
+  int num_units;      // scheduling units (tiles + lag)
+  int P;              // num_post_padded
+  int trace_count;    // trace records written
+  int pad[7];
+};
+
+// Task kinds in the ring.
+constexpr int kTaskUp = 0;     // up/gate GEMM + SwiGLU -> h
+constexpr int kTaskDown = 1;   // down GEMM + weighted combine -> out
+constexpr int kTaskStop = -1;
+
+struct Task {
+  int32_t kind;
+  int32_t tile;    // m-tile index
+  int32_t expert;  // routed expert, or E for the shared expert
+  int32_t row0;    // first sorted row (routed) or first token (shared)
+  int32_t nrows;   // valid rows in the tile (1..128)
+  int32_t n0;      // first output column (D for up tasks, H for down tasks)
+  int32_t nk;      // K stages
+  int32_t id;      // global task id
+};
+
+// Pointers into the workspace handed to the kernels.
+struct Workspace {
+  DeviceMeta* meta;
+  float* logits;         // [T][E]
+  int32_t* topk_ids;     // [T][k]
+  float* topk_w;         // [T][k]
+  int32_t* chunk_hist;   // [kMaxChunks][E]
+  int32_t* chunk_base;   // [kMaxChunks][E]  exclusive prefix over chunks, per expert
+  int32_t* expert_off;   // [E+1]            padded segment offsets
+  int32_t* expert_kept;  // [E]              kept slots per expert
+  int32_t* sorted_ids;   // [sorted_len]
+  int32_t* expert_ids;   // [blocks_len]
+  int32_t* tile_expert;  // [max_tiles]
+  int32_t* tile_row0;    // [max_tiles]
+  int32_t* tile_nrows;   // [max_tiles]
+  int32_t* unit_start;   // [max_tiles + max_lag + 1]
+  int32_t* done1;        // [max_tiles]      finished up/gate tasks per tile
+  uint16_t* h;           // [max_tiles*128][ldh] bf16 SwiGLU activations
+  int64_t* trace;        // [trace_cap][4]
+  int32_t trace_cap;
+  int32_t ldh;           // row stride of h in elements (max(D, D_shared))
+};
+
+// Shapes and knobs of one forward, passed by value.
+struct Shape {
+  int32_t T, H, D, Ds, E, k, block_m;
+  int32_t capacity;      // C, 0 = dropless
+  int32_t chunk_tokens;  // tokens per histogram chunk
+  int32_t num_chunks;
+  int32_t sorted_len, blocks_len;
+  int32_t lag;           // scheduling lag in units between a tile's up and down tasks
+  int32_t dep_extra;     // testing hook: extra up completions a down task waits for
+  int64_t timeout_ns;
+};
+
+__host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// ---- error raising and bounded waits -------------------------------------------------------
+__device__ __forceinline__ void raise_error(DeviceMeta* meta, volatile int* s_abort, int code) {
+  atomicCAS(&meta->status, 0, code);
+  atomicExch(&meta->abort, 1);
+  if (s_abort) *s_abort = 1;
+}
+
+__device__ __forceinline__ bool aborted(const DeviceMeta* meta, const volatile int* s_abort) {
+  return (s_abort && *s_abort) || *reinterpret_cast<const volatile int*>(&meta->abort);
+}
+
+// Wait until the phase of parity `parity` of `bar` completed. Gives up (returns false) when
+// the kernel is aborting or after `limit_ns`, in which case it raises a timeout error.
+static __device__ __noinline__ bool wait_bar(uint64_t* bar, uint32_t parity, DeviceMeta* meta,
+                                      volatile int* s_abort, int64_t limit_ns, int site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  uint32_t n = 0;
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((++n & 7u) == 0) {
+      if (aborted(meta, s_abort)) return false;
+      if (static_cast<int64_t>(globaltimer_ns() - t0) > limit_ns) {
+        raise_error(meta, s_abort, kStatusTimeout | site);
+        return false;
+      }
+    }
+  }
+}
+
+// Teardown wait: ignores the abort flag (the work it waits for is already in flight and will
+// finish), bounded by `limit_ns`.
+static __device__ __noinline__ bool wait_bar_drain(uint64_t* bar, uint32_t parity, DeviceMeta* meta,
+                                            int64_t limit_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (static_cast<int64_t>(globaltimer_ns() - t0) > limit_ns) {
+      atomicCAS(&meta->status, 0, kStatusTimeout | kSiteDrain);
+      atomicExch(&meta->abort, 1);
+      return false;
+    }
+  }
+  return true;
+}
+
+// Wait for the last TMA fill of every stage of a ring that was filled `nfill` times in
+// round-robin order (fill f of stage s completes phase f of its `full` barrier).
+__device__ __forceinline__ void drain_fills(uint64_t* full, int nstages, uint32_t nfill,
+                                            DeviceMeta* meta, int64_t limit_ns) {
+  for (int s = 0; s < nstages; ++s) {
+    if (nfill <= static_cast<uint32_t>(s)) break;
+    const uint32_t fills = (nfill - 1u - s) / nstages + 1u;
+    wait_bar_drain(&full[s], (fills - 1u) & 1u, meta, limit_ns);
+  }
+}
+
+}  // namespace moe

@@ -1,0 +1,432 @@
+// gate_align.cu -- gating (top-k softmax, renormalised) and align (moe_align_block_size).
+//
+// Gating (Weave blog section 1.1; vLLM execution analysis, topk_softmax): one warp per
+// token; each lane holds E/32 logits; k rounds of a warp arg-max (ties to the lower expert
+// index) select the experts in descending order; the weights are the selected softmax
+// probabilities renormalised over the selection, i.e. exp(v_j - v_0) / sum_i exp(v_i - v_0).
+//
+// Align (vLLM PR #53280 summary: per-expert counts, exclusive cumsum, cooperative writes of
+// token ids and block ids; the reviewer's variant that uses every block of the grid):
+//   1. each CTA of the gating (or histogram) kernel counts the slots of its token chunk per
+//      expert;
+//   2. the last CTA to finish scans: per expert, the counts of earlier chunks (so writes stay
+//      stable), the capacity cut, the padded segment offsets, and for the forward also the
+//      m-tile list and the task schedule of the expert-GEMM kernel;
+//   3. a grid-wide kernel writes sorted_ids (one warp per chunk, 32 slots per round, ranks
+//      from __match_any_sync), the padding sentinels and expert_ids (one thread per entry).
+#include <algorithm>
+#include <climits>
+#include <cmath>
+
+#include "launch.h"
+
+namespace moe {
+
+// ------------------------------------------------------------------------------------------
+// warp top-k + renormalised softmax of one token; lane j < k returns choice j
+// ------------------------------------------------------------------------------------------
+template <int VPL>
+__device__ __forceinline__ void warp_topk_softmax(const float* __restrict__ row, int E, int k,
+                                                  int lane, int& out_id, float& out_w) {
+  float v[VPL];
+  uint32_t taken = 0;
+#pragma unroll
+  for (int j = 0; j < VPL; ++j) {
+    const int e = lane + 32 * j;
+    v[j] = (e < E) ? row[e] : -INFINITY;
+    if (e >= E) taken |= 1u << j;
+  }
+  float my_v = 0.f, top_v = 0.f;
+  int my_id = -1;
+  for (int r = 0; r < k; ++r) {
+    float bv = -INFINITY;
+    int bi = INT_MAX;
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) {
+      const int e = lane + 32 * j;
+      if (!((taken >> j) & 1u) && (v[j] > bv || (v[j] == bv && e < bi))) {
+        bv = v[j];
+        bi = e;
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+      if (ov > bv || (ov == bv && oi < bi)) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    if (bi != INT_MAX && (bi & 31) == lane) taken |= 1u << (bi >> 5);
+    if (lane == r) {
+      my_v = bv;
+      my_id = bi;
+    }
+    if (r == 0) top_v = bv;
+  }
+  const float ex = (lane < k) ? expf(my_v - top_v) : 0.f;
+  float s = ex;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+  out_id = my_id;
+  out_w = ex / s;
+}
+
+// ------------------------------------------------------------------------------------------
+// block-wide exclusive scan of a[0..n) in shared memory (any n), returns the total.
+// Uses `tmp` (>= blockDim/32 + 1 ints). All threads must call it.
+// ------------------------------------------------------------------------------------------
+__device__ int block_exclusive_scan(int* a, int n, int* tmp) {
+  const int tid = threadIdx.x, nthr = blockDim.x, lane = tid & 31, warp = tid >> 5;
+  const int nwarps = nthr >> 5;
+  int carry = 0;
+  for (int base = 0; base < n; base += nthr * 4) {
+    int loc[4];
+    int sum = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int idx = base + tid * 4 + i;
+      loc[i] = (idx < n) ? a[idx] : 0;
+      sum += loc[i];
+    }
+    int incl = sum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += y;
+    }
+    if (lane == 31) tmp[warp] = incl;
+    __syncthreads();
+    if (tid == 0) {
+      int run = 0;
+      for (int w = 0; w < nwarps; ++w) {
+        const int x = tmp[w];
+        tmp[w] = run;
+        run += x;
+      }
+      tmp[nwarps] = run;
+    }
+    __syncthreads();
+    int run = carry + tmp[warp] + incl - sum;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int idx = base + tid * 4 + i;
+      if (idx < n) a[idx] = run;
+      run += loc[i];
+    }
+    carry += tmp[nwarps];
+    __syncthreads();
+  }
+  return carry;
+}
+
+// ------------------------------------------------------------------------------------------
+// The scans, run by the last CTA of the histogram pass. Shared memory layout (ints):
+//   tmp[64] | cnt[E] | kept[E] | buf[max(E+1, units+1)]
+// ------------------------------------------------------------------------------------------
+__device__ void align_scans(const Workspace& ws, const Shape& sh, bool tiles, int* sm) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
+  const int E = sh.E;
+  int* tmp = sm;
+  int* cnt = tmp + 64;
+  int* kept = cnt + E;
+  int* buf = kept + E;
+  const int nch = sh.num_chunks;
+
+  // 1. per expert: exclusive prefix of the chunk counts (chunk_base) and the total n_e
+  const int cpw = ceil_div(nch, nwarps);
+  for (int eg = 0; eg < E; eg += 32) {
+    const int e = eg + lane;
+    const int c0 = warp * cpw, c1 = min(nch, c0 + cpw);
+    int sum = 0;
+    if (e < E)
+      for (int c = c0; c < c1; ++c) sum += __ldcg(ws.chunk_hist + (size_t)c * E + e);
+    buf[warp * 32 + lane] = sum;
+    __syncthreads();
+    if (warp == 0) {
+      int run = 0;
+      for (int w = 0; w < nwarps; ++w) {
+        const int x = buf[w * 32 + lane];
+        buf[w * 32 + lane] = run;
+        run += x;
+      }
+      if (e < E) cnt[e] = run;
+    }
+    __syncthreads();
+    int run = buf[warp * 32 + lane];
+    if (e < E)
+      for (int c = c0; c < c1; ++c) {
+        ws.chunk_base[(size_t)c * E + e] = run;
+        run += __ldcg(ws.chunk_hist + (size_t)c * E + e);
+      }
+    __syncthreads();
+  }
+
+  // 2. capacity cut and padded segment lengths
+  for (int e = tid; e < E; e += blockDim.x) {
+    const int n = cnt[e];
+    const int kp = (sh.capacity > 0) ? min(n, sh.capacity) : n;
+    kept[e] = kp;
+    ws.expert_kept[e] = kp;
+    buf[e] = ceil_div(kp, sh.block_m) * sh.block_m;
+  }
+  __syncthreads();
+  const int P = block_exclusive_scan(buf, E, tmp);
+  for (int e = tid; e < E; e += blockDim.x) ws.expert_off[e] = buf[e];
+  if (tid == 0) {
+    ws.expert_off[E] = P;
+    ws.meta->P = P;
+  }
+  __syncthreads();
+  if (!tiles) return;
+
+  // 3. m-tiles: routed experts (ceil(kept/128) each), then the shared expert over all tokens
+  for (int e = tid; e < E; e += blockDim.x) buf[e] = ceil_div(kept[e], kBM);
+  __syncthreads();
+  const int Mr = block_exclusive_scan(buf, E, tmp);
+  for (int e = tid; e < E; e += blockDim.x) {
+    const int first = buf[e], nt = ceil_div(kept[e], kBM);
+    const int off = ws.expert_off[e];
+    for (int i = 0; i < nt; ++i) {
+      ws.tile_expert[first + i] = e;
+      ws.tile_row0[first + i] = off + i * kBM;
+      ws.tile_nrows[first + i] = min(kBM, kept[e] - i * kBM);
+    }
+  }
+  const int Ms = (sh.Ds > 0) ? ceil_div(sh.T, kBM) : 0;
+  for (int j = tid; j < Ms; j += blockDim.x) {
+    ws.tile_expert[Mr + j] = E;
+    ws.tile_row0[Mr + j] = j * kBM;
+    ws.tile_nrows[Mr + j] = min(kBM, sh.T - j * kBM);
+  }
+  const int Mt = Mr + Ms;
+  __syncthreads();
+
+  // 4. schedule units: unit u holds the up/gate tasks of tile u, then the down tasks of tile
+  //    u - lag. Task ids are unit-major, so every down task's dependencies have lower ids.
+  const int U = (Mt > 0) ? Mt + sh.lag : 0;
+  const int n2 = ceil_div(sh.H, kBN2);
+  for (int u = tid; u < U; u += blockDim.x) {
+    int c = 0;
+    if (u < Mt) c += ceil_div(ws.tile_expert[u] == E ? sh.Ds : sh.D, kBN1);
+    if (u >= sh.lag && u - sh.lag < Mt) c += n2;
+    buf[u] = c;
+  }
+  __syncthreads();
+  const int total = block_exclusive_scan(buf, U, tmp);
+  for (int u = tid; u < U; u += blockDim.x) ws.unit_start[u] = buf[u];
+  for (int i = tid; i < Mt; i += blockDim.x) ws.done1[i] = 0;
+  if (tid == 0) {
+    ws.unit_start[U] = total;
+    ws.meta->num_tiles = Mt;
+    ws.meta->num_units = U;
+    ws.meta->total_tasks = total;
+    ws.meta->task_counter = 0;
+    ws.meta->abort = 0;
+    ws.meta->trace_count = 0;
+  }
+}
+
+// Publish this CTA's chunk histogram; the last CTA runs the scans.
+__device__ void finish_histogram(const Workspace& ws, const Shape& sh, bool tiles, const int* hist,
+                                 int* sm) {
+  __shared__ int s_last;
+  for (int e = threadIdx.x; e < sh.E; e += blockDim.x)
+    ws.chunk_hist[(size_t)blockIdx.x * sh.E + e] = hist[e];
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = (atomicAdd(&ws.meta->hist_done, 1) == (int)gridDim.x - 1);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  align_scans(ws, sh, tiles, sm);
+  if (threadIdx.x == 0) ws.meta->hist_done = 0;
+}
+
+// ------------------------------------------------------------------------------------------
+// kernels
+// ------------------------------------------------------------------------------------------
+// smem: hist[E] | scan area
+template <int VPL>
+__global__ void __launch_bounds__(kGateThreads)
+    gate_kernel(const float* __restrict__ logits, int32_t* __restrict__ topk_ids,
+                float* __restrict__ topk_w, Workspace ws, Shape sh, int hist_on, int tiles) {
+  extern __shared__ int smem_i[];
+  int* hist = smem_i;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t0 = blockIdx.x * sh.chunk_tokens;
+  const int t1 = min(sh.T, t0 + sh.chunk_tokens);
+  if (hist_on) {
+    for (int e = threadIdx.x; e < sh.E; e += blockDim.x) hist[e] = 0;
+    __syncthreads();
+  }
+  for (int t = t0 + warp; t < t1; t += kGateThreads / 32) {
+    int id;
+    float w;
+    warp_topk_softmax<VPL>(logits + (size_t)t * sh.E, sh.E, sh.k, lane, id, w);
+    if (lane < sh.k) {
+      topk_ids[(size_t)t * sh.k + lane] = id;
+      topk_w[(size_t)t * sh.k + lane] = w;
+      if (hist_on) atomicAdd(&hist[id], 1);
+    }
+  }
+  if (!hist_on) return;
+  __syncthreads();
+  finish_histogram(ws, sh, tiles != 0, hist, smem_i + sh.E);
+}
+
+__global__ void __launch_bounds__(kGateThreads)
+    hist_kernel(const int32_t* __restrict__ topk_ids, Workspace ws, Shape sh) {
+  extern __shared__ int smem_i[];
+  int* hist = smem_i;
+  for (int e = threadIdx.x; e < sh.E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const int64_t s0 = (int64_t)blockIdx.x * sh.chunk_tokens * sh.k;
+  const int64_t s1 = (int64_t)min(sh.T, (int)(blockIdx.x + 1) * sh.chunk_tokens) * sh.k;
+  for (int64_t s = s0 + threadIdx.x; s < s1; s += blockDim.x) {
+    const int e = topk_ids[s];
+    if (e >= 0 && e < sh.E) atomicAdd(&hist[e], 1);  // ids outside [0, E) are skipped
+  }
+  __syncthreads();
+  finish_histogram(ws, sh, false, hist, smem_i + sh.E);
+}
+
+__device__ __forceinline__ int segment_of(const int* off, int E, int i) {
+  // largest e with off[e] <= i (off non-decreasing, off[E] = P > i)
+  int lo = 0, hi = E;  // answer in [lo, hi)
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (off[mid] <= i) lo = mid;
+    else hi = mid;
+  }
+  return lo;
+}
+
+// smem: off[E+1] | kept[E] | per-warp counters [8][E]
+__global__ void __launch_bounds__(256)
+    scatter_kernel(const int32_t* __restrict__ topk_ids, int32_t* __restrict__ sorted_ids,
+                   int32_t* __restrict__ expert_ids, int32_t* __restrict__ num_post_padded,
+                   float* __restrict__ out_zero, int64_t n4, Workspace ws, Shape sh) {
+  extern __shared__ int smem_i[];
+  const int E = sh.E;
+  int* off = smem_i;
+  int* kept = off + E + 1;
+  int* cnt_all = kept + E;
+  for (int e = threadIdx.x; e <= E; e += blockDim.x) off[e] = __ldcg(ws.expert_off + e);
+  for (int e = threadIdx.x; e < E; e += blockDim.x) kept[e] = __ldcg(ws.expert_kept + e);
+  __syncthreads();
+  const int P = off[E];
+  const int S = sh.T * sh.k;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // (a) stable scatter of the slot ids, one warp per chunk
+  int* cnt = cnt_all + warp * E;
+  const int gw = blockIdx.x * (blockDim.x >> 5) + warp;
+  const int nw = gridDim.x * (blockDim.x >> 5);
+  for (int c = gw; c < sh.num_chunks; c += nw) {
+    for (int e = lane; e < E; e += 32) cnt[e] = __ldcg(ws.chunk_base + (size_t)c * E + e);
+    __syncwarp();
+    const int s0 = c * sh.chunk_tokens * sh.k;
+    const int s1 = min(sh.T, (c + 1) * sh.chunk_tokens) * sh.k;
+    for (int base = s0; base < s1; base += 32) {
+      const int s = base + lane;
+      int e = (s < s1) ? topk_ids[s] : -1;
+      if (e >= E) e = -1;
+      const bool valid = e >= 0;
+      const unsigned mask = __match_any_sync(0xffffffffu, e);
+      const int rank = __popc(mask & ((1u << lane) - 1u));
+      const int c0 = valid ? cnt[e] : 0;
+      __syncwarp();
+      if (valid) {
+        const int r = c0 + rank;
+        if (sh.capacity == 0 || r < sh.capacity) sorted_ids[off[e] + r] = s;
+        if (rank == 0) cnt[e] = c0 + __popc(mask);
+      }
+      __syncwarp();
+    }
+  }
+
+  // (b) padding sentinels, (c) block -> expert ids, one thread per entry
+  const int gt = blockIdx.x * blockDim.x + threadIdx.x;
+  const int nt = gridDim.x * blockDim.x;
+  for (int i = gt; i < sh.sorted_len; i += nt) {
+    bool pad = true;
+    if (i < P) {
+      const int e = segment_of(off, E, i);
+      pad = (i - off[e]) >= kept[e];
+    }
+    if (pad) sorted_ids[i] = S;
+  }
+  for (int b = gt; b < sh.blocks_len; b += nt) {
+    const int i = b * sh.block_m;
+    expert_ids[b] = (i < P) ? segment_of(off, E, i) : -1;
+  }
+  if (gt == 0 && num_post_padded) *num_post_padded = P;
+
+  // (d) zero the layer output (the expert GEMMs accumulate into it)
+  if (out_zero) {
+    float4* o4 = reinterpret_cast<float4*>(out_zero);
+    for (int64_t i = gt; i < n4; i += nt) o4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// launchers
+// ------------------------------------------------------------------------------------------
+size_t gate_smem_bytes(const Shape& sh, int max_units) {
+  const int buf = std::max(std::max(sh.E + 1, max_units + 1), 8 * 32);
+  return sizeof(int) * (size_t)(sh.E /*hist*/ + 64 + 2 * sh.E + buf);
+}
+
+size_t scatter_smem_bytes(int E) { return sizeof(int) * (size_t)(E + 1 + E + 8 * E); }
+
+template <int VPL>
+static cudaError_t launch_gate_vpl(const float* logits, int32_t* ids, float* w, const Workspace& ws,
+                                   const Shape& sh, bool hist, bool tiles, size_t smem,
+                                   cudaStream_t st) {
+  gate_kernel<VPL><<<sh.num_chunks, kGateThreads, hist ? smem : 0, st>>>(logits, ids, w, ws, sh,
+                                                                          hist ? 1 : 0, tiles ? 1 : 0);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gate(const float* logits, int32_t* topk_ids, float* topk_w, const Workspace& ws,
+                        const Shape& sh, bool hist, bool tiles, size_t smem, cudaStream_t st) {
+  if (sh.num_chunks <= 0) return cudaSuccess;
+  if (sh.E <= 32) return launch_gate_vpl<1>(logits, topk_ids, topk_w, ws, sh, hist, tiles, smem, st);
+  if (sh.E <= 64) return launch_gate_vpl<2>(logits, topk_ids, topk_w, ws, sh, hist, tiles, smem, st);
+  if (sh.E <= 128) return launch_gate_vpl<4>(logits, topk_ids, topk_w, ws, sh, hist, tiles, smem, st);
+  if (sh.E <= 256) return launch_gate_vpl<8>(logits, topk_ids, topk_w, ws, sh, hist, tiles, smem, st);
+  if (sh.E <= 512) return launch_gate_vpl<16>(logits, topk_ids, topk_w, ws, sh, hist, tiles, smem, st);
+  return launch_gate_vpl<32>(logits, topk_ids, topk_w, ws, sh, hist, tiles, smem, st);
+}
+
+cudaError_t launch_hist(const int32_t* topk_ids, const Workspace& ws, const Shape& sh, size_t smem,
+                        cudaStream_t st) {
+  hist_kernel<<<sh.num_chunks, kGateThreads, smem, st>>>(topk_ids, ws, sh);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_scatter(const int32_t* topk_ids, int32_t* sorted_ids, int32_t* expert_ids,
+                           int32_t* num_post_padded, float* out_zero, int64_t n4,
+                           const Workspace& ws, const Shape& sh, int grid, cudaStream_t st) {
+  scatter_kernel<<<grid, 256, scatter_smem_bytes(sh.E), st>>>(topk_ids, sorted_ids, expert_ids,
+                                                              num_post_padded, out_zero, n4, ws, sh);
+  return cudaGetLastError();
+}
+
+cudaError_t configure_gate_kernels(size_t gate_smem) {
+  cudaError_t err = cudaSuccess;
+  const int s = (int)gate_smem;
+  if ((err = cudaFuncSetAttribute(gate_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, s))) return err;
+  if ((err = cudaFuncSetAttribute(gate_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, s))) return err;
+  if ((err = cudaFuncSetAttribute(gate_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, s))) return err;
+  if ((err = cudaFuncSetAttribute(gate_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, s))) return err;
+  if ((err = cudaFuncSetAttribute(gate_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, s))) return err;
+  if ((err = cudaFuncSetAttribute(gate_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, s))) return err;
+  if ((err = cudaFuncSetAttribute(hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, s))) return err;
+  return cudaFuncSetAttribute(scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)scatter_smem_bytes(kMaxExperts));
+}
+
+}  // namespace moe

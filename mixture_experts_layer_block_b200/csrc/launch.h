@@ -1,0 +1,53 @@
+// launch.h -- host-side launchers of the kernels (implemented next to each kernel).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+// Tensor maps of the persistent expert-GEMM kernel.
+struct alignas(64) GemmMaps {
+  CUtensorMap x_gather;  // x [T][H], box {64, 1} (row gather)
+  CUtensorMap w_up;      // [E*D][H], box {64, 128}
+  CUtensorMap w_gate;    // [E*D][H], box {64, 128}
+  CUtensorMap w_down;    // [E*H][D], box {64, 256}
+  CUtensorMap h_routed;  // h [rows][D], row stride ldh, box {64, 128}
+  CUtensorMap ws_up;     // [Ds][H]
+  CUtensorMap ws_gate;   // [Ds][H]
+  CUtensorMap ws_down;   // [H][Ds]
+  CUtensorMap h_shared;  // h [rows][Ds], row stride ldh
+};
+
+// Router projection: logits[T][E] = x W^T (+ bias). x_map box {64,128}, w_map box {64,BN}.
+size_t router_smem_bytes(int BN);
+cudaError_t launch_router(const CUtensorMap& x_map, const CUtensorMap& w_map, const float* bias,
+                          float* logits, int T, int E, int H, int BN, DeviceMeta* meta,
+                          int64_t timeout_ns, cudaStream_t stream);
+
+// Gating. With `hist`, also the per-chunk expert histogram and, in the last CTA, the scans
+// (and the tile/task tables when `tiles`).
+size_t gate_smem_bytes(const Shape& sh, int max_units);
+cudaError_t launch_gate(const float* logits, int32_t* topk_ids, float* topk_w, const Workspace& ws,
+                        const Shape& sh, bool hist, bool tiles, size_t smem, cudaStream_t stream);
+
+// Histogram of given topk_ids (standalone align), with the same last-CTA scans (no tiles).
+cudaError_t launch_hist(const int32_t* topk_ids, const Workspace& ws, const Shape& sh, size_t smem,
+                        cudaStream_t stream);
+
+// Grid-wide align writes, plus zeroing of `out_zero` (n4 float4s) when non-null.
+size_t scatter_smem_bytes(int E);
+cudaError_t launch_scatter(const int32_t* topk_ids, int32_t* sorted_ids, int32_t* expert_ids,
+                           int32_t* num_post_padded, float* out_zero, int64_t n4,
+                           const Workspace& ws, const Shape& sh, int grid, cudaStream_t stream);
+
+// Persistent expert GEMMs.
+size_t gemm_smem_bytes();
+cudaError_t launch_moe_gemm(const GemmMaps& maps, const Workspace& ws, const Shape& sh, float* out,
+                            int grid, cudaStream_t stream);
+
+// One-time kernel attribute setup (dynamic shared memory limits).
+cudaError_t configure_kernels(size_t gate_smem);
+
+}  // namespace moe

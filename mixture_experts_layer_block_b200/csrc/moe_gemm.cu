@@ -1,0 +1,380 @@
+// moe_gemm.cu -- the persistent grouped expert GEMM with the atomic tile scheduler.
+//
+// What it computes (Mixture-of-Kittens blog, "Overlapping compute and communication in
+// MoE"): for every kept slot s = (t, j) routed to expert e,
+//     h_s  = SiLU(W_up^e x_t) (.) (W_gate^e x_t)                   (bf16, kept in HBM/L2)
+//     out_t += w_s * W_down^e h_s                                  (fp32 reduction)
+// plus the shared expert over every token with weight 1.
+//
+// How (Weave blog, sections 2.1-2.2 and 5.1: tile decomposition, an atomic task counter,
+// one persistent CTA per SM that claims tasks until the queue is empty):
+//  - m-tile: up to 128 sorted rows of one expert (align output), or 128 tokens of the
+//    shared expert.
+//  - up task   (tile, n): A = the tile's x rows, gathered with TMA tile::gather4 from the
+//    sorted slot ids; B = 128 rows of W_up^e stacked on 128 rows of W_gate^e; one
+//    tcgen05.mma of N = 256 per K step, so TMEM holds U | G; the epilogue writes
+//    h = SiLU(U) * G (bf16) for columns n*128 .. n*128+127 and counts the tile's done1.
+//  - down task (tile, n): waits until done1[tile] covers every up task of the tile (bounded
+//    spin), then A = the tile's h rows, B = 256 rows of W_down^e; the epilogue scales each
+//    row by its router weight and adds it into out[token] (fp32 vector atomics).
+//  - task ids are numbered in units: unit u = up tasks of tile u, then down tasks of tile
+//    u - lag. A down task's dependencies always have smaller ids, and claims are monotone,
+//    so the earliest unfinished task can always make progress (no deadlock).
+//
+// Warp roles (192 threads, one CTA per SM): warp 0 claims tasks and issues TMA into a
+// 4-stage ring (48 KB / stage); warp 1 allocates 512 TMEM columns (two 256-column fp32
+// accumulators) and issues tcgen05.mma from one lane; warps 2-5 drain TMEM (tcgen05.ld)
+// in the epilogue. Producer -> consumers: a 4-entry task ring guarded by mbarriers.
+// Every wait is bounded (globaltimer); a wait that runs out records a status code, sets the
+// abort flag, and every CTA drains its in-flight copies and MMAs and exits.
+#include "launch.h"
+
+namespace moe {
+
+namespace {
+
+struct SmemLayout {
+  static constexpr int kBarOff = kStages * kStageBytes;
+  // barriers: full[S], empty[S], acc_full[2], acc_empty[2], task_full[R], task_empty[R], drain
+  static constexpr int kNumBars = 2 * kStages + 4 + 2 * kTaskSlots + 1;
+  static constexpr int kRingOff = kBarOff + ((kNumBars * 8 + 63) & ~63);
+  static constexpr int kMiscOff = kRingOff + kTaskSlots * (int)sizeof(Task);
+  static constexpr int kBytes = kMiscOff + 64;
+};
+
+__device__ __forceinline__ int n1_of(int expert, const Shape& sh) {
+  return ceil_div(expert == sh.E ? sh.Ds : sh.D, kBN1);
+}
+
+// Bounded wait until *p >= need (acquire). Raises a timeout error on expiry.
+__device__ __noinline__ bool wait_count(const int* p, int need, DeviceMeta* meta,
+                                        volatile int* s_abort, int64_t limit_ns) {
+  if (ld_acquire_gpu(p) >= need) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    __nanosleep(128);
+    if (ld_acquire_gpu(p) >= need) return true;
+    if (aborted(meta, s_abort)) return false;
+    if (static_cast<int64_t>(globaltimer_ns() - t0) > limit_ns) {
+      raise_error(meta, s_abort, kStatusTimeout | kSiteDependency);
+      return false;
+    }
+  }
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    moe_gemm_kernel(const __grid_constant__ GemmMaps maps, Workspace ws, Shape sh,
+                    float* __restrict__ out) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SmemLayout::kBarOff);
+  uint64_t* full = bars;
+  uint64_t* empty = full + kStages;
+  uint64_t* acc_full = empty + kStages;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* task_full = acc_empty + 2;
+  uint64_t* task_empty = task_full + kTaskSlots;
+  uint64_t* drain = task_empty + kTaskSlots;
+  Task* ring = reinterpret_cast<Task*>(smem + SmemLayout::kRingOff);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + SmemLayout::kMiscOff);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + SmemLayout::kMiscOff + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  DeviceMeta* meta = ws.meta;
+  const int64_t limit = sh.timeout_ns;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 4);  // one arrival per epilogue warp
+    }
+    for (int i = 0; i < kTaskSlots; ++i) {
+      mbar_init(&task_full[i], 1);
+      mbar_init(&task_empty[i], 5);  // MMA lane + 4 epilogue warps
+    }
+    mbar_init(drain, 1);
+    *s_abort = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&maps.x_gather);
+    tma_prefetch_desc(&maps.w_up);
+    tma_prefetch_desc(&maps.w_gate);
+    tma_prefetch_desc(&maps.w_down);
+    tma_prefetch_desc(&maps.h_routed);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(s_tmem), 2 * kAccCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *s_tmem;
+  uint32_t nfill = 0;  // TMA stage fills issued by this CTA (producer warp)
+  bool mma_issued = false;
+
+  if (warp == 0) {
+    // ===================================== producer =====================================
+    const int total = __ldcg(&meta->total_tasks);
+    const int Mt = __ldcg(&meta->num_tiles);
+    const int nk1 = ceil_div(sh.H, kBK);
+    int u_cur = 0;
+    uint32_t stage = 0, phase = 0, slot = 0, slot_phase = 0;
+    while (true) {
+      int tau = 0;
+      if (lane == 0) tau = aborted(meta, s_abort) ? total : atomicAdd(&meta->task_counter, 1);
+      tau = __shfl_sync(0xffffffffu, tau, 0);
+      Task t;
+      t.id = tau;
+      if (tau >= total) {
+        t.kind = kTaskStop;
+      } else {
+        while (__ldcg(&ws.unit_start[u_cur + 1]) <= tau) ++u_cur;
+        const int off = tau - __ldcg(&ws.unit_start[u_cur]);
+        const int n1u = (u_cur < Mt) ? n1_of(__ldcg(&ws.tile_expert[u_cur]), sh) : 0;
+        int nt;
+        if (off < n1u) {
+          t.kind = kTaskUp;
+          t.tile = u_cur;
+          nt = off;
+        } else {
+          t.kind = kTaskDown;
+          t.tile = u_cur - sh.lag;
+          nt = off - n1u;
+        }
+        t.expert = __ldcg(&ws.tile_expert[t.tile]);
+        t.row0 = __ldcg(&ws.tile_row0[t.tile]);
+        t.nrows = __ldcg(&ws.tile_nrows[t.tile]);
+        const int Dt = (t.expert == sh.E) ? sh.Ds : sh.D;
+        if (t.kind == kTaskUp) {
+          t.n0 = nt * kBN1;
+          t.nk = nk1;
+        } else {
+          t.n0 = nt * kBN2;
+          t.nk = ceil_div(Dt, kBK);
+        }
+      }
+      // publish the task to the MMA and epilogue warps
+      bool ok = true;
+      if (lane == 0) {
+        ok = wait_bar(&task_empty[slot], slot_phase ^ 1, meta, s_abort, limit, kSiteProducerTask);
+        if (ok) {
+          ring[slot] = t;
+          mbar_arrive(&task_full[slot]);
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok || t.kind == kTaskStop) break;
+      if (++slot == kTaskSlots) { slot = 0; slot_phase ^= 1; }
+      if (ws.trace_cap > 0 && lane == 0) {
+        // claim time goes to the trace slot of this task id (written again at completion)
+        if (tau < ws.trace_cap) {
+          ws.trace[(size_t)tau * 4 + 0] = blockIdx.x;
+          ws.trace[(size_t)tau * 4 + 1] = tau;
+          ws.trace[(size_t)tau * 4 + 2] = (int64_t)globaltimer_ns();
+        }
+      }
+      const bool shared = (t.expert == sh.E);
+      // a down task needs every up task of its tile
+      if (t.kind == kTaskDown) {
+        if (lane == 0) {
+          ok = wait_count(&ws.done1[t.tile], n1_of(t.expert, sh) + sh.dep_extra, meta, s_abort, limit);
+          if (ok) fence_proxy_async_global();
+        }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
+      }
+      // x rows of the up task: lane l gathers rows 4l..4l+3; rows past nrows repeat row 0
+      // (their results are never read)
+      int r[4] = {0, 0, 0, 0};
+      if (t.kind == kTaskUp) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int row = lane * 4 + i;
+          const int rr = row < t.nrows ? row : 0;
+          r[i] = shared ? (t.row0 + rr) : (__ldcg(&ws.sorted_ids[t.row0 + rr]) / sh.k);
+        }
+      }
+      const int wrow_up = shared ? t.n0 : t.expert * sh.D + t.n0;
+      const int wrow_dn = shared ? t.n0 : t.expert * sh.H + t.n0;
+      for (int kb = 0; kb < t.nk; ++kb) {
+        if (lane == 0) ok = wait_bar(&empty[stage], phase ^ 1, meta, s_abort, limit, kSiteProducerEmpty);
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
+        const uint32_t a = smem_u32(smem + stage * kStageBytes);
+        const uint32_t b = a + kABytes;
+        if (lane == 0) mbar_arrive_expect_tx(&full[stage], kStageBytes);
+        __syncwarp();
+        if (t.kind == kTaskUp) {
+          tma_gather4(a + lane * 512, &maps.x_gather, &full[stage], kb * kBK, r[0], r[1], r[2], r[3]);
+          if (lane == 0) {
+            tma_load_2d(b, shared ? &maps.ws_up : &maps.w_up, &full[stage], kb * kBK, wrow_up);
+            tma_load_2d(b + kBN1 * 128, shared ? &maps.ws_gate : &maps.w_gate, &full[stage], kb * kBK,
+                        wrow_up);
+          }
+        } else if (lane == 0) {
+          tma_load_2d(a, shared ? &maps.h_shared : &maps.h_routed, &full[stage], kb * kBK, t.tile * kBM);
+          tma_load_2d(b, shared ? &maps.ws_down : &maps.w_down, &full[stage], kb * kBK, wrow_dn);
+        }
+        ++nfill;
+        if (++stage == kStages) { stage = 0; phase ^= 1; }
+      }
+      if (!ok) break;
+    }
+  } else if (warp == 1) {
+    // ===================================== MMA issuer ===================================
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kBM, kUmmaN);
+      uint32_t stage = 0, phase = 0, slot = 0, slot_phase = 0, acc = 0, acc_phase = 0;
+      while (true) {
+        if (!wait_bar(&task_full[slot], slot_phase, meta, s_abort, limit, kSiteMmaTask)) break;
+        const Task t = ring[slot];
+        if (t.kind == kTaskStop) break;
+        if (!wait_bar(&acc_empty[acc], acc_phase ^ 1, meta, s_abort, limit, kSiteMmaAcc)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + acc * kAccCols;
+        bool ok = true;
+        for (int kb = 0; kb < t.nk; ++kb) {
+          if (!wait_bar(&full[stage], phase, meta, s_abort, limit, kSiteMmaFull)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a = smem_u32(smem + stage * kStageBytes);
+          const uint32_t b = a + kABytes;
+#pragma unroll
+          for (int kk = 0; kk < kBK / kUK; ++kk)
+            umma_bf16(d, sdesc_kmajor_sw128(a + kk * 32), sdesc_kmajor_sw128(b + kk * 32), idesc,
+                      (kb | kk) != 0);
+          mma_issued = true;
+          umma_commit(&empty[stage]);
+          if (++stage == kStages) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        umma_commit(&acc_full[acc]);
+        mbar_arrive(&task_empty[slot]);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+        if (++slot == kTaskSlots) { slot = 0; slot_phase ^= 1; }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ===================================== epilogue =====================================
+    const int q = warp & 3;          // TMEM lane quarter this warp may read
+    const int row = q * 32 + lane;   // tile row owned by this thread
+    uint32_t slot = 0, slot_phase = 0, acc = 0, acc_phase = 0;
+    while (true) {
+      if (!wait_bar(&task_full[slot], slot_phase, meta, s_abort, limit, kSiteEpiTask)) break;
+      const Task t = ring[slot];
+      if (t.kind == kTaskStop) break;
+      if (!wait_bar(&acc_full[acc], acc_phase, meta, s_abort, limit, kSiteEpiAcc)) break;
+      tc_fence_after();
+      const uint32_t tacc = tmem_base + acc * kAccCols + (static_cast<uint32_t>(q * 32) << 16);
+      const bool shared = (t.expert == sh.E);
+      if (t.kind == kTaskUp) {
+        const int Dt = shared ? sh.Ds : sh.D;
+        uint16_t* hrow = ws.h + (size_t)(t.tile * kBM + row) * ws.ldh;
+#pragma unroll 1
+        for (int c = 0; c < kBN1; c += 32) {
+          uint32_t u[32], g[32];
+          tmem_ld_32x32b_x32(tacc + c, u);
+          tmem_ld_32x32b_x32(tacc + kBN1 + c, g);
+          tmem_ld_wait();
+          uint32_t pk[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float u0 = __uint_as_float(u[2 * j]), u1 = __uint_as_float(u[2 * j + 1]);
+            const float g0 = __uint_as_float(g[2 * j]), g1 = __uint_as_float(g[2 * j + 1]);
+            const float h0 = u0 / (1.0f + __expf(-u0)) * g0;
+            const float h1 = u1 / (1.0f + __expf(-u1)) * g1;
+            pk[j] = pack_bf16x2(h0, h1);
+          }
+          const int col = t.n0 + c;
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            if (col + 8 * v + 8 <= Dt)
+              *reinterpret_cast<uint4*>(hrow + col + 8 * v) =
+                  make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[acc]);
+        // publish h: this tile's down tasks read it with TMA (async proxy) on other SMs
+        fence_proxy_async_global();
+        __threadfence();
+        named_bar_sync(1, 128);
+        if (warp == 2 && lane == 0) red_release_add_gpu(&ws.done1[t.tile], 1);
+      } else {
+        const bool valid = row < t.nrows;
+        int tok = 0;
+        float w = 0.f;
+        if (valid) {
+          if (shared) {
+            tok = t.row0 + row;
+            w = 1.f;
+          } else {
+            const int s = __ldcg(&ws.sorted_ids[t.row0 + row]);
+            tok = s / sh.k;
+            w = __ldcg(&ws.topk_w[s]);
+          }
+        }
+        float* orow = out + (size_t)tok * sh.H;
+#pragma unroll 1
+        for (int c = 0; c < kBN2; c += 32) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tacc + c, v);
+          tmem_ld_wait();
+          const int col = t.n0 + c;
+          if (valid) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              if (col + 4 * j + 4 <= sh.H)
+                atomicAdd(reinterpret_cast<float4*>(orow + col + 4 * j),
+                          make_float4(w * __uint_as_float(v[4 * j]), w * __uint_as_float(v[4 * j + 1]),
+                                      w * __uint_as_float(v[4 * j + 2]), w * __uint_as_float(v[4 * j + 3])));
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[acc]);
+      }
+      if (lane == 0) mbar_arrive(&task_empty[slot]);
+      if (ws.trace_cap > 0 && warp == 2 && lane == 0 && t.id < ws.trace_cap)
+        ws.trace[(size_t)t.id * 4 + 3] = (int64_t)globaltimer_ns();
+      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+      if (++slot == kTaskSlots) { slot = 0; slot_phase ^= 1; }
+    }
+  }
+
+  // teardown: every TMA fill and tcgen05 op issued by this CTA must be complete before the
+  // CTA releases TMEM and exits (this only waits after an abort)
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0) drain_fills(full, kStages, nfill, meta, limit);
+  if (threadIdx.x == 32) {
+    if (mma_issued) {
+      umma_commit(drain);
+      wait_bar_drain(drain, 0, meta, limit);
+    }
+  }
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, 2 * kAccCols);
+}
+
+size_t gemm_smem_bytes() { return (size_t)SmemLayout::kBytes + 1024; }
+
+cudaError_t launch_moe_gemm(const GemmMaps& maps, const Workspace& ws, const Shape& sh, float* out,
+                            int grid, cudaStream_t stream) {
+  moe_gemm_kernel<<<grid, kGemmThreads, gemm_smem_bytes(), stream>>>(maps, ws, sh, out);
+  return cudaGetLastError();
+}
+
+cudaError_t configure_gemm_kernel() {
+  return cudaFuncSetAttribute(moe_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)gemm_smem_bytes());
+}
+
+}  // namespace moe

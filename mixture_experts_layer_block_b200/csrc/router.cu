@@ -1,0 +1,168 @@
+// router.cu -- router projection logits[T][E] = x[T][H] . W_router[E][H]^T (+ bias[E]).
+//
+// Router projection of the Mixture-of-Kittens layer ("Overlapping compute and communication
+// in MoE": the router projection picks the top-k routed experts of each token). A dense
+// contraction, so it runs on the tensor cores: one CTA per 128 x BN output tile, TMA-fed
+// 4-stage smem ring (x tile 128 x 64, W tile BN x 64, both 128-byte swizzled), tcgen05.mma
+// with the fp32 accumulator in TMEM, and an epilogue warpgroup that adds the bias and
+// stores fp32 rows.
+//
+// Warp roles: warp 0 TMA producer, warp 1 TMEM allocator + MMA issuer, warps 2-5 epilogue.
+#include "launch.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kRThreads = 192;
+constexpr int kRABytes = kBM * kBK * 2;
+
+__device__ __forceinline__ uint32_t tmem_cols_for(int bn) { return bn <= 32 ? 32u : 64u; }
+
+// 32 lanes x 16 columns
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(kRThreads, 1)
+    router_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CUtensorMap w_map,
+                  const float* __restrict__ bias, float* __restrict__ logits, int T, int E, int H,
+                  int BN, DeviceMeta* meta, int64_t timeout_ns) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int b_bytes = BN * kBK * 2;
+  const int stage_bytes = kRABytes + ((b_bytes + 1023) & ~1023);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kRouterStages * stage_bytes);
+  uint64_t* empty = full + kRouterStages;
+  uint64_t* acc_full = empty + kRouterStages;
+  uint64_t* drain = acc_full + 1;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * kBM, n0 = blockIdx.y * BN;
+  const int nk = ceil_div(H, kBK);
+  const uint32_t ncols = tmem_cols_for(BN);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kRouterStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(drain, 1);
+    *s_abort = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&x_map);
+    tma_prefetch_desc(&w_map);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(s_tmem), ncols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+  uint32_t nfill = 0;  // TMA fills issued (producer lane)
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0;
+      for (int kb = 0; kb < nk; ++kb, ++nfill) {
+        if (!wait_bar(&empty[stage], phase ^ 1, meta, s_abort, timeout_ns, kSiteRouter)) break;
+        const uint32_t a = smem_u32(smem + stage * stage_bytes);
+        mbar_arrive_expect_tx(&full[stage], kRABytes + b_bytes);
+        tma_load_2d(a, &x_map, &full[stage], kb * kBK, m0);
+        tma_load_2d(a + kRABytes, &w_map, &full[stage], kb * kBK, n0);
+        if (++stage == kRouterStages) { stage = 0; phase ^= 1; }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(kBM, BN);
+      uint32_t stage = 0, phase = 0;
+      bool ok = true;
+      for (int kb = 0; kb < nk; ++kb) {
+        if (!wait_bar(&full[stage], phase, meta, s_abort, timeout_ns, kSiteRouter)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a = smem_u32(smem + stage * stage_bytes);
+        const uint32_t b = a + kRABytes;
+#pragma unroll
+        for (int kk = 0; kk < kBK / kUK; ++kk)
+          umma_bf16(tmem, sdesc_kmajor_sw128(a + kk * 32), sdesc_kmajor_sw128(b + kk * 32), idesc,
+                    (kb | kk) != 0);
+        umma_commit(&empty[stage]);
+        if (++stage == kRouterStages) { stage = 0; phase ^= 1; }
+      }
+      if (ok) umma_commit(acc_full);
+    }
+    __syncwarp();
+  } else {
+    // epilogue: thread owns one output row
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const bool ok = wait_bar(acc_full, 0, meta, s_abort, timeout_ns, kSiteRouter);
+    tc_fence_after();
+    if (ok) {
+      const int t = m0 + row;
+      for (int c = 0; c < BN; c += 16) {
+        uint32_t v[16];
+        tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(q * 32) << 16) + c, v);
+        tmem_ld_wait();
+        if (t < T) {
+          float* dst = logits + (size_t)t * E;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int e = n0 + c + j;
+            if (e < E) dst[e] = __uint_as_float(v[j]) + (bias ? bias[e] : 0.f);
+          }
+        }
+      }
+    }
+  }
+
+  // teardown: every TMA fill and every MMA this CTA issued must have landed before the
+  // shared memory and TMEM are released (only waits after an abort)
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0) drain_fills(full, kRouterStages, nfill, meta, timeout_ns);
+  if (threadIdx.x == 32) {
+    umma_commit(drain);
+    wait_bar_drain(drain, 0, meta, timeout_ns);
+  }
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, ncols);
+}
+
+size_t router_smem_bytes(int BN) {
+  const int b_bytes = BN * kBK * 2;
+  const int stage_bytes = kRABytes + ((b_bytes + 1023) & ~1023);
+  return (size_t)kRouterStages * stage_bytes + 1024 /*align*/ + 256 /*barriers*/;
+}
+
+cudaError_t launch_router(const CUtensorMap& x_map, const CUtensorMap& w_map, const float* bias,
+                          float* logits, int T, int E, int H, int BN, DeviceMeta* meta,
+                          int64_t timeout_ns, cudaStream_t stream) {
+  dim3 grid(ceil_div(T, kBM), ceil_div(E, BN));
+  router_kernel<<<grid, kRThreads, router_smem_bytes(BN), stream>>>(x_map, w_map, bias, logits, T, E,
+                                                                     H, BN, meta, timeout_ns);
+  return cudaGetLastError();
+}
+
+cudaError_t configure_router_kernel() {
+  return cudaFuncSetAttribute(router_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)router_smem_bytes(kRouterMaxN));
+}
+
+}  // namespace moe
