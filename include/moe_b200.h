@@ -102,7 +102,7 @@ MOE_API void moe_destroy(moe_handle *h);
  * over the selected experts; moe_align_block_size-style sort padded to cfg.block_m;
  * dropless unless cfg.capacity_factor > 0, in which case a slot whose rank inside its
  * expert, in ascending slot order s = t*top_k + j, is >= C is dropped and contributes 0).
- *   x           device bf16 [T][H]
+ *   x           device bf16 [T][H] (may be NULL when T == 0)
  *   T           0..cfg.max_tokens
  *   w_router    device bf16 [E][H]
  *   router_bias device fp32 [E], added to the logits before selection and softmax; nullable
@@ -110,7 +110,7 @@ MOE_API void moe_destroy(moe_handle *h);
  *   w_down      device bf16 [E][H][D]
  *   w_shared    nullable; required (all three non-null) iff cfg.inter_shared > 0
  *   top_k       1..cfg.top_k
- *   out         device fp32 [T][H]; fully overwritten with x'
+ *   out         device fp32 [T][H]; fully overwritten with x' (may be NULL when T == 0)
  * Asynchronous on `stream`; no host synchronisation, so it may be captured in a CUDA graph
  * once the handle's tensor-map cache holds the weight pointers. */
 MOE_API int moe_forward(moe_handle *h, const void *x, int32_t T, const void *w_router,

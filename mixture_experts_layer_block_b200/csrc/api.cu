@@ -330,7 +330,8 @@ static int forward_impl(moe_handle* h, const void* x, int32_t T, const void* w_r
   const moe_config& c = h->cfg;
   int rc;
   if ((rc = check_tokens(h, T, top_k))) return rc;
-  if (!x || !w_router || !w_up || !w_gate || !w_down || !out) return MOE_ERR_INVALID_ARG;
+  if (!w_router || !w_up || !w_gate || !w_down) return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (!x || !out)) return MOE_ERR_INVALID_ARG;  // an empty batch may pass null x / out
   const bool has_shared = c.inter_shared > 0;
   if (has_shared && (!w_shared || !w_shared->up || !w_shared->gate || !w_shared->down))
     return MOE_ERR_INVALID_ARG;
