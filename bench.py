@@ -4,8 +4,8 @@ dominant kernel's fraction of the HBM (or tensor) roofline.
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mine|reference]
                   [--workload flashmoe_prefill] [--no-cpu-baseline] [--e2e-steps M]
 
-One step = one whole layer forward (router projection, gating, align, expert GEMMs with the
-fused SwiGLU and weighted combine) over one batch of seeded synthetic input already resident
+One step = one whole layer forward (router projection, gating, align, row gather, expert
+GEMMs with the fused SwiGLU and router weighting, and the combine) over one batch of seeded synthetic input already resident
 in HBM. The default workload is the FlashMoE-shaped prefill layer (T=4096, H=2048, D=2048,
 E=64, top-2, capacity factor 1.0); its 1.6 GB of expert weights exceed the 126 MB L2, so no
 L2 flush is needed between steps. With N > 1 (torchrun) every rank runs an independent
@@ -56,6 +56,42 @@ def algorithmic_bytes_gemm(w, hit_experts: int) -> float:
     b += 3.0 * w.D_shared * w.H * 2
     b += w.T * w.H * 2 + w.T * w.H * 4
     return b
+
+
+def sm_busy_fraction(records: np.ndarray, n_ctas: int) -> dict:
+    """SM-busy fraction of one traced forward of the expert-GEMM kernel: per CTA the union of
+    its tasks' [claim, done] intervals, summed, over n_ctas x (last done - first claim)."""
+    if records.size == 0:
+        return {"sm_busy": None}
+    r = records[(records[:, 2] > 0) & (records[:, 3] >= records[:, 2])]
+    t0, t1 = r[:, 2].min(), r[:, 3].max()
+    busy = 0
+    for cta in np.unique(r[:, 0]):
+        iv = r[r[:, 0] == cta][:, 2:4]
+        iv = iv[np.argsort(iv[:, 0])]
+        cur_s, cur_e = iv[0]
+        for s_, e_ in iv[1:]:
+            if s_ > cur_e:
+                busy += cur_e - cur_s
+                cur_s, cur_e = s_, e_
+            else:
+                cur_e = max(cur_e, e_)
+        busy += cur_e - cur_s
+    return {"sm_busy": float(busy / (n_ctas * (t1 - t0))), "makespan_us": float((t1 - t0) / 1e3),
+            "tasks": int(r.shape[0])}
+
+
+def traced_forward(w, wts, x, out):
+    """One extra forward with per-task tracing (outside the timed region)."""
+    from mixture_experts_layer_block_b200.native import MOE_FLAG_TRACE, MoELayer
+    layer = MoELayer.for_workload(w, flags=MOE_FLAG_TRACE)
+    for _ in range(2):
+        layer.forward(x, wts, out)
+    torch.cuda.synchronize()
+    rec = layer.trace(1 << 20)
+    n_ctas = layer.query(1)
+    layer.close()
+    return sm_busy_fraction(rec, n_ctas)
 
 
 def routing_stats(layer, w, dev):
@@ -228,6 +264,7 @@ def main():
     ap.add_argument("--impl", choices=["mine", "reference"], default="mine")
     ap.add_argument("--workload", default="flashmoe_prefill", choices=sorted(configs.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-trace", action="store_true", help="skip the traced forward (SM-busy)")
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--ref-tokens", type=int, default=256)
     ap.add_argument("--traffic-bytes", type=float, default=None,
@@ -300,7 +337,7 @@ def run_mine(args, world, rank, local):
     layer.stage_times()
 
     peaks, peak_src = load_peaks()
-    gemm_ms = stage_ms[3]
+    gemm_ms = stage_ms[4]
     gbytes = algorithmic_bytes_gemm(w, stats["hit_experts"])
     gemm_flops = flops - 2.0 * w.T * w.H * w.E
     hbm_t = gbytes / (peaks["hbm_gbs"] * 1e9)
@@ -324,13 +361,14 @@ def run_mine(args, world, rank, local):
                        "parallelism": f"replicas{world}",
                        "l2": "inputs larger than L2 (expert weights read each step exceed 126 MB)"},
             "tflops": tflops, "tflops_frac_of_bf16_peak": tflops / peaks["bf16_tflops"],
-            "stage_ms": {"router": stage_ms[0], "gating": stage_ms[1], "align_scatter": stage_ms[2],
-                         "expert_gemm": stage_ms[3]},
+            "stage_ms": dict(zip(MoELayer.STAGES, stage_ms)),
             "routing": stats, "roofline": roof,
             "e2e": {"value": world * w.T / (e2e_ms * 1e-3), "unit": UNIT,
                     "h2d_bytes_per_step": w.T * w.H * 2, "d2h_bytes_per_step": w.T * w.H * 4},
-            "gpu_launches": 4 * args.steps,
+            "gpu_launches": len(MoELayer.STAGES) * args.steps,
             "clocks": clk.summary()}
+    if not args.no_trace:
+        line["scheduler"] = traced_forward(w, wts, x, out)
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, wts, x)
     layer.close()

@@ -7,15 +7,18 @@
  *     x' = W_shared(x) + sum_{e in top-k(x)} w_e * W_down^e * SwiGLU(W_up^e x, W_gate^e x),
  *     SwiGLU(u, g) = SiLU(u) (.) g.
  *
- * It runs as four stream-ordered kernels with no host synchronisation and no allocation:
+ * It runs as six stream-ordered kernels with no host synchronisation and no allocation:
  *   1. router projection  logits = x W_router^T (+ bias)     tcgen05 GEMM, fp32 out
  *   2. gating             warp-level top-k + renormalised softmax, per-chunk expert
  *                         histogram, and (last CTA) the expert/block/tile scans
- *   3. align scatter      grid-wide writes of sorted_ids / expert_ids (+ zeroing of out)
- *   4. expert GEMMs       one persistent kernel; its CTAs claim (expert, m-tile, n-tile)
+ *   3. align scatter      grid-wide writes of sorted_ids / expert_ids and each slot's row
+ *   4. row gather         x rows copied into expert-tile order
+ *   5. expert GEMMs       one persistent kernel; its CTAs claim (expert, m-tile, n-tile)
  *                         tasks from an atomic counter (Weave blog, sections 2.1-2.2):
- *                         up/gate GEMM with SwiGLU in the epilogue, then down GEMM with
- *                         the router-weighted combine in the epilogue.
+ *                         up/gate GEMM with SwiGLU in the epilogue, then down GEMM whose
+ *                         epilogue applies the router weight to each slot's row
+ *   6. combine            per token, the shared row plus its k weighted slot rows, summed
+ *                         in slot order (deterministic)
  *
  * Conventions for every entry point below
  *  - Tensors are dense, row-major and contiguous. "bf16" buffers hold IEEE bfloat16 values
@@ -176,9 +179,10 @@ MOE_API int moe_debug_outputs(moe_handle *h, float *logits, int32_t *topk_ids, f
 
 /* Mean durations in milliseconds of the kernels of the forwards recorded since the previous
  * call (the first 256 of them; needs MOE_FLAG_STAGE_TIMING; synchronises, then starts a new
- * recording window): ms[0] router, ms[1] gating, ms[2] align scatter, ms[3] expert GEMMs.
- * n = entries of ms (up to 4). Each duration is measured with CUDA events recorded on the
- * forward's stream around the kernel. MOE_ERR_NOT_READY when nothing was recorded. */
+ * recording window): ms[0] router, ms[1] gating, ms[2] align scatter, ms[3] row gather,
+ * ms[4] expert GEMMs, ms[5] combine. n = entries of ms (up to 6). Each duration is measured
+ * with CUDA events recorded on the forward's stream around the kernel. MOE_ERR_NOT_READY
+ * when nothing was recorded. */
 MOE_API int moe_stage_times(moe_handle *h, float *ms, int32_t n);
 
 /* Handle facts: which = 0 SM count, 1 persistent-kernel CTAs, 2 workspace bytes,

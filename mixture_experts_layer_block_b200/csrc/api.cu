@@ -46,6 +46,7 @@ struct MapEntry {
 constexpr int64_t kDefaultTimeoutNs = 2000000000LL;
 constexpr size_t kMapCacheMax = 64;
 constexpr int kTimingRing = 256;  // forwards whose kernel durations moe_stage_times averages
+constexpr int kNumStages = 6;     // router, gating, align scatter, row gather, expert GEMMs, combine
 
 // Dynamic shared memory limit already granted to the gating kernels (shared by all handles).
 size_t g_gate_smem_granted = 0;
@@ -64,8 +65,9 @@ struct moe_handle {
   size_t gate_smem = 0;
   EncodeTiledFn encode = nullptr;
   std::vector<MapEntry> cache;
-  CUtensorMap h_routed{}, h_shared{};
-  std::vector<cudaEvent_t> ev;  // kTimingRing x 5 events (router, gate, scatter, gemm, end)
+  CUtensorMap h_routed{}, h_shared{}, xs_map{}, y_map{};
+  int max_routed_tiles = 0;
+  std::vector<cudaEvent_t> ev;  // kTimingRing x (kNumStages + 1) events around the kernels
   int timed = 0;                // forwards recorded since the last moe_stage_times
   bool timing = false;
   cudaStream_t last_stream = nullptr;
@@ -82,12 +84,13 @@ namespace {
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int encode_map(moe_handle* h, CUtensorMap* out, const void* ptr, uint64_t inner, uint64_t outer,
-               uint64_t stride_bytes, uint32_t box0, uint32_t box1) {
+               uint64_t stride_bytes, uint32_t box0, uint32_t box1,
+               CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {stride_bytes};
   cuuint32_t box[2] = {box0, box1};
   cuuint32_t es[2] = {1, 1};
-  CUresult r = h->encode(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims,
+  CUresult r = h->encode(out, dtype, 2, const_cast<void*>(ptr), dims,
                          strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
@@ -217,7 +220,8 @@ int moe_init(const moe_config* cfg, moe_handle** out) {
   const int E = c.num_experts;
   h->sorted_len_max = sorted_len_max;
   h->blocks_len_max = ceil_div((int)sorted_len_max, c.block_m);
-  h->max_tiles = (int)(ceil_div((int)S_max, kBM) + E + (c.inter_shared > 0 ? ceil_div(c.max_tokens, kBM) : 0));
+  h->max_routed_tiles = ceil_div((int)S_max, kBM) + E;
+  h->max_tiles = h->max_routed_tiles + (c.inter_shared > 0 ? ceil_div(c.max_tokens, kBM) : 0);
   h->max_lag = 2 * h->num_sms;
   h->max_units = h->max_tiles + h->max_lag;
   const int ldh = std::max(c.inter, c.inter_shared);
@@ -247,6 +251,10 @@ int moe_init(const moe_config* cfg, moe_handle** out) {
       {(void**)&w.unit_start, (size_t)(h->max_units + 1) * 4},
       {(void**)&w.done1, (size_t)h->max_tiles * 4},
       {(void**)&w.h, (size_t)h->max_tiles * kBM * ldh * 2},
+      {(void**)&w.expert_tile0, E_ * 4},
+      {(void**)&w.row_of_slot, (size_t)S_max * 4},
+      {(void**)&w.xs, (size_t)h->max_routed_tiles * kBM * c.hidden * 2},
+      {(void**)&w.y, (size_t)h->max_tiles * kBM * c.hidden * 4},
       {(void**)&w.trace, (size_t)trace_cap * 4 * 8},
       {(void**)&h->x_stage, (c.flags & MOE_FLAG_HOST_STAGING) ? T_ * c.hidden * 2 : 0},
       {(void**)&h->out_stage, (c.flags & MOE_FLAG_HOST_STAGING) ? T_ * c.hidden * 4 : 0},
@@ -276,6 +284,12 @@ int moe_init(const moe_config* cfg, moe_handle** out) {
   } else {
     h->h_shared = h->h_routed;
   }
+  if ((rc = encode_map(h, &h->xs_map, w.xs, c.hidden, (uint64_t)h->max_routed_tiles * kBM,
+                       (uint64_t)c.hidden * 2, kBK, kBM)))
+    return fail(rc);
+  if ((rc = encode_map(h, &h->y_map, w.y, c.hidden, h_rows, (uint64_t)c.hidden * 4, 32, kBM,
+                       CU_TENSOR_MAP_DATA_TYPE_FLOAT32)))
+    return fail(rc);
 
   // kernel attributes
   Shape sh = make_shape(h, c.max_tokens, c.top_k);
@@ -286,7 +300,7 @@ int moe_init(const moe_config* cfg, moe_handle** out) {
   }
   if (check_cuda(configure_router_kernel()) || check_cuda(configure_gemm_kernel())) return fail(MOE_ERR_CUDA);
   if (h->timing) {
-    h->ev.assign((size_t)kTimingRing * 5, nullptr);
+    h->ev.assign((size_t)kTimingRing * (kNumStages + 1), nullptr);
     for (auto& e : h->ev)
       if (cudaEventCreate(&e) != cudaSuccess) return fail(MOE_ERR_CUDA);
   }
@@ -355,11 +369,12 @@ static int forward_impl(moe_handle* h, const void* x, int32_t T, const void* w_r
   const Workspace& w = h->ws;
 
   // tensor maps
-  CUtensorMap x_router, wr_map;
+  CUtensorMap wr_map;
   GemmMaps maps;
   const int bn = router_bn(E);
-  if ((rc = encode_map(h, &x_router, x, H, T, (uint64_t)H * 2, kBK, kBM))) return rc;
-  if ((rc = encode_map(h, &maps.x_gather, x, H, T, (uint64_t)H * 2, kBK, 1))) return rc;
+  if ((rc = encode_map(h, &maps.x_tile, x, H, T, (uint64_t)H * 2, kBK, kBM))) return rc;
+  maps.xs = h->xs_map;
+  maps.y = h->y_map;
   if ((rc = cached_map(h, &wr_map, w_router, H, E, (uint64_t)H * 2, kBK, bn))) return rc;
   if ((rc = cached_map(h, &maps.w_up, w_up, H, (uint64_t)E * D, (uint64_t)H * 2, kBK, kBN1))) return rc;
   if ((rc = cached_map(h, &maps.w_gate, w_gate, H, (uint64_t)E * D, (uint64_t)H * 2, kBK, kBN1))) return rc;
@@ -378,21 +393,27 @@ static int forward_impl(moe_handle* h, const void* x, int32_t T, const void* w_r
   }
 
   cudaEvent_t* ev = nullptr;
-  if (h->timing && h->timed < kTimingRing) ev = &h->ev[(size_t)h->timed++ * 5];
-  if (ev && cudaEventRecord(ev[0], st) != cudaSuccess) return MOE_ERR_CUDA;
-  if ((rc = check_cuda(launch_router(x_router, wr_map, router_bias, w.logits, T, E, H, bn, w.meta,
+  if (h->timing && h->timed < kTimingRing) ev = &h->ev[(size_t)h->timed++ * (kNumStages + 1)];
+  auto mark = [&](int i) { return (ev && cudaEventRecord(ev[i], st) != cudaSuccess) ? MOE_ERR_CUDA : MOE_OK; };
+  const uint16_t* x16 = static_cast<const uint16_t*>(x);
+  if ((rc = mark(0))) return rc;
+  if ((rc = check_cuda(launch_router(maps.x_tile, wr_map, router_bias, w.logits, T, E, H, bn, w.meta,
                                      h->timeout_ns, st))))
     return rc;
-  if (ev && cudaEventRecord(ev[1], st) != cudaSuccess) return MOE_ERR_CUDA;
+  if ((rc = mark(1))) return rc;
   if ((rc = check_cuda(launch_gate(w.logits, w.topk_ids, w.topk_w, w, sh, true, true, h->gate_smem, st))))
     return rc;
-  if (ev && cudaEventRecord(ev[2], st) != cudaSuccess) return MOE_ERR_CUDA;
-  if ((rc = check_cuda(launch_scatter(w.topk_ids, w.sorted_ids, w.expert_ids, nullptr, out,
-                                      (int64_t)T * H / 4, w, sh, 2 * h->num_sms, st))))
+  if ((rc = mark(2))) return rc;
+  if ((rc = check_cuda(launch_scatter(w.topk_ids, w.sorted_ids, w.expert_ids, nullptr, w.row_of_slot, w,
+                                      sh, 2 * h->num_sms, st))))
     return rc;
-  if (ev && cudaEventRecord(ev[3], st) != cudaSuccess) return MOE_ERR_CUDA;
-  if ((rc = check_cuda(launch_moe_gemm(maps, w, sh, out, h->num_sms, st)))) return rc;
-  if (ev && cudaEventRecord(ev[4], st) != cudaSuccess) return MOE_ERR_CUDA;
+  if ((rc = mark(3))) return rc;
+  if ((rc = check_cuda(launch_gather_rows(x16, w, sh, 4 * h->num_sms, st)))) return rc;
+  if ((rc = mark(4))) return rc;
+  if ((rc = check_cuda(launch_moe_gemm(maps, w, sh, h->num_sms, st)))) return rc;
+  if ((rc = mark(5))) return rc;
+  if ((rc = check_cuda(launch_combine(out, w, sh, st)))) return rc;
+  if ((rc = mark(6))) return rc;
   return MOE_OK;
 }
 
@@ -488,8 +509,8 @@ int moe_align_block_size(moe_handle* h, const int32_t* topk_ids, int32_t T, int3
   h->last_stream = st;
   const Shape sh = make_shape(h, T, top_k);
   if ((rc = check_cuda(launch_hist(topk_ids, h->ws, sh, h->gate_smem, st)))) return rc;
-  return check_cuda(launch_scatter(topk_ids, sorted_ids, expert_ids, num_post_padded, nullptr, 0,
-                                   h->ws, sh, 2 * h->num_sms, st));
+  return check_cuda(launch_scatter(topk_ids, sorted_ids, expert_ids, num_post_padded, nullptr, h->ws, sh,
+                                   2 * h->num_sms, st));
 }
 
 int moe_debug_outputs(moe_handle* h, float* logits, int32_t* topk_ids, float* topk_w,
@@ -519,13 +540,14 @@ int moe_stage_times(moe_handle* h, float* ms, int32_t n) {
   if (!h || !ms || n < 1) return MOE_ERR_INVALID_ARG;
   if (!h->timing || h->timed == 0) return MOE_ERR_NOT_READY;
   const int m = h->timed;
+  const size_t K = kNumStages + 1;
   h->timed = 0;
-  for (int i = 0; i < std::min(n, 4); ++i) ms[i] = 0.f;
-  if (cudaEventSynchronize(h->ev[(size_t)(m - 1) * 5 + 4]) != cudaSuccess) return MOE_ERR_CUDA;
+  for (int i = 0; i < std::min(n, kNumStages); ++i) ms[i] = 0.f;
+  if (cudaEventSynchronize(h->ev[(size_t)(m - 1) * K + kNumStages]) != cudaSuccess) return MOE_ERR_CUDA;
   for (int f = 0; f < m; ++f)
-    for (int i = 0; i < std::min(n, 4); ++i) {
+    for (int i = 0; i < std::min(n, kNumStages); ++i) {
       float t = 0.f;
-      if (cudaEventElapsedTime(&t, h->ev[(size_t)f * 5 + i], h->ev[(size_t)f * 5 + i + 1]) != cudaSuccess)
+      if (cudaEventElapsedTime(&t, h->ev[(size_t)f * K + i], h->ev[(size_t)f * K + i + 1]) != cudaSuccess)
         return MOE_ERR_CUDA;
       ms[i] += t / m;
     }

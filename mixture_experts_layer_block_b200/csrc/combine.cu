@@ -1,0 +1,84 @@
+// combine.cu -- the two memory-bound steps around the expert GEMMs.
+//
+// gather_rows_kernel: copies every kept slot's token row x[t] into the tile-ordered buffer
+//   xs (row = first tile of its expert * 128 + its rank in the expert), so that the up/gate
+//   GEMM reads its A operand as plain 128-row TMA boxes. One warp per slot, 16-byte vectors.
+//
+// combine_kernel: the sum over experts of the Mixture-of-Kittens layer equation
+//   x' = W_shared(x) + sum_{e in top-k} w_e (W_down^e SwiGLU(...)).
+//   The down-GEMM epilogue already wrote w_s * (W_down^e h_s) for every kept slot s into its
+//   tile row of y (fp32); this kernel adds, per token, the shared-expert row first and then
+//   the slots j = 0..k-1 in order (dropped slots skipped), in fp32. The order is fixed, so
+//   the result does not depend on the schedule. One warp per (token, 128 columns).
+#include <algorithm>
+
+#include "launch.h"
+
+namespace moe {
+
+__global__ void __launch_bounds__(256)
+    gather_rows_kernel(const uint16_t* __restrict__ x, Workspace ws, Shape sh) {
+  const int lane = threadIdx.x & 31;
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int nw = (gridDim.x * blockDim.x) >> 5;
+  const int S = sh.T * sh.k;
+  const int nvec = sh.H / 8;  // 16-byte vectors per row (H is a multiple of 8)
+  for (int s = gw; s < S; s += nw) {
+    const int row = __ldcg(ws.row_of_slot + s);
+    if (row < 0) continue;
+    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)(s / sh.k) * sh.H);
+    uint4* dst = reinterpret_cast<uint4*>(ws.xs + (size_t)row * sh.H);
+    int i = lane;
+    for (; i + 96 < nvec; i += 128) {
+      const uint4 a = __ldg(src + i), b = __ldg(src + i + 32), c = __ldg(src + i + 64),
+                  d = __ldg(src + i + 96);
+      dst[i] = a;
+      dst[i + 32] = b;
+      dst[i + 64] = c;
+      dst[i + 96] = d;
+    }
+    for (; i < nvec; i += 32) dst[i] = __ldg(src + i);
+  }
+}
+
+__global__ void __launch_bounds__(256)
+    combine_kernel(float* __restrict__ out, Workspace ws, Shape sh) {
+  const int lane = threadIdx.x & 31;
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int nw = (gridDim.x * blockDim.x) >> 5;
+  const int nch = ceil_div(sh.H, 128);
+  const int Mr = __ldcg(&ws.meta->num_routed_tiles);
+  const int64_t total = (int64_t)sh.T * nch;
+  for (int64_t w = gw; w < total; w += nw) {
+    const int t = (int)(w / nch);
+    const int c = (int)(w % nch) * 128 + lane * 4;
+    if (c >= sh.H) continue;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (sh.Ds > 0) {
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(ws.y + ((size_t)Mr * kBM + t) * sh.H + c));
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    for (int j = 0; j < sh.k; ++j) {
+      const int row = __ldcg(ws.row_of_slot + (size_t)t * sh.k + j);
+      if (row < 0) continue;
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(ws.y + (size_t)row * sh.H + c));
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    *reinterpret_cast<float4*>(out + (size_t)t * sh.H + c) = acc;
+  }
+}
+
+cudaError_t launch_gather_rows(const uint16_t* x, const Workspace& ws, const Shape& sh, int grid,
+                               cudaStream_t stream) {
+  gather_rows_kernel<<<grid, 256, 0, stream>>>(x, ws, sh);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(float* out, const Workspace& ws, const Shape& sh, cudaStream_t stream) {
+  const int64_t warps = (int64_t)sh.T * ceil_div(sh.H, 128);
+  const int grid = (int)std::min<int64_t>((warps + 7) / 8, 148 * 32);
+  combine_kernel<<<grid, 256, 0, stream>>>(out, ws, sh);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -20,6 +20,8 @@ constexpr int kABytes = kBM * kBK * 2;       // 16 KB
 constexpr int kBBytes = kUmmaN * kBK * 2;    // 32 KB
 constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kTaskSlots = 4;   // depth of the producer -> MMA/epilogue task ring
+constexpr int kStagingBytes = 128 * 128;  // one epilogue staging buffer: 128 rows x 128 B
+constexpr int kNumStaging = 2;            // double-buffered epilogue -> TMA store staging
 constexpr int kAccCols = 256;   // TMEM columns per accumulator buffer (2 buffers)
 constexpr int kGemmThreads = 192;  // warp 0 producer, warp 1 MMA, warps 2-5 epilogue
 
@@ -59,7 +61,8 @@ struct DeviceMeta {
   int num_units;      // scheduling units (tiles + lag)
   int P;              // num_post_padded
   int trace_count;    // trace records written
-  int pad[7];
+  int num_routed_tiles;  // m-tiles of routed experts (shared-expert tiles follow them)
+  int pad[6];
 };
 
 // Task kinds in the ring.
@@ -95,7 +98,11 @@ struct Workspace {
   int32_t* tile_nrows;   // [max_tiles]
   int32_t* unit_start;   // [max_tiles + max_lag + 1]
   int32_t* done1;        // [max_tiles]      finished up/gate tasks per tile
+  int32_t* expert_tile0; // [E]              first m-tile of each expert
+  int32_t* row_of_slot;  // [S]              tile row (tile*128 + r) of each kept slot, -1 if dropped
+  uint16_t* xs;          // [max_routed_tiles*128][H] bf16 x rows gathered in tile order
   uint16_t* h;           // [max_tiles*128][ldh] bf16 SwiGLU activations
+  float* y;              // [max_tiles*128][H] fp32 router-weighted expert outputs per tile row
   int64_t* trace;        // [trace_cap][4]
   int32_t trace_cap;
   int32_t ldh;           // row stride of h in elements (max(D, D_shared))

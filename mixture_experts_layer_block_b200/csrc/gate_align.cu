@@ -188,6 +188,7 @@ __device__ void align_scans(const Workspace& ws, const Shape& sh, bool tiles, in
   for (int e = tid; e < E; e += blockDim.x) {
     const int first = buf[e], nt = ceil_div(kept[e], kBM);
     const int off = ws.expert_off[e];
+    ws.expert_tile0[e] = first;
     for (int i = 0; i < nt; ++i) {
       ws.tile_expert[first + i] = e;
       ws.tile_row0[first + i] = off + i * kBM;
@@ -220,6 +221,7 @@ __device__ void align_scans(const Workspace& ws, const Shape& sh, bool tiles, in
   if (tid == 0) {
     ws.unit_start[U] = total;
     ws.meta->num_tiles = Mt;
+    ws.meta->num_routed_tiles = Mr;
     ws.meta->num_units = U;
     ws.meta->total_tasks = total;
     ws.meta->task_counter = 0;
@@ -303,18 +305,23 @@ __device__ __forceinline__ int segment_of(const int* off, int E, int i) {
   return lo;
 }
 
-// smem: off[E+1] | kept[E] | per-warp counters [8][E]
+// smem: off[E+1] | kept[E] | tile0[E] | per-warp counters [8][E]
+// With `row_of_slot` non-null, also records for every slot its row in the tile-ordered
+// buffers (first tile of its expert * 128 + its rank), or -1 when the slot was dropped.
 __global__ void __launch_bounds__(256)
     scatter_kernel(const int32_t* __restrict__ topk_ids, int32_t* __restrict__ sorted_ids,
                    int32_t* __restrict__ expert_ids, int32_t* __restrict__ num_post_padded,
-                   float* __restrict__ out_zero, int64_t n4, Workspace ws, Shape sh) {
+                   int32_t* __restrict__ row_of_slot, Workspace ws, Shape sh) {
   extern __shared__ int smem_i[];
   const int E = sh.E;
   int* off = smem_i;
   int* kept = off + E + 1;
-  int* cnt_all = kept + E;
+  int* tile0 = kept + E;
+  int* cnt_all = tile0 + E;
   for (int e = threadIdx.x; e <= E; e += blockDim.x) off[e] = __ldcg(ws.expert_off + e);
   for (int e = threadIdx.x; e < E; e += blockDim.x) kept[e] = __ldcg(ws.expert_kept + e);
+  if (row_of_slot)
+    for (int e = threadIdx.x; e < E; e += blockDim.x) tile0[e] = __ldcg(ws.expert_tile0 + e);
   __syncthreads();
   const int P = off[E];
   const int S = sh.T * sh.k;
@@ -340,8 +347,12 @@ __global__ void __launch_bounds__(256)
       __syncwarp();
       if (valid) {
         const int r = c0 + rank;
-        if (sh.capacity == 0 || r < sh.capacity) sorted_ids[off[e] + r] = s;
+        const bool keep = sh.capacity == 0 || r < sh.capacity;
+        if (keep) sorted_ids[off[e] + r] = s;
+        if (row_of_slot) row_of_slot[s] = keep ? tile0[e] * kBM + r : -1;
         if (rank == 0) cnt[e] = c0 + __popc(mask);
+      } else if (row_of_slot && s < s1) {
+        row_of_slot[s] = -1;  // an expert id outside [0, E)
       }
       __syncwarp();
     }
@@ -363,12 +374,6 @@ __global__ void __launch_bounds__(256)
     expert_ids[b] = (i < P) ? segment_of(off, E, i) : -1;
   }
   if (gt == 0 && num_post_padded) *num_post_padded = P;
-
-  // (d) zero the layer output (the expert GEMMs accumulate into it)
-  if (out_zero) {
-    float4* o4 = reinterpret_cast<float4*>(out_zero);
-    for (int64_t i = gt; i < n4; i += nt) o4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-  }
 }
 
 // ------------------------------------------------------------------------------------------
@@ -379,7 +384,7 @@ size_t gate_smem_bytes(const Shape& sh, int max_units) {
   return sizeof(int) * (size_t)(sh.E /*hist*/ + 64 + 2 * sh.E + buf);
 }
 
-size_t scatter_smem_bytes(int E) { return sizeof(int) * (size_t)(E + 1 + E + 8 * E); }
+size_t scatter_smem_bytes(int E) { return sizeof(int) * (size_t)(E + 1 + 2 * E + 8 * E); }
 
 template <int VPL>
 static cudaError_t launch_gate_vpl(const float* logits, int32_t* ids, float* w, const Workspace& ws,
@@ -408,10 +413,10 @@ cudaError_t launch_hist(const int32_t* topk_ids, const Workspace& ws, const Shap
 }
 
 cudaError_t launch_scatter(const int32_t* topk_ids, int32_t* sorted_ids, int32_t* expert_ids,
-                           int32_t* num_post_padded, float* out_zero, int64_t n4,
-                           const Workspace& ws, const Shape& sh, int grid, cudaStream_t st) {
+                           int32_t* num_post_padded, int32_t* row_of_slot, const Workspace& ws,
+                           const Shape& sh, int grid, cudaStream_t st) {
   scatter_kernel<<<grid, 256, scatter_smem_bytes(sh.E), st>>>(topk_ids, sorted_ids, expert_ids,
-                                                              num_post_padded, out_zero, n4, ws, sh);
+                                                              num_post_padded, row_of_slot, ws, sh);
   return cudaGetLastError();
 }
 

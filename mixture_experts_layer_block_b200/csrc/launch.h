@@ -9,7 +9,9 @@ namespace moe {
 
 // Tensor maps of the persistent expert-GEMM kernel.
 struct alignas(64) GemmMaps {
-  CUtensorMap x_gather;  // x [T][H], box {64, 1} (row gather)
+  CUtensorMap x_tile;    // x [T][H], box {64, 128} (shared-expert tiles)
+  CUtensorMap xs;        // gathered rows [routed_rows][H], box {64, 128}
+  CUtensorMap y;         // y [rows][H] fp32, box {32, 128} (store)
   CUtensorMap w_up;      // [E*D][H], box {64, 128}
   CUtensorMap w_gate;    // [E*D][H], box {64, 128}
   CUtensorMap w_down;    // [E*H][D], box {64, 256}
@@ -36,16 +38,23 @@ cudaError_t launch_gate(const float* logits, int32_t* topk_ids, float* topk_w, c
 cudaError_t launch_hist(const int32_t* topk_ids, const Workspace& ws, const Shape& sh, size_t smem,
                         cudaStream_t stream);
 
-// Grid-wide align writes, plus zeroing of `out_zero` (n4 float4s) when non-null.
+// Grid-wide align writes (and the tile row of every slot when row_of_slot is non-null).
 size_t scatter_smem_bytes(int E);
 cudaError_t launch_scatter(const int32_t* topk_ids, int32_t* sorted_ids, int32_t* expert_ids,
-                           int32_t* num_post_padded, float* out_zero, int64_t n4,
-                           const Workspace& ws, const Shape& sh, int grid, cudaStream_t stream);
+                           int32_t* num_post_padded, int32_t* row_of_slot, const Workspace& ws,
+                           const Shape& sh, int grid, cudaStream_t stream);
+
+// Copy each kept slot's x row into the tile-ordered buffer ws.xs.
+cudaError_t launch_gather_rows(const uint16_t* x, const Workspace& ws, const Shape& sh, int grid,
+                               cudaStream_t stream);
+
+// out[t] = (shared row of t) + sum_j y[row_of_slot[t*k+j]], in that order, fp32.
+cudaError_t launch_combine(float* out, const Workspace& ws, const Shape& sh, cudaStream_t stream);
 
 // Persistent expert GEMMs.
 size_t gemm_smem_bytes();
-cudaError_t launch_moe_gemm(const GemmMaps& maps, const Workspace& ws, const Shape& sh, float* out,
-                            int grid, cudaStream_t stream);
+cudaError_t launch_moe_gemm(const GemmMaps& maps, const Workspace& ws, const Shape& sh, int grid,
+                            cudaStream_t stream);
 
 // One-time kernel attribute setup (dynamic shared memory limits).
 cudaError_t configure_kernels(size_t gate_smem);

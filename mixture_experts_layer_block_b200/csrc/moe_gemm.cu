@@ -3,20 +3,25 @@
 // What it computes (Mixture-of-Kittens blog, "Overlapping compute and communication in
 // MoE"): for every kept slot s = (t, j) routed to expert e,
 //     h_s  = SiLU(W_up^e x_t) (.) (W_gate^e x_t)                   (bf16, kept in HBM/L2)
-//     out_t += w_s * W_down^e h_s                                  (fp32 reduction)
+//     y_s   = w_s * W_down^e h_s                                   (fp32, per slot row)
 // plus the shared expert over every token with weight 1.
 //
 // How (Weave blog, sections 2.1-2.2 and 5.1: tile decomposition, an atomic task counter,
 // one persistent CTA per SM that claims tasks until the queue is empty):
 //  - m-tile: up to 128 sorted rows of one expert (align output), or 128 tokens of the
 //    shared expert.
-//  - up task   (tile, n): A = the tile's x rows, gathered with TMA tile::gather4 from the
-//    sorted slot ids; B = 128 rows of W_up^e stacked on 128 rows of W_gate^e; one
-//    tcgen05.mma of N = 256 per K step, so TMEM holds U | G; the epilogue writes
-//    h = SiLU(U) * G (bf16) for columns n*128 .. n*128+127 and counts the tile's done1.
+//  - up task   (tile, n): A = the tile's 128 x rows (pre-gathered in tile order into xs by
+//    the gather kernel; shared-expert tiles read x directly); B = 128 rows of W_up^e stacked
+//    on 128 rows of W_gate^e; one tcgen05.mma of N = 256 per K step, so TMEM holds U | G; the
+//    epilogue writes h = SiLU(U) * G (bf16) for columns n*128 .. n*128+127 and counts the
+//    tile's done1.
 //  - down task (tile, n): waits until done1[tile] covers every up task of the tile (bounded
 //    spin), then A = the tile's h rows, B = 256 rows of W_down^e; the epilogue scales each
-//    row by its router weight and adds it into out[token] (fp32 vector atomics).
+//    row by its router weight and writes it (fp32) to the tile's rows of y. The combine
+//    kernel sums each token's rows in slot order.
+//  - epilogue results go through two 16 KB shared-memory staging buffers (128-byte swizzled)
+//    and asynchronous TMA tensor stores, so the epilogue warps release TMEM and move on
+//    while the stores drain.
 //  - task ids are numbered in units: unit u = up tasks of tile u, then down tasks of tile
 //    u - lag. A down task's dependencies always have smaller ids, and claims are monotone,
 //    so the earliest unfinished task can always make progress (no deadlock).
@@ -34,7 +39,8 @@ namespace moe {
 namespace {
 
 struct SmemLayout {
-  static constexpr int kBarOff = kStages * kStageBytes;
+  static constexpr int kStagingOff = kStages * kStageBytes;
+  static constexpr int kBarOff = kStagingOff + kNumStaging * kStagingBytes;
   // barriers: full[S], empty[S], acc_full[2], acc_empty[2], task_full[R], task_empty[R], drain
   static constexpr int kNumBars = 2 * kStages + 4 + 2 * kTaskSlots + 1;
   static constexpr int kRingOff = kBarOff + ((kNumBars * 8 + 63) & ~63);
@@ -65,8 +71,7 @@ __device__ __noinline__ bool wait_count(const int* p, int need, DeviceMeta* meta
 }  // namespace
 
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    moe_gemm_kernel(const __grid_constant__ GemmMaps maps, Workspace ws, Shape sh,
-                    float* __restrict__ out) {
+    moe_gemm_kernel(const __grid_constant__ GemmMaps maps, Workspace ws, Shape sh) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SmemLayout::kBarOff);
@@ -101,7 +106,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     mbar_init(drain, 1);
     *s_abort = 0;
     fence_mbar_init();
-    tma_prefetch_desc(&maps.x_gather);
+    tma_prefetch_desc(&maps.xs);
+    tma_prefetch_desc(&maps.y);
     tma_prefetch_desc(&maps.w_up);
     tma_prefetch_desc(&maps.w_gate);
     tma_prefetch_desc(&maps.w_down);
@@ -189,38 +195,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         if (!ok) break;
       }
-      // x rows of the up task: lane l gathers rows 4l..4l+3; rows past nrows repeat row 0
-      // (their results are never read)
-      int r[4] = {0, 0, 0, 0};
-      if (t.kind == kTaskUp) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int row = lane * 4 + i;
-          const int rr = row < t.nrows ? row : 0;
-          r[i] = shared ? (t.row0 + rr) : (__ldcg(&ws.sorted_ids[t.row0 + rr]) / sh.k);
-        }
-      }
       const int wrow_up = shared ? t.n0 : t.expert * sh.D + t.n0;
       const int wrow_dn = shared ? t.n0 : t.expert * sh.H + t.n0;
       for (int kb = 0; kb < t.nk; ++kb) {
         if (lane == 0) ok = wait_bar(&empty[stage], phase ^ 1, meta, s_abort, limit, kSiteProducerEmpty);
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         if (!ok) break;
-        const uint32_t a = smem_u32(smem + stage * kStageBytes);
-        const uint32_t b = a + kABytes;
-        if (lane == 0) mbar_arrive_expect_tx(&full[stage], kStageBytes);
-        __syncwarp();
-        if (t.kind == kTaskUp) {
-          tma_gather4(a + lane * 512, &maps.x_gather, &full[stage], kb * kBK, r[0], r[1], r[2], r[3]);
-          if (lane == 0) {
+        if (lane == 0) {
+          const uint32_t a = smem_u32(smem + stage * kStageBytes);
+          const uint32_t b = a + kABytes;
+          mbar_arrive_expect_tx(&full[stage], kStageBytes);
+          if (t.kind == kTaskUp) {
+            // A: 128 rows of x in tile order (routed: gathered copy; shared: the tokens)
+            if (shared) tma_load_2d(a, &maps.x_tile, &full[stage], kb * kBK, t.row0);
+            else tma_load_2d(a, &maps.xs, &full[stage], kb * kBK, t.tile * kBM);
             tma_load_2d(b, shared ? &maps.ws_up : &maps.w_up, &full[stage], kb * kBK, wrow_up);
             tma_load_2d(b + kBN1 * 128, shared ? &maps.ws_gate : &maps.w_gate, &full[stage], kb * kBK,
                         wrow_up);
+          } else {
+            tma_load_2d(a, shared ? &maps.h_shared : &maps.h_routed, &full[stage], kb * kBK, t.tile * kBM);
+            tma_load_2d(b, shared ? &maps.ws_down : &maps.w_down, &full[stage], kb * kBK, wrow_dn);
           }
-        } else if (lane == 0) {
-          tma_load_2d(a, shared ? &maps.h_shared : &maps.h_routed, &full[stage], kb * kBK, t.tile * kBM);
-          tma_load_2d(b, shared ? &maps.ws_down : &maps.w_down, &full[stage], kb * kBK, wrow_dn);
         }
+        __syncwarp();
         ++nfill;
         if (++stage == kStages) { stage = 0; phase ^= 1; }
       }
@@ -262,9 +259,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncwarp();
   } else {
     // ===================================== epilogue =====================================
+    // Each thread owns one tile row (its TMEM lane). Per chunk of 128 bytes per row: drain
+    // TMEM to registers, convert, write the row into a 128-byte-swizzled staging buffer, and
+    // let one thread issue the TMA store of the 128-row box.
     const int q = warp & 3;          // TMEM lane quarter this warp may read
     const int row = q * 32 + lane;   // tile row owned by this thread
-    uint32_t slot = 0, slot_phase = 0, acc = 0, acc_phase = 0;
+    const bool leader = (warp == 2 && lane == 0);
+    uint8_t* staging = smem + SmemLayout::kStagingOff;
+    uint32_t slot = 0, slot_phase = 0, acc = 0, acc_phase = 0, sb = 0;
+    // write 8 x 16 bytes (one 128-byte row) into staging buffer `buf` with the 128B swizzle
+    auto put_row = [&](uint8_t* buf, const uint32_t (&w)[32]) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        *reinterpret_cast<uint4*>(buf + row * 128 + ((j ^ (row & 7)) << 4)) =
+            make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+    };
     while (true) {
       if (!wait_bar(&task_full[slot], slot_phase, meta, s_abort, limit, kSiteEpiTask)) break;
       const Task t = ring[slot];
@@ -274,78 +283,93 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint32_t tacc = tmem_base + acc * kAccCols + (static_cast<uint32_t>(q * 32) << 16);
       const bool shared = (t.expert == sh.E);
       if (t.kind == kTaskUp) {
-        const int Dt = shared ? sh.Ds : sh.D;
-        uint16_t* hrow = ws.h + (size_t)(t.tile * kBM + row) * ws.ldh;
+        // h = SiLU(U) * G, two chunks of 64 bf16 columns
 #pragma unroll 1
-        for (int c = 0; c < kBN1; c += 32) {
-          uint32_t u[32], g[32];
-          tmem_ld_32x32b_x32(tacc + c, u);
-          tmem_ld_32x32b_x32(tacc + kBN1 + c, g);
-          tmem_ld_wait();
-          uint32_t pk[16];
+        for (int cc = 0; cc < kBN1 / 64; ++cc) {
+          uint8_t* buf = staging + sb * kStagingBytes;
+          uint32_t pk[32];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float u0 = __uint_as_float(u[2 * j]), u1 = __uint_as_float(u[2 * j + 1]);
-            const float g0 = __uint_as_float(g[2 * j]), g1 = __uint_as_float(g[2 * j + 1]);
-            const float h0 = u0 / (1.0f + __expf(-u0)) * g0;
-            const float h1 = u1 / (1.0f + __expf(-u1)) * g1;
-            pk[j] = pack_bf16x2(h0, h1);
+          for (int half = 0; half < 2; ++half) {
+            uint32_t u[32], g[32];
+            tmem_ld_32x32b_x32(tacc + cc * 64 + half * 32, u);
+            tmem_ld_32x32b_x32(tacc + kBN1 + cc * 64 + half * 32, g);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const float u0 = __uint_as_float(u[2 * j]), u1 = __uint_as_float(u[2 * j + 1]);
+              const float g0 = __uint_as_float(g[2 * j]), g1 = __uint_as_float(g[2 * j + 1]);
+              pk[half * 16 + j] = pack_bf16x2(u0 / (1.0f + __expf(-u0)) * g0, u1 / (1.0f + __expf(-u1)) * g1);
+            }
           }
-          const int col = t.n0 + c;
-#pragma unroll
-          for (int v = 0; v < 4; ++v)
-            if (col + 8 * v + 8 <= Dt)
-              *reinterpret_cast<uint4*>(hrow + col + 8 * v) =
-                  make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          if (cc == kBN1 / 64 - 1) {  // every TMEM read of this task is done: release it
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[acc]);
+          }
+          if (leader) bulk_wait_group_read<kNumStaging - 1>();  // buffer sb no longer read
+          named_bar_sync(1, 128);
+          put_row(buf, pk);
+          fence_proxy_async_shared();
+          named_bar_sync(1, 128);
+          if (leader) {
+            tma_store_2d(shared ? &maps.h_shared : &maps.h_routed, smem_u32(buf), t.n0 + cc * 64,
+                         t.tile * kBM);
+            bulk_commit_group();
+          }
+          sb ^= 1;
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[acc]);
-        // publish h: this tile's down tasks read it with TMA (async proxy) on other SMs
-        fence_proxy_async_global();
-        __threadfence();
-        named_bar_sync(1, 128);
-        if (warp == 2 && lane == 0) red_release_add_gpu(&ws.done1[t.tile], 1);
+        // publish h: the stores must be complete and visible to other SMs' TMA loads before
+        // the tile's counter moves
+        if (leader) {
+          bulk_wait_group<0>();
+          fence_proxy_async_global();
+          __threadfence();
+          red_release_add_gpu(&ws.done1[t.tile], 1);
+        }
       } else {
-        const bool valid = row < t.nrows;
-        int tok = 0;
+        // y = w * (h W_down^T), eight chunks of 32 fp32 columns
         float w = 0.f;
-        if (valid) {
+        if (row < t.nrows) {
           if (shared) {
-            tok = t.row0 + row;
             w = 1.f;
           } else {
             const int s = __ldcg(&ws.sorted_ids[t.row0 + row]);
-            tok = s / sh.k;
             w = __ldcg(&ws.topk_w[s]);
           }
         }
-        float* orow = out + (size_t)tok * sh.H;
 #pragma unroll 1
-        for (int c = 0; c < kBN2; c += 32) {
+        for (int cc = 0; cc < kBN2 / 32; ++cc) {
+          uint8_t* buf = staging + sb * kStagingBytes;
           uint32_t v[32];
-          tmem_ld_32x32b_x32(tacc + c, v);
+          tmem_ld_32x32b_x32(tacc + cc * 32, v);
           tmem_ld_wait();
-          const int col = t.n0 + c;
-          if (valid) {
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-              if (col + 4 * j + 4 <= sh.H)
-                atomicAdd(reinterpret_cast<float4*>(orow + col + 4 * j),
-                          make_float4(w * __uint_as_float(v[4 * j]), w * __uint_as_float(v[4 * j + 1]),
-                                      w * __uint_as_float(v[4 * j + 2]), w * __uint_as_float(v[4 * j + 3])));
+          if (cc == kBN2 / 32 - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[acc]);
           }
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(w * __uint_as_float(v[j]));
+          if (leader) bulk_wait_group_read<kNumStaging - 1>();
+          named_bar_sync(1, 128);
+          put_row(buf, v);
+          fence_proxy_async_shared();
+          named_bar_sync(1, 128);
+          if (leader) {
+            tma_store_2d(&maps.y, smem_u32(buf), t.n0 + cc * 32, t.tile * kBM);
+            bulk_commit_group();
+          }
+          sb ^= 1;
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[acc]);
       }
       if (lane == 0) mbar_arrive(&task_empty[slot]);
-      if (ws.trace_cap > 0 && warp == 2 && lane == 0 && t.id < ws.trace_cap)
+      if (ws.trace_cap > 0 && leader && t.id < ws.trace_cap)
         ws.trace[(size_t)t.id * 4 + 3] = (int64_t)globaltimer_ns();
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }
       if (++slot == kTaskSlots) { slot = 0; slot_phase ^= 1; }
     }
+    // the staging buffers must not be released while a store still reads them
+    if (leader) bulk_wait_group<0>();
   }
 
   // teardown: every TMA fill and tcgen05 op issued by this CTA must be complete before the
@@ -366,9 +390,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
 size_t gemm_smem_bytes() { return (size_t)SmemLayout::kBytes + 1024; }
 
-cudaError_t launch_moe_gemm(const GemmMaps& maps, const Workspace& ws, const Shape& sh, float* out,
-                            int grid, cudaStream_t stream) {
-  moe_gemm_kernel<<<grid, kGemmThreads, gemm_smem_bytes(), stream>>>(maps, ws, sh, out);
+cudaError_t launch_moe_gemm(const GemmMaps& maps, const Workspace& ws, const Shape& sh, int grid,
+                            cudaStream_t stream) {
+  moe_gemm_kernel<<<grid, kGemmThreads, gemm_smem_bytes(), stream>>>(maps, ws, sh);
   return cudaGetLastError();
 }
 

@@ -11,7 +11,8 @@ import ctypes
 import os
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libmoe_b200.so")
+# MOE_B200_LIBRARY may name another build of the same library (for A/B timing of builds)
+LIB_PATH = os.environ.get("MOE_B200_LIBRARY") or os.path.join(_PKG, "libmoe_b200.so")
 
 MOE_OK = 0
 MOE_ERR_INVALID_ARG = -1
@@ -198,9 +199,11 @@ class MoELayer:
         rc = lib.moe_get_status(self.h, ctypes.byref(st))
         return rc, st.value
 
+    STAGES = ("router", "gating", "align_scatter", "row_gather", "expert_gemm", "combine")
+
     def stage_times(self):
-        ms = (ctypes.c_float * 4)()
-        check(lib.moe_stage_times(self.h, ms, 4), "moe_stage_times")
+        ms = (ctypes.c_float * 6)()
+        check(lib.moe_stage_times(self.h, ms, 6), "moe_stage_times")
         return list(ms)
 
     def query(self, which):
