@@ -14,7 +14,7 @@
 #include "moe_b200.h"
 
 namespace moe {
-cudaError_t configure_gate_kernels(size_t gate_smem);
+cudaError_t configure_gate_kernels(size_t gate_smem, size_t scatter_smem);
 cudaError_t configure_router_kernel();
 cudaError_t configure_gemm_kernel();
 }  // namespace moe
@@ -48,8 +48,9 @@ constexpr size_t kMapCacheMax = 64;
 constexpr int kTimingRing = 256;  // forwards whose kernel durations moe_stage_times averages
 constexpr int kNumStages = 6;     // router, gating, align scatter, row gather, expert GEMMs, combine
 
-// Dynamic shared memory limit already granted to the gating kernels (shared by all handles).
-size_t g_gate_smem_granted = 0;
+// Dynamic shared memory limits already granted to the gating and scatter kernels (shared by
+// all handles).
+size_t g_gate_smem_granted = 0, g_scatter_smem_granted = 0;
 
 }  // namespace
 
@@ -67,6 +68,7 @@ struct moe_handle {
   std::vector<MapEntry> cache;
   CUtensorMap h_routed{}, h_shared{}, xs_map{}, y_map{};
   int max_routed_tiles = 0;
+  int parts_rows = 0;  // rows of the K-split partial logits buffer
   std::vector<cudaEvent_t> ev;  // kTimingRing x (kNumStages + 1) events around the kernels
   int timed = 0;                // forwards recorded since the last moe_stage_times
   bool timing = false;
@@ -132,7 +134,9 @@ Shape make_shape(const moe_handle* h, int T, int k) {
   sh.k = k;
   sh.block_m = c.block_m;
   sh.capacity = capacity_of(c, T, k);
-  sh.chunk_tokens = std::max(kMinChunkTokens, ceil_div(std::max(T, 1), kMaxChunks));
+  // a chunk holds a whole number of gating CTAs (kGateTokensPerCta tokens each)
+  sh.chunk_tokens = ceil_div(std::max(kMinChunkTokens, ceil_div(std::max(T, 1), kMaxChunks)),
+                             kGateTokensPerCta) * kGateTokensPerCta;
   sh.num_chunks = std::max(1, ceil_div(T, sh.chunk_tokens));
   sh.sorted_len = T * k + c.num_experts * (c.block_m - 1);
   sh.blocks_len = ceil_div(sh.sorted_len, c.block_m);
@@ -221,6 +225,8 @@ int moe_init(const moe_config* cfg, moe_handle** out) {
   h->sorted_len_max = sorted_len_max;
   h->blocks_len_max = ceil_div((int)sorted_len_max, c.block_m);
   h->max_routed_tiles = ceil_div((int)S_max, kBM) + E;
+  // splits * T <= #SMs * 128 (see router_splits) and splits <= 4
+  h->parts_rows = std::min(kMaxRouterSplits * c.max_tokens, (h->num_sms + 1) * kBM);
   h->max_tiles = h->max_routed_tiles + (c.inter_shared > 0 ? ceil_div(c.max_tokens, kBM) : 0);
   h->max_lag = 2 * h->num_sms;
   h->max_units = h->max_tiles + h->max_lag;
@@ -237,6 +243,7 @@ int moe_init(const moe_config* cfg, moe_handle** out) {
   std::vector<Piece> pieces = {
       {(void**)&w.meta, sizeof(DeviceMeta)},
       {(void**)&w.logits, T_ * E_ * 4},
+      {(void**)&w.logit_parts, (size_t)h->parts_rows * E_ * 4},
       {(void**)&w.topk_ids, T_ * K_ * 4},
       {(void**)&w.topk_w, T_ * K_ * 4},
       {(void**)&w.chunk_hist, (size_t)kMaxChunks * E_ * 4},
@@ -254,7 +261,7 @@ int moe_init(const moe_config* cfg, moe_handle** out) {
       {(void**)&w.expert_tile0, E_ * 4},
       {(void**)&w.row_of_slot, (size_t)S_max * 4},
       {(void**)&w.xs, (size_t)h->max_routed_tiles * kBM * c.hidden * 2},
-      {(void**)&w.y, (size_t)h->max_tiles * kBM * c.hidden * 4},
+      {(void**)&w.y, (size_t)h->max_tiles * kBM * c.hidden * 2},
       {(void**)&w.trace, (size_t)trace_cap * 4 * 8},
       {(void**)&h->x_stage, (c.flags & MOE_FLAG_HOST_STAGING) ? T_ * c.hidden * 2 : 0},
       {(void**)&h->out_stage, (c.flags & MOE_FLAG_HOST_STAGING) ? T_ * c.hidden * 4 : 0},
@@ -287,16 +294,17 @@ int moe_init(const moe_config* cfg, moe_handle** out) {
   if ((rc = encode_map(h, &h->xs_map, w.xs, c.hidden, (uint64_t)h->max_routed_tiles * kBM,
                        (uint64_t)c.hidden * 2, kBK, kBM)))
     return fail(rc);
-  if ((rc = encode_map(h, &h->y_map, w.y, c.hidden, h_rows, (uint64_t)c.hidden * 4, 32, kBM,
-                       CU_TENSOR_MAP_DATA_TYPE_FLOAT32)))
-    return fail(rc);
+  if ((rc = encode_map(h, &h->y_map, w.y, c.hidden, h_rows, (uint64_t)c.hidden * 2, kBK, kBM))) return fail(rc);
 
   // kernel attributes
   Shape sh = make_shape(h, c.max_tokens, c.top_k);
   h->gate_smem = gate_smem_bytes(sh, h->max_units);
-  if (h->gate_smem > g_gate_smem_granted) {
-    if (check_cuda(configure_gate_kernels(h->gate_smem))) return fail(MOE_ERR_CUDA);
-    g_gate_smem_granted = h->gate_smem;
+  const size_t scatter_smem = scatter_smem_bytes(E, sh.chunk_tokens * c.top_k);
+  if (h->gate_smem > g_gate_smem_granted || scatter_smem > g_scatter_smem_granted) {
+    g_gate_smem_granted = std::max(g_gate_smem_granted, h->gate_smem);
+    g_scatter_smem_granted = std::max(g_scatter_smem_granted, scatter_smem);
+    if (check_cuda(configure_gate_kernels(g_gate_smem_granted, g_scatter_smem_granted)))
+      return fail(MOE_ERR_CUDA);
   }
   if (check_cuda(configure_router_kernel()) || check_cuda(configure_gemm_kernel())) return fail(MOE_ERR_CUDA);
   if (h->timing) {
@@ -397,11 +405,15 @@ static int forward_impl(moe_handle* h, const void* x, int32_t T, const void* w_r
   auto mark = [&](int i) { return (ev && cudaEventRecord(ev[i], st) != cudaSuccess) ? MOE_ERR_CUDA : MOE_OK; };
   const uint16_t* x16 = static_cast<const uint16_t*>(x);
   if ((rc = mark(0))) return rc;
-  if ((rc = check_cuda(launch_router(maps.x_tile, wr_map, router_bias, w.logits, T, E, H, bn, w.meta,
+  int splits = router_splits(T, E, H, bn, h->num_sms);
+  while (splits > 1 && (int64_t)splits * T > h->parts_rows) splits /= 2;
+  float* parts = splits > 1 ? w.logit_parts : w.logits;
+  if ((rc = check_cuda(launch_router(maps.x_tile, wr_map, router_bias, parts, T, E, H, bn, splits, w.meta,
                                      h->timeout_ns, st))))
     return rc;
   if ((rc = mark(1))) return rc;
-  if ((rc = check_cuda(launch_gate(w.logits, w.topk_ids, w.topk_w, w, sh, true, true, h->gate_smem, st))))
+  if ((rc = check_cuda(launch_gate(parts, splits, splits > 1 ? w.logits : nullptr, w.topk_ids, w.topk_w, w,
+                                   sh, true, true, h->gate_smem, st))))
     return rc;
   if ((rc = mark(2))) return rc;
   if ((rc = check_cuda(launch_scatter(w.topk_ids, w.sorted_ids, w.expert_ids, nullptr, w.row_of_slot, w,
@@ -480,7 +492,7 @@ int moe_router_logits(moe_handle* h, const void* x, int32_t T, const void* w_rou
   if ((rc = cached_map(h, &wm, w_router, H, E, (uint64_t)H * 2, kBK, bn))) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   h->last_stream = st;
-  return check_cuda(launch_router(xm, wm, router_bias, logits, T, E, H, bn, h->ws.meta, h->timeout_ns, st));
+  return check_cuda(launch_router(xm, wm, router_bias, logits, T, E, H, bn, 1, h->ws.meta, h->timeout_ns, st));
 }
 
 int moe_gate_topk(moe_handle* h, const float* logits, int32_t T, int32_t top_k, int32_t* topk_ids,
@@ -494,7 +506,7 @@ int moe_gate_topk(moe_handle* h, const float* logits, int32_t T, int32_t top_k, 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   h->last_stream = st;
   const Shape sh = make_shape(h, T, top_k);
-  return check_cuda(launch_gate(logits, topk_ids, topk_w, h->ws, sh, false, false, 0, st));
+  return check_cuda(launch_gate(logits, 1, nullptr, topk_ids, topk_w, h->ws, sh, false, false, 0, st));
 }
 
 int moe_align_block_size(moe_handle* h, const int32_t* topk_ids, int32_t T, int32_t top_k,

@@ -7,9 +7,10 @@
 // combine_kernel: the sum over experts of the Mixture-of-Kittens layer equation
 //   x' = W_shared(x) + sum_{e in top-k} w_e (W_down^e SwiGLU(...)).
 //   The down-GEMM epilogue already wrote w_s * (W_down^e h_s) for every kept slot s into its
-//   tile row of y (fp32); this kernel adds, per token, the shared-expert row first and then
-//   the slots j = 0..k-1 in order (dropped slots skipped), in fp32. The order is fixed, so
-//   the result does not depend on the schedule. One warp per (token, 128 columns).
+//   tile row of y (bf16, like the per-slot intermediate cache of the vLLM execution
+//   analysis); this kernel adds, per token, the shared-expert row first and then the slots
+//   j = 0..k-1 in order (dropped slots skipped), in fp32. The order is fixed, so the result
+//   does not depend on the schedule. One warp per (token, 256 columns).
 #include <algorithm>
 
 #include "launch.h"
@@ -41,30 +42,39 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+__device__ __forceinline__ void add_bf16x8(float (&acc)[8], const uint4 v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    acc[2 * i] += __uint_as_float(w[i] << 16);
+    acc[2 * i + 1] += __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
+// One warp per (token, 256 columns); each lane sums 8 columns.
 __global__ void __launch_bounds__(256)
     combine_kernel(float* __restrict__ out, Workspace ws, Shape sh) {
   const int lane = threadIdx.x & 31;
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int nw = (gridDim.x * blockDim.x) >> 5;
-  const int nch = ceil_div(sh.H, 128);
+  const int nch = ceil_div(sh.H, 256);
   const int Mr = __ldcg(&ws.meta->num_routed_tiles);
   const int64_t total = (int64_t)sh.T * nch;
   for (int64_t w = gw; w < total; w += nw) {
     const int t = (int)(w / nch);
-    const int c = (int)(w % nch) * 128 + lane * 4;
+    const int c = (int)(w % nch) * 256 + lane * 8;
     if (c >= sh.H) continue;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (sh.Ds > 0) {
-      const float4 v = __ldcg(reinterpret_cast<const float4*>(ws.y + ((size_t)Mr * kBM + t) * sh.H + c));
-      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-    }
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (sh.Ds > 0)
+      add_bf16x8(acc, __ldcg(reinterpret_cast<const uint4*>(ws.y + ((size_t)Mr * kBM + t) * sh.H + c)));
     for (int j = 0; j < sh.k; ++j) {
       const int row = __ldcg(ws.row_of_slot + (size_t)t * sh.k + j);
       if (row < 0) continue;
-      const float4 v = __ldcg(reinterpret_cast<const float4*>(ws.y + (size_t)row * sh.H + c));
-      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+      add_bf16x8(acc, __ldcg(reinterpret_cast<const uint4*>(ws.y + (size_t)row * sh.H + c)));
     }
-    *reinterpret_cast<float4*>(out + (size_t)t * sh.H + c) = acc;
+    float4* o = reinterpret_cast<float4*>(out + (size_t)t * sh.H + c);
+    o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    o[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
   }
 }
 
@@ -75,7 +85,7 @@ cudaError_t launch_gather_rows(const uint16_t* x, const Workspace& ws, const Sha
 }
 
 cudaError_t launch_combine(float* out, const Workspace& ws, const Shape& sh, cudaStream_t stream) {
-  const int64_t warps = (int64_t)sh.T * ceil_div(sh.H, 128);
+  const int64_t warps = (int64_t)sh.T * ceil_div(sh.H, 256);
   const int grid = (int)std::min<int64_t>((warps + 7) / 8, 148 * 32);
   combine_kernel<<<grid, 256, 0, stream>>>(out, ws, sh);
   return cudaGetLastError();

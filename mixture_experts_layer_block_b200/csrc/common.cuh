@@ -26,13 +26,15 @@ constexpr int kAccCols = 256;   // TMEM columns per accumulator buffer (2 buffer
 constexpr int kGemmThreads = 192;  // warp 0 producer, warp 1 MMA, warps 2-5 epilogue
 
 // ---- router GEMM -------------------------------------------------------------------------
-constexpr int kRouterStages = 4;
+constexpr int kRouterStages = 6;
 constexpr int kRouterMaxN = 64;
+constexpr int kMaxRouterSplits = 4;
 
 // ---- gating / align ------------------------------------------------------------------------
-constexpr int kGateThreads = 256;
-constexpr int kMaxChunks = 128;    // token chunks of the histogram (chunk = ceil(T/128) >= 64)
+constexpr int kGateThreads = 512;
+constexpr int kMaxChunks = 32;     // token chunks of the histogram (chunk = ceil(T/32) >= 64)
 constexpr int kMinChunkTokens = 64;
+constexpr int kGateTokensPerCta = 64;  // gating CTAs: 16 warps x 4 tokens
 constexpr int kMaxExperts = 1024;
 
 // ---- device status word --------------------------------------------------------------------
@@ -85,6 +87,7 @@ struct Task {
 struct Workspace {
   DeviceMeta* meta;
   float* logits;         // [T][E]
+  float* logit_parts;    // [splits*T][E]    K-split partial router logits
   int32_t* topk_ids;     // [T][k]
   float* topk_w;         // [T][k]
   int32_t* chunk_hist;   // [kMaxChunks][E]
@@ -102,7 +105,7 @@ struct Workspace {
   int32_t* row_of_slot;  // [S]              tile row (tile*128 + r) of each kept slot, -1 if dropped
   uint16_t* xs;          // [max_routed_tiles*128][H] bf16 x rows gathered in tile order
   uint16_t* h;           // [max_tiles*128][ldh] bf16 SwiGLU activations
-  float* y;              // [max_tiles*128][H] fp32 router-weighted expert outputs per tile row
+  uint16_t* y;           // [max_tiles*128][H] bf16 router-weighted expert outputs per tile row
   int64_t* trace;        // [trace_cap][4]
   int32_t trace_cap;
   int32_t ldh;           // row stride of h in elements (max(D, D_shared))

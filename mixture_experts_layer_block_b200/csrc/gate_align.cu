@@ -1,19 +1,24 @@
 // gate_align.cu -- gating (top-k softmax, renormalised) and align (moe_align_block_size).
 //
 // Gating (Weave blog section 1.1; vLLM execution analysis, topk_softmax): one warp per
-// token; each lane holds E/32 logits; k rounds of a warp arg-max (ties to the lower expert
-// index) select the experts in descending order; the weights are the selected softmax
-// probabilities renormalised over the selection, i.e. exp(v_j - v_0) / sum_i exp(v_i - v_0).
+// token, 64 tokens per CTA; each lane holds E/32 logits (adding the router's K-split
+// partials in split order); k rounds of a warp arg-max (ties to
+// the lower expert index) select the experts in descending order; the weights are the
+// selected softmax probabilities renormalised over the selection, i.e.
+// exp(v_j - v_0) / sum_i exp(v_i - v_0). Each warp loads its next token while it selects
+// the current one.
 //
 // Align (vLLM PR #53280 summary: per-expert counts, exclusive cumsum, cooperative writes of
 // token ids and block ids; the reviewer's variant that uses every block of the grid):
-//   1. each CTA of the gating (or histogram) kernel counts the slots of its token chunk per
-//      expert;
-//   2. the last CTA to finish scans: per expert, the counts of earlier chunks (so writes stay
-//      stable), the capacity cut, the padded segment offsets, and for the forward also the
-//      m-tile list and the task schedule of the expert-GEMM kernel;
-//   3. a grid-wide kernel writes sorted_ids (one warp per chunk, 32 slots per round, ranks
-//      from __match_any_sync), the padding sentinels and expert_ids (one thread per entry).
+//   1. each CTA of the gating (or histogram) kernel counts its slots per expert and adds the
+//      counts into its token chunk's histogram (integer atomics; at most 32 chunks);
+//   2. the last CTA to finish scans: per expert, the counts of earlier chunks (loaded in
+//      parallel into shared memory), the capacity cut, the padded segment offsets, and for
+//      the forward also the m-tile list and the task schedule of the expert-GEMM kernel;
+//   3. a grid-wide kernel writes sorted_ids: one CTA per chunk, one warp per sub-chunk,
+//      ranks from __match_any_sync, warp offsets from a per-chunk prefix over warps; and
+//      every CTA writes its share of the padding sentinels and expert_ids (one thread per
+//      entry).
 #include <algorithm>
 #include <climits>
 #include <cmath>
@@ -23,19 +28,36 @@
 namespace moe {
 
 // ------------------------------------------------------------------------------------------
-// warp top-k + renormalised softmax of one token; lane j < k returns choice j
+// warp top-k + renormalised softmax of one token held in registers; lane j < k returns
+// choice j
 // ------------------------------------------------------------------------------------------
-template <int VPL>
-__device__ __forceinline__ void warp_topk_softmax(const float* __restrict__ row, int E, int k,
-                                                  int lane, int& out_id, float& out_w) {
-  float v[VPL];
-  uint32_t taken = 0;
+template <int VPL, int S>
+__device__ __forceinline__ void load_token(const float* __restrict__ row, size_t part_stride, int E,
+                                           int lane, float (&v)[VPL]) {
+  float p[S][VPL];
+#pragma unroll
+  for (int s = 0; s < S; ++s)
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) {
+      const int e = lane + 32 * j;
+      p[s][j] = (e < E) ? __ldcg(row + s * part_stride + e) : 0.f;
+    }
 #pragma unroll
   for (int j = 0; j < VPL; ++j) {
-    const int e = lane + 32 * j;
-    v[j] = (e < E) ? row[e] : -INFINITY;
-    if (e >= E) taken |= 1u << j;
+    float a = p[0][j];
+#pragma unroll
+    for (int s = 1; s < S; ++s) a += p[s][j];
+    v[j] = (lane + 32 * j < E) ? a : -INFINITY;
   }
+}
+
+template <int VPL>
+__device__ __forceinline__ void warp_topk_softmax(const float (&v)[VPL], int E, int k, int lane,
+                                                  int& out_id, float& out_w) {
+  uint32_t taken = 0;
+#pragma unroll
+  for (int j = 0; j < VPL; ++j)
+    if (lane + 32 * j >= E) taken |= 1u << j;
   float my_v = 0.f, top_v = 0.f;
   int my_id = -1;
   for (int r = 0; r < k; ++r) {
@@ -123,48 +145,48 @@ __device__ int block_exclusive_scan(int* a, int n, int* tmp) {
 
 // ------------------------------------------------------------------------------------------
 // The scans, run by the last CTA of the histogram pass. Shared memory layout (ints):
-//   tmp[64] | cnt[E] | kept[E] | buf[max(E+1, units+1)]
+//   tmp[64] | cnt[E] | kept[E] | tile[kMaxChunks * kScanGroup] | buf[max(E+1, units+1)]
 // ------------------------------------------------------------------------------------------
+constexpr int kScanGroup = 256;  // experts scanned per pass (tile of [chunks][256] counts)
+
 __device__ void align_scans(const Workspace& ws, const Shape& sh, bool tiles, int* sm) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
+  const int tid = threadIdx.x, nthr = blockDim.x;
   const int E = sh.E;
   int* tmp = sm;
   int* cnt = tmp + 64;
   int* kept = cnt + E;
-  int* buf = kept + E;
+  int* tile = kept + E;
+  int* buf = tile + kMaxChunks * kScanGroup;
   const int nch = sh.num_chunks;
 
-  // 1. per expert: exclusive prefix of the chunk counts (chunk_base) and the total n_e
-  const int cpw = ceil_div(nch, nwarps);
-  for (int eg = 0; eg < E; eg += 32) {
-    const int e = eg + lane;
-    const int c0 = warp * cpw, c1 = min(nch, c0 + cpw);
-    int sum = 0;
-    if (e < E)
-      for (int c = c0; c < c1; ++c) sum += __ldcg(ws.chunk_hist + (size_t)c * E + e);
-    buf[warp * 32 + lane] = sum;
-    __syncthreads();
-    if (warp == 0) {
-      int run = 0;
-      for (int w = 0; w < nwarps; ++w) {
-        const int x = buf[w * 32 + lane];
-        buf[w * 32 + lane] = run;
-        run += x;
-      }
-      if (e < E) cnt[e] = run;
+  // 1. per expert: exclusive prefix of the chunk counts (chunk_base) and the total n_e.
+  //    The [chunks][group] block of counts is loaded with independent loads, then each
+  //    thread scans one expert's column in shared memory.
+  for (int g0 = 0; g0 < E; g0 += kScanGroup) {
+    const int G = min(kScanGroup, E - g0);
+    const int n = nch * G;
+#pragma unroll 4
+    for (int i = tid; i < n; i += nthr) {
+      const int c = i / G, e = i - c * G;
+      int* p = ws.chunk_hist + (size_t)c * E + g0 + e;
+      tile[i] = __ldcg(p);
+      *p = 0;  // the histograms start from zero at the next call
     }
     __syncthreads();
-    int run = buf[warp * 32 + lane];
-    if (e < E)
-      for (int c = c0; c < c1; ++c) {
-        ws.chunk_base[(size_t)c * E + e] = run;
-        run += __ldcg(ws.chunk_hist + (size_t)c * E + e);
+    if (tid < G) {
+      int run = 0;
+      for (int c = 0; c < nch; ++c) {
+        const int v = tile[c * G + tid];
+        ws.chunk_base[(size_t)c * E + g0 + tid] = run;
+        run += v;
       }
+      cnt[g0 + tid] = run;
+    }
     __syncthreads();
   }
 
   // 2. capacity cut and padded segment lengths
-  for (int e = tid; e < E; e += blockDim.x) {
+  for (int e = tid; e < E; e += nthr) {
     const int n = cnt[e];
     const int kp = (sh.capacity > 0) ? min(n, sh.capacity) : n;
     kept[e] = kp;
@@ -173,7 +195,7 @@ __device__ void align_scans(const Workspace& ws, const Shape& sh, bool tiles, in
   }
   __syncthreads();
   const int P = block_exclusive_scan(buf, E, tmp);
-  for (int e = tid; e < E; e += blockDim.x) ws.expert_off[e] = buf[e];
+  for (int e = tid; e < E; e += nthr) ws.expert_off[e] = buf[e];
   if (tid == 0) {
     ws.expert_off[E] = P;
     ws.meta->P = P;
@@ -182,10 +204,10 @@ __device__ void align_scans(const Workspace& ws, const Shape& sh, bool tiles, in
   if (!tiles) return;
 
   // 3. m-tiles: routed experts (ceil(kept/128) each), then the shared expert over all tokens
-  for (int e = tid; e < E; e += blockDim.x) buf[e] = ceil_div(kept[e], kBM);
+  for (int e = tid; e < E; e += nthr) buf[e] = ceil_div(kept[e], kBM);
   __syncthreads();
   const int Mr = block_exclusive_scan(buf, E, tmp);
-  for (int e = tid; e < E; e += blockDim.x) {
+  for (int e = tid; e < E; e += nthr) {
     const int first = buf[e], nt = ceil_div(kept[e], kBM);
     const int off = ws.expert_off[e];
     ws.expert_tile0[e] = first;
@@ -196,7 +218,7 @@ __device__ void align_scans(const Workspace& ws, const Shape& sh, bool tiles, in
     }
   }
   const int Ms = (sh.Ds > 0) ? ceil_div(sh.T, kBM) : 0;
-  for (int j = tid; j < Ms; j += blockDim.x) {
+  for (int j = tid; j < Ms; j += nthr) {
     ws.tile_expert[Mr + j] = E;
     ws.tile_row0[Mr + j] = j * kBM;
     ws.tile_nrows[Mr + j] = min(kBM, sh.T - j * kBM);
@@ -208,7 +230,7 @@ __device__ void align_scans(const Workspace& ws, const Shape& sh, bool tiles, in
   //    u - lag. Task ids are unit-major, so every down task's dependencies have lower ids.
   const int U = (Mt > 0) ? Mt + sh.lag : 0;
   const int n2 = ceil_div(sh.H, kBN2);
-  for (int u = tid; u < U; u += blockDim.x) {
+  for (int u = tid; u < U; u += nthr) {
     int c = 0;
     if (u < Mt) c += ceil_div(ws.tile_expert[u] == E ? sh.Ds : sh.D, kBN1);
     if (u >= sh.lag && u - sh.lag < Mt) c += n2;
@@ -216,8 +238,8 @@ __device__ void align_scans(const Workspace& ws, const Shape& sh, bool tiles, in
   }
   __syncthreads();
   const int total = block_exclusive_scan(buf, U, tmp);
-  for (int u = tid; u < U; u += blockDim.x) ws.unit_start[u] = buf[u];
-  for (int i = tid; i < Mt; i += blockDim.x) ws.done1[i] = 0;
+  for (int u = tid; u < U; u += nthr) ws.unit_start[u] = buf[u];
+  for (int i = tid; i < Mt; i += nthr) ws.done1[i] = 0;
   if (tid == 0) {
     ws.unit_start[U] = total;
     ws.meta->num_tiles = Mt;
@@ -230,12 +252,12 @@ __device__ void align_scans(const Workspace& ws, const Shape& sh, bool tiles, in
   }
 }
 
-// Publish this CTA's chunk histogram; the last CTA runs the scans.
+// Add this CTA's counts into its chunk's histogram; the last CTA runs the scans.
 __device__ void finish_histogram(const Workspace& ws, const Shape& sh, bool tiles, const int* hist,
-                                 int* sm) {
+                                 int chunk, int* sm) {
   __shared__ int s_last;
   for (int e = threadIdx.x; e < sh.E; e += blockDim.x)
-    ws.chunk_hist[(size_t)blockIdx.x * sh.E + e] = hist[e];
+    if (hist[e]) atomicAdd(ws.chunk_hist + (size_t)chunk * sh.E + e, hist[e]);
   __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) s_last = (atomicAdd(&ws.meta->hist_done, 1) == (int)gridDim.x - 1);
@@ -249,24 +271,41 @@ __device__ void finish_histogram(const Workspace& ws, const Shape& sh, bool tile
 // ------------------------------------------------------------------------------------------
 // kernels
 // ------------------------------------------------------------------------------------------
-// smem: hist[E] | scan area
-template <int VPL>
+// smem: hist[E] | scan area. One CTA per kGateTokensPerCta tokens (a chunk holds a whole
+// number of CTAs). `parts` holds S partial logits [S][T][E]; with logits_out non-null the
+// sums are written there.
+template <int VPL, int S>
 __global__ void __launch_bounds__(kGateThreads)
-    gate_kernel(const float* __restrict__ logits, int32_t* __restrict__ topk_ids,
-                float* __restrict__ topk_w, Workspace ws, Shape sh, int hist_on, int tiles) {
+    gate_kernel(const float* __restrict__ parts, float* __restrict__ logits_out,
+                int32_t* __restrict__ topk_ids, float* __restrict__ topk_w, Workspace ws, Shape sh,
+                int hist_on, int tiles) {
   extern __shared__ int smem_i[];
   int* hist = smem_i;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t0 = blockIdx.x * sh.chunk_tokens;
-  const int t1 = min(sh.T, t0 + sh.chunk_tokens);
+  constexpr int kWarps = kGateThreads / 32;
+  const int t0 = blockIdx.x * kGateTokensPerCta;
+  const int t1 = min(sh.T, t0 + kGateTokensPerCta);
+  const size_t pstride = (size_t)sh.T * sh.E;
   if (hist_on) {
     for (int e = threadIdx.x; e < sh.E; e += blockDim.x) hist[e] = 0;
     __syncthreads();
   }
-  for (int t = t0 + warp; t < t1; t += kGateThreads / 32) {
+  float vnext[VPL];
+  int t = t0 + warp;
+  if (t < t1) load_token<VPL, S>(parts + (size_t)t * sh.E, pstride, sh.E, lane, vnext);
+  for (; t < t1; t += kWarps) {
+    float v[VPL];
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) v[j] = vnext[j];
+    if (t + kWarps < t1) load_token<VPL, S>(parts + (size_t)(t + kWarps) * sh.E, pstride, sh.E, lane, vnext);
+    if (logits_out) {
+#pragma unroll
+      for (int j = 0; j < VPL; ++j)
+        if (lane + 32 * j < sh.E) logits_out[(size_t)t * sh.E + lane + 32 * j] = v[j];
+    }
     int id;
     float w;
-    warp_topk_softmax<VPL>(logits + (size_t)t * sh.E, sh.E, sh.k, lane, id, w);
+    warp_topk_softmax<VPL>(v, sh.E, sh.k, lane, id, w);
     if (lane < sh.k) {
       topk_ids[(size_t)t * sh.k + lane] = id;
       topk_w[(size_t)t * sh.k + lane] = w;
@@ -275,7 +314,7 @@ __global__ void __launch_bounds__(kGateThreads)
   }
   if (!hist_on) return;
   __syncthreads();
-  finish_histogram(ws, sh, tiles != 0, hist, smem_i + sh.E);
+  finish_histogram(ws, sh, tiles != 0, hist, t0 / sh.chunk_tokens, smem_i + sh.E);
 }
 
 __global__ void __launch_bounds__(kGateThreads)
@@ -284,14 +323,15 @@ __global__ void __launch_bounds__(kGateThreads)
   int* hist = smem_i;
   for (int e = threadIdx.x; e < sh.E; e += blockDim.x) hist[e] = 0;
   __syncthreads();
-  const int64_t s0 = (int64_t)blockIdx.x * sh.chunk_tokens * sh.k;
-  const int64_t s1 = (int64_t)min(sh.T, (int)(blockIdx.x + 1) * sh.chunk_tokens) * sh.k;
+  const int t0 = blockIdx.x * kGateTokensPerCta;
+  const int64_t s0 = (int64_t)t0 * sh.k;
+  const int64_t s1 = (int64_t)min(sh.T, t0 + kGateTokensPerCta) * sh.k;
   for (int64_t s = s0 + threadIdx.x; s < s1; s += blockDim.x) {
     const int e = topk_ids[s];
     if (e >= 0 && e < sh.E) atomicAdd(&hist[e], 1);  // ids outside [0, E) are skipped
   }
   __syncthreads();
-  finish_histogram(ws, sh, false, hist, smem_i + sh.E);
+  finish_histogram(ws, sh, false, hist, t0 / sh.chunk_tokens, smem_i + sh.E);
 }
 
 __device__ __forceinline__ int segment_of(const int* off, int E, int i) {
@@ -305,60 +345,89 @@ __device__ __forceinline__ int segment_of(const int* off, int E, int i) {
   return lo;
 }
 
-// smem: off[E+1] | kept[E] | tile0[E] | per-warp counters [8][E]
-// With `row_of_slot` non-null, also records for every slot its row in the tile-ordered
-// buffers (first tile of its expert * 128 + its rank), or -1 when the slot was dropped.
-__global__ void __launch_bounds__(256)
+// smem: off[E+1] | kept[E] | tile0[E] | wcnt[16][E] | ids[chunk slots]
+// CTA c < num_chunks sorts the slots of token chunk c: warp w owns a contiguous run of the
+// chunk's slots; pass 1 counts them per expert, a per-expert prefix over the warps (seeded
+// with the chunk prefix of the scan) gives every warp its first rank, pass 2 writes. With
+// `row_of_slot` non-null, also records for every slot its row in the tile-ordered buffers
+// (first tile of its expert * 128 + its rank), or -1 when the slot was dropped. Every CTA
+// then writes its share of the padding sentinels and of expert_ids.
+__global__ void __launch_bounds__(kGateThreads)
     scatter_kernel(const int32_t* __restrict__ topk_ids, int32_t* __restrict__ sorted_ids,
                    int32_t* __restrict__ expert_ids, int32_t* __restrict__ num_post_padded,
                    int32_t* __restrict__ row_of_slot, Workspace ws, Shape sh) {
   extern __shared__ int smem_i[];
+  constexpr int kWarps = kGateThreads / 32;
   const int E = sh.E;
   int* off = smem_i;
   int* kept = off + E + 1;
   int* tile0 = kept + E;
-  int* cnt_all = tile0 + E;
-  for (int e = threadIdx.x; e <= E; e += blockDim.x) off[e] = __ldcg(ws.expert_off + e);
-  for (int e = threadIdx.x; e < E; e += blockDim.x) kept[e] = __ldcg(ws.expert_kept + e);
-  if (row_of_slot)
-    for (int e = threadIdx.x; e < E; e += blockDim.x) tile0[e] = __ldcg(ws.expert_tile0 + e);
-  __syncthreads();
-  const int P = off[E];
-  const int S = sh.T * sh.k;
+  int* wcnt = tile0 + E;
+  int* ids = wcnt + kWarps * E;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int e = threadIdx.x; e <= E; e += blockDim.x) off[e] = __ldcg(ws.expert_off + e);
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    kept[e] = __ldcg(ws.expert_kept + e);
+    if (row_of_slot) tile0[e] = __ldcg(ws.expert_tile0 + e);
+  }
+  const int P = __ldcg(ws.expert_off + E);
+  const int S = sh.T * sh.k;
 
-  // (a) stable scatter of the slot ids, one warp per chunk
-  int* cnt = cnt_all + warp * E;
-  const int gw = blockIdx.x * (blockDim.x >> 5) + warp;
-  const int nw = gridDim.x * (blockDim.x >> 5);
-  for (int c = gw; c < sh.num_chunks; c += nw) {
-    for (int e = lane; e < E; e += 32) cnt[e] = __ldcg(ws.chunk_base + (size_t)c * E + e);
-    __syncwarp();
+  const int c = blockIdx.x;
+  if (c < sh.num_chunks) {
     const int s0 = c * sh.chunk_tokens * sh.k;
-    const int s1 = min(sh.T, (c + 1) * sh.chunk_tokens) * sh.k;
-    for (int base = s0; base < s1; base += 32) {
-      const int s = base + lane;
-      int e = (s < s1) ? topk_ids[s] : -1;
-      if (e >= E) e = -1;
-      const bool valid = e >= 0;
+    const int n = min(sh.T, (c + 1) * sh.chunk_tokens) * sh.k - s0;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      const int e = topk_ids[s0 + i];
+      ids[i] = (e >= 0 && e < E) ? e : -1;
+    }
+    for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) wcnt[i] = 0;
+    __syncthreads();
+    const int per = ceil_div(ceil_div(n, kWarps), 32) * 32;
+    const int w0 = min(n, warp * per), w1 = min(n, w0 + per);
+    int* cnt = wcnt + warp * E;
+    // pass 1: per-warp counts
+    for (int base = w0; base < w1; base += 32) {
+      const int e = (base + lane < w1) ? ids[base + lane] : -1;
+      const unsigned mask = __match_any_sync(0xffffffffu, e);
+      if (e >= 0 && lane == __ffs(mask) - 1) cnt[e] += __popc(mask);
+    }
+    __syncthreads();
+    // per expert: first rank of every warp = chunk prefix + counts of the earlier warps
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+      int run = __ldcg(ws.chunk_base + (size_t)c * E + e);
+      for (int w = 0; w < kWarps; ++w) {
+        const int x = wcnt[w * E + e];
+        wcnt[w * E + e] = run;
+        run += x;
+      }
+    }
+    __syncthreads();
+    // pass 2: stable writes
+    for (int base = w0; base < w1; base += 32) {
+      const bool in = base + lane < w1;
+      const int e = in ? ids[base + lane] : -1;
       const unsigned mask = __match_any_sync(0xffffffffu, e);
       const int rank = __popc(mask & ((1u << lane) - 1u));
-      const int c0 = valid ? cnt[e] : 0;
+      const int c0 = (e >= 0) ? cnt[e] : 0;
       __syncwarp();
-      if (valid) {
+      const int s = s0 + base + lane;
+      if (e >= 0) {
         const int r = c0 + rank;
         const bool keep = sh.capacity == 0 || r < sh.capacity;
         if (keep) sorted_ids[off[e] + r] = s;
         if (row_of_slot) row_of_slot[s] = keep ? tile0[e] * kBM + r : -1;
         if (rank == 0) cnt[e] = c0 + __popc(mask);
-      } else if (row_of_slot && s < s1) {
+      } else if (in && row_of_slot) {
         row_of_slot[s] = -1;  // an expert id outside [0, E)
       }
       __syncwarp();
     }
+  } else {
+    __syncthreads();
   }
 
-  // (b) padding sentinels, (c) block -> expert ids, one thread per entry
+  // padding sentinels and block -> expert ids, one thread per entry, grid-wide
   const int gt = blockIdx.x * blockDim.x + threadIdx.x;
   const int nt = gridDim.x * blockDim.x;
   for (int i = gt; i < sh.sorted_len; i += nt) {
@@ -380,58 +449,79 @@ __global__ void __launch_bounds__(256)
 // launchers
 // ------------------------------------------------------------------------------------------
 size_t gate_smem_bytes(const Shape& sh, int max_units) {
-  const int buf = std::max(std::max(sh.E + 1, max_units + 1), 8 * 32);
-  return sizeof(int) * (size_t)(sh.E /*hist*/ + 64 + 2 * sh.E + buf);
+  const int buf = std::max(sh.E + 1, max_units + 1);
+  return sizeof(int) * (size_t)(sh.E /*hist*/ + 64 + 2 * sh.E + kMaxChunks * kScanGroup + buf);
 }
 
-size_t scatter_smem_bytes(int E) { return sizeof(int) * (size_t)(E + 1 + 2 * E + 8 * E); }
+size_t scatter_smem_bytes(int E, int chunk_slots) {
+  return sizeof(int) * (size_t)(E + 1 + 2 * E + (kGateThreads / 32) * E + chunk_slots);
+}
 
-template <int VPL>
-static cudaError_t launch_gate_vpl(const float* logits, int32_t* ids, float* w, const Workspace& ws,
-                                   const Shape& sh, bool hist, bool tiles, size_t smem,
-                                   cudaStream_t st) {
-  gate_kernel<VPL><<<sh.num_chunks, kGateThreads, hist ? smem : 0, st>>>(logits, ids, w, ws, sh,
-                                                                          hist ? 1 : 0, tiles ? 1 : 0);
+static int gate_grid(const Shape& sh) { return std::max(1, ceil_div(sh.T, kGateTokensPerCta)); }
+
+template <int VPL, int S>
+static cudaError_t launch_gate_vs(const float* parts, float* logits_out, int32_t* ids, float* w,
+                                  const Workspace& ws, const Shape& sh, bool hist, bool tiles,
+                                  size_t smem, cudaStream_t st) {
+  gate_kernel<VPL, S><<<gate_grid(sh), kGateThreads, hist ? smem : 0, st>>>(
+      parts, logits_out, ids, w, ws, sh, hist ? 1 : 0, tiles ? 1 : 0);
   return cudaGetLastError();
 }
 
-cudaError_t launch_gate(const float* logits, int32_t* topk_ids, float* topk_w, const Workspace& ws,
-                        const Shape& sh, bool hist, bool tiles, size_t smem, cudaStream_t st) {
-  if (sh.num_chunks <= 0) return cudaSuccess;
-  if (sh.E <= 32) return launch_gate_vpl<1>(logits, topk_ids, topk_w, ws, sh, hist, tiles, smem, st);
-  if (sh.E <= 64) return launch_gate_vpl<2>(logits, topk_ids, topk_w, ws, sh, hist, tiles, smem, st);
-  if (sh.E <= 128) return launch_gate_vpl<4>(logits, topk_ids, topk_w, ws, sh, hist, tiles, smem, st);
-  if (sh.E <= 256) return launch_gate_vpl<8>(logits, topk_ids, topk_w, ws, sh, hist, tiles, smem, st);
-  if (sh.E <= 512) return launch_gate_vpl<16>(logits, topk_ids, topk_w, ws, sh, hist, tiles, smem, st);
-  return launch_gate_vpl<32>(logits, topk_ids, topk_w, ws, sh, hist, tiles, smem, st);
+template <int VPL>
+static cudaError_t launch_gate_v(const float* parts, int splits, float* logits_out, int32_t* ids,
+                                 float* w, const Workspace& ws, const Shape& sh, bool hist,
+                                 bool tiles, size_t smem, cudaStream_t st) {
+  if (splits == 4) return launch_gate_vs<VPL, 4>(parts, logits_out, ids, w, ws, sh, hist, tiles, smem, st);
+  if (splits == 2) return launch_gate_vs<VPL, 2>(parts, logits_out, ids, w, ws, sh, hist, tiles, smem, st);
+  return launch_gate_vs<VPL, 1>(parts, logits_out, ids, w, ws, sh, hist, tiles, smem, st);
+}
+
+cudaError_t launch_gate(const float* parts, int splits, float* logits_out, int32_t* topk_ids,
+                        float* topk_w, const Workspace& ws, const Shape& sh, bool hist, bool tiles,
+                        size_t smem, cudaStream_t st) {
+#define MOE_GATE(V) \
+  launch_gate_v<V>(parts, splits, logits_out, topk_ids, topk_w, ws, sh, hist, tiles, smem, st)
+  if (sh.E <= 32) return MOE_GATE(1);
+  if (sh.E <= 64) return MOE_GATE(2);
+  if (sh.E <= 128) return MOE_GATE(4);
+  if (sh.E <= 256) return MOE_GATE(8);
+  if (sh.E <= 512) return MOE_GATE(16);
+  return MOE_GATE(32);
+#undef MOE_GATE
 }
 
 cudaError_t launch_hist(const int32_t* topk_ids, const Workspace& ws, const Shape& sh, size_t smem,
                         cudaStream_t st) {
-  hist_kernel<<<sh.num_chunks, kGateThreads, smem, st>>>(topk_ids, ws, sh);
+  hist_kernel<<<gate_grid(sh), kGateThreads, smem, st>>>(topk_ids, ws, sh);
   return cudaGetLastError();
 }
 
 cudaError_t launch_scatter(const int32_t* topk_ids, int32_t* sorted_ids, int32_t* expert_ids,
                            int32_t* num_post_padded, int32_t* row_of_slot, const Workspace& ws,
                            const Shape& sh, int grid, cudaStream_t st) {
-  scatter_kernel<<<grid, 256, scatter_smem_bytes(sh.E), st>>>(topk_ids, sorted_ids, expert_ids,
-                                                              num_post_padded, row_of_slot, ws, sh);
+  const size_t smem = scatter_smem_bytes(sh.E, sh.chunk_tokens * sh.k);
+  scatter_kernel<<<std::max(grid, sh.num_chunks), kGateThreads, smem, st>>>(
+      topk_ids, sorted_ids, expert_ids, num_post_padded, row_of_slot, ws, sh);
   return cudaGetLastError();
 }
 
-cudaError_t configure_gate_kernels(size_t gate_smem) {
+template <int VPL>
+static cudaError_t set_gate_smem(int s) {
+  cudaError_t err;
+  if ((err = cudaFuncSetAttribute(gate_kernel<VPL, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, s))) return err;
+  if ((err = cudaFuncSetAttribute(gate_kernel<VPL, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, s))) return err;
+  return cudaFuncSetAttribute(gate_kernel<VPL, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, s);
+}
+
+cudaError_t configure_gate_kernels(size_t gate_smem, size_t scatter_smem) {
   cudaError_t err = cudaSuccess;
   const int s = (int)gate_smem;
-  if ((err = cudaFuncSetAttribute(gate_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, s))) return err;
-  if ((err = cudaFuncSetAttribute(gate_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, s))) return err;
-  if ((err = cudaFuncSetAttribute(gate_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, s))) return err;
-  if ((err = cudaFuncSetAttribute(gate_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, s))) return err;
-  if ((err = cudaFuncSetAttribute(gate_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, s))) return err;
-  if ((err = cudaFuncSetAttribute(gate_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, s))) return err;
+  if ((err = set_gate_smem<1>(s)) || (err = set_gate_smem<2>(s)) || (err = set_gate_smem<4>(s)) ||
+      (err = set_gate_smem<8>(s)) || (err = set_gate_smem<16>(s)) || (err = set_gate_smem<32>(s)))
+    return err;
   if ((err = cudaFuncSetAttribute(hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, s))) return err;
-  return cudaFuncSetAttribute(scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)scatter_smem_bytes(kMaxExperts));
+  return cudaFuncSetAttribute(scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)scatter_smem);
 }
 
 }  // namespace moe

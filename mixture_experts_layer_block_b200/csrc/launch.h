@@ -11,7 +11,7 @@ namespace moe {
 struct alignas(64) GemmMaps {
   CUtensorMap x_tile;    // x [T][H], box {64, 128} (shared-expert tiles)
   CUtensorMap xs;        // gathered rows [routed_rows][H], box {64, 128}
-  CUtensorMap y;         // y [rows][H] fp32, box {32, 128} (store)
+  CUtensorMap y;         // y [rows][H] bf16, box {64, 128} (store)
   CUtensorMap w_up;      // [E*D][H], box {64, 128}
   CUtensorMap w_gate;    // [E*D][H], box {64, 128}
   CUtensorMap w_down;    // [E*H][D], box {64, 256}
@@ -23,23 +23,29 @@ struct alignas(64) GemmMaps {
 };
 
 // Router projection: logits[T][E] = x W^T (+ bias). x_map box {64,128}, w_map box {64,BN}.
+// With splits > 1 (1, 2 or 4) the K loop is split over blockIdx.z and `logits` receives the
+// partials [splits][T][E] (bias in partial 0).
 size_t router_smem_bytes(int BN);
+int router_splits(int T, int E, int H, int BN, int num_sms);
 cudaError_t launch_router(const CUtensorMap& x_map, const CUtensorMap& w_map, const float* bias,
-                          float* logits, int T, int E, int H, int BN, DeviceMeta* meta,
+                          float* logits, int T, int E, int H, int BN, int splits, DeviceMeta* meta,
                           int64_t timeout_ns, cudaStream_t stream);
 
-// Gating. With `hist`, also the per-chunk expert histogram and, in the last CTA, the scans
-// (and the tile/task tables when `tiles`).
+// Gating of logits given as `splits` partials [splits][T][E] (1, 2 or 4; summed in split
+// order, and the sums written to logits_out when it is non-null). With `hist`, also the
+// per-chunk expert histogram and, in the last CTA, the scans (and the tile/task tables when
+// `tiles`).
 size_t gate_smem_bytes(const Shape& sh, int max_units);
-cudaError_t launch_gate(const float* logits, int32_t* topk_ids, float* topk_w, const Workspace& ws,
-                        const Shape& sh, bool hist, bool tiles, size_t smem, cudaStream_t stream);
+cudaError_t launch_gate(const float* parts, int splits, float* logits_out, int32_t* topk_ids,
+                        float* topk_w, const Workspace& ws, const Shape& sh, bool hist, bool tiles,
+                        size_t smem, cudaStream_t stream);
 
 // Histogram of given topk_ids (standalone align), with the same last-CTA scans (no tiles).
 cudaError_t launch_hist(const int32_t* topk_ids, const Workspace& ws, const Shape& sh, size_t smem,
                         cudaStream_t stream);
 
 // Grid-wide align writes (and the tile row of every slot when row_of_slot is non-null).
-size_t scatter_smem_bytes(int E);
+size_t scatter_smem_bytes(int E, int chunk_slots);
 cudaError_t launch_scatter(const int32_t* topk_ids, int32_t* sorted_ids, int32_t* expert_ids,
                            int32_t* num_post_padded, int32_t* row_of_slot, const Workspace& ws,
                            const Shape& sh, int grid, cudaStream_t stream);

@@ -3,7 +3,7 @@
 // What it computes (Mixture-of-Kittens blog, "Overlapping compute and communication in
 // MoE"): for every kept slot s = (t, j) routed to expert e,
 //     h_s  = SiLU(W_up^e x_t) (.) (W_gate^e x_t)                   (bf16, kept in HBM/L2)
-//     y_s   = w_s * W_down^e h_s                                   (fp32, per slot row)
+//     y_s   = w_s * W_down^e h_s                                   (bf16, per slot row)
 // plus the shared expert over every token with weight 1.
 //
 // How (Weave blog, sections 2.1-2.2 and 5.1: tile decomposition, an atomic task counter,
@@ -17,8 +17,8 @@
 //    tile's done1.
 //  - down task (tile, n): waits until done1[tile] covers every up task of the tile (bounded
 //    spin), then A = the tile's h rows, B = 256 rows of W_down^e; the epilogue scales each
-//    row by its router weight and writes it (fp32) to the tile's rows of y. The combine
-//    kernel sums each token's rows in slot order.
+//    row by its router weight and writes it (bf16) to the tile's rows of y. The combine
+//    kernel sums each token's rows in slot order in fp32.
 //  - epilogue results go through two 16 KB shared-memory staging buffers (128-byte swizzled)
 //    and asynchronous TMA tensor stores, so the epilogue warps release TMEM and move on
 //    while the stores drain.
@@ -327,7 +327,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           red_release_add_gpu(&ws.done1[t.tile], 1);
         }
       } else {
-        // y = w * (h W_down^T), eight chunks of 32 fp32 columns
+        // y = w * (h W_down^T) rounded to bf16, four chunks of 64 columns
         float w = 0.f;
         if (row < t.nrows) {
           if (shared) {
@@ -338,25 +338,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
 #pragma unroll 1
-        for (int cc = 0; cc < kBN2 / 32; ++cc) {
+        for (int cc = 0; cc < kBN2 / 64; ++cc) {
           uint8_t* buf = staging + sb * kStagingBytes;
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(tacc + cc * 32, v);
-          tmem_ld_wait();
-          if (cc == kBN2 / 32 - 1) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(tacc + cc * 64 + half * 32, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              pk[half * 16 + j] = pack_bf16x2(w * __uint_as_float(v[2 * j]), w * __uint_as_float(v[2 * j + 1]));
+          }
+          if (cc == kBN2 / 64 - 1) {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[acc]);
           }
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(w * __uint_as_float(v[j]));
           if (leader) bulk_wait_group_read<kNumStaging - 1>();
           named_bar_sync(1, 128);
-          put_row(buf, v);
+          put_row(buf, pk);
           fence_proxy_async_shared();
           named_bar_sync(1, 128);
           if (leader) {
-            tma_store_2d(&maps.y, smem_u32(buf), t.n0 + cc * 32, t.tile * kBM);
+            tma_store_2d(&maps.y, smem_u32(buf), t.n0 + cc * 64, t.tile * kBM);
             bulk_commit_group();
           }
           sb ^= 1;

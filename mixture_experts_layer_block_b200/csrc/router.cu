@@ -2,12 +2,16 @@
 //
 // Router projection of the Mixture-of-Kittens layer ("Overlapping compute and communication
 // in MoE": the router projection picks the top-k routed experts of each token). A dense
-// contraction, so it runs on the tensor cores: one CTA per 128 x BN output tile, TMA-fed
-// 4-stage smem ring (x tile 128 x 64, W tile BN x 64, both 128-byte swizzled), tcgen05.mma
-// with the fp32 accumulator in TMEM, and an epilogue warpgroup that adds the bias and
-// stores fp32 rows.
+// contraction, so it runs on the tensor cores: one CTA per 128 x BN output tile and K split
+// (blockIdx.z), TMA-fed smem ring (x tile 128 x 64, W tile BN x 64, both 128-byte swizzled),
+// tcgen05.mma with the fp32 accumulator in TMEM, and an epilogue warpgroup that stores fp32
+// rows. With K split S ways (S = 1, 2 or 4, so that few tokens still fill the GPU) CTA z
+// writes partial z of [S][T][E] (the bias goes into partial 0); the gating kernel adds the
+// partials in split order, so the sum does not depend on which CTA finished first.
 //
 // Warp roles: warp 0 TMA producer, warp 1 TMEM allocator + MMA issuer, warps 2-5 epilogue.
+#include <algorithm>
+
 #include "launch.h"
 
 namespace moe {
@@ -35,7 +39,7 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)
 __global__ void __launch_bounds__(kRThreads, 1)
     router_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CUtensorMap w_map,
                   const float* __restrict__ bias, float* __restrict__ logits, int T, int E, int H,
-                  int BN, DeviceMeta* meta, int64_t timeout_ns) {
+                  int BN, int kb_per_split, DeviceMeta* meta, int64_t timeout_ns) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int b_bytes = BN * kBK * 2;
@@ -49,7 +53,10 @@ __global__ void __launch_bounds__(kRThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * kBM, n0 = blockIdx.y * BN;
-  const int nk = ceil_div(H, kBK);
+  const int kb0 = blockIdx.z * kb_per_split;
+  const int nk = min(ceil_div(H, kBK) - kb0, kb_per_split);  // >= 1 by construction of the grid
+  logits += (size_t)blockIdx.z * T * E;
+  if (blockIdx.z != 0) bias = nullptr;
   const uint32_t ncols = tmem_cols_for(BN);
 
   if (threadIdx.x == 0) {
@@ -81,8 +88,8 @@ __global__ void __launch_bounds__(kRThreads, 1)
         if (!wait_bar(&empty[stage], phase ^ 1, meta, s_abort, timeout_ns, kSiteRouter)) break;
         const uint32_t a = smem_u32(smem + stage * stage_bytes);
         mbar_arrive_expect_tx(&full[stage], kRABytes + b_bytes);
-        tma_load_2d(a, &x_map, &full[stage], kb * kBK, m0);
-        tma_load_2d(a + kRABytes, &w_map, &full[stage], kb * kBK, n0);
+        tma_load_2d(a, &x_map, &full[stage], (kb0 + kb) * kBK, m0);
+        tma_load_2d(a + kRABytes, &w_map, &full[stage], (kb0 + kb) * kBK, n0);
         if (++stage == kRouterStages) { stage = 0; phase ^= 1; }
       }
     }
@@ -111,20 +118,19 @@ __global__ void __launch_bounds__(kRThreads, 1)
     // epilogue: thread owns one output row
     const int q = warp & 3;
     const int row = q * 32 + lane;
+    const int t = m0 + row;
     const bool ok = wait_bar(acc_full, 0, meta, s_abort, timeout_ns, kSiteRouter);
     tc_fence_after();
     if (ok) {
-      const int t = m0 + row;
       for (int c = 0; c < BN; c += 16) {
         uint32_t v[16];
         tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(q * 32) << 16) + c, v);
         tmem_ld_wait();
         if (t < T) {
-          float* dst = logits + (size_t)t * E;
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int e = n0 + c + j;
-            if (e < E) dst[e] = __uint_as_float(v[j]) + (bias ? bias[e] : 0.f);
+            if (e < E) logits[(size_t)t * E + e] = __uint_as_float(v[j]) + (bias ? bias[e] : 0.f);
           }
         }
       }
@@ -151,12 +157,24 @@ size_t router_smem_bytes(int BN) {
   return (size_t)kRouterStages * stage_bytes + 1024 /*align*/ + 256 /*barriers*/;
 }
 
+int router_splits(int T, int E, int H, int BN, int num_sms) {
+  const int tiles = ceil_div(T, kBM) * ceil_div(E, BN);
+  const int nk = ceil_div(H, kBK);
+  // S in {1, 2, 4}: about one wave of CTAs, and at least kRouterStages K steps per CTA
+  int S = 1;
+  while (S < kMaxRouterSplits && 2 * S * tiles <= num_sms && nk / (2 * S) >= kRouterStages) S *= 2;
+  return S;
+}
+
 cudaError_t launch_router(const CUtensorMap& x_map, const CUtensorMap& w_map, const float* bias,
-                          float* logits, int T, int E, int H, int BN, DeviceMeta* meta,
+                          float* logits, int T, int E, int H, int BN, int splits, DeviceMeta* meta,
                           int64_t timeout_ns, cudaStream_t stream) {
-  dim3 grid(ceil_div(T, kBM), ceil_div(E, BN));
+  const int nk = ceil_div(H, kBK);
+  const int kps = ceil_div(nk, splits);  // splits divides the K steps evenly or leaves a short tail
+  dim3 grid(ceil_div(T, kBM), ceil_div(E, BN), ceil_div(nk, kps));
+  if ((int)grid.z != splits) return cudaErrorInvalidValue;  // the gating sums exactly `splits` partials
   router_kernel<<<grid, kRThreads, router_smem_bytes(BN), stream>>>(x_map, w_map, bias, logits, T, E,
-                                                                     H, BN, meta, timeout_ns);
+                                                                     H, BN, kps, meta, timeout_ns);
   return cudaGetLastError();
 }
 
