@@ -201,6 +201,30 @@ MOE_API int moe_trace_read(moe_handle *h, int64_t *records, int64_t cap, int64_t
  * moe_get_status. The hook clears itself after one forward. */
 MOE_API int moe_debug_inject_stall(moe_handle *h, int32_t extra);
 
+/* Allocation-free variant of moe_align_block_size. The pages have no counterpart: this entry
+ * exists for callers that cannot let this library allocate device memory, such as a serving
+ * runtime that owns all of HBM through its own allocator, or a latency-critical path that
+ * cannot afford a cudaMalloc (which may synchronise the device). It needs no handle and never
+ * allocates: the kernels' scratch memory is a fixed array of about 68 KB compiled into the
+ * library, which every GPU that loads the library keeps until the process exits.
+ *   topk_ids        device int32 [T][top_k], expert ids in [0, num_experts)
+ *   num_experts     1..256;  T * top_k <= 131072  (larger: MOE_ERR_UNSUPPORTED)
+ *   block_m, capacity_factor   as moe_config.block_m / capacity_factor
+ *   sorted_ids      device int32 [T*top_k + num_experts*(block_m-1)]
+ *   expert_ids      device int32 [ceil(that / block_m)]
+ *   num_post_padded device int32 [1]
+ * Outputs are those of moe_align_block_size for the same arguments. The first call on each
+ * device looks up the array's device address and the SM count on the calling thread's current
+ * device; make that first call before any stream capture. Every call uses the same array:
+ * each call clears what it needs, but calls whose work overlaps on the GPU (different streams,
+ * or different host threads without ordering) race on it and must be serialised by the
+ * caller. */
+MOE_API int moe_align_block_size_noalloc(const int32_t *topk_ids, int32_t T, int32_t top_k,
+                                         int32_t num_experts, int32_t block_m,
+                                         float capacity_factor, int32_t *sorted_ids,
+                                         int32_t *expert_ids, int32_t *num_post_padded,
+                                         void *stream);
+
 /* Human-readable name of a MOE_* status code. */
 MOE_API const char *moe_status_string(int code);
 

@@ -506,6 +506,23 @@ cudaError_t launch_scatter(const int32_t* topk_ids, int32_t* sorted_ids, int32_t
   return cudaGetLastError();
 }
 
+// Raise (never lower) the dynamic shared memory limits of the histogram and scatter kernels
+// to what one launch needs; the limit is per kernel and process-wide, and a handle may have
+// set it to its own, smaller, need.
+cudaError_t ensure_align_smem(size_t hist_bytes, size_t scatter_bytes) {
+  cudaFuncAttributes a{};
+  cudaError_t err;
+  if ((err = cudaFuncGetAttributes(&a, hist_kernel))) return err;
+  if ((size_t)a.maxDynamicSharedSizeBytes < hist_bytes &&
+      (err = cudaFuncSetAttribute(hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hist_bytes)))
+    return err;
+  if ((err = cudaFuncGetAttributes(&a, scatter_kernel))) return err;
+  if ((size_t)a.maxDynamicSharedSizeBytes < scatter_bytes &&
+      (err = cudaFuncSetAttribute(scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)scatter_bytes)))
+    return err;
+  return cudaSuccess;
+}
+
 template <int VPL>
 static cudaError_t set_gate_smem(int s) {
   cudaError_t err;

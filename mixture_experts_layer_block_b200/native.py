@@ -62,6 +62,8 @@ SIGNATURES = {
     "moe_trace_read": (ctypes.c_int, [_P, _P, _I64, ctypes.POINTER(ctypes.c_int64)]),
     "moe_debug_inject_stall": (ctypes.c_int, [_P, _I32]),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "moe_align_block_size_noalloc": (ctypes.c_int, [_P, _I32, _I32, _I32, _I32, ctypes.c_float, _P, _P, _P,
+                                                    _P]),
 }
 
 
@@ -79,6 +81,15 @@ def _load():
 
 
 lib = _load()
+
+
+def align_block_size_noalloc(topk_ids, num_experts, block_m, capacity_factor, sorted_ids, expert_ids,
+                             num_post_padded, stream=None):
+    """moe_align_block_size_noalloc on torch CUDA tensors (no handle, no allocation)."""
+    T, k = topk_ids.shape
+    check(lib.moe_align_block_size_noalloc(_ptr(topk_ids), T, k, num_experts, block_m, float(capacity_factor),
+                                           _ptr(sorted_ids), _ptr(expert_ids), _ptr(num_post_padded),
+                                           _stream(stream)), "moe_align_block_size_noalloc")
 
 
 class MoEError(RuntimeError):
