@@ -36,6 +36,32 @@ UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one expert-GEMM launch, from
+# the ncu captures summarised under profiles/, with the hash of the kernel sources it was taken
+# on. A different hash (the kernel changed since) reports null.
+KERNEL_SOURCES = ["mixture_experts_layer_block_b200/csrc/moe_gemm.cu",
+                  "mixture_experts_layer_block_b200/csrc/common.cuh",
+                  "mixture_experts_layer_block_b200/csrc/ptx.cuh",
+                  "mixture_experts_layer_block_b200/csrc/launch.h"]
+MEASURED_TRAFFIC = {"flashmoe_prefill": ("ab2282bf59bc49fc", 1.676179e9 + 0.064273e9)}
+
+
+def kernel_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(workload: str):
+    rec = MEASURED_TRAFFIC.get(workload)
+    if rec is None or rec[0] != kernel_source_hash():
+        return None
+    return rec[1]
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -234,7 +260,7 @@ def barrier(world: int):
 def run_reference(args, world, rank):
     if rank != 0:
         return 0
-    w = configs.WORKLOADS[args.workload]
+    w = workload_of(args)
     wts = gen.make_weights(w, "cpu")
     x = gen.make_x(w, "cpu")
     from oracle import oracle
@@ -267,6 +293,8 @@ def main():
     ap.add_argument("--no-trace", action="store_true", help="skip the traced forward (SM-busy)")
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--ref-tokens", type=int, default=256)
+    ap.add_argument("--T", type=int, default=None, help="override the workload's token count (profiling)")
+    ap.add_argument("--E", type=int, default=None, help="override the workload's expert count (profiling)")
     ap.add_argument("--traffic-bytes", type=float, default=None,
                     help="ncu dram bytes per launch of the expert-GEMM kernel, if captured")
     args = ap.parse_args()
@@ -281,10 +309,19 @@ def main():
             dist.destroy_process_group()
 
 
+def workload_of(args):
+    w = configs.WORKLOADS[args.workload]
+    if args.T is not None:
+        w = w.replace(T=args.T)
+    if args.E is not None:
+        w = w.replace(E=args.E)
+    return w
+
+
 def run_mine(args, world, rank, local):
     from mixture_experts_layer_block_b200.native import (MOE_FLAG_HOST_STAGING, MOE_FLAG_STAGE_TIMING,
                                                          MoELayer)
-    w = configs.WORKLOADS[args.workload]
+    w = workload_of(args)
     dev = torch.device("cuda", local)
     wts = gen.make_weights(w, dev)
     x = gen.make_x(w.replace(seed=w.seed + 1000 * rank) if rank else w, dev)  # each replica its own tokens
@@ -350,7 +387,8 @@ def run_mine(args, world, rank, local):
         achieved = gemm_flops / (gemm_ms * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": achieved / peaks["bf16_tflops"]}
-    roof.update({"traffic": args.traffic_bytes, "kernel": "moe_gemm_kernel",
+    traffic = args.traffic_bytes if args.traffic_bytes is not None else measured_traffic(w.name)
+    roof.update({"traffic": traffic, "kernel": "moe_gemm_kernel",
                  "algorithmic_bytes": gbytes, "kernel_ms": gemm_ms, "peak_source": peak_src})
 
     line = {"metric": METRIC, "value": tokens_per_s, "unit": UNIT, "n_gpus": world, "steps": args.steps,

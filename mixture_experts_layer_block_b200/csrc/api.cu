@@ -140,8 +140,12 @@ Shape make_shape(const moe_handle* h, int T, int k) {
   sh.num_chunks = std::max(1, ceil_div(T, sh.chunk_tokens));
   sh.sorted_len = T * k + c.num_experts * (c.block_m - 1);
   sh.blocks_len = ceil_div(sh.sorted_len, c.block_m);
+  // A tile's down tasks are numbered `lag` units after its up tasks: at least two waves of
+  // tasks and one and a half waves of up tasks in between, so that a claimed down task rarely
+  // finds its tile's up tasks still running.
   const int n1 = ceil_div(c.inter, kBN1), n2 = ceil_div(c.hidden, kBN2);
-  sh.lag = std::max(1, std::min(h->max_lag, ceil_div(2 * h->num_sms, n1 + n2)));
+  const int lag = std::max(ceil_div(2 * h->num_sms, n1 + n2), ceil_div(3 * h->num_sms, 2 * n1));
+  sh.lag = std::max(1, std::min(h->max_lag, lag));
   sh.dep_extra = 0;
   sh.timeout_ns = h->timeout_ns;
   return sh;

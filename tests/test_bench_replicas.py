@@ -38,6 +38,8 @@ def _worker(rank, world, port, q):
         warmup = 1
         gpus = world
         ref_tokens = 8
+        T = None
+        E = None
     buf = io.StringIO()
     with redirect_stdout(buf):
         rc = bench.run_reference(A, w, r)
