@@ -19,6 +19,8 @@ namespace moe {
 
 __global__ void __launch_bounds__(256)
     gather_rows_kernel(const uint16_t* __restrict__ x, Workspace ws, Shape sh) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int nw = (gridDim.x * blockDim.x) >> 5;
@@ -54,6 +56,8 @@ __device__ __forceinline__ void add_bf16x8(float (&acc)[8], const uint4 v) {
 // One warp per (token, 256 columns); each lane sums 8 columns.
 __global__ void __launch_bounds__(256)
     combine_kernel(float* __restrict__ out, Workspace ws, Shape sh) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int nw = (gridDim.x * blockDim.x) >> 5;
@@ -80,15 +84,13 @@ __global__ void __launch_bounds__(256)
 
 cudaError_t launch_gather_rows(const uint16_t* x, const Workspace& ws, const Shape& sh, int grid,
                                cudaStream_t stream) {
-  gather_rows_kernel<<<grid, 256, 0, stream>>>(x, ws, sh);
-  return cudaGetLastError();
+  return launch_k(gather_rows_kernel, dim3(grid), dim3(256), 0, stream, x, ws, sh);
 }
 
 cudaError_t launch_combine(float* out, const Workspace& ws, const Shape& sh, cudaStream_t stream) {
   const int64_t warps = (int64_t)sh.T * ceil_div(sh.H, 256);
   const int grid = (int)std::min<int64_t>((warps + 7) / 8, 148 * 32);
-  combine_kernel<<<grid, 256, 0, stream>>>(out, ws, sh);
-  return cudaGetLastError();
+  return launch_k(combine_kernel, dim3(grid), dim3(256), 0, stream, out, ws, sh);
 }
 
 }  // namespace moe

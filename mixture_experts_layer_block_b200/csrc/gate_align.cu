@@ -279,6 +279,8 @@ __global__ void __launch_bounds__(kGateThreads)
     gate_kernel(const float* __restrict__ parts, float* __restrict__ logits_out,
                 int32_t* __restrict__ topk_ids, float* __restrict__ topk_w, Workspace ws, Shape sh,
                 int hist_on, int tiles) {
+  griddep_wait();
+  griddep_launch_dependents();
   extern __shared__ int smem_i[];
   int* hist = smem_i;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -319,6 +321,8 @@ __global__ void __launch_bounds__(kGateThreads)
 
 __global__ void __launch_bounds__(kGateThreads)
     hist_kernel(const int32_t* __restrict__ topk_ids, Workspace ws, Shape sh) {
+  griddep_wait();
+  griddep_launch_dependents();
   extern __shared__ int smem_i[];
   int* hist = smem_i;
   for (int e = threadIdx.x; e < sh.E; e += blockDim.x) hist[e] = 0;
@@ -356,6 +360,8 @@ __global__ void __launch_bounds__(kGateThreads)
     scatter_kernel(const int32_t* __restrict__ topk_ids, int32_t* __restrict__ sorted_ids,
                    int32_t* __restrict__ expert_ids, int32_t* __restrict__ num_post_padded,
                    int32_t* __restrict__ row_of_slot, Workspace ws, Shape sh) {
+  griddep_wait();
+  griddep_launch_dependents();
   extern __shared__ int smem_i[];
   constexpr int kWarps = kGateThreads / 32;
   const int E = sh.E;
@@ -463,9 +469,8 @@ template <int VPL, int S>
 static cudaError_t launch_gate_vs(const float* parts, float* logits_out, int32_t* ids, float* w,
                                   const Workspace& ws, const Shape& sh, bool hist, bool tiles,
                                   size_t smem, cudaStream_t st) {
-  gate_kernel<VPL, S><<<gate_grid(sh), kGateThreads, hist ? smem : 0, st>>>(
-      parts, logits_out, ids, w, ws, sh, hist ? 1 : 0, tiles ? 1 : 0);
-  return cudaGetLastError();
+  return launch_k(gate_kernel<VPL, S>, dim3(gate_grid(sh)), dim3(kGateThreads), hist ? smem : 0, st, parts,
+                  logits_out, ids, w, ws, sh, hist ? 1 : 0, tiles ? 1 : 0);
 }
 
 template <int VPL>
@@ -493,17 +498,15 @@ cudaError_t launch_gate(const float* parts, int splits, float* logits_out, int32
 
 cudaError_t launch_hist(const int32_t* topk_ids, const Workspace& ws, const Shape& sh, size_t smem,
                         cudaStream_t st) {
-  hist_kernel<<<gate_grid(sh), kGateThreads, smem, st>>>(topk_ids, ws, sh);
-  return cudaGetLastError();
+  return launch_k(hist_kernel, dim3(gate_grid(sh)), dim3(kGateThreads), smem, st, topk_ids, ws, sh);
 }
 
 cudaError_t launch_scatter(const int32_t* topk_ids, int32_t* sorted_ids, int32_t* expert_ids,
                            int32_t* num_post_padded, int32_t* row_of_slot, const Workspace& ws,
                            const Shape& sh, int grid, cudaStream_t st) {
   const size_t smem = scatter_smem_bytes(sh.E, sh.chunk_tokens * sh.k);
-  scatter_kernel<<<std::max(grid, sh.num_chunks), kGateThreads, smem, st>>>(
-      topk_ids, sorted_ids, expert_ids, num_post_padded, row_of_slot, ws, sh);
-  return cudaGetLastError();
+  return launch_k(scatter_kernel, dim3(std::max(grid, sh.num_chunks)), dim3(kGateThreads), smem, st, topk_ids,
+                  sorted_ids, expert_ids, num_post_padded, row_of_slot, ws, sh);
 }
 
 // Raise (never lower) the dynamic shared memory limits of the histogram and scatter kernels

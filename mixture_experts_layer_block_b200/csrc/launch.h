@@ -3,9 +3,30 @@
 
 #include <cuda_runtime.h>
 
+#include <utility>
+
 #include "common.cuh"
 
 namespace moe {
+
+// Launch with programmatic stream serialisation: the kernel may be scheduled while the previous
+// kernel of the stream finishes, runs its prologue, and waits (griddep_wait) before it touches
+// global memory; the previous kernel lets it in with griddep_launch_dependents.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                     Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Tensor maps of the persistent expert-GEMM kernel.
 struct alignas(64) GemmMaps {

@@ -121,6 +121,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
+  griddep_wait();  // inputs of earlier kernels are complete from here on
   uint32_t nfill = 0;  // TMA stage fills issued by this CTA (producer warp)
   bool mma_issued = false;
 
@@ -379,6 +380,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (leader) bulk_wait_group<0>();
   }
 
+  // the next kernel may start its prologue once every CTA has finished its tasks (not earlier:
+  // its waiting CTAs would share the SMs with the tensor-core pipeline)
+  griddep_launch_dependents();
   // teardown: every TMA fill and tcgen05 op issued by this CTA must be complete before the
   // CTA releases TMEM and exits (this only waits after an abort)
   tc_fence_before();
@@ -399,8 +403,7 @@ size_t gemm_smem_bytes() { return (size_t)SmemLayout::kBytes + 1024; }
 
 cudaError_t launch_moe_gemm(const GemmMaps& maps, const Workspace& ws, const Shape& sh, int grid,
                             cudaStream_t stream) {
-  moe_gemm_kernel<<<grid, kGemmThreads, gemm_smem_bytes(), stream>>>(maps, ws, sh);
-  return cudaGetLastError();
+  return launch_k(moe_gemm_kernel, dim3(grid), dim3(kGemmThreads), gemm_smem_bytes(), stream, maps, ws, sh);
 }
 
 cudaError_t configure_gemm_kernel() {

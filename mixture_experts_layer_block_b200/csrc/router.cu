@@ -80,6 +80,8 @@ __global__ void __launch_bounds__(kRThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
   uint32_t nfill = 0;  // TMA fills issued (producer lane)
+  griddep_wait();  // inputs of earlier kernels are complete from here on
+  griddep_launch_dependents();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -173,9 +175,8 @@ cudaError_t launch_router(const CUtensorMap& x_map, const CUtensorMap& w_map, co
   const int kps = ceil_div(nk, splits);  // splits divides the K steps evenly or leaves a short tail
   dim3 grid(ceil_div(T, kBM), ceil_div(E, BN), ceil_div(nk, kps));
   if ((int)grid.z != splits) return cudaErrorInvalidValue;  // the gating sums exactly `splits` partials
-  router_kernel<<<grid, kRThreads, router_smem_bytes(BN), stream>>>(x_map, w_map, bias, logits, T, E,
-                                                                     H, BN, kps, meta, timeout_ns);
-  return cudaGetLastError();
+  return launch_k(router_kernel, grid, dim3(kRThreads), router_smem_bytes(BN), stream, x_map, w_map, bias,
+                  logits, T, E, H, BN, kps, meta, timeout_ns);
 }
 
 cudaError_t configure_router_kernel() {
