@@ -67,6 +67,7 @@ struct moe_handle {
   EncodeTiledFn encode = nullptr;
   std::vector<MapEntry> cache;
   CUtensorMap h_routed{}, h_shared{}, xs_map{}, y_map{};
+  CUtensorMap h_routed16{}, h_shared16{}, xs_map16{};  // 16-row boxes for batches of <= 16 tokens
   int max_routed_tiles = 0;
   int parts_rows = 0;  // rows of the K-split partial logits buffer
   std::vector<cudaEvent_t> ev;  // kTimingRing x (kNumStages + 1) events around the kernels
@@ -298,6 +299,17 @@ int moe_init(const moe_config* cfg, moe_handle** out) {
   if ((rc = encode_map(h, &h->xs_map, w.xs, c.hidden, (uint64_t)h->max_routed_tiles * kBM,
                        (uint64_t)c.hidden * 2, kBK, kBM)))
     return fail(rc);
+  if ((rc = encode_map(h, &h->xs_map16, w.xs, c.hidden, (uint64_t)h->max_routed_tiles * kBM,
+                       (uint64_t)c.hidden * 2, kBK, kSmallRows)))
+    return fail(rc);
+  if ((rc = encode_map(h, &h->h_routed16, w.h, c.inter, h_rows, (uint64_t)ldh * 2, kBK, kSmallRows)))
+    return fail(rc);
+  if (c.inter_shared > 0) {
+    if ((rc = encode_map(h, &h->h_shared16, w.h, c.inter_shared, h_rows, (uint64_t)ldh * 2, kBK, kSmallRows)))
+      return fail(rc);
+  } else {
+    h->h_shared16 = h->h_routed16;
+  }
   if ((rc = encode_map(h, &h->y_map, w.y, c.hidden, h_rows, (uint64_t)c.hidden * 2, kBK, kBM))) return fail(rc);
 
   // kernel attributes
@@ -384,24 +396,33 @@ static int forward_impl(moe_handle* h, const void* x, int32_t T, const void* w_r
   CUtensorMap wr_map;
   GemmMaps maps;
   const int bn = router_bn(E);
-  if ((rc = encode_map(h, &maps.x_tile, x, H, T, (uint64_t)H * 2, kBK, kBM))) return rc;
-  maps.xs = h->xs_map;
+  // With at most 16 tokens every m-tile has at most 16 rows (an expert appears once per token):
+  // the expert GEMMs use their small-tile shape with 16-row A boxes.
+  const bool small = T <= kSmallRows;
+  CUtensorMap x_router;
+  if ((rc = encode_map(h, &x_router, x, H, T, (uint64_t)H * 2, kBK, kBM))) return rc;
+  if (small) {
+    if ((rc = encode_map(h, &maps.x_tile, x, H, T, (uint64_t)H * 2, kBK, kSmallRows))) return rc;
+  } else {
+    maps.x_tile = x_router;
+  }
+  maps.xs = small ? h->xs_map16 : h->xs_map;
   maps.y = h->y_map;
   if ((rc = cached_map(h, &wr_map, w_router, H, E, (uint64_t)H * 2, kBK, bn))) return rc;
   if ((rc = cached_map(h, &maps.w_up, w_up, H, (uint64_t)E * D, (uint64_t)H * 2, kBK, kBN1))) return rc;
   if ((rc = cached_map(h, &maps.w_gate, w_gate, H, (uint64_t)E * D, (uint64_t)H * 2, kBK, kBN1))) return rc;
   if ((rc = cached_map(h, &maps.w_down, w_down, D, (uint64_t)E * H, (uint64_t)D * 2, kBK, kBN2))) return rc;
-  maps.h_routed = h->h_routed;
+  maps.h_routed = small ? h->h_routed16 : h->h_routed;
   if (has_shared) {
     if ((rc = cached_map(h, &maps.ws_up, w_shared->up, H, Ds, (uint64_t)H * 2, kBK, kBN1))) return rc;
     if ((rc = cached_map(h, &maps.ws_gate, w_shared->gate, H, Ds, (uint64_t)H * 2, kBK, kBN1))) return rc;
     if ((rc = cached_map(h, &maps.ws_down, w_shared->down, Ds, H, (uint64_t)Ds * 2, kBK, kBN2))) return rc;
-    maps.h_shared = h->h_shared;
+    maps.h_shared = small ? h->h_shared16 : h->h_shared;
   } else {
     maps.ws_up = maps.w_up;
     maps.ws_gate = maps.w_gate;
     maps.ws_down = maps.w_down;
-    maps.h_shared = h->h_routed;
+    maps.h_shared = maps.h_routed;
   }
 
   cudaEvent_t* ev = nullptr;
@@ -412,7 +433,7 @@ static int forward_impl(moe_handle* h, const void* x, int32_t T, const void* w_r
   int splits = router_splits(T, E, H, bn, h->num_sms);
   while (splits > 1 && (int64_t)splits * T > h->parts_rows) splits /= 2;
   float* parts = splits > 1 ? w.logit_parts : w.logits;
-  if ((rc = check_cuda(launch_router(maps.x_tile, wr_map, router_bias, parts, T, E, H, bn, splits, w.meta,
+  if ((rc = check_cuda(launch_router(x_router, wr_map, router_bias, parts, T, E, H, bn, splits, w.meta,
                                      h->timeout_ns, st))))
     return rc;
   if ((rc = mark(1))) return rc;
@@ -426,7 +447,7 @@ static int forward_impl(moe_handle* h, const void* x, int32_t T, const void* w_r
   if ((rc = mark(3))) return rc;
   if ((rc = check_cuda(launch_gather_rows(x16, w, sh, 4 * h->num_sms, st)))) return rc;
   if ((rc = mark(4))) return rc;
-  if ((rc = check_cuda(launch_moe_gemm(maps, w, sh, h->num_sms, st)))) return rc;
+  if ((rc = check_cuda(launch_moe_gemm(maps, w, sh, h->num_sms, small, st)))) return rc;
   if ((rc = mark(5))) return rc;
   if ((rc = check_cuda(launch_combine(out, w, sh, st)))) return rc;
   if ((rc = mark(6))) return rc;

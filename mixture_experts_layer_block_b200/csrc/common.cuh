@@ -24,6 +24,7 @@ constexpr int kStagingBytes = 128 * 128;  // one epilogue staging buffer: 128 ro
 constexpr int kNumStaging = 2;            // double-buffered epilogue -> TMA store staging
 constexpr int kAccCols = 256;   // TMEM columns per accumulator buffer (2 buffers)
 constexpr int kGemmThreads = 192;  // warp 0 producer, warp 1 MMA, warps 2-5 epilogue
+constexpr int kSmallRows = 16;     // A-tile rows of the expert GEMMs' small-tile shape (T <= 16)
 
 // ---- router GEMM -------------------------------------------------------------------------
 constexpr int kRouterStages = 6;

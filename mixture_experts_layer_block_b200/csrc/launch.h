@@ -81,10 +81,11 @@ cudaError_t launch_gather_rows(const uint16_t* x, const Workspace& ws, const Sha
 // out[t] = (shared row of t) + sum_j y[row_of_slot[t*k+j]], in that order, fp32.
 cudaError_t launch_combine(float* out, const Workspace& ws, const Shape& sh, cudaStream_t stream);
 
-// Persistent expert GEMMs.
-size_t gemm_smem_bytes();
+// Persistent expert GEMMs. `small` selects the shape for batches of at most 16 tokens (its
+// maps must use 16-row boxes for x_tile, xs, h_routed and h_shared).
+size_t gemm_smem_bytes(bool small);
 cudaError_t launch_moe_gemm(const GemmMaps& maps, const Workspace& ws, const Shape& sh, int grid,
-                            cudaStream_t stream);
+                            bool small, cudaStream_t stream);
 
 // One-time kernel attribute setup (dynamic shared memory limits).
 cudaError_t configure_kernels(size_t gate_smem);

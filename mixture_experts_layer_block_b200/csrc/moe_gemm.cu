@@ -38,14 +38,29 @@ namespace moe {
 
 namespace {
 
-struct SmemLayout {
-  static constexpr int kStagingOff = kStages * kStageBytes;
-  static constexpr int kBarOff = kStagingOff + kNumStaging * kStagingBytes;
+// Two shapes of the kernel. The general one moves 128-row A tiles through a 4 x 48 KB ring
+// and writes its epilogue results with TMA stores from two staging buffers. The small-tile
+// one serves batches of at most 16 tokens (every m-tile then holds at most 16 rows): it moves
+// 16-row A boxes (2 KB), so the same shared memory holds a 6 x 34 KB ring and 50% more weight
+// bytes in flight per SM, and its epilogue stores the valid rows directly. Its MMAs stay
+// M=128: rows 16..127 read the stage's B bytes (finite values) and their results are never
+// stored.
+template <bool kSmall>
+struct Cfg {
+  static constexpr int kStagesN = kSmall ? 6 : kStages;
+  static constexpr int kARows = kSmall ? 16 : kBM;
+  static constexpr int kABytesN = kARows * kBK * 2;
+  static constexpr int kStageBytesN = kABytesN + kBBytes;
+  static constexpr int kNumStagingN = kSmall ? 0 : kNumStaging;
+  static constexpr int kStagingOff = kStagesN * kStageBytesN;
+  static constexpr int kBarOff = kStagingOff + kNumStagingN * kStagingBytes;
   // barriers: full[S], empty[S], acc_full[2], acc_empty[2], task_full[R], task_empty[R], drain
-  static constexpr int kNumBars = 2 * kStages + 4 + 2 * kTaskSlots + 1;
+  static constexpr int kNumBars = 2 * kStagesN + 4 + 2 * kTaskSlots + 1;
   static constexpr int kRingOff = kBarOff + ((kNumBars * 8 + 63) & ~63);
   static constexpr int kMiscOff = kRingOff + kTaskSlots * (int)sizeof(Task);
   static constexpr int kBytes = kMiscOff + 64;
+  static_assert(kStageBytesN % 1024 == 0 && kABytesN % 1024 == 0, "1024-byte aligned operand tiles");
+  static_assert(kBytes + 1024 <= 227 * 1024, "shared memory budget");
 };
 
 __device__ __forceinline__ int n1_of(int expert, const Shape& sh) {
@@ -70,11 +85,16 @@ __device__ __noinline__ bool wait_count(const int* p, int need, DeviceMeta* meta
 
 }  // namespace
 
+template <bool kSmall>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     moe_gemm_kernel(const __grid_constant__ GemmMaps maps, Workspace ws, Shape sh) {
+  using C = Cfg<kSmall>;
+  constexpr int kStages = C::kStagesN;
+  constexpr int kStageBytes = C::kStageBytesN;
+  constexpr int kABytes = C::kABytesN;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SmemLayout::kBarOff);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
   uint64_t* full = bars;
   uint64_t* empty = full + kStages;
   uint64_t* acc_full = empty + kStages;
@@ -82,9 +102,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* task_full = acc_empty + 2;
   uint64_t* task_empty = task_full + kTaskSlots;
   uint64_t* drain = task_empty + kTaskSlots;
-  Task* ring = reinterpret_cast<Task*>(smem + SmemLayout::kRingOff);
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + SmemLayout::kMiscOff);
-  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + SmemLayout::kMiscOff + 4);
+  Task* ring = reinterpret_cast<Task*>(smem + C::kRingOff);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   DeviceMeta* meta = ws.meta;
@@ -266,8 +286,105 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int q = warp & 3;          // TMEM lane quarter this warp may read
     const int row = q * 32 + lane;   // tile row owned by this thread
     const bool leader = (warp == 2 && lane == 0);
-    uint8_t* staging = smem + SmemLayout::kStagingOff;
+    uint8_t* staging = smem + C::kStagingOff;
     uint32_t slot = 0, slot_phase = 0, acc = 0, acc_phase = 0, sb = 0;
+    if constexpr (kSmall) {
+      // at most 16 valid rows per tile: only the warp of TMEM lanes 0-31 has work, and the
+      // valid rows are stored straight from registers (no staging, no TMA stores)
+      while (true) {
+        if (!wait_bar(&task_full[slot], slot_phase, meta, s_abort, limit, kSiteEpiTask)) break;
+        const Task t = ring[slot];
+        if (t.kind == kTaskStop) break;
+        if (!wait_bar(&acc_full[acc], acc_phase, meta, s_abort, limit, kSiteEpiAcc)) break;
+        tc_fence_after();
+        const uint32_t tacc = tmem_base + acc * kAccCols + (static_cast<uint32_t>(q * 32) << 16);
+        const bool shared = (t.expert == sh.E);
+        const bool has_rows = q * 32 < t.nrows;  // warp-uniform
+        const bool valid = row < t.nrows;
+        if (t.kind == kTaskUp) {
+          const int Dt = shared ? sh.Ds : sh.D;
+          uint16_t* hrow = ws.h + (size_t)(t.tile * kBM + row) * ws.ldh;
+          if (has_rows) {
+#pragma unroll 1
+            for (int cc = 0; cc < kBN1 / 64; ++cc) {
+              uint32_t pk[32];
+#pragma unroll
+              for (int half = 0; half < 2; ++half) {
+                uint32_t u[32], g[32];
+                tmem_ld_32x32b_x32(tacc + cc * 64 + half * 32, u);
+                tmem_ld_32x32b_x32(tacc + kBN1 + cc * 64 + half * 32, g);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                  const float u0 = __uint_as_float(u[2 * j]), u1 = __uint_as_float(u[2 * j + 1]);
+                  const float g0 = __uint_as_float(g[2 * j]), g1 = __uint_as_float(g[2 * j + 1]);
+                  pk[half * 16 + j] = pack_bf16x2(__fdividef(u0, 1.0f + __expf(-u0)) * g0,
+                                                  __fdividef(u1, 1.0f + __expf(-u1)) * g1);
+                }
+              }
+              const int col = t.n0 + cc * 64;
+              if (valid) {
+#pragma unroll
+                for (int v = 0; v < 8; ++v)
+                  if (col + 8 * v + 8 <= Dt)
+                    *reinterpret_cast<uint4*>(hrow + col + 8 * v) =
+                        make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+              }
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[acc]);
+          // publish h: this tile's down tasks read it with TMA (async proxy) on other SMs
+          fence_proxy_async_global();
+          __threadfence();
+          named_bar_sync(1, 128);
+          if (leader) red_release_add_gpu(&ws.done1[t.tile], 1);
+        } else {
+          float w = 0.f;
+          if (valid) {
+            if (shared) {
+              w = 1.f;
+            } else {
+              const int s = __ldcg(&ws.sorted_ids[t.row0 + row]);
+              w = __ldcg(&ws.topk_w[s]);
+            }
+          }
+          uint16_t* yrow = ws.y + (size_t)(t.tile * kBM + row) * sh.H;
+          if (has_rows) {
+#pragma unroll 1
+            for (int cc = 0; cc < kBN2 / 64; ++cc) {
+              uint32_t pk[32];
+#pragma unroll
+              for (int half = 0; half < 2; ++half) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(tacc + cc * 64 + half * 32, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                  pk[half * 16 + j] = pack_bf16x2(w * __uint_as_float(v[2 * j]), w * __uint_as_float(v[2 * j + 1]));
+              }
+              const int col = t.n0 + cc * 64;
+              if (valid) {
+#pragma unroll
+                for (int v = 0; v < 8; ++v)
+                  if (col + 8 * v + 8 <= sh.H)
+                    *reinterpret_cast<uint4*>(yrow + col + 8 * v) =
+                        make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+              }
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[acc]);
+        }
+        if (lane == 0) mbar_arrive(&task_empty[slot]);
+        if (ws.trace_cap > 0 && leader && t.id < ws.trace_cap)
+          ws.trace[(size_t)t.id * 4 + 3] = (int64_t)globaltimer_ns();
+        if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+        if (++slot == kTaskSlots) { slot = 0; slot_phase ^= 1; }
+      }
+    } else {
     // write 8 x 16 bytes (one 128-byte row) into staging buffer `buf` with the 128B swizzle
     auto put_row = [&](uint8_t* buf, const uint32_t (&w)[32]) {
 #pragma unroll
@@ -378,6 +495,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     // the staging buffers must not be released while a store still reads them
     if (leader) bulk_wait_group<0>();
+    }
   }
 
   // the next kernel may start its prologue once every CTA has finished its tasks (not earlier:
@@ -399,16 +517,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 1) tmem_dealloc(tmem_base, 2 * kAccCols);
 }
 
-size_t gemm_smem_bytes() { return (size_t)SmemLayout::kBytes + 1024; }
+size_t gemm_smem_bytes(bool small) { return (size_t)(small ? Cfg<true>::kBytes : Cfg<false>::kBytes) + 1024; }
 
 cudaError_t launch_moe_gemm(const GemmMaps& maps, const Workspace& ws, const Shape& sh, int grid,
-                            cudaStream_t stream) {
-  return launch_k(moe_gemm_kernel, dim3(grid), dim3(kGemmThreads), gemm_smem_bytes(), stream, maps, ws, sh);
+                            bool small, cudaStream_t stream) {
+  if (small)
+    return launch_k(moe_gemm_kernel<true>, dim3(grid), dim3(kGemmThreads), gemm_smem_bytes(true), stream, maps,
+                    ws, sh);
+  return launch_k(moe_gemm_kernel<false>, dim3(grid), dim3(kGemmThreads), gemm_smem_bytes(false), stream, maps,
+                  ws, sh);
 }
 
 cudaError_t configure_gemm_kernel() {
-  return cudaFuncSetAttribute(moe_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)gemm_smem_bytes());
+  cudaError_t e = cudaFuncSetAttribute(moe_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)gemm_smem_bytes(true));
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(moe_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)gemm_smem_bytes(false));
 }
 
 }  // namespace moe

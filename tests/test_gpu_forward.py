@@ -23,6 +23,11 @@ SMALL = {
     "skew_small": configs.SKEW.replace(name="skew_small", T=2000, H=512, D=256),
     "one_token": configs.DECODE.replace(name="one_token", T=1),
     "k_equals_E": configs.MoEWorkload("k_equals_E", T=200, H=256, D=128, E=4, top_k=4, block_m=16),
+    # at most 16 tokens: the expert GEMMs take their small-tile shape
+    "small_tokens_shared": configs.DSV3.replace(name="small_tokens_shared", T=12, H=512, D=256, E=16, top_k=4,
+                                                D_shared=256),
+    "small_tokens_ragged": configs.MoEWorkload("small_tokens_ragged", T=5, H=320, D=200, E=5, top_k=2,
+                                               block_m=48, D_shared=136, sigma_w=0.05, capacity_factor=1.0),
 }
 
 
