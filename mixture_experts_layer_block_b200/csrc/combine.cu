@@ -10,7 +10,7 @@
 //   tile row of y (bf16, like the per-slot intermediate cache of the vLLM execution
 //   analysis); this kernel adds, per token, the shared-expert row first and then the slots
 //   j = 0..k-1 in order (dropped slots skipped), in fp32. The order is fixed, so the result
-//   does not depend on the schedule. One warp per (token, 256 columns).
+//   does not depend on the schedule. One warp per (token, 512 columns).
 #include <algorithm>
 
 #include "launch.h"
@@ -53,7 +53,7 @@ __device__ __forceinline__ void add_bf16x8(float (&acc)[8], const uint4 v) {
   }
 }
 
-// One warp per (token, 256 columns); each lane sums 8 columns.
+// One warp per (token, 512 columns); each lane sums 8 columns in each 256-column half.
 __global__ void __launch_bounds__(256)
     combine_kernel(float* __restrict__ out, Workspace ws, Shape sh) {
   griddep_wait();
@@ -61,24 +61,40 @@ __global__ void __launch_bounds__(256)
   const int lane = threadIdx.x & 31;
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int nw = (gridDim.x * blockDim.x) >> 5;
-  const int nch = ceil_div(sh.H, 256);
   const int Mr = __ldcg(&ws.meta->num_routed_tiles);
-  const int64_t total = (int64_t)sh.T * nch;
-  for (int64_t w = gw; w < total; w += nw) {
-    const int t = (int)(w / nch);
-    const int c = (int)(w % nch) * 256 + lane * 8;
-    if (c >= sh.H) continue;
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    if (sh.Ds > 0)
-      add_bf16x8(acc, __ldcg(reinterpret_cast<const uint4*>(ws.y + ((size_t)Mr * kBM + t) * sh.H + c)));
-    for (int j = 0; j < sh.k; ++j) {
-      const int row = __ldcg(ws.row_of_slot + (size_t)t * sh.k + j);
-      if (row < 0) continue;
-      add_bf16x8(acc, __ldcg(reinterpret_cast<const uint4*>(ws.y + (size_t)row * sh.H + c)));
+  const int nblk = ceil_div(sh.H, 512);
+  const int64_t items = (int64_t)sh.T * nblk;
+  for (int64_t it = gw; it < items; it += nw) {
+    const int t = (int)(it / nblk);
+    const int c0 = (int)(it % nblk) * 512 + lane * 8, c1 = c0 + 256;
+    // this token's rows in y: the shared-expert row first, then its slots in order
+    const int myrow = (lane < sh.k) ? __ldcg(ws.row_of_slot + (size_t)t * sh.k + lane) : -1;
+    if (c0 >= sh.H) continue;
+    const bool has1 = c1 < sh.H;
+    float a0[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    float a1[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (sh.Ds > 0) {
+      const uint16_t* srow = ws.y + ((size_t)Mr * kBM + t) * sh.H;
+      add_bf16x8(a0, __ldcg(reinterpret_cast<const uint4*>(srow + c0)));
+      if (has1) add_bf16x8(a1, __ldcg(reinterpret_cast<const uint4*>(srow + c1)));
     }
-    float4* o = reinterpret_cast<float4*>(out + (size_t)t * sh.H + c);
-    o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-    o[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    for (int j = 0; j < sh.k; ++j) {
+      const int row = __shfl_sync(0xffffffffu, myrow, j);
+      if (row < 0) continue;
+      const uint16_t* yr = ws.y + (size_t)row * sh.H;
+      const uint4 v0 = __ldcg(reinterpret_cast<const uint4*>(yr + c0));
+      if (has1) add_bf16x8(a1, __ldcg(reinterpret_cast<const uint4*>(yr + c1)));
+      add_bf16x8(a0, v0);
+    }
+    float* orow = out + (size_t)t * sh.H;
+    float4* o0 = reinterpret_cast<float4*>(orow + c0);
+    o0[0] = make_float4(a0[0], a0[1], a0[2], a0[3]);
+    o0[1] = make_float4(a0[4], a0[5], a0[6], a0[7]);
+    if (has1) {
+      float4* o1 = reinterpret_cast<float4*>(orow + c1);
+      o1[0] = make_float4(a1[0], a1[1], a1[2], a1[3]);
+      o1[1] = make_float4(a1[4], a1[5], a1[6], a1[7]);
+    }
   }
 }
 
@@ -88,8 +104,8 @@ cudaError_t launch_gather_rows(const uint16_t* x, const Workspace& ws, const Sha
 }
 
 cudaError_t launch_combine(float* out, const Workspace& ws, const Shape& sh, cudaStream_t stream) {
-  const int64_t warps = (int64_t)sh.T * ceil_div(sh.H, 256);
-  const int grid = (int)std::min<int64_t>((warps + 7) / 8, 148 * 32);
+  const int64_t warps = (int64_t)sh.T * ceil_div(sh.H, 512);
+  const int grid = (int)std::min<int64_t>((warps + 7) / 8, 148 * 16);
   return launch_k(combine_kernel, dim3(grid), dim3(256), 0, stream, out, ws, sh);
 }
 

@@ -145,7 +145,8 @@ __device__ int block_exclusive_scan(int* a, int n, int* tmp) {
 
 // ------------------------------------------------------------------------------------------
 // The scans, run by the last CTA of the histogram pass. Shared memory layout (ints):
-//   tmp[64] | cnt[E] | kept[E] | tile[kMaxChunks * kScanGroup] | buf[max(E+1, units+1)]
+//   tmp[64] | cnt[E] | kept[E] | offs[E] | tile[kMaxChunks * kScanGroup] | buf[max(E+1, units+1)]
+// Everything the later steps need stays in shared memory (no reads of just-written globals).
 // ------------------------------------------------------------------------------------------
 constexpr int kScanGroup = 256;  // experts scanned per pass (tile of [chunks][256] counts)
 
@@ -155,7 +156,8 @@ __device__ void align_scans(const Workspace& ws, const Shape& sh, bool tiles, in
   int* tmp = sm;
   int* cnt = tmp + 64;
   int* kept = cnt + E;
-  int* tile = kept + E;
+  int* offs = kept + E;
+  int* tile = offs + E;
   int* buf = tile + kMaxChunks * kScanGroup;
   const int nch = sh.num_chunks;
 
@@ -195,7 +197,10 @@ __device__ void align_scans(const Workspace& ws, const Shape& sh, bool tiles, in
   }
   __syncthreads();
   const int P = block_exclusive_scan(buf, E, tmp);
-  for (int e = tid; e < E; e += nthr) ws.expert_off[e] = buf[e];
+  for (int e = tid; e < E; e += nthr) {
+    ws.expert_off[e] = buf[e];
+    offs[e] = buf[e];
+  }
   if (tid == 0) {
     ws.expert_off[E] = P;
     ws.meta->P = P;
@@ -209,7 +214,7 @@ __device__ void align_scans(const Workspace& ws, const Shape& sh, bool tiles, in
   const int Mr = block_exclusive_scan(buf, E, tmp);
   for (int e = tid; e < E; e += nthr) {
     const int first = buf[e], nt = ceil_div(kept[e], kBM);
-    const int off = ws.expert_off[e];
+    const int off = offs[e];
     ws.expert_tile0[e] = first;
     for (int i = 0; i < nt; ++i) {
       ws.tile_expert[first + i] = e;
@@ -230,9 +235,10 @@ __device__ void align_scans(const Workspace& ws, const Shape& sh, bool tiles, in
   //    u - lag. Task ids are unit-major, so every down task's dependencies have lower ids.
   const int U = (Mt > 0) ? Mt + sh.lag : 0;
   const int n2 = ceil_div(sh.H, kBN2);
+  const int n1r = ceil_div(sh.D, kBN1), n1s = ceil_div(sh.Ds, kBN1);
   for (int u = tid; u < U; u += nthr) {
     int c = 0;
-    if (u < Mt) c += ceil_div(ws.tile_expert[u] == E ? sh.Ds : sh.D, kBN1);
+    if (u < Mt) c += (u < Mr) ? n1r : n1s;  // routed tiles come first, then the shared ones
     if (u >= sh.lag && u - sh.lag < Mt) c += n2;
     buf[u] = c;
   }
@@ -456,7 +462,7 @@ __global__ void __launch_bounds__(kGateThreads)
 // ------------------------------------------------------------------------------------------
 size_t gate_smem_bytes(const Shape& sh, int max_units) {
   const int buf = std::max(sh.E + 1, max_units + 1);
-  return sizeof(int) * (size_t)(sh.E /*hist*/ + 64 + 2 * sh.E + kMaxChunks * kScanGroup + buf);
+  return sizeof(int) * (size_t)(sh.E /*hist*/ + 64 + 3 * sh.E + kMaxChunks * kScanGroup + buf);
 }
 
 size_t scatter_smem_bytes(int E, int chunk_slots) {

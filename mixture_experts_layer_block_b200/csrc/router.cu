@@ -129,10 +129,27 @@ __global__ void __launch_bounds__(kRThreads, 1)
         tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(q * 32) << 16) + c, v);
         tmem_ld_wait();
         if (t < T) {
+          float* dst = logits + (size_t)t * E + n0 + c;
+          if ((E & 3) == 0) {  // rows are 16-byte aligned: vector stores of 4 logits
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int e = n0 + c + j;
-            if (e < E) logits[(size_t)t * E + e] = __uint_as_float(v[j]) + (bias ? bias[e] : 0.f);
+            for (int j = 0; j < 16; j += 4) {
+              if (n0 + c + j >= E) break;
+              float4 o = make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]), __uint_as_float(v[j + 2]),
+                                     __uint_as_float(v[j + 3]));
+              if (bias) {
+                o.x += bias[n0 + c + j];
+                o.y += bias[n0 + c + j + 1];
+                o.z += bias[n0 + c + j + 2];
+                o.w += bias[n0 + c + j + 3];
+              }
+              *reinterpret_cast<float4*>(dst + j) = o;
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int e = n0 + c + j;
+              if (e < E) dst[j] = __uint_as_float(v[j]) + (bias ? bias[e] : 0.f);
+            }
           }
         }
       }
