@@ -107,10 +107,16 @@ def sm_busy_fraction(records: np.ndarray, n_ctas: int) -> dict:
             "tasks": int(r.shape[0])}
 
 
-def traced_forward(w, wts, x, out):
+def tile_flags(args) -> int:
+    from mixture_experts_layer_block_b200 import native
+    return {"auto": 0, "pair": native.MOE_FLAG_PAIR_TILES, "single": native.MOE_FLAG_SINGLE_TILES}[
+        getattr(args, "tiles", "auto")]
+
+
+def traced_forward(w, wts, x, out, extra_flags=0):
     """One extra forward with per-task tracing (outside the timed region)."""
     from mixture_experts_layer_block_b200.native import MOE_FLAG_TRACE, MoELayer
-    layer = MoELayer.for_workload(w, flags=MOE_FLAG_TRACE)
+    layer = MoELayer.for_workload(w, flags=MOE_FLAG_TRACE | extra_flags)
     for _ in range(2):
         layer.forward(x, wts, out)
     torch.cuda.synchronize()
@@ -295,6 +301,9 @@ def main():
     ap.add_argument("--ref-tokens", type=int, default=256)
     ap.add_argument("--T", type=int, default=None, help="override the workload's token count (profiling)")
     ap.add_argument("--E", type=int, default=None, help="override the workload's expert count (profiling)")
+    ap.add_argument("--tiles", choices=["auto", "pair", "single"], default="auto",
+                    help="expert-GEMM shape: the library's choice, 256-row tiles on SM pairs, or "
+                         "128-row tiles on single SMs")
     ap.add_argument("--traffic-bytes", type=float, default=None,
                     help="ncu dram bytes per launch of the expert-GEMM kernel, if captured")
     args = ap.parse_args()
@@ -326,7 +335,7 @@ def run_mine(args, world, rank, local):
     wts = gen.make_weights(w, dev)
     x = gen.make_x(w.replace(seed=w.seed + 1000 * rank) if rank else w, dev)  # each replica its own tokens
     out = torch.empty((w.T, w.H), dtype=torch.float32, device=dev)
-    layer = MoELayer.for_workload(w, flags=MOE_FLAG_HOST_STAGING)
+    layer = MoELayer.for_workload(w, flags=MOE_FLAG_HOST_STAGING | tile_flags(args))
     stream = torch.cuda.current_stream(dev)
 
     for _ in range(args.warmup):
@@ -334,6 +343,8 @@ def run_mine(args, world, rank, local):
     torch.cuda.synchronize()
     rc, st = layer.status()
     assert rc == 0 and st == 0, (rc, st)
+    gemm_shape = {"tile_m": layer.query(6), "workers": layer.query(1),
+                  "kind": "SM pairs (2-CTA clusters)" if layer.query(6) == 256 else "single SMs"}
     stats = routing_stats(layer, w, dev)
 
     # headline: K whole forwards back to back, nothing recorded between the kernels
@@ -375,7 +386,7 @@ def run_mine(args, world, rank, local):
     # per-kernel durations: a second timed pass whose handle records CUDA events around every
     # kernel on the launching stream (events between kernels stop them from overlapping, so
     # this pass is kept apart from the headline one)
-    layer_t = MoELayer.for_workload(w, flags=MOE_FLAG_STAGE_TIMING)
+    layer_t = MoELayer.for_workload(w, flags=MOE_FLAG_STAGE_TIMING | tile_flags(args))
     for _ in range(3):
         layer_t.forward(x, wts, out)
     torch.cuda.synchronize()
@@ -421,9 +432,10 @@ def run_mine(args, world, rank, local):
             "e2e": {"value": world * w.T / (e2e_ms * 1e-3), "unit": UNIT,
                     "h2d_bytes_per_step": w.T * w.H * 2, "d2h_bytes_per_step": w.T * w.H * 4},
             "gpu_launches": len(MoELayer.STAGES) * args.steps,
+            "gemm_shape": gemm_shape,
             "clocks": clk.summary()}
     if not args.no_trace:
-        line["scheduler"] = traced_forward(w, wts, x, out)
+        line["scheduler"] = traced_forward(w, wts, x, out, tile_flags(args))
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, wts, x)
     if rank == 0:

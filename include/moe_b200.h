@@ -62,6 +62,12 @@ extern "C" {
 #define MOE_FLAG_STAGE_TIMING  1u  /* record CUDA events around each kernel (moe_stage_times) */
 #define MOE_FLAG_HOST_STAGING  2u  /* allocate device staging buffers for moe_forward_host */
 #define MOE_FLAG_TRACE         4u  /* record per-task claim/finish times (moe_trace_read) */
+/* Shape of the expert GEMMs of batches of more than 16 tokens. By default a forward computes
+ * 256-row m-tiles on pairs of SMs (2-CTA clusters) when its experts receive more than 128 slots
+ * on average and the capacity allows more than 128, else 128-row m-tiles on single SMs. The
+ * two flags force one shape (both set: single SMs). Either shape computes the same result. */
+#define MOE_FLAG_PAIR_TILES    8u
+#define MOE_FLAG_SINGLE_TILES 16u
 
 typedef struct moe_config {
     int32_t hidden;           /* H: model dimension; multiple of 8 */
@@ -185,9 +191,11 @@ MOE_API int moe_debug_outputs(moe_handle *h, float *logits, int32_t *topk_ids, f
  * when nothing was recorded. */
 MOE_API int moe_stage_times(moe_handle *h, float *ms, int32_t n);
 
-/* Handle facts: which = 0 SM count, 1 persistent-kernel CTAs, 2 workspace bytes,
+/* Handle facts: which = 0 SM count, 1 workers of the last forward's expert GEMMs (CTAs on
+ * single SMs, or SM pairs; the SM count before any forward), 2 workspace bytes,
  * 3 tasks of the last forward (synchronises), 4 m-tiles of the last forward (synchronises),
- * 5 dependency lag (units) of the last forward. */
+ * 5 dependency lag (units) of the last forward, 6 rows per m-tile of the last forward
+ * (128 or 256), 7 SM pairs the device can run at once for the pair shape (0 = none). */
 MOE_API int moe_query(const moe_handle *h, int32_t which, int64_t *value);
 
 /* Per-task trace of the last forward (needs MOE_FLAG_TRACE; synchronises). Fills up to

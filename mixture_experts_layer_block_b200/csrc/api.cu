@@ -17,6 +17,7 @@ namespace moe {
 cudaError_t configure_gate_kernels(size_t gate_smem, size_t scatter_smem);
 cudaError_t configure_router_kernel();
 cudaError_t configure_gemm_kernel();
+cudaError_t configure_gemm_pair_kernel(int* max_pairs);
 }  // namespace moe
 
 using namespace moe;
@@ -68,7 +69,11 @@ struct moe_handle {
   std::vector<MapEntry> cache;
   CUtensorMap h_routed{}, h_shared{}, xs_map{}, y_map{};
   CUtensorMap h_routed16{}, h_shared16{}, xs_map16{};  // 16-row boxes for batches of <= 16 tokens
+  CUtensorMap h_routed32{}, h_shared32{}, xs_map32{}, y_map32{};  // 32-row boxes (SM-pair tiles)
   int max_routed_tiles = 0;
+  int64_t routed_rows = 0, tile_rows = 0;  // rows of xs, and of h and y, for either tile height
+  int max_pairs = 0;                       // 2-CTA clusters of the pair kernel that fit at once
+  int last_workers = 0, last_tile_m = kBM;
   int parts_rows = 0;  // rows of the K-split partial logits buffer
   std::vector<cudaEvent_t> ev;  // kTimingRing x (kNumStages + 1) events around the kernels
   int timed = 0;                // forwards recorded since the last moe_stage_times
@@ -124,7 +129,7 @@ int capacity_of(const moe_config& c, int T, int k) {
   return (int)std::min<double>(v, (double)T * k);
 }
 
-Shape make_shape(const moe_handle* h, int T, int k) {
+Shape make_shape(const moe_handle* h, int T, int k, int tile_m = kBM, int workers = 0) {
   const moe_config& c = h->cfg;
   Shape sh{};
   sh.T = T;
@@ -145,9 +150,11 @@ Shape make_shape(const moe_handle* h, int T, int k) {
   // tasks and one and a half waves of up tasks in between, so that a claimed down task rarely
   // finds its tile's up tasks still running.
   const int n1 = ceil_div(c.inter, kBN1), n2 = ceil_div(c.hidden, kBN2);
-  const int lag = std::max(ceil_div(2 * h->num_sms, n1 + n2), ceil_div(3 * h->num_sms, 2 * n1));
+  const int W = workers > 0 ? workers : h->num_sms;  // SMs, or SM pairs
+  const int lag = std::max(ceil_div(2 * W, n1 + n2), ceil_div(3 * W, 2 * n1));
   sh.lag = std::max(1, std::min(h->max_lag, lag));
   sh.dep_extra = 0;
+  sh.tile_m = tile_m;
   sh.timeout_ns = h->timeout_ns;
   return sh;
 }
@@ -229,7 +236,10 @@ int moe_init(const moe_config* cfg, moe_handle** out) {
   const int E = c.num_experts;
   h->sorted_len_max = sorted_len_max;
   h->blocks_len_max = ceil_div((int)sorted_len_max, c.block_m);
-  h->max_routed_tiles = ceil_div((int)S_max, kBM) + E;
+  h->max_routed_tiles = ceil_div((int)S_max, kBM) + E;  // tile count (128-row tiles: the most)
+  // rows: 256-row tiles pad the most (at most 255 rows per expert and per batch)
+  h->routed_rows = (int64_t)(ceil_div((int)S_max, 2 * kBM) + E) * 2 * kBM;
+  h->tile_rows = h->routed_rows + (c.inter_shared > 0 ? (int64_t)ceil_div(c.max_tokens, 2 * kBM) * 2 * kBM : 0);
   // splits * T <= #SMs * 128 (see router_splits) and splits <= 4
   h->parts_rows = std::min(kMaxRouterSplits * c.max_tokens, (h->num_sms + 1) * kBM);
   h->max_tiles = h->max_routed_tiles + (c.inter_shared > 0 ? ceil_div(c.max_tokens, kBM) : 0);
@@ -262,11 +272,11 @@ int moe_init(const moe_config* cfg, moe_handle** out) {
       {(void**)&w.tile_nrows, (size_t)h->max_tiles * 4},
       {(void**)&w.unit_start, (size_t)(h->max_units + 1) * 4},
       {(void**)&w.done1, (size_t)h->max_tiles * 4},
-      {(void**)&w.h, (size_t)h->max_tiles * kBM * ldh * 2},
+      {(void**)&w.h, (size_t)h->tile_rows * ldh * 2},
       {(void**)&w.expert_tile0, E_ * 4},
       {(void**)&w.row_of_slot, (size_t)S_max * 4},
-      {(void**)&w.xs, (size_t)h->max_routed_tiles * kBM * c.hidden * 2},
-      {(void**)&w.y, (size_t)h->max_tiles * kBM * c.hidden * 2},
+      {(void**)&w.xs, (size_t)h->routed_rows * c.hidden * 2},
+      {(void**)&w.y, (size_t)h->tile_rows * c.hidden * 2},
       {(void**)&w.trace, (size_t)trace_cap * 4 * 8},
       {(void**)&h->x_stage, (c.flags & MOE_FLAG_HOST_STAGING) ? T_ * c.hidden * 2 : 0},
       {(void**)&h->out_stage, (c.flags & MOE_FLAG_HOST_STAGING) ? T_ * c.hidden * 4 : 0},
@@ -288,7 +298,8 @@ int moe_init(const moe_config* cfg, moe_handle** out) {
   if (cudaMemset(h->ws_mem, 0, total) != cudaSuccess) return fail(MOE_ERR_CUDA);
 
   // h tensor maps (fixed for the handle's lifetime)
-  const uint64_t h_rows = (uint64_t)h->max_tiles * kBM;
+  const uint64_t h_rows = (uint64_t)h->tile_rows;
+  const uint64_t xs_rows = (uint64_t)h->routed_rows;
   if ((rc = encode_map(h, &h->h_routed, w.h, c.inter, h_rows, (uint64_t)ldh * 2, kBK, kBM))) return fail(rc);
   if (c.inter_shared > 0) {
     if ((rc = encode_map(h, &h->h_shared, w.h, c.inter_shared, h_rows, (uint64_t)ldh * 2, kBK, kBM)))
@@ -296,11 +307,21 @@ int moe_init(const moe_config* cfg, moe_handle** out) {
   } else {
     h->h_shared = h->h_routed;
   }
-  if ((rc = encode_map(h, &h->xs_map, w.xs, c.hidden, (uint64_t)h->max_routed_tiles * kBM,
-                       (uint64_t)c.hidden * 2, kBK, kBM)))
+  if ((rc = encode_map(h, &h->xs_map, w.xs, c.hidden, xs_rows, (uint64_t)c.hidden * 2, kBK, kBM)))
     return fail(rc);
-  if ((rc = encode_map(h, &h->xs_map16, w.xs, c.hidden, (uint64_t)h->max_routed_tiles * kBM,
-                       (uint64_t)c.hidden * 2, kBK, kSmallRows)))
+  if ((rc = encode_map(h, &h->xs_map16, w.xs, c.hidden, xs_rows, (uint64_t)c.hidden * 2, kBK, kSmallRows)))
+    return fail(rc);
+  if ((rc = encode_map(h, &h->xs_map32, w.xs, c.hidden, xs_rows, (uint64_t)c.hidden * 2, kBK, kPairBoxRows)))
+    return fail(rc);
+  if ((rc = encode_map(h, &h->h_routed32, w.h, c.inter, h_rows, (uint64_t)ldh * 2, kBK, kPairBoxRows)))
+    return fail(rc);
+  if (c.inter_shared > 0) {
+    if ((rc = encode_map(h, &h->h_shared32, w.h, c.inter_shared, h_rows, (uint64_t)ldh * 2, kBK, kPairBoxRows)))
+      return fail(rc);
+  } else {
+    h->h_shared32 = h->h_routed32;
+  }
+  if ((rc = encode_map(h, &h->y_map32, w.y, c.hidden, h_rows, (uint64_t)c.hidden * 2, kBK, kPairBoxRows)))
     return fail(rc);
   if ((rc = encode_map(h, &h->h_routed16, w.h, c.inter, h_rows, (uint64_t)ldh * 2, kBK, kSmallRows)))
     return fail(rc);
@@ -323,6 +344,9 @@ int moe_init(const moe_config* cfg, moe_handle** out) {
       return fail(MOE_ERR_CUDA);
   }
   if (check_cuda(configure_router_kernel()) || check_cuda(configure_gemm_kernel())) return fail(MOE_ERR_CUDA);
+  if (check_cuda(configure_gemm_pair_kernel(&h->max_pairs))) return fail(MOE_ERR_CUDA);
+  h->max_pairs = std::min(h->max_pairs, h->num_sms / 2);
+  h->last_workers = h->num_sms;
   if (h->timing) {
     h->ev.assign((size_t)kTimingRing * (kNumStages + 1), nullptr);
     for (auto& e : h->ev)
@@ -386,7 +410,23 @@ static int forward_impl(moe_handle* h, const void* x, int32_t T, const void* w_r
   if (T == 0) return MOE_OK;
 
   const int E = c.num_experts, H = c.hidden, D = c.inter, Ds = c.inter_shared;
-  Shape sh = make_shape(h, T, top_k);
+  // With at most 16 tokens every m-tile has at most 16 rows (an expert appears once per token):
+  // the expert GEMMs use their small-tile shape with 16-row A boxes.
+  const bool small = T <= kSmallRows;
+  bool pair = false;
+  if (!small && h->max_pairs > 0 && !(c.flags & MOE_FLAG_SINGLE_TILES)) {
+    if (c.flags & MOE_FLAG_PAIR_TILES) {
+      pair = true;
+    } else {
+      // 256-row tiles pay off once experts receive more than one 128-row tile on average
+      const int cap = capacity_of(c, T, top_k);
+      pair = (int64_t)T * top_k >= (int64_t)kBM * E && (cap == 0 || cap > kBM);
+    }
+  }
+  const int workers = pair ? h->max_pairs : h->num_sms;
+  Shape sh = make_shape(h, T, top_k, pair ? 2 * kBM : kBM, workers);
+  h->last_workers = workers;
+  h->last_tile_m = sh.tile_m;
   sh.dep_extra = h->dep_extra_next;
   h->dep_extra_next = 0;
   h->last_lag = sh.lag;
@@ -396,28 +436,28 @@ static int forward_impl(moe_handle* h, const void* x, int32_t T, const void* w_r
   CUtensorMap wr_map;
   GemmMaps maps;
   const int bn = router_bn(E);
-  // With at most 16 tokens every m-tile has at most 16 rows (an expert appears once per token):
-  // the expert GEMMs use their small-tile shape with 16-row A boxes.
-  const bool small = T <= kSmallRows;
   CUtensorMap x_router;
   if ((rc = encode_map(h, &x_router, x, H, T, (uint64_t)H * 2, kBK, kBM))) return rc;
-  if (small) {
-    if ((rc = encode_map(h, &maps.x_tile, x, H, T, (uint64_t)H * 2, kBK, kSmallRows))) return rc;
+  if (small || pair) {
+    if ((rc = encode_map(h, &maps.x_tile, x, H, T, (uint64_t)H * 2, kBK, small ? kSmallRows : kPairBoxRows)))
+      return rc;
   } else {
     maps.x_tile = x_router;
   }
-  maps.xs = small ? h->xs_map16 : h->xs_map;
-  maps.y = h->y_map;
+  maps.xs = small ? h->xs_map16 : (pair ? h->xs_map32 : h->xs_map);
+  maps.y = pair ? h->y_map32 : h->y_map;
+  // the pair shape stages half of B (128 rows) per CTA
+  const uint32_t bn2 = pair ? (uint32_t)kBN2 / 2 : (uint32_t)kBN2;
   if ((rc = cached_map(h, &wr_map, w_router, H, E, (uint64_t)H * 2, kBK, bn))) return rc;
   if ((rc = cached_map(h, &maps.w_up, w_up, H, (uint64_t)E * D, (uint64_t)H * 2, kBK, kBN1))) return rc;
   if ((rc = cached_map(h, &maps.w_gate, w_gate, H, (uint64_t)E * D, (uint64_t)H * 2, kBK, kBN1))) return rc;
-  if ((rc = cached_map(h, &maps.w_down, w_down, D, (uint64_t)E * H, (uint64_t)D * 2, kBK, kBN2))) return rc;
-  maps.h_routed = small ? h->h_routed16 : h->h_routed;
+  if ((rc = cached_map(h, &maps.w_down, w_down, D, (uint64_t)E * H, (uint64_t)D * 2, kBK, bn2))) return rc;
+  maps.h_routed = small ? h->h_routed16 : (pair ? h->h_routed32 : h->h_routed);
   if (has_shared) {
     if ((rc = cached_map(h, &maps.ws_up, w_shared->up, H, Ds, (uint64_t)H * 2, kBK, kBN1))) return rc;
     if ((rc = cached_map(h, &maps.ws_gate, w_shared->gate, H, Ds, (uint64_t)H * 2, kBK, kBN1))) return rc;
-    if ((rc = cached_map(h, &maps.ws_down, w_shared->down, Ds, H, (uint64_t)Ds * 2, kBK, kBN2))) return rc;
-    maps.h_shared = small ? h->h_shared16 : h->h_shared;
+    if ((rc = cached_map(h, &maps.ws_down, w_shared->down, Ds, H, (uint64_t)Ds * 2, kBK, bn2))) return rc;
+    maps.h_shared = small ? h->h_shared16 : (pair ? h->h_shared32 : h->h_shared);
   } else {
     maps.ws_up = maps.w_up;
     maps.ws_gate = maps.w_gate;
@@ -447,7 +487,11 @@ static int forward_impl(moe_handle* h, const void* x, int32_t T, const void* w_r
   if ((rc = mark(3))) return rc;
   if ((rc = check_cuda(launch_gather_rows(x16, w, sh, 4 * h->num_sms, st)))) return rc;
   if ((rc = mark(4))) return rc;
-  if ((rc = check_cuda(launch_moe_gemm(maps, w, sh, h->num_sms, small, st)))) return rc;
+  if (pair) {
+    if ((rc = check_cuda(launch_moe_gemm_pair(maps, w, sh, h->max_pairs, st)))) return rc;
+  } else {
+    if ((rc = check_cuda(launch_moe_gemm(maps, w, sh, h->num_sms, small, st)))) return rc;
+  }
   if ((rc = mark(5))) return rc;
   if ((rc = check_cuda(launch_combine(out, w, sh, st)))) return rc;
   if ((rc = mark(6))) return rc;
@@ -595,7 +639,7 @@ int moe_query(const moe_handle* h, int32_t which, int64_t* value) {
   if (!h || !value) return MOE_ERR_INVALID_ARG;
   switch (which) {
     case 0: *value = h->num_sms; return MOE_OK;
-    case 1: *value = h->num_sms; return MOE_OK;
+    case 1: *value = h->last_workers; return MOE_OK;
     case 2: *value = (int64_t)h->ws_bytes; return MOE_OK;
     case 3:
     case 4: {
@@ -608,6 +652,8 @@ int moe_query(const moe_handle* h, int32_t which, int64_t* value) {
       return MOE_OK;
     }
     case 5: *value = h->last_lag; return MOE_OK;
+    case 6: *value = h->last_tile_m; return MOE_OK;
+    case 7: *value = h->max_pairs; return MOE_OK;
     default: return MOE_ERR_INVALID_ARG;
   }
 }

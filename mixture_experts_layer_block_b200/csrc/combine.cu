@@ -1,8 +1,8 @@
 // combine.cu -- the two memory-bound steps around the expert GEMMs.
 //
 // gather_rows_kernel: copies every kept slot's token row x[t] into the tile-ordered buffer
-//   xs (row = first tile of its expert * 128 + its rank in the expert), so that the up/gate
-//   GEMM reads its A operand as plain 128-row TMA boxes. One warp per slot, 16-byte vectors.
+//   xs (row = first tile of its expert * tile height + its rank in the expert), so that the
+//   up/gate GEMM reads its A operand as plain TMA boxes. One warp per slot, 16-byte vectors.
 //
 // combine_kernel: the sum over experts of the Mixture-of-Kittens layer equation
 //   x' = W_shared(x) + sum_{e in top-k} w_e (W_down^e SwiGLU(...)).
@@ -74,7 +74,7 @@ __global__ void __launch_bounds__(256)
     float a0[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     float a1[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     if (sh.Ds > 0) {
-      const uint16_t* srow = ws.y + ((size_t)Mr * kBM + t) * sh.H;
+      const uint16_t* srow = ws.y + ((size_t)Mr * sh.tile_m + t) * sh.H;
       add_bf16x8(a0, __ldcg(reinterpret_cast<const uint4*>(srow + c0)));
       if (has1) add_bf16x8(a1, __ldcg(reinterpret_cast<const uint4*>(srow + c1)));
     }

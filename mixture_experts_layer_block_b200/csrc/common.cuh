@@ -25,6 +25,7 @@ constexpr int kNumStaging = 2;            // double-buffered epilogue -> TMA sto
 constexpr int kAccCols = 256;   // TMEM columns per accumulator buffer (2 buffers)
 constexpr int kGemmThreads = 192;  // warp 0 producer, warp 1 MMA, warps 2-5 epilogue
 constexpr int kSmallRows = 16;     // A-tile rows of the expert GEMMs' small-tile shape (T <= 16)
+constexpr int kPairBoxRows = 32;   // rows per A load / result store box of the SM-pair shape
 
 // ---- router GEMM -------------------------------------------------------------------------
 constexpr int kRouterStages = 6;
@@ -103,10 +104,10 @@ struct Workspace {
   int32_t* unit_start;   // [max_tiles + max_lag + 1]
   int32_t* done1;        // [max_tiles]      finished up/gate tasks per tile
   int32_t* expert_tile0; // [E]              first m-tile of each expert
-  int32_t* row_of_slot;  // [S]              tile row (tile*128 + r) of each kept slot, -1 if dropped
-  uint16_t* xs;          // [max_routed_tiles*128][H] bf16 x rows gathered in tile order
-  uint16_t* h;           // [max_tiles*128][ldh] bf16 SwiGLU activations
-  uint16_t* y;           // [max_tiles*128][H] bf16 router-weighted expert outputs per tile row
+  int32_t* row_of_slot;  // [S]              tile row (tile*tile_m + r) of each kept slot, -1 if dropped
+  uint16_t* xs;          // [routed rows][H] bf16 x rows gathered in tile order
+  uint16_t* h;           // [rows][ldh] bf16 SwiGLU activations, tile order
+  uint16_t* y;           // [rows][H] bf16 router-weighted expert outputs per tile row
   int64_t* trace;        // [trace_cap][4]
   int32_t trace_cap;
   int32_t ldh;           // row stride of h in elements (max(D, D_shared))
@@ -121,6 +122,7 @@ struct Shape {
   int32_t sorted_len, blocks_len;
   int32_t lag;           // scheduling lag in units between a tile's up and down tasks
   int32_t dep_extra;     // testing hook: extra up completions a down task waits for
+  int32_t tile_m;        // rows per m-tile of the expert GEMMs: 128, or 256 on SM pairs
   int64_t timeout_ns;
 };
 
@@ -169,6 +171,22 @@ static __device__ __noinline__ bool wait_bar_drain(uint64_t* bar, uint32_t parit
     }
   }
   return true;
+}
+
+// Bounded wait until *p >= need (acquire). Raises a timeout error on expiry.
+static __device__ __noinline__ bool wait_count(const int* p, int need, DeviceMeta* meta,
+                                        volatile int* s_abort, int64_t limit_ns) {
+  if (ld_acquire_gpu(p) >= need) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    __nanosleep(128);
+    if (ld_acquire_gpu(p) >= need) return true;
+    if (aborted(meta, s_abort)) return false;
+    if (static_cast<int64_t>(globaltimer_ns() - t0) > limit_ns) {
+      raise_error(meta, s_abort, kStatusTimeout | kSiteDependency);
+      return false;
+    }
+  }
 }
 
 // Wait for the last TMA fill of every stage of a ring that was filled `nfill` times in

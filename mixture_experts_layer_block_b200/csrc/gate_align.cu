@@ -208,25 +208,27 @@ __device__ void align_scans(const Workspace& ws, const Shape& sh, bool tiles, in
   __syncthreads();
   if (!tiles) return;
 
-  // 3. m-tiles: routed experts (ceil(kept/128) each), then the shared expert over all tokens
-  for (int e = tid; e < E; e += nthr) buf[e] = ceil_div(kept[e], kBM);
+  // 3. m-tiles of tile_m rows: routed experts (ceil(kept/tile_m) each), then the shared expert
+  //    over all tokens
+  const int tm = sh.tile_m;
+  for (int e = tid; e < E; e += nthr) buf[e] = ceil_div(kept[e], tm);
   __syncthreads();
   const int Mr = block_exclusive_scan(buf, E, tmp);
   for (int e = tid; e < E; e += nthr) {
-    const int first = buf[e], nt = ceil_div(kept[e], kBM);
+    const int first = buf[e], nt = ceil_div(kept[e], tm);
     const int off = offs[e];
     ws.expert_tile0[e] = first;
     for (int i = 0; i < nt; ++i) {
       ws.tile_expert[first + i] = e;
-      ws.tile_row0[first + i] = off + i * kBM;
-      ws.tile_nrows[first + i] = min(kBM, kept[e] - i * kBM);
+      ws.tile_row0[first + i] = off + i * tm;
+      ws.tile_nrows[first + i] = min(tm, kept[e] - i * tm);
     }
   }
-  const int Ms = (sh.Ds > 0) ? ceil_div(sh.T, kBM) : 0;
+  const int Ms = (sh.Ds > 0) ? ceil_div(sh.T, tm) : 0;
   for (int j = tid; j < Ms; j += nthr) {
     ws.tile_expert[Mr + j] = E;
-    ws.tile_row0[Mr + j] = j * kBM;
-    ws.tile_nrows[Mr + j] = min(kBM, sh.T - j * kBM);
+    ws.tile_row0[Mr + j] = j * tm;
+    ws.tile_nrows[Mr + j] = min(tm, sh.T - j * tm);
   }
   const int Mt = Mr + Ms;
   __syncthreads();
@@ -428,7 +430,7 @@ __global__ void __launch_bounds__(kGateThreads)
         const int r = c0 + rank;
         const bool keep = sh.capacity == 0 || r < sh.capacity;
         if (keep) sorted_ids[off[e] + r] = s;
-        if (row_of_slot) row_of_slot[s] = keep ? tile0[e] * kBM + r : -1;
+        if (row_of_slot) row_of_slot[s] = keep ? tile0[e] * sh.tile_m + r : -1;
         if (rank == 0) cnt[e] = c0 + __popc(mask);
       } else if (in && row_of_slot) {
         row_of_slot[s] = -1;  // an expert id outside [0, E)

@@ -87,6 +87,12 @@ size_t gemm_smem_bytes(bool small);
 cudaError_t launch_moe_gemm(const GemmMaps& maps, const Workspace& ws, const Shape& sh, int grid,
                             bool small, cudaStream_t stream);
 
+// The same GEMMs with 256-row m-tiles on `pairs` 2-CTA clusters (sh.tile_m = 256; its maps use
+// 32-row boxes for x_tile, xs, h_routed, h_shared and y, and 128-row boxes for w_down, ws_down).
+size_t gemm_pair_smem_bytes();
+cudaError_t launch_moe_gemm_pair(const GemmMaps& maps, const Workspace& ws, const Shape& sh, int pairs,
+                                 cudaStream_t stream);
+
 // One-time kernel attribute setup (dynamic shared memory limits).
 cudaError_t configure_kernels(size_t gate_smem);
 

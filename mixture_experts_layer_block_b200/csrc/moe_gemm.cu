@@ -67,22 +67,6 @@ __device__ __forceinline__ int n1_of(int expert, const Shape& sh) {
   return ceil_div(expert == sh.E ? sh.Ds : sh.D, kBN1);
 }
 
-// Bounded wait until *p >= need (acquire). Raises a timeout error on expiry.
-__device__ __noinline__ bool wait_count(const int* p, int need, DeviceMeta* meta,
-                                        volatile int* s_abort, int64_t limit_ns) {
-  if (ld_acquire_gpu(p) >= need) return true;
-  const uint64_t t0 = globaltimer_ns();
-  while (true) {
-    __nanosleep(128);
-    if (ld_acquire_gpu(p) >= need) return true;
-    if (aborted(meta, s_abort)) return false;
-    if (static_cast<int64_t>(globaltimer_ns() - t0) > limit_ns) {
-      raise_error(meta, s_abort, kStatusTimeout | kSiteDependency);
-      return false;
-    }
-  }
-}
-
 }  // namespace
 
 template <bool kSmall>

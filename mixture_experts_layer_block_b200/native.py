@@ -25,6 +25,8 @@ MOE_ERR_NOT_READY = -7
 
 MOE_FLAG_STAGE_TIMING = 1
 MOE_FLAG_HOST_STAGING = 2
+MOE_FLAG_PAIR_TILES = 8
+MOE_FLAG_SINGLE_TILES = 16
 MOE_FLAG_TRACE = 4
 
 

@@ -36,6 +36,11 @@ def _layer(w, **kw):
     return MoELayer.for_workload(w, **kw)
 
 
+def _flags():
+    from mixture_experts_layer_block_b200 import native
+    return {"pair": native.MOE_FLAG_PAIR_TILES, "single": native.MOE_FLAG_SINGLE_TILES}
+
+
 @pytest.mark.parametrize("name", sorted(SMALL))
 def test_forward_small_all_tokens(name):
     w = SMALL[name]
@@ -46,6 +51,49 @@ def test_forward_small_all_tokens(name):
     res2 = check_forward(layer, w, inp)
     assert res2["out_err"] <= 1e-2
     print(name, res)
+
+
+# Both shapes of the expert GEMMs (256-row tiles on SM pairs, 128-row tiles on single SMs) on
+# every small case with more than 16 tokens: tiles of 1..256 rows, split between the two CTAs
+# of a pair at every boundary the split rule has.
+@pytest.mark.parametrize("shape", ["pair", "single"])
+@pytest.mark.parametrize("name", sorted(n for n, w in SMALL.items() if w.T > 16))
+def test_forward_small_tile_shapes(name, shape):
+    w = SMALL[name]
+    inp = {k: (v.cuda() if v is not None else None) for k, v in gen.make_inputs(w).items()}
+    layer = _layer(w, flags=_flags()[shape])
+    res = check_forward(layer, w, inp)
+    assert layer.query(6) == (256 if shape == "pair" else 128)
+    res2 = check_forward(layer, w, inp)
+    assert res2["out_err"] <= 1e-2
+    print(name, shape, res)
+
+
+@pytest.mark.parametrize("nrows", [17, 31, 32, 33, 64, 95, 127, 128, 129, 160, 200, 255, 256, 257, 300, 513])
+def test_pair_tiles_one_expert(nrows):
+    """Every token routed to expert 0 (top-1 of 2 experts with a large bias): one expert with
+    nrows rows, i.e. pair tiles of every size around the 32-row box and 128-row half boundaries."""
+    w = configs.MoEWorkload(f"one_expert_{nrows}", T=nrows, H=256, D=384, E=2, top_k=1, block_m=16,
+                            D_shared=128, sigma_w=0.05)
+    inp = {k: (v.cuda() if v is not None else None) for k, v in gen.make_inputs(w).items()}
+    inp["bias"] = torch.tensor([30.0, 0.0], dtype=torch.float32, device="cuda")
+    layer = _layer(w, flags=_flags()["pair"])
+    check_forward(layer, w, inp)
+    assert layer.query(6) == 256
+
+
+def test_tile_shape_heuristic():
+    """Experts with more than 128 slots on average take the pair shape; a capacity of at most
+    128 slots per expert keeps single SMs."""
+    w2 = SMALL["skew_small"].replace(E=64, name="skew_small_64")  # 2000 x top-8 / 64: 250 each
+    inp2 = {k: (v.cuda() if v is not None else None) for k, v in gen.make_inputs(w2).items()}
+    layer = _layer(w2)
+    check_forward(layer, w2, inp2)
+    assert layer.query(6) == 256 and layer.query(1) == layer.query(7) > 0
+    cap = w2.replace(capacity_factor=0.5, name="skew_small_64_cap")  # capacity 125
+    layer = _layer(cap)
+    check_forward(layer, cap, inp2)
+    assert layer.query(6) == 128 and layer.query(1) == layer.query(0)
 
 
 @pytest.mark.parametrize("name", ["flashmoe_prefill", "dsv3", "decode", "skew", "skew_uniform"])
