@@ -62,10 +62,10 @@ extern "C" {
 #define MOE_FLAG_STAGE_TIMING  1u  /* record CUDA events around each kernel (moe_stage_times) */
 #define MOE_FLAG_HOST_STAGING  2u  /* allocate device staging buffers for moe_forward_host */
 #define MOE_FLAG_TRACE         4u  /* record per-task claim/finish times (moe_trace_read) */
-/* Shape of the expert GEMMs of batches of more than 16 tokens. By default a forward computes
- * 256-row m-tiles on pairs of SMs (2-CTA clusters) when its experts receive more than 128 slots
- * on average and the capacity allows more than 128, else 128-row m-tiles on single SMs. The
- * two flags force one shape (both set: single SMs). Either shape computes the same result. */
+/* Shape of the expert GEMMs of batches of more than 16 tokens: 128-row m-tiles on single SMs
+ * (the default), or with MOE_FLAG_PAIR_TILES 256-row m-tiles on pairs of SMs (2-CTA clusters,
+ * tcgen05 cta_group::2; used only when the device fits such clusters). MOE_FLAG_SINGLE_TILES
+ * forces single SMs and wins over MOE_FLAG_PAIR_TILES. Both shapes compute the same result. */
 #define MOE_FLAG_PAIR_TILES    8u
 #define MOE_FLAG_SINGLE_TILES 16u
 

@@ -414,15 +414,11 @@ static int forward_impl(moe_handle* h, const void* x, int32_t T, const void* w_r
   // the expert GEMMs use their small-tile shape with 16-row A boxes.
   const bool small = T <= kSmallRows;
   bool pair = false;
-  if (!small && h->max_pairs > 0 && !(c.flags & MOE_FLAG_SINGLE_TILES)) {
-    if (c.flags & MOE_FLAG_PAIR_TILES) {
-      pair = true;
-    } else {
-      // 256-row tiles pay off once experts receive more than one 128-row tile on average
-      const int cap = capacity_of(c, T, top_k);
-      pair = (int64_t)T * top_k >= (int64_t)kBM * E && (cap == 0 || cap > kBM);
-    }
-  }
+  // The pair shape is chosen only on request: on the measured workloads (skewed routing, and
+  // 256 experts x top-8 with a shared expert) it was slower than single SMs, whose operand rings
+  // already keep the tensor pipe as busy as the memory system allows.
+  if (!small && h->max_pairs > 0 && (c.flags & MOE_FLAG_PAIR_TILES) && !(c.flags & MOE_FLAG_SINGLE_TILES))
+    pair = true;
   const int workers = pair ? h->max_pairs : h->num_sms;
   Shape sh = make_shape(h, T, top_k, pair ? 2 * kBM : kBM, workers);
   h->last_workers = workers;

@@ -189,6 +189,21 @@ static __device__ __noinline__ bool wait_count(const int* p, int need, DeviceMet
   }
 }
 
+// The scheduling unit u of task `tau` (unit_start[u] <= tau < unit_start[u + 1]), searched
+// forward from unit `u` (each CTA claims ever larger task ids). Executed by a whole warp: each
+// round compares the next 32 unit starts at once, so a claim costs one dependent load round
+// however many units it skips.
+__device__ __forceinline__ int find_unit(const int32_t* unit_start, int num_units, int tau, int u) {
+  const int lane = threadIdx.x & 31;
+  while (true) {
+    const int idx = u + 1 + lane;
+    const int v = idx <= num_units ? __ldcg(unit_start + idx) : 0x7fffffff;
+    const int adv = __popc(__ballot_sync(0xffffffffu, v <= tau));  // unit starts never decrease
+    u += adv;
+    if (adv < 32) return u;
+  }
+}
+
 // Wait for the last TMA fill of every stage of a ring that was filled `nfill` times in
 // round-robin order (fill f of stage s completes phase f of its `full` barrier).
 __device__ __forceinline__ void drain_fills(uint64_t* full, int nstages, uint32_t nfill,

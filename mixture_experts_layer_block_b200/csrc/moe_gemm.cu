@@ -133,6 +133,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ===================================== producer =====================================
     const int total = __ldcg(&meta->total_tasks);
     const int Mt = __ldcg(&meta->num_tiles);
+    const int U = __ldcg(&meta->num_units);
     const int nk1 = ceil_div(sh.H, kBK);
     int u_cur = 0;
     uint32_t stage = 0, phase = 0, slot = 0, slot_phase = 0;
@@ -145,7 +146,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (tau >= total) {
         t.kind = kTaskStop;
       } else {
-        while (__ldcg(&ws.unit_start[u_cur + 1]) <= tau) ++u_cur;
+        u_cur = find_unit(ws.unit_start, U, tau, u_cur);
         const int off = tau - __ldcg(&ws.unit_start[u_cur]);
         const int n1u = (u_cur < Mt) ? n1_of(__ldcg(&ws.tile_expert[u_cur]), sh) : 0;
         int nt;

@@ -166,6 +166,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t task_full_c1 = mapa_shared(smem_u32(task_full), 1);
     const int total = __ldcg(&meta->total_tasks);
     const int Mt = __ldcg(&meta->num_tiles);
+    const int U = __ldcg(&meta->num_units);
     int u_cur = 0;
     uint32_t stage = 0, phase = 0, slot = 0, slot_phase = 0;
     while (true) {
@@ -179,7 +180,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         t.kind = kTaskStop;
         t.tile = t.expert = t.row0 = t.nrows = t.n0 = t.nk = 0;
         if (tau < total) {
-          while (__ldcg(&ws.unit_start[u_cur + 1]) <= tau) ++u_cur;
+          u_cur = find_unit(ws.unit_start, U, tau, u_cur);
           const int off = tau - __ldcg(&ws.unit_start[u_cur]);
           const int n1u = (u_cur < Mt) ? n1_of(__ldcg(&ws.tile_expert[u_cur]), sh) : 0;
           int nt;

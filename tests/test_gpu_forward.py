@@ -82,18 +82,21 @@ def test_pair_tiles_one_expert(nrows):
     assert layer.query(6) == 256
 
 
-def test_tile_shape_heuristic():
-    """Experts with more than 128 slots on average take the pair shape; a capacity of at most
-    128 slots per expert keeps single SMs."""
-    w2 = SMALL["skew_small"].replace(E=64, name="skew_small_64")  # 2000 x top-8 / 64: 250 each
+def test_tile_shape_selection():
+    """Single SMs by default, SM pairs on request (when the device fits 2-CTA clusters), single
+    SMs when both flags are given; batches of at most 16 tokens keep the small-tile shape."""
+    w2 = SMALL["skew_small"].replace(E=64, name="skew_small_64")
     inp2 = {k: (v.cuda() if v is not None else None) for k, v in gen.make_inputs(w2).items()}
+    f = _flags()
     layer = _layer(w2)
     check_forward(layer, w2, inp2)
-    assert layer.query(6) == 256 and layer.query(1) == layer.query(7) > 0
-    cap = w2.replace(capacity_factor=0.5, name="skew_small_64_cap")  # capacity 125
-    layer = _layer(cap)
-    check_forward(layer, cap, inp2)
     assert layer.query(6) == 128 and layer.query(1) == layer.query(0)
+    layer = _layer(w2, flags=f["pair"])
+    check_forward(layer, w2, inp2)
+    assert layer.query(7) > 0 and layer.query(6) == 256 and layer.query(1) == layer.query(7)
+    layer = _layer(w2, flags=f["pair"] | f["single"])
+    check_forward(layer, w2, inp2)
+    assert layer.query(6) == 128
 
 
 @pytest.mark.parametrize("name", ["flashmoe_prefill", "dsv3", "decode", "skew", "skew_uniform"])
