@@ -89,6 +89,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   Task* ring = reinterpret_cast<Task*>(smem + C::kRingOff);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
+  volatile int* s_epi_go = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 8);  // [2]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   DeviceMeta* meta = ws.meta;
@@ -273,15 +274,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const bool leader = (warp == 2 && lane == 0);
     uint8_t* staging = smem + C::kStagingOff;
     uint32_t slot = 0, slot_phase = 0, acc = 0, acc_phase = 0, sb = 0;
+    // One thread waits for the next task and its accumulator and tells the other 127 through
+    // the named barrier, so the four warps always take the same branch (a warp that left the
+    // loop alone would strand the others at the next named barrier). The decision word is
+    // double-buffered: it is rewritten only after every thread passed the next loop barrier.
+    auto epilogue_next = [&](uint32_t it) -> bool {
+      if (leader) {
+        int go = 0;
+        if (wait_bar(&task_full[slot], slot_phase, meta, s_abort, limit, kSiteEpiTask) && ring[slot].kind != kTaskStop)
+          go = wait_bar(&acc_full[acc], acc_phase, meta, s_abort, limit, kSiteEpiAcc) ? 1 : 0;
+        s_epi_go[it & 1] = go;
+      }
+      named_bar_sync(1, 128);
+      if (s_epi_go[it & 1] == 0) return false;
+      tc_fence_after();
+      return true;
+    };
     if constexpr (kSmall) {
       // at most 16 valid rows per tile: only the warp of TMEM lanes 0-31 has work, and the
       // valid rows are stored straight from registers (no staging, no TMA stores)
-      while (true) {
-        if (!wait_bar(&task_full[slot], slot_phase, meta, s_abort, limit, kSiteEpiTask)) break;
+      for (uint32_t it = 0;; ++it) {
+        if (!epilogue_next(it)) break;
         const Task t = ring[slot];
-        if (t.kind == kTaskStop) break;
-        if (!wait_bar(&acc_full[acc], acc_phase, meta, s_abort, limit, kSiteEpiAcc)) break;
-        tc_fence_after();
         const uint32_t tacc = tmem_base + acc * kAccCols + (static_cast<uint32_t>(q * 32) << 16);
         const bool shared = (t.expert == sh.E);
         const bool has_rows = q * 32 < t.nrows;  // warp-uniform
@@ -377,12 +391,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         *reinterpret_cast<uint4*>(buf + row * 128 + ((j ^ (row & 7)) << 4)) =
             make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
     };
-    while (true) {
-      if (!wait_bar(&task_full[slot], slot_phase, meta, s_abort, limit, kSiteEpiTask)) break;
+    for (uint32_t it = 0;; ++it) {
+      if (!epilogue_next(it)) break;
       const Task t = ring[slot];
-      if (t.kind == kTaskStop) break;
-      if (!wait_bar(&acc_full[acc], acc_phase, meta, s_abort, limit, kSiteEpiAcc)) break;
-      tc_fence_after();
       const uint32_t tacc = tmem_base + acc * kAccCols + (static_cast<uint32_t>(q * 32) << 16);
       const bool shared = (t.expert == sh.E);
       if (t.kind == kTaskUp) {

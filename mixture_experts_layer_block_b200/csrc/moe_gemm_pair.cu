@@ -112,7 +112,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + kPMiscOff);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + kPMiscOff + 4);
   volatile uint32_t* s_peer_nfill = reinterpret_cast<volatile uint32_t*>(smem + kPMiscOff + 8);
-  volatile int* s_epi_go = reinterpret_cast<volatile int*>(smem + kPMiscOff + 12);
+  volatile int* s_epi_go = reinterpret_cast<volatile int*>(smem + kPMiscOff + 12);  // [2]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -327,20 +327,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         *reinterpret_cast<uint4*>(buf + row * 128 + ((j ^ (row & 7)) << 4)) =
             make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
     };
-    while (true) {
+    for (uint32_t it = 0;; ++it) {
       // one thread waits for the task and its accumulator and tells the other 127 through the
       // named barrier, so that the four warps always take the same branch (a warp that left
-      // the loop alone would strand the others at the next named barrier)
+      // the loop alone would strand the others at the next named barrier); the decision word
+      // is double-buffered, rewritten only after every thread passed the next loop barrier
       if (leader) {
         int go = 0;
         const bool got = rank == 0 ? wait_bar(&task_full[slot], slot_phase, meta, s_abort, limit, kSiteEpiTask)
                                    : wait_bar_cluster(&task_full[slot], slot_phase, meta, s_abort, limit, kSiteEpiTask);
         if (got && ring[slot].kind != kTaskStop)
           go = wait_bar(&acc_full[acc], acc_phase, meta, s_abort, limit, kSiteEpiAcc) ? 1 : 0;
-        *s_epi_go = go;
+        s_epi_go[it & 1] = go;
       }
       named_bar_sync(1, 128);
-      if (*s_epi_go == 0) break;
+      if (s_epi_go[it & 1] == 0) break;
       const Task t = ring[slot];
       tc_fence_after();
       const uint32_t tacc = tmem_base + acc * kAccCols + (static_cast<uint32_t>(q * 32) << 16);
