@@ -403,16 +403,23 @@ def run_mine(args, world, rank, local):
     gemm_ms = stage_ms[4]
     gbytes = algorithmic_bytes_gemm(w, stats["hit_experts"])
     gemm_flops = flops - 2.0 * w.T * w.H * w.E
+    # The GEMM is timed inside a loop of forwards. When that loop keeps the tensor cores busy for
+    # a second or more the 1 kW power cap sets the clock, and the sustained GEMM peak (a cuBLAS
+    # loop of seconds) is the fair denominator; a shorter pass is compared with the burst peak.
+    timed_pass_s = min(args.steps, 256) * ms * 1e-3
+    tc_kind = "sustained" if timed_pass_s >= 1.0 else "burst"
+    tc_peak = peaks["bf16_tflops_sustained"] if tc_kind == "sustained" else peaks["bf16_tflops"]
     hbm_t = gbytes / (peaks["hbm_gbs"] * 1e9)
-    tc_t = gemm_flops / (peaks["bf16_tflops"] * 1e12)
+    tc_t = gemm_flops / (tc_peak * 1e12)
     if hbm_t >= tc_t:
         achieved = gbytes / (gemm_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"]}
     else:
         achieved = gemm_flops / (gemm_ms * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": achieved / peaks["bf16_tflops"]}
+        roof = {"bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s",
+                "frac": achieved / tc_peak, "peak_kind": tc_kind,
+                "timed_pass_s": timed_pass_s, "frac_of_burst_peak": achieved / peaks["bf16_tflops"]}
     traffic = args.traffic_bytes if args.traffic_bytes is not None else measured_traffic(w.name)
     roof.update({"traffic": traffic, "kernel": "moe_gemm_kernel",
                  "algorithmic_bytes": gbytes, "kernel_ms": gemm_ms, "peak_source": peak_src,
