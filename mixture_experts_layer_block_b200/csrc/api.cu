@@ -270,6 +270,8 @@ int moe_init(const moe_config* cfg, moe_handle** out) {
       {(void**)&w.tile_expert, (size_t)h->max_tiles * 4},
       {(void**)&w.tile_row0, (size_t)h->max_tiles * 4},
       {(void**)&w.tile_nrows, (size_t)h->max_tiles * 4},
+      {(void**)&w.group_tile0, (size_t)h->max_tiles * 4},
+      {(void**)&w.group_ntiles, (size_t)h->max_tiles * 4},
       {(void**)&w.unit_start, (size_t)(h->max_units + 1) * 4},
       {(void**)&w.done1, (size_t)h->max_tiles * 4},
       {(void**)&w.h, (size_t)h->tile_rows * ldh * 2},
@@ -388,7 +390,7 @@ static int check_tokens(const moe_handle* h, int32_t T, int32_t top_k) {
 static int forward_impl(moe_handle* h, const void* x, int32_t T, const void* w_router,
                         const float* router_bias, const void* w_up, const void* w_gate,
                         const void* w_down, const moe_shared_w* w_shared, int32_t top_k,
-                        float* out, cudaStream_t st) {
+                        void* out, cudaStream_t st) {
   const moe_config& c = h->cfg;
   int rc;
   if ((rc = check_tokens(h, T, top_k))) return rc;
@@ -489,14 +491,14 @@ static int forward_impl(moe_handle* h, const void* x, int32_t T, const void* w_r
     if ((rc = check_cuda(launch_moe_gemm(maps, w, sh, h->num_sms, small, st)))) return rc;
   }
   if ((rc = mark(5))) return rc;
-  if ((rc = check_cuda(launch_combine(out, w, sh, st)))) return rc;
+  if ((rc = check_cuda(launch_combine(out, (c.flags & MOE_FLAG_OUT_BF16) != 0, w, sh, st)))) return rc;
   if ((rc = mark(6))) return rc;
   return MOE_OK;
 }
 
 int moe_forward(moe_handle* h, const void* x, int32_t T, const void* w_router,
                 const float* router_bias, const void* w_up, const void* w_gate, const void* w_down,
-                const moe_shared_w* w_shared, int32_t top_k, float* out, void* stream) {
+                const moe_shared_w* w_shared, int32_t top_k, void* out, void* stream) {
   if (!h) return MOE_ERR_INVALID_ARG;
   return forward_impl(h, x, T, w_router, router_bias, w_up, w_gate, w_down, w_shared, top_k, out,
                       static_cast<cudaStream_t>(stream));
@@ -505,7 +507,7 @@ int moe_forward(moe_handle* h, const void* x, int32_t T, const void* w_router,
 int moe_forward_host(moe_handle* h, const void* x_host, int32_t T, const void* w_router,
                      const float* router_bias, const void* w_up, const void* w_gate,
                      const void* w_down, const moe_shared_w* w_shared, int32_t top_k,
-                     float* out_host, void* stream) {
+                     void* out_host, void* stream) {
   if (!h) return MOE_ERR_INVALID_ARG;
   if (!h->x_stage || !h->out_stage) return MOE_ERR_NOT_READY;
   int rc;
@@ -513,7 +515,8 @@ int moe_forward_host(moe_handle* h, const void* x_host, int32_t T, const void* w
   if (!x_host || !out_host) return MOE_ERR_INVALID_ARG;
   if ((rc = select_device(h))) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const size_t xb = (size_t)T * h->cfg.hidden * 2, ob = (size_t)T * h->cfg.hidden * 4;
+  const size_t xb = (size_t)T * h->cfg.hidden * 2;
+  const size_t ob = (size_t)T * h->cfg.hidden * ((h->cfg.flags & MOE_FLAG_OUT_BF16) ? 2 : 4);
   if (T > 0 && cudaMemcpyAsync(h->x_stage, x_host, xb, cudaMemcpyHostToDevice, st) != cudaSuccess)
     return MOE_ERR_CUDA;
   if ((rc = forward_impl(h, h->x_stage, T, w_router, router_bias, w_up, w_gate, w_down, w_shared,

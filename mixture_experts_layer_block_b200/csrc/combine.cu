@@ -10,7 +10,8 @@
 //   tile row of y (bf16, like the per-slot intermediate cache of the vLLM execution
 //   analysis); this kernel adds, per token, the shared-expert row first and then the slots
 //   j = 0..k-1 in order (dropped slots skipped), in fp32. The order is fixed, so the result
-//   does not depend on the schedule. One warp per (token, 512 columns).
+//   does not depend on the schedule. The sum is stored as fp32, or rounded once to bf16.
+//   One warp per (token, 512 columns).
 #include <algorithm>
 
 #include "launch.h"
@@ -53,9 +54,24 @@ __device__ __forceinline__ void add_bf16x8(float (&acc)[8], const uint4 v) {
   }
 }
 
+// Stores 8 consecutive sums at element `off` of `out`: fp32, or bf16 rounded to nearest even.
+template <bool kBf16>
+__device__ __forceinline__ void store8(void* out, size_t off, const float (&a)[8]) {
+  if constexpr (kBf16) {
+    *reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + off) =
+        make_uint4(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]), pack_bf16x2(a[4], a[5]),
+                   pack_bf16x2(a[6], a[7]));
+  } else {
+    float4* o = reinterpret_cast<float4*>(static_cast<float*>(out) + off);
+    o[0] = make_float4(a[0], a[1], a[2], a[3]);
+    o[1] = make_float4(a[4], a[5], a[6], a[7]);
+  }
+}
+
 // One warp per (token, 512 columns); each lane sums 8 columns in each 256-column half.
+template <bool kBf16>
 __global__ void __launch_bounds__(256)
-    combine_kernel(float* __restrict__ out, Workspace ws, Shape sh) {
+    combine_kernel(void* __restrict__ out, Workspace ws, Shape sh) {
   griddep_wait();
   griddep_launch_dependents();
   const int lane = threadIdx.x & 31;
@@ -86,15 +102,9 @@ __global__ void __launch_bounds__(256)
       if (has1) add_bf16x8(a1, __ldcg(reinterpret_cast<const uint4*>(yr + c1)));
       add_bf16x8(a0, v0);
     }
-    float* orow = out + (size_t)t * sh.H;
-    float4* o0 = reinterpret_cast<float4*>(orow + c0);
-    o0[0] = make_float4(a0[0], a0[1], a0[2], a0[3]);
-    o0[1] = make_float4(a0[4], a0[5], a0[6], a0[7]);
-    if (has1) {
-      float4* o1 = reinterpret_cast<float4*>(orow + c1);
-      o1[0] = make_float4(a1[0], a1[1], a1[2], a1[3]);
-      o1[1] = make_float4(a1[4], a1[5], a1[6], a1[7]);
-    }
+    const size_t orow = (size_t)t * sh.H;
+    store8<kBf16>(out, orow + c0, a0);
+    if (has1) store8<kBf16>(out, orow + c1, a1);
   }
 }
 
@@ -103,10 +113,11 @@ cudaError_t launch_gather_rows(const uint16_t* x, const Workspace& ws, const Sha
   return launch_k(gather_rows_kernel, dim3(grid), dim3(256), 0, stream, x, ws, sh);
 }
 
-cudaError_t launch_combine(float* out, const Workspace& ws, const Shape& sh, cudaStream_t stream) {
+cudaError_t launch_combine(void* out, bool bf16_out, const Workspace& ws, const Shape& sh, cudaStream_t stream) {
   const int64_t warps = (int64_t)sh.T * ceil_div(sh.H, 512);
   const int grid = (int)std::min<int64_t>((warps + 7) / 8, 148 * 16);
-  return launch_k(combine_kernel, dim3(grid), dim3(256), 0, stream, out, ws, sh);
+  if (bf16_out) return launch_k(combine_kernel<true>, dim3(grid), dim3(256), 0, stream, out, ws, sh);
+  return launch_k(combine_kernel<false>, dim3(grid), dim3(256), 0, stream, out, ws, sh);
 }
 
 }  // namespace moe

@@ -20,6 +20,13 @@ constexpr int kABytes = kBM * kBK * 2;       // 16 KB
 constexpr int kBBytes = kUmmaN * kBK * 2;    // 32 KB
 constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kTaskSlots = 4;   // depth of the producer -> MMA/epilogue task ring
+#ifndef MOE_GROUP_TILES
+#define MOE_GROUP_TILES 2
+#endif
+// Consecutive m-tiles of one expert are scheduled as a group of up to this many: the group's
+// up (and down) tasks are numbered n-major across its tiles, so the tasks that read the same
+// weight rows are claimed back to back and stream those rows together through L2.
+constexpr int kGroupTiles = MOE_GROUP_TILES;
 constexpr int kStagingBytes = 128 * 128;  // one epilogue staging buffer: 128 rows x 128 B
 constexpr int kNumStaging = 2;            // double-buffered epilogue -> TMA store staging
 constexpr int kAccCols = 256;   // TMEM columns per accumulator buffer (2 buffers)
@@ -66,7 +73,9 @@ struct DeviceMeta {
   int P;              // num_post_padded
   int trace_count;    // trace records written
   int num_routed_tiles;  // m-tiles of routed experts (shared-expert tiles follow them)
-  int pad[6];
+  int num_groups;     // scheduling groups of up to kGroupTiles tiles of one expert
+  int num_routed_groups;  // groups of routed experts (shared-expert groups follow them)
+  int pad[4];
 };
 
 // Task kinds in the ring.
@@ -101,7 +110,9 @@ struct Workspace {
   int32_t* tile_expert;  // [max_tiles]
   int32_t* tile_row0;    // [max_tiles]
   int32_t* tile_nrows;   // [max_tiles]
-  int32_t* unit_start;   // [max_tiles + max_lag + 1]
+  int32_t* group_tile0;  // [max_tiles]      first m-tile of each scheduling group
+  int32_t* group_ntiles; // [max_tiles]      m-tiles in each group (1..kGroupTiles)
+  int32_t* unit_start;   // [max_groups + max_lag + 1]
   int32_t* done1;        // [max_tiles]      finished up/gate tasks per tile
   int32_t* expert_tile0; // [E]              first m-tile of each expert
   int32_t* row_of_slot;  // [S]              tile row (tile*tile_m + r) of each kept slot, -1 if dropped
@@ -202,6 +213,26 @@ __device__ __forceinline__ int find_unit(const int32_t* unit_start, int num_unit
     u += adv;
     if (adv < 32) return u;
   }
+}
+
+// Position of task `tau` of unit `u`: unit u holds the up tasks of group u, then the down tasks
+// of group u - lag; inside a group the tasks run n-major over its tiles.
+struct TaskPos {
+  int kind, tile, nt;
+};
+__device__ __forceinline__ TaskPos decode_task(const Workspace& ws, const Shape& sh, int u, int tau, int Mg,
+                                               int Mgr) {
+  const int off = tau - __ldcg(&ws.unit_start[u]);
+  int n1u = 0;
+  if (u < Mg) {
+    const int g = __ldcg(&ws.group_ntiles[u]);
+    n1u = ceil_div(u < Mgr ? sh.D : sh.Ds, kBN1) * g;
+    if (off < n1u) return TaskPos{kTaskUp, __ldcg(&ws.group_tile0[u]) + off % g, off / g};
+  }
+  const int gl = u - sh.lag;
+  const int g = __ldcg(&ws.group_ntiles[gl]);
+  const int o = off - n1u;
+  return TaskPos{kTaskDown, __ldcg(&ws.group_tile0[gl]) + o % g, o / g};
 }
 
 // Wait for the last TMA fill of every stage of a ring that was filled `nfill` times in

@@ -223,6 +223,7 @@ __device__ void align_scans(const Workspace& ws, const Shape& sh, bool tiles, in
       ws.tile_row0[first + i] = off + i * tm;
       ws.tile_nrows[first + i] = min(tm, kept[e] - i * tm);
     }
+    offs[e] = first;  // the segment offsets are no longer needed: keep the first tile instead
   }
   const int Ms = (sh.Ds > 0) ? ceil_div(sh.T, tm) : 0;
   for (int j = tid; j < Ms; j += nthr) {
@@ -233,15 +234,35 @@ __device__ void align_scans(const Workspace& ws, const Shape& sh, bool tiles, in
   const int Mt = Mr + Ms;
   __syncthreads();
 
-  // 4. schedule units: unit u holds the up/gate tasks of tile u, then the down tasks of tile
+  // 3b. scheduling groups: up to kGroupTiles consecutive tiles of one expert (the shared
+  //     expert's tiles are grouped the same way)
+  for (int e = tid; e < E; e += nthr) buf[e] = ceil_div(ceil_div(kept[e], tm), kGroupTiles);
+  __syncthreads();
+  const int Mgr = block_exclusive_scan(buf, E, tmp);
+  for (int e = tid; e < E; e += nthr) {
+    const int nt = ceil_div(kept[e], tm), first = offs[e], g0 = buf[e];
+    for (int i = 0; i * kGroupTiles < nt; ++i) {
+      ws.group_tile0[g0 + i] = first + i * kGroupTiles;
+      ws.group_ntiles[g0 + i] = min(kGroupTiles, nt - i * kGroupTiles);
+    }
+  }
+  const int Mgs = ceil_div(Ms, kGroupTiles);
+  for (int j = tid; j < Mgs; j += nthr) {
+    ws.group_tile0[Mgr + j] = Mr + j * kGroupTiles;
+    ws.group_ntiles[Mgr + j] = min(kGroupTiles, Ms - j * kGroupTiles);
+  }
+  const int Mg = Mgr + Mgs;
+  __syncthreads();
+
+  // 4. schedule units: unit u holds the up/gate tasks of group u, then the down tasks of group
   //    u - lag. Task ids are unit-major, so every down task's dependencies have lower ids.
-  const int U = (Mt > 0) ? Mt + sh.lag : 0;
+  const int U = (Mg > 0) ? Mg + sh.lag : 0;
   const int n2 = ceil_div(sh.H, kBN2);
   const int n1r = ceil_div(sh.D, kBN1), n1s = ceil_div(sh.Ds, kBN1);
   for (int u = tid; u < U; u += nthr) {
     int c = 0;
-    if (u < Mt) c += (u < Mr) ? n1r : n1s;  // routed tiles come first, then the shared ones
-    if (u >= sh.lag && u - sh.lag < Mt) c += n2;
+    if (u < Mg) c += ((u < Mgr) ? n1r : n1s) * ws.group_ntiles[u];  // routed groups first
+    if (u >= sh.lag && u - sh.lag < Mg) c += n2 * ws.group_ntiles[u - sh.lag];
     buf[u] = c;
   }
   __syncthreads();
@@ -252,6 +273,8 @@ __device__ void align_scans(const Workspace& ws, const Shape& sh, bool tiles, in
     ws.unit_start[U] = total;
     ws.meta->num_tiles = Mt;
     ws.meta->num_routed_tiles = Mr;
+    ws.meta->num_groups = Mg;
+    ws.meta->num_routed_groups = Mgr;
     ws.meta->num_units = U;
     ws.meta->total_tasks = total;
     ws.meta->task_counter = 0;

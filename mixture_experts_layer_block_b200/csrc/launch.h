@@ -78,8 +78,9 @@ cudaError_t ensure_align_smem(size_t hist_bytes, size_t scatter_bytes);
 cudaError_t launch_gather_rows(const uint16_t* x, const Workspace& ws, const Shape& sh, int grid,
                                cudaStream_t stream);
 
-// out[t] = (shared row of t) + sum_j y[row_of_slot[t*k+j]], in that order, fp32.
-cudaError_t launch_combine(float* out, const Workspace& ws, const Shape& sh, cudaStream_t stream);
+// out[t] = (shared row of t) + sum_j y[row_of_slot[t*k+j]], in that order, summed in fp32 and
+// stored as fp32 (or rounded to bf16 when bf16_out).
+cudaError_t launch_combine(void* out, bool bf16_out, const Workspace& ws, const Shape& sh, cudaStream_t stream);
 
 // Persistent expert GEMMs. `small` selects the shape for batches of at most 16 tokens (its
 // maps must use 16-row boxes for x_tile, xs, h_routed and h_shared).

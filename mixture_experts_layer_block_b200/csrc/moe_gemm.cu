@@ -133,7 +133,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 0) {
     // ===================================== producer =====================================
     const int total = __ldcg(&meta->total_tasks);
-    const int Mt = __ldcg(&meta->num_tiles);
+    const int Mg = __ldcg(&meta->num_groups), Mgr = __ldcg(&meta->num_routed_groups);
     const int U = __ldcg(&meta->num_units);
     const int nk1 = ceil_div(sh.H, kBK);
     int u_cur = 0;
@@ -148,18 +148,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         t.kind = kTaskStop;
       } else {
         u_cur = find_unit(ws.unit_start, U, tau, u_cur);
-        const int off = tau - __ldcg(&ws.unit_start[u_cur]);
-        const int n1u = (u_cur < Mt) ? n1_of(__ldcg(&ws.tile_expert[u_cur]), sh) : 0;
-        int nt;
-        if (off < n1u) {
-          t.kind = kTaskUp;
-          t.tile = u_cur;
-          nt = off;
-        } else {
-          t.kind = kTaskDown;
-          t.tile = u_cur - sh.lag;
-          nt = off - n1u;
-        }
+        const TaskPos pos = decode_task(ws, sh, u_cur, tau, Mg, Mgr);
+        t.kind = pos.kind;
+        t.tile = pos.tile;
+        const int nt = pos.nt;
         t.expert = __ldcg(&ws.tile_expert[t.tile]);
         t.row0 = __ldcg(&ws.tile_row0[t.tile]);
         t.nrows = __ldcg(&ws.tile_nrows[t.tile]);

@@ -165,7 +165,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t ring_c1 = mapa_shared(smem_u32(ring), 1);
     const uint32_t task_full_c1 = mapa_shared(smem_u32(task_full), 1);
     const int total = __ldcg(&meta->total_tasks);
-    const int Mt = __ldcg(&meta->num_tiles);
+    const int Mg = __ldcg(&meta->num_groups), Mgr = __ldcg(&meta->num_routed_groups);
     const int U = __ldcg(&meta->num_units);
     int u_cur = 0;
     uint32_t stage = 0, phase = 0, slot = 0, slot_phase = 0;
@@ -181,18 +181,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         t.tile = t.expert = t.row0 = t.nrows = t.n0 = t.nk = 0;
         if (tau < total) {
           u_cur = find_unit(ws.unit_start, U, tau, u_cur);
-          const int off = tau - __ldcg(&ws.unit_start[u_cur]);
-          const int n1u = (u_cur < Mt) ? n1_of(__ldcg(&ws.tile_expert[u_cur]), sh) : 0;
-          int nt;
-          if (off < n1u) {
-            t.kind = kTaskUp;
-            t.tile = u_cur;
-            nt = off;
-          } else {
-            t.kind = kTaskDown;
-            t.tile = u_cur - sh.lag;
-            nt = off - n1u;
-          }
+          const TaskPos pos = decode_task(ws, sh, u_cur, tau, Mg, Mgr);
+          t.kind = pos.kind;
+          t.tile = pos.tile;
+          const int nt = pos.nt;
           t.expert = __ldcg(&ws.tile_expert[t.tile]);
           t.row0 = __ldcg(&ws.tile_row0[t.tile]);
           t.nrows = __ldcg(&ws.tile_nrows[t.tile]);

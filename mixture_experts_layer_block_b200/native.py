@@ -27,6 +27,7 @@ MOE_FLAG_STAGE_TIMING = 1
 MOE_FLAG_HOST_STAGING = 2
 MOE_FLAG_PAIR_TILES = 8
 MOE_FLAG_SINGLE_TILES = 16
+MOE_FLAG_OUT_BF16 = 32
 MOE_FLAG_TRACE = 4
 
 
@@ -123,7 +124,7 @@ def _stream(stream):
 class MoELayer:
     """Owns one moe_handle. Tensors are torch CUDA tensors laid out as include/moe_b200.h
     states (x [T,H] bf16, W_router [E,H], W_up/W_gate [E,D,H], W_down [E,H,D] bf16, bias [E]
-    fp32, out [T,H] fp32)."""
+    fp32, out [T,H] fp32, or bf16 with MOE_FLAG_OUT_BF16)."""
 
     def __init__(self, hidden, inter, num_experts, top_k, block_m, max_tokens, inter_shared=0,
                  capacity_factor=0.0, flags=0, device=-1, timeout_ns=0):
@@ -132,6 +133,13 @@ class MoELayer:
         h = ctypes.c_void_p()
         check(lib.moe_init(ctypes.byref(self.cfg), ctypes.byref(h)), "moe_init")
         self.h = h
+        self.out_dtype = "bfloat16" if flags & MOE_FLAG_OUT_BF16 else "float32"
+
+    def _check_out(self, out):
+        # the library writes out in the dtype the handle was configured for
+        dt = getattr(out, "dtype", None)
+        if dt is not None and str(dt).split(".")[-1] != self.out_dtype:
+            raise TypeError(f"out must be {self.out_dtype} for this handle, got {dt}")
 
     @classmethod
     def for_workload(cls, w, max_tokens=None, **kw):
@@ -156,6 +164,7 @@ class MoELayer:
         return ctypes.byref(s), s
 
     def forward(self, x, wts, out, top_k=None, stream=None):
+        self._check_out(out)
         sh = self._shared(wts)
         check(lib.moe_forward(self.h, _ptr(x), x.shape[0], _ptr(wts["W_router"]), _ptr(wts.get("bias")),
                               _ptr(wts["W_up"]), _ptr(wts["W_gate"]), _ptr(wts["W_down"]),
@@ -164,6 +173,7 @@ class MoELayer:
         return out
 
     def forward_host(self, x_host, wts, out_host, top_k=None, stream=None):
+        self._check_out(out_host)
         sh = self._shared(wts)
         check(lib.moe_forward_host(self.h, _ptr(x_host), x_host.shape[0], _ptr(wts["W_router"]),
                                    _ptr(wts.get("bias")), _ptr(wts["W_up"]), _ptr(wts["W_gate"]),

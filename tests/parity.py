@@ -80,12 +80,12 @@ def compact_weights(inp: dict, experts: np.ndarray) -> dict:
     return out
 
 
-def check_forward(layer, w, inp: dict, tokens=None, out_tol: float = OUT_TOL):
+def check_forward(layer, w, inp: dict, tokens=None, out_tol: float = OUT_TOL, out_dtype=torch.float32):
     """Run the CUDA forward for workload `w` on `inp` (device tensors) and compare with the
     oracle on `tokens` (None = all). Returns a dict of the measured errors and counts."""
     dev = inp["x"].device
     T, H, k, E = w.T, w.H, w.top_k, w.E
-    out = torch.empty((T, H), dtype=torch.float32, device=dev)
+    out = torch.empty((T, H), dtype=out_dtype, device=dev)
     layer.forward(inp["x"], inp, out)
     dbg = layer.debug_outputs(T, k, dev)
     torch.cuda.synchronize()
@@ -137,7 +137,7 @@ def check_forward(layer, w, inp: dict, tokens=None, out_tol: float = OUT_TOL):
     cw = compact_weights(inp, experts)
     sub_ids = remap[ref_ids[tok]].astype(np.int32)
     ref_out = oracle.layer(x_h[torch.as_tensor(tok)], cw, sub_ids, ref_w[tok], ref_al["kept"][tok])
-    g_out = out.cpu().numpy()[tok].astype(np.float64)
+    g_out = out.float().cpu().numpy()[tok].astype(np.float64)
     out_err = rel_err(g_out, ref_out)
     assert np.all(np.isfinite(g_out))
     res = {"logit_err": logit_err, "weight_err": w_err, "out_err": out_err, "near_ties": n_tie,

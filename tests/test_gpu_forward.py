@@ -151,3 +151,27 @@ def test_forward_is_deterministic_in_routing():
     ref = outs[0].abs().max().item()
     for o in outs[1:]:
         assert (o - outs[0]).abs().max().item() <= 1e-5 * ref
+
+
+@pytest.mark.parametrize("name", ["tiny", "dsv3_small", "ragged_dims", "one_token", "small_tokens_shared"])
+def test_forward_bf16_out(name):
+    """MOE_FLAG_OUT_BF16: the combine's fp32 sums rounded once to bf16. Bit-identical to the fp32
+    output rounded to nearest even (same routing, same per-slot rows, same summation order), and
+    within tolerance of the oracle; the host-staged path returns the same bytes."""
+    from mixture_experts_layer_block_b200 import native
+    w = SMALL[name]
+    inp = {k: (v.cuda() if v is not None else None) for k, v in gen.make_inputs(w).items()}
+    l16 = _layer(w, flags=native.MOE_FLAG_OUT_BF16 | native.MOE_FLAG_HOST_STAGING)
+    check_forward(l16, w, inp, out_dtype=torch.bfloat16)
+    l32 = _layer(w)
+    o32 = torch.empty((w.T, w.H), dtype=torch.float32, device="cuda")
+    o16 = torch.empty((w.T, w.H), dtype=torch.bfloat16, device="cuda")
+    l32.forward(inp["x"], inp, o32)
+    l16.forward(inp["x"], inp, o16)
+    torch.cuda.synchronize()
+    assert torch.equal(o16, o32.to(torch.bfloat16))
+    oh = torch.empty((w.T, w.H), dtype=torch.bfloat16).pin_memory()
+    l16.forward_host(inp["x"].cpu().pin_memory(), inp, oh)
+    assert torch.equal(oh, o16.cpu())
+    with pytest.raises(TypeError):
+        l16.forward(inp["x"], inp, o32)
