@@ -68,6 +68,9 @@ extern "C" {
  * forces single SMs and wins over MOE_FLAG_PAIR_TILES. Both shapes compute the same result. */
 #define MOE_FLAG_PAIR_TILES    8u
 #define MOE_FLAG_SINGLE_TILES 16u
+/* moe_forward / moe_forward_host write `out` as bf16 [T][H] (the fp32 sum rounded to nearest
+ * even once) instead of fp32 [T][H]. */
+#define MOE_FLAG_OUT_BF16     32u
 
 typedef struct moe_config {
     int32_t hidden;           /* H: model dimension; multiple of 8 */
@@ -119,22 +122,23 @@ MOE_API void moe_destroy(moe_handle *h);
  *   w_down      device bf16 [E][H][D]
  *   w_shared    nullable; required (all three non-null) iff cfg.inter_shared > 0
  *   top_k       1..cfg.top_k
- *   out         device fp32 [T][H]; fully overwritten with x' (may be NULL when T == 0)
+ *   out         device fp32 [T][H], or bf16 [T][H] with MOE_FLAG_OUT_BF16; fully overwritten
+ *               with x' (may be NULL when T == 0)
  * Asynchronous on `stream`; no host synchronisation, so it may be captured in a CUDA graph
  * once the handle's tensor-map cache holds the weight pointers. */
 MOE_API int moe_forward(moe_handle *h, const void *x, int32_t T, const void *w_router,
                 const float *router_bias, const void *w_up, const void *w_gate,
-                const void *w_down, const moe_shared_w *w_shared, int32_t top_k, float *out,
+                const void *w_down, const moe_shared_w *w_shared, int32_t top_k, void *out,
                 void *stream);
 
 /* moe_forward with HOST activations: copies x_host (bf16 [T][H], pinned host memory for
  * full speed) to a device staging buffer, runs the forward, copies the result to out_host
- * (fp32 [T][H]) and synchronises `stream`. Weights stay device pointers. Needs
+ * (fp32 [T][H], or bf16 with MOE_FLAG_OUT_BF16) and synchronises `stream`. Weights stay device pointers. Needs
  * MOE_FLAG_HOST_STAGING at moe_init (else MOE_ERR_NOT_READY). */
 MOE_API int moe_forward_host(moe_handle *h, const void *x_host, int32_t T, const void *w_router,
                      const float *router_bias, const void *w_up, const void *w_gate,
                      const void *w_down, const moe_shared_w *w_shared, int32_t top_k,
-                     float *out_host, void *stream);
+                     void *out_host, void *stream);
 
 /* Synchronise the handle's last stream and report the device status word:
  * *device_status = 0 when every kernel since the last call finished normally, else a
