@@ -451,6 +451,14 @@ static int forward_impl(moe_handle* h, const void* x, int32_t T, const void* w_r
   if ((rc = cached_map(h, &maps.w_gate, w_gate, H, (uint64_t)E * D, (uint64_t)H * 2, kBK, kBN1))) return rc;
   if ((rc = cached_map(h, &maps.w_down, w_down, D, (uint64_t)E * H, (uint64_t)D * 2, kBK, bn2))) return rc;
   maps.h_routed = small ? h->h_routed16 : (pair ? h->h_routed32 : h->h_routed);
+  maps.xs32 = h->xs_map32;
+  maps.h_routed32 = h->h_routed32;
+  maps.h_shared32 = h->h_shared32;
+  if (small || pair) {
+    maps.x_tile32 = maps.x_tile;  // unused by these shapes (the pair shape's x_tile has 32-row boxes)
+  } else if ((rc = encode_map(h, &maps.x_tile32, x, H, T, (uint64_t)H * 2, kBK, kPairBoxRows))) {
+    return rc;
+  }
   if (has_shared) {
     if ((rc = cached_map(h, &maps.ws_up, w_shared->up, H, Ds, (uint64_t)H * 2, kBK, kBN1))) return rc;
     if ((rc = cached_map(h, &maps.ws_gate, w_shared->gate, H, Ds, (uint64_t)H * 2, kBK, kBN1))) return rc;

@@ -41,6 +41,9 @@ struct alignas(64) GemmMaps {
   CUtensorMap ws_gate;   // [Ds][H]
   CUtensorMap ws_down;   // [H][Ds]
   CUtensorMap h_shared;  // h [rows][Ds], row stride ldh
+  // the same four A operands with 32-row boxes: the one-SM kernel loads a tile of at most 96
+  // rows as whole 32-row boxes instead of one 128-row box
+  CUtensorMap x_tile32, xs32, h_routed32, h_shared32;
 };
 
 // Router projection: logits[T][E] = x W^T (+ bias). x_map box {64,128}, w_map box {64,BN}.

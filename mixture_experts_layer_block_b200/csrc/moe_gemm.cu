@@ -196,6 +196,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       const int wrow_up = shared ? t.n0 : t.expert * sh.D + t.n0;
       const int wrow_dn = shared ? t.n0 : t.expert * sh.H + t.n0;
+      // A operand: one box of kARows rows, or (general shape, tiles of at most 96 rows) only
+      // the 32-row boxes that hold the tile's rows; the rest of the A slot keeps stale rows,
+      // whose results land in output rows past the tile's end
+      const bool up = (t.kind == kTaskUp);
+      const int nbox = (!kSmall && t.nrows <= 3 * kPairBoxRows) ? ceil_div(t.nrows, kPairBoxRows) : 0;
+      const uint32_t stage_tx = (nbox ? (uint32_t)nbox * kPairBoxRows * kBK * 2 : (uint32_t)kABytes) + kBBytes;
+      const CUtensorMap* amap = up ? (shared ? &maps.x_tile : &maps.xs) : (shared ? &maps.h_shared : &maps.h_routed);
+      const CUtensorMap* amap32 =
+          up ? (shared ? &maps.x_tile32 : &maps.xs32) : (shared ? &maps.h_shared32 : &maps.h_routed32);
+      const int arow = (up && shared) ? t.row0 : t.tile * kBM;
       for (int kb = 0; kb < t.nk; ++kb) {
         if (lane == 0) ok = wait_bar(&empty[stage], phase ^ 1, meta, s_abort, limit, kSiteProducerEmpty);
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -203,16 +213,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (lane == 0) {
           const uint32_t a = smem_u32(smem + stage * kStageBytes);
           const uint32_t b = a + kABytes;
-          mbar_arrive_expect_tx(&full[stage], kStageBytes);
-          if (t.kind == kTaskUp) {
-            // A: 128 rows of x in tile order (routed: gathered copy; shared: the tokens)
-            if (shared) tma_load_2d(a, &maps.x_tile, &full[stage], kb * kBK, t.row0);
-            else tma_load_2d(a, &maps.xs, &full[stage], kb * kBK, t.tile * kBM);
+          mbar_arrive_expect_tx(&full[stage], stage_tx);
+          // A: the tile's rows of x in tile order (routed: gathered copy; shared: the tokens),
+          // or of h for down tasks
+          if (nbox == 0) {
+            tma_load_2d(a, amap, &full[stage], kb * kBK, arow);
+          } else {
+            for (int j = 0; j < nbox; ++j)
+              tma_load_2d(a + j * kPairBoxRows * 128, amap32, &full[stage], kb * kBK, arow + j * kPairBoxRows);
+          }
+          if (up) {
             tma_load_2d(b, shared ? &maps.ws_up : &maps.w_up, &full[stage], kb * kBK, wrow_up);
             tma_load_2d(b + kBN1 * 128, shared ? &maps.ws_gate : &maps.w_gate, &full[stage], kb * kBK,
                         wrow_up);
           } else {
-            tma_load_2d(a, shared ? &maps.h_shared : &maps.h_routed, &full[stage], kb * kBK, t.tile * kBM);
             tma_load_2d(b, shared ? &maps.ws_down : &maps.w_down, &full[stage], kb * kBK, wrow_dn);
           }
         }
