@@ -71,6 +71,13 @@ extern "C" {
 /* moe_forward / moe_forward_host write `out` as bf16 [T][H] (the fp32 sum rounded to nearest
  * even once) instead of fp32 [T][H]. */
 #define MOE_FLAG_OUT_BF16     32u
+/* The one-SM expert GEMMs can compute a tile's tail of at most 32 rows inside the tasks of the
+ * expert's previous tile, from the same weight stages (the "tail" shape). By default they do so
+ * when the mean load per expert is 96..384 slots and the capacity allows more than 128;
+ * MOE_FLAG_TAIL_TILES asks for it on every batch of more than 16 tokens, MOE_FLAG_NO_TAIL_TILES
+ * never (it wins). Both compute the same result. */
+#define MOE_FLAG_TAIL_TILES   64u
+#define MOE_FLAG_NO_TAIL_TILES 128u
 
 typedef struct moe_config {
     int32_t hidden;           /* H: model dimension; multiple of 8 */
@@ -199,7 +206,8 @@ MOE_API int moe_stage_times(moe_handle *h, float *ms, int32_t n);
  * single SMs, or SM pairs; the SM count before any forward), 2 workspace bytes,
  * 3 tasks of the last forward (synchronises), 4 m-tiles of the last forward (synchronises),
  * 5 dependency lag (units) of the last forward, 6 rows per m-tile of the last forward
- * (128 or 256), 7 SM pairs the device can run at once for the pair shape (0 = none). */
+ * (128 or 256), 7 SM pairs the device can run at once for the pair shape (0 = none),
+ * 8 expert-GEMM shape of the last forward (0 general, 1 small-tile, 2 tail, 3 SM pairs). */
 MOE_API int moe_query(const moe_handle *h, int32_t which, int64_t *value);
 
 /* Per-task trace of the last forward (needs MOE_FLAG_TRACE; synchronises). Fills up to

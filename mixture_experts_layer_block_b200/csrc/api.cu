@@ -74,6 +74,7 @@ struct moe_handle {
   int64_t routed_rows = 0, tile_rows = 0;  // rows of xs, and of h and y, for either tile height
   int max_pairs = 0;                       // 2-CTA clusters of the pair kernel that fit at once
   int last_workers = 0, last_tile_m = kBM;
+  int last_shape = 0;  // expert-GEMM shape of the last forward: 0 general, 1 small, 2 tail, 3 pair
   int parts_rows = 0;  // rows of the K-split partial logits buffer
   std::vector<cudaEvent_t> ev;  // kTimingRing x (kNumStages + 1) events around the kernels
   int timed = 0;                // forwards recorded since the last moe_stage_times
@@ -272,6 +273,7 @@ int moe_init(const moe_config* cfg, moe_handle** out) {
       {(void**)&w.tile_nrows, (size_t)h->max_tiles * 4},
       {(void**)&w.group_tile0, (size_t)h->max_tiles * 4},
       {(void**)&w.group_ntiles, (size_t)h->max_tiles * 4},
+      {(void**)&w.group_tasks, (size_t)h->max_tiles * 4},
       {(void**)&w.unit_start, (size_t)(h->max_units + 1) * 4},
       {(void**)&w.done1, (size_t)h->max_tiles * 4},
       {(void**)&w.h, (size_t)h->tile_rows * ldh * 2},
@@ -423,6 +425,19 @@ static int forward_impl(moe_handle* h, const void* x, int32_t T, const void* w_r
     pair = true;
   const int workers = pair ? h->max_pairs : h->num_sms;
   Shape sh = make_shape(h, T, top_k, pair ? 2 * kBM : kBM, workers);
+  // Merging tails of at most 32 rows into the previous tile's tasks pays when experts get a few
+  // 128-row tiles each (many of them then end in a short tail), and costs the general shape's
+  // second staging buffer: by default it is used when the mean load per expert is 96..384
+  // slots and the capacity allows more than one tile per expert.
+  int gemm_shape = small ? kShapeSmall : kShapeGeneral;
+  if (!small && !pair && !(c.flags & MOE_FLAG_NO_TAIL_TILES)) {
+    const int64_t load = (int64_t)T * top_k;  // slots over E experts
+    const int cap = capacity_of(c, T, top_k);
+    const bool fits = load > (int64_t)96 * E && load <= (int64_t)384 * E && (cap == 0 || cap > kBM);
+    if (fits || (c.flags & MOE_FLAG_TAIL_TILES)) gemm_shape = kShapeTail;
+  }
+  h->last_shape = pair ? 3 : gemm_shape;
+  sh.merge_tail = (gemm_shape == kShapeTail) ? 1 : 0;
   h->last_workers = workers;
   h->last_tile_m = sh.tile_m;
   sh.dep_extra = h->dep_extra_next;
@@ -496,7 +511,7 @@ static int forward_impl(moe_handle* h, const void* x, int32_t T, const void* w_r
   if (pair) {
     if ((rc = check_cuda(launch_moe_gemm_pair(maps, w, sh, h->max_pairs, st)))) return rc;
   } else {
-    if ((rc = check_cuda(launch_moe_gemm(maps, w, sh, h->num_sms, small, st)))) return rc;
+    if ((rc = check_cuda(launch_moe_gemm(maps, w, sh, h->num_sms, gemm_shape, st)))) return rc;
   }
   if ((rc = mark(5))) return rc;
   if ((rc = check_cuda(launch_combine(out, (c.flags & MOE_FLAG_OUT_BF16) != 0, w, sh, st)))) return rc;
@@ -661,6 +676,7 @@ int moe_query(const moe_handle* h, int32_t which, int64_t* value) {
     case 5: *value = h->last_lag; return MOE_OK;
     case 6: *value = h->last_tile_m; return MOE_OK;
     case 7: *value = h->max_pairs; return MOE_OK;
+    case 8: *value = h->last_shape; return MOE_OK;
     default: return MOE_ERR_INVALID_ARG;
   }
 }

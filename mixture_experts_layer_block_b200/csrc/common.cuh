@@ -92,7 +92,11 @@ struct Task {
   int32_t n0;      // first output column (D for up tasks, H for down tasks)
   int32_t nk;      // K stages
   int32_t id;      // global task id
+  int32_t ntiles;  // 1, or 2: the task also computes the next tile (rows row0 + 128 ...), a
+                   // tail of nrows2 <= kTailRows rows, from the same B stages
+  int32_t nrows2;  // valid rows of that second tile
 };
+constexpr int kTailRows = 32;  // a tile this short rides along with its expert's previous tile
 
 // Pointers into the workspace handed to the kernels.
 struct Workspace {
@@ -112,6 +116,9 @@ struct Workspace {
   int32_t* tile_nrows;   // [max_tiles]
   int32_t* group_tile0;  // [max_tiles]      first m-tile of each scheduling group
   int32_t* group_ntiles; // [max_tiles]      m-tiles in each group (1..kGroupTiles)
+  int32_t* group_tasks;  // [max_tiles]      task sets per n-tile: group_ntiles, or 1 when the
+                         //                  group's last tile is a tail merged into the tasks
+                         //                  of the tile before it
   int32_t* unit_start;   // [max_groups + max_lag + 1]
   int32_t* done1;        // [max_tiles]      finished up/gate tasks per tile
   int32_t* expert_tile0; // [E]              first m-tile of each expert
@@ -134,6 +141,8 @@ struct Shape {
   int32_t lag;           // scheduling lag in units between a tile's up and down tasks
   int32_t dep_extra;     // testing hook: extra up completions a down task waits for
   int32_t tile_m;        // rows per m-tile of the expert GEMMs: 128, or 256 on SM pairs
+  int32_t merge_tail;    // 1: a group of a full tile and a tail of <= kTailRows rows runs as one
+                         //    task set (the one-SM general shape only)
   int64_t timeout_ns;
 };
 
@@ -218,21 +227,26 @@ __device__ __forceinline__ int find_unit(const int32_t* unit_start, int num_unit
 // Position of task `tau` of unit `u`: unit u holds the up tasks of group u, then the down tasks
 // of group u - lag; inside a group the tasks run n-major over its tiles.
 struct TaskPos {
-  int kind, tile, nt;
+  int kind, tile, nt, ntiles;
 };
 __device__ __forceinline__ TaskPos decode_task(const Workspace& ws, const Shape& sh, int u, int tau, int Mg,
                                                int Mgr) {
-  const int off = tau - __ldcg(&ws.unit_start[u]);
-  int n1u = 0;
-  if (u < Mg) {
-    const int g = __ldcg(&ws.group_ntiles[u]);
-    n1u = ceil_div(u < Mgr ? sh.D : sh.Ds, kBN1) * g;
-    if (off < n1u) return TaskPos{kTaskUp, __ldcg(&ws.group_tile0[u]) + off % g, off / g};
-  }
+  // every load depends only on u: they go out together (one round trip per claim)
   const int gl = u - sh.lag;
-  const int g = __ldcg(&ws.group_ntiles[gl]);
+  const bool has_up = u < Mg, has_dn = gl >= 0 && gl < Mg;
+  const int us = __ldcg(&ws.unit_start[u]);
+  const int gu = has_up ? __ldcg(&ws.group_tasks[u]) : 1;
+  const int tu = has_up ? __ldcg(&ws.group_tile0[u]) : 0;
+  const int nu = has_up ? __ldcg(&ws.group_ntiles[u]) : 1;
+  const int gd = has_dn ? __ldcg(&ws.group_tasks[gl]) : 1;
+  const int td = has_dn ? __ldcg(&ws.group_tile0[gl]) : 0;
+  const int nd = has_dn ? __ldcg(&ws.group_ntiles[gl]) : 1;
+  const int off = tau - us;
+  const int n1u = has_up ? ceil_div(u < Mgr ? sh.D : sh.Ds, kBN1) * gu : 0;
+  // a merged group (one task set for two tiles) computes both tiles in each task
+  if (off < n1u) return TaskPos{kTaskUp, tu + off % gu, off / gu, gu == 1 ? nu : 1};
   const int o = off - n1u;
-  return TaskPos{kTaskDown, __ldcg(&ws.group_tile0[gl]) + o % g, o / g};
+  return TaskPos{kTaskDown, td + o % gd, o / gd, gd == 1 ? nd : 1};
 }
 
 // Wait for the last TMA fill of every stage of a ring that was filled `nfill` times in

@@ -239,17 +239,35 @@ __device__ void align_scans(const Workspace& ws, const Shape& sh, bool tiles, in
   for (int e = tid; e < E; e += nthr) buf[e] = ceil_div(ceil_div(kept[e], tm), kGroupTiles);
   __syncthreads();
   const int Mgr = block_exclusive_scan(buf, E, tmp);
+  // A group of two tiles whose second is a tail of at most kTailRows rows runs as one task set
+  // when sh.merge_tail: each task computes both tiles from the same weight stages. With pairs of
+  // tiles, a run of an odd number of tiles that ends in a tail starts with a single-tile group,
+  // so that the tail closes a pair.
+  auto put_group = [&](int gi, int t0, int g, int last_rows) {
+    ws.group_tile0[gi] = t0;
+    ws.group_ntiles[gi] = g;
+    ws.group_tasks[gi] = (sh.merge_tail && g == 2 && last_rows <= kTailRows) ? 1 : g;
+  };
+  // tiles [start, start + g) of group j of a run of nt tiles whose last tile has last_rows rows
+  auto group_span = [&](int j, int nt, int last_rows, int& start, int& g) {
+    const int f = (kGroupTiles == 2 && sh.merge_tail && nt > 1 && (nt & 1) && last_rows <= kTailRows) ? 1 : 0;
+    start = (f && j > 0) ? kGroupTiles * j - 1 : kGroupTiles * j;
+    g = (f && j == 0) ? 1 : min(kGroupTiles, nt - start);
+  };
   for (int e = tid; e < E; e += nthr) {
     const int nt = ceil_div(kept[e], tm), first = offs[e], g0 = buf[e];
+    const int last_rows = kept[e] - (nt - 1) * tm;
     for (int i = 0; i * kGroupTiles < nt; ++i) {
-      ws.group_tile0[g0 + i] = first + i * kGroupTiles;
-      ws.group_ntiles[g0 + i] = min(kGroupTiles, nt - i * kGroupTiles);
+      int st, g;
+      group_span(i, nt, last_rows, st, g);
+      put_group(g0 + i, first + st, g, min(tm, kept[e] - (st + g - 1) * tm));
     }
   }
   const int Mgs = ceil_div(Ms, kGroupTiles);
   for (int j = tid; j < Mgs; j += nthr) {
-    ws.group_tile0[Mgr + j] = Mr + j * kGroupTiles;
-    ws.group_ntiles[Mgr + j] = min(kGroupTiles, Ms - j * kGroupTiles);
+    int st, g;
+    group_span(j, Ms, sh.T - (Ms - 1) * tm, st, g);
+    put_group(Mgr + j, Mr + st, g, min(tm, sh.T - (st + g - 1) * tm));
   }
   const int Mg = Mgr + Mgs;
   __syncthreads();
@@ -261,8 +279,8 @@ __device__ void align_scans(const Workspace& ws, const Shape& sh, bool tiles, in
   const int n1r = ceil_div(sh.D, kBN1), n1s = ceil_div(sh.Ds, kBN1);
   for (int u = tid; u < U; u += nthr) {
     int c = 0;
-    if (u < Mg) c += ((u < Mgr) ? n1r : n1s) * ws.group_ntiles[u];  // routed groups first
-    if (u >= sh.lag && u - sh.lag < Mg) c += n2 * ws.group_ntiles[u - sh.lag];
+    if (u < Mg) c += ((u < Mgr) ? n1r : n1s) * ws.group_tasks[u];  // routed groups first
+    if (u >= sh.lag && u - sh.lag < Mg) c += n2 * ws.group_tasks[u - sh.lag];
     buf[u] = c;
   }
   __syncthreads();

@@ -85,11 +85,14 @@ cudaError_t launch_gather_rows(const uint16_t* x, const Workspace& ws, const Sha
 // stored as fp32 (or rounded to bf16 when bf16_out).
 cudaError_t launch_combine(void* out, bool bf16_out, const Workspace& ws, const Shape& sh, cudaStream_t stream);
 
-// Persistent expert GEMMs. `small` selects the shape for batches of at most 16 tokens (its
-// maps must use 16-row boxes for x_tile, xs, h_routed and h_shared).
-size_t gemm_smem_bytes(bool small);
-cudaError_t launch_moe_gemm(const GemmMaps& maps, const Workspace& ws, const Shape& sh, int grid,
-                            bool small, cudaStream_t stream);
+// Persistent expert GEMMs in one of three shapes: general (128-row tiles), tail (the same with
+// tails of at most 32 rows merged into the previous tile's tasks; needs sh.merge_tail = 1) and
+// small (batches of at most 16 tokens; its maps use 16-row boxes for x_tile, xs, h_routed and
+// h_shared).
+enum GemmShape : int { kShapeGeneral = 0, kShapeSmall = 1, kShapeTail = 2 };
+size_t gemm_smem_bytes(int shape);
+cudaError_t launch_moe_gemm(const GemmMaps& maps, const Workspace& ws, const Shape& sh, int grid, int shape,
+                            cudaStream_t stream);
 
 // The same GEMMs with 256-row m-tiles on `pairs` 2-CTA clusters (sh.tile_m = 256; its maps use
 // 32-row boxes for x_tile, xs, h_routed, h_shared and y, and 128-row boxes for w_down, ws_down).

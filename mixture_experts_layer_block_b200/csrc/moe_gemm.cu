@@ -38,20 +38,25 @@ namespace moe {
 
 namespace {
 
-// Two shapes of the kernel. The general one moves 128-row A tiles through a 4 x 48 KB ring
-// and writes its epilogue results with TMA stores from two staging buffers. The small-tile
-// one serves batches of at most 16 tokens (every m-tile then holds at most 16 rows): it moves
-// 16-row A boxes (2 KB), so the same shared memory holds a 6 x 34 KB ring and 50% more weight
-// bytes in flight per SM, and its epilogue stores the valid rows directly. Its MMAs stay
-// M=128: rows 16..127 read the stage's B bytes (finite values) and their results are never
-// stored.
-template <bool kSmall>
+// Three shapes of the kernel (GemmShape). The general one moves 128-row A tiles through a
+// 4 x 48 KB ring and writes its epilogue results with TMA stores from two staging buffers.
+// The tail shape adds a 4 KB slot per stage for the 32 rows of a tail tile that rides along in
+// the tasks of its expert's previous tile (4 x 52 KB ring), which leaves room for one staging
+// buffer only. The small-tile one serves batches of at most 16 tokens (every m-tile then holds
+// at most 16 rows): it moves 16-row A boxes (2 KB), so the same shared memory holds a
+// 6 x 34 KB ring and 50% more weight bytes in flight per SM, and its epilogue stores the valid
+// rows directly. Its MMAs stay M=128: rows 16..127 read the stage's B bytes (finite values)
+// and their results are never stored.
+template <int kShape>
 struct Cfg {
+  static constexpr bool kSmall = (kShape == kShapeSmall);
+  static constexpr bool kTail = (kShape == kShapeTail);
   static constexpr int kStagesN = kSmall ? 6 : kStages;
   static constexpr int kARows = kSmall ? 16 : kBM;
   static constexpr int kABytesN = kARows * kBK * 2;
-  static constexpr int kStageBytesN = kABytesN + kBBytes;
-  static constexpr int kNumStagingN = kSmall ? 0 : kNumStaging;
+  static constexpr int kTailBytesN = kTail ? kTailRows * kBK * 2 : 0;
+  static constexpr int kStageBytesN = kABytesN + kTailBytesN + kBBytes;
+  static constexpr int kNumStagingN = kSmall ? 0 : (kTail ? 1 : kNumStaging);
   static constexpr int kStagingOff = kStagesN * kStageBytesN;
   static constexpr int kBarOff = kStagingOff + kNumStagingN * kStagingBytes;
   // barriers: full[S], empty[S], acc_full[2], acc_empty[2], task_full[R], task_empty[R], drain
@@ -59,7 +64,8 @@ struct Cfg {
   static constexpr int kRingOff = kBarOff + ((kNumBars * 8 + 63) & ~63);
   static constexpr int kMiscOff = kRingOff + kTaskSlots * (int)sizeof(Task);
   static constexpr int kBytes = kMiscOff + 64;
-  static_assert(kStageBytesN % 1024 == 0 && kABytesN % 1024 == 0, "1024-byte aligned operand tiles");
+  static_assert(kStageBytesN % 1024 == 0 && kABytesN % 1024 == 0 && kTailBytesN % 1024 == 0,
+                "1024-byte aligned operand tiles");
   static_assert(kBytes + 1024 <= 227 * 1024, "shared memory budget");
 };
 
@@ -69,13 +75,16 @@ __device__ __forceinline__ int n1_of(int expert, const Shape& sh) {
 
 }  // namespace
 
-template <bool kSmall>
+template <int kShape>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     moe_gemm_kernel(const __grid_constant__ GemmMaps maps, Workspace ws, Shape sh) {
-  using C = Cfg<kSmall>;
+  using C = Cfg<kShape>;
+  constexpr bool kSmall = C::kSmall;
+  constexpr bool kTail = C::kTail;
   constexpr int kStages = C::kStagesN;
   constexpr int kStageBytes = C::kStageBytesN;
   constexpr int kABytes = C::kABytesN;
+  constexpr int kBOff = C::kABytesN + C::kTailBytesN;  // B's offset in a stage
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
@@ -144,6 +153,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tau = __shfl_sync(0xffffffffu, tau, 0);
       Task t;
       t.id = tau;
+      t.ntiles = 1;
+      t.nrows2 = 0;
       if (tau >= total) {
         t.kind = kTaskStop;
       } else {
@@ -155,6 +166,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         t.expert = __ldcg(&ws.tile_expert[t.tile]);
         t.row0 = __ldcg(&ws.tile_row0[t.tile]);
         t.nrows = __ldcg(&ws.tile_nrows[t.tile]);
+        t.ntiles = kTail ? pos.ntiles : 1;
+        t.nrows2 = (t.ntiles == 2) ? __ldcg(&ws.tile_nrows[t.tile + 1]) : 0;
         const int Dt = (t.expert == sh.E) ? sh.Ds : sh.D;
         if (t.kind == kTaskUp) {
           t.n0 = nt * kBN1;
@@ -185,10 +198,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
       }
       const bool shared = (t.expert == sh.E);
-      // a down task needs every up task of its tile
+      // a down task needs every up task of its tile(s)
       if (t.kind == kTaskDown) {
         if (lane == 0) {
-          ok = wait_count(&ws.done1[t.tile], n1_of(t.expert, sh) + sh.dep_extra, meta, s_abort, limit);
+          const int need = n1_of(t.expert, sh) + sh.dep_extra;
+          ok = wait_count(&ws.done1[t.tile], need, meta, s_abort, limit);
+          if (ok && t.ntiles == 2) ok = wait_count(&ws.done1[t.tile + 1], need, meta, s_abort, limit);
           if (ok) fence_proxy_async_global();
         }
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -201,18 +216,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // whose results land in output rows past the tile's end
       const bool up = (t.kind == kTaskUp);
       const int nbox = (!kSmall && t.nrows <= 3 * kPairBoxRows) ? ceil_div(t.nrows, kPairBoxRows) : 0;
-      const uint32_t stage_tx = (nbox ? (uint32_t)nbox * kPairBoxRows * kBK * 2 : (uint32_t)kABytes) + kBBytes;
+      const uint32_t stage_tx = (nbox ? (uint32_t)nbox * kPairBoxRows * kBK * 2 : (uint32_t)kABytes) + kBBytes +
+                                (t.ntiles == 2 ? (uint32_t)kTailRows * kBK * 2 : 0u);
       const CUtensorMap* amap = up ? (shared ? &maps.x_tile : &maps.xs) : (shared ? &maps.h_shared : &maps.h_routed);
       const CUtensorMap* amap32 =
           up ? (shared ? &maps.x_tile32 : &maps.xs32) : (shared ? &maps.h_shared32 : &maps.h_routed32);
       const int arow = (up && shared) ? t.row0 : t.tile * kBM;
+      const int arow2 = (up && shared) ? t.row0 + kBM : (t.tile + 1) * kBM;  // a merged tail's rows
       for (int kb = 0; kb < t.nk; ++kb) {
         if (lane == 0) ok = wait_bar(&empty[stage], phase ^ 1, meta, s_abort, limit, kSiteProducerEmpty);
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         if (!ok) break;
         if (lane == 0) {
           const uint32_t a = smem_u32(smem + stage * kStageBytes);
-          const uint32_t b = a + kABytes;
+          const uint32_t b = a + kBOff;
           mbar_arrive_expect_tx(&full[stage], stage_tx);
           // A: the tile's rows of x in tile order (routed: gathered copy; shared: the tokens),
           // or of h for down tasks
@@ -222,6 +239,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             for (int j = 0; j < nbox; ++j)
               tma_load_2d(a + j * kPairBoxRows * 128, amap32, &full[stage], kb * kBK, arow + j * kPairBoxRows);
           }
+          if (kTail && t.ntiles == 2) tma_load_2d(a + kABytes, amap32, &full[stage], kb * kBK, arow2);
           if (up) {
             tma_load_2d(b, shared ? &maps.ws_up : &maps.w_up, &full[stage], kb * kBK, wrow_up);
             tma_load_2d(b + kBN1 * 128, shared ? &maps.ws_gate : &maps.w_gate, &full[stage], kb * kBK,
@@ -238,34 +256,54 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else if (warp == 1) {
     // ===================================== MMA issuer ===================================
+    // A task uses the next accumulator, or both when it also computes a merged tail tile; each
+    // accumulator's barriers are phased by its own use count.
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(kBM, kUmmaN);
-      uint32_t stage = 0, phase = 0, slot = 0, slot_phase = 0, acc = 0, acc_phase = 0;
+      uint32_t stage = 0, phase = 0, slot = 0, slot_phase = 0, next = 0, use0 = 0, use1 = 0;
       while (true) {
         if (!wait_bar(&task_full[slot], slot_phase, meta, s_abort, limit, kSiteMmaTask)) break;
         const Task t = ring[slot];
         if (t.kind == kTaskStop) break;
-        if (!wait_bar(&acc_empty[acc], acc_phase ^ 1, meta, s_abort, limit, kSiteMmaAcc)) break;
+        const uint32_t a0 = next, a1 = next ^ 1u;
+        const bool two = kTail && (t.ntiles == 2);
+        if (!wait_bar(&acc_empty[a0], ((a0 ? use1 : use0) & 1u) ^ 1u, meta, s_abort, limit, kSiteMmaAcc)) break;
+        if (two && !wait_bar(&acc_empty[a1], ((a1 ? use1 : use0) & 1u) ^ 1u, meta, s_abort, limit, kSiteMmaAcc))
+          break;
         tc_fence_after();
-        const uint32_t d = tmem_base + acc * kAccCols;
+        const uint32_t d0 = tmem_base + a0 * kAccCols, d1 = tmem_base + a1 * kAccCols;
         bool ok = true;
         for (int kb = 0; kb < t.nk; ++kb) {
           if (!wait_bar(&full[stage], phase, meta, s_abort, limit, kSiteMmaFull)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a = smem_u32(smem + stage * kStageBytes);
-          const uint32_t b = a + kABytes;
+          const uint32_t b = a + kBOff;
 #pragma unroll
           for (int kk = 0; kk < kBK / kUK; ++kk)
-            umma_bf16(d, sdesc_kmajor_sw128(a + kk * 32), sdesc_kmajor_sw128(b + kk * 32), idesc,
+            umma_bf16(d0, sdesc_kmajor_sw128(a + kk * 32), sdesc_kmajor_sw128(b + kk * 32), idesc,
                       (kb | kk) != 0);
+          if (two) {
+            // the tail's 32 rows sit in the slot after A; its other 96 MMA rows read the start of
+            // B and land in accumulator rows that are never stored
+#pragma unroll
+            for (int kk = 0; kk < kBK / kUK; ++kk)
+              umma_bf16(d1, sdesc_kmajor_sw128(a + kABytes + kk * 32), sdesc_kmajor_sw128(b + kk * 32), idesc,
+                        (kb | kk) != 0);
+          }
           mma_issued = true;
           umma_commit(&empty[stage]);
           if (++stage == kStages) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
-        umma_commit(&acc_full[acc]);
+        umma_commit(&acc_full[a0]);
+        if (a0) ++use1; else ++use0;
+        if (two) {
+          umma_commit(&acc_full[a1]);
+          if (a1) ++use1; else ++use0;
+        } else {
+          next ^= 1u;
+        }
         mbar_arrive(&task_empty[slot]);
-        if (++acc == 2) { acc = 0; acc_phase ^= 1; }
         if (++slot == kTaskSlots) { slot = 0; slot_phase ^= 1; }
       }
     }
@@ -279,7 +317,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int row = q * 32 + lane;   // tile row owned by this thread
     const bool leader = (warp == 2 && lane == 0);
     uint8_t* staging = smem + C::kStagingOff;
-    uint32_t slot = 0, slot_phase = 0, acc = 0, acc_phase = 0, sb = 0;
+    // accumulator bookkeeping mirrors the MMA issuer: a task uses `next`, or both
+    // accumulators when it carries a merged tail tile; barriers are phased per accumulator
+    uint32_t slot = 0, slot_phase = 0, next = 0, use0 = 0, use1 = 0;
     // One thread waits for the next task and its accumulator and tells the other 127 through
     // the named barrier, so the four warps always take the same branch (a warp that left the
     // loop alone would strand the others at the next named barrier). The decision word is
@@ -287,8 +327,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     auto epilogue_next = [&](uint32_t it) -> bool {
       if (leader) {
         int go = 0;
-        if (wait_bar(&task_full[slot], slot_phase, meta, s_abort, limit, kSiteEpiTask) && ring[slot].kind != kTaskStop)
-          go = wait_bar(&acc_full[acc], acc_phase, meta, s_abort, limit, kSiteEpiAcc) ? 1 : 0;
+        if (wait_bar(&task_full[slot], slot_phase, meta, s_abort, limit, kSiteEpiTask) && ring[slot].kind != kTaskStop) {
+          const uint32_t a1 = next ^ 1u;
+          go = wait_bar(&acc_full[next], (next ? use1 : use0) & 1u, meta, s_abort, limit, kSiteEpiAcc) ? 1 : 0;
+          if (go && ring[slot].ntiles == 2)
+            go = wait_bar(&acc_full[a1], (a1 ? use1 : use0) & 1u, meta, s_abort, limit, kSiteEpiAcc) ? 1 : 0;
+        }
         s_epi_go[it & 1] = go;
       }
       named_bar_sync(1, 128);
@@ -296,13 +340,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       return true;
     };
+    // after a task: count the accumulators it used and move `next` past a single one
+    auto accs_done = [&](int ntiles) {
+      if (next) ++use1; else ++use0;
+      if (ntiles == 2) {
+        if (next) ++use0; else ++use1;
+      } else {
+        next ^= 1u;
+      }
+    };
     if constexpr (kSmall) {
       // at most 16 valid rows per tile: only the warp of TMEM lanes 0-31 has work, and the
       // valid rows are stored straight from registers (no staging, no TMA stores)
       for (uint32_t it = 0;; ++it) {
         if (!epilogue_next(it)) break;
         const Task t = ring[slot];
-        const uint32_t tacc = tmem_base + acc * kAccCols + (static_cast<uint32_t>(q * 32) << 16);
+        const uint32_t tacc = tmem_base + next * kAccCols + (static_cast<uint32_t>(q * 32) << 16);
         const bool shared = (t.expert == sh.E);
         const bool has_rows = q * 32 < t.nrows;  // warp-uniform
         const bool valid = row < t.nrows;
@@ -339,7 +392,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty[acc]);
+          if (lane == 0) mbar_arrive(&acc_empty[next]);
           // publish h: this tile's down tasks read it with TMA (async proxy) on other SMs
           fence_proxy_async_global();
           __threadfence();
@@ -381,12 +434,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty[acc]);
+          if (lane == 0) mbar_arrive(&acc_empty[next]);
         }
         if (lane == 0) mbar_arrive(&task_empty[slot]);
         if (ws.trace_cap > 0 && leader && t.id < ws.trace_cap)
           ws.trace[(size_t)t.id * 4 + 3] = (int64_t)globaltimer_ns();
-        if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+        accs_done(1);
         if (++slot == kTaskSlots) { slot = 0; slot_phase ^= 1; }
       }
     } else {
@@ -397,16 +450,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         *reinterpret_cast<uint4*>(buf + row * 128 + ((j ^ (row & 7)) << 4)) =
             make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
     };
-    for (uint32_t it = 0;; ++it) {
-      if (!epilogue_next(it)) break;
-      const Task t = ring[slot];
-      const uint32_t tacc = tmem_base + acc * kAccCols + (static_cast<uint32_t>(q * 32) << 16);
+    uint32_t sb = 0;  // staging buffer in use (the tail shape has one, the general shape two)
+    // One tile of the task: accumulator `a` holds its rows (lane = row); results go to rows
+    // tile*128 .. of h (up) or y (down).
+    auto process_tile = [&](const Task& t, int tile, int row0, int nrows, uint32_t a) {
+      const uint32_t tacc = tmem_base + a * kAccCols + (static_cast<uint32_t>(q * 32) << 16);
       const bool shared = (t.expert == sh.E);
       if (t.kind == kTaskUp) {
         // h = SiLU(U) * G, two chunks of 64 bf16 columns
 #pragma unroll 1
         for (int cc = 0; cc < kBN1 / 64; ++cc) {
-          uint8_t* buf = staging + sb * kStagingBytes;
           uint32_t pk[32];
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
@@ -423,22 +476,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                               __fdividef(u1, 1.0f + __expf(-u1)) * g1);
             }
           }
-          if (cc == kBN1 / 64 - 1) {  // every TMEM read of this task is done: release it
+          if (cc == kBN1 / 64 - 1) {  // every TMEM read of this accumulator is done: release it
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[acc]);
+            if (lane == 0) mbar_arrive(&acc_empty[a]);
           }
-          if (leader) bulk_wait_group_read<kNumStaging - 1>();  // buffer sb no longer read
+          uint8_t* buf = staging + sb * kStagingBytes;
+          if (leader) bulk_wait_group_read<C::kNumStagingN - 1>();  // buffer sb is no longer read
           named_bar_sync(1, 128);
           put_row(buf, pk);
           fence_proxy_async_shared();
           named_bar_sync(1, 128);
           if (leader) {
-            tma_store_2d(shared ? &maps.h_shared : &maps.h_routed, smem_u32(buf), t.n0 + cc * 64,
-                         t.tile * kBM);
+            tma_store_2d(shared ? &maps.h_shared : &maps.h_routed, smem_u32(buf), t.n0 + cc * 64, tile * kBM);
             bulk_commit_group();
           }
-          sb ^= 1;
+          if constexpr (C::kNumStagingN > 1) sb ^= 1;
         }
         // publish h: the stores must be complete and visible to other SMs' TMA loads before
         // the tile's counter moves
@@ -446,22 +499,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           bulk_wait_group<0>();
           fence_proxy_async_global();
           __threadfence();
-          red_release_add_gpu(&ws.done1[t.tile], 1);
+          red_release_add_gpu(&ws.done1[tile], 1);
         }
       } else {
         // y = w * (h W_down^T) rounded to bf16, four chunks of 64 columns
         float w = 0.f;
-        if (row < t.nrows) {
+        if (row < nrows) {
           if (shared) {
             w = 1.f;
           } else {
-            const int s = __ldcg(&ws.sorted_ids[t.row0 + row]);
+            const int s = __ldcg(&ws.sorted_ids[row0 + row]);
             w = __ldcg(&ws.topk_w[s]);
           }
         }
 #pragma unroll 1
         for (int cc = 0; cc < kBN2 / 64; ++cc) {
-          uint8_t* buf = staging + sb * kStagingBytes;
           uint32_t pk[32];
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
@@ -475,27 +527,34 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (cc == kBN2 / 64 - 1) {
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[acc]);
+            if (lane == 0) mbar_arrive(&acc_empty[a]);
           }
-          if (leader) bulk_wait_group_read<kNumStaging - 1>();
+          uint8_t* buf = staging + sb * kStagingBytes;
+          if (leader) bulk_wait_group_read<C::kNumStagingN - 1>();
           named_bar_sync(1, 128);
           put_row(buf, pk);
           fence_proxy_async_shared();
           named_bar_sync(1, 128);
           if (leader) {
-            tma_store_2d(&maps.y, smem_u32(buf), t.n0 + cc * 64, t.tile * kBM);
+            tma_store_2d(&maps.y, smem_u32(buf), t.n0 + cc * 64, tile * kBM);
             bulk_commit_group();
           }
-          sb ^= 1;
+          if constexpr (C::kNumStagingN > 1) sb ^= 1;
         }
       }
+    };
+    for (uint32_t it = 0;; ++it) {
+      if (!epilogue_next(it)) break;
+      const Task t = ring[slot];
+      process_tile(t, t.tile, t.row0, t.nrows, next);
+      if (kTail && t.ntiles == 2) process_tile(t, t.tile + 1, t.row0 + kBM, t.nrows2, next ^ 1u);
       if (lane == 0) mbar_arrive(&task_empty[slot]);
       if (ws.trace_cap > 0 && leader && t.id < ws.trace_cap)
         ws.trace[(size_t)t.id * 4 + 3] = (int64_t)globaltimer_ns();
-      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+      accs_done(kTail ? t.ntiles : 1);
       if (++slot == kTaskSlots) { slot = 0; slot_phase ^= 1; }
     }
-    // the staging buffers must not be released while a store still reads them
+    // the staging buffer must not be released while a store still reads it
     if (leader) bulk_wait_group<0>();
     }
   }
@@ -519,23 +578,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 1) tmem_dealloc(tmem_base, 2 * kAccCols);
 }
 
-size_t gemm_smem_bytes(bool small) { return (size_t)(small ? Cfg<true>::kBytes : Cfg<false>::kBytes) + 1024; }
+size_t gemm_smem_bytes(int shape) {
+  return (size_t)(shape == kShapeSmall ? Cfg<kShapeSmall>::kBytes
+                                       : (shape == kShapeTail ? Cfg<kShapeTail>::kBytes : Cfg<kShapeGeneral>::kBytes)) +
+         1024;
+}
 
-cudaError_t launch_moe_gemm(const GemmMaps& maps, const Workspace& ws, const Shape& sh, int grid,
-                            bool small, cudaStream_t stream) {
-  if (small)
-    return launch_k(moe_gemm_kernel<true>, dim3(grid), dim3(kGemmThreads), gemm_smem_bytes(true), stream, maps,
-                    ws, sh);
-  return launch_k(moe_gemm_kernel<false>, dim3(grid), dim3(kGemmThreads), gemm_smem_bytes(false), stream, maps,
-                  ws, sh);
+cudaError_t launch_moe_gemm(const GemmMaps& maps, const Workspace& ws, const Shape& sh, int grid, int shape,
+                            cudaStream_t stream) {
+  const size_t smem = gemm_smem_bytes(shape);
+  if (shape == kShapeSmall)
+    return launch_k(moe_gemm_kernel<kShapeSmall>, dim3(grid), dim3(kGemmThreads), smem, stream, maps, ws, sh);
+  if (shape == kShapeTail)
+    return launch_k(moe_gemm_kernel<kShapeTail>, dim3(grid), dim3(kGemmThreads), smem, stream, maps, ws, sh);
+  return launch_k(moe_gemm_kernel<kShapeGeneral>, dim3(grid), dim3(kGemmThreads), smem, stream, maps, ws, sh);
 }
 
 cudaError_t configure_gemm_kernel() {
-  cudaError_t e = cudaFuncSetAttribute(moe_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)gemm_smem_bytes(true));
+  cudaError_t e = cudaFuncSetAttribute(moe_gemm_kernel<kShapeSmall>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)gemm_smem_bytes(kShapeSmall));
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(moe_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)gemm_smem_bytes(false));
+  e = cudaFuncSetAttribute(moe_gemm_kernel<kShapeTail>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)gemm_smem_bytes(kShapeTail));
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(moe_gemm_kernel<kShapeGeneral>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)gemm_smem_bytes(kShapeGeneral));
 }
 
 }  // namespace moe

@@ -47,7 +47,8 @@ constexpr int kPMiscOff = kPRingOff + kTaskSlots * (int)sizeof(Task);
 constexpr int kPBytes = kPMiscOff + 64;
 static_assert(kPStageBytes % 1024 == 0 && kPABytes % 1024 == 0, "1024-byte aligned operand tiles");
 static_assert(kPBytes + 1024 <= 227 * 1024, "shared memory budget");
-static_assert(sizeof(Task) == 32, "task ring entries are copied as 8 words");
+static_assert(sizeof(Task) % 4 == 0, "task ring entries are copied as words");
+constexpr int kTaskWords = (int)sizeof(Task) / 4;
 
 __device__ __forceinline__ int n1_of(int expert, const Shape& sh) {
   return ceil_div(expert == sh.E ? sh.Ds : sh.D, kBN1);
@@ -81,14 +82,10 @@ __device__ __noinline__ bool wait_bar_cluster(uint64_t* bar, uint32_t parity, De
 
 __device__ __forceinline__ Task shfl_task(const Task& t) {
   Task r;
-  r.kind = __shfl_sync(0xffffffffu, t.kind, 0);
-  r.tile = __shfl_sync(0xffffffffu, t.tile, 0);
-  r.expert = __shfl_sync(0xffffffffu, t.expert, 0);
-  r.row0 = __shfl_sync(0xffffffffu, t.row0, 0);
-  r.nrows = __shfl_sync(0xffffffffu, t.nrows, 0);
-  r.n0 = __shfl_sync(0xffffffffu, t.n0, 0);
-  r.nk = __shfl_sync(0xffffffffu, t.nk, 0);
-  r.id = __shfl_sync(0xffffffffu, t.id, 0);
+  const int32_t* a = reinterpret_cast<const int32_t*>(&t);
+  int32_t* b = reinterpret_cast<int32_t*>(&r);
+#pragma unroll
+  for (int i = 0; i < kTaskWords; ++i) b[i] = __shfl_sync(0xffffffffu, a[i], 0);
   return r;
 }
 
@@ -178,7 +175,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tau = __shfl_sync(0xffffffffu, tau, 0);
         t.id = tau;
         t.kind = kTaskStop;
-        t.tile = t.expert = t.row0 = t.nrows = t.n0 = t.nk = 0;
+        t.tile = t.expert = t.row0 = t.nrows = t.n0 = t.nk = t.nrows2 = 0;
+        t.ntiles = 1;
         if (tau < total) {
           u_cur = find_unit(ws.unit_start, U, tau, u_cur);
           const TaskPos pos = decode_task(ws, sh, u_cur, tau, Mg, Mgr);
@@ -204,7 +202,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             ring[slot] = t;
             const uint32_t* w = reinterpret_cast<const uint32_t*>(&t);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) st_cluster_u32(ring_c1 + slot * (uint32_t)sizeof(Task) + 4u * i, w[i]);
+            for (int i = 0; i < kTaskWords; ++i)
+              st_cluster_u32(ring_c1 + slot * (uint32_t)sizeof(Task) + 4u * i, w[i]);
             mbar_arrive(&task_full[slot]);
             mbar_arrive_release_cluster(task_full_c1 + 8u * slot);
           }

@@ -38,7 +38,12 @@ def _layer(w, **kw):
 
 def _flags():
     from mixture_experts_layer_block_b200 import native
-    return {"pair": native.MOE_FLAG_PAIR_TILES, "single": native.MOE_FLAG_SINGLE_TILES}
+    return {"pair": native.MOE_FLAG_PAIR_TILES, "single": native.MOE_FLAG_SINGLE_TILES,
+            "general": native.MOE_FLAG_SINGLE_TILES | native.MOE_FLAG_NO_TAIL_TILES,
+            "tail": native.MOE_FLAG_SINGLE_TILES | native.MOE_FLAG_TAIL_TILES}
+
+
+SHAPE_CODE = {"general": 0, "small": 1, "tail": 2, "pair": 3}
 
 
 @pytest.mark.parametrize("name", sorted(SMALL))
@@ -53,10 +58,10 @@ def test_forward_small_all_tokens(name):
     print(name, res)
 
 
-# Both shapes of the expert GEMMs (256-row tiles on SM pairs, 128-row tiles on single SMs) on
-# every small case with more than 16 tokens: tiles of 1..256 rows, split between the two CTAs
-# of a pair at every boundary the split rule has.
-@pytest.mark.parametrize("shape", ["pair", "single"])
+# Every shape of the expert GEMMs for batches of more than 16 tokens (256-row tiles on SM
+# pairs; 128-row tiles on single SMs, with or without merged tails) on every small case: tiles
+# of 1..256 rows, split between the two CTAs of a pair at every boundary the split rule has.
+@pytest.mark.parametrize("shape", ["pair", "general", "tail"])
 @pytest.mark.parametrize("name", sorted(n for n, w in SMALL.items() if w.T > 16))
 def test_forward_small_tile_shapes(name, shape):
     w = SMALL[name]
@@ -64,6 +69,7 @@ def test_forward_small_tile_shapes(name, shape):
     layer = _layer(w, flags=_flags()[shape])
     res = check_forward(layer, w, inp)
     assert layer.query(6) == (256 if shape == "pair" else 128)
+    assert layer.query(8) == SHAPE_CODE[shape]
     res2 = check_forward(layer, w, inp)
     assert res2["out_err"] <= 1e-2
     print(name, shape, res)
@@ -85,12 +91,18 @@ def test_pair_tiles_one_expert(nrows):
 def test_tile_shape_selection():
     """Single SMs by default, SM pairs on request (when the device fits 2-CTA clusters), single
     SMs when both flags are given; batches of at most 16 tokens keep the small-tile shape."""
-    w2 = SMALL["skew_small"].replace(E=64, name="skew_small_64")
+    w2 = SMALL["skew_small"].replace(E=64, name="skew_small_64")  # 250 slots per expert
     inp2 = {k: (v.cuda() if v is not None else None) for k, v in gen.make_inputs(w2).items()}
     f = _flags()
     layer = _layer(w2)
     check_forward(layer, w2, inp2)
     assert layer.query(6) == 128 and layer.query(1) == layer.query(0)
+    assert layer.query(8) == SHAPE_CODE["tail"]  # 96..384 slots per expert: merged tails
+    wide = w2.replace(E=16, name="skew_small_16")  # 1000 slots per expert
+    inp3 = {k: (v.cuda() if v is not None else None) for k, v in gen.make_inputs(wide).items()}
+    layer = _layer(wide)
+    check_forward(layer, wide, inp3)
+    assert layer.query(8) == SHAPE_CODE["general"]
     layer = _layer(w2, flags=f["pair"])
     check_forward(layer, w2, inp2)
     assert layer.query(7) > 0 and layer.query(6) == 256 and layer.query(1) == layer.query(7)
@@ -175,3 +187,20 @@ def test_forward_bf16_out(name):
     assert torch.equal(oh, o16.cpu())
     with pytest.raises(TypeError):
         l16.forward(inp["x"], inp, o32)
+
+
+@pytest.mark.parametrize("shape", ["tail", "general"])
+@pytest.mark.parametrize("nrows", [129, 140, 160, 161, 256, 288, 289, 300, 416, 417, 513])
+def test_single_sm_merged_tails_one_expert(nrows, shape):
+    """Every token routed to expert 0 (top-1 of 2 with a large bias) and the shared expert over
+    the same tokens: runs of 128-row tiles ending in tails of 1..33+ rows. A tail of at most 32
+    rows rides in the tasks of the tile before it (an odd run starts with a single tile so the
+    tail closes a pair); a longer one keeps its own tasks."""
+    w = configs.MoEWorkload(f"tails_{nrows}", T=nrows, H=256, D=384, E=2, top_k=1, block_m=16,
+                            D_shared=128, sigma_w=0.05)
+    inp = {k: (v.cuda() if v is not None else None) for k, v in gen.make_inputs(w).items()}
+    inp["bias"] = torch.tensor([30.0, 0.0], dtype=torch.float32, device="cuda")
+    layer = _layer(w, flags=_flags()[shape])
+    check_forward(layer, w, inp)
+    assert layer.query(8) == SHAPE_CODE[shape]
+    check_forward(layer, w, inp)  # the same handle again
