@@ -43,7 +43,14 @@ KERNEL_SOURCES = ["mixture_experts_layer_block_b200/csrc/moe_gemm.cu",
                   "mixture_experts_layer_block_b200/csrc/common.cuh",
                   "mixture_experts_layer_block_b200/csrc/ptx.cuh",
                   "mixture_experts_layer_block_b200/csrc/launch.h"]
-MEASURED_TRAFFIC = {"flashmoe_prefill": ("eef3a95d38d8c053", 1.676879e9 + 0.060522e9)}
+MEASURED_TRAFFIC = {
+    "flashmoe_prefill": ("7348e6e4a3ec4c8c", 1.676500e9 + 0.061459e9, "one full-size launch"),
+    "decode": ("7348e6e4a3ec4c8c", 0.337754e9 + 0.003711e9, "one full-size launch"),
+    # full DSV3 holds 22.6 GB of weights, too large for a multi-pass capture: the T=512, E=32
+    # case of the same layer (the same per-expert load, 1/8 of the experts and tokens) scaled
+    # by the 8x more units of a full launch
+    "dsv3": ("7348e6e4a3ec4c8c", 8 * (3.041209e9 + 0.113897e9), "T=512, E=32 capture x 8"),
+}
 
 
 def kernel_source_hash() -> str:
@@ -60,6 +67,11 @@ def measured_traffic(workload: str):
     if rec is None or rec[0] != kernel_source_hash():
         return None
     return rec[1]
+
+
+def measured_traffic_note(workload: str):
+    rec = MEASURED_TRAFFIC.get(workload)
+    return rec[2] if rec is not None and rec[0] == kernel_source_hash() else None
 
 
 def load_peaks():
@@ -421,7 +433,8 @@ def run_mine(args, world, rank, local):
                 "frac": achieved / tc_peak, "peak_kind": tc_kind,
                 "timed_pass_s": timed_pass_s, "frac_of_burst_peak": achieved / peaks["bf16_tflops"]}
     traffic = args.traffic_bytes if args.traffic_bytes is not None else measured_traffic(w.name)
-    roof.update({"traffic": traffic, "kernel": "moe_gemm_kernel",
+    roof.update({"traffic": traffic, "traffic_source": measured_traffic_note(w.name) if args.traffic_bytes is None
+                 else "--traffic-bytes", "kernel": "moe_gemm_kernel",
                  "algorithmic_bytes": gbytes, "kernel_ms": gemm_ms, "peak_source": peak_src,
                  "kernel_timing": f"CUDA events around the kernel over {min(args.steps, 256)} timed forwards "
                                   "of a second pass"})
