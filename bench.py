@@ -121,8 +121,11 @@ def sm_busy_fraction(records: np.ndarray, n_ctas: int) -> dict:
 
 def tile_flags(args) -> int:
     from mixture_experts_layer_block_b200 import native
-    return {"auto": 0, "pair": native.MOE_FLAG_PAIR_TILES, "single": native.MOE_FLAG_SINGLE_TILES}[
+    f = {"auto": 0, "pair": native.MOE_FLAG_PAIR_TILES, "single": native.MOE_FLAG_SINGLE_TILES}[
         getattr(args, "tiles", "auto")]
+    if getattr(args, "sched", "dynamic") == "static":
+        f |= native.MOE_FLAG_STATIC_QUOTA
+    return f
 
 
 def traced_forward(w, wts, x, out, extra_flags=0):
@@ -316,6 +319,9 @@ def main():
     ap.add_argument("--tiles", choices=["auto", "pair", "single"], default="auto",
                     help="expert-GEMM shape: the library's choice, 256-row tiles on SM pairs, or "
                          "128-row tiles on single SMs")
+    ap.add_argument("--sched", choices=["dynamic", "static"], default="dynamic",
+                    help="task scheduling of the expert GEMMs: the atomic queue, or the static "
+                         "per-expert SM quota baseline (ablation)")
     ap.add_argument("--traffic-bytes", type=float, default=None,
                     help="ncu dram bytes per launch of the expert-GEMM kernel, if captured")
     args = ap.parse_args()
@@ -355,7 +361,8 @@ def run_mine(args, world, rank, local):
     torch.cuda.synchronize()
     rc, st = layer.status()
     assert rc == 0 and st == 0, (rc, st)
-    gemm_shape = {"tile_m": layer.query(6), "workers": layer.query(1),
+    gemm_shape = {"tile_m": layer.query(6), "workers": layer.query(1), "shape": layer.query(8),
+                  "scheduler": getattr(args, "sched", "dynamic"),
                   "kind": "SM pairs (2-CTA clusters)" if layer.query(6) == 256 else "single SMs"}
     stats = routing_stats(layer, w, dev)
 

@@ -78,6 +78,13 @@ extern "C" {
  * never (it wins). Both compute the same result. */
 #define MOE_FLAG_TAIL_TILES   64u
 #define MOE_FLAG_NO_TAIL_TILES 128u
+/* Ablation baseline, not for production (the static per-expert SM quota of a fused MoE kernel
+ * that the Weave blog, section 1.2, measures against): instead of claiming tasks from the shared
+ * counter, each persistent CTA is given a fixed share of the experts at launch — with G CTAs and
+ * X = E (+1 for the shared expert), floor(G/X) CTAs per expert and the rest idle, or with
+ * X > G the experts c, c+G, ... for CTA c — and works through only its experts' tasks.
+ * Single-SM expert GEMMs only (ignored for SM pairs). Same result, slower under skew. */
+#define MOE_FLAG_STATIC_QUOTA 256u
 
 typedef struct moe_config {
     int32_t hidden;           /* H: model dimension; multiple of 8 */

@@ -274,6 +274,7 @@ int moe_init(const moe_config* cfg, moe_handle** out) {
       {(void**)&w.group_tile0, (size_t)h->max_tiles * 4},
       {(void**)&w.group_ntiles, (size_t)h->max_tiles * 4},
       {(void**)&w.group_tasks, (size_t)h->max_tiles * 4},
+      {(void**)&w.expert_group0, (E_ + 2) * 4},
       {(void**)&w.unit_start, (size_t)(h->max_units + 1) * 4},
       {(void**)&w.done1, (size_t)h->max_tiles * 4},
       {(void**)&w.h, (size_t)h->tile_rows * ldh * 2},
@@ -438,6 +439,7 @@ static int forward_impl(moe_handle* h, const void* x, int32_t T, const void* w_r
   }
   h->last_shape = pair ? 3 : gemm_shape;
   sh.merge_tail = (gemm_shape == kShapeTail) ? 1 : 0;
+  sh.static_quota = (!pair && (c.flags & MOE_FLAG_STATIC_QUOTA)) ? 1 : 0;
   h->last_workers = workers;
   h->last_tile_m = sh.tile_m;
   sh.dep_extra = h->dep_extra_next;

@@ -119,6 +119,8 @@ struct Workspace {
   int32_t* group_tasks;  // [max_tiles]      task sets per n-tile: group_ntiles, or 1 when the
                          //                  group's last tile is a tail merged into the tasks
                          //                  of the tile before it
+  int32_t* expert_group0;  // [E + 2]        first scheduling group of each expert; [E] the
+                           //                shared expert's first group, [E + 1] all groups
   int32_t* unit_start;   // [max_groups + max_lag + 1]
   int32_t* done1;        // [max_tiles]      finished up/gate tasks per tile
   int32_t* expert_tile0; // [E]              first m-tile of each expert
@@ -143,6 +145,7 @@ struct Shape {
   int32_t tile_m;        // rows per m-tile of the expert GEMMs: 128, or 256 on SM pairs
   int32_t merge_tail;    // 1: a group of a full tile and a tail of <= kTailRows rows runs as one
                          //    task set (the one-SM general shape only)
+  int32_t static_quota;  // 1: each CTA works through a fixed share of the experts (ablation)
   int64_t timeout_ns;
 };
 
@@ -248,6 +251,47 @@ __device__ __forceinline__ TaskPos decode_task(const Workspace& ws, const Shape&
   const int o = off - n1u;
   return TaskPos{kTaskDown, td + o % gd, o / gd, gd == 1 ? nd : 1};
 }
+
+// The tasks of one "slot" (a routed expert, or E for the shared expert) in task-id order, for
+// the static per-expert quota (ablation). The slot's groups are [g0, g1); unit u holds the up
+// tasks of group u, then the down tasks of group u - lag.
+struct SlotIter {
+  int g0, g1, u, part, k;
+  __device__ void start(const Workspace& ws, int slot) {
+    g0 = __ldcg(&ws.expert_group0[slot]);
+    g1 = __ldcg(&ws.expert_group0[slot + 1]);
+    u = g0;
+    part = 0;
+    k = 0;
+  }
+  // The slot's next task id (and its unit in `unit`), or -1 when the slot has no more.
+  __device__ int next(const Workspace& ws, const Shape& sh, int Mg, int Mgr, int& unit) {
+    while (u < g1 + sh.lag) {
+      const int us = __ldcg(&ws.unit_start[u]);
+      const int n1u = (u < Mg) ? ceil_div(u < Mgr ? sh.D : sh.Ds, kBN1) * __ldcg(&ws.group_tasks[u]) : 0;
+      if (part == 0) {
+        if (u >= g0 && u < g1 && k < n1u) {
+          unit = u;
+          return us + k++;
+        }
+        part = 1;
+        k = 0;
+      }
+      const int gl = u - sh.lag;
+      if (gl >= g0 && gl < g1) {
+        const int nd = __ldcg(&ws.unit_start[u + 1]) - us - n1u;
+        if (k < nd) {
+          unit = u;
+          return us + n1u + k++;
+        }
+      }
+      ++u;
+      part = 0;
+      k = 0;
+    }
+    return -1;
+  }
+};
 
 // Wait for the last TMA fill of every stage of a ring that was filled `nfill` times in
 // round-robin order (fill f of stage s completes phase f of its `full` barrier).

@@ -257,6 +257,7 @@ __device__ void align_scans(const Workspace& ws, const Shape& sh, bool tiles, in
   for (int e = tid; e < E; e += nthr) {
     const int nt = ceil_div(kept[e], tm), first = offs[e], g0 = buf[e];
     const int last_rows = kept[e] - (nt - 1) * tm;
+    ws.expert_group0[e] = g0;
     for (int i = 0; i * kGroupTiles < nt; ++i) {
       int st, g;
       group_span(i, nt, last_rows, st, g);
@@ -270,6 +271,10 @@ __device__ void align_scans(const Workspace& ws, const Shape& sh, bool tiles, in
     put_group(Mgr + j, Mr + st, g, min(tm, sh.T - (st + g - 1) * tm));
   }
   const int Mg = Mgr + Mgs;
+  if (tid == 0) {
+    ws.expert_group0[E] = Mgr;
+    ws.expert_group0[E + 1] = Mg;
+  }
   __syncthreads();
 
   // 4. schedule units: unit u holds the up/gate tasks of group u, then the down tasks of group

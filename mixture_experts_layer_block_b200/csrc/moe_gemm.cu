@@ -147,9 +147,42 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int nk1 = ceil_div(sh.H, kBK);
     int u_cur = 0;
     uint32_t stage = 0, phase = 0, slot = 0, slot_phase = 0;
+    // Static per-expert quota (ablation): X slots (experts, plus the shared expert) over G CTAs.
+    // With G >= X each slot gets floor(G/X) CTAs, which take its tasks in turn, and the CTAs
+    // left over stay idle; with G < X, CTA c takes slots c, c+G, ... one after the other.
+    const int X = sh.E + (sh.Ds > 0 ? 1 : 0), G = (int)gridDim.x;
+    const int q = (G >= X) ? G / X : 1;
+    int sq_slot = (G >= X) ? (int)blockIdx.x / q : (int)blockIdx.x;
+    const int sq_r = (G >= X) ? (int)blockIdx.x % q : 0;
+    const int sq_stride = (G >= X) ? X : G;
+    SlotIter sq_it;
+    int sq_j = 0;
+    if (sh.static_quota && lane == 0 && sq_slot < X) sq_it.start(ws, sq_slot);
     while (true) {
-      int tau = 0;
-      if (lane == 0) tau = aborted(meta, s_abort) ? total : atomicAdd(&meta->task_counter, 1);
+      int tau = 0, unit = 0;
+      if (sh.static_quota) {
+        if (lane == 0) {
+          tau = total;  // stop unless a task of this CTA's slots remains
+          while (!aborted(meta, s_abort) && sq_slot < X) {
+            int u = 0;
+            const int cand = sq_it.next(ws, sh, Mg, Mgr, u);
+            if (cand < 0) {
+              sq_slot += sq_stride;
+              sq_j = 0;
+              if (sq_slot < X) sq_it.start(ws, sq_slot);
+              continue;
+            }
+            if (sq_j++ % q == sq_r) {
+              tau = cand;
+              unit = u;
+              break;
+            }
+          }
+        }
+        unit = __shfl_sync(0xffffffffu, unit, 0);
+      } else if (lane == 0) {
+        tau = aborted(meta, s_abort) ? total : atomicAdd(&meta->task_counter, 1);
+      }
       tau = __shfl_sync(0xffffffffu, tau, 0);
       Task t;
       t.id = tau;
@@ -158,7 +191,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (tau >= total) {
         t.kind = kTaskStop;
       } else {
-        u_cur = find_unit(ws.unit_start, U, tau, u_cur);
+        u_cur = sh.static_quota ? unit : find_unit(ws.unit_start, U, tau, u_cur);
         const TaskPos pos = decode_task(ws, sh, u_cur, tau, Mg, Mgr);
         t.kind = pos.kind;
         t.tile = pos.tile;

@@ -30,6 +30,7 @@ MOE_FLAG_SINGLE_TILES = 16
 MOE_FLAG_OUT_BF16 = 32
 MOE_FLAG_TAIL_TILES = 64
 MOE_FLAG_NO_TAIL_TILES = 128
+MOE_FLAG_STATIC_QUOTA = 256
 MOE_FLAG_TRACE = 4
 
 

@@ -204,3 +204,26 @@ def test_single_sm_merged_tails_one_expert(nrows, shape):
     check_forward(layer, w, inp)
     assert layer.query(8) == SHAPE_CODE[shape]
     check_forward(layer, w, inp)  # the same handle again
+
+
+STATIC_CASES = {
+    "tiny": SMALL["tiny"],                      # 8 experts: 18 CTAs each
+    "dsv3_small": SMALL["dsv3_small"],          # 32 experts + shared: 4 CTAs each
+    "skew_small": SMALL["skew_small"],          # 128 experts: one CTA each, 20 idle
+    "small_tokens_shared": SMALL["small_tokens_shared"],  # small-tile shape
+    "many_experts": configs.MoEWorkload("many_experts", T=200, H=256, D=128, E=300, top_k=4,
+                                        block_m=16, D_shared=128, sigma_w=0.05),  # 301 > 148 CTAs
+}
+
+
+@pytest.mark.parametrize("name", sorted(STATIC_CASES))
+def test_forward_static_quota(name):
+    """MOE_FLAG_STATIC_QUOTA (the static per-expert SM quota baseline): same results as the
+    dynamic queue, for fewer experts than CTAs, one CTA per expert and more experts than CTAs."""
+    from mixture_experts_layer_block_b200 import native
+    w = STATIC_CASES[name]
+    inp = {k: (v.cuda() if v is not None else None) for k, v in gen.make_inputs(w).items()}
+    for extra in (0, native.MOE_FLAG_TAIL_TILES):
+        layer = _layer(w, flags=native.MOE_FLAG_STATIC_QUOTA | extra)
+        check_forward(layer, w, inp)
+        check_forward(layer, w, inp)
