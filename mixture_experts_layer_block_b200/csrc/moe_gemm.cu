@@ -19,19 +19,27 @@
 //    spin), then A = the tile's h rows, B = 256 rows of W_down^e; the epilogue scales each
 //    row by its router weight and writes it (bf16) to the tile's rows of y. The combine
 //    kernel sums each token's rows in slot order in fp32.
-//  - epilogue results go through two 16 KB shared-memory staging buffers (128-byte swizzled)
+//  - epilogue results go through 16 KB shared-memory staging buffers (128-byte swizzled)
 //    and asynchronous TMA tensor stores, so the epilogue warps release TMEM and move on
 //    while the stores drain.
-//  - task ids are numbered in units: unit u = up tasks of tile u, then down tasks of tile
+//  - consecutive tiles of one expert are scheduled as groups of two whose tasks are numbered
+//    n-major (the two tasks that read the same weight rows are claimed back to back); in the
+//    tail shape a group of a full tile and a tail of at most 32 rows runs as one task set that
+//    computes both tiles from the same B stages into the two TMEM accumulators.
+//  - task ids are numbered in units: unit u = up tasks of group u, then down tasks of group
 //    u - lag. A down task's dependencies always have smaller ids, and claims are monotone,
-//    so the earliest unfinished task can always make progress (no deadlock).
+//    so the earliest unfinished task can always make progress (no deadlock). A claim finds
+//    its unit with one warp-wide round of loads.
+//  - ablation (MOE_FLAG_STATIC_QUOTA): CTAs walk a fixed share of the experts' tasks instead
+//    of claiming from the counter.
 //
-// Warp roles (192 threads, one CTA per SM): warp 0 claims tasks and issues TMA into a
-// 4-stage ring (48 KB / stage); warp 1 allocates 512 TMEM columns (two 256-column fp32
-// accumulators) and issues tcgen05.mma from one lane; warps 2-5 drain TMEM (tcgen05.ld)
-// in the epilogue. Producer -> consumers: a 4-entry task ring guarded by mbarriers.
-// Every wait is bounded (globaltimer); a wait that runs out records a status code, sets the
-// abort flag, and every CTA drains its in-flight copies and MMAs and exits.
+// Warp roles (192 threads, one CTA per SM): warp 0 claims tasks and issues TMA into the
+// operand ring (general shape 4 x 48 KB, tail shape 4 x 52 KB, small-tile shape 6 x 34 KB);
+// warp 1 allocates 512 TMEM columns (two 256-column fp32 accumulators) and issues tcgen05.mma
+// from one lane; warps 2-5 drain TMEM (tcgen05.ld) in the epilogue. Producer -> consumers: a
+// 4-entry task ring guarded by mbarriers. Every wait is bounded (globaltimer); a wait that
+// runs out records a status code, sets the abort flag, and every CTA drains its in-flight
+// copies and MMAs and exits.
 #include "launch.h"
 
 namespace moe {
