@@ -162,7 +162,16 @@ Shape make_shape(const moe_handle* h, int T, int k, int tile_m = kBM, int worker
 
 int check_cuda(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
-int router_bn(int E) { return E <= 16 ? 16 : (E <= 32 ? 32 : kRouterMaxN); }
+// Router N tile: the narrowest power of two >= E (at most kRouterMaxN, so that x is read once
+// per K split), narrowed while the m-tiles x N tiles x the deepest K split give less than half
+// a wave of CTAs (a few tokens then still spread the router weights over many SMs).
+int router_bn(int E, int T, int num_sms) {
+  int bn = 16;
+  while (bn < E && bn < kRouterMaxN) bn *= 2;
+  const int mt = ceil_div(std::max(T, 1), kBM);
+  while (bn > 16 && (int64_t)mt * ceil_div(E, bn) * kMaxRouterSplits < num_sms / 2) bn /= 2;
+  return bn;
+}
 
 int select_device(moe_handle* h) { return check_cuda(cudaSetDevice(h->device)); }
 
@@ -450,7 +459,7 @@ static int forward_impl(moe_handle* h, const void* x, int32_t T, const void* w_r
   // tensor maps
   CUtensorMap wr_map;
   GemmMaps maps;
-  const int bn = router_bn(E);
+  const int bn = router_bn(E, T, h->num_sms);
   CUtensorMap x_router;
   if ((rc = encode_map(h, &x_router, x, H, T, (uint64_t)H * 2, kBK, kBM))) return rc;
   if (small || pair) {
@@ -579,7 +588,7 @@ int moe_router_logits(moe_handle* h, const void* x, int32_t T, const void* w_rou
   int rc;
   if ((rc = select_device(h))) return rc;
   if (T == 0) return MOE_OK;
-  const int E = h->cfg.num_experts, H = h->cfg.hidden, bn = router_bn(E);
+  const int E = h->cfg.num_experts, H = h->cfg.hidden, bn = router_bn(E, T, h->num_sms);
   CUtensorMap xm, wm;
   if ((rc = encode_map(h, &xm, x, H, T, (uint64_t)H * 2, kBK, kBM))) return rc;
   if ((rc = cached_map(h, &wm, w_router, H, E, (uint64_t)H * 2, kBK, bn))) return rc;

@@ -36,14 +36,14 @@ constexpr int kPairBoxRows = 32;   // rows per A load / result store box of the 
 
 // ---- router GEMM -------------------------------------------------------------------------
 constexpr int kRouterStages = 6;
-constexpr int kRouterMaxN = 64;
+constexpr int kRouterMaxN = 256;  // one N tile covers up to 256 experts: x is read once per split
 constexpr int kMaxRouterSplits = 4;
 
 // ---- gating / align ------------------------------------------------------------------------
 constexpr int kGateThreads = 512;
 constexpr int kMaxChunks = 32;     // token chunks of the histogram (chunk = ceil(T/32) >= 64)
 constexpr int kMinChunkTokens = 64;
-constexpr int kGateTokensPerCta = 64;  // gating CTAs: 16 warps x 4 tokens
+constexpr int kGateTokensPerCta = 16;  // gating CTAs: 16 warps x 1 token
 constexpr int kMaxExperts = 1024;
 
 // ---- device status word --------------------------------------------------------------------

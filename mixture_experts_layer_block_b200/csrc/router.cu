@@ -3,7 +3,8 @@
 // Router projection of the Mixture-of-Kittens layer ("Overlapping compute and communication
 // in MoE": the router projection picks the top-k routed experts of each token). A dense
 // contraction, so it runs on the tensor cores: one CTA per 128 x BN output tile and K split
-// (blockIdx.z), TMA-fed smem ring (x tile 128 x 64, W tile BN x 64, both 128-byte swizzled),
+// (blockIdx.z), TMA-fed smem ring (x tile 128 x 64, W tile BN x 64, both 128-byte swizzled;
+// BN = 16..256, one N tile for up to 256 experts),
 // tcgen05.mma with the fp32 accumulator in TMEM, and an epilogue warpgroup that stores fp32
 // rows. With K split S ways (S = 1, 2 or 4, so that few tokens still fill the GPU) CTA z
 // writes partial z of [S][T][E] (the bias goes into partial 0); the gating kernel adds the
@@ -21,7 +22,17 @@ namespace {
 constexpr int kRThreads = 192;
 constexpr int kRABytes = kBM * kBK * 2;
 
-__device__ __forceinline__ uint32_t tmem_cols_for(int bn) { return bn <= 32 ? 32u : 64u; }
+__device__ __forceinline__ uint32_t tmem_cols_for(int bn) {
+  return bn <= 32 ? 32u : (bn <= 64 ? 64u : (bn <= 128 ? 128u : 256u));
+}
+
+// Ring depth for an N tile of BN rows: kRouterStages, or fewer so that the ring stays within
+// 192 KB of shared memory (4 stages of 48 KB at BN = 256).
+__host__ __device__ inline int router_stages(int BN) {
+  const int stage_bytes = kRABytes + ((BN * kBK * 2 + 1023) & ~1023);
+  const int fit = (192 * 1024) / stage_bytes;
+  return fit < kRouterStages ? fit : kRouterStages;
+}
 
 // 32 lanes x 16 columns
 __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
@@ -44,8 +55,9 @@ __global__ void __launch_bounds__(kRThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int b_bytes = BN * kBK * 2;
   const int stage_bytes = kRABytes + ((b_bytes + 1023) & ~1023);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kRouterStages * stage_bytes);
-  uint64_t* empty = full + kRouterStages;
+  const int nst = router_stages(BN);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + nst * stage_bytes);
+  uint64_t* empty = full + kRouterStages;  // barrier arrays sized for the deepest ring
   uint64_t* acc_full = empty + kRouterStages;
   uint64_t* drain = acc_full + 1;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
@@ -60,7 +72,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
   const uint32_t ncols = tmem_cols_for(BN);
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kRouterStages; ++i) {
+    for (int i = 0; i < nst; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
@@ -92,7 +104,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
         mbar_arrive_expect_tx(&full[stage], kRABytes + b_bytes);
         tma_load_2d(a, &x_map, &full[stage], (kb0 + kb) * kBK, m0);
         tma_load_2d(a + kRABytes, &w_map, &full[stage], (kb0 + kb) * kBK, n0);
-        if (++stage == kRouterStages) { stage = 0; phase ^= 1; }
+        if (++stage == (uint32_t)nst) { stage = 0; phase ^= 1; }
       }
     }
     __syncwarp();
@@ -111,7 +123,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
           umma_bf16(tmem, sdesc_kmajor_sw128(a + kk * 32), sdesc_kmajor_sw128(b + kk * 32), idesc,
                     (kb | kk) != 0);
         umma_commit(&empty[stage]);
-        if (++stage == kRouterStages) { stage = 0; phase ^= 1; }
+        if (++stage == (uint32_t)nst) { stage = 0; phase ^= 1; }
       }
       if (ok) umma_commit(acc_full);
     }
@@ -160,7 +172,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
   // shared memory and TMEM are released (only waits after an abort)
   tc_fence_before();
   __syncthreads();
-  if (threadIdx.x == 0) drain_fills(full, kRouterStages, nfill, meta, timeout_ns);
+  if (threadIdx.x == 0) drain_fills(full, nst, nfill, meta, timeout_ns);
   if (threadIdx.x == 32) {
     umma_commit(drain);
     wait_bar_drain(drain, 0, meta, timeout_ns);
@@ -173,7 +185,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
 size_t router_smem_bytes(int BN) {
   const int b_bytes = BN * kBK * 2;
   const int stage_bytes = kRABytes + ((b_bytes + 1023) & ~1023);
-  return (size_t)kRouterStages * stage_bytes + 1024 /*align*/ + 256 /*barriers*/;
+  return (size_t)router_stages(BN) * stage_bytes + 1024 /*align*/ + 256 /*barriers*/;
 }
 
 int router_splits(int T, int E, int H, int BN, int num_sms) {
@@ -181,7 +193,7 @@ int router_splits(int T, int E, int H, int BN, int num_sms) {
   const int nk = ceil_div(H, kBK);
   // S in {1, 2, 4}: about one wave of CTAs, and at least kRouterStages K steps per CTA
   int S = 1;
-  while (S < kMaxRouterSplits && 2 * S * tiles <= num_sms && nk / (2 * S) >= kRouterStages) S *= 2;
+  while (S < kMaxRouterSplits && 2 * S * tiles <= num_sms && nk / (2 * S) >= router_stages(BN)) S *= 2;
   return S;
 }
 
@@ -197,8 +209,9 @@ cudaError_t launch_router(const CUtensorMap& x_map, const CUtensorMap& w_map, co
 }
 
 cudaError_t configure_router_kernel() {
-  return cudaFuncSetAttribute(router_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)router_smem_bytes(kRouterMaxN));
+  size_t most = 0;
+  for (int bn = 16; bn <= kRouterMaxN; bn *= 2) most = std::max(most, router_smem_bytes(bn));
+  return cudaFuncSetAttribute(router_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)most);
 }
 
 }  // namespace moe
