@@ -44,12 +44,12 @@ KERNEL_SOURCES = ["mixture_experts_layer_block_b200/csrc/moe_gemm.cu",
                   "mixture_experts_layer_block_b200/csrc/ptx.cuh",
                   "mixture_experts_layer_block_b200/csrc/launch.h"]
 MEASURED_TRAFFIC = {
-    "flashmoe_prefill": ("7348e6e4a3ec4c8c", 1.676500e9 + 0.061459e9, "one full-size launch"),
-    "decode": ("7348e6e4a3ec4c8c", 0.337754e9 + 0.003711e9, "one full-size launch"),
+    "flashmoe_prefill": ("8e58c2e2d8dae369", 1.677245e9 + 0.061002e9, "one full-size launch"),
+    "decode": ("8e58c2e2d8dae369", 0.337762e9 + 0.004001e9, "one full-size launch"),
     # full DSV3 holds 22.6 GB of weights, too large for a multi-pass capture: the T=512, E=32
     # case of the same layer (the same per-expert load, 1/8 of the experts and tokens) scaled
     # by the 8x more units of a full launch
-    "dsv3": ("7348e6e4a3ec4c8c", 8 * (3.041209e9 + 0.113897e9), "T=512, E=32 capture x 8"),
+    "dsv3": ("8e58c2e2d8dae369", 8 * (3.063093e9 + 0.115249e9), "T=512, E=32 capture x 8"),
 }
 
 
