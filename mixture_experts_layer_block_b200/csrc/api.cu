@@ -147,12 +147,13 @@ Shape make_shape(const moe_handle* h, int T, int k, int tile_m = kBM, int worker
   sh.num_chunks = std::max(1, ceil_div(T, sh.chunk_tokens));
   sh.sorted_len = T * k + c.num_experts * (c.block_m - 1);
   sh.blocks_len = ceil_div(sh.sorted_len, c.block_m);
-  // A tile's down tasks are numbered `lag` units after its up tasks: at least two waves of
-  // tasks and one and a half waves of up tasks in between, so that a claimed down task rarely
-  // finds its tile's up tasks still running.
+  // A group's down tasks are numbered `lag` units after its up tasks: at least four waves of
+  // tasks and three waves of up tasks in between, so that a claimed down task rarely finds its
+  // tile's up tasks still running (measured: half this lag was 1% slower on the prefill layer,
+  // a quarter of it up to 16% slower on the decode layer).
   const int n1 = ceil_div(c.inter, kBN1), n2 = ceil_div(c.hidden, kBN2);
   const int W = workers > 0 ? workers : h->num_sms;  // SMs, or SM pairs
-  const int lag = std::max(ceil_div(2 * W, n1 + n2), ceil_div(3 * W, 2 * n1));
+  const int lag = std::max(ceil_div(4 * W, n1 + n2), ceil_div(3 * W, n1));
   sh.lag = std::max(1, std::min(h->max_lag, lag));
   sh.dep_extra = 0;
   sh.tile_m = tile_m;
