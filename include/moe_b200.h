@@ -154,6 +154,22 @@ MOE_API int moe_forward_host(moe_handle *h, const void *x_host, int32_t T, const
                      const void *w_down, const moe_shared_w *w_shared, int32_t top_k,
                      void *out_host, void *stream);
 
+/* moe_forward_host without the synchronisation, for a caller that feeds batches back to back:
+ * consecutive calls pipeline, so that the copy of call i+1's x to the device and the copy of
+ * call i-1's result to the host overlap call i's forward (two device staging slots, two copy
+ * streams of the handle, ordered by events; the forwards themselves run in order on `stream`).
+ * Returns once the work is queued. x_host and out_host (pinned for the copies to overlap) must
+ * stay valid and x_host unchanged until moe_forward_host_join has returned; a call's result is
+ * in out_host from then on. Needs MOE_FLAG_HOST_STAGING (else MOE_ERR_NOT_READY). */
+MOE_API int moe_forward_host_async(moe_handle *h, const void *x_host, int32_t T, const void *w_router,
+                                   const float *router_bias, const void *w_up, const void *w_gate,
+                                   const void *w_down, const moe_shared_w *w_shared, int32_t top_k,
+                                   void *out_host, void *stream);
+
+/* Makes `stream` wait for every copy back queued by moe_forward_host_async on this handle; with
+ * `block` non-zero the host also waits for them. */
+MOE_API int moe_forward_host_join(moe_handle *h, void *stream, int32_t block);
+
 /* Synchronise the handle's last stream and report the device status word:
  * *device_status = 0 when every kernel since the last call finished normally, else a
  * device error code (bit 30 set, low bits naming the wait that ran out). The word is

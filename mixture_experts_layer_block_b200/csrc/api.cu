@@ -82,8 +82,16 @@ struct moe_handle {
   cudaStream_t last_stream = nullptr;
   bool have_forward = false;
   int last_T = 0, last_k = 0, last_lag = 0;
-  void* x_stage = nullptr;
-  float* out_stage = nullptr;
+  void* x_stage = nullptr;   // [2 slots][max_tokens][H] bf16 (slot 0 for moe_forward_host)
+  float* out_stage = nullptr;  // [2 slots][max_tokens][H] fp32 or bf16
+  size_t x_slot_bytes = 0, out_slot_bytes = 0;
+  // moe_forward_host_async: copy streams and, per staging slot, the events that order the
+  // copy in, the forward and the copy back
+  cudaStream_t copy_in = nullptr, copy_out = nullptr;
+  cudaEvent_t ev_in[2] = {nullptr, nullptr}, ev_done[2] = {nullptr, nullptr}, ev_out[2] = {nullptr, nullptr};
+  bool slot_used[2] = {false, false};
+  int async_slot = 0;
+  bool async_pending = false;
   int dep_extra_next = 0;
   int64_t timeout_ns = kDefaultTimeoutNs;
 };
@@ -293,8 +301,8 @@ int moe_init(const moe_config* cfg, moe_handle** out) {
       {(void**)&w.xs, (size_t)h->routed_rows * c.hidden * 2},
       {(void**)&w.y, (size_t)h->tile_rows * c.hidden * 2},
       {(void**)&w.trace, (size_t)trace_cap * 4 * 8},
-      {(void**)&h->x_stage, (c.flags & MOE_FLAG_HOST_STAGING) ? T_ * c.hidden * 2 : 0},
-      {(void**)&h->out_stage, (c.flags & MOE_FLAG_HOST_STAGING) ? T_ * c.hidden * 4 : 0},
+      {(void**)&h->x_stage, (c.flags & MOE_FLAG_HOST_STAGING) ? 2 * T_ * c.hidden * 2 : 0},
+      {(void**)&h->out_stage, (c.flags & MOE_FLAG_HOST_STAGING) ? 2 * T_ * c.hidden * 4 : 0},
   };
   size_t total = 0;
   for (const Piece& p : pieces) total += (p.bytes + 255) & ~size_t(255);
@@ -310,6 +318,18 @@ int moe_init(const moe_config* cfg, moe_handle** out) {
   }
   w.trace_cap = trace_cap;
   w.ldh = ldh;
+  h->x_slot_bytes = T_ * c.hidden * 2;
+  h->out_slot_bytes = T_ * c.hidden * 4;
+  if (c.flags & MOE_FLAG_HOST_STAGING) {
+    if (cudaStreamCreateWithFlags(&h->copy_in, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&h->copy_out, cudaStreamNonBlocking) != cudaSuccess)
+      return fail(MOE_ERR_CUDA);
+    for (int i = 0; i < 2; ++i)
+      if (cudaEventCreateWithFlags(&h->ev_in[i], cudaEventDisableTiming) != cudaSuccess ||
+          cudaEventCreateWithFlags(&h->ev_done[i], cudaEventDisableTiming) != cudaSuccess ||
+          cudaEventCreateWithFlags(&h->ev_out[i], cudaEventDisableTiming) != cudaSuccess)
+        return fail(MOE_ERR_CUDA);
+  }
   if (cudaMemset(h->ws_mem, 0, total) != cudaSuccess) return fail(MOE_ERR_CUDA);
 
   // h tensor maps (fixed for the handle's lifetime)
@@ -379,6 +399,13 @@ void moe_destroy(moe_handle* h) {
   }
   for (auto& e : h->ev)
     if (e) cudaEventDestroy(e);
+  for (int i = 0; i < 2; ++i) {
+    if (h->ev_in[i]) cudaEventDestroy(h->ev_in[i]);
+    if (h->ev_done[i]) cudaEventDestroy(h->ev_done[i]);
+    if (h->ev_out[i]) cudaEventDestroy(h->ev_out[i]);
+  }
+  if (h->copy_in) cudaStreamDestroy(h->copy_in);
+  if (h->copy_out) cudaStreamDestroy(h->copy_out);
   if (h->ws_mem) cudaFree(h->ws_mem);
   delete h;
 }
@@ -550,6 +577,8 @@ int moe_forward_host(moe_handle* h, const void* x_host, int32_t T, const void* w
   if (!x_host || !out_host) return MOE_ERR_INVALID_ARG;
   if ((rc = select_device(h))) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // staging slot 0 may still be in use by queued asynchronous calls
+  if (h->async_pending && (rc = moe_forward_host_join(h, stream, 1))) return rc;
   const size_t xb = (size_t)T * h->cfg.hidden * 2;
   const size_t ob = (size_t)T * h->cfg.hidden * ((h->cfg.flags & MOE_FLAG_OUT_BF16) ? 2 : 4);
   if (T > 0 && cudaMemcpyAsync(h->x_stage, x_host, xb, cudaMemcpyHostToDevice, st) != cudaSuccess)
@@ -560,6 +589,59 @@ int moe_forward_host(moe_handle* h, const void* x_host, int32_t T, const void* w
   if (T > 0 && cudaMemcpyAsync(out_host, h->out_stage, ob, cudaMemcpyDeviceToHost, st) != cudaSuccess)
     return MOE_ERR_CUDA;
   return check_cuda(cudaStreamSynchronize(st));
+}
+
+int moe_forward_host_async(moe_handle* h, const void* x_host, int32_t T, const void* w_router,
+                           const float* router_bias, const void* w_up, const void* w_gate,
+                           const void* w_down, const moe_shared_w* w_shared, int32_t top_k,
+                           void* out_host, void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  if (!h->x_stage || !h->out_stage || !h->copy_in) return MOE_ERR_NOT_READY;
+  int rc;
+  if ((rc = check_tokens(h, T, top_k))) return rc;
+  if (!x_host || !out_host) return MOE_ERR_INVALID_ARG;
+  if ((rc = select_device(h))) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int s = h->async_slot;
+  h->async_slot ^= 1;
+  void* xs = static_cast<char*>(h->x_stage) + (size_t)s * h->x_slot_bytes;
+  void* os = reinterpret_cast<char*>(h->out_stage) + (size_t)s * h->out_slot_bytes;
+  const size_t xb = (size_t)T * h->cfg.hidden * 2;
+  const size_t ob = (size_t)T * h->cfg.hidden * ((h->cfg.flags & MOE_FLAG_OUT_BF16) ? 2 : 4);
+  // copy in: this slot's x buffer is free once the forward that read it two calls ago is done
+  if (h->slot_used[s] && cudaStreamWaitEvent(h->copy_in, h->ev_done[s], 0) != cudaSuccess) return MOE_ERR_CUDA;
+  if (T > 0 && cudaMemcpyAsync(xs, x_host, xb, cudaMemcpyHostToDevice, h->copy_in) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (cudaEventRecord(h->ev_in[s], h->copy_in) != cudaSuccess) return MOE_ERR_CUDA;
+  // forward on the caller's stream, once x is in and this slot's previous result is copied out
+  if (cudaStreamWaitEvent(st, h->ev_in[s], 0) != cudaSuccess) return MOE_ERR_CUDA;
+  if (h->slot_used[s] && cudaStreamWaitEvent(st, h->ev_out[s], 0) != cudaSuccess) return MOE_ERR_CUDA;
+  if ((rc = forward_impl(h, xs, T, w_router, router_bias, w_up, w_gate, w_down, w_shared, top_k, os, st)))
+    return rc;
+  if (cudaEventRecord(h->ev_done[s], st) != cudaSuccess) return MOE_ERR_CUDA;
+  // copy back
+  if (cudaStreamWaitEvent(h->copy_out, h->ev_done[s], 0) != cudaSuccess) return MOE_ERR_CUDA;
+  if (T > 0 && cudaMemcpyAsync(out_host, os, ob, cudaMemcpyDeviceToHost, h->copy_out) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (cudaEventRecord(h->ev_out[s], h->copy_out) != cudaSuccess) return MOE_ERR_CUDA;
+  h->slot_used[s] = true;
+  h->async_pending = true;
+  return MOE_OK;
+}
+
+int moe_forward_host_join(moe_handle* h, void* stream, int32_t block) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  int rc;
+  if ((rc = select_device(h))) return rc;
+  if (!h->async_pending) return MOE_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  for (int s = 0; s < 2; ++s)
+    if (h->slot_used[s] && cudaStreamWaitEvent(st, h->ev_out[s], 0) != cudaSuccess) return MOE_ERR_CUDA;
+  if (block) {
+    if (cudaStreamSynchronize(h->copy_out) != cudaSuccess) return MOE_ERR_CUDA;
+    h->async_pending = false;
+  }
+  return MOE_OK;
 }
 
 int moe_get_status(moe_handle* h, int32_t* device_status) {

@@ -56,6 +56,9 @@ SIGNATURES = {
                                    _I32, _P, _P]),
     "moe_forward_host": (ctypes.c_int, [_P, _P, _I32, _P, _P, _P, _P, _P,
                                         ctypes.POINTER(moe_shared_w), _I32, _P, _P]),
+    "moe_forward_host_async": (ctypes.c_int, [_P, _P, _I32, _P, _P, _P, _P, _P,
+                                              ctypes.POINTER(moe_shared_w), _I32, _P, _P]),
+    "moe_forward_host_join": (ctypes.c_int, [_P, _P, _I32]),
     "moe_get_status": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_int32)]),
     "moe_router_logits": (ctypes.c_int, [_P, _P, _I32, _P, _P, _P, _P]),
     "moe_gate_topk": (ctypes.c_int, [_P, _P, _I32, _I32, _P, _P, _P]),
@@ -183,6 +186,21 @@ class MoELayer:
                                    _ptr(wts["W_down"]), sh[0] if sh else None, top_k or self.cfg.top_k,
                                    _ptr(out_host), _stream(stream)), "moe_forward_host")
         return out_host
+
+    def forward_host_async(self, x_host, wts, out_host, top_k=None, stream=None):
+        """Queue a host-buffer forward; consecutive calls overlap their copies with the
+        previous forward. x_host / out_host must stay alive until forward_host_join."""
+        self._check_out(out_host)
+        sh = self._shared(wts)
+        check(lib.moe_forward_host_async(self.h, _ptr(x_host), x_host.shape[0], _ptr(wts["W_router"]),
+                                         _ptr(wts.get("bias")), _ptr(wts["W_up"]), _ptr(wts["W_gate"]),
+                                         _ptr(wts["W_down"]), sh[0] if sh else None,
+                                         top_k or self.cfg.top_k, _ptr(out_host), _stream(stream)),
+              "moe_forward_host_async")
+        return out_host
+
+    def forward_host_join(self, stream=None, block=True):
+        check(lib.moe_forward_host_join(self.h, _stream(stream), 1 if block else 0), "moe_forward_host_join")
 
     def router_logits(self, x, w_router, bias, logits, stream=None):
         check(lib.moe_router_logits(self.h, _ptr(x), x.shape[0], _ptr(w_router), _ptr(bias), _ptr(logits),

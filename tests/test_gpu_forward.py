@@ -227,3 +227,34 @@ def test_forward_static_quota(name):
         layer = _layer(w, flags=native.MOE_FLAG_STATIC_QUOTA | extra)
         check_forward(layer, w, inp)
         check_forward(layer, w, inp)
+
+
+def test_forward_host_async_pipelined():
+    """moe_forward_host_async: back-to-back calls on different batches (copies overlapping the
+    neighbouring forwards) give exactly the synchronous call's outputs; a synchronous call after
+    queued ones waits for them first."""
+    from mixture_experts_layer_block_b200 import native
+    w = SMALL["dsv3_small"]
+    inp = {k: (v.cuda() if v is not None else None) for k, v in gen.make_inputs(w).items()}
+    layer = _layer(w, flags=native.MOE_FLAG_HOST_STAGING)
+    xs = [gen.make_x(w.replace(seed=w.seed + i)).pin_memory() for i in range(5)]
+    ref = []
+    for x in xs:
+        o = torch.empty((w.T, w.H), dtype=torch.float32).pin_memory()
+        layer.forward_host(x, inp, o)
+        ref.append(o.clone())
+    outs = [torch.full((w.T, w.H), float("nan"), dtype=torch.float32).pin_memory() for _ in xs]
+    stream = torch.cuda.current_stream()
+    for x, o in zip(xs, outs):
+        layer.forward_host_async(x, inp, o, stream=stream)
+    layer.forward_host_join(stream=stream, block=True)
+    for o, r in zip(outs, ref):
+        assert torch.equal(o, r)
+    # queued calls, then a synchronous one: every result lands
+    layer.forward_host_async(xs[0], inp, outs[0], stream=stream)
+    last = torch.empty((w.T, w.H), dtype=torch.float32).pin_memory()
+    layer.forward_host(xs[1], inp, last)
+    layer.forward_host_join(block=True)
+    assert torch.equal(outs[0], ref[0]) and torch.equal(last, ref[1])
+    rc, st = layer.status()
+    assert rc == 0 and st == 0
