@@ -85,25 +85,24 @@ __global__ void __launch_bounds__(256)
     const int c0 = (int)(it % nblk) * 512 + lane * 8, c1 = c0 + 256;
     // this token's rows in y: the shared-expert row first, then its slots in order
     const int myrow = (lane < sh.k) ? __ldcg(ws.row_of_slot + (size_t)t * sh.k + lane) : -1;
-    if (c0 >= sh.H) continue;
-    const bool has1 = c1 < sh.H;
+    // every lane stays for the shuffles below; lanes past the row's end only skip memory
+    const bool has0 = c0 < sh.H, has1 = c1 < sh.H;
     float a0[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     float a1[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     if (sh.Ds > 0) {
       const uint16_t* srow = ws.y + ((size_t)Mr * sh.tile_m + t) * sh.H;
-      add_bf16x8(a0, __ldcg(reinterpret_cast<const uint4*>(srow + c0)));
+      if (has0) add_bf16x8(a0, __ldcg(reinterpret_cast<const uint4*>(srow + c0)));
       if (has1) add_bf16x8(a1, __ldcg(reinterpret_cast<const uint4*>(srow + c1)));
     }
     for (int j = 0; j < sh.k; ++j) {
       const int row = __shfl_sync(0xffffffffu, myrow, j);
-      if (row < 0) continue;
+      if (row < 0) continue;  // the same for every lane
       const uint16_t* yr = ws.y + (size_t)row * sh.H;
-      const uint4 v0 = __ldcg(reinterpret_cast<const uint4*>(yr + c0));
+      if (has0) add_bf16x8(a0, __ldcg(reinterpret_cast<const uint4*>(yr + c0)));
       if (has1) add_bf16x8(a1, __ldcg(reinterpret_cast<const uint4*>(yr + c1)));
-      add_bf16x8(a0, v0);
     }
     const size_t orow = (size_t)t * sh.H;
-    store8<kBf16>(out, orow + c0, a0);
+    if (has0) store8<kBf16>(out, orow + c0, a0);
     if (has1) store8<kBf16>(out, orow + c1, a1);
   }
 }

@@ -28,6 +28,9 @@ SMALL = {
                                                 D_shared=256),
     "small_tokens_ragged": configs.MoEWorkload("small_tokens_ragged", T=5, H=320, D=200, E=5, top_k=2,
                                                block_m=48, D_shared=136, sigma_w=0.05, capacity_factor=1.0),
+    # H = 640: a 512-column block of a row ends inside the first 256 columns of its second half
+    "h640": configs.MoEWorkload("h640", T=90, H=640, D=192, E=6, top_k=2, block_m=16, D_shared=64,
+                                sigma_w=0.05),
 }
 
 
