@@ -242,6 +242,194 @@ ORACLE_API void moe_oracle_layer(const uint16_t *x, int64_t T, int64_t H, int64_
     }
 }
 
+/* ---------------------------------------------------------------------------------------
+ * MXFP8 experts.  The pages name MXFP8 support (Mixture-of-Kittens blog, introduction and its
+ * MXFP8 section heading; FlashMoE review, "future directions": FP8 and lower precisions) but do
+ * not define the format; the reading taken is the OCP Microscaling (MX) format, MXFP8 with E4M3
+ * elements:
+ *  - a block is 32 consecutive elements along the contraction dimension; it shares one E8M0
+ *    scale X = 2^s (code s + 127, s in [-127, 127]);
+ *  - s = floor(log2(max |v|)) - 8 (8 = the exponent of E4M3's largest normal, 448 = 1.75 * 2^8),
+ *    clamped to [-127, 127]; an all-zero block takes s = -127;
+ *  - each element is v / X rounded to E4M3, to nearest with ties to even, magnitudes above 448
+ *    clamped to 448 (saturating conversion);
+ *  - the value of an element is its E4M3 value times X.
+ * In the layer, x (along H), h (along D or Ds) and every expert weight matrix (along its
+ * contraction dimension) are quantised this way; the products, SwiGLU, the router weights and
+ * the combine stay exact (double). h is quantised from its value rounded to fp32, the
+ * precision in which the GPU path takes the same decision.
+ * ------------------------------------------------------------------------------------- */
+
+/* E4M3: sign, 4 exponent bits (bias 7), 3 mantissa bits; exponent field 0 holds the
+ * subnormals m * 2^-9; S.1111.111 is NaN (there is no infinity). */
+ORACLE_API double moe_oracle_e4m3_value(uint8_t c)
+{
+    const int sgn = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m, -9);
+    else v = ldexp(1.0 + m / 8.0, e - 7);
+    return sgn ? -v : v;
+}
+
+/* Nearest E4M3 code to v, ties to the even code, |v| > 448 clamped to 448. */
+ORACLE_API uint8_t moe_oracle_e4m3_encode(double v)
+{
+    const uint8_t sgn = (v < 0 || (v == 0 && signbit(v))) ? 0x80 : 0;
+    double a = fabs(v);
+    if (a > 448.0) a = 448.0;
+    /* spacing of the representable values around a: 2^-9 below 2^-6, else 2^(floor(log2 a) - 3) */
+    int ex;
+    double q;
+    if (a < ldexp(1.0, -6)) {
+        q = ldexp(1.0, -9);
+    } else {
+        frexp(a, &ex); /* a = f * 2^ex, f in [0.5, 1): floor(log2 a) = ex - 1 */
+        q = ldexp(1.0, ex - 1 - 3);
+    }
+    const double r = a / q; /* exact: q is a power of two */
+    double n = floor(r);
+    const double frac = r - n;
+    if (frac > 0.5 || (frac == 0.5 && fmod(n, 2.0) != 0.0)) n += 1.0;
+    const double val = n * q; /* a representable magnitude (may be the next binade's first) */
+    uint8_t code;
+    if (val < ldexp(1.0, -6)) {
+        code = (uint8_t)(val / ldexp(1.0, -9)); /* subnormal: m = val / 2^-9 */
+    } else {
+        frexp(val, &ex);
+        const int e = ex - 1;                                   /* val = 2^e * (1 + m/8) */
+        const int m = (int)(ldexp(val, -e) * 8.0 - 8.0);
+        code = (uint8_t)(((e + 7) << 3) | m);
+    }
+    return (uint8_t)(sgn | code);
+}
+
+/* Quantise n values (n a multiple of 32) block by block: codes[n] and the E8M0 scale codes
+ * scales[n / 32]. */
+ORACLE_API void moe_oracle_mx_quantize(const double *v, int64_t n, uint8_t *codes, uint8_t *scales)
+{
+    for (int64_t b = 0; b < n / 32; ++b) {
+        const double *blk = v + b * 32;
+        double amax = 0.0;
+        for (int i = 0; i < 32; ++i) if (fabs(blk[i]) > amax) amax = fabs(blk[i]);
+        int s = -127;
+        if (amax > 0.0) {
+            int ex;
+            frexp(amax, &ex);
+            s = (ex - 1) - 8;
+            if (s < -127) s = -127;
+            if (s > 127) s = 127;
+        }
+        scales[b] = (uint8_t)(s + 127);
+        for (int i = 0; i < 32; ++i) codes[b * 32 + i] = moe_oracle_e4m3_encode(ldexp(blk[i], -s));
+    }
+}
+
+/* Value of element i of a quantised vector. */
+static double mx_value(const uint8_t *codes, const uint8_t *scales, int64_t i)
+{
+    return ldexp(moe_oracle_e4m3_value(codes[i]), (int)scales[i / 32] - 127);
+}
+
+/* v <- the values of its MX quantisation (n a multiple of 32); scratch: n + n/32 bytes. */
+static void mx_round_trip(double *v, int64_t n, uint8_t *scratch)
+{
+    uint8_t *codes = scratch, *scales = scratch + n;
+    moe_oracle_mx_quantize(v, n, codes, scales);
+    for (int64_t i = 0; i < n; ++i) v[i] = mx_value(codes, scales, i);
+}
+
+/* Quantise the rows of a bf16 matrix [R][K] (K a multiple of 32): codes [R][K], scale codes
+ * [R][K/32]. */
+ORACLE_API void moe_oracle_mx_quantize_bf16_rows(const uint16_t *src, int64_t R, int64_t K,
+                                                 uint8_t *codes, uint8_t *scales)
+{
+#pragma omp parallel
+    {
+        double *row = (double *)malloc(sizeof(double) * (size_t)K);
+#pragma omp for schedule(static)
+        for (int64_t r = 0; r < R; ++r) {
+            for (int64_t i = 0; i < K; ++i) row[i] = bf16_to_double(src[r * K + i]);
+            moe_oracle_mx_quantize(row, K, codes + r * K, scales + r * (K / 32));
+        }
+        free(row);
+    }
+}
+
+/* One expert FFN on one MX-quantised token row xq (values):
+ *   h = SwiGLU(Wq_up xq, Wq_gate xq), hq = MX(fp32(h)), y = Wq_down hq,
+ * with every weight row quantised along its contraction dimension. */
+static void expert_ffn_mx(const double *xq, const uint16_t *w_up, const uint16_t *w_gate,
+                          const uint16_t *w_down, int64_t H, int64_t D, double *wrow,
+                          uint8_t *scratch, double *a, double *y)
+{
+    for (int64_t d = 0; d < D; ++d) {
+        double u = 0.0, g = 0.0;
+        for (int64_t h = 0; h < H; ++h) wrow[h] = bf16_to_double(w_up[d * H + h]);
+        mx_round_trip(wrow, H, scratch);
+        for (int64_t h = 0; h < H; ++h) u += wrow[h] * xq[h];
+        for (int64_t h = 0; h < H; ++h) wrow[h] = bf16_to_double(w_gate[d * H + h]);
+        mx_round_trip(wrow, H, scratch);
+        for (int64_t h = 0; h < H; ++h) g += wrow[h] * xq[h];
+        a[d] = (double)(float)((u / (1.0 + exp(-u))) * g);
+    }
+    mx_round_trip(a, D, scratch);
+    for (int64_t h = 0; h < H; ++h) {
+        for (int64_t d = 0; d < D; ++d) wrow[d] = bf16_to_double(w_down[h * D + d]);
+        mx_round_trip(wrow, D, scratch);
+        double s = 0.0;
+        for (int64_t d = 0; d < D; ++d) s += wrow[d] * a[d];
+        y[h] = s;
+    }
+}
+
+/* moe_oracle_layer with MXFP8 experts (H, D and Ds multiples of 32). */
+ORACLE_API void moe_oracle_layer_mxfp8(const uint16_t *x, int64_t T, int64_t H, int64_t D, int64_t E,
+                                       int64_t k, const int32_t *topk_ids, const double *topk_w,
+                                       const uint8_t *kept, const uint16_t *w_up,
+                                       const uint16_t *w_gate, const uint16_t *w_down, int64_t Ds,
+                                       const uint16_t *ws_up, const uint16_t *ws_gate,
+                                       const uint16_t *ws_down, const int64_t *tokens,
+                                       int64_t n_tokens, double *out)
+{
+    (void)T; (void)E;
+    const int64_t Dmax = Ds > D ? Ds : D;
+    const int64_t W = H > Dmax ? H : Dmax;
+#pragma omp parallel
+    {
+        double *xt = (double *)malloc(sizeof(double) * (size_t)H);
+        double *a = (double *)malloc(sizeof(double) * (size_t)Dmax);
+        double *y = (double *)malloc(sizeof(double) * (size_t)H);
+        double *wrow = (double *)malloc(sizeof(double) * (size_t)W);
+        uint8_t *scratch = (uint8_t *)malloc((size_t)(W + W / 32));
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t i = 0; i < n_tokens; ++i) {
+            const int64_t t = tokens[i];
+            double *o = out + i * H;
+            for (int64_t h = 0; h < H; ++h) xt[h] = bf16_to_double(x[t * H + h]);
+            mx_round_trip(xt, H, scratch);
+            for (int64_t h = 0; h < H; ++h) o[h] = 0.0;
+            if (Ds > 0) {
+                expert_ffn_mx(xt, ws_up, ws_gate, ws_down, H, Ds, wrow, scratch, a, y);
+                for (int64_t h = 0; h < H; ++h) o[h] += y[h];
+            }
+            for (int64_t j = 0; j < k; ++j) {
+                const int64_t s = t * k + j;
+                if (!kept[s]) continue;
+                const int64_t e = topk_ids[s];
+                expert_ffn_mx(xt, w_up + e * D * H, w_gate + e * D * H, w_down + e * H * D, H, D,
+                              wrow, scratch, a, y);
+                for (int64_t h = 0; h < H; ++h) o[h] += topk_w[s] * y[h];
+            }
+        }
+        free(scratch);
+        free(wrow);
+        free(y);
+        free(a);
+        free(xt);
+    }
+}
+
 /* Threads the OpenMP loops above use (1 when built without OpenMP). */
 ORACLE_API int moe_oracle_num_threads(void)
 {

@@ -42,6 +42,16 @@ def _bind(L):
     L.moe_oracle_layer.argtypes = [_p, _i64, _i64, _i64, _i64, _i64, _p, _p, _p, _p, _p, _p,
                                    _i64, _p, _p, _p, _p, _i64, _p]
     L.moe_oracle_layer.restype = None
+    L.moe_oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+    L.moe_oracle_e4m3_value.restype = ctypes.c_double
+    L.moe_oracle_e4m3_encode.argtypes = [ctypes.c_double]
+    L.moe_oracle_e4m3_encode.restype = ctypes.c_uint8
+    L.moe_oracle_mx_quantize.argtypes = [_p, _i64, _p, _p]
+    L.moe_oracle_mx_quantize.restype = None
+    L.moe_oracle_mx_quantize_bf16_rows.argtypes = [_p, _i64, _i64, _p, _p]
+    L.moe_oracle_mx_quantize_bf16_rows.restype = None
+    L.moe_oracle_layer_mxfp8.argtypes = L.moe_oracle_layer.argtypes
+    L.moe_oracle_layer_mxfp8.restype = None
     L.moe_oracle_num_threads.argtypes = []
     L.moe_oracle_num_threads.restype = ctypes.c_int
     return L
@@ -141,9 +151,51 @@ def align(topk_ids: np.ndarray, E: int, block_m: int, cap: int = 0,
             "kept": kept.reshape(T, k).astype(bool)}
 
 
+def e4m3_value(code: int) -> float:
+    """Value of an E4M3 code (NaN for S.1111.111)."""
+    return float(lib().moe_oracle_e4m3_value(int(code)))
+
+
+def e4m3_encode(v: float) -> int:
+    """Nearest E4M3 code (ties to even, magnitudes above 448 clamped to 448)."""
+    return int(lib().moe_oracle_e4m3_encode(float(v)))
+
+
+def mx_quantize(v) -> tuple[np.ndarray, np.ndarray]:
+    """MXFP8 (E4M3, 32-element blocks, E8M0 scales) of a float64 vector whose length is a
+    multiple of 32: (codes uint8 [n], scale codes uint8 [n/32])."""
+    a = np.ascontiguousarray(np.asarray(v, dtype=np.float64).ravel())
+    assert a.size % 32 == 0
+    codes = np.empty(a.size, dtype=np.uint8)
+    scales = np.empty(a.size // 32, dtype=np.uint8)
+    lib().moe_oracle_mx_quantize(_ptr(a), a.size, _ptr(codes), _ptr(scales))
+    return codes, scales
+
+
+def mx_values(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """Values of MXFP8 data: E4M3 value of each code times 2^(scale code - 127) of its block."""
+    c = np.asarray(codes, dtype=np.uint8).ravel()
+    sc = np.repeat(np.asarray(scales, dtype=np.int64).ravel() - 127, 32)
+    ev = np.array([e4m3_value(i) for i in range(256)], dtype=np.float64)
+    return np.ldexp(ev[c], sc)
+
+
+def mx_quantize_bf16_rows(m) -> tuple[np.ndarray, np.ndarray]:
+    """MXFP8 of each row of a bf16 matrix [R][K] (K a multiple of 32): codes [R][K] and scale
+    codes [R][K/32]."""
+    b = bf16_bits(m)
+    R, K = b.shape
+    assert K % 32 == 0
+    codes = np.empty((R, K), dtype=np.uint8)
+    scales = np.empty((R, K // 32), dtype=np.uint8)
+    lib().moe_oracle_mx_quantize_bf16_rows(_ptr(b), R, K, _ptr(codes), _ptr(scales))
+    return codes, scales
+
+
 def layer(x, weights: dict, topk_ids: np.ndarray, topk_w: np.ndarray, kept: np.ndarray,
-          tokens=None) -> np.ndarray:
-    """Layer output rows (float64 [n, H]) for `tokens` (default: all)."""
+          tokens=None, mxfp8: bool = False) -> np.ndarray:
+    """Layer output rows (float64 [n, H]) for `tokens` (default: all). With `mxfp8`, x, h and
+    every expert weight are MXFP8-quantised first (moe_oracle_layer_mxfp8)."""
     xb = bf16_bits(x)
     T, H = xb.shape
     wu, wg, wd = (bf16_bits(weights[n]) for n in ("W_up", "W_gate", "W_down"))
@@ -161,19 +213,24 @@ def layer(x, weights: dict, topk_ids: np.ndarray, topk_w: np.ndarray, kept: np.n
     w = np.ascontiguousarray(topk_w, dtype=np.float64)
     kp = np.ascontiguousarray(kept, dtype=np.uint8)
     out = np.empty((tok.size, H), dtype=np.float64)
-    lib().moe_oracle_layer(_ptr(xb), T, H, D, E, k, _ptr(ids), _ptr(w), _ptr(kp), _ptr(wu), _ptr(wg),
-                           _ptr(wd), Ds, _ptr(su), _ptr(sg), _ptr(sd), _ptr(tok), tok.size, _ptr(out))
+    fn = lib().moe_oracle_layer_mxfp8 if mxfp8 else lib().moe_oracle_layer
+    if mxfp8:
+        assert H % 32 == 0 and D % 32 == 0 and Ds % 32 == 0
+    fn(_ptr(xb), T, H, D, E, k, _ptr(ids), _ptr(w), _ptr(kp), _ptr(wu), _ptr(wg), _ptr(wd), Ds, _ptr(su),
+       _ptr(sg), _ptr(sd), _ptr(tok), tok.size, _ptr(out))
     return out
 
 
-def forward(inputs: dict, top_k: int, block_m: int, capacity_factor: float = 0.0, tokens=None):
+def forward(inputs: dict, top_k: int, block_m: int, capacity_factor: float = 0.0, tokens=None,
+            mxfp8: bool = False):
     """Whole layer: router logits -> top-k softmax -> align (capacity) -> expert FFNs and the
-    weighted combine for `tokens` (default all). Returns every intermediate."""
+    weighted combine for `tokens` (default all). Returns every intermediate. With `mxfp8` the
+    expert FFNs run on MXFP8-quantised x, h and weights (the router stays bf16)."""
     logits, absdot = router_logits(inputs["x"], inputs["W_router"], inputs.get("bias"), with_absdot=True)
     T, E = logits.shape
     ids, w = topk_softmax(logits, top_k)
     cap = capacity(T, top_k, E, capacity_factor)
     al = align(ids, E, block_m, cap)
-    out = layer(inputs["x"], inputs, ids, w, al["kept"], tokens)
+    out = layer(inputs["x"], inputs, ids, w, al["kept"], tokens, mxfp8=mxfp8)
     return {"logits": logits, "absdot": absdot, "topk_ids": ids, "topk_w": w, "capacity": cap,
             **al, "out": out}

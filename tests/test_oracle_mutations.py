@@ -48,6 +48,68 @@ PIN_TESTS = [
 ]
 
 
+# planted mistakes in the MXFP8 arithmetic, checked against the pins of test_oracle_mx_pins.py
+MX_MUTANTS = {
+    "mx_ties_away_from_zero": ("if (frac > 0.5 || (frac == 0.5 && fmod(n, 2.0) != 0.0)) n += 1.0;",
+                               "if (frac >= 0.5) n += 1.0;"),
+    "mx_emax_7": ("s = (ex - 1) - 8;", "s = (ex - 1) - 7;"),
+    "mx_no_saturation": ("if (a > 448.0) a = 448.0;", "if (a > 1e300) a = 448.0;"),
+    "mx_h_not_quantised": ("    mx_round_trip(a, D, scratch);\n", "    (void)a;\n"),
+    "mx_x_not_quantised": ("mx_round_trip(xt, H, scratch);", "(void)xt;"),
+    "mx_amax_over_16": ("for (int i = 0; i < 32; ++i) if (fabs(blk[i]) > amax)",
+                        "for (int i = 0; i < 16; ++i) if (fabs(blk[i]) > amax)"),
+    "mx_scale_applied_inverted": ("moe_oracle_e4m3_encode(ldexp(blk[i], -s))",
+                                  "moe_oracle_e4m3_encode(ldexp(blk[i], s))"),
+    "mx_subnormal_step": ("if (e == 0) v = ldexp((double)m, -9);", "if (e == 0) v = ldexp((double)m, -10);"),
+    "mx_exponent_bias": ("else v = ldexp(1.0 + m / 8.0, e - 7);", "else v = ldexp(1.0 + m / 8.0, e - 8);"),
+    "mx_down_weights_not_quantised": ("        for (int64_t d = 0; d < D; ++d) wrow[d] = bf16_to_double(w_down[h * D + d]);\n        mx_round_trip(wrow, D, scratch);",
+                                      "        for (int64_t d = 0; d < D; ++d) wrow[d] = bf16_to_double(w_down[h * D + d]);"),
+}
+
+
+def _mx_pin_tests():
+    import test_oracle_mx_pins as mx
+    return [
+        lambda: mx.test_hand_worked_mx_layer(),
+        lambda: mx.test_e4m3_every_finite_code_round_trips(),
+        lambda: mx.test_e4m3_ties_go_to_the_even_code(),
+        lambda: mx.test_e4m3_saturates_at_448(),
+        lambda: mx.test_e4m3_matches_torch_float8_conversion(),
+        lambda: [mx.test_e4m3_decode_table(c, v) for c, v in ((0x01, 2.0 ** -9), (0x38, 1.0), (0x7E, 448.0))],
+        lambda: [mx.test_scale_code_is_floor_log2_amax_minus_8(j, p) for j in (-7, 0, 5) for p in (0, 31)],
+        lambda: mx.test_small_element_under_a_large_maximum(),
+        lambda: mx.test_rounding_error_bound(),
+    ]
+
+
+def _compile_and_count_failures(src, tmp_path, pin_tests):
+    mut = tmp_path / "mut.c"
+    mut.write_text(src)
+    so = tmp_path / "libmut.so"
+    subprocess.check_call(["gcc", "-O1", "-std=c99", "-fPIC", "-shared", "-fopenmp", str(mut),
+                           "-o", str(so), "-lm"])
+    failed = 0
+    oracle.use_library(str(so))
+    try:
+        for pin in pin_tests:
+            try:
+                pin()
+            except AssertionError:
+                failed += 1
+    finally:
+        oracle.use_library(None)
+    return failed
+
+
+@pytest.mark.parametrize("name", sorted(MX_MUTANTS))
+def test_planted_mx_mistake_fails_a_pin(name, tmp_path):
+    old, new = MX_MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation anchor not unique: {old}"
+    failed = _compile_and_count_failures(src.replace(old, new), tmp_path, _mx_pin_tests())
+    assert failed > 0, f"mutant {name} passed every pin"
+
+
 @pytest.mark.parametrize("name", sorted(MUTANTS))
 def test_planted_mistake_fails_a_pin(name, tmp_path):
     old, new = MUTANTS[name]
