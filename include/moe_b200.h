@@ -85,6 +85,9 @@ extern "C" {
  * X > G the experts c, c+G, ... for CTA c — and works through only its experts' tasks.
  * Single-SM expert GEMMs only (ignored for SM pairs). Same result, slower under skew. */
 #define MOE_FLAG_STATIC_QUOTA 256u
+/* Allocate the MXFP8 workspace at moe_init (x and h quantised to MXFP8, with their scales), for
+ * moe_forward_mxfp8. Needs H, D and D_shared multiples of 128 (else MOE_ERR_UNSUPPORTED). */
+#define MOE_FLAG_MXFP8        512u
 
 typedef struct moe_config {
     int32_t hidden;           /* H: model dimension; multiple of 8 */
@@ -166,6 +169,56 @@ MOE_API int moe_forward_host_async(moe_handle *h, const void *x_host, int32_t T,
                                    const void *w_down, const moe_shared_w *w_shared, int32_t top_k,
                                    void *out_host, void *stream);
 
+/* ---- MXFP8 experts ------------------------------------------------------------------------
+ * The pages name MXFP8 expert weights (Mixture-of-Kittens blog, introduction; FlashMoE review,
+ * "future directions": FP8 and lower precisions) without defining the format. It is read as the
+ * OCP Microscaling format MXFP8: E4M3 elements (exponent bias 7, largest value 448, no
+ * infinity) in blocks of 32 consecutive elements along the contraction dimension, each block
+ * with one E8M0 scale 2^(floor(log2 amax) - 8) (scale code = exponent + 127, 0 for a block of
+ * zeros); an element is v / scale rounded to nearest even and clamped to +-448.
+ * A quantised matrix [R][K] (R and K multiples of 128) is a pair of device buffers, both
+ * 16-byte aligned and owned by the caller:
+ *   q       E4M3 codes, uint8 [R][K], row-major
+ *   scales  E8M0 codes in 512-byte atoms, moe_mxfp8_scale_bytes(R, K) bytes in all: atom
+ *           (r / 128) * (K / 128) + b / 4 holds the scale of row r, block b (columns 32b ..
+ *           32b + 31) at byte (r % 32) * 16 + ((r / 32) % 4) * 4 + b % 4.
+ */
+typedef struct moe_mxfp8_mat {
+    const void *q;
+    const void *scales;
+} moe_mxfp8_mat;
+
+/* The experts of moe_forward_mxfp8, each a quantised matrix: up and gate [E*D][H] (the bf16
+ * [E][D][H] tensors viewed as [E*D][H]), down [E*H][D]; the shared expert's [D_shared][H],
+ * [D_shared][H] and [H][D_shared] (ignored when D_shared == 0). */
+typedef struct moe_mxfp8_experts {
+    moe_mxfp8_mat up, gate, down;
+    moe_mxfp8_mat shared_up, shared_gate, shared_down;
+} moe_mxfp8_experts;
+
+/* Bytes of the scale array of an [rows][cols] quantised matrix: rows * cols / 32; -1 unless
+ * both are positive multiples of 128. */
+MOE_API int64_t moe_mxfp8_scale_bytes(int64_t rows, int64_t cols);
+
+/* Quantise the device bf16 matrix src [rows][cols] to MXFP8, writing q [rows][cols] and its
+ * scales (layout above), asynchronously on `stream`. rows and cols positive multiples of 128
+ * (else MOE_ERR_UNSUPPORTED); pointers 16-byte aligned (else MOE_ERR_MISALIGNED). Any handle
+ * works (MOE_FLAG_MXFP8 is not needed); nothing is kept. */
+MOE_API int moe_quantize_mxfp8(moe_handle *h, const void *src, int64_t rows, int64_t cols, void *q,
+                               void *scales, void *stream);
+
+/* moe_forward with MXFP8 experts. The router projection and gating run on the bf16 x and
+ * W_router exactly as in moe_forward; then each token's x row is quantised to MXFP8 (blocks
+ * along H), the expert GEMMs read the quantised weights `w`, h = SwiGLU(W_up x, W_gate x) is
+ * computed in fp32 and quantised to MXFP8 (blocks along D) before the down projection, and the
+ * router-weighted rows are combined as in moe_forward (fp32 sums; `out` fp32 [T][H], or bf16
+ * with MOE_FLAG_OUT_BF16). x, w_router, router_bias, top_k, out and stream as in moe_forward.
+ * Needs MOE_FLAG_MXFP8 at moe_init (else MOE_ERR_NOT_READY). Asynchronous, no host
+ * synchronisation, no allocation. */
+MOE_API int moe_forward_mxfp8(moe_handle *h, const void *x, int32_t T, const void *w_router,
+                              const float *router_bias, const moe_mxfp8_experts *w, int32_t top_k,
+                              void *out, void *stream);
+
 /* Makes `stream` wait for every copy back queued by moe_forward_host_async on this handle; with
  * `block` non-zero the host also waits for them. */
 MOE_API int moe_forward_host_join(moe_handle *h, void *stream, int32_t block);
@@ -230,7 +283,8 @@ MOE_API int moe_stage_times(moe_handle *h, float *ms, int32_t n);
  * 3 tasks of the last forward (synchronises), 4 m-tiles of the last forward (synchronises),
  * 5 dependency lag (units) of the last forward, 6 rows per m-tile of the last forward
  * (128 or 256), 7 SM pairs the device can run at once for the pair shape (0 = none),
- * 8 expert-GEMM shape of the last forward (0 general, 1 small-tile, 2 tail, 3 SM pairs). */
+ * 8 expert-GEMM shape of the last forward (0 general, 1 small-tile, 2 tail, 3 SM pairs,
+ * 4 MXFP8). */
 MOE_API int moe_query(const moe_handle *h, int32_t which, int64_t *value);
 
 /* Per-task trace of the last forward (needs MOE_FLAG_TRACE; synchronises). Fills up to

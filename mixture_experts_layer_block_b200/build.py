@@ -17,7 +17,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmoe_b200.so")
 OBJDIR = os.path.join(PKG, "_build")
 SOURCES = ["api.cu", "router.cu", "gate_align.cu", "moe_gemm.cu", "moe_gemm_pair.cu", "combine.cu",
-           "align_noalloc.cu"]
+           "align_noalloc.cu", "mx_quant.cu", "moe_gemm_mx.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-fvisibility=hidden",

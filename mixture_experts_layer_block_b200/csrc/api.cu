@@ -12,6 +12,7 @@
 
 #include "launch.h"
 #include "moe_b200.h"
+#include "mx.cuh"
 
 namespace moe {
 cudaError_t configure_gate_kernels(size_t gate_smem, size_t scatter_smem);
@@ -33,9 +34,10 @@ struct MapKey {
   const void* ptr;
   uint64_t inner, outer, stride;
   uint32_t box0, box1;
+  int dtype;
   bool operator==(const MapKey& o) const {
     return ptr == o.ptr && inner == o.inner && outer == o.outer && stride == o.stride &&
-           box0 == o.box0 && box1 == o.box1;
+           box0 == o.box0 && box1 == o.box1 && dtype == o.dtype;
   }
 };
 
@@ -94,6 +96,9 @@ struct moe_handle {
   bool async_pending = false;
   int dep_extra_next = 0;
   int64_t timeout_ns = kDefaultTimeoutNs;
+  // MXFP8 workspace (MOE_FLAG_MXFP8): x in token order and in tile order, h, with their scales
+  MxBuffers mx{};
+  CUtensorMap mx_xs_map{}, mx_h_map{};
 };
 
 namespace {
@@ -116,15 +121,16 @@ int encode_map(moe_handle* h, CUtensorMap* out, const void* ptr, uint64_t inner,
 // Weight maps are cached by (pointer, shape, box): encoding is cheap, but caching keeps the
 // per-call host work to a lookup.
 int cached_map(moe_handle* h, CUtensorMap* out, const void* ptr, uint64_t inner, uint64_t outer,
-               uint64_t stride_bytes, uint32_t box0, uint32_t box1) {
-  const MapKey key{ptr, inner, outer, stride_bytes, box0, box1};
+               uint64_t stride_bytes, uint32_t box0, uint32_t box1,
+               CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
+  const MapKey key{ptr, inner, outer, stride_bytes, box0, box1, (int)dtype};
   for (const MapEntry& e : h->cache)
     if (e.key == key) {
       *out = e.map;
       return MOE_OK;
     }
   MapEntry e{key, {}};
-  const int rc = encode_map(h, &e.map, ptr, inner, outer, stride_bytes, box0, box1);
+  const int rc = encode_map(h, &e.map, ptr, inner, outer, stride_bytes, box0, box1, dtype);
   if (rc != MOE_OK) return rc;
   if (h->cache.size() >= kMapCacheMax) h->cache.erase(h->cache.begin());
   h->cache.push_back(e);
@@ -220,6 +226,9 @@ int moe_init(const moe_config* cfg, moe_handle** out) {
   if (sorted_len_max > (int64_t)INT32_MAX / 2) return MOE_ERR_UNSUPPORTED;
   if ((int64_t)c.num_experts * std::max(c.inter, c.hidden) > (int64_t)INT32_MAX / 2) return MOE_ERR_UNSUPPORTED;
   if ((int64_t)c.max_tokens * c.hidden > ((int64_t)1 << 40)) return MOE_ERR_UNSUPPORTED;
+  const bool mxfp8 = (c.flags & MOE_FLAG_MXFP8) != 0;
+  if (mxfp8 && (c.hidden % kMxBK != 0 || c.inter % kMxBK != 0 || c.inter_shared % kMxBK != 0))
+    return MOE_ERR_UNSUPPORTED;
 
   moe_handle* h = new (std::nothrow) moe_handle();
   if (!h) return MOE_ERR_OUT_OF_MEMORY;
@@ -274,6 +283,7 @@ int moe_init(const moe_config* cfg, moe_handle** out) {
   };
   Workspace& w = h->ws;
   const size_t T_ = (size_t)c.max_tokens, K_ = (size_t)c.top_k, E_ = (size_t)E;
+  const size_t T_pad = (size_t)ceil_div(c.max_tokens, kBM) * kBM;
   std::vector<Piece> pieces = {
       {(void**)&w.meta, sizeof(DeviceMeta)},
       {(void**)&w.logits, T_ * E_ * 4},
@@ -303,6 +313,13 @@ int moe_init(const moe_config* cfg, moe_handle** out) {
       {(void**)&w.trace, (size_t)trace_cap * 4 * 8},
       {(void**)&h->x_stage, (c.flags & MOE_FLAG_HOST_STAGING) ? 2 * T_ * c.hidden * 2 : 0},
       {(void**)&h->out_stage, (c.flags & MOE_FLAG_HOST_STAGING) ? 2 * T_ * c.hidden * 4 : 0},
+      // MXFP8: codes plus scales (1 byte per 32 elements); token rows padded to whole atoms
+      {(void**)&h->mx.xq, mxfp8 && c.inter_shared > 0 ? T_pad * c.hidden : 0},
+      {(void**)&h->mx.sf_xq, mxfp8 && c.inter_shared > 0 ? T_pad * c.hidden / kMxBlock : 0},
+      {(void**)&h->mx.xs, mxfp8 ? (size_t)h->routed_rows * c.hidden : 0},
+      {(void**)&h->mx.sf_xs, mxfp8 ? (size_t)h->routed_rows * c.hidden / kMxBlock : 0},
+      {(void**)&h->mx.h, mxfp8 ? (size_t)h->tile_rows * ldh : 0},
+      {(void**)&h->mx.sf_h, mxfp8 ? (size_t)h->tile_rows * ldh / kMxBlock : 0},
   };
   size_t total = 0;
   for (const Piece& p : pieces) total += (p.bytes + 255) & ~size_t(255);
@@ -367,6 +384,15 @@ int moe_init(const moe_config* cfg, moe_handle** out) {
     h->h_shared16 = h->h_routed16;
   }
   if ((rc = encode_map(h, &h->y_map, w.y, c.hidden, h_rows, (uint64_t)c.hidden * 2, kBK, kBM))) return fail(rc);
+  if (mxfp8) {
+    if ((rc = encode_map(h, &h->mx_xs_map, h->mx.xs, c.hidden, xs_rows, (uint64_t)c.hidden, kMxBK, kBM,
+                         CU_TENSOR_MAP_DATA_TYPE_UINT8)))
+      return fail(rc);
+    if ((rc = encode_map(h, &h->mx_h_map, h->mx.h, ldh, h_rows, (uint64_t)ldh, kMxBK, kBM,
+                         CU_TENSOR_MAP_DATA_TYPE_UINT8)))
+      return fail(rc);
+    if (check_cuda(configure_gemm_mx_kernel())) return fail(MOE_ERR_CUDA);
+  }
 
   // kernel attributes
   Shape sh = make_shape(h, c.max_tokens, c.top_k);
@@ -552,6 +578,127 @@ static int forward_impl(moe_handle* h, const void* x, int32_t T, const void* w_r
   } else {
     if ((rc = check_cuda(launch_moe_gemm(maps, w, sh, h->num_sms, gemm_shape, st)))) return rc;
   }
+  if ((rc = mark(5))) return rc;
+  if ((rc = check_cuda(launch_combine(out, (c.flags & MOE_FLAG_OUT_BF16) != 0, w, sh, st)))) return rc;
+  if ((rc = mark(6))) return rc;
+  return MOE_OK;
+}
+
+int64_t moe_mxfp8_scale_bytes(int64_t rows, int64_t cols) {
+  if (rows <= 0 || cols <= 0 || rows % kMxBK != 0 || cols % kMxBK != 0) return -1;
+  return rows * cols / kMxBlock;
+}
+
+int moe_quantize_mxfp8(moe_handle* h, const void* src, int64_t rows, int64_t cols, void* q, void* scales,
+                       void* stream) {
+  if (!h || !src || !q || !scales) return MOE_ERR_INVALID_ARG;
+  if (moe_mxfp8_scale_bytes(rows, cols) < 0 || cols > INT32_MAX) return MOE_ERR_UNSUPPORTED;
+  if (!aligned16(src) || !aligned16(q) || !aligned16(scales)) return MOE_ERR_MISALIGNED;
+  int rc;
+  if ((rc = select_device(h))) return rc;
+  // one warp per row, 8 rows per CTA, grid-stride beyond 16 CTAs per SM
+  const int grid = (int)std::min<int64_t>((rows + 7) / 8, (int64_t)16 * h->num_sms);
+  return check_cuda(launch_mx_quantize(static_cast<const uint16_t*>(src), rows, (int)cols, static_cast<uint8_t*>(q),
+                                       static_cast<uint8_t*>(scales), grid,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+int moe_forward_mxfp8(moe_handle* h, const void* x, int32_t T, const void* w_router, const float* router_bias,
+                      const moe_mxfp8_experts* wq, int32_t top_k, void* out, void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  const moe_config& c = h->cfg;
+  if (!(c.flags & MOE_FLAG_MXFP8)) return MOE_ERR_NOT_READY;
+  int rc;
+  if ((rc = check_tokens(h, T, top_k))) return rc;
+  if (!w_router || !wq || !wq->up.q || !wq->up.scales || !wq->gate.q || !wq->gate.scales || !wq->down.q ||
+      !wq->down.scales)
+    return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (!x || !out)) return MOE_ERR_INVALID_ARG;
+  const bool has_shared = c.inter_shared > 0;
+  if (has_shared && (!wq->shared_up.q || !wq->shared_up.scales || !wq->shared_gate.q || !wq->shared_gate.scales ||
+                     !wq->shared_down.q || !wq->shared_down.scales))
+    return MOE_ERR_INVALID_ARG;
+  const moe_mxfp8_mat* mats[6] = {&wq->up, &wq->gate, &wq->down, &wq->shared_up, &wq->shared_gate, &wq->shared_down};
+  for (int i = 0; i < (has_shared ? 6 : 3); ++i)
+    if (!aligned16(mats[i]->q) || !aligned16(mats[i]->scales)) return MOE_ERR_MISALIGNED;
+  if (!aligned16(x) || !aligned16(w_router) || !aligned16(out) || (router_bias && !aligned16(router_bias)))
+    return MOE_ERR_MISALIGNED;
+  if ((rc = select_device(h))) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  h->last_stream = st;
+  h->last_T = T;
+  h->last_k = top_k;
+  h->have_forward = true;
+  if (T == 0) return MOE_OK;
+
+  const int E = c.num_experts, H = c.hidden, D = c.inter, Ds = c.inter_shared;
+  Shape sh = make_shape(h, T, top_k);
+  sh.dep_extra = h->dep_extra_next;
+  h->dep_extra_next = 0;
+  h->last_shape = 4;
+  h->last_workers = h->num_sms;
+  h->last_tile_m = kBM;
+  h->last_lag = sh.lag;
+  const Workspace& w = h->ws;
+  constexpr CUtensorMapDataType kU8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+
+  CUtensorMap x_router, wr_map;
+  MxMaps maps;
+  const int bn = router_bn(E, T, h->num_sms);
+  if ((rc = encode_map(h, &x_router, x, H, T, (uint64_t)H * 2, kBK, kBM))) return rc;
+  if ((rc = cached_map(h, &wr_map, w_router, H, E, (uint64_t)H * 2, kBK, bn))) return rc;
+  maps.xs = h->mx_xs_map;
+  maps.h = h->mx_h_map;
+  maps.y = h->y_map;
+  if ((rc = cached_map(h, &maps.w_up, wq->up.q, H, (uint64_t)E * D, H, kMxBK, kBN1, kU8))) return rc;
+  if ((rc = cached_map(h, &maps.w_gate, wq->gate.q, H, (uint64_t)E * D, H, kMxBK, kBN1, kU8))) return rc;
+  if ((rc = cached_map(h, &maps.w_down, wq->down.q, D, (uint64_t)E * H, D, kMxBK, kBN2, kU8))) return rc;
+  MxBuffers mx = h->mx;
+  mx.sf_up = static_cast<const uint8_t*>(wq->up.scales);
+  mx.sf_gate = static_cast<const uint8_t*>(wq->gate.scales);
+  mx.sf_down = static_cast<const uint8_t*>(wq->down.scales);
+  if (has_shared) {
+    if ((rc = encode_map(h, &maps.x_tile, mx.xq, H, T, H, kMxBK, kBM, kU8))) return rc;
+    if ((rc = cached_map(h, &maps.ws_up, wq->shared_up.q, H, Ds, H, kMxBK, kBN1, kU8))) return rc;
+    if ((rc = cached_map(h, &maps.ws_gate, wq->shared_gate.q, H, Ds, H, kMxBK, kBN1, kU8))) return rc;
+    if ((rc = cached_map(h, &maps.ws_down, wq->shared_down.q, Ds, H, Ds, kMxBK, kBN2, kU8))) return rc;
+    mx.sfs_up = static_cast<const uint8_t*>(wq->shared_up.scales);
+    mx.sfs_gate = static_cast<const uint8_t*>(wq->shared_gate.scales);
+    mx.sfs_down = static_cast<const uint8_t*>(wq->shared_down.scales);
+  } else {
+    maps.x_tile = maps.xs;
+    maps.ws_up = maps.w_up;
+    maps.ws_gate = maps.w_gate;
+    maps.ws_down = maps.w_down;
+    mx.sfs_up = mx.sf_up;
+    mx.sfs_gate = mx.sf_gate;
+    mx.sfs_down = mx.sf_down;
+  }
+
+  cudaEvent_t* ev = nullptr;
+  if (h->timing && h->timed < kTimingRing) ev = &h->ev[(size_t)h->timed++ * (kNumStages + 1)];
+  auto mark = [&](int i) { return (ev && cudaEventRecord(ev[i], st) != cudaSuccess) ? MOE_ERR_CUDA : MOE_OK; };
+  if ((rc = mark(0))) return rc;
+  int splits = router_splits(T, E, H, bn, h->num_sms);
+  while (splits > 1 && (int64_t)splits * T > h->parts_rows) splits /= 2;
+  float* parts = splits > 1 ? w.logit_parts : w.logits;
+  if ((rc = check_cuda(launch_router(x_router, wr_map, router_bias, parts, T, E, H, bn, splits, w.meta,
+                                     h->timeout_ns, st))))
+    return rc;
+  if ((rc = mark(1))) return rc;
+  if ((rc = check_cuda(launch_gate(parts, splits, splits > 1 ? w.logits : nullptr, w.topk_ids, w.topk_w, w,
+                                   sh, true, true, h->gate_smem, st))))
+    return rc;
+  if ((rc = mark(2))) return rc;
+  if ((rc = check_cuda(launch_scatter(w.topk_ids, w.sorted_ids, w.expert_ids, nullptr, w.row_of_slot, w,
+                                      sh, 2 * h->num_sms, st))))
+    return rc;
+  if ((rc = mark(3))) return rc;
+  if ((rc = check_cuda(launch_mx_gather(static_cast<const uint16_t*>(x), w, mx, sh, has_shared,
+                                        4 * h->num_sms, st))))
+    return rc;
+  if ((rc = mark(4))) return rc;
+  if ((rc = check_cuda(launch_moe_gemm_mx(maps, w, mx, sh, h->num_sms, st)))) return rc;
   if ((rc = mark(5))) return rc;
   if ((rc = check_cuda(launch_combine(out, (c.flags & MOE_FLAG_OUT_BF16) != 0, w, sh, st)))) return rc;
   if ((rc = mark(6))) return rc;

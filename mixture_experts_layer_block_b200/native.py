@@ -31,6 +31,7 @@ MOE_FLAG_OUT_BF16 = 32
 MOE_FLAG_TAIL_TILES = 64
 MOE_FLAG_NO_TAIL_TILES = 128
 MOE_FLAG_STATIC_QUOTA = 256
+MOE_FLAG_MXFP8 = 512
 MOE_FLAG_TRACE = 4
 
 
@@ -47,6 +48,14 @@ class moe_shared_w(ctypes.Structure):
     _fields_ = [("up", ctypes.c_void_p), ("gate", ctypes.c_void_p), ("down", ctypes.c_void_p)]
 
 
+class moe_mxfp8_mat(ctypes.Structure):
+    _fields_ = [("q", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
+
+
+class moe_mxfp8_experts(ctypes.Structure):
+    _fields_ = [(n, moe_mxfp8_mat) for n in ("up", "gate", "down", "shared_up", "shared_gate", "shared_down")]
+
+
 # every symbol the header declares, with its C signature
 _P, _I32, _I64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
 SIGNATURES = {
@@ -60,6 +69,9 @@ SIGNATURES = {
                                               ctypes.POINTER(moe_shared_w), _I32, _P, _P]),
     "moe_forward_host_join": (ctypes.c_int, [_P, _P, _I32]),
     "moe_get_status": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_int32)]),
+    "moe_mxfp8_scale_bytes": (_I64, [_I64, _I64]),
+    "moe_quantize_mxfp8": (ctypes.c_int, [_P, _P, _I64, _I64, _P, _P, _P]),
+    "moe_forward_mxfp8": (ctypes.c_int, [_P, _P, _I32, _P, _P, ctypes.POINTER(moe_mxfp8_experts), _I32, _P, _P]),
     "moe_router_logits": (ctypes.c_int, [_P, _P, _I32, _P, _P, _P, _P]),
     "moe_gate_topk": (ctypes.c_int, [_P, _P, _I32, _I32, _P, _P, _P]),
     "moe_align_block_size": (ctypes.c_int, [_P, _P, _I32, _I32, _P, _P, _P, _P]),
@@ -198,6 +210,40 @@ class MoELayer:
                                          top_k or self.cfg.top_k, _ptr(out_host), _stream(stream)),
               "moe_forward_host_async")
         return out_host
+
+    # ---- MXFP8 experts ----
+    def quantize_mxfp8(self, src, stream=None):
+        """MXFP8 of a bf16 CUDA matrix [R, K] (a 3-D tensor is viewed as [-1, K]): returns
+        (codes uint8 [R, K], scales uint8 [R*K/32] in the header's atom layout)."""
+        import torch
+        m = src.reshape(-1, src.shape[-1])
+        R, K = m.shape
+        nb = lib.moe_mxfp8_scale_bytes(R, K)
+        if nb < 0:
+            raise ValueError(f"MXFP8 needs both dimensions multiples of 128, got {R}x{K}")
+        q = torch.empty(R, K, dtype=torch.uint8, device=src.device)
+        sf = torch.empty(nb, dtype=torch.uint8, device=src.device)
+        check(lib.moe_quantize_mxfp8(self.h, _ptr(m), R, K, _ptr(q), _ptr(sf), _stream(stream)),
+              "moe_quantize_mxfp8")
+        return q, sf
+
+    def quantize_experts_mxfp8(self, wts, stream=None):
+        """The quantised experts of a weight dict (keys W_up, W_gate, W_down and, with a
+        shared expert, Ws_up, Ws_gate, Ws_down) as {name: (codes, scales)}."""
+        names = ["W_up", "W_gate", "W_down"] + (["Ws_up", "Ws_gate", "Ws_down"] if wts.get("Ws_up") is not None else [])
+        return {n: self.quantize_mxfp8(wts[n], stream) for n in names}
+
+    def forward_mxfp8(self, x, w_router, bias, wq, out, top_k=None, stream=None):
+        """moe_forward_mxfp8: wq as returned by quantize_experts_mxfp8 (needs MOE_FLAG_MXFP8)."""
+        self._check_out(out)
+        mats = []
+        for n in ("W_up", "W_gate", "W_down", "Ws_up", "Ws_gate", "Ws_down"):
+            q, sf = wq.get(n, (None, None))
+            mats.append(moe_mxfp8_mat(None if q is None else q.data_ptr(), None if sf is None else sf.data_ptr()))
+        ex = moe_mxfp8_experts(*mats)
+        check(lib.moe_forward_mxfp8(self.h, _ptr(x), x.shape[0], _ptr(w_router), _ptr(bias), ctypes.byref(ex),
+                                    top_k or self.cfg.top_k, _ptr(out), _stream(stream)), "moe_forward_mxfp8")
+        return out
 
     def forward_host_join(self, stream=None, block=True):
         check(lib.moe_forward_host_join(self.h, _stream(stream), 1 if block else 0), "moe_forward_host_join")

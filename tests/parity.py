@@ -80,13 +80,20 @@ def compact_weights(inp: dict, experts: np.ndarray) -> dict:
     return out
 
 
-def check_forward(layer, w, inp: dict, tokens=None, out_tol: float = OUT_TOL, out_dtype=torch.float32):
+def check_forward(layer, w, inp: dict, tokens=None, out_tol: float = OUT_TOL, out_dtype=torch.float32,
+                  wq: dict | None = None):
     """Run the CUDA forward for workload `w` on `inp` (device tensors) and compare with the
-    oracle on `tokens` (None = all). Returns a dict of the measured errors and counts."""
+    oracle on `tokens` (None = all). With `wq` (the library's MXFP8 quantisation of the experts,
+    from layer.quantize_experts_mxfp8) the MXFP8 forward runs instead, against the oracle's
+    MXFP8 layer (which quantises the bf16 weights itself). Returns a dict of the measured errors
+    and counts."""
     dev = inp["x"].device
     T, H, k, E = w.T, w.H, w.top_k, w.E
     out = torch.empty((T, H), dtype=out_dtype, device=dev)
-    layer.forward(inp["x"], inp, out)
+    if wq is None:
+        layer.forward(inp["x"], inp, out)
+    else:
+        layer.forward_mxfp8(inp["x"], inp["W_router"], inp.get("bias"), wq, out)
     dbg = layer.debug_outputs(T, k, dev)
     torch.cuda.synchronize()
     rc, st = layer.status()
@@ -136,7 +143,8 @@ def check_forward(layer, w, inp: dict, tokens=None, out_tol: float = OUT_TOL, ou
     remap[experts] = np.arange(experts.size)
     cw = compact_weights(inp, experts)
     sub_ids = remap[ref_ids[tok]].astype(np.int32)
-    ref_out = oracle.layer(x_h[torch.as_tensor(tok)], cw, sub_ids, ref_w[tok], ref_al["kept"][tok])
+    ref_out = oracle.layer(x_h[torch.as_tensor(tok)], cw, sub_ids, ref_w[tok], ref_al["kept"][tok],
+                           mxfp8=wq is not None)
     g_out = out.float().cpu().numpy()[tok].astype(np.float64)
     out_err = rel_err(g_out, ref_out)
     assert np.all(np.isfinite(g_out))

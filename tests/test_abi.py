@@ -68,3 +68,24 @@ def test_null_arguments(native):
 def test_status_strings(native):
     for code in range(-7, 1):
         assert native.lib.moe_status_string(code)
+
+
+@pytest.mark.parametrize("bad", [dict(hidden=320), dict(inter=200), dict(inter_shared=64)])
+def test_mxfp8_init_needs_multiples_of_128_before_cuda(native, bad):
+    h = ctypes.c_void_p()
+    rc = native.lib.moe_init(ctypes.byref(_cfg(native, flags=native.MOE_FLAG_MXFP8, **bad)), ctypes.byref(h))
+    assert rc == native.MOE_ERR_UNSUPPORTED
+    assert not h.value
+
+
+def test_mxfp8_scale_bytes(native):
+    f = native.lib.moe_mxfp8_scale_bytes
+    assert f(128, 128) == 512
+    assert f(7168, 2048) == 7168 * 2048 // 32
+    for r, c in ((0, 128), (128, 0), (100, 128), (128, 96), (-128, 128)):
+        assert f(r, c) == -1
+
+
+def test_mxfp8_null_arguments(native):
+    assert native.lib.moe_forward_mxfp8(None, None, 0, None, None, None, 1, None, None) == native.MOE_ERR_INVALID_ARG
+    assert native.lib.moe_quantize_mxfp8(None, None, 128, 128, None, None, None) == native.MOE_ERR_INVALID_ARG
