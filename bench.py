@@ -87,12 +87,14 @@ def load_peaks():
 # workload arithmetic (reporting only)
 # ------------------------------------------------------------------------------------------
 
-def algorithmic_bytes_gemm(w, hit_experts: int) -> float:
-    """Bytes the expert-GEMM kernel must move at least once: the bf16 weights of the experts
-    that receive tokens, the shared expert's weights, x (bf16) and out (fp32)."""
-    b = 3.0 * hit_experts * w.D * w.H * 2
-    b += 3.0 * w.D_shared * w.H * 2
-    b += w.T * w.H * 2 + w.T * w.H * 4
+def algorithmic_bytes_gemm(w, hit_experts: int, mxfp8: bool = False) -> float:
+    """Bytes the expert-GEMM kernel must move at least once: the weights of the experts that
+    receive tokens, the shared expert's weights, x and out (fp32). Weights and x are bf16, or
+    with MXFP8 experts one byte per element plus one scale byte per 32 elements."""
+    e = (1.0 + 1.0 / 32.0) if mxfp8 else 2.0
+    b = 3.0 * hit_experts * w.D * w.H * e
+    b += 3.0 * w.D_shared * w.H * e
+    b += w.T * w.H * e + w.T * w.H * 4
     return b
 
 
@@ -128,12 +130,20 @@ def tile_flags(args) -> int:
     return f
 
 
-def traced_forward(w, wts, x, out, extra_flags=0):
+def run_forward(layer, x, wts, out, wq=None):
+    """One layer forward: bf16 experts, or MXFP8 experts when `wq` holds their quantisation."""
+    if wq is None:
+        layer.forward(x, wts, out)
+    else:
+        layer.forward_mxfp8(x, wts["W_router"], wts.get("bias"), wq, out)
+
+
+def traced_forward(w, wts, x, out, extra_flags=0, wq=None):
     """One extra forward with per-task tracing (outside the timed region)."""
     from mixture_experts_layer_block_b200.native import MOE_FLAG_TRACE, MoELayer
     layer = MoELayer.for_workload(w, flags=MOE_FLAG_TRACE | extra_flags)
     for _ in range(2):
-        layer.forward(x, wts, out)
+        run_forward(layer, x, wts, out, wq)
     torch.cuda.synchronize()
     rec = layer.trace(1 << 20)
     n_ctas = layer.query(1)
@@ -216,27 +226,27 @@ class ClockSampler:
 # CPU oracle timing (the reported baseline, and the reference arm)
 # ------------------------------------------------------------------------------------------
 
-def oracle_sample_time(w, wts_host, x_host, n_tokens):
+def oracle_sample_time(w, wts_host, x_host, n_tokens, mxfp8=False):
     from oracle import oracle
     sub = w.replace(T=n_tokens)
     inp = dict(wts_host, x=x_host[:n_tokens])
     t0 = time.perf_counter()
-    oracle.forward(inp, sub.top_k, sub.block_m, sub.capacity_factor)
+    oracle.forward(inp, sub.top_k, sub.block_m, sub.capacity_factor, mxfp8=mxfp8)
     return time.perf_counter() - t0
 
 
-def cpu_baseline(w, wts_dev, x_dev, budget_s=12.0):
+def cpu_baseline(w, wts_dev, x_dev, budget_s=12.0, mxfp8=False):
     """Time the oracle, as it stands, on the first n tokens of the batch (a smaller batch of
     the same layer), n sized for about `budget_s` of CPU work."""
     from oracle import oracle
     wts_host = {k: (v.cpu() if v is not None else None) for k, v in wts_dev.items()}
     x_host = x_dev.cpu()
-    n = min(w.T, 16)
-    dt = oracle_sample_time(w, wts_host, x_host, n)
+    n = min(w.T, 4 if mxfp8 else 16)
+    dt = oracle_sample_time(w, wts_host, x_host, n, mxfp8)
     n2 = int(min(w.T, max(n, n * budget_s / max(dt, 1e-3))))
     if n2 > n:
         n = n2
-        dt = oracle_sample_time(w, wts_host, x_host, n)
+        dt = oracle_sample_time(w, wts_host, x_host, n, mxfp8)
     return {"value": n / dt, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
             "sample": f"oracle forward (fp64 C, OpenMP) on the first {n} tokens of the {w.name} batch "
                       f"as a batch of its own ({dt:.1f} s)"}
@@ -286,16 +296,18 @@ def run_reference(args, world, rank):
     x = gen.make_x(w, "cpu")
     from oracle import oracle
     n = min(w.T, args.ref_tokens)
+    mx = getattr(args, "precision", "bf16") == "mxfp8"
     for _ in range(max(0, min(args.warmup, 1))):
-        oracle_sample_time(w, wts, x, min(n, 8))
-    times = [oracle_sample_time(w, wts, x, n) for _ in range(args.steps)]
+        oracle_sample_time(w, wts, x, min(n, 8), mx)
+    times = [oracle_sample_time(w, wts, x, n, mx) for _ in range(args.steps)]
     per_tok = float(np.mean(times)) / n
     value = 1.0 / per_tok
     ms_step = per_tok * w.T * 1e3
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": w.name, **w.describe()},
+            "data": "synthetic", "config": {"workload": w.name, **w.describe(),
+                                            "precision": getattr(args, "precision", "bf16")},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
                              "sample": f"each step: oracle forward on the first {n} tokens of the batch"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -322,6 +334,8 @@ def main():
     ap.add_argument("--sched", choices=["dynamic", "static"], default="dynamic",
                     help="task scheduling of the expert GEMMs: the atomic queue, or the static "
                          "per-expert SM quota baseline (ablation)")
+    ap.add_argument("--precision", choices=["bf16", "mxfp8"], default="bf16",
+                    help="expert weights and activations in bf16, or MXFP8 (E4M3, 32-element blocks)")
     ap.add_argument("--traffic-bytes", type=float, default=None,
                     help="ncu dram bytes per launch of the expert-GEMM kernel, if captured")
     args = ap.parse_args()
@@ -346,18 +360,22 @@ def workload_of(args):
 
 
 def run_mine(args, world, rank, local):
-    from mixture_experts_layer_block_b200.native import (MOE_FLAG_HOST_STAGING, MOE_FLAG_STAGE_TIMING,
-                                                         MoELayer)
+    from mixture_experts_layer_block_b200.native import (MOE_FLAG_HOST_STAGING, MOE_FLAG_MXFP8,
+                                                         MOE_FLAG_STAGE_TIMING, MoELayer)
     w = workload_of(args)
+    mx = args.precision == "mxfp8"
+    prec_flags = MOE_FLAG_MXFP8 if mx else 0
     dev = torch.device("cuda", local)
     wts = gen.make_weights(w, dev)
     x = gen.make_x(w.replace(seed=w.seed + 1000 * rank) if rank else w, dev)  # each replica its own tokens
     out = torch.empty((w.T, w.H), dtype=torch.float32, device=dev)
-    layer = MoELayer.for_workload(w, flags=MOE_FLAG_HOST_STAGING | tile_flags(args))
+    layer = MoELayer.for_workload(w, flags=MOE_FLAG_HOST_STAGING | prec_flags | tile_flags(args))
     stream = torch.cuda.current_stream(dev)
+    # MXFP8 experts: the weights are quantised once, before any timing (a model stores them so)
+    wq = layer.quantize_experts_mxfp8(wts) if mx else None
 
     for _ in range(args.warmup):
-        layer.forward(x, wts, out)
+        run_forward(layer, x, wts, out, wq)
     torch.cuda.synchronize()
     rc, st = layer.status()
     assert rc == 0 and st == 0, (rc, st)
@@ -373,7 +391,7 @@ def run_mine(args, world, rank, local):
     with ClockSampler(local) as clk:
         e0.record(stream)
         for _ in range(args.steps):
-            layer.forward(x, wts, out)
+            run_forward(layer, x, wts, out, wq)
         e1.record(stream)
         torch.cuda.synchronize()
     barrier(world)
@@ -392,37 +410,56 @@ def run_mine(args, world, rank, local):
     # and the final join. Also the synchronous moe_forward_host (upload, forward, download, wait).
     x_pin = x.cpu().pin_memory()
     out_pin = torch.empty((w.T, w.H), dtype=torch.float32).pin_memory()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if not mx:
+        for _ in range(3):
+            layer.forward_host(x_pin, wts, out_pin)
+        barrier(world)
+        torch.cuda.synchronize()
+        f0.record(stream)
+        for _ in range(args.e2e_steps):
+            layer.forward_host_async(x_pin, wts, out_pin, stream=stream)
+        layer.forward_host_join(stream=stream, block=False)
+        f1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(f0.elapsed_time(f1) / args.e2e_steps, world)
+    # synchronous: upload, forward, download, wait (for MXFP8 experts, which have no host-buffer
+    # entry point, the caller's own copies around moe_forward_mxfp8)
+    x_dev = torch.empty_like(x)
+
+    def host_step():
+        if mx:
+            x_dev.copy_(x_pin, non_blocking=True)
+            run_forward(layer, x_dev, wts, out, wq)
+            out_pin.copy_(out, non_blocking=True)
+            stream.synchronize()
+        else:
+            layer.forward_host(x_pin, wts, out_pin)
     for _ in range(3):
-        layer.forward_host(x_pin, wts, out_pin)
+        host_step()
     barrier(world)
     torch.cuda.synchronize()
-    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     f0.record(stream)
     for _ in range(args.e2e_steps):
-        layer.forward_host_async(x_pin, wts, out_pin, stream=stream)
-    layer.forward_host_join(stream=stream, block=False)
-    f1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(f0.elapsed_time(f1) / args.e2e_steps, world)
-    f0.record(stream)
-    for _ in range(args.e2e_steps):
-        layer.forward_host(x_pin, wts, out_pin)
+        host_step()
     f1.record(stream)
     torch.cuda.synchronize()
     e2e_sync_ms = max_over_ranks(f0.elapsed_time(f1) / args.e2e_steps, world)
+    if mx:
+        e2e_ms = e2e_sync_ms
     layer.close()
 
     # per-kernel durations: a second timed pass whose handle records CUDA events around every
     # kernel on the launching stream (events between kernels stop them from overlapping, so
     # this pass is kept apart from the headline one)
-    layer_t = MoELayer.for_workload(w, flags=MOE_FLAG_STAGE_TIMING | tile_flags(args))
+    layer_t = MoELayer.for_workload(w, flags=MOE_FLAG_STAGE_TIMING | prec_flags | tile_flags(args))
     for _ in range(3):
-        layer_t.forward(x, wts, out)
+        run_forward(layer_t, x, wts, out, wq)
     torch.cuda.synchronize()
     layer_t.stage_times()  # drop the warm-up window
     barrier(world)
     for _ in range(min(args.steps, 256)):
-        layer_t.forward(x, wts, out)
+        run_forward(layer_t, x, wts, out, wq)
     stage_ms = layer_t.stage_times()
     rc, st = layer_t.status()
     assert rc == 0 and st == 0, (rc, st)
@@ -430,7 +467,7 @@ def run_mine(args, world, rank, local):
 
     peaks, peak_src = load_peaks()
     gemm_ms = stage_ms[4]
-    gbytes = algorithmic_bytes_gemm(w, stats["hit_experts"])
+    gbytes = algorithmic_bytes_gemm(w, stats["hit_experts"], mx)
     gemm_flops = flops - 2.0 * w.T * w.H * w.E
     # The GEMM is timed inside a loop of forwards. When that loop keeps the tensor cores busy for
     # a second or more the 1 kW power cap sets the clock, and the sustained GEMM peak (a cuBLAS
@@ -438,6 +475,9 @@ def run_mine(args, world, rank, local):
     timed_pass_s = min(args.steps, 256) * ms * 1e-3
     tc_kind = "sustained" if timed_pass_s >= 1.0 else "burst"
     tc_peak = peaks["bf16_tflops_sustained"] if tc_kind == "sustained" else peaks["bf16_tflops"]
+    # MXFP8 MMAs: the measured bf16 peak times the nominal fp8 / bf16 ratio (4.5 / 2.25 PFLOP/s)
+    tc_ratio = 2.0 if mx else 1.0
+    tc_peak *= tc_ratio
     hbm_t = gbytes / (peaks["hbm_gbs"] * 1e9)
     tc_t = gemm_flops / (tc_peak * 1e12)
     if hbm_t >= tc_t:
@@ -448,19 +488,23 @@ def run_mine(args, world, rank, local):
         achieved = gemm_flops / (gemm_ms * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s",
                 "frac": achieved / tc_peak, "peak_kind": tc_kind,
-                "timed_pass_s": timed_pass_s, "frac_of_burst_peak": achieved / peaks["bf16_tflops"]}
-    traffic = args.traffic_bytes if args.traffic_bytes is not None else measured_traffic(w.name)
+                "timed_pass_s": timed_pass_s, "frac_of_burst_peak": achieved / (tc_ratio * peaks["bf16_tflops"])}
+        if mx:
+            roof["peak_dtype"] = "mxfp8: measured bf16 peak x 2 (nominal 4.5 / 2.25 PFLOP/s)"
+    traffic = args.traffic_bytes if args.traffic_bytes is not None else (None if mx else measured_traffic(w.name))
     roof.update({"traffic": traffic, "traffic_source": measured_traffic_note(w.name) if args.traffic_bytes is None
-                 else "--traffic-bytes", "kernel": "moe_gemm_kernel",
+                 else "--traffic-bytes", "kernel": "moe_gemm_mx_kernel" if mx else "moe_gemm_kernel",
                  "algorithmic_bytes": gbytes, "kernel_ms": gemm_ms, "peak_source": peak_src,
                  "kernel_timing": f"CUDA events around the kernel over {min(args.steps, 256)} timed forwards "
                                   "of a second pass"})
 
     line = {"metric": METRIC, "value": tokens_per_s, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "vs_baseline": None, "dtype": "mxfp8-e4m3 experts, bf16 router" if mx else "bf16",
+            "data": "synthetic",
             "config": {"workload": w.name, "T": w.T, "H": w.H, "D": w.D, "E": w.E, "top_k": w.top_k,
                        "block_m": w.block_m, "D_shared": w.D_shared, "capacity_factor": w.capacity_factor,
+                       "precision": args.precision,
                        "parallelism": f"replicas{world}",
                        "l2": "inputs larger than L2 (expert weights read each step exceed 126 MB)"},
             "tflops": tflops, "tflops_frac_of_bf16_peak": tflops / peaks["bf16_tflops"],
@@ -468,16 +512,19 @@ def run_mine(args, world, rank, local):
             "routing": stats, "roofline": roof,
             "e2e": {"value": world * w.T / (e2e_ms * 1e-3), "unit": UNIT,
                     "h2d_bytes_per_step": w.T * w.H * 2, "d2h_bytes_per_step": w.T * w.H * 4,
-                    "api": "moe_forward_host_async, steps pipelined (copies overlap the previous "
-                           "and next forwards), joined inside the timed region",
-                    "synchronous": {"value": world * w.T / (e2e_sync_ms * 1e-3), "api": "moe_forward_host"}},
+                    "api": ("moe_forward_mxfp8 between the caller's pinned-host copies of x and out, "
+                            "synchronised every step") if mx else
+                           ("moe_forward_host_async, steps pipelined (copies overlap the previous "
+                            "and next forwards), joined inside the timed region"),
+                    "synchronous": {"value": world * w.T / (e2e_sync_ms * 1e-3),
+                                    "api": "as above" if mx else "moe_forward_host"}},
             "gpu_launches": len(MoELayer.STAGES) * args.steps,
             "gemm_shape": gemm_shape,
             "clocks": clk.summary()}
     if not args.no_trace:
-        line["scheduler"] = traced_forward(w, wts, x, out, tile_flags(args))
+        line["scheduler"] = traced_forward(w, wts, x, out, tile_flags(args) | prec_flags, wq)
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, wts, x)
+        line["cpu_baseline"] = cpu_baseline(w, wts, x, mxfp8=mx)
     if rank == 0:
         print(json.dumps(line))
     return 0
