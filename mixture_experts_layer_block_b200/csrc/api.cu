@@ -98,7 +98,7 @@ struct moe_handle {
   int64_t timeout_ns = kDefaultTimeoutNs;
   // MXFP8 workspace (MOE_FLAG_MXFP8): x in token order and in tile order, h, with their scales
   MxBuffers mx{};
-  CUtensorMap mx_xs_map{}, mx_h_map{};
+  CUtensorMap mx_xs_map{}, mx_h_map{}, mx_xs_map32{}, mx_h_map32{};
 };
 
 namespace {
@@ -391,6 +391,12 @@ int moe_init(const moe_config* cfg, moe_handle** out) {
     if ((rc = encode_map(h, &h->mx_h_map, h->mx.h, ldh, h_rows, (uint64_t)ldh, kMxBK, kBM,
                          CU_TENSOR_MAP_DATA_TYPE_UINT8)))
       return fail(rc);
+    if ((rc = encode_map(h, &h->mx_xs_map32, h->mx.xs, c.hidden, xs_rows, (uint64_t)c.hidden, kMxBK, kPairBoxRows,
+                         CU_TENSOR_MAP_DATA_TYPE_UINT8)))
+      return fail(rc);
+    if ((rc = encode_map(h, &h->mx_h_map32, h->mx.h, ldh, h_rows, (uint64_t)ldh, kMxBK, kPairBoxRows,
+                         CU_TENSOR_MAP_DATA_TYPE_UINT8)))
+      return fail(rc);
     if (check_cuda(configure_gemm_mx_kernel())) return fail(MOE_ERR_CUDA);
   }
 
@@ -649,6 +655,8 @@ int moe_forward_mxfp8(moe_handle* h, const void* x, int32_t T, const void* w_rou
   if ((rc = cached_map(h, &wr_map, w_router, H, E, (uint64_t)H * 2, kBK, bn))) return rc;
   maps.xs = h->mx_xs_map;
   maps.h = h->mx_h_map;
+  maps.xs32 = h->mx_xs_map32;
+  maps.h32 = h->mx_h_map32;
   maps.y = h->y_map;
   if ((rc = cached_map(h, &maps.w_up, wq->up.q, H, (uint64_t)E * D, H, kMxBK, kBN1, kU8))) return rc;
   if ((rc = cached_map(h, &maps.w_gate, wq->gate.q, H, (uint64_t)E * D, H, kMxBK, kBN1, kU8))) return rc;
@@ -659,6 +667,7 @@ int moe_forward_mxfp8(moe_handle* h, const void* x, int32_t T, const void* w_rou
   mx.sf_down = static_cast<const uint8_t*>(wq->down.scales);
   if (has_shared) {
     if ((rc = encode_map(h, &maps.x_tile, mx.xq, H, T, H, kMxBK, kBM, kU8))) return rc;
+    if ((rc = encode_map(h, &maps.x_tile32, mx.xq, H, T, H, kMxBK, kPairBoxRows, kU8))) return rc;
     if ((rc = cached_map(h, &maps.ws_up, wq->shared_up.q, H, Ds, H, kMxBK, kBN1, kU8))) return rc;
     if ((rc = cached_map(h, &maps.ws_gate, wq->shared_gate.q, H, Ds, H, kMxBK, kBN1, kU8))) return rc;
     if ((rc = cached_map(h, &maps.ws_down, wq->shared_down.q, Ds, H, Ds, kMxBK, kBN2, kU8))) return rc;
@@ -667,6 +676,7 @@ int moe_forward_mxfp8(moe_handle* h, const void* x, int32_t T, const void* w_rou
     mx.sfs_down = static_cast<const uint8_t*>(wq->shared_down.scales);
   } else {
     maps.x_tile = maps.xs;
+    maps.x_tile32 = maps.xs32;
     maps.ws_up = maps.w_up;
     maps.ws_gate = maps.w_gate;
     maps.ws_down = maps.w_down;

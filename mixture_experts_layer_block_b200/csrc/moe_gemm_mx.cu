@@ -175,7 +175,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int wrow_up = shared ? t.n0 : t.expert * sh.D + t.n0;
       const int wrow_dn = shared ? t.n0 : t.expert * H + t.n0;
       const CUtensorMap* amap = up ? (shared ? &maps.x_tile : &maps.xs) : &maps.h;
+      const CUtensorMap* amap32 = up ? (shared ? &maps.x_tile32 : &maps.xs32) : &maps.h32;
       const int arow = (up && shared) ? t.row0 : t.tile * kBM;
+      // A: one 128-row box, or (tiles of at most 96 rows) only the 32-row boxes that hold the
+      // tile's rows; the rest of the A slot keeps stale rows, whose results land in accumulator
+      // rows that are never stored
+      const int nbox = (t.nrows <= 3 * kPairBoxRows) ? ceil_div(t.nrows, kPairBoxRows) : 0;
+      const uint32_t a_bytes = nbox ? (uint32_t)(nbox * kPairBoxRows * kMxBK) : (uint32_t)C::kABytes;
       // scale atoms: A's row block (128-aligned rows), B's row blocks
       const uint8_t* sfa = up ? (shared ? mx.sf_xq + mx_atom_offset(t.row0 >> 7, 0, H)
                                         : mx.sf_xs + mx_atom_offset(t.tile, 0, H))
@@ -194,7 +200,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // scales of those rows (results in columns that are never stored) are not fetched
         if (wrow_dn + kBM >= rows_dn) sfb_bytes = kSfAtomBytes;
       }
-      const uint32_t stage_tx = (uint32_t)C::kStageBytes + kSfAtomBytes + sfb_bytes;
+      const uint32_t stage_tx = a_bytes + (uint32_t)C::kBBytes + kSfAtomBytes + sfb_bytes;
       for (int kb = 0; kb < t.nk; ++kb) {
         if (lane == 0) ok = wait_bar(&empty[stage], phase ^ 1, meta, s_abort, limit, kSiteProducerEmpty);
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -204,7 +210,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint32_t b = a + C::kABytes;
           const uint32_t sf = smem_u32(smem + C::kSfOff + stage * C::kSfStageBytes);
           mbar_arrive_expect_tx(&full[stage], stage_tx);
-          tma_load_2d(a, amap, &full[stage], kb * kMxBK, arow);
+          if (nbox == 0) {
+            tma_load_2d(a, amap, &full[stage], kb * kMxBK, arow);
+          } else {
+            for (int j = 0; j < nbox; ++j)
+              tma_load_2d(a + j * kPairBoxRows * kMxBK, amap32, &full[stage], kb * kMxBK, arow + j * kPairBoxRows);
+          }
           if (up) {
             tma_load_2d(b, shared ? &maps.ws_up : &maps.w_up, &full[stage], kb * kMxBK, wrow_up);
             tma_load_2d(b + kBN1 * kMxBK, shared ? &maps.ws_gate : &maps.w_gate, &full[stage], kb * kMxBK, wrow_up);

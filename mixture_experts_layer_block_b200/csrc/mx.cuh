@@ -49,6 +49,8 @@ struct alignas(64) MxMaps {
   CUtensorMap w_down;          // [E*H][D], box {128, 256}
   CUtensorMap ws_up, ws_gate;  // [Ds][H]
   CUtensorMap ws_down;         // [H][Ds]
+  // the A operands with 32-row boxes: a tile of at most 96 rows is loaded as whole 32-row boxes
+  CUtensorMap x_tile32, xs32, h32;
 };
 
 // Quantised activations (workspace) and the weights' scale arrays.
