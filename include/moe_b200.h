@@ -213,8 +213,10 @@ MOE_API int moe_quantize_mxfp8(moe_handle *h, const void *src, int64_t rows, int
  * computed in fp32 and quantised to MXFP8 (blocks along D) before the down projection, and the
  * router-weighted rows are combined as in moe_forward (fp32 sums; `out` fp32 [T][H], or bf16
  * with MOE_FLAG_OUT_BF16). x, w_router, router_bias, top_k, out and stream as in moe_forward.
- * Needs MOE_FLAG_MXFP8 at moe_init (else MOE_ERR_NOT_READY). Asynchronous, no host
- * synchronisation, no allocation. */
+ * The expert GEMMs run on single SMs with 128-row tiles and the atomic task counter
+ * (MOE_FLAG_PAIR_TILES, MOE_FLAG_TAIL_TILES and MOE_FLAG_STATIC_QUOTA do not apply; moe_query
+ * 8 reports 4). Needs MOE_FLAG_MXFP8 at moe_init (else MOE_ERR_NOT_READY). Asynchronous, no
+ * host synchronisation, no allocation. */
 MOE_API int moe_forward_mxfp8(moe_handle *h, const void *x, int32_t T, const void *w_router,
                               const float *router_bias, const moe_mxfp8_experts *w, int32_t top_k,
                               void *out, void *stream);
