@@ -136,3 +136,30 @@ def test_forward_mxfp8_full_size_sampled(name):
     res = check_forward(layer, w, inp, tokens=sample_tokens(w.T, 12, seed=5), wq=wq)
     print(name, res)
     layer.close()
+
+
+def test_forward_mxfp8_zero_tokens_then_a_batch():
+    """An empty batch launches nothing and leaves the handle usable."""
+    w = MX_SMALL["tiny"]
+    layer, inp, wq = _setup(w)
+    out = torch.empty((0, w.H), dtype=torch.float32, device="cuda")
+    layer.forward_mxfp8(inp["x"][:0], inp["W_router"], inp.get("bias"), wq, out)
+    torch.cuda.synchronize()
+    assert layer.status() == (0, 0)
+    check_forward(layer, w, inp, wq=wq)
+    layer.close()
+
+
+def test_forward_mxfp8_is_deterministic():
+    """Every slot's row is summed in slot order: repeated forwards agree bit for bit."""
+    w = MX_SMALL["skew_small"]
+    layer, inp, wq = _setup(w)
+    outs = []
+    for _ in range(3):
+        out = torch.empty((w.T, w.H), dtype=torch.float32, device="cuda")
+        layer.forward_mxfp8(inp["x"], inp["W_router"], inp.get("bias"), wq, out)
+        outs.append(out)
+    torch.cuda.synchronize()
+    assert layer.status() == (0, 0)
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
+    layer.close()
