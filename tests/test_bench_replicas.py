@@ -68,3 +68,15 @@ def test_two_gloo_ranks():
     line = json.loads(res[0][2].strip())
     assert line["impl"] == "reference" and line["unit"] == "tokens/s" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_reference_arm_mxfp8_line():
+    """--impl reference --precision mxfp8 times the oracle's MXFP8 layer and says so."""
+    import subprocess
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--precision",
+                        "mxfp8", "--workload", "tiny", "--steps", "1", "--warmup", "0", "--ref-tokens", "4"],
+                       capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert r.returncode == 0, r.stderr
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["config"]["precision"] == "mxfp8" and line["config"]["workload"] == "tiny"
