@@ -288,6 +288,9 @@ def barrier(world: int):
         dist.barrier()
 
 
+REF_BUDGET_S = 150.0  # CPU seconds of the reference arm's timed steps, whatever --steps is
+
+
 def run_reference(args, world, rank):
     if rank != 0:
         return 0
@@ -295,10 +298,14 @@ def run_reference(args, world, rank):
     wts = gen.make_weights(w, "cpu")
     x = gen.make_x(w, "cpu")
     from oracle import oracle
-    n = min(w.T, args.ref_tokens)
     mx = getattr(args, "precision", "bf16") == "mxfp8"
-    for _ in range(max(0, min(args.warmup, 1))):
-        oracle_sample_time(w, wts, x, min(n, 8), mx)
+    # each step is a bounded sample: at most --ref-tokens tokens, and few enough that the K
+    # timed steps take about REF_BUDGET_S in all (sized from a probe that is also the warm-up)
+    n_max = min(w.T, args.ref_tokens)
+    n_probe = min(n_max, 8)
+    t_probe = oracle_sample_time(w, wts, x, n_probe, mx)
+    per_step = REF_BUDGET_S / max(args.steps, 1)
+    n = int(min(n_max, max(1, n_probe * per_step / max(t_probe, 1e-6))))
     times = [oracle_sample_time(w, wts, x, n, mx) for _ in range(args.steps)]
     per_tok = float(np.mean(times)) / n
     value = 1.0 / per_tok
