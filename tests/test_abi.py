@@ -89,3 +89,13 @@ def test_mxfp8_scale_bytes(native):
 def test_mxfp8_null_arguments(native):
     assert native.lib.moe_forward_mxfp8(None, None, 0, None, None, None, 1, None, None) == native.MOE_ERR_INVALID_ARG
     assert native.lib.moe_quantize_mxfp8(None, None, 128, 128, None, None, None) == native.MOE_ERR_INVALID_ARG
+
+
+def test_binding_constants_match_the_header(native):
+    """Every MOE_FLAG_* and MOE_ERR_* / MOE_OK value the header defines has the same value in
+    the Python binding."""
+    text = open(HEADER).read()
+    defs = dict(re.findall(r"^#define\s+(MOE_(?:FLAG|ERR)_\w+|MOE_OK)\s+(-?\d+)u?\b", text, flags=re.M))
+    assert len(defs) >= 15
+    for name, value in defs.items():
+        assert getattr(native, name) == int(value), name
