@@ -1,0 +1,58 @@
+"""The benchmark's roofline arithmetic against the per-layer figures worked out by hand for the
+workloads (useful FLOPs per kept slot 6*H*D plus router and shared expert; algorithmic bytes =
+the weights of the experts actually hit, plus x and out), so the reported fractions rest on
+checked numbers (no GPU needed)."""
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from mixture_experts_layer_block_b200 import configs  # noqa: E402
+
+
+def test_prefill_figures():
+    w = configs.FLASHMOE_PREFILL
+    kept = w.T * w.top_k  # the upper bound: no slot dropped by the capacity limit
+    flops = configs.useful_flops(w, kept)
+    assert flops - 2.0 * w.T * w.H * w.E == pytest.approx(206.2e9, rel=1e-3)
+    assert 2.0 * w.T * w.H * w.E == pytest.approx(1.07e9, rel=1e-2)
+    weights = 3.0 * w.E * w.D * w.H * 2
+    assert weights == pytest.approx(1.611e9, rel=1e-3)
+    assert bench.algorithmic_bytes_gemm(w, w.E) == pytest.approx(weights + w.T * w.H * 6, rel=1e-12)
+
+
+def test_dsv3_figures():
+    w = configs.DSV3
+    flops = configs.useful_flops(w, w.T * w.top_k)
+    routed = 6.0 * w.T * w.top_k * w.H * w.D
+    shared = 6.0 * w.T * w.H * w.D_shared
+    assert routed == pytest.approx(2.886e12, rel=1e-3)
+    assert shared == pytest.approx(0.361e12, rel=1e-3)
+    assert flops == pytest.approx(2.886e12 + 0.361e12 + 0.015e12, rel=2e-3)
+    per_expert = 3.0 * w.D * w.H * 2
+    assert per_expert == pytest.approx(88.08e6, rel=1e-3)
+    b = bench.algorithmic_bytes_gemm(w, w.E)
+    assert b - w.T * w.H * 6 == pytest.approx(257 * per_expert, rel=1e-12)
+    assert 257 * per_expert == pytest.approx(22.64e9, rel=1e-3)
+
+
+def test_mxfp8_bytes_are_one_byte_plus_a_scale_per_32():
+    w = configs.FLASHMOE_PREFILL
+    b16 = bench.algorithmic_bytes_gemm(w, 10)
+    b8 = bench.algorithmic_bytes_gemm(w, 10, mxfp8=True)
+    out = w.T * w.H * 4
+    assert (b8 - out) == pytest.approx((b16 - out) * (1 + 1 / 32) / 2, rel=1e-12)
+
+
+def test_skew_is_tensor_bound_and_prefill_hbm_bound():
+    peaks = {"hbm_gbs": 6459.3, "bf16_tflops": 1653.5}
+    for name, bound in (("skew", "tensor"), ("flashmoe_prefill", "hbm"), ("dsv3", "hbm")):
+        w = configs.WORKLOADS[name]
+        flops = configs.useful_flops(w, w.T * w.top_k) - 2.0 * w.T * w.H * w.E
+        t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+        t_hbm = bench.algorithmic_bytes_gemm(w, w.E) / (peaks["hbm_gbs"] * 1e9)
+        assert (t_tc > t_hbm) == (bound == "tensor"), name
