@@ -314,10 +314,12 @@ MOE_API int moe_debug_inject_stall(moe_handle *h, int32_t extra);
  *   num_post_padded device int32 [1]
  * Outputs are those of moe_align_block_size for the same arguments. The first call on each
  * device looks up the array's device address and the SM count on the calling thread's current
- * device; make that first call before any stream capture. Every call uses the same array:
- * each call clears what it needs, but calls whose work overlaps on the GPU (different streams,
- * or different host threads without ordering) race on it and must be serialised by the
- * caller. */
+ * device; make that first call before any stream capture. The look-up is repeated, on the next
+ * call, when the device's context has changed since (after a cudaDeviceReset). Every call uses
+ * the same array: each call clears what it needs, but calls whose work overlaps on the GPU
+ * (different streams, or different host threads without ordering) race on it and must be
+ * serialised by the caller. T = 0 is allowed (topk_ids may then be NULL): every sorted_ids
+ * entry is the sentinel 0, every expert_ids entry -1, and num_post_padded 0. */
 MOE_API int moe_align_block_size_noalloc(const int32_t *topk_ids, int32_t T, int32_t top_k,
                                          int32_t num_experts, int32_t block_m,
                                          float capacity_factor, int32_t *sorted_ids,

@@ -12,6 +12,7 @@
 //
 // Limits: num_experts <= 256 and T * top_k <= 131072 (the array holds 32 chunk histograms of
 // 256 experts); larger sizes are rejected with MOE_ERR_UNSUPPORTED.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -39,26 +40,64 @@ static __device__ __align__(256) int32_t g_align_scratch[kNaScratchInts];
 constexpr int kNaMaxDevices = 64;
 struct DeviceSetup {
   bool ready = false;
-  int32_t* scratch = nullptr;  // device address of g_align_scratch on this device
+  unsigned long long ctx_id = 0;  // the device context the address below belongs to
+  int32_t* scratch = nullptr;     // device address of g_align_scratch in that context
   int num_sms = 0;
 };
 DeviceSetup g_setup[kNaMaxDevices];
 std::mutex g_setup_mu;
 
-// Once per device, with that device current: the array's device address. The name of the
-// array in host code is only a host-side stand-in, never a device pointer.
+// Driver entry points (through the runtime, so no link-time dependency on libcuda) that name
+// the calling thread's current context. A cudaDeviceReset destroys the context whose address
+// was cached; the next context of the same device gets a new id, which triggers a new set-up.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+CtxGetCurrentFn g_ctx_get_current = nullptr;
+CtxGetIdFn g_ctx_get_id = nullptr;
+
+// Id of the current context, 0 when the runtime has not made one current yet.
+int current_ctx_id(unsigned long long* id) {
+  *id = 0;
+  if (!g_ctx_get_current || !g_ctx_get_id) {
+    void* f1 = nullptr;
+    void* f2 = nullptr;
+    cudaDriverEntryPointQueryResult q1{}, q2{};
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1) != cudaSuccess ||
+        q1 != cudaDriverEntryPointSuccess || !f1 ||
+        cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2) != cudaSuccess ||
+        q2 != cudaDriverEntryPointSuccess || !f2)
+      return MOE_ERR_CUDA;
+    g_ctx_get_current = reinterpret_cast<CtxGetCurrentFn>(f1);
+    g_ctx_get_id = reinterpret_cast<CtxGetIdFn>(f2);
+  }
+  CUcontext ctx = nullptr;
+  if (g_ctx_get_current(&ctx) != CUDA_SUCCESS) return MOE_ERR_CUDA;
+  if (ctx && g_ctx_get_id(ctx, id) != CUDA_SUCCESS) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+// Once per device context, with that device current: the array's device address (the name of
+// the array in host code is only a host-side stand-in, never a device pointer) and the SM
+// count. Done again when the device's context has changed since (after a cudaDeviceReset).
 int device_setup(int dev, DeviceSetup** out) {
   if (dev < 0 || dev >= kNaMaxDevices) return MOE_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_setup_mu);
   DeviceSetup& s = g_setup[dev];
-  if (!s.ready) {
+  unsigned long long id = 0;
+  int rc = current_ctx_id(&id);
+  if (rc != MOE_OK) return rc;
+  if (!s.ready || id == 0 || id != s.ctx_id) {
+    s.ready = false;
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_align_scratch) != cudaSuccess || p == nullptr) return MOE_ERR_CUDA;
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
       return MOE_ERR_CUDA;
+    // the symbol lookup made the device's context current if it was not yet
+    if ((rc = current_ctx_id(&id)) != MOE_OK) return rc;
     s.scratch = static_cast<int32_t*>(p);
     s.num_sms = sms;
+    s.ctx_id = id;
     s.ready = true;
   }
   *out = &s;
@@ -103,12 +142,13 @@ extern "C" MOE_API int moe_align_block_size_noalloc(const int32_t* topk_ids, int
   sh.sorted_len = T * top_k + E * (block_m - 1);
   sh.blocks_len = ceil_div(sh.sorted_len, block_m);
 
-  // every launch fits in 48 KB of dynamic shared memory (the default limit; a handle created
-  // earlier may have lowered a kernel's limit, so it is raised back when needed)
+  // every launch fits in 48 KB of dynamic shared memory (the default limit); the limits are
+  // only ever raised, under the same lock moe_init takes, so a concurrent moe_init cannot
+  // lower them between this check and the launches
   const size_t hist_smem = gate_smem_bytes(sh, 0);
   const size_t scatter_smem = scatter_smem_bytes(E, sh.chunk_tokens * top_k);
   if (hist_smem > 48 * 1024 || scatter_smem > 48 * 1024) return MOE_ERR_UNSUPPORTED;
-  if (ensure_align_smem(hist_smem, scatter_smem) != cudaSuccess) return MOE_ERR_CUDA;
+  if (raise_align_smem(0, hist_smem, scatter_smem) != cudaSuccess) return MOE_ERR_CUDA;
 
   Workspace ws{};
   int32_t* base = ds->scratch;

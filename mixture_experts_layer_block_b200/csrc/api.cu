@@ -15,7 +15,6 @@
 #include "mx.cuh"
 
 namespace moe {
-cudaError_t configure_gate_kernels(size_t gate_smem, size_t scatter_smem);
 cudaError_t configure_router_kernel();
 cudaError_t configure_gemm_kernel();
 cudaError_t configure_gemm_pair_kernel(int* max_pairs);
@@ -50,10 +49,6 @@ constexpr int64_t kDefaultTimeoutNs = 2000000000LL;
 constexpr size_t kMapCacheMax = 64;
 constexpr int kTimingRing = 256;  // forwards whose kernel durations moe_stage_times averages
 constexpr int kNumStages = 6;     // router, gating, align scatter, row gather, expert GEMMs, combine
-
-// Dynamic shared memory limits already granted to the gating and scatter kernels (shared by
-// all handles).
-size_t g_gate_smem_granted = 0, g_scatter_smem_granted = 0;
 
 }  // namespace
 
@@ -404,12 +399,8 @@ int moe_init(const moe_config* cfg, moe_handle** out) {
   Shape sh = make_shape(h, c.max_tokens, c.top_k);
   h->gate_smem = gate_smem_bytes(sh, h->max_units);
   const size_t scatter_smem = scatter_smem_bytes(E, sh.chunk_tokens * c.top_k);
-  if (h->gate_smem > g_gate_smem_granted || scatter_smem > g_scatter_smem_granted) {
-    g_gate_smem_granted = std::max(g_gate_smem_granted, h->gate_smem);
-    g_scatter_smem_granted = std::max(g_scatter_smem_granted, scatter_smem);
-    if (check_cuda(configure_gate_kernels(g_gate_smem_granted, g_scatter_smem_granted)))
-      return fail(MOE_ERR_CUDA);
-  }
+  // on the handle's device (current here); raise-only, so no other handle or call loses out
+  if (check_cuda(raise_align_smem(h->gate_smem, h->gate_smem, scatter_smem))) return fail(MOE_ERR_CUDA);
   if (check_cuda(configure_router_kernel()) || check_cuda(configure_gemm_kernel())) return fail(MOE_ERR_CUDA);
   if (check_cuda(configure_gemm_pair_kernel(&h->max_pairs))) return fail(MOE_ERR_CUDA);
   h->max_pairs = std::min(h->max_pairs, h->num_sms / 2);

@@ -22,6 +22,7 @@
 #include <algorithm>
 #include <climits>
 #include <cmath>
+#include <mutex>
 
 #include "launch.h"
 
@@ -563,39 +564,43 @@ cudaError_t launch_scatter(const int32_t* topk_ids, int32_t* sorted_ids, int32_t
                   sorted_ids, expert_ids, num_post_padded, row_of_slot, ws, sh);
 }
 
-// Raise (never lower) the dynamic shared memory limits of the histogram and scatter kernels
-// to what one launch needs; the limit is per kernel and process-wide, and a handle may have
-// set it to its own, smaller, need.
-cudaError_t ensure_align_smem(size_t hist_bytes, size_t scatter_bytes) {
+namespace {
+
+// One lock for every change of these kernels' shared memory limits: moe_init (any thread, any
+// device) and the allocation-free align both go through raise_align_smem.
+std::mutex g_align_smem_mu;
+
+// Raise (never lower) one kernel's dynamic shared memory limit on the current device. The
+// limit is kept per kernel and per device context, so a handle on another device, or an
+// earlier call with a larger need, never leaves a launch with less than it asked for.
+template <typename K>
+cudaError_t raise_one(K* kernel, size_t bytes) {
+  if (bytes == 0) return cudaSuccess;
   cudaFuncAttributes a{};
-  cudaError_t err;
-  if ((err = cudaFuncGetAttributes(&a, hist_kernel))) return err;
-  if ((size_t)a.maxDynamicSharedSizeBytes < hist_bytes &&
-      (err = cudaFuncSetAttribute(hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hist_bytes)))
-    return err;
-  if ((err = cudaFuncGetAttributes(&a, scatter_kernel))) return err;
-  if ((size_t)a.maxDynamicSharedSizeBytes < scatter_bytes &&
-      (err = cudaFuncSetAttribute(scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)scatter_bytes)))
-    return err;
-  return cudaSuccess;
+  cudaError_t err = cudaFuncGetAttributes(&a, kernel);
+  if (err != cudaSuccess) return err;
+  if ((size_t)a.maxDynamicSharedSizeBytes >= bytes) return cudaSuccess;
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
 template <int VPL>
-static cudaError_t set_gate_smem(int s) {
+cudaError_t raise_gate(size_t s) {
   cudaError_t err;
-  if ((err = cudaFuncSetAttribute(gate_kernel<VPL, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, s))) return err;
-  if ((err = cudaFuncSetAttribute(gate_kernel<VPL, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, s))) return err;
-  return cudaFuncSetAttribute(gate_kernel<VPL, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, s);
+  if ((err = raise_one(gate_kernel<VPL, 1>, s))) return err;
+  if ((err = raise_one(gate_kernel<VPL, 2>, s))) return err;
+  return raise_one(gate_kernel<VPL, 4>, s);
 }
 
-cudaError_t configure_gate_kernels(size_t gate_smem, size_t scatter_smem) {
+}  // namespace
+
+cudaError_t raise_align_smem(size_t gate_bytes, size_t hist_bytes, size_t scatter_bytes) {
+  std::lock_guard<std::mutex> lock(g_align_smem_mu);
   cudaError_t err = cudaSuccess;
-  const int s = (int)gate_smem;
-  if ((err = set_gate_smem<1>(s)) || (err = set_gate_smem<2>(s)) || (err = set_gate_smem<4>(s)) ||
-      (err = set_gate_smem<8>(s)) || (err = set_gate_smem<16>(s)) || (err = set_gate_smem<32>(s)))
+  if ((err = raise_gate<1>(gate_bytes)) || (err = raise_gate<2>(gate_bytes)) || (err = raise_gate<4>(gate_bytes)) ||
+      (err = raise_gate<8>(gate_bytes)) || (err = raise_gate<16>(gate_bytes)) || (err = raise_gate<32>(gate_bytes)))
     return err;
-  if ((err = cudaFuncSetAttribute(hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, s))) return err;
-  return cudaFuncSetAttribute(scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)scatter_smem);
+  if ((err = raise_one(hist_kernel, hist_bytes))) return err;
+  return raise_one(scatter_kernel, scatter_bytes);
 }
 
 }  // namespace moe

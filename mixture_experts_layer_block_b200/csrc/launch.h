@@ -74,8 +74,10 @@ cudaError_t launch_scatter(const int32_t* topk_ids, int32_t* sorted_ids, int32_t
                            int32_t* num_post_padded, int32_t* row_of_slot, const Workspace& ws,
                            const Shape& sh, int grid, cudaStream_t stream);
 
-// Raise the histogram and scatter kernels' dynamic shared memory limits to at least these.
-cudaError_t ensure_align_smem(size_t hist_bytes, size_t scatter_bytes);
+// Raise (never lower) the dynamic shared memory limits of the gating, histogram and scatter
+// kernels on the current device to at least these (0 = leave as is), under one process-wide
+// lock, so that concurrent callers on any thread or device only ever raise them.
+cudaError_t raise_align_smem(size_t gate_bytes, size_t hist_bytes, size_t scatter_bytes);
 
 // Copy each kept slot's x row into the tile-ordered buffer ws.xs.
 cudaError_t launch_gather_rows(const uint16_t* x, const Workspace& ws, const Shape& sh, int grid,

@@ -60,6 +60,24 @@ def test_noalloc_matches_handle_align_twice_in_a_row(first, second):
             assert torch.equal(g, r), name
 
 
+def test_noalloc_empty_batch_between_two_batches():
+    """T = 0 between two real batches: the empty call writes only sentinels (0), -1 block ids and
+    P = 0, exactly like the handle align, and leaves nothing behind for the next call."""
+    runs = []
+    for i, T in ((1, None), (1, 0), (0, None)):
+        T0, E, k, bm, cf, dist = CASES[i]
+        T = T0 if T is None else T
+        ids = gen.make_topk_ids(T, E, k, seed=21 + i, dist=dist).cuda()
+        runs.append((ids, E, k, bm, cf, _run_noalloc(ids, E, k, bm, cf)))
+    torch.cuda.synchronize()
+    for ids, E, k, bm, cf, got in runs:
+        ref = _run_handle(ids, E, k, bm, cf)
+        for g, r, name in zip(got, ref, ("sorted_ids", "expert_ids", "num_post_padded")):
+            assert torch.equal(g, r), name
+    s0, e0, n0 = runs[1][5]
+    assert int(n0.item()) == 0 and bool((s0 == 0).all()) and bool((e0 == -1).all())
+
+
 def test_noalloc_rejects_sizes_beyond_its_limit():
     from mixture_experts_layer_block_b200.native import MOE_ERR_UNSUPPORTED, MoEError, align_block_size_noalloc
     ids = torch.zeros((8, 2), dtype=torch.int32, device="cuda")
