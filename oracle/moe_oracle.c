@@ -176,10 +176,13 @@ ORACLE_API int64_t moe_oracle_align(const int32_t *topk_ids, int64_t T, int64_t 
     return P;
 }
 
-/* One expert FFN on one token: y = W_down . SwiGLU(W_up x, W_gate x), SiLU(u) = u/(1+e^-u).
- * w_up, w_gate: [D][H]; w_down: [H][D]; a: scratch [D]. */
-static void expert_ffn(const double *x, const uint16_t *w_up, const uint16_t *w_gate,
-                       const uint16_t *w_down, int64_t H, int64_t D, double *a, double *y)
+/* First half of one expert FFN on one token (the SwiGLU of the layer equation):
+ *   a[d] = SiLU(u_d) * g_d,  u_d = sum_h W_up[d][h] x[h],  g_d = sum_h W_gate[d][h] x[h],
+ * SiLU(u) = u / (1 + e^-u), sums in ascending h. au[d] = sum_h |W_up[d][h] x[h]| and ag[d]
+ * likewise (both nullable): they bound the rounding error of any fp32 evaluation of u_d, g_d.
+ * w_up, w_gate: [D][H]. */
+static void swiglu_row(const double *x, const uint16_t *w_up, const uint16_t *w_gate, int64_t H,
+                       int64_t D, double *a, double *au, double *ag)
 {
     for (int64_t d = 0; d < D; ++d) {
         const uint16_t *ru = w_up + d * H, *rg = w_gate + d * H;
@@ -189,13 +192,44 @@ static void expert_ffn(const double *x, const uint16_t *w_up, const uint16_t *w_
             g += bf16_to_double(rg[h]) * x[h];
         }
         a[d] = (u / (1.0 + exp(-u))) * g;
+        if (au) {
+            double m = 0.0;
+            for (int64_t h = 0; h < H; ++h) m += fabs(bf16_to_double(ru[h]) * x[h]);
+            au[d] = m;
+        }
+        if (ag) {
+            double m = 0.0;
+            for (int64_t h = 0; h < H; ++h) m += fabs(bf16_to_double(rg[h]) * x[h]);
+            ag[d] = m;
+        }
     }
+}
+
+/* Second half: y[h] = sum_d W_down[h][d] a[d] (ascending d); ay[h] = sum_d |W_down[h][d] a[d]|
+ * (nullable). w_down: [H][D]. */
+static void down_row(const double *a, const uint16_t *w_down, int64_t H, int64_t D, double *y,
+                     double *ay)
+{
     for (int64_t h = 0; h < H; ++h) {
         const uint16_t *rd = w_down + h * D;
         double s = 0.0;
         for (int64_t d = 0; d < D; ++d) s += bf16_to_double(rd[d]) * a[d];
         y[h] = s;
+        if (ay) {
+            double m = 0.0;
+            for (int64_t d = 0; d < D; ++d) m += fabs(bf16_to_double(rd[d]) * a[d]);
+            ay[h] = m;
+        }
     }
+}
+
+/* One expert FFN on one token: y = W_down . SwiGLU(W_up x, W_gate x).
+ * w_up, w_gate: [D][H]; w_down: [H][D]; a: scratch [D]. */
+static void expert_ffn(const double *x, const uint16_t *w_up, const uint16_t *w_gate,
+                       const uint16_t *w_down, int64_t H, int64_t D, double *a, double *y)
+{
+    swiglu_row(x, w_up, w_gate, H, D, a, NULL, NULL);
+    down_row(a, w_down, H, D, y, NULL);
 }
 
 /* The layer output for a list of tokens:
@@ -239,6 +273,79 @@ ORACLE_API void moe_oracle_layer(const uint16_t *x, int64_t T, int64_t H, int64_
         free(y);
         free(a);
         free(xt);
+    }
+}
+
+/* ---------------------------------------------------------------------------------------
+ * The layer equation stage by stage, for checking the GPU path's intermediates one step at a
+ * time (each stage is fed the GPU's own output of the stage before it).
+ * ------------------------------------------------------------------------------------- */
+
+/* GEMM1 + SwiGLU for n (token, expert) pairs: h[i][0..Dt) = SwiGLU(W_up^e x_t, W_gate^e x_t),
+ * t = tokens[i], e = experts[i]; e == E selects the shared expert (ws_up, ws_gate, Dt = Ds),
+ * else Dt = D. au, ag (nullable) as in swiglu_row. h, au, ag: [n][ld] (ld >= max(D, Ds)). */
+ORACLE_API void moe_oracle_expert_h(const uint16_t *x, int64_t H, int64_t D, int64_t E,
+                                    const uint16_t *w_up, const uint16_t *w_gate, int64_t Ds,
+                                    const uint16_t *ws_up, const uint16_t *ws_gate,
+                                    const int64_t *tokens, const int32_t *experts, int64_t n,
+                                    int64_t ld, double *h, double *au, double *ag)
+{
+#pragma omp parallel
+    {
+        double *xt = (double *)malloc(sizeof(double) * (size_t)H);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t i = 0; i < n; ++i) {
+            const int64_t t = tokens[i], e = experts[i];
+            for (int64_t c = 0; c < H; ++c) xt[c] = bf16_to_double(x[t * H + c]);
+            if (e == E)
+                swiglu_row(xt, ws_up, ws_gate, H, Ds, h + i * ld, au ? au + i * ld : NULL,
+                           ag ? ag + i * ld : NULL);
+            else
+                swiglu_row(xt, w_up + e * D * H, w_gate + e * D * H, H, D, h + i * ld,
+                           au ? au + i * ld : NULL, ag ? ag + i * ld : NULL);
+        }
+        free(xt);
+    }
+}
+
+/* GEMM2 with the router weight for n rows: y[i][c] = wts[i] * sum_d W_down^e[c][d] a[i][d],
+ * e = experts[i] (E selects the shared expert, ws_down [H][Ds]); a: [n][lda], its first Dt
+ * entries used. ay[i][c] = |wts[i]| * sum_d |W_down^e[c][d] a[i][d]| (nullable). y, ay: [n][H]. */
+ORACLE_API void moe_oracle_expert_down(const double *a, int64_t lda, int64_t H, int64_t D, int64_t E,
+                                       const uint16_t *w_down, int64_t Ds, const uint16_t *ws_down,
+                                       const int32_t *experts, const double *wts, int64_t n, double *y,
+                                       double *ay)
+{
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t i = 0; i < n; ++i) {
+        const int64_t e = experts[i];
+        double *yi = y + i * H, *ai = ay ? ay + i * H : NULL;
+        if (e == E)
+            down_row(a + i * lda, ws_down, H, Ds, yi, ai);
+        else
+            down_row(a + i * lda, w_down + e * H * D, H, D, yi, ai);
+        for (int64_t c = 0; c < H; ++c) {
+            yi[c] = wts[i] * yi[c];
+            if (ai) ai[c] = fabs(wts[i]) * ai[c];
+        }
+    }
+}
+
+/* Combine: out[i] = sum_{j < m, idx[i][j] >= 0} rows[idx[i][j]], summed in j order (the shared
+ * expert's row first, then the token's slots j = 0..k-1, as in moe_oracle_layer).
+ * rows: [*][H]; idx: [n][m]; out: [n][H]. */
+ORACLE_API void moe_oracle_combine(const double *rows, int64_t H, const int64_t *idx, int64_t n,
+                                   int64_t m, double *out)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) {
+        double *o = out + i * H;
+        for (int64_t c = 0; c < H; ++c) o[c] = 0.0;
+        for (int64_t j = 0; j < m; ++j) {
+            const int64_t r = idx[i * m + j];
+            if (r < 0) continue;
+            for (int64_t c = 0; c < H; ++c) o[c] += rows[r * H + c];
+        }
     }
 }
 

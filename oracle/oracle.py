@@ -52,6 +52,13 @@ def _bind(L):
     L.moe_oracle_mx_quantize_bf16_rows.restype = None
     L.moe_oracle_layer_mxfp8.argtypes = L.moe_oracle_layer.argtypes
     L.moe_oracle_layer_mxfp8.restype = None
+    L.moe_oracle_expert_h.argtypes = [_p, _i64, _i64, _i64, _p, _p, _i64, _p, _p, _p, _p, _i64, _i64, _p,
+                                      _p, _p]
+    L.moe_oracle_expert_h.restype = None
+    L.moe_oracle_expert_down.argtypes = [_p, _i64, _i64, _i64, _i64, _p, _i64, _p, _p, _p, _i64, _p, _p]
+    L.moe_oracle_expert_down.restype = None
+    L.moe_oracle_combine.argtypes = [_p, _i64, _p, _i64, _i64, _p]
+    L.moe_oracle_combine.restype = None
     L.moe_oracle_num_threads.argtypes = []
     L.moe_oracle_num_threads.restype = ctypes.c_int
     return L
@@ -218,6 +225,65 @@ def layer(x, weights: dict, topk_ids: np.ndarray, topk_w: np.ndarray, kept: np.n
         assert H % 32 == 0 and D % 32 == 0 and Ds % 32 == 0
     fn(_ptr(xb), T, H, D, E, k, _ptr(ids), _ptr(w), _ptr(kp), _ptr(wu), _ptr(wg), _ptr(wd), Ds, _ptr(su),
        _ptr(sg), _ptr(sd), _ptr(tok), tok.size, _ptr(out))
+    return out
+
+
+# --------------------------------------------------------------------------------------
+# the expert FFN and the combine stage by stage (each stage can be fed another path's output
+# of the stage before it)
+# --------------------------------------------------------------------------------------
+
+def _expert_mats(weights: dict):
+    wu, wg, wd = (bf16_bits(weights[n]) for n in ("W_up", "W_gate", "W_down"))
+    if weights.get("Ws_up") is not None:
+        su, sg, sd = (bf16_bits(weights[n]) for n in ("Ws_up", "Ws_gate", "Ws_down"))
+        Ds = su.shape[0]
+    else:
+        su = sg = sd = None
+        Ds = 0
+    return wu, wg, wd, su, sg, sd, Ds
+
+
+def expert_h(x, weights: dict, tokens, experts, with_absdot: bool = False):
+    """SwiGLU(W_up^e x_t, W_gate^e x_t) (float64 [n, max(D, Ds)]) for each (tokens[i],
+    experts[i]); expert E (the number of routed experts) is the shared expert, whose rows hold
+    Ds valid entries. With `with_absdot` also sum_h |W x| of the up and gate projections."""
+    xb = bf16_bits(x)
+    H = xb.shape[1]
+    wu, wg, wd, su, sg, sd, Ds = _expert_mats(weights)
+    E, D, _ = wu.shape
+    tok = np.ascontiguousarray(tokens, dtype=np.int64)
+    ex = np.ascontiguousarray(experts, dtype=np.int32)
+    ld = max(D, Ds)
+    h = np.zeros((tok.size, ld), dtype=np.float64)
+    au = np.zeros_like(h) if with_absdot else None
+    ag = np.zeros_like(h) if with_absdot else None
+    lib().moe_oracle_expert_h(_ptr(xb), H, D, E, _ptr(wu), _ptr(wg), Ds, _ptr(su), _ptr(sg), _ptr(tok), _ptr(ex),
+                              tok.size, ld, _ptr(h), _ptr(au), _ptr(ag))
+    return (h, au, ag) if with_absdot else h
+
+
+def expert_down(a: np.ndarray, weights: dict, experts, wts, with_absdot: bool = False):
+    """wts[i] * W_down^e a[i] (float64 [n, H]) with e = experts[i] (E = the shared expert); a is
+    float64 [n, >= D (Ds)]. With `with_absdot` also |wts[i]| * sum_d |W_down^e a[i]|."""
+    wu, wg, wd, su, sg, sd, Ds = _expert_mats(weights)
+    E, H, D = wd.shape
+    A = np.ascontiguousarray(a, dtype=np.float64)
+    ex = np.ascontiguousarray(experts, dtype=np.int32)
+    w = np.ascontiguousarray(wts, dtype=np.float64)
+    y = np.empty((ex.size, H), dtype=np.float64)
+    ay = np.empty_like(y) if with_absdot else None
+    lib().moe_oracle_expert_down(_ptr(A), A.shape[1], H, D, E, _ptr(wd), Ds, _ptr(sd), _ptr(ex), _ptr(w), ex.size,
+                                 _ptr(y), _ptr(ay))
+    return (y, ay) if with_absdot else y
+
+
+def combine(rows: np.ndarray, idx: np.ndarray) -> np.ndarray:
+    """out[i] = sum over j of rows[idx[i, j]] in j order, entries < 0 skipped (float64 [n, H])."""
+    R = np.ascontiguousarray(rows, dtype=np.float64)
+    I = np.ascontiguousarray(idx, dtype=np.int64)
+    out = np.empty((I.shape[0], R.shape[1]), dtype=np.float64)
+    lib().moe_oracle_combine(_ptr(R), R.shape[1], _ptr(I), I.shape[0], I.shape[1], _ptr(out))
     return out
 
 

@@ -31,6 +31,10 @@ MUTANTS = {
     "unstable_segment_order": ("sorted_ids[offset[e] + fill[e]++] = (int32_t)s;",
                                "sorted_ids[offset[e] + kept_n[e] - 1 - fill[e]++] = (int32_t)s;"),
     "router_row_index": ("const double *w = wr + e * H;", "const double *w = wr + (E - 1 - e) * H;"),
+    "combine_skips_first_row": ("for (int64_t j = 0; j < m; ++j) {", "for (int64_t j = 1; j < m; ++j) {"),
+    "down_weight_dropped": ("yi[c] = wts[i] * yi[c];", "yi[c] = yi[c];"),
+    "shared_up_gate_swapped": ("swiglu_row(xt, ws_up, ws_gate, H, Ds, h + i * ld,",
+                               "swiglu_row(xt, ws_gate, ws_up, H, Ds, h + i * ld,"),
 }
 
 PIN_TESTS = [
@@ -45,6 +49,10 @@ PIN_TESTS = [
     lambda: pins.test_brute_force_with_capacity_and_shared(),
     lambda: pins.test_brute_force_with_bias(),
     lambda: pins.test_top_k_equals_E_is_dense_softmax_mixture(),
+    lambda: pins.test_expert_h_is_swiglu_of_two_matmuls(),
+    lambda: pins.test_expert_down_is_weighted_matmul(),
+    lambda: pins.test_combine_sums_listed_rows_in_order(),
+    lambda: pins.test_stages_compose_to_the_layer(),
 ]
 
 

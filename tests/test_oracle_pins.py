@@ -254,6 +254,79 @@ def test_top_k_equals_E_is_dense_softmax_mixture():
     np.testing.assert_allclose(res["out"], ref.numpy(), rtol=1e-11, atol=1e-13)
 
 
+# ----------------------------------------------------------------------------------------
+# the expert FFN stage by stage (GEMM1 + SwiGLU, GEMM2 with the router weight, combine)
+# ----------------------------------------------------------------------------------------
+
+def _stage_case():
+    w, inp = _small_inputs(T=20, H=64, D=32, E=5, Ds=48, seed=3)
+    rng = np.random.default_rng(4)
+    tokens = rng.integers(0, w.T, size=40)
+    experts = rng.integers(0, w.E + 1, size=40).astype(np.int32)  # E = the shared expert
+    return w, inp, tokens, experts
+
+
+def test_expert_h_is_swiglu_of_two_matmuls():
+    """GEMM1 + SwiGLU against torch fp64: SiLU(x W_up^T) * (x W_gate^T), SiLU on the up side;
+    the shared expert's rows (expert E) hold Ds entries; |W x| sums against abs matmuls."""
+    w, inp, tokens, experts = _stage_case()
+    h, au, ag = oracle.expert_h(inp["x"], inp, tokens, experts, with_absdot=True)
+    x = inp["x"].double()
+    for i, (t, e) in enumerate(zip(tokens, experts)):
+        wu = inp["Ws_up"] if e == w.E else inp["W_up"][e]
+        wg = inp["Ws_gate"] if e == w.E else inp["W_gate"][e]
+        u = x[t] @ wu.double().T
+        g = x[t] @ wg.double().T
+        n = u.shape[0]
+        np.testing.assert_allclose(h[i, :n], (torch.nn.functional.silu(u) * g).numpy(), rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(au[i, :n], (x[t].abs() @ wu.double().abs().T).numpy(), rtol=1e-12)
+        np.testing.assert_allclose(ag[i, :n], (x[t].abs() @ wg.double().abs().T).numpy(), rtol=1e-12)
+
+
+def test_expert_down_is_weighted_matmul():
+    """GEMM2 against numpy fp64: wts[i] * W_down^e a[i] (W_down is [H][D]: out row c, in d)."""
+    w, inp, tokens, experts = _stage_case()
+    rng = np.random.default_rng(5)
+    a = rng.standard_normal((tokens.size, max(w.D, w.D_shared)))
+    wts = rng.uniform(-1.0, 1.0, size=tokens.size)
+    y, ay = oracle.expert_down(a, inp, experts, wts, with_absdot=True)
+    for i, e in enumerate(experts):
+        wd = _f64(inp["Ws_down"] if e == w.E else inp["W_down"][e])
+        n = wd.shape[1]
+        np.testing.assert_allclose(y[i], wts[i] * (wd @ a[i, :n]), rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(ay[i], abs(wts[i]) * (np.abs(wd) @ np.abs(a[i, :n])), rtol=1e-12)
+
+
+def test_combine_sums_listed_rows_in_order():
+    rng = np.random.default_rng(6)
+    rows = rng.standard_normal((30, 17))
+    idx = rng.integers(-1, 30, size=(9, 5))
+    out = oracle.combine(rows, idx)
+    for i in range(idx.shape[0]):
+        ref = np.zeros(17)
+        for r in idx[i]:
+            if r >= 0:
+                ref = ref + rows[r]
+        np.testing.assert_array_equal(out[i], ref)
+
+
+def test_stages_compose_to_the_layer():
+    """Shared row, then the kept slots' weighted rows in j order, through the three stage
+    functions, give the layer's output (capacity drops included)."""
+    w, inp = _small_inputs(T=40, H=64, D=32, E=4, Ds=24, seed=7)
+    res = oracle.forward(inp, 2, 16, capacity_factor=1.0)
+    T, k = res["topk_ids"].shape
+    tok = np.repeat(np.arange(T), k + 1)
+    ex = np.concatenate([np.full((T, 1), w.E), res["topk_ids"]], axis=1).reshape(-1).astype(np.int32)
+    wts = np.concatenate([np.ones((T, 1)), res["topk_w"]], axis=1).reshape(-1)
+    h = oracle.expert_h(inp["x"], inp, tok, ex)
+    y = oracle.expert_down(h, inp, ex, wts)
+    keep = np.concatenate([np.ones((T, 1), dtype=bool), res["kept"]], axis=1)
+    idx = np.where(keep, np.arange(T * (k + 1)).reshape(T, k + 1), -1)
+    assert not keep.all()  # the case has capacity drops
+    np.testing.assert_allclose(oracle.combine(y, idx), res["out"], rtol=1e-13, atol=1e-15)
+
+
 def _brute_force(inp, k, cap_factor=0.0):
     """Dense per-token loop: every expert's FFN for every token, then the top-k sum.
     No sort of slots and no align; capacity applied by counting in token order."""
