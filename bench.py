@@ -2,16 +2,23 @@
 dominant kernel's fraction of the HBM (or tensor) roofline.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mine|reference]
-                  [--workload flashmoe_prefill] [--no-cpu-baseline] [--e2e-steps M]
+                  [--workload dsv3] [--no-per-config] [--no-cpu-baseline] [--e2e-steps M]
 
 One step = one whole layer forward (router projection, gating, align, row gather, expert
-GEMMs with the fused SwiGLU and router weighting, and the combine) over one batch of seeded synthetic input already resident
-in HBM. The default workload is the FlashMoE-shaped prefill layer (T=4096, H=2048, D=2048,
-E=64, top-2, capacity factor 1.0); its 1.6 GB of expert weights exceed the 126 MB L2, so no
-L2 flush is needed between steps. With N > 1 (torchrun) every rank runs an independent
-replica on its own GPU (no collective on the data path; weak scaling); rank 0 prints one
-JSON line. `--impl reference` times the CPU oracle instead, on a bounded sample of the same
-workload.
+GEMMs with the fused SwiGLU and router weighting, and the combine) over one batch of seeded
+synthetic input already resident in HBM. The headline workload is the largest single-GPU
+layer, the DeepSeek-V3-style one (T=4096, H=7168, 256 routed experts top-8 plus a shared
+expert, 22.6 GB of expert weights, far larger than the 126 MB L2). The line also carries a
+`per_config` object: every other workload (the FlashMoE-shaped prefill, decode on seeds 0, 1
+and 2, the skewed router and the same router without its bias, and the tiny layer), the
+static per-expert-quota ablation and the MXFP8 experts, each with its own timing, roofline
+fractions and SM-busy fraction, plus the skew overhead. Every timing is given twice: K
+forwards back to back (the headline), and K forwards each after a write of a buffer twice the
+L2 size (outside the timed events).
+
+With N > 1 (torchrun) every rank runs an independent replica on its own GPU (no collective on
+the data path; weak scaling); rank 0 prints one JSON line. `--impl reference` times the CPU
+oracle instead, on a bounded token sample of the same workload.
 """
 from __future__ import annotations
 
@@ -34,6 +41,7 @@ from mixture_experts_layer_block_b200 import configs, inputs as gen  # noqa: E40
 METRIC = "MoE layer tokens/s and TFLOP/s on 1 B200; % of bf16/HBM roofline"
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 1024 * 1024
 
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one expert-GEMM launch, from
@@ -98,6 +106,21 @@ def algorithmic_bytes_gemm(w, hit_experts: int, mxfp8: bool = False) -> float:
     return b
 
 
+def algorithmic_bytes_layer(w, hit_experts: int, mxfp8: bool = False) -> float:
+    """The whole layer's algorithmic bytes: the expert GEMMs' (hit experts' and shared weights,
+    x and out) plus the router weights (bf16 [E][H])."""
+    return algorithmic_bytes_gemm(w, hit_experts, mxfp8) + 2.0 * w.E * w.H
+
+
+def config_of(w, precision: str, world: int) -> dict:
+    """The `config` object of the JSON line: the workload only, identical in both arms."""
+    return {"workload": w.name, "T": w.T, "H": w.H, "D": w.D, "E": w.E, "top_k": w.top_k,
+            "block_m": w.block_m, "D_shared": w.D_shared, "capacity_factor": w.capacity_factor,
+            "seed": w.seed, "precision": precision, "parallelism": f"replicas{world}",
+            "l2": "inputs larger than L2 (the expert weights read each step exceed 126 MB); "
+                  "L2-flushed timings reported beside"}
+
+
 def sm_busy_fraction(records: np.ndarray, n_ctas: int) -> dict:
     """SM-busy fraction of one traced forward of the expert-GEMM kernel: per CTA the union of
     its tasks' [claim, done] intervals, summed, over n_ctas x (last done - first claim)."""
@@ -121,6 +144,48 @@ def sm_busy_fraction(records: np.ndarray, n_ctas: int) -> dict:
             "tasks": int(r.shape[0])}
 
 
+def roofline(w, peaks, gemm_ms, kept, hit, mx, timed_pass_s):
+    """Roofline of the dominant kernel (the expert GEMMs): HBM- or tensor-bound, whichever
+    roofline time is longer; achieved = algorithmic bytes (or useful FLOPs) / kernel time."""
+    flops = configs.useful_flops(w, kept)
+    gemm_flops = flops - 2.0 * w.T * w.H * w.E
+    gbytes = algorithmic_bytes_gemm(w, hit, mx)
+    # A GEMM timed inside a loop that keeps the tensor cores busy for a second or more runs at
+    # the clock the 1 kW power cap allows: the sustained GEMM peak (a cuBLAS loop of seconds) is
+    # then the fair denominator; a shorter pass is compared with the burst peak.
+    tc_kind = "sustained" if timed_pass_s >= 1.0 else "burst"
+    tc_peak = peaks["bf16_tflops_sustained"] if tc_kind == "sustained" else peaks["bf16_tflops"]
+    tc_ratio = 2.0 if mx else 1.0  # MXFP8 MMAs: the measured bf16 peak x nominal fp8/bf16 (4.5/2.25)
+    tc_peak *= tc_ratio
+    hbm_t = gbytes / (peaks["hbm_gbs"] * 1e9)
+    tc_t = gemm_flops / (tc_peak * 1e12)
+    if hbm_t >= tc_t:
+        achieved = gbytes / (gemm_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"]}
+    else:
+        achieved = gemm_flops / (gemm_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s",
+                "frac": achieved / tc_peak, "peak_kind": tc_kind, "timed_pass_s": timed_pass_s,
+                "frac_of_burst_peak": achieved / (tc_ratio * peaks["bf16_tflops"])}
+        if mx:
+            roof["peak_dtype"] = "mxfp8: measured bf16 peak x 2 (nominal 4.5 / 2.25 PFLOP/s)"
+    roof["algorithmic_bytes"] = gbytes
+    roof["kernel_ms"] = gemm_ms
+    return roof
+
+
+def layer_fraction(w, peaks, ms, kept, hit, mx):
+    """The whole step against its own roofline: max(useful FLOPs / tensor peak, algorithmic
+    bytes / HBM peak) over the measured step time (the burst tensor peak)."""
+    flops = configs.useful_flops(w, kept)
+    b = algorithmic_bytes_layer(w, hit, mx)
+    t_hbm = b / (peaks["hbm_gbs"] * 1e9)
+    t_tc = flops / ((2.0 if mx else 1.0) * peaks["bf16_tflops"] * 1e12)
+    return {"bound": "hbm" if t_hbm >= t_tc else "tensor", "frac": max(t_hbm, t_tc) / (ms * 1e-3),
+            "algorithmic_bytes": b, "useful_flops": flops}
+
+
 def tile_flags(args) -> int:
     from mixture_experts_layer_block_b200 import native
     f = {"auto": 0, "pair": native.MOE_FLAG_PAIR_TILES, "single": native.MOE_FLAG_SINGLE_TILES}[
@@ -140,8 +205,8 @@ def run_forward(layer, x, wts, out, wq=None):
 
 def traced_forward(w, wts, x, out, extra_flags=0, wq=None):
     """One extra forward with per-task tracing (outside the timed region)."""
-    from mixture_experts_layer_block_b200.native import MOE_FLAG_TRACE, MoELayer
-    layer = MoELayer.for_workload(w, flags=MOE_FLAG_TRACE | extra_flags)
+    from mixture_experts_layer_block_b200.native import MOE_FLAG_MXFP8, MOE_FLAG_TRACE, MoELayer
+    layer = MoELayer.for_workload(w, flags=MOE_FLAG_TRACE | extra_flags | (MOE_FLAG_MXFP8 if wq else 0))
     for _ in range(2):
         run_forward(layer, x, wts, out, wq)
     torch.cuda.synchronize()
@@ -226,7 +291,18 @@ class ClockSampler:
 # CPU oracle timing (the reported baseline, and the reference arm)
 # ------------------------------------------------------------------------------------------
 
+def host_inputs(w, device):
+    """The workload's seeded inputs drawn on `device` (the same values the timed GPU arm uses
+    when that is the GPU) and copied to host memory for the oracle."""
+    wts = gen.make_weights(w, device)
+    x = gen.make_x(w, device)
+    wts = {k: (v.cpu() if v is not None else None) for k, v in wts.items()}
+    return wts, x.cpu()
+
+
 def oracle_sample_time(w, wts_host, x_host, n_tokens, mxfp8=False):
+    """Seconds of one oracle forward (router, gating, align, experts, combine) on the first
+    n_tokens tokens as a batch of their own."""
     from oracle import oracle
     sub = w.replace(T=n_tokens)
     inp = dict(wts_host, x=x_host[:n_tokens])
@@ -235,13 +311,11 @@ def oracle_sample_time(w, wts_host, x_host, n_tokens, mxfp8=False):
     return time.perf_counter() - t0
 
 
-def cpu_baseline(w, wts_dev, x_dev, budget_s=12.0, mxfp8=False):
+def cpu_baseline(w, wts_host, x_host, budget_s=12.0, mxfp8=False):
     """Time the oracle, as it stands, on the first n tokens of the batch (a smaller batch of
     the same layer), n sized for about `budget_s` of CPU work."""
     from oracle import oracle
-    wts_host = {k: (v.cpu() if v is not None else None) for k, v in wts_dev.items()}
-    x_host = x_dev.cpu()
-    n = min(w.T, 4 if mxfp8 else 16)
+    n = min(w.T, 16)
     dt = oracle_sample_time(w, wts_host, x_host, n, mxfp8)
     n2 = int(min(w.T, max(n, n * budget_s / max(dt, 1e-3))))
     if n2 > n:
@@ -249,11 +323,11 @@ def cpu_baseline(w, wts_dev, x_dev, budget_s=12.0, mxfp8=False):
         dt = oracle_sample_time(w, wts_host, x_host, n, mxfp8)
     return {"value": n / dt, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
             "sample": f"oracle forward (fp64 C, OpenMP) on the first {n} tokens of the {w.name} batch "
-                      f"as a batch of its own ({dt:.1f} s)"}
+                      f"as a batch of their own ({dt:.1f} s)"}
 
 
 # ------------------------------------------------------------------------------------------
-# main
+# process plumbing
 # ------------------------------------------------------------------------------------------
 
 def dist_setup():
@@ -266,7 +340,7 @@ def dist_setup():
         backend = "nccl" if torch.cuda.is_available() else "gloo"
         if torch.cuda.is_available():
             torch.cuda.set_device(local)
-        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=300))
     elif torch.cuda.is_available():
         torch.cuda.set_device(local)
     return world, rank, local
@@ -288,50 +362,339 @@ def barrier(world: int):
         dist.barrier()
 
 
-REF_BUDGET_S = 150.0  # CPU seconds of the reference arm's timed steps, whatever --steps is
+REF_BUDGET_S = 60.0  # CPU seconds of the reference arm's timed steps, whatever --steps is
 
 
 def run_reference(args, world, rank):
+    """The reference arm: the CPU oracle, as it stands, on the host cores, on the same
+    workload and config as the GPU arm. Each timed step runs the oracle's whole forward on the
+    first n tokens of the batch, n sized so that the K steps take about REF_BUDGET_S; the line
+    reports the measured seconds per step and the sampled tokens per second."""
     if rank != 0:
         return 0
     w = workload_of(args)
-    wts = gen.make_weights(w, "cpu")
-    x = gen.make_x(w, "cpu")
     from oracle import oracle
     mx = getattr(args, "precision", "bf16") == "mxfp8"
-    # each step is a bounded sample: at most --ref-tokens tokens, and few enough that the K
-    # timed steps take about REF_BUDGET_S in all (sized from a probe that is also the warm-up)
+    wts, x = host_inputs(w, "cuda" if torch.cuda.is_available() else "cpu")
     n_max = min(w.T, args.ref_tokens)
     n_probe = min(n_max, 8)
+    oracle_sample_time(w, wts, x, n_probe, mx)  # warm-up (also loads the oracle)
     t_probe = oracle_sample_time(w, wts, x, n_probe, mx)
     per_step = REF_BUDGET_S / max(args.steps, 1)
     n = int(min(n_max, max(1, n_probe * per_step / max(t_probe, 1e-6))))
+    for _ in range(max(0, min(args.warmup, 1))):
+        oracle_sample_time(w, wts, x, n, mx)
     times = [oracle_sample_time(w, wts, x, n, mx) for _ in range(args.steps)]
-    per_tok = float(np.mean(times)) / n
-    value = 1.0 / per_tok
-    ms_step = per_tok * w.T * 1e3
+    step_s = float(np.mean(times))
+    value = n / step_s
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": w.name, **w.describe(),
-                                            "precision": getattr(args, "precision", "bf16")},
+            "data": "synthetic", "config": config_of(w, getattr(args, "precision", "bf16"), world),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
-                             "sample": f"each step: oracle forward on the first {n} tokens of the batch"},
+                             "sample": f"each step: the oracle's forward on the first {n} of the batch's "
+                                       f"{w.T} tokens (a batch of their own); ms_per_step is that step's "
+                                       f"measured time"},
+            "tokens_per_step": n,
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
+    return 0
+
+
+def workload_of(args, name=None):
+    w = configs.WORKLOADS[name or args.workload]
+    if getattr(args, "T", None) is not None:
+        w = w.replace(T=args.T)
+    if getattr(args, "E", None) is not None:
+        w = w.replace(E=args.E)
+    return w
+
+
+# ------------------------------------------------------------------------------------------
+# the GPU arm
+# ------------------------------------------------------------------------------------------
+
+class Flusher:
+    """Writes a buffer of twice the L2 size, so that nothing of the previous step stays in L2."""
+
+    def __init__(self, dev):
+        try:
+            l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        except (AttributeError, RuntimeError):
+            l2 = L2_BYTES
+        self.buf = torch.empty(2 * max(l2, L2_BYTES) // 4, dtype=torch.float32, device=dev)
+
+    def __call__(self):
+        self.buf.fill_(1.0)
+
+
+def timed_steps(layer, x, wts, out, wq, steps, stream, world, flusher=None):
+    """Device time per step (ms), max over ranks. Without `flusher`: K forwards back to back
+    between two events. With it: each forward between its own pair of events, after an L2 flush
+    outside them; the per-step times are summed."""
+    barrier(world)
+    torch.cuda.synchronize()
+    if flusher is None:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            run_forward(layer, x, wts, out, wq)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / steps
+    else:
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for a, b in evs:
+            flusher()
+            a.record(stream)
+            run_forward(layer, x, wts, out, wq)
+            b.record(stream)
+        torch.cuda.synchronize()
+        ms = sum(a.elapsed_time(b) for a, b in evs) / steps
+    barrier(world)
+    return max_over_ranks(ms, world)
+
+
+def measure(w, dev, world, rank, steps, warmup, peaks, flusher, mx=False, flags=0, trace=True,
+            keep=False, sched="dynamic"):
+    """One workload: warm-up, K steps back to back (clocks sampled), K steps with L2 flushes,
+    a per-kernel timing pass, a traced forward (SM-busy); the roofline of the expert GEMMs and
+    of the whole step. With `keep`, also returns the layer and inputs (for the e2e legs)."""
+    from mixture_experts_layer_block_b200.native import (MOE_FLAG_HOST_STAGING, MOE_FLAG_MXFP8,
+                                                         MOE_FLAG_STAGE_TIMING, MoELayer)
+    prec = MOE_FLAG_MXFP8 if mx else 0
+    wts = gen.make_weights(w, dev)
+    x = gen.make_x(w.replace(seed=w.seed + 1000 * rank) if rank else w, dev)  # each replica its own tokens
+    out = torch.empty((w.T, w.H), dtype=torch.float32, device=dev)
+    layer = MoELayer.for_workload(w, flags=(MOE_FLAG_HOST_STAGING if keep else 0) | prec | flags)
+    stream = torch.cuda.current_stream(dev)
+    wq = layer.quantize_experts_mxfp8(wts) if mx else None  # weights are stored quantised
+    for _ in range(warmup):
+        run_forward(layer, x, wts, out, wq)
+    torch.cuda.synchronize()
+    rc, st = layer.status()
+    assert rc == 0 and st == 0, (w.name, rc, st)
+    stats = routing_stats(layer, w, dev)
+    shape = {"tile_m": layer.query(6), "workers": layer.query(1), "shape": layer.query(8), "scheduler": sched}
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        ms = timed_steps(layer, x, wts, out, wq, steps, stream, world)
+    ms_flushed = timed_steps(layer, x, wts, out, wq, steps, stream, world, flusher)
+    rc, st = layer.status()
+    assert rc == 0 and st == 0, (w.name, rc, st)
+
+    # per-kernel durations: a separate pass whose handle records CUDA events around every kernel
+    # on the launching stream (events between kernels stop them from overlapping)
+    lt = MoELayer.for_workload(w, flags=MOE_FLAG_STAGE_TIMING | prec | flags)
+    for _ in range(3):
+        run_forward(lt, x, wts, out, wq)
+    torch.cuda.synchronize()
+    lt.stage_times()  # drop the warm-up window
+    barrier(world)
+    n_stage = min(steps, 256)
+    for _ in range(n_stage):
+        run_forward(lt, x, wts, out, wq)
+    stage_ms = lt.stage_times()
+    rc, st = lt.status()
+    assert rc == 0 and st == 0, (w.name, rc, st)
+    lt.close()
+    stage_ms = [max_over_ranks(v, world) for v in stage_ms]
+
+    kept, hit = stats["kept_slots"], stats["hit_experts"]
+    flops = configs.useful_flops(w, kept)
+    roof = roofline(w, peaks, stage_ms[4], kept, hit, mx, n_stage * ms * 1e-3)
+    res = {"workload": w.name, "seed": w.seed, "precision": "mxfp8" if mx else "bf16", "steps": steps,
+           "warmup": warmup, "ms_per_step": ms, "ms_per_step_l2_flushed": ms_flushed,
+           "tokens_per_s": world * w.T / (ms * 1e-3), "tflops": flops / (ms * 1e-3) / 1e12,
+           "stage_ms": dict(zip(MoELayer.STAGES, stage_ms)), "routing": stats, "gemm_shape": shape,
+           "roofline": roof, "layer_roofline": layer_fraction(w, peaks, ms, kept, hit, mx),
+           "layer_roofline_l2_flushed": layer_fraction(w, peaks, ms_flushed, kept, hit, mx),
+           "clocks": clk.summary(), "kernel_timing": f"CUDA events around each kernel, {n_stage} forwards"}
+    if trace:
+        res["scheduler"] = traced_forward(w, wts, x, out, flags, wq)
+    if keep:
+        return res, (layer, x, wts, out, wq, stream)
+    layer.close()
+    del wts, x, out, wq
+    torch.cuda.empty_cache()
+    return res
+
+
+def e2e_legs(w, layer, x, wts, out, wq, stream, world, steps, mx):
+    """End to end through the C ABI with host buffers: every step copies x from pinned host
+    memory to the device and the step's out back. Pipelined: moe_forward_host_async overlaps step
+    i+1's upload and step i-1's download with step i's forward; the events bracket all steps and
+    the final join. Also the synchronous moe_forward_host (upload, forward, download, wait)."""
+    x_pin = x.cpu().pin_memory()
+    out_pin = torch.empty((w.T, w.H), dtype=torch.float32).pin_memory()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_ms = None
+    if not mx:
+        for _ in range(3):
+            layer.forward_host(x_pin, wts, out_pin)
+        barrier(world)
+        torch.cuda.synchronize()
+        f0.record(stream)
+        for _ in range(steps):
+            layer.forward_host_async(x_pin, wts, out_pin, stream=stream)
+        layer.forward_host_join(stream=stream, block=False)
+        f1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(f0.elapsed_time(f1) / steps, world)
+    x_dev = torch.empty_like(x)
+
+    def host_step():
+        if mx:  # MXFP8 experts have no host-buffer entry point: the caller's own copies
+            x_dev.copy_(x_pin, non_blocking=True)
+            run_forward(layer, x_dev, wts, out, wq)
+            out_pin.copy_(out, non_blocking=True)
+            stream.synchronize()
+        else:
+            layer.forward_host(x_pin, wts, out_pin)
+    for _ in range(3):
+        host_step()
+    barrier(world)
+    torch.cuda.synchronize()
+    f0.record(stream)
+    for _ in range(steps):
+        host_step()
+    f1.record(stream)
+    torch.cuda.synchronize()
+    sync_ms = max_over_ranks(f0.elapsed_time(f1) / steps, world)
+    if mx:
+        e2e_ms = sync_ms
+    return {"value": world * w.T / (e2e_ms * 1e-3), "unit": UNIT,
+            "h2d_bytes_per_step": w.T * w.H * 2, "d2h_bytes_per_step": w.T * w.H * 4,
+            "api": ("moe_forward_mxfp8 between the caller's pinned-host copies of x and out, synchronised every "
+                    "step") if mx else
+                   ("moe_forward_host_async, steps pipelined (copies overlap the previous and next forwards), "
+                    "joined inside the timed region"),
+            "synchronous": {"value": world * w.T / (sync_ms * 1e-3), "api": "as above" if mx else "moe_forward_host"}}
+
+
+# per_config entries: (key, workload name, seed, precision, extra flags, scheduler)
+def per_config_plan():
+    from mixture_experts_layer_block_b200.native import MOE_FLAG_STATIC_QUOTA as SQ
+    return [
+        ("tiny", "tiny", 0, "bf16", 0, "dynamic"),
+        ("flashmoe_prefill", "flashmoe_prefill", 0, "bf16", 0, "dynamic"),
+        ("decode", "decode", 0, "bf16", 0, "dynamic"),
+        ("decode_seed1", "decode", 1, "bf16", 0, "dynamic"),
+        ("decode_seed2", "decode", 2, "bf16", 0, "dynamic"),
+        ("skew", "skew", 0, "bf16", 0, "dynamic"),
+        ("skew_uniform", "skew_uniform", 0, "bf16", 0, "dynamic"),
+        # the static per-expert SM quota baseline (Weave blog, section 1.2) on the same layers
+        ("static_quota/skew", "skew", 0, "bf16", SQ, "static"),
+        ("static_quota/skew_uniform", "skew_uniform", 0, "bf16", SQ, "static"),
+        ("static_quota/dsv3", "dsv3", 0, "bf16", SQ, "static"),
+        ("static_quota/flashmoe_prefill", "flashmoe_prefill", 0, "bf16", SQ, "static"),
+        ("static_quota/decode", "decode", 0, "bf16", SQ, "static"),
+        # MXFP8 experts
+        ("mxfp8/dsv3", "dsv3", 0, "mxfp8", 0, "dynamic"),
+        ("mxfp8/flashmoe_prefill", "flashmoe_prefill", 0, "mxfp8", 0, "dynamic"),
+        ("mxfp8/decode", "decode", 0, "mxfp8", 0, "dynamic"),
+        ("mxfp8/skew", "skew", 0, "mxfp8", 0, "dynamic"),
+    ]
+
+
+def compact(entry):
+    """A per_config entry without the bulky parts."""
+    keep = ("workload", "seed", "precision", "steps", "ms_per_step", "ms_per_step_l2_flushed", "tokens_per_s",
+            "tflops", "stage_ms", "routing", "gemm_shape", "scheduler", "clocks")
+    d = {k: entry[k] for k in keep if k in entry}
+    r = entry["roofline"]
+    d["gemm_roofline"] = {k: r[k] for k in ("bound", "achieved", "unit", "peak", "frac", "peak_kind",
+                                            "frac_of_burst_peak", "kernel_ms") if k in r}
+    d["layer_roofline"] = {"bound": entry["layer_roofline"]["bound"], "frac": entry["layer_roofline"]["frac"],
+                           "frac_l2_flushed": entry["layer_roofline_l2_flushed"]["frac"]}
+    return d
+
+
+def run_mine(args, world, rank, local):
+    from mixture_experts_layer_block_b200.native import MoELayer
+    dev = torch.device("cuda", local)
+    peaks, peak_src = load_peaks()
+    flusher = Flusher(dev)
+    w = workload_of(args)
+    mx = args.precision == "mxfp8"
+    head, (layer, x, wts, out, wq, stream) = measure(
+        w, dev, world, rank, args.steps, args.warmup, peaks, flusher, mx, tile_flags(args),
+        trace=not args.no_trace, keep=True, sched=args.sched)
+    e2e = e2e_legs(w, layer, x, wts, out, wq, stream, world, args.e2e_steps, mx)
+    layer.close()
+    cpu = None
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        wts_h = {k: (v.cpu() if v is not None else None) for k, v in wts.items()}
+        x_h = x.cpu()
+        del layer, x, wts, out, wq
+        torch.cuda.empty_cache()
+        cpu = cpu_baseline(w, wts_h, x_h, mxfp8=mx)
+        del wts_h, x_h
+    else:
+        del layer, x, wts, out, wq
+        torch.cuda.empty_cache()
+
+    roof = dict(head["roofline"])
+    traffic = args.traffic_bytes if args.traffic_bytes is not None else (None if mx else measured_traffic(w.name))
+    roof.update({"traffic": traffic,
+                 "traffic_source": (measured_traffic_note(w.name) if args.traffic_bytes is None else "--traffic-bytes"),
+                 "kernel": "moe_gemm_mx_kernel" if mx else "moe_gemm_kernel", "peak_source": peak_src,
+                 "kernel_timing": head["kernel_timing"] + " of a second pass"})
+    line = {"metric": METRIC, "value": head["tokens_per_s"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "mxfp8-e4m3 experts, bf16 router" if mx else "bf16", "data": "synthetic",
+            "config": config_of(w, args.precision, world),
+            "ms_per_step_l2_flushed": head["ms_per_step_l2_flushed"],
+            "tflops": head["tflops"], "tflops_frac_of_bf16_peak": head["tflops"] / peaks["bf16_tflops"],
+            "stage_ms": head["stage_ms"], "routing": head["routing"], "roofline": roof,
+            "layer_roofline": head["layer_roofline"], "layer_roofline_l2_flushed": head["layer_roofline_l2_flushed"],
+            "e2e": e2e, "gpu_launches": len(MoELayer.STAGES) * args.steps, "gemm_shape": head["gemm_shape"],
+            "clocks": head["clocks"]}
+    if "scheduler" in head:
+        line["scheduler"] = head["scheduler"]
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+
+    if not args.no_per_config:
+        pc = {}
+        for key, name, seed, prec, flags, sched in per_config_plan():
+            if name == w.name and seed == w.seed and prec == args.precision and flags == tile_flags(args):
+                continue  # the headline itself
+            wk = configs.WORKLOADS[name].replace(seed=seed)
+            slow = sched == "static"
+            e = measure(wk, dev, world, rank, max(5, args.steps // 2) if slow else args.steps,
+                        min(args.warmup, 3) if slow else args.warmup, peaks, flusher, prec == "mxfp8", flags,
+                        trace=not args.no_trace, sched=sched)
+            pc[key] = compact(e)
+        pc[w.name if not mx else f"mxfp8/{w.name}"] = compact(head)
+        line["per_config"] = pc
+        if "skew" in pc and "skew_uniform" in pc:
+            s, u = pc["skew"], pc["skew_uniform"]
+            line["skew_overhead"] = {
+                "layer": s["ms_per_step"] / u["ms_per_step"] - 1.0,
+                "layer_l2_flushed": s["ms_per_step_l2_flushed"] / u["ms_per_step_l2_flushed"] - 1.0,
+                "expert_gemm": s["stage_ms"]["expert_gemm"] / u["stage_ms"]["expert_gemm"] - 1.0,
+                "useful_flops_ratio": (configs.useful_flops(configs.SKEW, s["routing"]["kept_slots"]) /
+                                       configs.useful_flops(configs.SKEW_UNIFORM, u["routing"]["kept_slots"])),
+                "sm_busy": {"skew": s.get("scheduler", {}).get("sm_busy"),
+                            "uniform": u.get("scheduler", {}).get("sm_busy")},
+                "target": "<= 0.15 (time under skewed routing over uniform routing at equal useful FLOPs, minus 1)"}
+    if rank == 0:
+        print(json.dumps(line))
     return 0
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["mine", "reference"], default="mine")
-    ap.add_argument("--workload", default="flashmoe_prefill", choices=sorted(configs.WORKLOADS))
+    ap.add_argument("--workload", default="dsv3", choices=sorted(configs.WORKLOADS))
+    ap.add_argument("--no-per-config", action="store_true", help="time only the headline workload")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-trace", action="store_true", help="skip the traced forward (SM-busy)")
-    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--no-trace", action="store_true", help="skip the traced forwards (SM-busy)")
+    ap.add_argument("--e2e-steps", type=int, default=30)
     ap.add_argument("--ref-tokens", type=int, default=256)
     ap.add_argument("--T", type=int, default=None, help="override the workload's token count (profiling)")
     ap.add_argument("--E", type=int, default=None, help="override the workload's expert count (profiling)")
@@ -355,186 +718,6 @@ def main():
         if world > 1:
             import torch.distributed as dist
             dist.destroy_process_group()
-
-
-def workload_of(args):
-    w = configs.WORKLOADS[args.workload]
-    if args.T is not None:
-        w = w.replace(T=args.T)
-    if args.E is not None:
-        w = w.replace(E=args.E)
-    return w
-
-
-def run_mine(args, world, rank, local):
-    from mixture_experts_layer_block_b200.native import (MOE_FLAG_HOST_STAGING, MOE_FLAG_MXFP8,
-                                                         MOE_FLAG_STAGE_TIMING, MoELayer)
-    w = workload_of(args)
-    mx = args.precision == "mxfp8"
-    prec_flags = MOE_FLAG_MXFP8 if mx else 0
-    dev = torch.device("cuda", local)
-    wts = gen.make_weights(w, dev)
-    x = gen.make_x(w.replace(seed=w.seed + 1000 * rank) if rank else w, dev)  # each replica its own tokens
-    out = torch.empty((w.T, w.H), dtype=torch.float32, device=dev)
-    layer = MoELayer.for_workload(w, flags=MOE_FLAG_HOST_STAGING | prec_flags | tile_flags(args))
-    stream = torch.cuda.current_stream(dev)
-    # MXFP8 experts: the weights are quantised once, before any timing (a model stores them so)
-    wq = layer.quantize_experts_mxfp8(wts) if mx else None
-
-    for _ in range(args.warmup):
-        run_forward(layer, x, wts, out, wq)
-    torch.cuda.synchronize()
-    rc, st = layer.status()
-    assert rc == 0 and st == 0, (rc, st)
-    gemm_shape = {"tile_m": layer.query(6), "workers": layer.query(1), "shape": layer.query(8),
-                  "scheduler": getattr(args, "sched", "dynamic"),
-                  "kind": "SM pairs (2-CTA clusters)" if layer.query(6) == 256 else "single SMs"}
-    stats = routing_stats(layer, w, dev)
-
-    # headline: K whole forwards back to back, nothing recorded between the kernels
-    barrier(world)
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clk:
-        e0.record(stream)
-        for _ in range(args.steps):
-            run_forward(layer, x, wts, out, wq)
-        e1.record(stream)
-        torch.cuda.synchronize()
-    barrier(world)
-    ms = e0.elapsed_time(e1) / args.steps
-    ms = max_over_ranks(ms, world)
-    rc, st = layer.status()
-    assert rc == 0 and st == 0, (rc, st)
-
-    tokens_per_s = world * w.T / (ms * 1e-3)
-    flops = configs.useful_flops(w, stats["kept_slots"])
-    tflops = flops / (ms * 1e-3) / 1e12
-
-    # end to end through the C ABI with host buffers: every step copies x from pinned host memory
-    # to the device and the step's out back. Pipelined: moe_forward_host_async overlaps step
-    # i+1's upload and step i-1's download with step i's forward; the events bracket all steps
-    # and the final join. Also the synchronous moe_forward_host (upload, forward, download, wait).
-    x_pin = x.cpu().pin_memory()
-    out_pin = torch.empty((w.T, w.H), dtype=torch.float32).pin_memory()
-    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if not mx:
-        for _ in range(3):
-            layer.forward_host(x_pin, wts, out_pin)
-        barrier(world)
-        torch.cuda.synchronize()
-        f0.record(stream)
-        for _ in range(args.e2e_steps):
-            layer.forward_host_async(x_pin, wts, out_pin, stream=stream)
-        layer.forward_host_join(stream=stream, block=False)
-        f1.record(stream)
-        torch.cuda.synchronize()
-        e2e_ms = max_over_ranks(f0.elapsed_time(f1) / args.e2e_steps, world)
-    # synchronous: upload, forward, download, wait (for MXFP8 experts, which have no host-buffer
-    # entry point, the caller's own copies around moe_forward_mxfp8)
-    x_dev = torch.empty_like(x)
-
-    def host_step():
-        if mx:
-            x_dev.copy_(x_pin, non_blocking=True)
-            run_forward(layer, x_dev, wts, out, wq)
-            out_pin.copy_(out, non_blocking=True)
-            stream.synchronize()
-        else:
-            layer.forward_host(x_pin, wts, out_pin)
-    for _ in range(3):
-        host_step()
-    barrier(world)
-    torch.cuda.synchronize()
-    f0.record(stream)
-    for _ in range(args.e2e_steps):
-        host_step()
-    f1.record(stream)
-    torch.cuda.synchronize()
-    e2e_sync_ms = max_over_ranks(f0.elapsed_time(f1) / args.e2e_steps, world)
-    if mx:
-        e2e_ms = e2e_sync_ms
-    layer.close()
-
-    # per-kernel durations: a second timed pass whose handle records CUDA events around every
-    # kernel on the launching stream (events between kernels stop them from overlapping, so
-    # this pass is kept apart from the headline one)
-    layer_t = MoELayer.for_workload(w, flags=MOE_FLAG_STAGE_TIMING | prec_flags | tile_flags(args))
-    for _ in range(3):
-        run_forward(layer_t, x, wts, out, wq)
-    torch.cuda.synchronize()
-    layer_t.stage_times()  # drop the warm-up window
-    barrier(world)
-    for _ in range(min(args.steps, 256)):
-        run_forward(layer_t, x, wts, out, wq)
-    stage_ms = layer_t.stage_times()
-    rc, st = layer_t.status()
-    assert rc == 0 and st == 0, (rc, st)
-    layer_t.close()
-
-    peaks, peak_src = load_peaks()
-    gemm_ms = stage_ms[4]
-    gbytes = algorithmic_bytes_gemm(w, stats["hit_experts"], mx)
-    gemm_flops = flops - 2.0 * w.T * w.H * w.E
-    # The GEMM is timed inside a loop of forwards. When that loop keeps the tensor cores busy for
-    # a second or more the 1 kW power cap sets the clock, and the sustained GEMM peak (a cuBLAS
-    # loop of seconds) is the fair denominator; a shorter pass is compared with the burst peak.
-    timed_pass_s = min(args.steps, 256) * ms * 1e-3
-    tc_kind = "sustained" if timed_pass_s >= 1.0 else "burst"
-    tc_peak = peaks["bf16_tflops_sustained"] if tc_kind == "sustained" else peaks["bf16_tflops"]
-    # MXFP8 MMAs: the measured bf16 peak times the nominal fp8 / bf16 ratio (4.5 / 2.25 PFLOP/s)
-    tc_ratio = 2.0 if mx else 1.0
-    tc_peak *= tc_ratio
-    hbm_t = gbytes / (peaks["hbm_gbs"] * 1e9)
-    tc_t = gemm_flops / (tc_peak * 1e12)
-    if hbm_t >= tc_t:
-        achieved = gbytes / (gemm_ms * 1e-3) / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"]}
-    else:
-        achieved = gemm_flops / (gemm_ms * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s",
-                "frac": achieved / tc_peak, "peak_kind": tc_kind,
-                "timed_pass_s": timed_pass_s, "frac_of_burst_peak": achieved / (tc_ratio * peaks["bf16_tflops"])}
-        if mx:
-            roof["peak_dtype"] = "mxfp8: measured bf16 peak x 2 (nominal 4.5 / 2.25 PFLOP/s)"
-    traffic = args.traffic_bytes if args.traffic_bytes is not None else (None if mx else measured_traffic(w.name))
-    roof.update({"traffic": traffic, "traffic_source": measured_traffic_note(w.name) if args.traffic_bytes is None
-                 else "--traffic-bytes", "kernel": "moe_gemm_mx_kernel" if mx else "moe_gemm_kernel",
-                 "algorithmic_bytes": gbytes, "kernel_ms": gemm_ms, "peak_source": peak_src,
-                 "kernel_timing": f"CUDA events around the kernel over {min(args.steps, 256)} timed forwards "
-                                  "of a second pass"})
-
-    line = {"metric": METRIC, "value": tokens_per_s, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "mxfp8-e4m3 experts, bf16 router" if mx else "bf16",
-            "data": "synthetic",
-            "config": {"workload": w.name, "T": w.T, "H": w.H, "D": w.D, "E": w.E, "top_k": w.top_k,
-                       "block_m": w.block_m, "D_shared": w.D_shared, "capacity_factor": w.capacity_factor,
-                       "precision": args.precision,
-                       "parallelism": f"replicas{world}",
-                       "l2": "inputs larger than L2 (expert weights read each step exceed 126 MB)"},
-            "tflops": tflops, "tflops_frac_of_bf16_peak": tflops / peaks["bf16_tflops"],
-            "stage_ms": dict(zip(MoELayer.STAGES, stage_ms)),
-            "routing": stats, "roofline": roof,
-            "e2e": {"value": world * w.T / (e2e_ms * 1e-3), "unit": UNIT,
-                    "h2d_bytes_per_step": w.T * w.H * 2, "d2h_bytes_per_step": w.T * w.H * 4,
-                    "api": ("moe_forward_mxfp8 between the caller's pinned-host copies of x and out, "
-                            "synchronised every step") if mx else
-                           ("moe_forward_host_async, steps pipelined (copies overlap the previous "
-                            "and next forwards), joined inside the timed region"),
-                    "synchronous": {"value": world * w.T / (e2e_sync_ms * 1e-3),
-                                    "api": "as above" if mx else "moe_forward_host"}},
-            "gpu_launches": len(MoELayer.STAGES) * args.steps,
-            "gemm_shape": gemm_shape,
-            "clocks": clk.summary()}
-    if not args.no_trace:
-        line["scheduler"] = traced_forward(w, wts, x, out, tile_flags(args) | prec_flags, wq)
-    if world == 1 and rank == 0 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, wts, x, mxfp8=mx)
-    if rank == 0:
-        print(json.dumps(line))
-    return 0
 
 
 if __name__ == "__main__":

@@ -272,6 +272,22 @@ MOE_API int moe_debug_outputs(moe_handle *h, float *logits, int32_t *topk_ids, f
                       int32_t *sorted_ids, int32_t *expert_ids, int32_t *num_post_padded,
                       void *stream);
 
+/* Copy the expert GEMMs' per-row results of the most recent forward on `stream` into caller
+ * device buffers (each nullable), for checking the layer stage by stage:
+ *   h_rows            bf16 [moe_query 9][moe_query 10]: SwiGLU(W_up^e x_t, W_gate^e x_t) of
+ *                     every GEMM row (the up/gate GEMM's output; bf16 experts only: after
+ *                     moe_forward_mxfp8, h_rows must be NULL, else MOE_ERR_NOT_READY)
+ *   y_rows            bf16 [moe_query 9][H]: w_s * W_down^e h of every row (the down GEMM's
+ *                     output, router weight applied; weight 1 for shared-expert rows)
+ *   row_of_slot       int32 [T][k]: the GEMM row of slot s = t*k + j, or -1 if it was dropped
+ *   num_routed_tiles  int32 [1]: M_r, the routed experts' m-tiles; the shared expert's tile i
+ *                     (tokens i*tile_m ...) follows at rows (M_r + i) * tile_m (moe_query 6)
+ * Rows are grouped in m-tiles of moe_query 6 rows; rows past a tile's valid rows hold no
+ * result. (Layer equation of the Mixture-of-Kittens blog, its two GEMMs taken one by one.)
+ * Returns MOE_ERR_NOT_READY before the first forward. */
+MOE_API int moe_debug_expert_rows(moe_handle *h, void *h_rows, void *y_rows, int32_t *row_of_slot,
+                                  int32_t *num_routed_tiles, void *stream);
+
 /* Mean durations in milliseconds of the kernels of the forwards recorded since the previous
  * call (the first 256 of them; needs MOE_FLAG_STAGE_TIMING; synchronises, then starts a new
  * recording window): ms[0] router, ms[1] gating, ms[2] align scatter, ms[3] row gather,
@@ -286,7 +302,8 @@ MOE_API int moe_stage_times(moe_handle *h, float *ms, int32_t n);
  * 5 dependency lag (units) of the last forward, 6 rows per m-tile of the last forward
  * (128 or 256), 7 SM pairs the device can run at once for the pair shape (0 = none),
  * 8 expert-GEMM shape of the last forward (0 general, 1 small-tile, 2 tail, 3 SM pairs,
- * 4 MXFP8). */
+ * 4 MXFP8), 9 rows of the per-row buffers of moe_debug_expert_rows, 10 their h row stride
+ * (elements, max(D, D_shared)). */
 MOE_API int moe_query(const moe_handle *h, int32_t which, int64_t *value);
 
 /* Per-task trace of the last forward (needs MOE_FLAG_TRACE; synchronises). Fills up to

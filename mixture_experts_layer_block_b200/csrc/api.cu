@@ -881,6 +881,27 @@ int moe_debug_outputs(moe_handle* h, float* logits, int32_t* topk_ids, float* to
   return MOE_OK;
 }
 
+int moe_debug_expert_rows(moe_handle* h, void* h_rows, void* y_rows, int32_t* row_of_slot,
+                          int32_t* num_routed_tiles, void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  if (!h->have_forward) return MOE_ERR_NOT_READY;
+  if (h_rows && h->last_shape == 4) return MOE_ERR_NOT_READY;  // MXFP8 keeps h quantised
+  int rc;
+  if ((rc = select_device(h))) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Workspace& w = h->ws;
+  auto cp = [&](void* dst, const void* src, size_t bytes) {
+    if (!dst || bytes == 0) return MOE_OK;
+    return check_cuda(cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, st));
+  };
+  const size_t rows = (size_t)h->tile_rows;
+  if ((rc = cp(h_rows, w.h, rows * w.ldh * 2))) return rc;
+  if ((rc = cp(y_rows, w.y, rows * h->cfg.hidden * 2))) return rc;
+  if ((rc = cp(row_of_slot, w.row_of_slot, (size_t)h->last_T * h->last_k * 4))) return rc;
+  if ((rc = cp(num_routed_tiles, &w.meta->num_routed_tiles, 4))) return rc;
+  return MOE_OK;
+}
+
 int moe_stage_times(moe_handle* h, float* ms, int32_t n) {
   if (!h || !ms || n < 1) return MOE_ERR_INVALID_ARG;
   if (!h->timing || h->timed == 0) return MOE_ERR_NOT_READY;
@@ -919,6 +940,8 @@ int moe_query(const moe_handle* h, int32_t which, int64_t* value) {
     case 6: *value = h->last_tile_m; return MOE_OK;
     case 7: *value = h->max_pairs; return MOE_OK;
     case 8: *value = h->last_shape; return MOE_OK;
+    case 9: *value = h->tile_rows; return MOE_OK;
+    case 10: *value = h->ws.ldh; return MOE_OK;
     default: return MOE_ERR_INVALID_ARG;
   }
 }

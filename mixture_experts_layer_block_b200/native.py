@@ -78,6 +78,7 @@ SIGNATURES = {
     "moe_sorted_len": (_I64, [_P, _I32, _I32]),
     "moe_blocks_len": (_I64, [_P, _I32, _I32]),
     "moe_debug_outputs": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_debug_expert_rows": (ctypes.c_int, [_P, _P, _P, _P, _P, _P]),
     "moe_stage_times": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_float), _I32]),
     "moe_query": (ctypes.c_int, [_P, _I32, ctypes.POINTER(ctypes.c_int64)]),
     "moe_trace_read": (ctypes.c_int, [_P, _P, _I64, ctypes.POINTER(ctypes.c_int64)]),
@@ -282,6 +283,19 @@ class MoELayer:
                                                                     "sorted_ids", "expert_ids",
                                                                     "num_post_padded")),
                                     _stream(stream)), "moe_debug_outputs")
+        return d
+
+    def debug_expert_rows(self, T, k, device, with_h=True, stream=None):
+        """moe_debug_expert_rows: the GEMM rows of the last forward, as torch tensors (h and y
+        bf16 [rows, ...], row_of_slot int32 [T*k], num_routed_tiles int)."""
+        import torch
+        rows, ldh = self.query(9), self.query(10)
+        d = {"h": torch.empty((rows, ldh), dtype=torch.bfloat16, device=device) if with_h else None,
+             "y": torch.empty((rows, self.cfg.hidden), dtype=torch.bfloat16, device=device),
+             "row_of_slot": torch.empty((T * k,), dtype=torch.int32, device=device),
+             "num_routed_tiles": torch.empty((1,), dtype=torch.int32, device=device)}
+        check(lib.moe_debug_expert_rows(self.h, _ptr(d["h"]), _ptr(d["y"]), _ptr(d["row_of_slot"]),
+                                        _ptr(d["num_routed_tiles"]), _stream(stream)), "moe_debug_expert_rows")
         return d
 
     def status(self):

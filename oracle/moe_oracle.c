@@ -178,11 +178,11 @@ ORACLE_API int64_t moe_oracle_align(const int32_t *topk_ids, int64_t T, int64_t 
 
 /* First half of one expert FFN on one token (the SwiGLU of the layer equation):
  *   a[d] = SiLU(u_d) * g_d,  u_d = sum_h W_up[d][h] x[h],  g_d = sum_h W_gate[d][h] x[h],
- * SiLU(u) = u / (1 + e^-u), sums in ascending h. au[d] = sum_h |W_up[d][h] x[h]| and ag[d]
- * likewise (both nullable): they bound the rounding error of any fp32 evaluation of u_d, g_d.
- * w_up, w_gate: [D][H]. */
+ * SiLU(u) = u / (1 + e^-u), sums in ascending h. Optional outputs (nullable): uo[d] = u_d,
+ * go[d] = g_d, and au[d] = sum_h |W_up[d][h] x[h]|, ag[d] likewise, which bound the rounding
+ * error of any fp32 evaluation of u_d and g_d. w_up, w_gate: [D][H]. */
 static void swiglu_row(const double *x, const uint16_t *w_up, const uint16_t *w_gate, int64_t H,
-                       int64_t D, double *a, double *au, double *ag)
+                       int64_t D, double *a, double *uo, double *go, double *au, double *ag)
 {
     for (int64_t d = 0; d < D; ++d) {
         const uint16_t *ru = w_up + d * H, *rg = w_gate + d * H;
@@ -192,6 +192,8 @@ static void swiglu_row(const double *x, const uint16_t *w_up, const uint16_t *w_
             g += bf16_to_double(rg[h]) * x[h];
         }
         a[d] = (u / (1.0 + exp(-u))) * g;
+        if (uo) uo[d] = u;
+        if (go) go[d] = g;
         if (au) {
             double m = 0.0;
             for (int64_t h = 0; h < H; ++h) m += fabs(bf16_to_double(ru[h]) * x[h]);
@@ -228,7 +230,7 @@ static void down_row(const double *a, const uint16_t *w_down, int64_t H, int64_t
 static void expert_ffn(const double *x, const uint16_t *w_up, const uint16_t *w_gate,
                        const uint16_t *w_down, int64_t H, int64_t D, double *a, double *y)
 {
-    swiglu_row(x, w_up, w_gate, H, D, a, NULL, NULL);
+    swiglu_row(x, w_up, w_gate, H, D, a, NULL, NULL, NULL, NULL);
     down_row(a, w_down, H, D, y, NULL);
 }
 
@@ -283,12 +285,14 @@ ORACLE_API void moe_oracle_layer(const uint16_t *x, int64_t T, int64_t H, int64_
 
 /* GEMM1 + SwiGLU for n (token, expert) pairs: h[i][0..Dt) = SwiGLU(W_up^e x_t, W_gate^e x_t),
  * t = tokens[i], e = experts[i]; e == E selects the shared expert (ws_up, ws_gate, Dt = Ds),
- * else Dt = D. au, ag (nullable) as in swiglu_row. h, au, ag: [n][ld] (ld >= max(D, Ds)). */
+ * else Dt = D. u, g, au, ag (nullable) as uo, go, au, ag of swiglu_row. Every output is
+ * [n][ld] (ld >= max(D, Ds)). */
 ORACLE_API void moe_oracle_expert_h(const uint16_t *x, int64_t H, int64_t D, int64_t E,
                                     const uint16_t *w_up, const uint16_t *w_gate, int64_t Ds,
                                     const uint16_t *ws_up, const uint16_t *ws_gate,
                                     const int64_t *tokens, const int32_t *experts, int64_t n,
-                                    int64_t ld, double *h, double *au, double *ag)
+                                    int64_t ld, double *h, double *u, double *g, double *au,
+                                    double *ag)
 {
 #pragma omp parallel
     {
@@ -296,13 +300,13 @@ ORACLE_API void moe_oracle_expert_h(const uint16_t *x, int64_t H, int64_t D, int
 #pragma omp for schedule(dynamic, 1)
         for (int64_t i = 0; i < n; ++i) {
             const int64_t t = tokens[i], e = experts[i];
+            double *ui = u ? u + i * ld : NULL, *gi = g ? g + i * ld : NULL;
+            double *aui = au ? au + i * ld : NULL, *agi = ag ? ag + i * ld : NULL;
             for (int64_t c = 0; c < H; ++c) xt[c] = bf16_to_double(x[t * H + c]);
             if (e == E)
-                swiglu_row(xt, ws_up, ws_gate, H, Ds, h + i * ld, au ? au + i * ld : NULL,
-                           ag ? ag + i * ld : NULL);
+                swiglu_row(xt, ws_up, ws_gate, H, Ds, h + i * ld, ui, gi, aui, agi);
             else
-                swiglu_row(xt, w_up + e * D * H, w_gate + e * D * H, H, D, h + i * ld,
-                           au ? au + i * ld : NULL, ag ? ag + i * ld : NULL);
+                swiglu_row(xt, w_up + e * D * H, w_gate + e * D * H, H, D, h + i * ld, ui, gi, aui, agi);
         }
         free(xt);
     }
@@ -463,34 +467,60 @@ ORACLE_API void moe_oracle_mx_quantize_bf16_rows(const uint16_t *src, int64_t R,
     }
 }
 
-/* One expert FFN on one MX-quantised token row xq (values):
- *   h = SwiGLU(Wq_up xq, Wq_gate xq), hq = MX(fp32(h)), y = Wq_down hq,
- * with every weight row quantised along its contraction dimension. */
-static void expert_ffn_mx(const double *xq, const uint16_t *w_up, const uint16_t *w_gate,
-                          const uint16_t *w_down, int64_t H, int64_t D, double *wrow,
-                          uint8_t *scratch, double *a, double *y)
+/* One expert's FFN on n MX-quantised token rows (values; row l is xq + rows[l] * H):
+ *   a_l = SwiGLU(Wq_up xq_l, Wq_gate xq_l) rounded to fp32 and quantised along Dt,
+ *   y_l = Wq_down a_l,
+ * where every weight row is quantised along its contraction dimension -- once, and used for
+ * all n rows. w_up, w_gate: [Dt][H]; w_down: [H][Dt]; a: [n][Dt]; y: [n][H]. */
+static void expert_rows_mx(const double *xq, const int64_t *rows, int64_t n, int64_t H, int64_t Dt,
+                           const uint16_t *w_up, const uint16_t *w_gate, const uint16_t *w_down,
+                           double *a, double *y)
 {
-    for (int64_t d = 0; d < D; ++d) {
-        double u = 0.0, g = 0.0;
-        for (int64_t h = 0; h < H; ++h) wrow[h] = bf16_to_double(w_up[d * H + h]);
-        mx_round_trip(wrow, H, scratch);
-        for (int64_t h = 0; h < H; ++h) u += wrow[h] * xq[h];
-        for (int64_t h = 0; h < H; ++h) wrow[h] = bf16_to_double(w_gate[d * H + h]);
-        mx_round_trip(wrow, H, scratch);
-        for (int64_t h = 0; h < H; ++h) g += wrow[h] * xq[h];
-        a[d] = (double)(float)((u / (1.0 + exp(-u))) * g);
-    }
-    mx_round_trip(a, D, scratch);
-    for (int64_t h = 0; h < H; ++h) {
-        for (int64_t d = 0; d < D; ++d) wrow[d] = bf16_to_double(w_down[h * D + d]);
-        mx_round_trip(wrow, D, scratch);
-        double s = 0.0;
-        for (int64_t d = 0; d < D; ++d) s += wrow[d] * a[d];
-        y[h] = s;
+    const int64_t W = H > Dt ? H : Dt;
+#pragma omp parallel
+    {
+        double *wu = (double *)malloc(sizeof(double) * (size_t)W);
+        double *wg = (double *)malloc(sizeof(double) * (size_t)W);
+        double *wd = (double *)malloc(sizeof(double) * (size_t)W);
+        uint8_t *scratch = (uint8_t *)malloc((size_t)(W + W / 32));
+#pragma omp for schedule(dynamic, 4)
+        for (int64_t d = 0; d < Dt; ++d) {
+            for (int64_t h = 0; h < H; ++h) wu[h] = bf16_to_double(w_up[d * H + h]);
+            mx_round_trip(wu, H, scratch);
+            for (int64_t h = 0; h < H; ++h) wg[h] = bf16_to_double(w_gate[d * H + h]);
+            mx_round_trip(wg, H, scratch);
+            for (int64_t l = 0; l < n; ++l) {
+                const double *xl = xq + rows[l] * H;
+                double u = 0.0, g = 0.0;
+                for (int64_t h = 0; h < H; ++h) u += wu[h] * xl[h];
+                for (int64_t h = 0; h < H; ++h) g += wg[h] * xl[h];
+                a[l * Dt + d] = (double)(float)((u / (1.0 + exp(-u))) * g);
+            }
+        }
+#pragma omp for schedule(static)
+        for (int64_t l = 0; l < n; ++l) mx_round_trip(a + l * Dt, Dt, scratch);
+#pragma omp for schedule(dynamic, 4)
+        for (int64_t h = 0; h < H; ++h) {
+            for (int64_t d = 0; d < Dt; ++d) wd[d] = bf16_to_double(w_down[h * Dt + d]);
+            mx_round_trip(wd, Dt, scratch);
+            for (int64_t l = 0; l < n; ++l) {
+                double s = 0.0;
+                for (int64_t d = 0; d < Dt; ++d) s += wd[d] * a[l * Dt + d];
+                y[l * H + h] = s;
+            }
+        }
+        free(scratch);
+        free(wd);
+        free(wg);
+        free(wu);
     }
 }
 
-/* moe_oracle_layer with MXFP8 experts (H, D and Ds multiples of 32). */
+/* moe_oracle_layer with MXFP8 experts (H, D and Ds multiples of 32): x, every expert weight
+ * row and h are quantised as above; per token the shared expert's row first, then the kept
+ * slots j = 0..k-1 weighted by topk_w, as in moe_oracle_layer. The experts are taken one at a
+ * time (each weight row is quantised once per call); each slot's result is kept until the
+ * per-token sums, which run in the order just stated. */
 ORACLE_API void moe_oracle_layer_mxfp8(const uint16_t *x, int64_t T, int64_t H, int64_t D, int64_t E,
                                        int64_t k, const int32_t *topk_ids, const double *topk_w,
                                        const uint8_t *kept, const uint16_t *w_up,
@@ -499,42 +529,69 @@ ORACLE_API void moe_oracle_layer_mxfp8(const uint16_t *x, int64_t T, int64_t H, 
                                        const uint16_t *ws_down, const int64_t *tokens,
                                        int64_t n_tokens, double *out)
 {
-    (void)T; (void)E;
+    (void)T;
+    const int64_t m = k + 1; /* per token: slots 0..k-1, then the shared expert */
     const int64_t Dmax = Ds > D ? Ds : D;
-    const int64_t W = H > Dmax ? H : Dmax;
+    double *xq = (double *)malloc(sizeof(double) * (size_t)(n_tokens * H));
+    double *ys = (double *)calloc((size_t)(n_tokens * m * H), sizeof(double));
+    double *a = (double *)malloc(sizeof(double) * (size_t)(n_tokens * Dmax));
+    double *ye = (double *)malloc(sizeof(double) * (size_t)(n_tokens * H));
+    int64_t *rows = (int64_t *)malloc(sizeof(int64_t) * (size_t)n_tokens);
+    int64_t *dest = (int64_t *)malloc(sizeof(int64_t) * (size_t)n_tokens);
 #pragma omp parallel
     {
-        double *xt = (double *)malloc(sizeof(double) * (size_t)H);
-        double *a = (double *)malloc(sizeof(double) * (size_t)Dmax);
-        double *y = (double *)malloc(sizeof(double) * (size_t)H);
-        double *wrow = (double *)malloc(sizeof(double) * (size_t)W);
-        uint8_t *scratch = (uint8_t *)malloc((size_t)(W + W / 32));
-#pragma omp for schedule(dynamic, 1)
+        uint8_t *scratch = (uint8_t *)malloc((size_t)(H + H / 32));
+#pragma omp for schedule(static)
         for (int64_t i = 0; i < n_tokens; ++i) {
-            const int64_t t = tokens[i];
-            double *o = out + i * H;
-            for (int64_t h = 0; h < H; ++h) xt[h] = bf16_to_double(x[t * H + h]);
-            mx_round_trip(xt, H, scratch);
-            for (int64_t h = 0; h < H; ++h) o[h] = 0.0;
-            if (Ds > 0) {
-                expert_ffn_mx(xt, ws_up, ws_gate, ws_down, H, Ds, wrow, scratch, a, y);
-                for (int64_t h = 0; h < H; ++h) o[h] += y[h];
-            }
-            for (int64_t j = 0; j < k; ++j) {
-                const int64_t s = t * k + j;
-                if (!kept[s]) continue;
-                const int64_t e = topk_ids[s];
-                expert_ffn_mx(xt, w_up + e * D * H, w_gate + e * D * H, w_down + e * H * D, H, D,
-                              wrow, scratch, a, y);
-                for (int64_t h = 0; h < H; ++h) o[h] += topk_w[s] * y[h];
-            }
+            for (int64_t h = 0; h < H; ++h) xq[i * H + h] = bf16_to_double(x[tokens[i] * H + h]);
+            mx_round_trip(xq + i * H, H, scratch);
         }
         free(scratch);
-        free(wrow);
-        free(y);
-        free(a);
-        free(xt);
     }
+    for (int64_t e = 0; e <= E; ++e) {
+        const int shared = (e == E);
+        if (shared && Ds == 0) break;
+        int64_t n = 0;
+        for (int64_t i = 0; i < n_tokens; ++i) {
+            if (shared) {
+                rows[n] = i;
+                dest[n++] = i * m + k;
+                continue;
+            }
+            for (int64_t j = 0; j < k; ++j) {
+                const int64_t s = tokens[i] * k + j;
+                if (kept[s] && topk_ids[s] == e) {
+                    rows[n] = i;
+                    dest[n++] = i * m + j;
+                }
+            }
+        }
+        if (n == 0) continue;
+        if (shared)
+            expert_rows_mx(xq, rows, n, H, Ds, ws_up, ws_gate, ws_down, a, ye);
+        else
+            expert_rows_mx(xq, rows, n, H, D, w_up + e * D * H, w_gate + e * D * H, w_down + e * H * D, a, ye);
+        for (int64_t l = 0; l < n; ++l) memcpy(ys + dest[l] * H, ye + l * H, sizeof(double) * (size_t)H);
+    }
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n_tokens; ++i) {
+        const int64_t t = tokens[i];
+        double *o = out + i * H;
+        for (int64_t h = 0; h < H; ++h) o[h] = 0.0;
+        if (Ds > 0)
+            for (int64_t h = 0; h < H; ++h) o[h] += ys[(i * m + k) * H + h];
+        for (int64_t j = 0; j < k; ++j) {
+            const int64_t s = t * k + j;
+            if (!kept[s]) continue;
+            for (int64_t h = 0; h < H; ++h) o[h] += topk_w[s] * ys[(i * m + j) * H + h];
+        }
+    }
+    free(dest);
+    free(rows);
+    free(ye);
+    free(a);
+    free(ys);
+    free(xq);
 }
 
 /* Threads the OpenMP loops above use (1 when built without OpenMP). */

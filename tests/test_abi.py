@@ -62,6 +62,7 @@ def test_null_arguments(native):
     assert native.lib.moe_forward(None, None, 0, None, None, None, None, None, None, 1, None, None) \
         == native.MOE_ERR_INVALID_ARG
     assert native.lib.moe_sorted_len(None, 4, 2) == -1
+    assert native.lib.moe_debug_expert_rows(None, None, None, None, None, None) == native.MOE_ERR_INVALID_ARG
     native.lib.moe_destroy(None)
 
 

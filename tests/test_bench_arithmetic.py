@@ -56,3 +56,34 @@ def test_skew_is_tensor_bound_and_prefill_hbm_bound():
         t_tc = flops / (peaks["bf16_tflops"] * 1e12)
         t_hbm = bench.algorithmic_bytes_gemm(w, w.E) / (peaks["hbm_gbs"] * 1e9)
         assert (t_tc > t_hbm) == (bound == "tensor"), name
+
+
+def test_layer_fraction_adds_the_router_weights():
+    peaks = {"hbm_gbs": 6459.3, "bf16_tflops": 1653.5}
+    w = configs.DECODE
+    b = bench.algorithmic_bytes_layer(w, 53)
+    assert b == pytest.approx(bench.algorithmic_bytes_gemm(w, 53) + 2.0 * w.E * w.H, rel=1e-12)
+    # 53 hit experts of 6.29 MB, the router weights, x and out: about 334.6 MB
+    assert b == pytest.approx(334.6e6, rel=2e-3)
+    f = bench.layer_fraction(w, peaks, 0.074, w.T * w.top_k, 53, False)
+    assert f["bound"] == "hbm" and f["frac"] == pytest.approx(b / 6459.3e9 / 0.074e-3, rel=1e-12)
+    assert f["frac"] == pytest.approx(0.70, abs=0.005)
+
+
+def test_config_object_is_the_same_in_both_arms():
+    """The reference arm and the GPU arm print the same config object for the same workload."""
+    w = configs.DSV3
+    a = bench.config_of(w, "bf16", 1)
+    assert a == bench.config_of(configs.WORKLOADS["dsv3"], "bf16", 1)
+    assert a["workload"] == "dsv3" and a["T"] == 4096 and a["E"] == 256 and a["D_shared"] == 2048
+    assert bench.config_of(w, "bf16", 2)["parallelism"] == "replicas2"
+
+
+def test_per_config_plan_covers_every_workload_and_the_decode_seeds():
+    names = {(n, s) for _, n, s, p, f, _ in bench.per_config_plan() if p == "bf16" and f == 0}
+    for n in ("tiny", "flashmoe_prefill", "skew", "skew_uniform"):
+        assert (n, 0) in names
+    assert {("decode", 0), ("decode", 1), ("decode", 2)} <= names
+    keys = [k for k, *_ in bench.per_config_plan()]
+    assert len(keys) == len(set(keys))
+    assert any(k.startswith("static_quota/") for k in keys) and any(k.startswith("mxfp8/") for k in keys)

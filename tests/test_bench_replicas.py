@@ -68,6 +68,12 @@ def test_two_gloo_ranks():
     line = json.loads(res[0][2].strip())
     assert line["impl"] == "reference" and line["unit"] == "tokens/s" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+    # the measured step time of the sampled tokens, and the main arm's config object
+    import bench
+    from mixture_experts_layer_block_b200 import configs
+    assert line["config"] == bench.config_of(configs.TINY, "bf16", 2)
+    n = line["tokens_per_step"]
+    assert 1 <= n <= 8 and abs(line["value"] * line["ms_per_step"] * 1e-3 - n) < 1e-6 * n
 
 
 def test_reference_arm_mxfp8_line():

@@ -18,7 +18,7 @@ import torch
 
 from mixture_experts_layer_block_b200 import configs, inputs as gen
 from oracle import oracle
-from parity import check_forward, sample_tokens
+from parity import check_forward
 
 pytestmark = pytest.mark.gpu
 
@@ -133,7 +133,8 @@ def test_forward_mxfp8_differs_from_bf16_by_quantisation_only():
 def test_forward_mxfp8_full_size_sampled(name):
     w = configs.WORKLOADS[name]
     layer, inp, wq = _setup(w)
-    res = check_forward(layer, w, inp, tokens=sample_tokens(w.T, 12, seed=5), wq=wq)
+    res = check_forward(layer, w, inp, tokens="tiles", min_tokens=128, wq=wq)
+    assert res["compared_tokens"] >= 128 - res["near_ties"]
     print(name, res)
     layer.close()
 

@@ -35,6 +35,7 @@ MUTANTS = {
     "down_weight_dropped": ("yi[c] = wts[i] * yi[c];", "yi[c] = yi[c];"),
     "shared_up_gate_swapped": ("swiglu_row(xt, ws_up, ws_gate, H, Ds, h + i * ld,",
                                "swiglu_row(xt, ws_gate, ws_up, H, Ds, h + i * ld,"),
+    "up_projection_reported_as_gate": ("if (uo) uo[d] = u;", "if (uo) uo[d] = g;"),
 }
 
 PIN_TESTS = [
@@ -65,16 +66,15 @@ MX_MUTANTS = {
                                "if (frac >= 0.5) n += 1.0;"),
     "mx_emax_7": ("s = (ex - 1) - 8;", "s = (ex - 1) - 7;"),
     "mx_no_saturation": ("if (a > 448.0) a = 448.0;", "if (a > 1e300) a = 448.0;"),
-    "mx_h_not_quantised": ("    mx_round_trip(a, D, scratch);\n", "    (void)a;\n"),
-    "mx_x_not_quantised": ("mx_round_trip(xt, H, scratch);", "(void)xt;"),
+    "mx_h_not_quantised": ("mx_round_trip(a + l * Dt, Dt, scratch);", "(void)scratch;"),
+    "mx_x_not_quantised": ("mx_round_trip(xq + i * H, H, scratch);", "(void)scratch;"),
     "mx_amax_over_16": ("for (int i = 0; i < 32; ++i) if (fabs(blk[i]) > amax)",
                         "for (int i = 0; i < 16; ++i) if (fabs(blk[i]) > amax)"),
     "mx_scale_applied_inverted": ("moe_oracle_e4m3_encode(ldexp(blk[i], -s))",
                                   "moe_oracle_e4m3_encode(ldexp(blk[i], s))"),
     "mx_subnormal_step": ("if (e == 0) v = ldexp((double)m, -9);", "if (e == 0) v = ldexp((double)m, -10);"),
     "mx_exponent_bias": ("else v = ldexp(1.0 + m / 8.0, e - 7);", "else v = ldexp(1.0 + m / 8.0, e - 8);"),
-    "mx_down_weights_not_quantised": ("        for (int64_t d = 0; d < D; ++d) wrow[d] = bf16_to_double(w_down[h * D + d]);\n        mx_round_trip(wrow, D, scratch);",
-                                      "        for (int64_t d = 0; d < D; ++d) wrow[d] = bf16_to_double(w_down[h * D + d]);"),
+    "mx_down_weights_not_quantised": ("mx_round_trip(wd, Dt, scratch);", "(void)wd;"),
 }
 
 

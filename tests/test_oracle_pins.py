@@ -268,9 +268,10 @@ def _stage_case():
 
 def test_expert_h_is_swiglu_of_two_matmuls():
     """GEMM1 + SwiGLU against torch fp64: SiLU(x W_up^T) * (x W_gate^T), SiLU on the up side;
-    the shared expert's rows (expert E) hold Ds entries; |W x| sums against abs matmuls."""
+    the shared expert's rows (expert E) hold Ds entries; the projections and their |W x| sums
+    against plain and abs matmuls."""
     w, inp, tokens, experts = _stage_case()
-    h, au, ag = oracle.expert_h(inp["x"], inp, tokens, experts, with_absdot=True)
+    h, uo, go, au, ag = oracle.expert_h(inp["x"], inp, tokens, experts, with_parts=True)
     x = inp["x"].double()
     for i, (t, e) in enumerate(zip(tokens, experts)):
         wu = inp["Ws_up"] if e == w.E else inp["W_up"][e]
@@ -279,6 +280,8 @@ def test_expert_h_is_swiglu_of_two_matmuls():
         g = x[t] @ wg.double().T
         n = u.shape[0]
         np.testing.assert_allclose(h[i, :n], (torch.nn.functional.silu(u) * g).numpy(), rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(uo[i, :n], u.numpy(), rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(go[i, :n], g.numpy(), rtol=1e-12, atol=1e-14)
         np.testing.assert_allclose(au[i, :n], (x[t].abs() @ wu.double().abs().T).numpy(), rtol=1e-12)
         np.testing.assert_allclose(ag[i, :n], (x[t].abs() @ wg.double().abs().T).numpy(), rtol=1e-12)
 

@@ -70,3 +70,135 @@ def test_inputs_have_the_stated_scale():
     d = gen.make_inputs(w)
     assert abs(d["x"].float().std().item() - w.sigma_x) < 0.02 * w.sigma_x
     assert abs(d["W_up"].float().std().item() - w.sigma_w) < 0.02 * w.sigma_w
+
+
+# ------------------------------------------------------------------------------------------
+# tile-aware sampling and the stage-by-stage checker, against a stand-in layer on the CPU
+# ------------------------------------------------------------------------------------------
+
+def test_gemm_tiles_cut_each_expert_segment_into_tiles():
+    from oracle import oracle
+    from parity import gemm_tiles
+    ids = gen.make_topk_ids(300, 6, 2, seed=3, dist="skewed").numpy()
+    al = oracle.align(ids, 6, 16)
+    S = 600
+    tiles = gemm_tiles(al["sorted_ids"], al["expert_ids"], al["num_post_padded"], S, 16, tile_m=128)
+    flat = ids.reshape(-1)
+    seen = np.concatenate(tiles)
+    np.testing.assert_array_equal(np.sort(seen), np.arange(S))  # every slot once
+    for tl in tiles:
+        assert 1 <= tl.size <= 128 and np.all(flat[tl] == flat[tl[0]]) and np.all(np.diff(tl) > 0)
+    counts = np.bincount(flat, minlength=6)
+    assert len(tiles) == sum((c + 127) // 128 for c in counts)
+
+
+def test_tile_sample_covers_first_and_last_row_of_every_tile():
+    from parity import tile_sample
+    rng = np.random.default_rng(0)
+    tiles = [np.sort(rng.choice(4000, size=n, replace=False)) for n in (128, 128, 5, 1, 77)]
+    tokens, slots, shared = tile_sample(tiles, T=1000, k=4, has_shared=True, min_tokens=300)
+    for tl in tiles:
+        assert tl[0] in slots and tl[-1] in slots
+    assert {0, 127, 128, 255, 896, 999} <= set(shared.tolist())
+    assert set((slots // 4).tolist()) <= set(tokens.tolist()) and tokens.size >= 300
+    assert np.all(np.diff(tokens) > 0)
+
+
+class _StandIn:
+    """Plays the CUDA layer's part for check_stages: per-row results computed by the oracle and
+    rounded the way the GPU stores them (h and y bf16, out fp32), laid out like the library's
+    tile-ordered buffers."""
+
+    def __init__(self, w, inp, res):
+        from oracle import oracle
+        T, k, E = w.T, w.top_k, w.E
+        self.T, self.k = T, k
+        kept = res["kept"].reshape(-1)
+        slots = np.flatnonzero(kept)
+        self.Mr = (slots.size + 127) // 128
+        rows = self.Mr * 128 + ((T + 127) // 128) * 128
+        ros = np.full(T * k, -1, dtype=np.int32)
+        ros[slots] = np.arange(slots.size)
+        tok = np.concatenate([slots // k, np.arange(T)])
+        ex = np.concatenate([res["topk_ids"].reshape(-1)[slots], np.full(T, E)]).astype(np.int32)
+        wts = np.concatenate([res["topk_w"].reshape(-1)[slots].astype(np.float32).astype(np.float64), np.ones(T)])
+        r = np.concatenate([np.arange(slots.size), self.Mr * 128 + np.arange(T)])
+        h = oracle.expert_h(inp["x"], inp, tok, ex)
+        hb = torch.from_numpy(h).to(torch.bfloat16)
+        y = oracle.expert_down(hb.double().numpy(), inp, ex, wts)
+        ld = h.shape[1]
+        self.h = torch.zeros((rows, ld), dtype=torch.bfloat16)
+        self.y = torch.zeros((rows, w.H), dtype=torch.bfloat16)
+        self.h[torch.as_tensor(r)] = hb
+        self.y[torch.as_tensor(r)] = torch.from_numpy(y).to(torch.bfloat16)
+        self.ros = torch.from_numpy(ros)
+        out = np.zeros((T, w.H), dtype=np.float32)
+        for t in range(T):
+            acc = self.y[self.Mr * 128 + t].float().numpy().copy()
+            for j in range(k):
+                if ros[t * k + j] >= 0:
+                    acc = acc + self.y[ros[t * k + j]].float().numpy()
+            out[t] = acc
+        self.out = torch.from_numpy(out)
+        self.gw = res["topk_w"].astype(np.float32)
+
+    def query(self, which):
+        return 128
+
+    def debug_expert_rows(self, T, k, device, with_h=True, stream=None):
+        return {"h": self.h if with_h else None, "y": self.y, "row_of_slot": self.ros,
+                "num_routed_tiles": torch.tensor([self.Mr], dtype=torch.int32)}
+
+
+def _stage_setup():
+    from oracle import oracle
+    w = configs.MoEWorkload("stage_cpu", T=70, H=96, D=64, E=5, top_k=2, block_m=16, D_shared=32,
+                            sigma_w=0.1, capacity_factor=1.0)
+    inp = gen.make_inputs(w)
+    res = oracle.forward(inp, w.top_k, w.block_m, w.capacity_factor)
+    return w, inp, res, _StandIn(w, inp, res)
+
+
+def _run_stages(w, inp, res, layer):
+    from parity import check_stages, compact_weights
+    T, k, E = w.T, w.top_k, w.E
+    experts = np.arange(E)
+    remap = np.arange(E + 1)
+    cw = compact_weights(inp, experts)
+    return check_stages(layer, w, inp, res["topk_ids"], layer.gw, layer.out, np.arange(T * k), np.arange(T),
+                        np.arange(T), 128, cw, remap, inp["x"])
+
+
+def test_stage_checker_accepts_values_rounded_like_the_gpu():
+    w, inp, res, layer = _stage_setup()
+    r = _run_stages(w, inp, res, layer)
+    assert r["h_match"] == 1.0 and r["y_match"] == 1.0 and r["combine_err"] <= 1e-6
+
+
+def _bump(t, row, col, ulps):
+    """t[row, col] moved by `ulps` bf16 steps."""
+    v = t[row, col].view(torch.int16)
+    t[row, col] = (v + ulps).view(torch.bfloat16)
+
+
+def test_stage_checker_rejects_planted_errors():
+    import pytest
+    w, inp, res, layer = _stage_setup()
+    slot = int(np.flatnonzero(res["kept"].reshape(-1))[7])
+    row = int(layer.ros[slot])
+    # h three bf16 steps off in one element of one row
+    _bump(layer.h, row, 5, 3)
+    with pytest.raises(AssertionError, match="GEMM1"):
+        _run_stages(w, inp, res, layer)
+    _bump(layer.h, row, 5, -3)
+    # y of one slot without its router weight
+    saved = layer.y[row].clone()
+    layer.y[row] = (layer.y[row].double() / float(layer.gw.reshape(-1)[slot])).to(torch.bfloat16)
+    with pytest.raises(AssertionError, match="GEMM2"):
+        _run_stages(w, inp, res, layer)
+    layer.y[row] = saved
+    # out of one token missing its shared-expert row
+    t = 3
+    layer.out[t] -= layer.y[layer.Mr * 128 + t].float()
+    with pytest.raises(AssertionError, match="combine"):
+        _run_stages(w, inp, res, layer)
