@@ -467,14 +467,32 @@ ORACLE_API void moe_oracle_mx_quantize_bf16_rows(const uint16_t *src, int64_t R,
     }
 }
 
+/* xq[i] = the values of the MX quantisation of token row x[tokens[i]] (along H), i < n. */
+static void mx_token_rows(const uint16_t *x, int64_t H, const int64_t *tokens, int64_t n, double *xq)
+{
+#pragma omp parallel
+    {
+        uint8_t *scratch = (uint8_t *)malloc((size_t)(H + H / 32));
+#pragma omp for schedule(static)
+        for (int64_t i = 0; i < n; ++i) {
+            for (int64_t h = 0; h < H; ++h) xq[i * H + h] = bf16_to_double(x[tokens[i] * H + h]);
+            mx_round_trip(xq + i * H, H, scratch);
+        }
+        free(scratch);
+    }
+}
+
 /* One expert's FFN on n MX-quantised token rows (values; row l is xq + rows[l] * H):
  *   a_l = SwiGLU(Wq_up xq_l, Wq_gate xq_l) rounded to fp32 and quantised along Dt,
  *   y_l = Wq_down a_l,
  * where every weight row is quantised along its contraction dimension -- once, and used for
- * all n rows. w_up, w_gate: [Dt][H]; w_down: [H][Dt]; a: [n][Dt]; y: [n][H]. */
+ * all n rows. w_up, w_gate: [Dt][H]; w_down: [H][Dt] (NULL: stop after a); a: [n][Dt];
+ * y: [n][H]. Optional outputs ([n][Dt], nullable): a_pre = a before its quantisation, uo / go
+ * = the up / gate projections, au / ag = their sums of |Wq xq| (rounding-error bounds). */
 static void expert_rows_mx(const double *xq, const int64_t *rows, int64_t n, int64_t H, int64_t Dt,
                            const uint16_t *w_up, const uint16_t *w_gate, const uint16_t *w_down,
-                           double *a, double *y)
+                           double *a, double *y, double *a_pre, double *uo, double *go, double *au,
+                           double *ag)
 {
     const int64_t W = H > Dt ? H : Dt;
 #pragma omp parallel
@@ -495,12 +513,25 @@ static void expert_rows_mx(const double *xq, const int64_t *rows, int64_t n, int
                 for (int64_t h = 0; h < H; ++h) u += wu[h] * xl[h];
                 for (int64_t h = 0; h < H; ++h) g += wg[h] * xl[h];
                 a[l * Dt + d] = (double)(float)((u / (1.0 + exp(-u))) * g);
+                if (a_pre) a_pre[l * Dt + d] = a[l * Dt + d];
+                if (uo) uo[l * Dt + d] = u;
+                if (go) go[l * Dt + d] = g;
+                if (au) {
+                    double m = 0.0;
+                    for (int64_t h = 0; h < H; ++h) m += fabs(wu[h] * xl[h]);
+                    au[l * Dt + d] = m;
+                }
+                if (ag) {
+                    double m = 0.0;
+                    for (int64_t h = 0; h < H; ++h) m += fabs(wg[h] * xl[h]);
+                    ag[l * Dt + d] = m;
+                }
             }
         }
 #pragma omp for schedule(static)
         for (int64_t l = 0; l < n; ++l) mx_round_trip(a + l * Dt, Dt, scratch);
 #pragma omp for schedule(dynamic, 4)
-        for (int64_t h = 0; h < H; ++h) {
+        for (int64_t h = 0; h < (w_down ? H : 0); ++h) {
             for (int64_t d = 0; d < Dt; ++d) wd[d] = bf16_to_double(w_down[h * Dt + d]);
             mx_round_trip(wd, Dt, scratch);
             for (int64_t l = 0; l < n; ++l) {
@@ -514,6 +545,52 @@ static void expert_rows_mx(const double *xq, const int64_t *rows, int64_t n, int
         free(wg);
         free(wu);
     }
+}
+
+/* The MXFP8 layer's GEMM1 + SwiGLU for n (token, expert) pairs (expert E = the shared expert):
+ * h[i] = SwiGLU(Wq_up^e xq_t, Wq_gate^e xq_t) rounded to fp32, i.e. the values that the layer then
+ * quantises, with the projections u, g and their magnitude sums au, ag (each nullable). Every
+ * output is [n][ld], ld >= max(D, Ds). */
+ORACLE_API void moe_oracle_expert_h_mxfp8(const uint16_t *x, int64_t H, int64_t D, int64_t E,
+                                          const uint16_t *w_up, const uint16_t *w_gate, int64_t Ds,
+                                          const uint16_t *ws_up, const uint16_t *ws_gate,
+                                          const int64_t *tokens, const int32_t *experts, int64_t n,
+                                          int64_t ld, double *h, double *u, double *g, double *au,
+                                          double *ag)
+{
+    const int64_t Dmax = Ds > D ? Ds : D;
+    double *xq = (double *)malloc(sizeof(double) * (size_t)(n * H));
+    int64_t *rows = (int64_t *)malloc(sizeof(int64_t) * (size_t)n);
+    int64_t *dest = (int64_t *)malloc(sizeof(int64_t) * (size_t)n);
+    double *abuf = (double *)malloc(sizeof(double) * (size_t)(n * Dmax));
+    double *part[5];
+    for (int q = 0; q < 5; ++q) part[q] = (double *)malloc(sizeof(double) * (size_t)(n * Dmax));
+    double *outs[5] = {h, u, g, au, ag};
+    mx_token_rows(x, H, tokens, n, xq);
+    for (int64_t e = 0; e <= E; ++e) {
+        int64_t m = 0;
+        for (int64_t i = 0; i < n; ++i)
+            if (experts[i] == e) {
+                rows[m] = i;
+                dest[m++] = i;
+            }
+        if (m == 0) continue;
+        const int64_t Dt = (e == E) ? Ds : D;
+        if (e == E)
+            expert_rows_mx(xq, rows, m, H, Dt, ws_up, ws_gate, NULL, abuf, NULL, part[0], part[1], part[2],
+                           au ? part[3] : NULL, ag ? part[4] : NULL);
+        else
+            expert_rows_mx(xq, rows, m, H, Dt, w_up + e * D * H, w_gate + e * D * H, NULL, abuf, NULL, part[0],
+                           part[1], part[2], au ? part[3] : NULL, ag ? part[4] : NULL);
+        for (int64_t l = 0; l < m; ++l)
+            for (int q = 0; q < 5; ++q)
+                if (outs[q]) memcpy(outs[q] + dest[l] * ld, part[q] + l * Dt, sizeof(double) * (size_t)Dt);
+    }
+    for (int q = 0; q < 5; ++q) free(part[q]);
+    free(abuf);
+    free(dest);
+    free(rows);
+    free(xq);
 }
 
 /* moe_oracle_layer with MXFP8 experts (H, D and Ds multiples of 32): x, every expert weight
@@ -538,16 +615,7 @@ ORACLE_API void moe_oracle_layer_mxfp8(const uint16_t *x, int64_t T, int64_t H, 
     double *ye = (double *)malloc(sizeof(double) * (size_t)(n_tokens * H));
     int64_t *rows = (int64_t *)malloc(sizeof(int64_t) * (size_t)n_tokens);
     int64_t *dest = (int64_t *)malloc(sizeof(int64_t) * (size_t)n_tokens);
-#pragma omp parallel
-    {
-        uint8_t *scratch = (uint8_t *)malloc((size_t)(H + H / 32));
-#pragma omp for schedule(static)
-        for (int64_t i = 0; i < n_tokens; ++i) {
-            for (int64_t h = 0; h < H; ++h) xq[i * H + h] = bf16_to_double(x[tokens[i] * H + h]);
-            mx_round_trip(xq + i * H, H, scratch);
-        }
-        free(scratch);
-    }
+    mx_token_rows(x, H, tokens, n_tokens, xq);
     for (int64_t e = 0; e <= E; ++e) {
         const int shared = (e == E);
         if (shared && Ds == 0) break;
@@ -568,9 +636,10 @@ ORACLE_API void moe_oracle_layer_mxfp8(const uint16_t *x, int64_t T, int64_t H, 
         }
         if (n == 0) continue;
         if (shared)
-            expert_rows_mx(xq, rows, n, H, Ds, ws_up, ws_gate, ws_down, a, ye);
+            expert_rows_mx(xq, rows, n, H, Ds, ws_up, ws_gate, ws_down, a, ye, NULL, NULL, NULL, NULL, NULL);
         else
-            expert_rows_mx(xq, rows, n, H, D, w_up + e * D * H, w_gate + e * D * H, w_down + e * H * D, a, ye);
+            expert_rows_mx(xq, rows, n, H, D, w_up + e * D * H, w_gate + e * D * H, w_down + e * H * D, a, ye,
+                           NULL, NULL, NULL, NULL, NULL);
         for (int64_t l = 0; l < n; ++l) memcpy(ys + dest[l] * H, ye + l * H, sizeof(double) * (size_t)H);
     }
 #pragma omp parallel for schedule(static)

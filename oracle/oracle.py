@@ -55,6 +55,8 @@ def _bind(L):
     L.moe_oracle_expert_h.argtypes = [_p, _i64, _i64, _i64, _p, _p, _i64, _p, _p, _p, _p, _i64, _i64, _p,
                                       _p, _p, _p, _p]
     L.moe_oracle_expert_h.restype = None
+    L.moe_oracle_expert_h_mxfp8.argtypes = L.moe_oracle_expert_h.argtypes
+    L.moe_oracle_expert_h_mxfp8.restype = None
     L.moe_oracle_expert_down.argtypes = [_p, _i64, _i64, _i64, _i64, _p, _i64, _p, _p, _p, _i64, _p, _p]
     L.moe_oracle_expert_down.restype = None
     L.moe_oracle_combine.argtypes = [_p, _i64, _p, _i64, _i64, _p]
@@ -244,11 +246,13 @@ def _expert_mats(weights: dict):
     return wu, wg, wd, su, sg, sd, Ds
 
 
-def expert_h(x, weights: dict, tokens, experts, with_parts: bool = False):
+def expert_h(x, weights: dict, tokens, experts, with_parts: bool = False, mxfp8: bool = False):
     """SwiGLU(W_up^e x_t, W_gate^e x_t) (float64 [n, max(D, Ds)]) for each (tokens[i],
     experts[i]); expert E (the number of routed experts) is the shared expert, whose rows hold
     Ds valid entries. With `with_parts` returns (h, u, g, au, ag): also the up and gate
-    projections u = W_up x, g = W_gate x and their magnitude sums sum_h |W x|."""
+    projections u = W_up x, g = W_gate x and their magnitude sums sum_h |W x|. With `mxfp8`, the
+    MXFP8 layer's stage: x and the weight rows quantised, h rounded to fp32 (the values the layer
+    then quantises)."""
     xb = bf16_bits(x)
     H = xb.shape[1]
     wu, wg, wd, su, sg, sd, Ds = _expert_mats(weights)
@@ -258,8 +262,9 @@ def expert_h(x, weights: dict, tokens, experts, with_parts: bool = False):
     ld = max(D, Ds)
     h = np.zeros((tok.size, ld), dtype=np.float64)
     parts = [np.zeros_like(h) for _ in range(4)] if with_parts else [None] * 4
-    lib().moe_oracle_expert_h(_ptr(xb), H, D, E, _ptr(wu), _ptr(wg), Ds, _ptr(su), _ptr(sg), _ptr(tok), _ptr(ex),
-                              tok.size, ld, _ptr(h), *(_ptr(q) for q in parts))
+    fn = lib().moe_oracle_expert_h_mxfp8 if mxfp8 else lib().moe_oracle_expert_h
+    fn(_ptr(xb), H, D, E, _ptr(wu), _ptr(wg), Ds, _ptr(su), _ptr(sg), _ptr(tok), _ptr(ex), tok.size, ld, _ptr(h),
+       *(_ptr(q) for q in parts))
     return (h, *parts) if with_parts else h
 
 

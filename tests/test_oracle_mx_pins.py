@@ -242,3 +242,47 @@ def test_grid_weights_and_inputs_leave_only_h_rounding():
             bound[t] += mx["topk_w"][t, j] * (np.abs(g["W_down"][e].double().numpy()) @ (np.abs(h) * 2.0 ** -4 * 1.0001 + 1e-30))
     assert np.all(np.abs(mx["out"] - ex["out"]) <= bound)
     assert np.any(mx["out"] != ex["out"])
+
+
+def _mx_rows(t):
+    """Values of the MX quantisation of each row of a bf16 matrix, float64."""
+    m = t.reshape(-1, t.shape[-1])
+    c, s = oracle.mx_quantize_bf16_rows(m)
+    return oracle.mx_values(c.ravel(), s.ravel()).reshape(m.shape)
+
+
+def test_mx_expert_h_is_swiglu_of_the_quantised_operands():
+    """The MXFP8 layer's GEMM1 stage against numpy on the quantiser's own values: u = Wq_up xq,
+    g = Wq_gate xq, h = fp32(SiLU(u) g), with the |Wq xq| sums; the shared expert's rows hold Ds
+    entries; and from h, the layer's remaining steps (h quantised, Wq_down, weighted sum in slot
+    order) written out with numpy give the layer's output."""
+    inp = _rand_inputs(T=10, H=64, D=64, E=4, Ds=32, seed=9)
+    E = 4
+    rng = np.random.default_rng(2)
+    tokens = rng.integers(0, 10, size=24)
+    experts = rng.integers(0, E + 1, size=24).astype(np.int32)
+    h, u, g, au, ag = oracle.expert_h(inp["x"], inp, tokens, experts, with_parts=True, mxfp8=True)
+    xq = _mx_rows(inp["x"])
+    for i, (t, e) in enumerate(zip(tokens, experts)):
+        wu = _mx_rows(inp["Ws_up"] if e == E else inp["W_up"][e])
+        wg = _mx_rows(inp["Ws_gate"] if e == E else inp["W_gate"][e])
+        n = wu.shape[0]
+        ur, gr = wu @ xq[t], wg @ xq[t]
+        np.testing.assert_allclose(u[i, :n], ur, rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(g[i, :n], gr, rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(au[i, :n], np.abs(wu) @ np.abs(xq[t]), rtol=1e-12)
+        np.testing.assert_allclose(ag[i, :n], np.abs(wg) @ np.abs(xq[t]), rtol=1e-12)
+        np.testing.assert_allclose(h[i, :n], (ur / (1 + np.exp(-ur)) * gr).astype(np.float32), rtol=2e-7, atol=1e-30)
+    res = oracle.forward(inp, 2, block_m=16, mxfp8=True)
+    T = inp["x"].shape[0]
+    tk = np.repeat(np.arange(T), 3)
+    ex = np.concatenate([np.full((T, 1), E), res["topk_ids"]], axis=1).reshape(-1).astype(np.int32)
+    hh = oracle.expert_h(inp["x"], inp, tk, ex, mxfp8=True)
+    out = np.zeros((T, inp["x"].shape[1]))
+    for i, (t, e) in enumerate(zip(tk, ex)):
+        wd = _mx_rows(inp["Ws_down"] if e == E else inp["W_down"][e])
+        c, s = oracle.mx_quantize(hh[i, :wd.shape[1]])
+        y = wd @ oracle.mx_values(c, s)
+        j = i % 3
+        out[t] += y if j == 0 else res["topk_w"][t, j - 1] * y
+    np.testing.assert_allclose(out, res["out"], rtol=1e-12, atol=1e-13)

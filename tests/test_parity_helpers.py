@@ -202,3 +202,45 @@ def test_stage_checker_rejects_planted_errors():
     layer.out[t] -= layer.y[layer.Mr * 128 + t].float()
     with pytest.raises(AssertionError, match="combine"):
         _run_stages(w, inp, res, layer)
+
+
+# ------------------------------------------------------------------------------------------
+# MXFP8: certified h-code flips
+# ------------------------------------------------------------------------------------------
+
+def test_mx_flip_steps_mark_only_elements_near_a_rounding_midpoint():
+    from parity import mx_flip_steps
+    # one block whose maximum is 3 (scale 2^(1-8) = 2^-7): value / scale = 128 * h
+    h = np.zeros((1, 32))
+    h[0, 0] = 230.4 / 128.0     # between the codes 224 and 240, 1.6 from their midpoint
+    h[0, 1] = 3.0               # the maximum (code 384)
+    h[0, 2] = 232.0 / 128.0     # exactly the midpoint of 224 and 240 (spacing 16)
+    slack = np.full((1, 32), 1e-6)
+    st = mx_flip_steps(h, slack)
+    assert st[0, 2] == 16.0 / 128.0   # one E4M3 step, in h units
+    assert st[0, 0] == 0.0 and st[0, 1] == 0.0 and np.count_nonzero(st) == 1
+    # a block maximum within its slack of a power of two: the whole block is uncertain
+    h2 = h.copy()
+    h2[0, 1] = 4.0 * (1 - 1e-9)
+    st2 = mx_flip_steps(h2, slack)
+    assert np.all(st2[0, :3] > 0) and st2[0, 1] >= 4.0 / 8 * (1 - 1e-9)
+
+
+def test_mx_certification_rejects_an_unexplained_error():
+    import pytest
+    from oracle import oracle
+    from parity import certify_mx_flips, compact_weights
+    w = configs.MoEWorkload("mx_cert", T=40, H=64, D=64, E=4, top_k=2, block_m=16, D_shared=32, sigma_w=0.1)
+    inp = gen.make_inputs(w)
+    res = oracle.forward(inp, w.top_k, w.block_m, mxfp8=True)
+    tok = np.arange(w.T)
+    cw = compact_weights(inp, np.arange(w.E))
+    g_out = res["out"].copy()
+    g_out[5, 7] += 0.05 * np.abs(res["out"]).max()  # 5% off in one element, no flip explains it
+    with pytest.raises(AssertionError, match="exceed the tolerance"):
+        certify_mx_flips(inp["x"], cw, tok, res["topk_ids"], res["topk_w"], res["kept"], g_out, res["out"], 1e-2, w)
+    g_out[5, 7] = res["out"][5, 7]
+    for t in range(3):  # too many tokens over the tolerance at all
+        g_out[t, 0] += 0.05 * np.abs(res["out"]).max()
+    with pytest.raises(AssertionError, match="over the tolerance"):
+        certify_mx_flips(inp["x"], cw, tok, res["topk_ids"], res["topk_w"], res["kept"], g_out, res["out"], 1e-2, w)
