@@ -192,6 +192,8 @@ def tile_flags(args) -> int:
         getattr(args, "tiles", "auto")]
     if getattr(args, "sched", "dynamic") == "static":
         f |= native.MOE_FLAG_STATIC_QUOTA
+    if getattr(args, "unfused_small", False):
+        f |= native.MOE_FLAG_UNFUSED_SMALL
     return f
 
 
@@ -212,8 +214,42 @@ def traced_forward(w, wts, x, out, extra_flags=0, wq=None):
     torch.cuda.synchronize()
     rec = layer.trace(1 << 20)
     n_ctas = layer.query(1)
+    res = sm_busy_fraction(rec, n_ctas)
+    if wq is None and layer.query(8) != 3:
+        res["waits"] = wait_fractions(layer.trace_waits(), MoELayer.WAITS)
     layer.close()
-    return sm_busy_fraction(rec, n_ctas)
+    return res
+
+
+def wait_fractions(w: np.ndarray, names) -> dict:
+    """Where each role's issuing thread spent its loop, summed over the CTAs: the fraction of
+    the MMA lane's loop spent waiting for operands, for a free accumulator, for tasks (the rest
+    is issuing MMAs), and likewise for the producer and the epilogue."""
+    if w.size == 0:
+        return {}
+    tot = w.sum(axis=0).astype(np.float64)
+    col = {n: tot[i] for i, n in enumerate(names)}
+    f = lambda a, b: float(col[a] / col[b]) if col[b] > 0 else None
+    return {"mma": {"operands": f("mma_full", "mma_loop"), "accumulator": f("mma_acc", "mma_loop"),
+                    "task": f("mma_task", "mma_loop")},
+            "producer": {"free_stage": f("prod_empty", "prod_loop"), "dependency": f("prod_dep", "prod_loop"),
+                         "ring": f("prod_ring", "prod_loop"), "claim_decode": f("prod_claim", "prod_loop")},
+            "epilogue": {"task": f("epi_task", "epi_loop"), "accumulator": f("epi_acc", "epi_loop")},
+            **({"front_us": front_timeline(w, names)} if col["front_to_end"] > 0 else {})}
+
+
+def front_timeline(w: np.ndarray, names) -> dict:
+    """The fused small-batch forward's front in microseconds: the median CTA's router slice and
+    gather, the schedule's computation in the CTA that did it, the median wait for it, and the
+    median time from the front's start to the end of the epilogue loop."""
+    c = {n: w[:, i] for i, n in enumerate(names)}
+    last = c["front_last"] == 1
+    med = lambda v: float(np.median(v) / 1e3) if v.size else None
+    steps = {n[6:]: med(c[n][last]) for n in names if n.startswith("sched_")}
+    return {"router": med(c["front_router"]), "schedule_compute": med(c["front_schedule"][last]),
+            "schedule_steps": steps, "schedule_wait": med(c["front_schedule"][~last]),
+            "gather": med(c["front_gather"]), "front_to_end": med(c["front_to_end"]),
+            "max_front_to_end": float(c["front_to_end"].max() / 1e3)}
 
 
 def routing_stats(layer, w, dev):
@@ -475,7 +511,8 @@ def measure(w, dev, world, rank, steps, warmup, peaks, flusher, mx=False, flags=
     rc, st = layer.status()
     assert rc == 0 and st == 0, (w.name, rc, st)
     stats = routing_stats(layer, w, dev)
-    shape = {"tile_m": layer.query(6), "workers": layer.query(1), "shape": layer.query(8), "scheduler": sched}
+    shape = {"tile_m": layer.query(6), "workers": layer.query(1), "shape": layer.query(8), "scheduler": sched,
+             "kernels_per_forward": layer.query(11)}
     with ClockSampler(dev.index if dev.index is not None else 0) as clk:
         ms = timed_steps(layer, x, wts, out, wq, steps, stream, world)
     ms_flushed = timed_steps(layer, x, wts, out, wq, steps, stream, world, flusher)
@@ -609,8 +646,31 @@ def compact(entry):
     return d
 
 
+def run_profile(args, local):
+    """--profile: the workload's warm-up and K timed forwards and nothing else (no flushed pass,
+    no per-kernel timing pass, no host-buffer legs, no traced forward), for profiler captures."""
+    from mixture_experts_layer_block_b200.native import MOE_FLAG_MXFP8, MoELayer
+    dev = torch.device("cuda", local)
+    w = workload_of(args)
+    mx = args.precision == "mxfp8"
+    wts = gen.make_weights(w, dev)
+    x = gen.make_x(w, dev)
+    out = torch.empty((w.T, w.H), dtype=torch.float32, device=dev)
+    layer = MoELayer.for_workload(w, flags=(MOE_FLAG_MXFP8 if mx else 0) | tile_flags(args))
+    wq = layer.quantize_experts_mxfp8(wts) if mx else None
+    for _ in range(args.warmup):
+        run_forward(layer, x, wts, out, wq)
+    torch.cuda.synchronize()
+    ms = timed_steps(layer, x, wts, out, wq, args.steps, torch.cuda.current_stream(dev), 1)
+    rc, st = layer.status()
+    assert rc == 0 and st == 0, (rc, st)
+    print(json.dumps({"profile": True, "workload": w.name, "T": w.T, "E": w.E, "precision": args.precision,
+                      "ms_per_step": ms, "kernels_per_forward": layer.query(11)}))
+    layer.close()
+    return 0
+
+
 def run_mine(args, world, rank, local):
-    from mixture_experts_layer_block_b200.native import MoELayer
     dev = torch.device("cuda", local)
     peaks, peak_src = load_peaks()
     flusher = Flusher(dev)
@@ -648,7 +708,8 @@ def run_mine(args, world, rank, local):
             "tflops": head["tflops"], "tflops_frac_of_bf16_peak": head["tflops"] / peaks["bf16_tflops"],
             "stage_ms": head["stage_ms"], "routing": head["routing"], "roofline": roof,
             "layer_roofline": head["layer_roofline"], "layer_roofline_l2_flushed": head["layer_roofline_l2_flushed"],
-            "e2e": e2e, "gpu_launches": len(MoELayer.STAGES) * args.steps, "gemm_shape": head["gemm_shape"],
+            "e2e": e2e, "gpu_launches": head["gemm_shape"]["kernels_per_forward"] * args.steps,
+            "gemm_shape": head["gemm_shape"],
             "clocks": head["clocks"]}
     if "scheduler" in head:
         line["scheduler"] = head["scheduler"]
@@ -704,15 +765,21 @@ def main():
     ap.add_argument("--sched", choices=["dynamic", "static"], default="dynamic",
                     help="task scheduling of the expert GEMMs: the atomic queue, or the static "
                          "per-expert SM quota baseline (ablation)")
+    ap.add_argument("--unfused-small", action="store_true",
+                    help="run batches of at most 16 tokens as six kernels instead of one fused launch")
     ap.add_argument("--precision", choices=["bf16", "mxfp8"], default="bf16",
                     help="expert weights and activations in bf16, or MXFP8 (E4M3, 32-element blocks)")
     ap.add_argument("--traffic-bytes", type=float, default=None,
                     help="ncu dram bytes per launch of the expert-GEMM kernel, if captured")
+    ap.add_argument("--profile", action="store_true",
+                    help="only the warm-up and the K timed forwards of --workload (for profiler captures)")
     args = ap.parse_args()
     world, rank, local = dist_setup()
     try:
         if args.impl == "reference":
             return run_reference(args, world, rank)
+        if args.profile:
+            return run_profile(args, local)
         return run_mine(args, world, rank, local)
     finally:
         if world > 1:

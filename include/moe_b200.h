@@ -88,6 +88,17 @@ extern "C" {
 /* Allocate the MXFP8 workspace at moe_init (x and h quantised to MXFP8, with their scales), for
  * moe_forward_mxfp8. Needs H, D and D_shared multiples of 128 (else MOE_ERR_UNSUPPORTED). */
 #define MOE_FLAG_MXFP8        512u
+/* Batches of at most 16 tokens normally run as ONE launch (on devices that allow a cooperative
+ * launch of one CTA per SM, and with E <= 256): every CTA computes the router logits of a slice
+ * of the experts, the last one to finish takes the gating and the align and publishes the
+ * schedule, every CTA gathers its share of the x rows, then all claim the expert-GEMM tasks, and
+ * the CTA that finishes the last down task of a 256-column block combines that block for every
+ * token (moe_query 11 reports 1 kernel). MOE_FLAG_UNFUSED_SMALL runs such batches as the six
+ * separate kernels instead. The fused router (fp32 on the CUDA cores) sums each logit in
+ * another order than the separate router kernel (fp32 on the tensor cores): logits and gating
+ * weights differ in the last bits, and an exact near-tie may go the other way; both are
+ * deterministic. */
+#define MOE_FLAG_UNFUSED_SMALL 1024u
 
 typedef struct moe_config {
     int32_t hidden;           /* H: model dimension; multiple of 8 */
@@ -292,8 +303,9 @@ MOE_API int moe_debug_expert_rows(moe_handle *h, void *h_rows, void *y_rows, int
  * call (the first 256 of them; needs MOE_FLAG_STAGE_TIMING; synchronises, then starts a new
  * recording window): ms[0] router, ms[1] gating, ms[2] align scatter, ms[3] row gather,
  * ms[4] expert GEMMs, ms[5] combine. n = entries of ms (up to 6). Each duration is measured
- * with CUDA events recorded on the forward's stream around the kernel. MOE_ERR_NOT_READY
- * when nothing was recorded. */
+ * with CUDA events recorded on the forward's stream around the kernel; a fused small batch
+ * (one launch) is timed whole in ms[4], with 0 in the others. MOE_ERR_NOT_READY when nothing
+ * was recorded. */
 MOE_API int moe_stage_times(moe_handle *h, float *ms, int32_t n);
 
 /* Handle facts: which = 0 SM count, 1 workers of the last forward's expert GEMMs (CTAs on
@@ -303,13 +315,31 @@ MOE_API int moe_stage_times(moe_handle *h, float *ms, int32_t n);
  * (128 or 256), 7 SM pairs the device can run at once for the pair shape (0 = none),
  * 8 expert-GEMM shape of the last forward (0 general, 1 small-tile, 2 tail, 3 SM pairs,
  * 4 MXFP8), 9 rows of the per-row buffers of moe_debug_expert_rows, 10 their h row stride
- * (elements, max(D, D_shared)). */
+ * (elements, max(D, D_shared)), 11 kernels the last forward launched (1 for a fused small
+ * batch, else 6), 12 whether batches of at most 16 tokens run fused on this handle (1) or not. */
 MOE_API int moe_query(const moe_handle *h, int32_t which, int64_t *value);
 
 /* Per-task trace of the last forward (needs MOE_FLAG_TRACE; synchronises). Fills up to
  * `cap` records of 4 int64 each: {cta, task, t_claim_ns, t_done_ns} (device globaltimer),
  * sets *n to the records written. */
 MOE_API int moe_trace_read(moe_handle *h, int64_t *records, int64_t cap, int64_t *n);
+
+/* Wait accounting of the last bf16 forward's expert-GEMM kernel (needs MOE_FLAG_TRACE;
+ * synchronises): per CTA (row) int64 %globaltimer ns summed over its tasks --
+ *   0 producer waiting for a free operand stage     1 producer waiting for a down task's up
+ *   2 producer waiting for a free task-ring entry      tasks (fused: for a tile's gathered rows)
+ *   3 producer claiming and decoding tasks           4 MMA lane waiting for a filled stage
+ *   5 MMA lane waiting for a free accumulator        6 MMA lane waiting for the next task
+ *   7 epilogue waiting for the next task             8 epilogue waiting for a finished accumulator
+ *   9 / 10 / 11 the producer / MMA / epilogue loop durations;
+ * and for a fused small batch: 12 the CTA's router slice, 13 waiting for the schedule (or, in
+ * the CTA that computed it, computing it), 14 its share of the row gather, 15 1 for the CTA that
+ * computed the schedule, 16 from the start of the front to the end of the epilogue loop,
+ * and in the CTA that computed the schedule its steps: 17 the arrival count, 18 loading the
+ * logits, 19 gating, 20 the count / offset / tile / unit tables, 21 the writes of sorted_ids,
+ * the sentinels, expert_ids and the task table, 22 publishing the schedule. (23 per row.) Writes up to `rows` rows (at most one per SM) into the host buffer
+ * `waits` and their number to *n_rows. The SM-pair and MXFP8 kernels leave zeros. */
+MOE_API int moe_trace_waits(moe_handle *h, int64_t *waits, int32_t rows, int32_t *n_rows);
 
 /* Testing hook: when `extra` > 0, the down-projection tasks of the next moe_forward wait
  * for `extra` more up-projection completions than can ever arrive, so their bounded wait

@@ -18,6 +18,7 @@ namespace moe {
 cudaError_t configure_router_kernel();
 cudaError_t configure_gemm_kernel();
 cudaError_t configure_gemm_pair_kernel(int* max_pairs);
+int small_fused_blocks_per_sm();
 }  // namespace moe
 
 using namespace moe;
@@ -72,6 +73,9 @@ struct moe_handle {
   int max_pairs = 0;                       // 2-CTA clusters of the pair kernel that fit at once
   int last_workers = 0, last_tile_m = kBM;
   int last_shape = 0;  // expert-GEMM shape of the last forward: 0 general, 1 small, 2 tail, 3 pair
+  int last_kernels = 0;  // kernels launched by the last forward
+  bool fused_ok = false;  // batches of <= 16 tokens may run as one fused launch on this device
+  int32_t epoch = 0;      // fused forwards launched (the schedule flag's value of the last one)
   int parts_rows = 0;  // rows of the K-split partial logits buffer
   std::vector<cudaEvent_t> ev;  // kTimingRing x (kNumStages + 1) events around the kernels
   int timed = 0;                // forwards recorded since the last moe_stage_times
@@ -306,6 +310,11 @@ int moe_init(const moe_config* cfg, moe_handle** out) {
       {(void**)&w.xs, (size_t)h->routed_rows * c.hidden * 2},
       {(void**)&w.y, (size_t)h->tile_rows * c.hidden * 2},
       {(void**)&w.trace, (size_t)trace_cap * 4 * 8},
+      {(void**)&w.waits, (c.flags & MOE_FLAG_TRACE) ? (size_t)h->num_sms * kNumWaits * 8 : 0},
+      {(void**)&w.task_tab, (size_t)h->max_tiles * n_task_max * sizeof(int4)},
+      {(void**)&w.front, sizeof(FrontSync)},
+      {(void**)&w.col_done, (size_t)ceil_div(c.hidden, kBN2) * 4},
+      {(void**)&w.gather_done, (size_t)h->max_tiles * 4},
       {(void**)&h->x_stage, (c.flags & MOE_FLAG_HOST_STAGING) ? 2 * T_ * c.hidden * 2 : 0},
       {(void**)&h->out_stage, (c.flags & MOE_FLAG_HOST_STAGING) ? 2 * T_ * c.hidden * 4 : 0},
       // MXFP8: codes plus scales (1 byte per 32 elements); token rows padded to whole atoms
@@ -329,6 +338,7 @@ int moe_init(const moe_config* cfg, moe_handle** out) {
     off += (p.bytes + 255) & ~size_t(255);
   }
   w.trace_cap = trace_cap;
+  w.task_cap = h->max_tiles * n_task_max;
   w.ldh = ldh;
   h->x_slot_bytes = T_ * c.hidden * 2;
   h->out_slot_bytes = T_ * c.hidden * 4;
@@ -403,6 +413,11 @@ int moe_init(const moe_config* cfg, moe_handle** out) {
   if (check_cuda(raise_align_smem(h->gate_smem, h->gate_smem, scatter_smem))) return fail(MOE_ERR_CUDA);
   if (check_cuda(configure_router_kernel()) || check_cuda(configure_gemm_kernel())) return fail(MOE_ERR_CUDA);
   if (check_cuda(configure_gemm_pair_kernel(&h->max_pairs))) return fail(MOE_ERR_CUDA);
+  // the fused small-batch forward needs one resident CTA per SM at once (cooperative launch)
+  int coop = 0;
+  if (cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, h->device) != cudaSuccess) return fail(MOE_ERR_CUDA);
+  h->fused_ok = coop != 0 && E <= kFusedMaxExperts && small_fused_blocks_per_sm() >= 1 &&
+                !(c.flags & MOE_FLAG_UNFUSED_SMALL) && !(c.flags & MOE_FLAG_STATIC_QUOTA);
   h->max_pairs = std::min(h->max_pairs, h->num_sms / 2);
   h->last_workers = h->num_sms;
   if (h->timing) {
@@ -476,8 +491,10 @@ static int forward_impl(moe_handle* h, const void* x, int32_t T, const void* w_r
 
   const int E = c.num_experts, H = c.hidden, D = c.inter, Ds = c.inter_shared;
   // With at most 16 tokens every m-tile has at most 16 rows (an expert appears once per token):
-  // the expert GEMMs use their small-tile shape with 16-row A boxes.
+  // the expert GEMMs use their small-tile shape with 16-row A boxes, and the whole forward runs
+  // as one fused launch where the device allows it.
   const bool small = T <= kSmallRows;
+  const bool fused = small && h->fused_ok;
   bool pair = false;
   // The pair shape is chosen only on request: on the measured workloads (skewed routing, and
   // 256 experts x top-8 with a shared expert) it was slower than single SMs, whose operand rings
@@ -552,6 +569,35 @@ static int forward_impl(moe_handle* h, const void* x, int32_t T, const void* w_r
   if (h->timing && h->timed < kTimingRing) ev = &h->ev[(size_t)h->timed++ * (kNumStages + 1)];
   auto mark = [&](int i) { return (ev && cudaEventRecord(ev[i], st) != cudaSuccess) ? MOE_ERR_CUDA : MOE_OK; };
   const uint16_t* x16 = static_cast<const uint16_t*>(x);
+  // tracing: the per-CTA wait accounting of this forward starts from zero
+  if (w.waits && cudaMemsetAsync(w.waits, 0, (size_t)h->num_sms * kNumWaits * 8, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (fused) {
+    // one launch: the stage events before it time nothing, the expert-GEMM slot times the launch
+    for (int i = 0; i <= 4; ++i)
+      if ((rc = mark(i))) return rc;
+    FrontArgs fa{};
+    fa.x = x16;
+    fa.w_router = static_cast<const uint16_t*>(w_router);
+    fa.bias = router_bias;
+    fa.out = out;
+    fa.out_bf16 = (c.flags & MOE_FLAG_OUT_BF16) ? 1 : 0;
+    fa.epoch = h->epoch + 1;
+    const cudaError_t le = launch_moe_small_fused(maps, w, sh, fa, h->num_sms, st);
+    if (le == cudaSuccess) {
+      h->epoch = fa.epoch;
+      h->last_kernels = 1;
+      if ((rc = mark(5))) return rc;
+      return mark(6);
+    }
+    // the device refused the cooperative launch (nothing ran): the separate kernels from now on
+    cudaGetLastError();
+    h->fused_ok = false;
+    if (ev) --h->timed;
+    h->dep_extra_next = sh.dep_extra;
+    return forward_impl(h, x, T, w_router, router_bias, w_up, w_gate, w_down, w_shared, top_k, out, st);
+  }
+  h->last_kernels = 6;
   if ((rc = mark(0))) return rc;
   int splits = router_splits(T, E, H, bn, h->num_sms);
   while (splits > 1 && (int64_t)splits * T > h->parts_rows) splits /= 2;
@@ -633,6 +679,7 @@ int moe_forward_mxfp8(moe_handle* h, const void* x, int32_t T, const void* w_rou
   sh.dep_extra = h->dep_extra_next;
   h->dep_extra_next = 0;
   h->last_shape = 4;
+  h->last_kernels = 6;
   h->last_workers = h->num_sms;
   h->last_tile_m = kBM;
   h->last_lag = sh.lag;
@@ -942,6 +989,8 @@ int moe_query(const moe_handle* h, int32_t which, int64_t* value) {
     case 8: *value = h->last_shape; return MOE_OK;
     case 9: *value = h->tile_rows; return MOE_OK;
     case 10: *value = h->ws.ldh; return MOE_OK;
+    case 11: *value = h->last_kernels; return MOE_OK;
+    case 12: *value = h->fused_ok ? 1 : 0; return MOE_OK;
     default: return MOE_ERR_INVALID_ARG;
   }
 }
@@ -956,6 +1005,19 @@ int moe_trace_read(moe_handle* h, int64_t* records, int64_t cap, int64_t* n) {
   if (m > 0 && cudaMemcpy(records, h->ws.trace, (size_t)m * 4 * 8, cudaMemcpyDeviceToHost) != cudaSuccess)
     return MOE_ERR_CUDA;
   *n = m;
+  return MOE_OK;
+}
+
+int moe_trace_waits(moe_handle* h, int64_t* waits, int32_t rows, int32_t* n_rows) {
+  if (!h || !waits || !n_rows || rows < 0) return MOE_ERR_INVALID_ARG;
+  if (!h->ws.waits || !h->have_forward) return MOE_ERR_NOT_READY;
+  int rc;
+  if ((rc = select_device(h))) return rc;
+  if (cudaStreamSynchronize(h->last_stream) != cudaSuccess) return MOE_ERR_CUDA;
+  const int m = std::min(rows, h->num_sms);
+  if (m > 0 && cudaMemcpy(waits, h->ws.waits, (size_t)m * kNumWaits * 8, cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  *n_rows = m;
   return MOE_OK;
 }
 

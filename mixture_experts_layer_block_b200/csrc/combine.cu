@@ -45,29 +45,6 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-__device__ __forceinline__ void add_bf16x8(float (&acc)[8], const uint4 v) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    acc[2 * i] += __uint_as_float(w[i] << 16);
-    acc[2 * i + 1] += __uint_as_float(w[i] & 0xffff0000u);
-  }
-}
-
-// Stores 8 consecutive sums at element `off` of `out`: fp32, or bf16 rounded to nearest even.
-template <bool kBf16>
-__device__ __forceinline__ void store8(void* out, size_t off, const float (&a)[8]) {
-  if constexpr (kBf16) {
-    *reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + off) =
-        make_uint4(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]), pack_bf16x2(a[4], a[5]),
-                   pack_bf16x2(a[6], a[7]));
-  } else {
-    float4* o = reinterpret_cast<float4*>(static_cast<float*>(out) + off);
-    o[0] = make_float4(a[0], a[1], a[2], a[3]);
-    o[1] = make_float4(a[4], a[5], a[6], a[7]);
-  }
-}
-
 // One warp per (token, 512 columns); each lane sums 8 columns in each 256-column half.
 template <bool kBf16>
 __global__ void __launch_bounds__(256)

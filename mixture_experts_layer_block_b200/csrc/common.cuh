@@ -45,6 +45,7 @@ constexpr int kMaxChunks = 32;     // token chunks of the histogram (chunk = cei
 constexpr int kMinChunkTokens = 64;
 constexpr int kGateTokensPerCta = 16;  // gating CTAs: 16 warps x 1 token
 constexpr int kMaxExperts = 1024;
+constexpr int kFusedMaxExperts = 256;  // the fused small-batch forward's gating holds 8 logits per lane
 
 // ---- device status word --------------------------------------------------------------------
 constexpr int kStatusTimeout = 1 << 30;     // | where-code
@@ -59,6 +60,7 @@ enum WaitSite : int {
   kSiteEpiAcc = 8,
   kSiteDrain = 9,
   kSiteRouter = 10,
+  kSiteFront = 11,  // fused small-batch forward: the schedule was not published in time
 };
 
 // Counters and scalars that live in device memory (one int each).
@@ -76,6 +78,47 @@ struct DeviceMeta {
   int num_groups;     // scheduling groups of up to kGroupTiles tiles of one expert
   int num_routed_groups;  // groups of routed experts (shared-expert groups follow them)
   int pad[4];
+};
+
+// The fused small-batch forward's two synchronisation words, each on a 128-byte line of its own
+// (the CTAs poll the flag while the scheduling CTA writes the DeviceMeta fields).
+struct FrontSync {
+  int front_done;      // CTAs that finished their router slice
+  int pad0[31];
+  int sched_flag;      // number of the last forward whose schedule is published (the CTAs wait
+                       // for their forward's number)
+  int pad1[31];
+};
+
+// Per-CTA wait accounting of the expert-GEMM kernel while tracing (ns of %globaltimer, summed
+// over the CTA's tasks): what each role's issuing thread waited for, and how long its loop ran.
+enum WaitKind : int {
+  kWaitProdEmpty = 0,  // producer: a free operand stage
+  kWaitProdDep = 1,    // producer: a down task's up tasks (or, fused, a tile's gathered rows)
+  kWaitProdRing = 2,   // producer: a free task-ring entry
+  kWaitProdClaim = 3,  // producer: claiming and decoding the next task
+  kWaitMmaFull = 4,    // MMA lane: a filled operand stage
+  kWaitMmaAcc = 5,     // MMA lane: a free accumulator (the epilogue of the task before)
+  kWaitMmaTask = 6,    // MMA lane: the next task
+  kWaitEpiTask = 7,    // epilogue: the next task
+  kWaitEpiAcc = 8,     // epilogue: a finished accumulator
+  kWaitProdLoop = 9,   // producer loop duration
+  kWaitMmaLoop = 10,   // MMA loop duration
+  kWaitEpiLoop = 11,   // epilogue loop duration
+  // the fused small-batch forward's front, per CTA (0 for the other kernels)
+  kFrontRouter = 12,   // this CTA's router slice
+  kFrontSchedule = 13, // waiting for the schedule, or (the last CTA) computing it
+  kFrontGather = 14,   // this CTA's share of the row gather
+  kFrontLast = 15,     // 1 for the CTA that computed the schedule
+  kFrontToEnd = 16,    // from the front's start to the end of the epilogue loop
+  // the scheduling CTA's steps (0 elsewhere)
+  kSchedArrive = 17,   // arrival count and CTA barrier
+  kSchedLogits = 18,   // loading every token's logits
+  kSchedGating = 19,   // top-k and softmax of every token
+  kSchedTables = 20,   // counts, offsets, tiles, groups and units (one warp)
+  kSchedWrites = 21,   // sorted_ids, sentinels, expert_ids, task table, counter resets
+  kSchedPublish = 22,  // memory fence, barrier and the flag
+  kNumWaits = 23,
 };
 
 // Task kinds in the ring.
@@ -131,6 +174,24 @@ struct Workspace {
   int64_t* trace;        // [trace_cap][4]
   int32_t trace_cap;
   int32_t ldh;           // row stride of h in elements (max(D, D_shared))
+  FrontSync* front;      // fused small-batch forward's counters
+  int4* task_tab;        // [task_cap] every task of the forward, decoded (task_entry), or null
+  int32_t task_cap;
+  int64_t* waits;        // [grid][kNumWaits] per-CTA wait accounting while tracing, or null
+  int32_t* col_done;     // [ceil(H / kBN2)]  fused small-batch forward: down tasks finished per
+                         //                   256-column block (the last one combines the block)
+  int32_t* gather_done;  // [max_tiles]       fused small-batch forward: x rows gathered per tile
+};
+
+// What the fused small-batch forward (router, gating, align, gather, expert GEMMs and combine
+// in one launch) reads and writes besides the workspace.
+struct FrontArgs {
+  const uint16_t* x;         // [T][H] bf16
+  const uint16_t* w_router;  // [E][H] bf16
+  const float* bias;         // [E] fp32, or null
+  void* out;                 // [T][H] fp32, or bf16 when out_bf16
+  int32_t out_bf16;
+  int32_t epoch;             // this forward's number: the value of the published schedule flag
 };
 
 // Shapes and knobs of one forward, passed by value.
@@ -227,6 +288,40 @@ __device__ __forceinline__ int find_unit(const int32_t* unit_start, int num_unit
   }
 }
 
+// A task, decoded once by the schedule so that a claim costs one load: {tile, expert, first
+// row, bits}, bits = nrows | nrows2 << 9 | (ntiles == 2) << 18 | kind << 19 | n-tile << 20.
+__host__ __device__ inline int4 task_entry(int kind, int tile, int nt, int ntiles, int expert, int row0, int nrows,
+                                           int nrows2) {
+  return make_int4(tile, expert, row0,
+                   nrows | (nrows2 << 9) | ((ntiles == 2 ? 1 : 0) << 18) | (kind << 19) | (nt << 20));
+}
+
+// Write the entries of unit u's tasks (ids unit_start[u] ...): the up tasks of group u, then the
+// down tasks of group u - lag, in the order decode_task gives them.
+__device__ inline void write_unit_tasks(const Workspace& ws, const Shape& sh, int u, int us, int Mg, int Mgr) {
+  const int gl = u - sh.lag;
+  int tau = us;
+  for (int part = 0; part < 2; ++part) {
+    const int g = part == 0 ? u : gl;
+    if (g < 0 || g >= Mg) continue;
+    const int gt = __ldcg(&ws.group_tasks[g]), t0 = __ldcg(&ws.group_tile0[g]), nt_ = __ldcg(&ws.group_ntiles[g]);
+    const int ntiles = gt == 1 ? nt_ : 1;
+    int ex[2], r0[2], nr[2];
+    for (int i = 0; i < gt; ++i) {
+      ex[i] = __ldcg(&ws.tile_expert[t0 + i]);
+      r0[i] = __ldcg(&ws.tile_row0[t0 + i]);
+      nr[i] = __ldcg(&ws.tile_nrows[t0 + i]);
+    }
+    const int nr2 = ntiles == 2 ? __ldcg(&ws.tile_nrows[t0 + 1]) : 0;
+    const int n = part == 0 ? ceil_div(g < Mgr ? sh.D : sh.Ds, kBN1) : ceil_div(sh.H, kBN2);
+    for (int o = 0; o < n * gt; ++o) {
+      const int i = o % gt;
+      ws.task_tab[tau++] = task_entry(part == 0 ? kTaskUp : kTaskDown, t0 + i, o / gt, ntiles, ex[i], r0[i], nr[i],
+                                      ntiles == 2 ? nr2 : 0);
+    }
+  }
+}
+
 // Position of task `tau` of unit `u`: unit u holds the up tasks of group u, then the down tasks
 // of group u - lag; inside a group the tasks run n-major over its tiles.
 struct TaskPos {
@@ -301,6 +396,31 @@ __device__ __forceinline__ void drain_fills(uint64_t* full, int nstages, uint32_
     if (nfill <= static_cast<uint32_t>(s)) break;
     const uint32_t fills = (nfill - 1u - s) / nstages + 1u;
     wait_bar_drain(&full[s], (fills - 1u) & 1u, meta, limit_ns);
+  }
+}
+
+// ---- rows of bf16 values summed in fp32 (the combine) -----------------------------------------
+// acc[i] += the i-th of 8 bf16 values packed in v (widened exactly).
+__device__ __forceinline__ void add_bf16x8(float (&acc)[8], const uint4 v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    acc[2 * i] += __uint_as_float(w[i] << 16);
+    acc[2 * i + 1] += __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
+// Stores 8 consecutive sums at element `off` of `out`: fp32, or bf16 rounded to nearest even.
+template <bool kBf16>
+__device__ __forceinline__ void store8(void* out, size_t off, const float (&a)[8]) {
+  if constexpr (kBf16) {
+    *reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + off) =
+        make_uint4(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]), pack_bf16x2(a[4], a[5]),
+                   pack_bf16x2(a[6], a[7]));
+  } else {
+    float4* o = reinterpret_cast<float4*>(static_cast<float*>(out) + off);
+    o[0] = make_float4(a[0], a[1], a[2], a[3]);
+    o[1] = make_float4(a[4], a[5], a[6], a[7]);
   }
 }
 

@@ -25,12 +25,13 @@
 #include <mutex>
 
 #include "launch.h"
+#include "route.cuh"
 
 namespace moe {
 
 // ------------------------------------------------------------------------------------------
-// warp top-k + renormalised softmax of one token held in registers; lane j < k returns
-// choice j
+// one token's logits (the sum of the router's S K-split partials, in split order) into the
+// registers of a warp: lane l holds experts l, l + 32, ...
 // ------------------------------------------------------------------------------------------
 template <int VPL, int S>
 __device__ __forceinline__ void load_token(const float* __restrict__ row, size_t part_stride, int E,
@@ -49,261 +50,6 @@ __device__ __forceinline__ void load_token(const float* __restrict__ row, size_t
 #pragma unroll
     for (int s = 1; s < S; ++s) a += p[s][j];
     v[j] = (lane + 32 * j < E) ? a : -INFINITY;
-  }
-}
-
-template <int VPL>
-__device__ __forceinline__ void warp_topk_softmax(const float (&v)[VPL], int E, int k, int lane,
-                                                  int& out_id, float& out_w) {
-  uint32_t taken = 0;
-#pragma unroll
-  for (int j = 0; j < VPL; ++j)
-    if (lane + 32 * j >= E) taken |= 1u << j;
-  float my_v = 0.f, top_v = 0.f;
-  int my_id = -1;
-  for (int r = 0; r < k; ++r) {
-    float bv = -INFINITY;
-    int bi = INT_MAX;
-#pragma unroll
-    for (int j = 0; j < VPL; ++j) {
-      const int e = lane + 32 * j;
-      if (!((taken >> j) & 1u) && (v[j] > bv || (v[j] == bv && e < bi))) {
-        bv = v[j];
-        bi = e;
-      }
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-      if (ov > bv || (ov == bv && oi < bi)) {
-        bv = ov;
-        bi = oi;
-      }
-    }
-    if (bi != INT_MAX && (bi & 31) == lane) taken |= 1u << (bi >> 5);
-    if (lane == r) {
-      my_v = bv;
-      my_id = bi;
-    }
-    if (r == 0) top_v = bv;
-  }
-  const float ex = (lane < k) ? expf(my_v - top_v) : 0.f;
-  float s = ex;
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-  out_id = my_id;
-  out_w = ex / s;
-}
-
-// ------------------------------------------------------------------------------------------
-// block-wide exclusive scan of a[0..n) in shared memory (any n), returns the total.
-// Uses `tmp` (>= blockDim/32 + 1 ints). All threads must call it.
-// ------------------------------------------------------------------------------------------
-__device__ int block_exclusive_scan(int* a, int n, int* tmp) {
-  const int tid = threadIdx.x, nthr = blockDim.x, lane = tid & 31, warp = tid >> 5;
-  const int nwarps = nthr >> 5;
-  int carry = 0;
-  for (int base = 0; base < n; base += nthr * 4) {
-    int loc[4];
-    int sum = 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int idx = base + tid * 4 + i;
-      loc[i] = (idx < n) ? a[idx] : 0;
-      sum += loc[i];
-    }
-    int incl = sum;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += y;
-    }
-    if (lane == 31) tmp[warp] = incl;
-    __syncthreads();
-    if (tid == 0) {
-      int run = 0;
-      for (int w = 0; w < nwarps; ++w) {
-        const int x = tmp[w];
-        tmp[w] = run;
-        run += x;
-      }
-      tmp[nwarps] = run;
-    }
-    __syncthreads();
-    int run = carry + tmp[warp] + incl - sum;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int idx = base + tid * 4 + i;
-      if (idx < n) a[idx] = run;
-      run += loc[i];
-    }
-    carry += tmp[nwarps];
-    __syncthreads();
-  }
-  return carry;
-}
-
-// ------------------------------------------------------------------------------------------
-// The scans, run by the last CTA of the histogram pass. Shared memory layout (ints):
-//   tmp[64] | cnt[E] | kept[E] | offs[E] | tile[kMaxChunks * kScanGroup] | buf[max(E+1, units+1)]
-// Everything the later steps need stays in shared memory (no reads of just-written globals).
-// ------------------------------------------------------------------------------------------
-constexpr int kScanGroup = 256;  // experts scanned per pass (tile of [chunks][256] counts)
-
-__device__ void align_scans(const Workspace& ws, const Shape& sh, bool tiles, int* sm) {
-  const int tid = threadIdx.x, nthr = blockDim.x;
-  const int E = sh.E;
-  int* tmp = sm;
-  int* cnt = tmp + 64;
-  int* kept = cnt + E;
-  int* offs = kept + E;
-  int* tile = offs + E;
-  int* buf = tile + kMaxChunks * kScanGroup;
-  const int nch = sh.num_chunks;
-
-  // 1. per expert: exclusive prefix of the chunk counts (chunk_base) and the total n_e.
-  //    The [chunks][group] block of counts is loaded with independent loads, then each
-  //    thread scans one expert's column in shared memory.
-  for (int g0 = 0; g0 < E; g0 += kScanGroup) {
-    const int G = min(kScanGroup, E - g0);
-    const int n = nch * G;
-#pragma unroll 4
-    for (int i = tid; i < n; i += nthr) {
-      const int c = i / G, e = i - c * G;
-      int* p = ws.chunk_hist + (size_t)c * E + g0 + e;
-      tile[i] = __ldcg(p);
-      *p = 0;  // the histograms start from zero at the next call
-    }
-    __syncthreads();
-    if (tid < G) {
-      int run = 0;
-      for (int c = 0; c < nch; ++c) {
-        const int v = tile[c * G + tid];
-        ws.chunk_base[(size_t)c * E + g0 + tid] = run;
-        run += v;
-      }
-      cnt[g0 + tid] = run;
-    }
-    __syncthreads();
-  }
-
-  // 2. capacity cut and padded segment lengths
-  for (int e = tid; e < E; e += nthr) {
-    const int n = cnt[e];
-    const int kp = (sh.capacity > 0) ? min(n, sh.capacity) : n;
-    kept[e] = kp;
-    ws.expert_kept[e] = kp;
-    buf[e] = ceil_div(kp, sh.block_m) * sh.block_m;
-  }
-  __syncthreads();
-  const int P = block_exclusive_scan(buf, E, tmp);
-  for (int e = tid; e < E; e += nthr) {
-    ws.expert_off[e] = buf[e];
-    offs[e] = buf[e];
-  }
-  if (tid == 0) {
-    ws.expert_off[E] = P;
-    ws.meta->P = P;
-  }
-  __syncthreads();
-  if (!tiles) return;
-
-  // 3. m-tiles of tile_m rows: routed experts (ceil(kept/tile_m) each), then the shared expert
-  //    over all tokens
-  const int tm = sh.tile_m;
-  for (int e = tid; e < E; e += nthr) buf[e] = ceil_div(kept[e], tm);
-  __syncthreads();
-  const int Mr = block_exclusive_scan(buf, E, tmp);
-  for (int e = tid; e < E; e += nthr) {
-    const int first = buf[e], nt = ceil_div(kept[e], tm);
-    const int off = offs[e];
-    ws.expert_tile0[e] = first;
-    for (int i = 0; i < nt; ++i) {
-      ws.tile_expert[first + i] = e;
-      ws.tile_row0[first + i] = off + i * tm;
-      ws.tile_nrows[first + i] = min(tm, kept[e] - i * tm);
-    }
-    offs[e] = first;  // the segment offsets are no longer needed: keep the first tile instead
-  }
-  const int Ms = (sh.Ds > 0) ? ceil_div(sh.T, tm) : 0;
-  for (int j = tid; j < Ms; j += nthr) {
-    ws.tile_expert[Mr + j] = E;
-    ws.tile_row0[Mr + j] = j * tm;
-    ws.tile_nrows[Mr + j] = min(tm, sh.T - j * tm);
-  }
-  const int Mt = Mr + Ms;
-  __syncthreads();
-
-  // 3b. scheduling groups: up to kGroupTiles consecutive tiles of one expert (the shared
-  //     expert's tiles are grouped the same way)
-  for (int e = tid; e < E; e += nthr) buf[e] = ceil_div(ceil_div(kept[e], tm), kGroupTiles);
-  __syncthreads();
-  const int Mgr = block_exclusive_scan(buf, E, tmp);
-  // A group of two tiles whose second is a tail of at most kTailRows rows runs as one task set
-  // when sh.merge_tail: each task computes both tiles from the same weight stages. With pairs of
-  // tiles, a run of an odd number of tiles that ends in a tail starts with a single-tile group,
-  // so that the tail closes a pair.
-  auto put_group = [&](int gi, int t0, int g, int last_rows) {
-    ws.group_tile0[gi] = t0;
-    ws.group_ntiles[gi] = g;
-    ws.group_tasks[gi] = (sh.merge_tail && g == 2 && last_rows <= kTailRows) ? 1 : g;
-  };
-  // tiles [start, start + g) of group j of a run of nt tiles whose last tile has last_rows rows
-  auto group_span = [&](int j, int nt, int last_rows, int& start, int& g) {
-    const int f = (kGroupTiles == 2 && sh.merge_tail && nt > 1 && (nt & 1) && last_rows <= kTailRows) ? 1 : 0;
-    start = (f && j > 0) ? kGroupTiles * j - 1 : kGroupTiles * j;
-    g = (f && j == 0) ? 1 : min(kGroupTiles, nt - start);
-  };
-  for (int e = tid; e < E; e += nthr) {
-    const int nt = ceil_div(kept[e], tm), first = offs[e], g0 = buf[e];
-    const int last_rows = kept[e] - (nt - 1) * tm;
-    ws.expert_group0[e] = g0;
-    for (int i = 0; i * kGroupTiles < nt; ++i) {
-      int st, g;
-      group_span(i, nt, last_rows, st, g);
-      put_group(g0 + i, first + st, g, min(tm, kept[e] - (st + g - 1) * tm));
-    }
-  }
-  const int Mgs = ceil_div(Ms, kGroupTiles);
-  for (int j = tid; j < Mgs; j += nthr) {
-    int st, g;
-    group_span(j, Ms, sh.T - (Ms - 1) * tm, st, g);
-    put_group(Mgr + j, Mr + st, g, min(tm, sh.T - (st + g - 1) * tm));
-  }
-  const int Mg = Mgr + Mgs;
-  if (tid == 0) {
-    ws.expert_group0[E] = Mgr;
-    ws.expert_group0[E + 1] = Mg;
-  }
-  __syncthreads();
-
-  // 4. schedule units: unit u holds the up/gate tasks of group u, then the down tasks of group
-  //    u - lag. Task ids are unit-major, so every down task's dependencies have lower ids.
-  const int U = (Mg > 0) ? Mg + sh.lag : 0;
-  const int n2 = ceil_div(sh.H, kBN2);
-  const int n1r = ceil_div(sh.D, kBN1), n1s = ceil_div(sh.Ds, kBN1);
-  for (int u = tid; u < U; u += nthr) {
-    int c = 0;
-    if (u < Mg) c += ((u < Mgr) ? n1r : n1s) * ws.group_tasks[u];  // routed groups first
-    if (u >= sh.lag && u - sh.lag < Mg) c += n2 * ws.group_tasks[u - sh.lag];
-    buf[u] = c;
-  }
-  __syncthreads();
-  const int total = block_exclusive_scan(buf, U, tmp);
-  for (int u = tid; u < U; u += nthr) ws.unit_start[u] = buf[u];
-  for (int i = tid; i < Mt; i += nthr) ws.done1[i] = 0;
-  if (tid == 0) {
-    ws.unit_start[U] = total;
-    ws.meta->num_tiles = Mt;
-    ws.meta->num_routed_tiles = Mr;
-    ws.meta->num_groups = Mg;
-    ws.meta->num_routed_groups = Mgr;
-    ws.meta->num_units = U;
-    ws.meta->total_tasks = total;
-    ws.meta->task_counter = 0;
-    ws.meta->abort = 0;
-    ws.meta->trace_count = 0;
   }
 }
 
@@ -391,17 +137,6 @@ __global__ void __launch_bounds__(kGateThreads)
   }
   __syncthreads();
   finish_histogram(ws, sh, false, hist, t0 / sh.chunk_tokens, smem_i + sh.E);
-}
-
-__device__ __forceinline__ int segment_of(const int* off, int E, int i) {
-  // largest e with off[e] <= i (off non-decreasing, off[E] = P > i)
-  int lo = 0, hi = E;  // answer in [lo, hi)
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (off[mid] <= i) lo = mid;
-    else hi = mid;
-  }
-  return lo;
 }
 
 // smem: off[E+1] | kept[E] | tile0[E] | wcnt[16][E] | ids[chunk slots]
@@ -504,6 +239,15 @@ __global__ void __launch_bounds__(kGateThreads)
     expert_ids[b] = (i < P) ? segment_of(off, E, i) : -1;
   }
   if (gt == 0 && num_post_padded) *num_post_padded = P;
+  // a forward's task table: one thread per scheduling unit, starting with the CTAs that sort no
+  // chunk (the schedule's scans ran in the gating kernel)
+  if (row_of_slot && ws.task_tab) {
+    const int U = __ldcg(&ws.meta->num_units), Mg = __ldcg(&ws.meta->num_groups);
+    const int Mgr = __ldcg(&ws.meta->num_routed_groups);
+    const int first = (int)((blockIdx.x + gridDim.x - min(sh.num_chunks, (int)gridDim.x)) % gridDim.x);
+    for (int u = first * blockDim.x + threadIdx.x; u < U; u += nt)
+      write_unit_tasks(ws, sh, u, __ldcg(&ws.unit_start[u]), Mg, Mgr);
+  }
 }
 
 // ------------------------------------------------------------------------------------------

@@ -91,10 +91,19 @@ cudaError_t launch_combine(void* out, bool bf16_out, const Workspace& ws, const 
 // tails of at most 32 rows merged into the previous tile's tasks; needs sh.merge_tail = 1) and
 // small (batches of at most 16 tokens; its maps use 16-row boxes for x_tile, xs, h_routed and
 // h_shared).
-enum GemmShape : int { kShapeGeneral = 0, kShapeSmall = 1, kShapeTail = 2 };
+enum GemmShape : int { kShapeGeneral = 0, kShapeSmall = 1, kShapeTail = 2, kShapeSmallFused = 3 };
 size_t gemm_smem_bytes(int shape);
 cudaError_t launch_moe_gemm(const GemmMaps& maps, const Workspace& ws, const Shape& sh, int grid, int shape,
                             cudaStream_t stream);
+
+// The whole forward of a batch of at most 16 tokens (and at most 256 experts) as one persistent
+// launch of `grid` CTAs, all resident at once (cooperative launch): every CTA computes the router
+// logits of a slice of the experts; the last to finish takes the gating, the align scans and
+// writes and publishes the schedule; every CTA gathers its share of the x rows, then claims
+// expert-GEMM tasks (small-tile shape) as the standalone kernel does; the CTA that finishes the
+// last down task of a 256-column block combines that block for every token.
+cudaError_t launch_moe_small_fused(const GemmMaps& maps, const Workspace& ws, const Shape& sh,
+                                   const FrontArgs& fa, int grid, cudaStream_t stream);
 
 // The same GEMMs with 256-row m-tiles on `pairs` 2-CTA clusters (sh.tile_m = 256; its maps use
 // 32-row boxes for x_tile, xs, h_routed, h_shared and y, and 128-row boxes for w_down, ws_down).

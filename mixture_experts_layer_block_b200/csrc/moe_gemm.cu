@@ -41,6 +41,7 @@
 // runs out records a status code, sets the abort flag, and every CTA drains its in-flight
 // copies and MMAs and exits.
 #include "launch.h"
+#include "route.cuh"
 
 namespace moe {
 
@@ -57,7 +58,7 @@ namespace {
 // and their results are never stored.
 template <int kShape>
 struct Cfg {
-  static constexpr bool kSmall = (kShape == kShapeSmall);
+  static constexpr bool kSmall = (kShape == kShapeSmall || kShape == kShapeSmallFused);
   static constexpr bool kTail = (kShape == kShapeTail);
   static constexpr int kStagesN = kSmall ? 6 : kStages;
   static constexpr int kARows = kSmall ? 16 : kBM;
@@ -81,13 +82,402 @@ __device__ __forceinline__ int n1_of(int expert, const Shape& sh) {
   return ceil_div(expert == sh.E ? sh.Ds : sh.D, kBN1);
 }
 
+// ---- the fused small-batch forward: the front (router, gating, align, gather) and the combine --
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4 v, float (&f)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
+// Router projection (Mixture-of-Kittens blog, "Overlapping compute and communication in MoE")
+// for this CTA's experts e = blockIdx.x + j * gridDim.x, two at a time: logits[t][e] =
+// sum_h x[t][h] W_router[e][h] (+ bias[e]) in fp32. Each thread takes 8-wide chunks of H for
+// all T <= 16 tokens; the partial sums are added over the warp, then over the warps in warp
+// order. red: shared scratch of [warps][2][16] floats.
+__device__ void front_router(const FrontArgs& fa, const Workspace& ws, const Shape& sh, float* red) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+  const int H = sh.H, E = sh.E, T = sh.T, nchunk = H / 8;
+  for (int e0 = blockIdx.x; e0 < E; e0 += 2 * gridDim.x) {
+    const int e1 = e0 + gridDim.x;
+    const bool two = e1 < E;
+    float a0[kSmallRows], a1[kSmallRows];
+#pragma unroll
+    for (int t = 0; t < kSmallRows; ++t) a0[t] = a1[t] = 0.f;
+    const uint4* w0p = reinterpret_cast<const uint4*>(fa.w_router + (size_t)e0 * H);
+    const uint4* w1p = reinterpret_cast<const uint4*>(fa.w_router + (size_t)(two ? e1 : e0) * H);
+    for (int c = tid; c < nchunk; c += blockDim.x) {
+      // every load of the chunk first (rows past T re-read row T-1; their sums are never used),
+      // so that they are all in flight together
+      uint4 xr[kSmallRows];
+#pragma unroll
+      for (int t = 0; t < kSmallRows; ++t)
+        xr[t] = __ldg(reinterpret_cast<const uint4*>(fa.x + (size_t)min(t, T - 1) * H) + c);
+      const uint4 wr0 = __ldg(w0p + c), wr1 = __ldg(w1p + c);
+      float w0[8], w1[8];
+      bf16x8_to_f32(wr0, w0);
+      bf16x8_to_f32(wr1, w1);
+#pragma unroll
+      for (int t = 0; t < kSmallRows; ++t) {
+        float xv[8];
+        bf16x8_to_f32(xr[t], xv);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          a0[t] = fmaf(w0[i], xv[i], a0[t]);
+          a1[t] = fmaf(w1[i], xv[i], a1[t]);
+        }
+      }
+    }
+    // transpose-reduce the 32 partial sums over the warp (31 shuffles): at each level a lane keeps
+    // the half of its values selected by its lane bit and adds its partner's copy of that half;
+    // lane l ends with the warp's total of value l (values 0-15: expert e0, 16-31: expert e1)
+    float v[2 * kSmallRows];
+#pragma unroll
+    for (int t = 0; t < kSmallRows; ++t) {
+      v[t] = a0[t];
+      v[kSmallRows + t] = a1[t];
+    }
+#pragma unroll
+    for (int sft = 16; sft >= 1; sft >>= 1) {
+      const bool upper = (lane & sft) != 0;
+#pragma unroll
+      for (int i = 0; i < sft; ++i) {
+        const float send = upper ? v[i] : v[i + sft];
+        const float keep = upper ? v[i + sft] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, sft);
+      }
+    }
+    red[warp * 2 * kSmallRows + lane] = v[0];
+    __syncthreads();
+    if (tid < 2 * T) {
+      const int which = tid >= T ? 1 : 0, t = tid - which * T;
+      if (!which || two) {
+        const int e = which ? e1 : e0;
+        float v = 0.f;
+        for (int w = 0; w < nw; ++w) v += red[(w * 2 + which) * kSmallRows + t];
+        if (fa.bias) v += fa.bias[e];
+        ws.logits[(size_t)t * E + e] = v;
+      }
+    }
+    __syncthreads();
+  }
+}
+
+// Exclusive prefix of v over the lanes of warp 0 (lane order); *total = the sum of all lanes.
+__device__ __forceinline__ int warp_exclusive(int v, int lane, int& total) {
+  int incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += y;
+  }
+  total = __shfl_sync(0xffffffffu, incl, 31);
+  return incl - v;
+}
+
+// First task id of unit u when every group is one m-tile (Mg groups, the first Mr routed): the up
+// tasks of the groups before u (ceil(D/128) each for a routed group, ceil(Ds/128) for the
+// shared one) plus the down tasks (ceil(H/256) each) of the groups before u - lag -- the
+// exclusive scan of the unit sizes, in closed form.
+__device__ __forceinline__ int unit_start_of(int u, int Mr, int Mg, const Shape& sh) {
+  const int n1r = ceil_div(sh.D, kBN1), n1s = ceil_div(sh.Ds, kBN1), n2 = ceil_div(sh.H, kBN2);
+  const int ups = min(u, Mg);
+  const int downs = max(0, min(u - sh.lag, Mg));
+  return n1r * min(ups, Mr) + n1s * max(0, ups - Mr) + n2 * downs;
+}
+
+// Run by the CTA that finished its router slice last, once every slice is in. For a batch of
+// at most 16 tokens every expert receives at most 16 slots, so each hit expert has one m-tile
+// and one scheduling group, and the whole schedule fits one warp's scans:
+//  - gating (Weave blog section 1.1: top-k, ties to the lower expert index, softmax
+//    renormalised over the selection), from the logits staged in shared memory;
+//  - the align (vLLM PR #53280 summary, implementation breakdown): per-expert counts, the
+//    capacity cut, padded segment offsets, the stable writes of sorted_ids in ascending slot
+//    order, the padding sentinels and expert_ids;
+//  - the tile and task schedule of the expert GEMMs: the same tables (tiles, groups, units with
+//    the dependency lag) that the align scans write for a larger batch;
+// then the reset of this forward's counters and the schedule flag. sm: shared scratch (ints).
+__device__ void front_schedule(const FrontArgs& fa, const Workspace& ws, const Shape& sh, int* sm, int64_t* ts) {
+  // ts (thread 0, tracing): the end times of the steps, for the wait accounting
+  const bool tracing = ws.trace_cap > 0;
+  auto stamp = [&](int i) {
+    if (tracing && threadIdx.x == 0) ts[i] = (int64_t)globaltimer_ns();
+  };
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5, nthr = blockDim.x;
+  const int E = sh.E, T = sh.T, k = sh.k, S = T * k;
+  int* ids_s = sm;           // [S]
+  int* cnt = ids_s + S;      // [E]
+  int* off = cnt + E;        // [E + 1]
+  int* kept = off + E + 1;   // [E]
+  int* tile0 = kept + E;     // [E]
+  int* run = tile0 + E;      // [E]  running count of the stable writes
+  int* s_mt = run + E;       // [2]  m-tiles, and routed m-tiles, of this forward
+  int* t_exp = s_mt + 2;     // [E + 1] per m-tile: expert, first sorted row, rows
+  int* t_r0 = t_exp + E + 1;
+  int* t_nr = t_r0 + E + 1;
+  for (int e = tid; e < E; e += nthr) {
+    cnt[e] = 0;
+    run[e] = 0;
+  }
+  // gating: warp w takes tokens w, w + nw, w + 2 nw (T <= 16 <= 3 * 6); the logits of all its
+  // tokens are loaded at once (one round trip), then each token's top-k
+  constexpr int kTokPerWarp = 3;
+  float v[kTokPerWarp][8];
+#pragma unroll
+  for (int i = 0; i < kTokPerWarp; ++i) {
+    const int t = min(warp + i * nw, T - 1);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = lane + 32 * j;
+      const float x = __ldcg(ws.logits + (size_t)t * E + min(e, E - 1));
+      v[i][j] = e < E ? x : -INFINITY;
+    }
+  }
+  __syncthreads();
+  stamp(0);
+  {
+    int id[kTokPerWarp];
+    float wt[kTokPerWarp];
+    warp_topk_softmax_n<8, kTokPerWarp>(v, E, k, lane, id, wt);
+#pragma unroll
+    for (int i = 0; i < kTokPerWarp; ++i) {
+      const int t = warp + i * nw;
+      if (t < T && lane < k) {
+        ws.topk_ids[t * k + lane] = id[i];
+        ws.topk_w[t * k + lane] = wt[i];
+        ids_s[t * k + lane] = id[i];
+        atomicAdd(&cnt[id[i]], 1);
+      }
+    }
+  }
+  __syncthreads();
+  stamp(1);
+  if (warp == 0) {
+    // lane l owns experts [8l, 8l + 8) (E <= 256), so lane order is expert order
+    const int e0 = lane * 8;
+    int kp[8], pad = 0, hit = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = e0 + j;
+      const int n = e < E ? cnt[e] : 0;
+      kp[j] = (sh.capacity > 0) ? min(n, sh.capacity) : n;
+      pad += ceil_div(kp[j], sh.block_m) * sh.block_m;
+      hit += kp[j] > 0 ? 1 : 0;
+    }
+    int P, Mr;
+    int o = warp_exclusive(pad, lane, P);
+    int ti = warp_exclusive(hit, lane, Mr);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = e0 + j;
+      if (e < E) {
+        off[e] = o;
+        kept[e] = kp[j];
+        tile0[e] = ti;
+        ws.expert_off[e] = o;
+        ws.expert_kept[e] = kp[j];
+        ws.expert_tile0[e] = ti;
+        ws.expert_group0[e] = ti;  // one tile per group
+        if (kp[j] > 0) {
+          t_exp[ti] = e;
+          t_r0[ti] = o;
+          t_nr[ti] = kp[j];
+          ws.tile_expert[ti] = e;
+          ws.tile_row0[ti] = o;
+          ws.tile_nrows[ti] = kp[j];
+          ws.group_tile0[ti] = ti;
+          ws.group_ntiles[ti] = 1;
+          ws.group_tasks[ti] = 1;
+        }
+        o += ceil_div(kp[j], sh.block_m) * sh.block_m;
+        ti += kp[j] > 0 ? 1 : 0;
+      }
+    }
+    // the shared expert: one tile (and group) of all T tokens after the routed ones
+    const int Ms = sh.Ds > 0 ? 1 : 0, Mt = Mr + Ms, Mg = Mt;
+    if (lane == 0) {
+      off[E] = P;
+      ws.expert_off[E] = P;
+      if (Ms) {
+        t_exp[Mr] = E;
+        t_r0[Mr] = 0;
+        t_nr[Mr] = T;
+        ws.tile_expert[Mr] = E;
+        ws.tile_row0[Mr] = 0;
+        ws.tile_nrows[Mr] = T;
+        ws.group_tile0[Mr] = Mr;
+        ws.group_ntiles[Mr] = 1;
+        ws.group_tasks[Mr] = 1;
+      }
+      ws.expert_group0[E] = Mr;
+      ws.expert_group0[E + 1] = Mg;
+    }
+    const int U = Mg > 0 ? Mg + sh.lag : 0;
+    if (lane == 0) {
+      *s_mt = Mt;
+      s_mt[1] = Mr;
+      DeviceMeta* m = ws.meta;
+      m->P = P;
+      m->num_tiles = Mt;
+      m->num_routed_tiles = Mr;
+      m->num_groups = Mg;
+      m->num_routed_groups = Mr;
+      m->num_units = U;
+      m->total_tasks = unit_start_of(U, Mr, Mg, sh);
+      m->task_counter = 0;
+      m->abort = 0;
+      m->trace_count = 0;
+    }
+  }
+  __syncthreads();
+  stamp(2);
+  const int P = off[E];
+  if (warp == 0) {
+    // slots in ascending order, 32 at a time: a slot's rank in its expert is the expert's running
+    // count plus its rank among this round's lanes of the same expert (stable)
+    for (int base = 0; base < S; base += 32) {
+      const int s = base + lane;
+      const int e = s < S ? ids_s[s] : -1;
+      const unsigned mask = __match_any_sync(0xffffffffu, e);
+      const int rank = __popc(mask & ((1u << lane) - 1u));
+      const int c0 = e >= 0 ? run[e] : 0;
+      __syncwarp();
+      if (e >= 0) {
+        const int r = c0 + rank;
+        const bool keep = sh.capacity == 0 || r < sh.capacity;
+        if (keep) ws.sorted_ids[off[e] + r] = s;
+        ws.row_of_slot[s] = keep ? tile0[e] * sh.tile_m + r : -1;
+        if (rank == 0) run[e] = c0 + __popc(mask);
+      }
+      __syncwarp();
+    }
+  }
+  for (int i = tid; i < sh.sorted_len; i += nthr) {
+    bool padding = true;
+    if (i < P) {
+      const int e = segment_of(off, E, i);
+      padding = (i - off[e]) >= kept[e];
+    }
+    if (padding) ws.sorted_ids[i] = S;
+  }
+  for (int b = tid; b < sh.blocks_len; b += nthr) {
+    const int i = b * sh.block_m;
+    ws.expert_ids[b] = (i < P) ? segment_of(off, E, i) : -1;
+  }
+  const int Mt = *s_mt, Mr = s_mt[1], U = Mt > 0 ? Mt + sh.lag : 0;
+  for (int i = tid; i < Mt; i += nthr) {
+    ws.gather_done[i] = 0;
+    ws.done1[i] = 0;
+  }
+  for (int u = tid; u <= U; u += nthr) ws.unit_start[u] = unit_start_of(u, Mr, Mt, sh);
+  // the task table: one m-tile per group here, so unit u's tasks are the up tasks of tile u, then
+  // the down tasks of tile u - lag (as write_unit_tasks lays them out)
+  if (ws.task_tab) {
+    for (int u = tid; u < U; u += nthr) {
+      int tau = unit_start_of(u, Mr, Mt, sh);
+      if (u < Mt) {
+        const int n1 = ceil_div(u < Mr ? sh.D : sh.Ds, kBN1);
+        for (int nt = 0; nt < n1; ++nt)
+          ws.task_tab[tau++] = task_entry(kTaskUp, u, nt, 1, t_exp[u], t_r0[u], t_nr[u], 0);
+      }
+      const int g = u - sh.lag;
+      if (g >= 0 && g < Mt)
+        for (int nt = 0; nt < ceil_div(sh.H, kBN2); ++nt)
+          ws.task_tab[tau++] = task_entry(kTaskDown, g, nt, 1, t_exp[g], t_r0[g], t_nr[g], 0);
+    }
+  }
+  for (int i = tid; i < ceil_div(sh.H, kBN2); i += nthr) ws.col_done[i] = 0;
+  stamp(3);
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    ws.front->front_done = 0;  // every CTA has arrived: ready for the next forward
+    st_release_gpu(&ws.front->sched_flag, fa.epoch);
+  }
+}
+
+// Bounded wait (one thread) until the schedule of forward `epoch` is published. Only the time
+// limit ends it early: the abort flag may still hold an earlier forward's value until the
+// schedule resets it.
+__device__ bool wait_schedule(const int* flag, int epoch, DeviceMeta* meta, int64_t limit_ns) {
+  // relaxed polls, then one acquire load once the value is there
+  if (ld_acquire_gpu(flag) == epoch) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    __nanosleep(128);
+    if (ld_relaxed_gpu(flag) == epoch && ld_acquire_gpu(flag) == epoch) return true;
+    if (static_cast<int64_t>(globaltimer_ns() - t0) > limit_ns) {
+      raise_error(meta, nullptr, kStatusTimeout | kSiteFront);
+      return false;
+    }
+  }
+}
+
+// This CTA's share of the row gather: the x row of every kept slot s = blockIdx.x + j * gridDim.x
+// into its tile row of xs; each row bumps its tile's gather count (release), which the tile's
+// up tasks wait for before their TMA loads.
+__device__ void front_gather(const FrontArgs& fa, const Workspace& ws, const Shape& sh) {
+  const int S = sh.T * sh.k, nvec = sh.H / 8;
+  for (int s = blockIdx.x; s < S; s += gridDim.x) {
+    const int row = __ldcg(ws.row_of_slot + s);
+    if (row < 0) continue;
+    const uint4* src = reinterpret_cast<const uint4*>(fa.x + (size_t)(s / sh.k) * sh.H);
+    uint4* dst = reinterpret_cast<uint4*>(ws.xs + (size_t)row * sh.H);
+    for (int i = threadIdx.x; i < nvec; i += 2 * blockDim.x) {  // two loads in flight per thread
+      const int i2 = i + blockDim.x;
+      const uint4 a = __ldg(src + i), b = __ldg(src + min(i2, nvec - 1));
+      dst[i] = a;
+      if (i2 < nvec) dst[i2] = b;
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) red_release_add_gpu(ws.gather_done + row / sh.tile_m, 1);
+  }
+}
+
+// The combine of columns [n0, n0 + kBN2) for every token, once every down task of that column
+// block is done: out[t] = y[shared row of t] + sum_j y[row of slot t*k + j], in this order, in
+// fp32 (the standalone combine kernel's order, so the result is the same bit for bit). Thread
+// i < 128: token i / 8, 32 columns.
+__device__ void fused_combine(const FrontArgs& fa, const Workspace& ws, const Shape& sh, int n0, int i, int Mr) {
+  const int t = i >> 3;
+  if (t >= sh.T) return;
+  const int c0 = n0 + (i & 7) * 32;
+  float acc[4][8];
+#pragma unroll
+  for (int v = 0; v < 4; ++v)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[v][j] = 0.f;
+  auto add_row = [&](int row) {
+    const uint16_t* yr = ws.y + (size_t)row * sh.H;
+#pragma unroll
+    for (int v = 0; v < 4; ++v)
+      if (c0 + 8 * v + 8 <= sh.H) add_bf16x8(acc[v], __ldcg(reinterpret_cast<const uint4*>(yr + c0 + 8 * v)));
+  };
+  if (sh.Ds > 0) add_row((Mr + t / sh.tile_m) * sh.tile_m + t % sh.tile_m);
+  for (int j = 0; j < sh.k; ++j) {
+    const int row = __ldcg(ws.row_of_slot + t * sh.k + j);
+    if (row >= 0) add_row(row);
+  }
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    if (c0 + 8 * v + 8 > sh.H) break;
+    if (fa.out_bf16) store8<true>(fa.out, (size_t)t * sh.H + c0 + 8 * v, acc[v]);
+    else store8<false>(fa.out, (size_t)t * sh.H + c0 + 8 * v, acc[v]);
+  }
+}
+
 }  // namespace
 
 template <int kShape>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    moe_gemm_kernel(const __grid_constant__ GemmMaps maps, Workspace ws, Shape sh) {
+    moe_gemm_kernel(const __grid_constant__ GemmMaps maps, Workspace ws, Shape sh, FrontArgs fa) {
   using C = Cfg<kShape>;
   constexpr bool kSmall = C::kSmall;
+  constexpr bool kFused = (kShape == kShapeSmallFused);
   constexpr bool kTail = C::kTail;
   constexpr int kStages = C::kStagesN;
   constexpr int kStageBytes = C::kStageBytesN;
@@ -107,6 +497,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
   volatile int* s_epi_go = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 8);  // [2]
+  volatile int* s_front = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 16);  // fused: last / ok
+  volatile int* s_comb = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 24);   // fused: combine
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   DeviceMeta* meta = ws.meta;
@@ -147,7 +539,61 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint32_t nfill = 0;  // TMA stage fills issued by this CTA (producer warp)
   bool mma_issued = false;
 
-  if (warp == 0) {
+  // wait accounting while tracing (globaltimer ns, per role thread; see kWait* in common.cuh)
+  const bool tracing = ws.trace_cap > 0;
+  int64_t wacc[kNumWaits];
+#pragma unroll
+  for (int i = 0; i < kNumWaits; ++i) wacc[i] = 0;
+  auto now = [&]() -> int64_t { return tracing ? (int64_t)globaltimer_ns() : 0; };
+
+  bool run_tasks = true;
+  const int64_t t_front = now();
+  if constexpr (kFused) {
+    // the front, by all 192 threads; the operand ring is free until the first TMA fill
+    int* fsm = reinterpret_cast<int*>(smem);
+    front_router(fa, ws, sh, reinterpret_cast<float*>(fsm));
+    const int64_t t_r = now();
+    if (threadIdx.x == 0) {
+      __threadfence();
+      s_front[0] = (atomicAdd(&ws.front->front_done, 1) == (int)gridDim.x - 1) ? 1 : 0;
+    }
+    __syncthreads();
+    int64_t ts[4] = {0, 0, 0, 0};
+    const int64_t t_arrived = now();
+    if (s_front[0]) {
+      __threadfence();
+      front_schedule(fa, ws, sh, fsm, ts);
+      if (threadIdx.x == 0) s_front[1] = 1;
+    } else if (threadIdx.x == 0) {
+      s_front[1] = wait_schedule(&ws.front->sched_flag, fa.epoch, meta, limit) ? 1 : 0;
+      __threadfence();
+    }
+    __syncthreads();
+    const int64_t t_s = now();
+    run_tasks = s_front[1] != 0;
+    if (run_tasks) front_gather(fa, ws, sh);
+    // the ring's generic-proxy writes come before the TMA fills that reuse it
+    fence_proxy_async_shared();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      wacc[kFrontRouter] = t_r - t_front;
+      wacc[kFrontSchedule] = t_s - t_r;
+      wacc[kFrontGather] = now() - t_s;
+      wacc[kFrontLast] = tracing ? s_front[0] : 0;
+      if (tracing && s_front[0]) {
+        wacc[kSchedArrive] = t_arrived - t_r;
+        wacc[kSchedLogits] = ts[0] - t_arrived;
+        wacc[kSchedGating] = ts[1] - ts[0];
+        wacc[kSchedTables] = ts[2] - ts[1];
+        wacc[kSchedWrites] = ts[3] - ts[2];
+        wacc[kSchedPublish] = t_s - ts[3];
+      }
+    }
+  }
+
+  if (!run_tasks) {
+    // the schedule never came (bounded wait ran out): nothing was issued, go to the teardown
+  } else if (warp == 0) {
     // ===================================== producer =====================================
     const int total = __ldcg(&meta->total_tasks);
     const int Mg = __ldcg(&meta->num_groups), Mgr = __ldcg(&meta->num_routed_groups);
@@ -166,7 +612,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     SlotIter sq_it;
     int sq_j = 0;
     if (sh.static_quota && lane == 0 && sq_slot < X) sq_it.start(ws, sq_slot);
+    // Claims run ahead by less than a ring: the id of the next task is fetched from the counter
+    // while the current task's last kStages stages are issued, so the atomic's round trip
+    // overlaps them, but a claimed task is never held for longer than one ring drains (a held
+    // task is one no idle CTA can take at the end of the queue). The held id is always the next
+    // task this producer starts, and every task it waits for has a smaller id, so the smallest
+    // unfinished task still always makes progress.
+    int next_tau = 0;
+    if (!sh.static_quota && lane == 0) next_tau = atomicAdd(&meta->task_counter, 1);
+    // with the task table, the claimed task's entry is loaded one stage after the claim
+    const bool use_tab = ws.task_tab != nullptr && !sh.static_quota;
+    int4 next_ent = make_int4(0, 0, 0, 0);
+    int ent_tau = -1;  // the claim whose entry next_ent holds
+    const int64_t t_loop = now();
     while (true) {
+      const int64_t t_top = now();
       int tau = 0, unit = 0;
       if (sh.static_quota) {
         if (lane == 0) {
@@ -189,7 +649,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         unit = __shfl_sync(0xffffffffu, unit, 0);
       } else if (lane == 0) {
-        tau = aborted(meta, s_abort) ? total : atomicAdd(&meta->task_counter, 1);
+        tau = aborted(meta, s_abort) ? total : next_tau;
       }
       tau = __shfl_sync(0xffffffffu, tau, 0);
       Task t;
@@ -198,6 +658,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       t.nrows2 = 0;
       if (tau >= total) {
         t.kind = kTaskStop;
+      } else if (use_tab) {
+        int4 ent = next_ent;
+        if (lane == 0 && ent_tau != tau) ent = __ldcg(ws.task_tab + tau);
+        ent.x = __shfl_sync(0xffffffffu, ent.x, 0);
+        ent.y = __shfl_sync(0xffffffffu, ent.y, 0);
+        ent.z = __shfl_sync(0xffffffffu, ent.z, 0);
+        ent.w = __shfl_sync(0xffffffffu, ent.w, 0);
+        t.tile = ent.x;
+        t.expert = ent.y;
+        t.row0 = ent.z;
+        t.nrows = ent.w & 511;
+        t.kind = (ent.w >> 19) & 1;
+        t.ntiles = kTail ? (((ent.w >> 18) & 1) ? 2 : 1) : 1;
+        t.nrows2 = t.ntiles == 2 ? (ent.w >> 9) & 511 : 0;
+        const int nt = ent.w >> 20;
+        if (t.kind == kTaskUp) {
+          t.n0 = nt * kBN1;
+          t.nk = nk1;
+        } else {
+          t.n0 = nt * kBN2;
+          t.nk = ceil_div(t.expert == sh.E ? sh.Ds : sh.D, kBK);
+        }
       } else {
         u_cur = sh.static_quota ? unit : find_unit(ws.unit_start, U, tau, u_cur);
         const TaskPos pos = decode_task(ws, sh, u_cur, tau, Mg, Mgr);
@@ -221,7 +703,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // publish the task to the MMA and epilogue warps
       bool ok = true;
       if (lane == 0) {
+        const int64_t t0 = now();
         ok = wait_bar(&task_empty[slot], slot_phase ^ 1, meta, s_abort, limit, kSiteProducerTask);
+        const int64_t t1 = now();
+        wacc[kWaitProdRing] += t1 - t0;
+        wacc[kWaitProdClaim] += t0 - t_top;
         if (ok) {
           ring[slot] = t;
           mbar_arrive(&task_full[slot]);
@@ -230,6 +716,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       if (!ok || t.kind == kTaskStop) break;
       if (++slot == kTaskSlots) { slot = 0; slot_phase ^= 1; }
+      const int claim_kb = t.nk > kStages ? t.nk - kStages : 0;  // stage at which the next id is claimed
       if (ws.trace_cap > 0 && lane == 0) {
         // claim time goes to the trace slot of this task id (written again at completion)
         if (tau < ws.trace_cap) {
@@ -239,12 +726,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
       }
       const bool shared = (t.expert == sh.E);
+      // fused small-batch forward: an up task of a routed tile needs the tile's gathered x rows
+      if (kFused && t.kind == kTaskUp && !shared) {
+        if (lane == 0) {
+          const int64_t t0 = now();
+          ok = wait_count(&ws.gather_done[t.tile], t.nrows, meta, s_abort, limit);
+          wacc[kWaitProdDep] += now() - t0;
+          if (ok) fence_proxy_async_global();
+        }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
+      }
       // a down task needs every up task of its tile(s)
       if (t.kind == kTaskDown) {
         if (lane == 0) {
           const int need = n1_of(t.expert, sh) + sh.dep_extra;
+          const int64_t t0 = now();
           ok = wait_count(&ws.done1[t.tile], need, meta, s_abort, limit);
           if (ok && t.ntiles == 2) ok = wait_count(&ws.done1[t.tile + 1], need, meta, s_abort, limit);
+          wacc[kWaitProdDep] += now() - t0;
           if (ok) fence_proxy_async_global();
         }
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -265,7 +765,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int arow = (up && shared) ? t.row0 : t.tile * kBM;
       const int arow2 = (up && shared) ? t.row0 + kBM : (t.tile + 1) * kBM;  // a merged tail's rows
       for (int kb = 0; kb < t.nk; ++kb) {
-        if (lane == 0) ok = wait_bar(&empty[stage], phase ^ 1, meta, s_abort, limit, kSiteProducerEmpty);
+        if (lane == 0) {
+          const int64_t t0 = now();
+          ok = wait_bar(&empty[stage], phase ^ 1, meta, s_abort, limit, kSiteProducerEmpty);
+          wacc[kWaitProdEmpty] += now() - t0;
+        }
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         if (!ok) break;
         if (lane == 0) {
@@ -289,12 +793,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             tma_load_2d(b, shared ? &maps.ws_down : &maps.w_down, &full[stage], kb * kBK, wrow_dn);
           }
         }
+        if (kb == claim_kb && !sh.static_quota && lane == 0) next_tau = atomicAdd(&meta->task_counter, 1);
+        if (kb == claim_kb + 1 && use_tab && lane == 0 && next_tau < total) {
+          next_ent = __ldcg(ws.task_tab + next_tau);
+          ent_tau = next_tau;
+        }
         __syncwarp();
         ++nfill;
         if (++stage == kStages) { stage = 0; phase ^= 1; }
       }
       if (!ok) break;
     }
+    wacc[kWaitProdLoop] = now() - t_loop;
   } else if (warp == 1) {
     // ===================================== MMA issuer ===================================
     // A task uses the next accumulator, or both when it also computes a merged tail tile; each
@@ -302,20 +812,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(kBM, kUmmaN);
       uint32_t stage = 0, phase = 0, slot = 0, slot_phase = 0, next = 0, use0 = 0, use1 = 0;
+      const int64_t t_loop = now();
       while (true) {
-        if (!wait_bar(&task_full[slot], slot_phase, meta, s_abort, limit, kSiteMmaTask)) break;
+        int64_t t0 = now();
+        const bool got = wait_bar(&task_full[slot], slot_phase, meta, s_abort, limit, kSiteMmaTask);
+        wacc[kWaitMmaTask] += now() - t0;
+        if (!got) break;
         const Task t = ring[slot];
         if (t.kind == kTaskStop) break;
         const uint32_t a0 = next, a1 = next ^ 1u;
         const bool two = kTail && (t.ntiles == 2);
+        t0 = now();
         if (!wait_bar(&acc_empty[a0], ((a0 ? use1 : use0) & 1u) ^ 1u, meta, s_abort, limit, kSiteMmaAcc)) break;
         if (two && !wait_bar(&acc_empty[a1], ((a1 ? use1 : use0) & 1u) ^ 1u, meta, s_abort, limit, kSiteMmaAcc))
           break;
+        wacc[kWaitMmaAcc] += now() - t0;
         tc_fence_after();
         const uint32_t d0 = tmem_base + a0 * kAccCols, d1 = tmem_base + a1 * kAccCols;
         bool ok = true;
         for (int kb = 0; kb < t.nk; ++kb) {
+          t0 = now();
           if (!wait_bar(&full[stage], phase, meta, s_abort, limit, kSiteMmaFull)) { ok = false; break; }
+          wacc[kWaitMmaFull] += now() - t0;
           tc_fence_after();
           const uint32_t a = smem_u32(smem + stage * kStageBytes);
           const uint32_t b = a + kBOff;
@@ -347,6 +865,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         mbar_arrive(&task_empty[slot]);
         if (++slot == kTaskSlots) { slot = 0; slot_phase ^= 1; }
       }
+      wacc[kWaitMmaLoop] = now() - t_loop;
     }
     __syncwarp();
   } else {
@@ -368,11 +887,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     auto epilogue_next = [&](uint32_t it) -> bool {
       if (leader) {
         int go = 0;
-        if (wait_bar(&task_full[slot], slot_phase, meta, s_abort, limit, kSiteEpiTask) && ring[slot].kind != kTaskStop) {
+        const int64_t t0 = now();
+        const bool got = wait_bar(&task_full[slot], slot_phase, meta, s_abort, limit, kSiteEpiTask);
+        const int64_t t1 = now();
+        wacc[kWaitEpiTask] += t1 - t0;
+        if (got && ring[slot].kind != kTaskStop) {
           const uint32_t a1 = next ^ 1u;
           go = wait_bar(&acc_full[next], (next ? use1 : use0) & 1u, meta, s_abort, limit, kSiteEpiAcc) ? 1 : 0;
           if (go && ring[slot].ntiles == 2)
             go = wait_bar(&acc_full[a1], (a1 ? use1 : use0) & 1u, meta, s_abort, limit, kSiteEpiAcc) ? 1 : 0;
+          wacc[kWaitEpiAcc] += now() - t1;
         }
         s_epi_go[it & 1] = go;
       }
@@ -390,6 +914,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         next ^= 1u;
       }
     };
+    const int64_t t_loop = now();
     if constexpr (kSmall) {
       // at most 16 valid rows per tile: only the warp of TMEM lanes 0-31 has work, and the
       // valid rows are stored straight from registers (no staging, no TMA stores)
@@ -476,6 +1001,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&acc_empty[next]);
+          if constexpr (kFused) {
+            // count this task's column block; the task that completes a block combines it
+            __threadfence();
+            named_bar_sync(1, 128);
+            if (leader)
+              *s_comb = (atomicAdd(&ws.col_done[t.n0 / kBN2], 1) == __ldcg(&meta->num_tiles) - 1) ? 1 : 0;
+            named_bar_sync(1, 128);
+            if (*s_comb) {
+              __threadfence();
+              fused_combine(fa, ws, sh, t.n0, (int)threadIdx.x - 64, __ldcg(&meta->num_routed_tiles));
+            }
+          }
         }
         if (lane == 0) mbar_arrive(&task_empty[slot]);
         if (ws.trace_cap > 0 && leader && t.id < ws.trace_cap)
@@ -598,6 +1135,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // the staging buffer must not be released while a store still reads it
     if (leader) bulk_wait_group<0>();
     }
+    wacc[kWaitEpiLoop] = now() - t_loop;
+    wacc[kFrontToEnd] = now() - t_front;
+  }
+  // wait accounting of this CTA: each role's recording thread adds its entries
+  if (tracing && ws.waits != nullptr && ((warp == 0 && lane == 0) || threadIdx.x == 32 || (warp == 2 && lane == 0))) {
+#pragma unroll
+    for (int i = 0; i < kNumWaits; ++i)
+      if (wacc[i]) atomicAdd(reinterpret_cast<unsigned long long*>(ws.waits + (size_t)blockIdx.x * kNumWaits + i),
+                             (unsigned long long)wacc[i]);
   }
 
   // the next kernel may start its prologue once every CTA has finished its tasks (not earlier:
@@ -620,24 +1166,57 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 }
 
 size_t gemm_smem_bytes(int shape) {
-  return (size_t)(shape == kShapeSmall ? Cfg<kShapeSmall>::kBytes
-                                       : (shape == kShapeTail ? Cfg<kShapeTail>::kBytes : Cfg<kShapeGeneral>::kBytes)) +
+  const bool small = shape == kShapeSmall || shape == kShapeSmallFused;
+  return (size_t)(small ? Cfg<kShapeSmall>::kBytes
+                        : (shape == kShapeTail ? Cfg<kShapeTail>::kBytes : Cfg<kShapeGeneral>::kBytes)) +
          1024;
 }
 
 cudaError_t launch_moe_gemm(const GemmMaps& maps, const Workspace& ws, const Shape& sh, int grid, int shape,
                             cudaStream_t stream) {
   const size_t smem = gemm_smem_bytes(shape);
+  const FrontArgs fa{};
   if (shape == kShapeSmall)
-    return launch_k(moe_gemm_kernel<kShapeSmall>, dim3(grid), dim3(kGemmThreads), smem, stream, maps, ws, sh);
+    return launch_k(moe_gemm_kernel<kShapeSmall>, dim3(grid), dim3(kGemmThreads), smem, stream, maps, ws, sh, fa);
   if (shape == kShapeTail)
-    return launch_k(moe_gemm_kernel<kShapeTail>, dim3(grid), dim3(kGemmThreads), smem, stream, maps, ws, sh);
-  return launch_k(moe_gemm_kernel<kShapeGeneral>, dim3(grid), dim3(kGemmThreads), smem, stream, maps, ws, sh);
+    return launch_k(moe_gemm_kernel<kShapeTail>, dim3(grid), dim3(kGemmThreads), smem, stream, maps, ws, sh, fa);
+  return launch_k(moe_gemm_kernel<kShapeGeneral>, dim3(grid), dim3(kGemmThreads), smem, stream, maps, ws, sh, fa);
+}
+
+cudaError_t launch_moe_small_fused(const GemmMaps& maps, const Workspace& ws, const Shape& sh,
+                                   const FrontArgs& fa, int grid, cudaStream_t stream) {
+  // every CTA waits for the schedule that one of them publishes: all must be resident at once
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = gemm_smem_bytes(kShapeSmallFused);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, moe_gemm_kernel<kShapeSmallFused>, maps, ws, sh, fa);
+}
+
+int small_fused_blocks_per_sm() {
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, moe_gemm_kernel<kShapeSmallFused>, kGemmThreads,
+                                                    gemm_smem_bytes(kShapeSmallFused)) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
 }
 
 cudaError_t configure_gemm_kernel() {
   cudaError_t e = cudaFuncSetAttribute(moe_gemm_kernel<kShapeSmall>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)gemm_smem_bytes(kShapeSmall));
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(moe_gemm_kernel<kShapeSmallFused>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)gemm_smem_bytes(kShapeSmallFused));
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(moe_gemm_kernel<kShapeTail>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)gemm_smem_bytes(kShapeTail));

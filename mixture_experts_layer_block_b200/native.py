@@ -32,6 +32,7 @@ MOE_FLAG_TAIL_TILES = 64
 MOE_FLAG_NO_TAIL_TILES = 128
 MOE_FLAG_STATIC_QUOTA = 256
 MOE_FLAG_MXFP8 = 512
+MOE_FLAG_UNFUSED_SMALL = 1024
 MOE_FLAG_TRACE = 4
 
 
@@ -83,6 +84,7 @@ SIGNATURES = {
     "moe_query": (ctypes.c_int, [_P, _I32, ctypes.POINTER(ctypes.c_int64)]),
     "moe_trace_read": (ctypes.c_int, [_P, _P, _I64, ctypes.POINTER(ctypes.c_int64)]),
     "moe_debug_inject_stall": (ctypes.c_int, [_P, _I32]),
+    "moe_trace_waits": (ctypes.c_int, [_P, _P, _I32, ctypes.POINTER(ctypes.c_int32)]),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "moe_align_block_size_noalloc": (ctypes.c_int, [_P, _I32, _I32, _I32, _I32, ctypes.c_float, _P, _P, _P,
                                                     _P]),
@@ -321,6 +323,20 @@ class MoELayer:
         n = ctypes.c_int64(0)
         check(lib.moe_trace_read(self.h, buf.ctypes.data_as(ctypes.c_void_p), cap, ctypes.byref(n)),
               "moe_trace_read")
+        return buf[: n.value]
+
+    WAITS = ("prod_empty", "prod_dep", "prod_ring", "prod_claim", "mma_full", "mma_acc", "mma_task",
+             "epi_task", "epi_acc", "prod_loop", "mma_loop", "epi_loop", "front_router", "front_schedule",
+             "front_gather", "front_last", "front_to_end", "sched_arrive", "sched_logits", "sched_gating",
+             "sched_tables", "sched_writes", "sched_publish")
+
+    def trace_waits(self):
+        """moe_trace_waits: [CTAs, 23] int64 ns (columns named by WAITS)."""
+        import numpy as np
+        buf = np.zeros((1024, len(self.WAITS)), dtype=np.int64)
+        n = ctypes.c_int32(0)
+        check(lib.moe_trace_waits(self.h, buf.ctypes.data_as(ctypes.c_void_p), 1024, ctypes.byref(n)),
+              "moe_trace_waits")
         return buf[: n.value]
 
     def inject_stall(self, extra):

@@ -271,3 +271,59 @@ def test_forward_host_async_pipelined():
     assert torch.equal(outs[0], ref[0]) and torch.equal(last, ref[1])
     rc, st = layer.status()
     assert rc == 0 and st == 0
+
+
+FUSED_CASES = {
+    "one_token": SMALL["one_token"],
+    "small_tokens_shared": SMALL["small_tokens_shared"],
+    "small_tokens_ragged": SMALL["small_tokens_ragged"],   # capacity drops, ragged H and D
+    "decode": configs.DECODE,                               # 256 experts top-8, router bias
+    "sixteen_rows_one_expert": configs.MoEWorkload("sixteen_rows_one_expert", T=16, H=256, D=384, E=2, top_k=1,
+                                                   block_m=16, D_shared=128, sigma_w=0.05),
+    "many_experts_few_ctas": configs.MoEWorkload("many_experts_few_ctas", T=9, H=512, D=256, E=200, top_k=6,
+                                                 block_m=16, sigma_w=0.05),
+}
+
+
+@pytest.mark.parametrize("name", sorted(FUSED_CASES))
+def test_small_batch_fused_and_unfused(name):
+    """Batches of at most 16 tokens run as one fused launch by default (router slices, gating and
+    align in the last CTA, gather, expert GEMMs, combine by the last down task of each column
+    block) and as the six kernels with MOE_FLAG_UNFUSED_SMALL: both match the oracle stage by
+    stage, and repeated fused forwards agree bit for bit."""
+    from mixture_experts_layer_block_b200 import native
+    w = FUSED_CASES[name]
+    inp = {k: (v.cuda() if v is not None else None) for k, v in gen.make_inputs(w).items()}
+    if name == "sixteen_rows_one_expert":
+        inp["bias"] = torch.tensor([30.0, 0.0], dtype=torch.float32, device="cuda")
+    fused = _layer(w)
+    assert fused.query(12) == 1
+    res = check_forward(fused, w, inp)
+    assert fused.query(11) == 1 and fused.query(8) == SHAPE_CODE["small"]
+    unfused = _layer(w, flags=native.MOE_FLAG_UNFUSED_SMALL)
+    check_forward(unfused, w, inp)
+    assert unfused.query(11) == 6 and unfused.query(12) == 0
+    outs = []
+    for _ in range(3):
+        o = torch.empty((w.T, w.H), dtype=torch.float32, device="cuda")
+        fused.forward(inp["x"], inp, o)
+        outs.append(o)
+    torch.cuda.synchronize()
+    assert fused.status() == (0, 0)
+    assert all(torch.equal(o, outs[0]) for o in outs[1:])
+    print(name, res)
+
+
+def test_small_batch_fused_stage_times_and_smaller_batches():
+    """The fused launch on a handle sized for more tokens, with shrinking batches in a row (the
+    per-forward counters start afresh each time), and its stage timing (all in the GEMM slot)."""
+    from mixture_experts_layer_block_b200 import native
+    w = configs.DECODE
+    inp = gen.make_inputs(w, device="cuda")
+    layer = _layer(w, flags=native.MOE_FLAG_STAGE_TIMING, max_tokens=64)
+    for T in (16, 7, 1, 16):
+        wt = w.replace(T=T)
+        check_forward(layer, wt, dict(inp, x=inp["x"][:T].contiguous()))
+        assert layer.query(11) == 1
+    ms = layer.stage_times()
+    assert ms[4] > 0 and all(abs(v) < 0.01 for i, v in enumerate(ms) if i != 4)
