@@ -188,8 +188,8 @@ def layer_fraction(w, peaks, ms, kept, hit, mx):
 
 def tile_flags(args) -> int:
     from mixture_experts_layer_block_b200 import native
-    f = {"auto": 0, "pair": native.MOE_FLAG_PAIR_TILES, "single": native.MOE_FLAG_SINGLE_TILES}[
-        getattr(args, "tiles", "auto")]
+    f = {"auto": 0, "pair": native.MOE_FLAG_PAIR_TILES, "single": native.MOE_FLAG_SINGLE_TILES,
+         "two": native.MOE_FLAG_TWO_TILES}[getattr(args, "tiles", "auto")]
     if getattr(args, "sched", "dynamic") == "static":
         f |= native.MOE_FLAG_STATIC_QUOTA
     if getattr(args, "unfused_small", False):
@@ -759,9 +759,9 @@ def main():
     ap.add_argument("--ref-tokens", type=int, default=256)
     ap.add_argument("--T", type=int, default=None, help="override the workload's token count (profiling)")
     ap.add_argument("--E", type=int, default=None, help="override the workload's expert count (profiling)")
-    ap.add_argument("--tiles", choices=["auto", "pair", "single"], default="auto",
-                    help="expert-GEMM shape: the library's choice, 256-row tiles on SM pairs, or "
-                         "128-row tiles on single SMs")
+    ap.add_argument("--tiles", choices=["auto", "pair", "single", "two"], default="auto",
+                    help="expert-GEMM shape: the library's choice, 256-row tiles on SM pairs, "
+                         "128-row tiles on single SMs, or two 128-row tiles per task on single SMs")
     ap.add_argument("--sched", choices=["dynamic", "static"], default="dynamic",
                     help="task scheduling of the expert GEMMs: the atomic queue, or the static "
                          "per-expert SM quota baseline (ablation)")

@@ -99,6 +99,11 @@ extern "C" {
  * weights differ in the last bits, and an exact near-tie may go the other way; both are
  * deterministic. */
 #define MOE_FLAG_UNFUSED_SMALL 1024u
+/* The one-SM expert GEMMs of batches of more than 16 tokens run every group of two m-tiles of one
+ * expert as one task set: each task computes both tiles from the same weight stages into the two
+ * TMEM accumulators (a 3-stage ring of 64 KB stages; the "two-tile" shape, moe_query 8 reports 5).
+ * It wins over the tail and general shapes; the same result. */
+#define MOE_FLAG_TWO_TILES    2048u
 
 typedef struct moe_config {
     int32_t hidden;           /* H: model dimension; multiple of 8 */
@@ -314,7 +319,7 @@ MOE_API int moe_stage_times(moe_handle *h, float *ms, int32_t n);
  * 5 dependency lag (units) of the last forward, 6 rows per m-tile of the last forward
  * (128 or 256), 7 SM pairs the device can run at once for the pair shape (0 = none),
  * 8 expert-GEMM shape of the last forward (0 general, 1 small-tile, 2 tail, 3 SM pairs,
- * 4 MXFP8), 9 rows of the per-row buffers of moe_debug_expert_rows, 10 their h row stride
+ * 4 MXFP8, 5 two-tile), 9 rows of the per-row buffers of moe_debug_expert_rows, 10 their h row stride
  * (elements, max(D, D_shared)), 11 kernels the last forward launched (1 for a fused small
  * batch, else 6), 12 whether batches of at most 16 tokens run fused on this handle (1) or not. */
 MOE_API int moe_query(const moe_handle *h, int32_t which, int64_t *value);

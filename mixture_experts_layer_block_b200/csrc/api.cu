@@ -508,14 +508,16 @@ static int forward_impl(moe_handle* h, const void* x, int32_t T, const void* w_r
   // second staging buffer: by default it is used when the mean load per expert is 96..384
   // slots and the capacity allows more than one tile per expert.
   int gemm_shape = small ? kShapeSmall : kShapeGeneral;
-  if (!small && !pair && !(c.flags & MOE_FLAG_NO_TAIL_TILES)) {
+  if (!small && !pair && (c.flags & MOE_FLAG_TWO_TILES)) {
+    gemm_shape = kShapeTwo;
+  } else if (!small && !pair && !(c.flags & MOE_FLAG_NO_TAIL_TILES)) {
     const int64_t load = (int64_t)T * top_k;  // slots over E experts
     const int cap = capacity_of(c, T, top_k);
     const bool fits = load > (int64_t)96 * E && load <= (int64_t)384 * E && (cap == 0 || cap > kBM);
     if (fits || (c.flags & MOE_FLAG_TAIL_TILES)) gemm_shape = kShapeTail;
   }
-  h->last_shape = pair ? 3 : gemm_shape;
-  sh.merge_tail = (gemm_shape == kShapeTail) ? 1 : 0;
+  h->last_shape = pair ? 3 : (gemm_shape == kShapeTwo ? 5 : gemm_shape);
+  sh.merge_tail = (gemm_shape == kShapeTail) ? 1 : (gemm_shape == kShapeTwo ? 2 : 0);
   sh.static_quota = (!pair && (c.flags & MOE_FLAG_STATIC_QUOTA)) ? 1 : 0;
   h->last_workers = workers;
   h->last_tile_m = sh.tile_m;

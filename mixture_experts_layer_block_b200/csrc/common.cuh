@@ -205,7 +205,8 @@ struct Shape {
   int32_t dep_extra;     // testing hook: extra up completions a down task waits for
   int32_t tile_m;        // rows per m-tile of the expert GEMMs: 128, or 256 on SM pairs
   int32_t merge_tail;    // 1: a group of a full tile and a tail of <= kTailRows rows runs as one
-                         //    task set (the one-SM general shape only)
+                         //    task set (the one-SM tail shape); 2: every group of two tiles does
+                         //    (the two-tile shape); 0: never
   int32_t static_quota;  // 1: each CTA works through a fixed share of the experts (ablation)
   int64_t timeout_ns;
 };

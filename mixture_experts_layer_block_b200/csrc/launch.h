@@ -91,7 +91,9 @@ cudaError_t launch_combine(void* out, bool bf16_out, const Workspace& ws, const 
 // tails of at most 32 rows merged into the previous tile's tasks; needs sh.merge_tail = 1) and
 // small (batches of at most 16 tokens; its maps use 16-row boxes for x_tile, xs, h_routed and
 // h_shared).
-enum GemmShape : int { kShapeGeneral = 0, kShapeSmall = 1, kShapeTail = 2, kShapeSmallFused = 3 };
+// kShapeTwo: every group of two m-tiles of one expert runs as one task set whose tasks compute
+// both tiles from the same weight stages (needs sh.merge_tail = 2).
+enum GemmShape : int { kShapeGeneral = 0, kShapeSmall = 1, kShapeTail = 2, kShapeSmallFused = 3, kShapeTwo = 4 };
 size_t gemm_smem_bytes(int shape);
 cudaError_t launch_moe_gemm(const GemmMaps& maps, const Workspace& ws, const Shape& sh, int grid, int shape,
                             cudaStream_t stream);

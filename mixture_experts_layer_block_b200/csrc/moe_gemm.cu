@@ -59,13 +59,14 @@ namespace {
 template <int kShape>
 struct Cfg {
   static constexpr bool kSmall = (kShape == kShapeSmall || kShape == kShapeSmallFused);
-  static constexpr bool kTail = (kShape == kShapeTail);
-  static constexpr int kStagesN = kSmall ? 6 : kStages;
+  static constexpr bool kTwo = (kShape == kShapeTwo);
+  static constexpr bool kTail = (kShape == kShapeTail) || kTwo;  // a task may carry a second tile
+  static constexpr int kStagesN = kSmall ? 6 : (kTwo ? 3 : kStages);
   static constexpr int kARows = kSmall ? 16 : kBM;
   static constexpr int kABytesN = kARows * kBK * 2;
-  static constexpr int kTailBytesN = kTail ? kTailRows * kBK * 2 : 0;
+  static constexpr int kTailBytesN = kTwo ? kBM * kBK * 2 : (kTail ? kTailRows * kBK * 2 : 0);
   static constexpr int kStageBytesN = kABytesN + kTailBytesN + kBBytes;
-  static constexpr int kNumStagingN = kSmall ? 0 : (kTail ? 1 : kNumStaging);
+  static constexpr int kNumStagingN = kSmall ? 0 : ((kTail && !kTwo) ? 1 : kNumStaging);
   static constexpr int kStagingOff = kStagesN * kStageBytesN;
   static constexpr int kBarOff = kStagingOff + kNumStagingN * kStagingBytes;
   // barriers: full[S], empty[S], acc_full[2], acc_empty[2], task_full[R], task_empty[R], drain
@@ -210,20 +211,17 @@ __device__ void front_schedule(const FrontArgs& fa, const Workspace& ws, const S
   const int E = sh.E, T = sh.T, k = sh.k, S = T * k;
   int* ids_s = sm;           // [S]
   int* cnt = ids_s + S;      // [E]
-  int* off = cnt + E;        // [E + 1]
+  unsigned* tmask = reinterpret_cast<unsigned*>(cnt + E);  // [E] tokens (bits) that chose e
+  int* off = reinterpret_cast<int*>(tmask + E);            // [E + 1]
   int* kept = off + E + 1;   // [E]
   int* tile0 = kept + E;     // [E]
-  int* run = tile0 + E;      // [E]  running count of the stable writes
-  int* s_mt = run + E;       // [2]  m-tiles, and routed m-tiles, of this forward
-  int* t_exp = s_mt + 2;     // [E + 1] per m-tile: expert, first sorted row, rows
-  int* t_r0 = t_exp + E + 1;
-  int* t_nr = t_r0 + E + 1;
+  int* s_mt = tile0 + E;     // [2]  m-tiles, and routed m-tiles, of this forward
   for (int e = tid; e < E; e += nthr) {
     cnt[e] = 0;
-    run[e] = 0;
+    tmask[e] = 0;
   }
   // gating: warp w takes tokens w, w + nw, w + 2 nw (T <= 16 <= 3 * 6); the logits of all its
-  // tokens are loaded at once (one round trip), then each token's top-k
+  // tokens are loaded at once (one round trip), then their top-k interleaved
   constexpr int kTokPerWarp = 3;
   float v[kTokPerWarp][8];
 #pragma unroll
@@ -250,21 +248,26 @@ __device__ void front_schedule(const FrontArgs& fa, const Workspace& ws, const S
         ws.topk_w[t * k + lane] = wt[i];
         ids_s[t * k + lane] = id[i];
         atomicAdd(&cnt[id[i]], 1);
+        atomicOr(&tmask[id[i]], 1u << t);
       }
     }
   }
   __syncthreads();
   stamp(1);
   if (warp == 0) {
-    // lane l owns experts [8l, 8l + 8) (E <= 256), so lane order is expert order
+    // the two scans over the experts; lane l owns experts [8l, 8l + 8) (E <= 256), so lane
+    // order is expert order
     const int e0 = lane * 8;
+    const int bm = sh.block_m;
+    const bool pow2 = (bm & (bm - 1)) == 0;
+    auto padded = [&](int n) { return pow2 ? (n + bm - 1) & ~(bm - 1) : ceil_div(n, bm) * bm; };
     int kp[8], pad = 0, hit = 0;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int e = e0 + j;
       const int n = e < E ? cnt[e] : 0;
       kp[j] = (sh.capacity > 0) ? min(n, sh.capacity) : n;
-      pad += ceil_div(kp[j], sh.block_m) * sh.block_m;
+      pad += padded(kp[j]);
       hit += kp[j] > 0 ? 1 : 0;
     }
     int P, Mr;
@@ -277,119 +280,109 @@ __device__ void front_schedule(const FrontArgs& fa, const Workspace& ws, const S
         off[e] = o;
         kept[e] = kp[j];
         tile0[e] = ti;
-        ws.expert_off[e] = o;
-        ws.expert_kept[e] = kp[j];
-        ws.expert_tile0[e] = ti;
-        ws.expert_group0[e] = ti;  // one tile per group
-        if (kp[j] > 0) {
-          t_exp[ti] = e;
-          t_r0[ti] = o;
-          t_nr[ti] = kp[j];
-          ws.tile_expert[ti] = e;
-          ws.tile_row0[ti] = o;
-          ws.tile_nrows[ti] = kp[j];
-          ws.group_tile0[ti] = ti;
-          ws.group_ntiles[ti] = 1;
-          ws.group_tasks[ti] = 1;
-        }
-        o += ceil_div(kp[j], sh.block_m) * sh.block_m;
+        o += padded(kp[j]);
         ti += kp[j] > 0 ? 1 : 0;
       }
     }
-    // the shared expert: one tile (and group) of all T tokens after the routed ones
-    const int Ms = sh.Ds > 0 ? 1 : 0, Mt = Mr + Ms, Mg = Mt;
     if (lane == 0) {
       off[E] = P;
-      ws.expert_off[E] = P;
-      if (Ms) {
-        t_exp[Mr] = E;
-        t_r0[Mr] = 0;
-        t_nr[Mr] = T;
-        ws.tile_expert[Mr] = E;
-        ws.tile_row0[Mr] = 0;
-        ws.tile_nrows[Mr] = T;
-        ws.group_tile0[Mr] = Mr;
-        ws.group_ntiles[Mr] = 1;
-        ws.group_tasks[Mr] = 1;
-      }
-      ws.expert_group0[E] = Mr;
-      ws.expert_group0[E + 1] = Mg;
-    }
-    const int U = Mg > 0 ? Mg + sh.lag : 0;
-    if (lane == 0) {
-      *s_mt = Mt;
+      s_mt[0] = Mr + (sh.Ds > 0 ? 1 : 0);  // the shared expert: one tile of all T tokens
       s_mt[1] = Mr;
-      DeviceMeta* m = ws.meta;
-      m->P = P;
-      m->num_tiles = Mt;
-      m->num_routed_tiles = Mr;
-      m->num_groups = Mg;
-      m->num_routed_groups = Mr;
-      m->num_units = U;
-      m->total_tasks = unit_start_of(U, Mr, Mg, sh);
-      m->task_counter = 0;
-      m->abort = 0;
-      m->trace_count = 0;
     }
   }
   __syncthreads();
   stamp(2);
-  const int P = off[E];
-  if (warp == 0) {
-    // slots in ascending order, 32 at a time: a slot's rank in its expert is the expert's running
-    // count plus its rank among this round's lanes of the same expert (stable)
-    for (int base = 0; base < S; base += 32) {
-      const int s = base + lane;
-      const int e = s < S ? ids_s[s] : -1;
-      const unsigned mask = __match_any_sync(0xffffffffu, e);
-      const int rank = __popc(mask & ((1u << lane) - 1u));
-      const int c0 = e >= 0 ? run[e] : 0;
-      __syncwarp();
-      if (e >= 0) {
-        const int r = c0 + rank;
-        const bool keep = sh.capacity == 0 || r < sh.capacity;
-        if (keep) ws.sorted_ids[off[e] + r] = s;
-        ws.row_of_slot[s] = keep ? tile0[e] * sh.tile_m + r : -1;
-        if (rank == 0) run[e] = c0 + __popc(mask);
-      }
-      __syncwarp();
+  // every write of the schedule, spread over the CTA
+  const int P = off[E], Mt = s_mt[0], Mr = s_mt[1], Mg = Mt, U = Mt > 0 ? Mt + sh.lag : 0;
+  const int bm = sh.block_m;
+  for (int e = tid; e < E; e += nthr) {
+    const int o = off[e], kp = kept[e], t0 = tile0[e], end = off[e + 1];
+    ws.expert_off[e] = o;
+    ws.expert_kept[e] = kp;
+    ws.expert_tile0[e] = t0;
+    ws.expert_group0[e] = t0;  // one tile per group
+    if (kp > 0) {
+      ws.tile_expert[t0] = e;
+      ws.tile_row0[t0] = o;
+      ws.tile_nrows[t0] = kp;
+      ws.group_tile0[t0] = t0;
+      ws.group_ntiles[t0] = 1;
+      ws.group_tasks[t0] = 1;
     }
+    for (int i = o + kp; i < end; ++i) ws.sorted_ids[i] = S;  // the segment's padding
+    for (int b = o / bm; b < end / bm; ++b) ws.expert_ids[b] = e;
   }
-  for (int i = tid; i < sh.sorted_len; i += nthr) {
-    bool padding = true;
-    if (i < P) {
-      const int e = segment_of(off, E, i);
-      padding = (i - off[e]) >= kept[e];
+  for (int i = P + tid; i < sh.sorted_len; i += nthr) ws.sorted_ids[i] = S;
+  for (int b = P / bm + tid; b < sh.blocks_len; b += nthr) ws.expert_ids[b] = -1;
+  // slot s = t*k + j: its rank in its expert is the number of earlier tokens that chose it
+  for (int s = tid; s < S; s += nthr) {
+    const int t = s / k, e = ids_s[s];
+    const int r = __popc(tmask[e] & ((1u << t) - 1u));
+    const bool keep = sh.capacity == 0 || r < sh.capacity;
+    if (keep) ws.sorted_ids[off[e] + r] = s;
+    ws.row_of_slot[s] = keep ? tile0[e] * sh.tile_m + r : -1;
+  }
+  if (tid == 0) {
+    ws.expert_off[E] = P;
+    if (sh.Ds > 0) {
+      ws.tile_expert[Mr] = E;
+      ws.tile_row0[Mr] = 0;
+      ws.tile_nrows[Mr] = T;
+      ws.group_tile0[Mr] = Mr;
+      ws.group_ntiles[Mr] = 1;
+      ws.group_tasks[Mr] = 1;
     }
-    if (padding) ws.sorted_ids[i] = S;
+    ws.expert_group0[E] = Mr;
+    ws.expert_group0[E + 1] = Mg;
+    DeviceMeta* m = ws.meta;
+    m->P = P;
+    m->num_tiles = Mt;
+    m->num_routed_tiles = Mr;
+    m->num_groups = Mg;
+    m->num_routed_groups = Mr;
+    m->num_units = U;
+    m->total_tasks = unit_start_of(U, Mr, Mg, sh);
+    m->task_counter = 0;
+    m->abort = 0;
+    m->trace_count = 0;
   }
-  for (int b = tid; b < sh.blocks_len; b += nthr) {
-    const int i = b * sh.block_m;
-    ws.expert_ids[b] = (i < P) ? segment_of(off, E, i) : -1;
-  }
-  const int Mt = *s_mt, Mr = s_mt[1], U = Mt > 0 ? Mt + sh.lag : 0;
   for (int i = tid; i < Mt; i += nthr) {
     ws.gather_done[i] = 0;
     ws.done1[i] = 0;
   }
-  for (int u = tid; u <= U; u += nthr) ws.unit_start[u] = unit_start_of(u, Mr, Mt, sh);
+  for (int i = tid; i < ceil_div(sh.H, kBN2); i += nthr) ws.col_done[i] = 0;
+  for (int u = tid; u <= U; u += nthr) ws.unit_start[u] = unit_start_of(u, Mr, Mg, sh);
   // the task table: one m-tile per group here, so unit u's tasks are the up tasks of tile u, then
-  // the down tasks of tile u - lag (as write_unit_tasks lays them out)
+  // the down tasks of tile u - lag (as write_unit_tasks lays them out); a tile's expert, first
+  // row and rows come from its expert's entries above (the shared tile: E, 0, T)
   if (ws.task_tab) {
+    // tile -> expert: the routed tiles are the hit experts in expert order
+    int* t_exp = s_mt + 2;  // [Mt]
+    for (int e = tid; e < E; e += nthr)
+      if (kept[e] > 0) t_exp[tile0[e]] = e;
+    if (tid == 0 && sh.Ds > 0) t_exp[Mr] = E;
+    __syncthreads();
+    auto tile_info = [&](int g, int& ex, int& r0, int& nr) {
+      ex = t_exp[g];
+      r0 = ex == E ? 0 : off[ex];
+      nr = ex == E ? T : kept[ex];
+    };
     for (int u = tid; u < U; u += nthr) {
-      int tau = unit_start_of(u, Mr, Mt, sh);
+      int tau = unit_start_of(u, Mr, Mg, sh);
+      int ex, r0, nr;
       if (u < Mt) {
+        tile_info(u, ex, r0, nr);
         const int n1 = ceil_div(u < Mr ? sh.D : sh.Ds, kBN1);
-        for (int nt = 0; nt < n1; ++nt)
-          ws.task_tab[tau++] = task_entry(kTaskUp, u, nt, 1, t_exp[u], t_r0[u], t_nr[u], 0);
+        for (int nt = 0; nt < n1; ++nt) ws.task_tab[tau++] = task_entry(kTaskUp, u, nt, 1, ex, r0, nr, 0);
       }
       const int g = u - sh.lag;
-      if (g >= 0 && g < Mt)
+      if (g >= 0 && g < Mt) {
+        tile_info(g, ex, r0, nr);
         for (int nt = 0; nt < ceil_div(sh.H, kBN2); ++nt)
-          ws.task_tab[tau++] = task_entry(kTaskDown, g, nt, 1, t_exp[g], t_r0[g], t_nr[g], 0);
+          ws.task_tab[tau++] = task_entry(kTaskDown, g, nt, 1, ex, r0, nr, 0);
+      }
     }
   }
-  for (int i = tid; i < ceil_div(sh.H, kBN2); i += nthr) ws.col_done[i] = 0;
   stamp(3);
   __threadfence();
   __syncthreads();
@@ -451,16 +444,43 @@ __device__ void fused_combine(const FrontArgs& fa, const Workspace& ws, const Sh
   for (int v = 0; v < 4; ++v)
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[v][j] = 0.f;
-  auto add_row = [&](int row) {
-    const uint16_t* yr = ws.y + (size_t)row * sh.H;
+  // the rows in summation order: the shared expert's, then slots j = 0..k-1 (-1: dropped); every
+  // index is loaded in one round, then the rows' data four rows at a time
+  constexpr int kMaxRows = 33;  // top_k <= 32, plus the shared row
+  int rows[kMaxRows];
+  const int nr = (sh.Ds > 0 ? 1 : 0) + sh.k;
 #pragma unroll
-    for (int v = 0; v < 4; ++v)
-      if (c0 + 8 * v + 8 <= sh.H) add_bf16x8(acc[v], __ldcg(reinterpret_cast<const uint4*>(yr + c0 + 8 * v)));
-  };
-  if (sh.Ds > 0) add_row((Mr + t / sh.tile_m) * sh.tile_m + t % sh.tile_m);
-  for (int j = 0; j < sh.k; ++j) {
-    const int row = __ldcg(ws.row_of_slot + t * sh.k + j);
-    if (row >= 0) add_row(row);
+  for (int j = 0; j < kMaxRows; ++j) {
+    if (j < nr) {
+      const int jj = sh.Ds > 0 ? j - 1 : j;
+      rows[j] = jj < 0 ? (Mr + t / sh.tile_m) * sh.tile_m + t % sh.tile_m
+                       : __ldcg(ws.row_of_slot + t * sh.k + jj);
+    } else {
+      rows[j] = -1;
+    }
+  }
+#pragma unroll
+  for (int j0 = 0; j0 < kMaxRows; j0 += 4) {
+    if (j0 >= nr) break;
+    uint4 d[4][4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int row = rows[j0 + q < kMaxRows ? j0 + q : 0];
+      const bool use = j0 + q < nr && row >= 0;
+      const uint16_t* yr = ws.y + (size_t)(use ? row : 0) * sh.H;
+#pragma unroll
+      for (int v = 0; v < 4; ++v)
+        d[q][v] = (use && c0 + 8 * v + 8 <= sh.H) ? __ldcg(reinterpret_cast<const uint4*>(yr + c0 + 8 * v))
+                                                   : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int row = rows[j0 + q < kMaxRows ? j0 + q : 0];
+      if (j0 + q < nr && row >= 0) {
+#pragma unroll
+        for (int v = 0; v < 4; ++v) add_bf16x8(acc[v], d[q][v]);
+      }
+    }
   }
 #pragma unroll
   for (int v = 0; v < 4; ++v) {
@@ -757,8 +777,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // whose results land in output rows past the tile's end
       const bool up = (t.kind == kTaskUp);
       const int nbox = (!kSmall && t.nrows <= 3 * kPairBoxRows) ? ceil_div(t.nrows, kPairBoxRows) : 0;
+      // the second tile of a two-tile task: one 32-row box (tail shape), or (two-tile shape) its
+      // 32-row boxes when it has at most 96 rows, else one 128-row box
+      const int nbox2 = t.ntiles != 2 ? 0
+                        : (!C::kTwo || t.nrows2 <= 3 * kPairBoxRows ? ceil_div(t.nrows2, kPairBoxRows) : -1);
       const uint32_t stage_tx = (nbox ? (uint32_t)nbox * kPairBoxRows * kBK * 2 : (uint32_t)kABytes) + kBBytes +
-                                (t.ntiles == 2 ? (uint32_t)kTailRows * kBK * 2 : 0u);
+                                (nbox2 < 0 ? (uint32_t)kABytes : (uint32_t)nbox2 * kPairBoxRows * kBK * 2);
       const CUtensorMap* amap = up ? (shared ? &maps.x_tile : &maps.xs) : (shared ? &maps.h_shared : &maps.h_routed);
       const CUtensorMap* amap32 =
           up ? (shared ? &maps.x_tile32 : &maps.xs32) : (shared ? &maps.h_shared32 : &maps.h_routed32);
@@ -784,7 +808,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             for (int j = 0; j < nbox; ++j)
               tma_load_2d(a + j * kPairBoxRows * 128, amap32, &full[stage], kb * kBK, arow + j * kPairBoxRows);
           }
-          if (kTail && t.ntiles == 2) tma_load_2d(a + kABytes, amap32, &full[stage], kb * kBK, arow2);
+          if (kTail && nbox2 < 0) {
+            tma_load_2d(a + kABytes, amap, &full[stage], kb * kBK, arow2);
+          } else if (kTail) {
+            for (int j = 0; j < nbox2; ++j)
+              tma_load_2d(a + kABytes + j * kPairBoxRows * 128, amap32, &full[stage], kb * kBK,
+                          arow2 + j * kPairBoxRows);
+          }
           if (up) {
             tma_load_2d(b, shared ? &maps.ws_up : &maps.w_up, &full[stage], kb * kBK, wrow_up);
             tma_load_2d(b + kBN1 * 128, shared ? &maps.ws_gate : &maps.w_gate, &full[stage], kb * kBK,
@@ -1168,7 +1198,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 size_t gemm_smem_bytes(int shape) {
   const bool small = shape == kShapeSmall || shape == kShapeSmallFused;
   return (size_t)(small ? Cfg<kShapeSmall>::kBytes
-                        : (shape == kShapeTail ? Cfg<kShapeTail>::kBytes : Cfg<kShapeGeneral>::kBytes)) +
+                        : (shape == kShapeTail ? Cfg<kShapeTail>::kBytes
+                                               : (shape == kShapeTwo ? Cfg<kShapeTwo>::kBytes
+                                                                     : Cfg<kShapeGeneral>::kBytes))) +
          1024;
 }
 
@@ -1180,6 +1212,8 @@ cudaError_t launch_moe_gemm(const GemmMaps& maps, const Workspace& ws, const Sha
     return launch_k(moe_gemm_kernel<kShapeSmall>, dim3(grid), dim3(kGemmThreads), smem, stream, maps, ws, sh, fa);
   if (shape == kShapeTail)
     return launch_k(moe_gemm_kernel<kShapeTail>, dim3(grid), dim3(kGemmThreads), smem, stream, maps, ws, sh, fa);
+  if (shape == kShapeTwo)
+    return launch_k(moe_gemm_kernel<kShapeTwo>, dim3(grid), dim3(kGemmThreads), smem, stream, maps, ws, sh, fa);
   return launch_k(moe_gemm_kernel<kShapeGeneral>, dim3(grid), dim3(kGemmThreads), smem, stream, maps, ws, sh, fa);
 }
 
@@ -1220,6 +1254,9 @@ cudaError_t configure_gemm_kernel() {
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(moe_gemm_kernel<kShapeTail>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)gemm_smem_bytes(kShapeTail));
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(moe_gemm_kernel<kShapeTwo>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)gemm_smem_bytes(kShapeTwo));
   if (e != cudaSuccess) return e;
   return cudaFuncSetAttribute(moe_gemm_kernel<kShapeGeneral>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               (int)gemm_smem_bytes(kShapeGeneral));

@@ -239,11 +239,11 @@ __device__ inline void align_scans(const Workspace& ws, const Shape& sh, bool ti
   auto put_group = [&](int gi, int t0, int g, int last_rows) {
     ws.group_tile0[gi] = t0;
     ws.group_ntiles[gi] = g;
-    ws.group_tasks[gi] = (sh.merge_tail && g == 2 && last_rows <= kTailRows) ? 1 : g;
+    ws.group_tasks[gi] = (g == 2 && (sh.merge_tail == 2 || (sh.merge_tail == 1 && last_rows <= kTailRows))) ? 1 : g;
   };
   // tiles [start, start + g) of group j of a run of nt tiles whose last tile has last_rows rows
   auto group_span = [&](int j, int nt, int last_rows, int& start, int& g) {
-    const int f = (kGroupTiles == 2 && sh.merge_tail && nt > 1 && (nt & 1) && last_rows <= kTailRows) ? 1 : 0;
+    const int f = (kGroupTiles == 2 && sh.merge_tail == 1 && nt > 1 && (nt & 1) && last_rows <= kTailRows) ? 1 : 0;
     start = (f && j > 0) ? kGroupTiles * j - 1 : kGroupTiles * j;
     g = (f && j == 0) ? 1 : min(kGroupTiles, nt - start);
   };

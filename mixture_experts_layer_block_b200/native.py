@@ -33,6 +33,7 @@ MOE_FLAG_NO_TAIL_TILES = 128
 MOE_FLAG_STATIC_QUOTA = 256
 MOE_FLAG_MXFP8 = 512
 MOE_FLAG_UNFUSED_SMALL = 1024
+MOE_FLAG_TWO_TILES = 2048
 MOE_FLAG_TRACE = 4
 
 

@@ -44,10 +44,11 @@ def _flags():
     from mixture_experts_layer_block_b200 import native
     return {"pair": native.MOE_FLAG_PAIR_TILES, "single": native.MOE_FLAG_SINGLE_TILES,
             "general": native.MOE_FLAG_SINGLE_TILES | native.MOE_FLAG_NO_TAIL_TILES,
-            "tail": native.MOE_FLAG_SINGLE_TILES | native.MOE_FLAG_TAIL_TILES}
+            "tail": native.MOE_FLAG_SINGLE_TILES | native.MOE_FLAG_TAIL_TILES,
+            "two": native.MOE_FLAG_SINGLE_TILES | native.MOE_FLAG_TWO_TILES}
 
 
-SHAPE_CODE = {"general": 0, "small": 1, "tail": 2, "pair": 3}
+SHAPE_CODE = {"general": 0, "small": 1, "tail": 2, "pair": 3, "two": 5}
 
 
 @pytest.mark.parametrize("name", sorted(SMALL))
@@ -65,7 +66,7 @@ def test_forward_small_all_tokens(name):
 # Every shape of the expert GEMMs for batches of more than 16 tokens (256-row tiles on SM
 # pairs; 128-row tiles on single SMs, with or without merged tails) on every small case: tiles
 # of 1..256 rows, split between the two CTAs of a pair at every boundary the split rule has.
-@pytest.mark.parametrize("shape", ["pair", "general", "tail"])
+@pytest.mark.parametrize("shape", ["pair", "general", "tail", "two"])
 @pytest.mark.parametrize("name", sorted(n for n, w in SMALL.items() if w.T > 16))
 def test_forward_small_tile_shapes(name, shape):
     w = SMALL[name]
@@ -202,13 +203,14 @@ def test_forward_bf16_out(name):
         l16.forward(inp["x"], inp, o32)
 
 
-@pytest.mark.parametrize("shape", ["tail", "general"])
-@pytest.mark.parametrize("nrows", [129, 140, 160, 161, 256, 288, 289, 300, 416, 417, 513])
+@pytest.mark.parametrize("shape", ["tail", "general", "two"])
+@pytest.mark.parametrize("nrows", [129, 140, 160, 161, 200, 225, 256, 288, 289, 300, 416, 417, 513])
 def test_single_sm_merged_tails_one_expert(nrows, shape):
     """Every token routed to expert 0 (top-1 of 2 with a large bias) and the shared expert over
-    the same tokens: runs of 128-row tiles ending in tails of 1..33+ rows. A tail of at most 32
-    rows rides in the tasks of the tile before it (an odd run starts with a single tile so the
-    tail closes a pair); a longer one keeps its own tasks."""
+    the same tokens: runs of 128-row tiles ending in tails of 1..128 rows. Tail shape: a tail of at
+    most 32 rows rides in the tasks of the tile before it (an odd run starts with a single tile so
+    the tail closes a pair), a longer one keeps its own tasks. Two-tile shape: every pair of tiles
+    (second tile of any size, loaded as 32-row boxes up to 96 rows) runs as one task set."""
     w = configs.MoEWorkload(f"tails_{nrows}", T=nrows, H=256, D=384, E=2, top_k=1, block_m=16,
                             D_shared=128, sigma_w=0.05)
     inp = {k: (v.cuda() if v is not None else None) for k, v in gen.make_inputs(w).items()}
