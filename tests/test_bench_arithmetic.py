@@ -87,3 +87,32 @@ def test_per_config_plan_covers_every_workload_and_the_decode_seeds():
     keys = [k for k, *_ in bench.per_config_plan()]
     assert len(keys) == len(set(keys))
     assert any(k.startswith("static_quota/") for k in keys) and any(k.startswith("mxfp8/") for k in keys)
+
+
+def test_wait_fractions_and_front_timeline():
+    """The traced forward's per-CTA wait totals become fractions of each role's loop, and the
+    fused front's timeline medians (the scheduling CTA's steps apart)."""
+    import numpy as np
+    names = ("prod_empty", "prod_dep", "prod_ring", "prod_claim", "mma_full", "mma_acc", "mma_task",
+             "epi_task", "epi_acc", "prod_loop", "mma_loop", "epi_loop", "front_router", "front_schedule",
+             "front_gather", "front_last", "front_to_end", "sched_arrive", "sched_logits", "sched_gating",
+             "sched_tables", "sched_writes", "sched_publish")
+    w = np.zeros((4, len(names)), dtype=np.int64)
+    col = {n: i for i, n in enumerate(names)}
+    w[:, col["mma_loop"]] = 1000
+    w[:, col["mma_full"]] = [600, 700, 500, 200]
+    w[:, col["prod_loop"]] = 1000
+    w[:, col["prod_empty"]] = 250
+    w[:, col["epi_loop"]] = 1000
+    w[:, col["front_router"]] = [3000, 4000, 5000, 6000]
+    w[:, col["front_schedule"]] = [10000, 12000, 14000, 9000]
+    w[:, col["front_last"]] = [0, 0, 0, 1]
+    w[:, col["front_to_end"]] = [80000, 81000, 82000, 90000]
+    w[3, col["sched_gating"]] = 4000
+    f = bench.wait_fractions(w, names)
+    assert f["mma"]["operands"] == pytest.approx(2000 / 4000)
+    assert f["producer"]["free_stage"] == pytest.approx(0.25)
+    fr = f["front_us"]
+    assert fr["schedule_compute"] == pytest.approx(9.0) and fr["schedule_wait"] == pytest.approx(12.0)
+    assert fr["router"] == pytest.approx(4.5) and fr["max_front_to_end"] == pytest.approx(90.0)
+    assert fr["schedule_steps"]["gating"] == pytest.approx(4.0)
