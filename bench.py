@@ -186,10 +186,15 @@ def layer_fraction(w, peaks, ms, kept, hit, mx):
             "algorithmic_bytes": b, "useful_flops": flops}
 
 
+# handle options the command line sets once for every layer bench.py builds
+LAYER_KW = {}
+
+
 def tile_flags(args) -> int:
     from mixture_experts_layer_block_b200 import native
     f = {"auto": 0, "pair": native.MOE_FLAG_PAIR_TILES, "single": native.MOE_FLAG_SINGLE_TILES,
-         "two": native.MOE_FLAG_TWO_TILES}[getattr(args, "tiles", "auto")]
+         "two": native.MOE_FLAG_TWO_TILES, "tail": native.MOE_FLAG_TAIL_TILES,
+         "general": native.MOE_FLAG_NO_TAIL_TILES}[getattr(args, "tiles", "auto")]
     if getattr(args, "sched", "dynamic") == "static":
         f |= native.MOE_FLAG_STATIC_QUOTA
     if getattr(args, "unfused_small", False):
@@ -208,14 +213,14 @@ def run_forward(layer, x, wts, out, wq=None):
 def traced_forward(w, wts, x, out, extra_flags=0, wq=None):
     """One extra forward with per-task tracing (outside the timed region)."""
     from mixture_experts_layer_block_b200.native import MOE_FLAG_MXFP8, MOE_FLAG_TRACE, MoELayer
-    layer = MoELayer.for_workload(w, flags=MOE_FLAG_TRACE | extra_flags | (MOE_FLAG_MXFP8 if wq else 0))
+    layer = MoELayer.for_workload(w, flags=MOE_FLAG_TRACE | extra_flags | (MOE_FLAG_MXFP8 if wq else 0), **LAYER_KW)
     for _ in range(2):
         run_forward(layer, x, wts, out, wq)
     torch.cuda.synchronize()
     rec = layer.trace(1 << 20)
     n_ctas = layer.query(1)
     res = sm_busy_fraction(rec, n_ctas)
-    if wq is None and layer.query(8) != 3:
+    if layer.query(8) != 3:  # every expert-GEMM kernel but the SM-pair one keeps wait accounting
         res["waits"] = wait_fractions(layer.trace_waits(), MoELayer.WAITS)
     layer.close()
     return res
@@ -502,7 +507,7 @@ def measure(w, dev, world, rank, steps, warmup, peaks, flusher, mx=False, flags=
     wts = gen.make_weights(w, dev)
     x = gen.make_x(w.replace(seed=w.seed + 1000 * rank) if rank else w, dev)  # each replica its own tokens
     out = torch.empty((w.T, w.H), dtype=torch.float32, device=dev)
-    layer = MoELayer.for_workload(w, flags=(MOE_FLAG_HOST_STAGING if keep else 0) | prec | flags)
+    layer = MoELayer.for_workload(w, flags=(MOE_FLAG_HOST_STAGING if keep else 0) | prec | flags, **LAYER_KW)
     stream = torch.cuda.current_stream(dev)
     wq = layer.quantize_experts_mxfp8(wts) if mx else None  # weights are stored quantised
     for _ in range(warmup):
@@ -512,7 +517,7 @@ def measure(w, dev, world, rank, steps, warmup, peaks, flusher, mx=False, flags=
     assert rc == 0 and st == 0, (w.name, rc, st)
     stats = routing_stats(layer, w, dev)
     shape = {"tile_m": layer.query(6), "workers": layer.query(1), "shape": layer.query(8), "scheduler": sched,
-             "kernels_per_forward": layer.query(11)}
+             "kernels_per_forward": layer.query(11), "claim_batch": max(1, LAYER_KW.get("claim_batch", 1))}
     with ClockSampler(dev.index if dev.index is not None else 0) as clk:
         ms = timed_steps(layer, x, wts, out, wq, steps, stream, world)
     ms_flushed = timed_steps(layer, x, wts, out, wq, steps, stream, world, flusher)
@@ -521,7 +526,7 @@ def measure(w, dev, world, rank, steps, warmup, peaks, flusher, mx=False, flags=
 
     # per-kernel durations: a separate pass whose handle records CUDA events around every kernel
     # on the launching stream (events between kernels stop them from overlapping)
-    lt = MoELayer.for_workload(w, flags=MOE_FLAG_STAGE_TIMING | prec | flags)
+    lt = MoELayer.for_workload(w, flags=MOE_FLAG_STAGE_TIMING | prec | flags, **LAYER_KW)
     for _ in range(3):
         run_forward(lt, x, wts, out, wq)
     torch.cuda.synchronize()
@@ -656,7 +661,7 @@ def run_profile(args, local):
     wts = gen.make_weights(w, dev)
     x = gen.make_x(w, dev)
     out = torch.empty((w.T, w.H), dtype=torch.float32, device=dev)
-    layer = MoELayer.for_workload(w, flags=(MOE_FLAG_MXFP8 if mx else 0) | tile_flags(args))
+    layer = MoELayer.for_workload(w, flags=(MOE_FLAG_MXFP8 if mx else 0) | tile_flags(args), **LAYER_KW)
     wq = layer.quantize_experts_mxfp8(wts) if mx else None
     for _ in range(args.warmup):
         run_forward(layer, x, wts, out, wq)
@@ -759,9 +764,10 @@ def main():
     ap.add_argument("--ref-tokens", type=int, default=256)
     ap.add_argument("--T", type=int, default=None, help="override the workload's token count (profiling)")
     ap.add_argument("--E", type=int, default=None, help="override the workload's expert count (profiling)")
-    ap.add_argument("--tiles", choices=["auto", "pair", "single", "two"], default="auto",
+    ap.add_argument("--tiles", choices=["auto", "pair", "single", "two", "tail", "general"], default="auto",
                     help="expert-GEMM shape: the library's choice, 256-row tiles on SM pairs, "
-                         "128-row tiles on single SMs, or two 128-row tiles per task on single SMs")
+                         "128-row tiles on single SMs (the library's merge choice), two 128-row tiles "
+                         "per task, tails of <= 32 rows merged into the previous tile, or no merging")
     ap.add_argument("--sched", choices=["dynamic", "static"], default="dynamic",
                     help="task scheduling of the expert GEMMs: the atomic queue, or the static "
                          "per-expert SM quota baseline (ablation)")
@@ -773,7 +779,11 @@ def main():
                     help="ncu dram bytes per launch of the expert-GEMM kernel, if captured")
     ap.add_argument("--profile", action="store_true",
                     help="only the warm-up and the K timed forwards of --workload (for profiler captures)")
+    ap.add_argument("--claim-batch", type=int, default=0,
+                    help="expert-GEMM task ids a CTA takes per claim on the shared counter (0 = 1)")
     args = ap.parse_args()
+    if args.claim_batch:
+        LAYER_KW["claim_batch"] = args.claim_batch
     world, rank, local = dist_setup()
     try:
         if args.impl == "reference":

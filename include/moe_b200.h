@@ -71,11 +71,13 @@ extern "C" {
 /* moe_forward / moe_forward_host write `out` as bf16 [T][H] (the fp32 sum rounded to nearest
  * even once) instead of fp32 [T][H]. */
 #define MOE_FLAG_OUT_BF16     32u
-/* The one-SM expert GEMMs can compute a tile's tail of at most 32 rows inside the tasks of the
- * expert's previous tile, from the same weight stages (the "tail" shape). By default they do so
- * when the mean load per expert is 96..384 slots and the capacity allows more than 128;
- * MOE_FLAG_TAIL_TILES asks for it on every batch of more than 16 tokens, MOE_FLAG_NO_TAIL_TILES
- * never (it wins). Both compute the same result. */
+/* The one-SM expert GEMMs can merge m-tiles of one expert into one task set, computed from the
+ * same weight stages: a tile's tail of at most 32 rows inside the tasks of the expert's previous
+ * tile (the "tail" shape, MOE_FLAG_TAIL_TILES), or every group of two tiles (the "two-tile"
+ * shape, MOE_FLAG_TWO_TILES, below). By default the two-tile shape runs when the mean load per
+ * expert is above 96 slots and the capacity allows more than 128, else neither;
+ * MOE_FLAG_NO_TAIL_TILES turns the default off (the flags that ask for a shape win over it). All
+ * compute the same result. */
 #define MOE_FLAG_TAIL_TILES   64u
 #define MOE_FLAG_NO_TAIL_TILES 128u
 /* Ablation baseline, not for production (the static per-expert SM quota of a fused MoE kernel
@@ -102,7 +104,7 @@ extern "C" {
 /* The one-SM expert GEMMs of batches of more than 16 tokens run every group of two m-tiles of one
  * expert as one task set: each task computes both tiles from the same weight stages into the two
  * TMEM accumulators (a 3-stage ring of 64 KB stages; the "two-tile" shape, moe_query 8 reports 5).
- * It wins over the tail and general shapes; the same result. */
+ * Wins over MOE_FLAG_TAIL_TILES; the same result. */
 #define MOE_FLAG_TWO_TILES    2048u
 
 typedef struct moe_config {
@@ -117,6 +119,11 @@ typedef struct moe_config {
     uint32_t flags;           /* MOE_FLAG_* */
     int32_t device;           /* CUDA device ordinal; -1 = the calling thread's current device */
     int64_t timeout_ns;       /* limit of every device-side wait; <= 0 = 2e9 (2 s) */
+    int32_t claim_batch;      /* expert-GEMM tasks a CTA takes per claim on the shared counter,
+                               * 0..64 (0 = 1). A CTA runs its batch's consecutive ids in order;
+                               * larger batches mean fewer atomics on the counter but coarser load
+                               * balance at the end of the queue (the two-level queue of the Weave
+                               * blog, section 5.2). Same result for every value. */
 } moe_config;
 
 typedef struct moe_handle moe_handle;
@@ -329,7 +336,7 @@ MOE_API int moe_query(const moe_handle *h, int32_t which, int64_t *value);
  * sets *n to the records written. */
 MOE_API int moe_trace_read(moe_handle *h, int64_t *records, int64_t cap, int64_t *n);
 
-/* Wait accounting of the last bf16 forward's expert-GEMM kernel (needs MOE_FLAG_TRACE;
+/* Wait accounting of the last forward's expert-GEMM kernel, bf16 or MXFP8 (needs MOE_FLAG_TRACE;
  * synchronises): per CTA (row) int64 %globaltimer ns summed over its tasks --
  *   0 producer waiting for a free operand stage     1 producer waiting for a down task's up
  *   2 producer waiting for a free task-ring entry      tasks (fused: for a tile's gathered rows)

@@ -195,6 +195,8 @@ struct FrontArgs {
 };
 
 // Shapes and knobs of one forward, passed by value.
+constexpr int kMaxClaimBatch = 64;  // largest moe_config.claim_batch
+
 struct Shape {
   int32_t T, H, D, Ds, E, k, block_m;
   int32_t capacity;      // C, 0 = dropless
@@ -208,6 +210,7 @@ struct Shape {
                          //    task set (the one-SM tail shape); 2: every group of two tiles does
                          //    (the two-tile shape); 0: never
   int32_t static_quota;  // 1: each CTA works through a fixed share of the experts (ablation)
+  int32_t claim_batch;   // consecutive task ids one claim on the counter takes (>= 1)
   int64_t timeout_ns;
 };
 

@@ -309,11 +309,7 @@ __device__ void front_schedule(const FrontArgs& fa, const Workspace& ws, const S
       ws.group_ntiles[t0] = 1;
       ws.group_tasks[t0] = 1;
     }
-    for (int i = o + kp; i < end; ++i) ws.sorted_ids[i] = S;  // the segment's padding
-    for (int b = o / bm; b < end / bm; ++b) ws.expert_ids[b] = e;
   }
-  for (int i = P + tid; i < sh.sorted_len; i += nthr) ws.sorted_ids[i] = S;
-  for (int b = P / bm + tid; b < sh.blocks_len; b += nthr) ws.expert_ids[b] = -1;
   // slot s = t*k + j: its rank in its expert is the number of earlier tokens that chose it
   for (int s = tid; s < S; s += nthr) {
     const int t = s / k, e = ids_s[s];
@@ -390,6 +386,15 @@ __device__ void front_schedule(const FrontArgs& fa, const Workspace& ws, const S
     ws.front->front_done = 0;  // every CTA has arrived: ready for the next forward
     st_release_gpu(&ws.front->sched_flag, fa.epoch);
   }
+  // the rest of the align outputs (the padding sentinels of sorted_ids and expert_ids), which
+  // nothing in this launch reads: after the schedule is out, before this CTA's own tasks
+  for (int e = tid; e < E; e += nthr) {
+    const int o = off[e], end = off[e + 1];
+    for (int i = o + kept[e]; i < end; ++i) ws.sorted_ids[i] = S;  // the segment's padding
+    for (int b = o / bm; b < end / bm; ++b) ws.expert_ids[b] = e;
+  }
+  for (int i = P + tid; i < sh.sorted_len; i += nthr) ws.sorted_ids[i] = S;
+  for (int b = P / bm + tid; b < sh.blocks_len; b += nthr) ws.expert_ids[b] = -1;
 }
 
 // Bounded wait (one thread) until the schedule of forward `epoch` is published. Only the time
@@ -638,8 +643,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // task is one no idle CTA can take at the end of the queue). The held id is always the next
     // task this producer starts, and every task it waits for has a smaller id, so the smallest
     // unfinished task still always makes progress.
-    int next_tau = 0;
-    if (!sh.static_quota && lane == 0) next_tau = atomicAdd(&meta->task_counter, 1);
+    // A claim takes sh.claim_batch consecutive ids; batch_end is one past the held batch.
+    const uint64_t w_policy = kSmall ? policy_evict_first() : 0;
+    int next_tau = 0, batch_end = 0;
+    if (!sh.static_quota && lane == 0) {
+      next_tau = atomicAdd(&meta->task_counter, sh.claim_batch);
+      batch_end = next_tau + sh.claim_batch;
+    }
     // with the task table, the claimed task's entry is loaded one stage after the claim
     const bool use_tab = ws.task_tab != nullptr && !sh.static_quota;
     int4 next_ent = make_int4(0, 0, 0, 0);
@@ -815,15 +825,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               tma_load_2d(a + kABytes + j * kPairBoxRows * 128, amap32, &full[stage], kb * kBK,
                           arow2 + j * kPairBoxRows);
           }
+          // B: weight rows. At most 16 tokens, every expert has one tile and its weights are read
+          // exactly once: they are loaded with an evict-first L2 hint, so that streaming them does
+          // not push out of L2 what the forward reads again (x, h, y, the schedule, its code)
+          auto load_w = [&](uint32_t dst, const CUtensorMap* map, int c1) {
+            if constexpr (kSmall)
+              tma_load_2d_hint(dst, map, &full[stage], kb * kBK, c1, w_policy);
+            else
+              tma_load_2d(dst, map, &full[stage], kb * kBK, c1);
+          };
           if (up) {
-            tma_load_2d(b, shared ? &maps.ws_up : &maps.w_up, &full[stage], kb * kBK, wrow_up);
-            tma_load_2d(b + kBN1 * 128, shared ? &maps.ws_gate : &maps.w_gate, &full[stage], kb * kBK,
-                        wrow_up);
+            load_w(b, shared ? &maps.ws_up : &maps.w_up, wrow_up);
+            load_w(b + kBN1 * 128, shared ? &maps.ws_gate : &maps.w_gate, wrow_up);
           } else {
-            tma_load_2d(b, shared ? &maps.ws_down : &maps.w_down, &full[stage], kb * kBK, wrow_dn);
+            load_w(b, shared ? &maps.ws_down : &maps.w_down, wrow_dn);
           }
         }
-        if (kb == claim_kb && !sh.static_quota && lane == 0) next_tau = atomicAdd(&meta->task_counter, 1);
+        if (kb == claim_kb && !sh.static_quota && lane == 0) {
+          if (tau + 1 < batch_end) {
+            next_tau = tau + 1;
+          } else {
+            next_tau = atomicAdd(&meta->task_counter, sh.claim_batch);
+            batch_end = next_tau + sh.claim_batch;
+          }
+        }
         if (kb == claim_kb + 1 && use_tab && lane == 0 && next_tau < total) {
           next_ent = __ldcg(ws.task_tab + next_tau);
           ent_tau = next_tau;

@@ -47,6 +47,7 @@ struct MxCfg {
   static constexpr uint32_t kSfColsPerStage = 16;
   static_assert(kStageBytes % 1024 == 0 && kSfOff % 1024 == 0, "1024-byte aligned operand tiles");
   static_assert(kBytes + 1024 <= 227 * 1024, "shared memory budget");
+  static_assert(kMiscOff % 8 == 0, "8-byte words in the misc area");
   static_assert(kSfCol0 + kStages * kSfColsPerStage <= 2 * kAccCols, "TMEM budget");
 };
 
@@ -110,6 +111,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint32_t nfill = 0;
   bool mma_issued = false;
 
+  // wait accounting while tracing, as in the bf16 kernel (globaltimer ns; each role's recording
+  // thread keeps its own sums and adds them to its CTA's row at the end of its loop)
+  const bool tracing = ws.trace_cap > 0;
+  auto now = [&]() -> int64_t { return tracing ? (int64_t)globaltimer_ns() : 0; };
+  auto add_wait = [&](int kind, int64_t v) {
+    if (tracing && ws.waits != nullptr && v != 0)
+      atomicAdd(reinterpret_cast<unsigned long long*>(ws.waits + (size_t)blockIdx.x * kNumWaits + kind),
+                (unsigned long long)v);
+  };
+
   if (warp == 0) {
     // ===================================== producer =====================================
     const int total = __ldcg(&meta->total_tasks);
@@ -118,9 +129,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int H = sh.H;
     int u_cur = 0;
     uint32_t stage = 0, phase = 0, slot = 0, slot_phase = 0;
+    // claims as in the bf16 kernel: the next id while the current task's last ring-depth of
+    // stages is issued, its task-table entry one stage later
+    const bool weights_once = sh.T <= kSmallRows;
+    const uint64_t w_policy = weights_once ? policy_evict_first() : 0;
+    int next_tau = 0, batch_end = 0;
+    if (lane == 0) {
+      next_tau = atomicAdd(&meta->task_counter, sh.claim_batch);
+      batch_end = next_tau + sh.claim_batch;
+    }
+    const bool use_tab = ws.task_tab != nullptr;
+    int4 next_ent = make_int4(0, 0, 0, 0);
+    int ent_tau = -1;
+    const int64_t t_loop = now();
+    int64_t w_empty = 0, w_dep = 0, w_ring = 0, w_claim = 0;
     while (true) {
+      const int64_t t_top = now();
       int tau = 0;
-      if (lane == 0) tau = aborted(meta, s_abort) ? total : atomicAdd(&meta->task_counter, 1);
+      if (lane == 0) tau = aborted(meta, s_abort) ? total : next_tau;
       tau = __shfl_sync(0xffffffffu, tau, 0);
       Task t;
       t.id = tau;
@@ -128,6 +154,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       t.nrows2 = 0;
       if (tau >= total) {
         t.kind = kTaskStop;
+      } else if (use_tab) {
+        int4 ent = next_ent;
+        if (lane == 0 && ent_tau != tau) ent = __ldcg(ws.task_tab + tau);
+        ent.x = __shfl_sync(0xffffffffu, ent.x, 0);
+        ent.y = __shfl_sync(0xffffffffu, ent.y, 0);
+        ent.z = __shfl_sync(0xffffffffu, ent.z, 0);
+        ent.w = __shfl_sync(0xffffffffu, ent.w, 0);
+        t.tile = ent.x;
+        t.expert = ent.y;
+        t.row0 = ent.z;
+        t.nrows = ent.w & 511;
+        t.kind = (ent.w >> 19) & 1;
+        const int nt = ent.w >> 20;
+        const int Dt = (t.expert == sh.E) ? sh.Ds : sh.D;
+        if (t.kind == kTaskUp) {
+          t.n0 = nt * kBN1;
+          t.nk = H / kMxBK;
+        } else {
+          t.n0 = nt * kBN2;
+          t.nk = Dt / kMxBK;
+        }
       } else {
         u_cur = find_unit(ws.unit_start, U, tau, u_cur);
         const TaskPos pos = decode_task(ws, sh, u_cur, tau, Mg, Mgr);
@@ -147,15 +194,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       bool ok = true;
       if (lane == 0) {
+        const int64_t t0 = now();
         ok = wait_bar(&task_empty[slot], slot_phase ^ 1, meta, s_abort, limit, kSiteProducerTask);
         if (ok) {
           ring[slot] = t;
           mbar_arrive(&task_full[slot]);
         }
+        w_ring += now() - t0;
+        w_claim += t0 - t_top;
       }
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       if (!ok || t.kind == kTaskStop) break;
       if (++slot == kTaskSlots) { slot = 0; slot_phase ^= 1; }
+      const int claim_kb = t.nk > kStages ? t.nk - kStages : 0;
       if (ws.trace_cap > 0 && lane == 0 && tau < ws.trace_cap) {
         ws.trace[(size_t)tau * 4 + 0] = blockIdx.x;
         ws.trace[(size_t)tau * 4 + 1] = tau;
@@ -165,8 +216,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const bool up = (t.kind == kTaskUp);
       if (!up) {
         if (lane == 0) {
+          const int64_t t0 = now();
           ok = wait_count(&ws.done1[t.tile], n1_of(t.expert, sh) + sh.dep_extra, meta, s_abort, limit);
           if (ok) fence_proxy_async_global();  // h (codes and scales) is read by the async proxy
+          w_dep += now() - t0;
         }
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         if (!ok) break;
@@ -202,7 +255,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       const uint32_t stage_tx = a_bytes + (uint32_t)C::kBBytes + kSfAtomBytes + sfb_bytes;
       for (int kb = 0; kb < t.nk; ++kb) {
-        if (lane == 0) ok = wait_bar(&empty[stage], phase ^ 1, meta, s_abort, limit, kSiteProducerEmpty);
+        if (lane == 0) {
+          const int64_t t0 = now();
+          ok = wait_bar(&empty[stage], phase ^ 1, meta, s_abort, limit, kSiteProducerEmpty);
+          w_empty += now() - t0;
+        }
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         if (!ok) break;
         if (lane == 0) {
@@ -216,16 +273,36 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             for (int j = 0; j < nbox; ++j)
               tma_load_2d(a + j * kPairBoxRows * kMxBK, amap32, &full[stage], kb * kMxBK, arow + j * kPairBoxRows);
           }
+          // weights read exactly once (at most 16 tokens: one tile per expert) carry an
+          // evict-first L2 hint, as in the bf16 kernel
+          auto load_w = [&](uint32_t dst, const CUtensorMap* map, int c1) {
+            if (weights_once)
+              tma_load_2d_hint(dst, map, &full[stage], kb * kMxBK, c1, w_policy);
+            else
+              tma_load_2d(dst, map, &full[stage], kb * kMxBK, c1);
+          };
           if (up) {
-            tma_load_2d(b, shared ? &maps.ws_up : &maps.w_up, &full[stage], kb * kMxBK, wrow_up);
-            tma_load_2d(b + kBN1 * kMxBK, shared ? &maps.ws_gate : &maps.w_gate, &full[stage], kb * kMxBK, wrow_up);
+            load_w(b, shared ? &maps.ws_up : &maps.w_up, wrow_up);
+            load_w(b + kBN1 * kMxBK, shared ? &maps.ws_gate : &maps.w_gate, wrow_up);
           } else {
-            tma_load_2d(b, shared ? &maps.ws_down : &maps.w_down, &full[stage], kb * kMxBK, wrow_dn);
+            load_w(b, shared ? &maps.ws_down : &maps.w_down, wrow_dn);
           }
           bulk_load(sf, sfa + (size_t)kb * kSfAtomBytes, kSfAtomBytes, &full[stage]);
           bulk_load(sf + kSfAtomBytes, sfb0 + (size_t)kb * kSfAtomBytes, kSfAtomBytes, &full[stage]);
           if (sfb_bytes > kSfAtomBytes)
             bulk_load(sf + 2 * kSfAtomBytes, sfb1 + (size_t)kb * kSfAtomBytes, kSfAtomBytes, &full[stage]);
+        }
+        if (kb == claim_kb && lane == 0) {
+          if (tau + 1 < batch_end) {
+            next_tau = tau + 1;
+          } else {
+            next_tau = atomicAdd(&meta->task_counter, sh.claim_batch);
+            batch_end = next_tau + sh.claim_batch;
+          }
+        }
+        if (kb == claim_kb + 1 && use_tab && lane == 0 && next_tau < total) {
+          next_ent = __ldcg(ws.task_tab + next_tau);
+          ent_tau = next_tau;
         }
         __syncwarp();
         ++nfill;
@@ -233,19 +310,34 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       if (!ok) break;
     }
+    if (lane == 0) {
+      add_wait(kWaitProdLoop, now() - t_loop);
+      add_wait(kWaitProdEmpty, w_empty);
+      add_wait(kWaitProdDep, w_dep);
+      add_wait(kWaitProdRing, w_ring);
+      add_wait(kWaitProdClaim, w_claim);
+    }
   } else if (warp == 1) {
     // ===================================== MMA issuer ===================================
     if (lane == 0) {
       uint32_t stage = 0, phase = 0, slot = 0, slot_phase = 0, use = 0;
+      const int64_t t_loop = now();
+      int64_t w_task = 0, w_acc = 0, w_full = 0;
       while (true) {
+        int64_t t0 = now();
         if (!wait_bar(&task_full[slot], slot_phase, meta, s_abort, limit, kSiteMmaTask)) break;
+        w_task += now() - t0;
         const Task t = ring[slot];
         if (t.kind == kTaskStop) break;
+        t0 = now();
         if (!wait_bar(acc_empty, (use & 1u) ^ 1u, meta, s_abort, limit, kSiteMmaAcc)) break;
+        w_acc += now() - t0;
         tc_fence_after();
         bool ok = true;
         for (int kb = 0; kb < t.nk; ++kb) {
+          t0 = now();
           if (!wait_bar(&full[stage], phase, meta, s_abort, limit, kSiteMmaFull)) { ok = false; break; }
+          w_full += now() - t0;
           tc_fence_after();
           const uint32_t a = smem_u32(smem + stage * C::kStageBytes);
           const uint32_t b = a + C::kABytes;
@@ -270,6 +362,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         mbar_arrive(&task_empty[slot]);
         if (++slot == kTaskSlots) { slot = 0; slot_phase ^= 1; }
       }
+      add_wait(kWaitMmaLoop, now() - t_loop);
+      add_wait(kWaitMmaTask, w_task);
+      add_wait(kWaitMmaAcc, w_acc);
+      add_wait(kWaitMmaFull, w_full);
     }
     __syncwarp();
   } else {
@@ -279,14 +375,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const bool leader = (warp == 2 && lane == 0);
     uint8_t* staging = smem + C::kStagingOff;
     uint32_t slot = 0, slot_phase = 0, use = 0;
+    // the leader's wait sums live in shared memory (no registers held across the loop)
+    int64_t* s_ewait = reinterpret_cast<int64_t*>(smem + C::kMiscOff + 16);  // [3]
+    if (leader) s_ewait[0] = s_ewait[1] = 0, s_ewait[2] = now();
     const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     // the leader waits for the next task and the accumulator and tells the others (the four
     // warps always take the same branch); the decision word is double-buffered
     auto epilogue_next = [&](uint32_t it) -> bool {
       if (leader) {
         int go = 0;
-        if (wait_bar(&task_full[slot], slot_phase, meta, s_abort, limit, kSiteEpiTask) && ring[slot].kind != kTaskStop)
+        const int64_t t0 = now();
+        if (wait_bar(&task_full[slot], slot_phase, meta, s_abort, limit, kSiteEpiTask) && ring[slot].kind != kTaskStop) {
+          const int64_t t1 = now();
+          s_ewait[0] += t1 - t0;
           go = wait_bar(acc_full, use & 1u, meta, s_abort, limit, kSiteEpiAcc) ? 1 : 0;
+          s_ewait[1] += now() - t1;
+        }
         s_epi_go[it & 1] = go;
       }
       named_bar_sync(1, 128);
@@ -323,34 +427,50 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (!epilogue_next(it)) break;
       const Task t = ring[slot];
       const bool shared = (t.expert == sh.E);
+      // a partial tile (decode batches, tails): warps without valid rows skip the accumulator,
+      // and the valid rows go straight from registers to global memory (no staging, no TMA
+      // store of 128 rows)
+      const bool direct = t.nrows < kBM;
+      const bool has_rows = q * 32 < t.nrows;  // warp-uniform
+      const bool valid = row < t.nrows;
       if (t.kind == kTaskUp) {
         // h = SiLU(U) * G for 128 columns, quantised per 32 columns
         uint32_t codes[32];
         uint32_t scales = 0;
+        if (has_rows || !direct) {
 #pragma unroll
-        for (int j = 0; j < kBN1 / kMxBlock; ++j) {
-          uint32_t u[32], g[32];
-          tmem_ld_32x32b_x32(tacc + j * 32, u);
-          tmem_ld_32x32b_x32(tacc + kBN1 + j * 32, g);
-          tmem_ld_wait();
-          if (j == kBN1 / kMxBlock - 1) release_acc();
-          float hv[32];
+          for (int j = 0; j < kBN1 / kMxBlock; ++j) {
+            uint32_t u[32], g[32];
+            tmem_ld_32x32b_x32(tacc + j * 32, u);
+            tmem_ld_32x32b_x32(tacc + kBN1 + j * 32, g);
+            tmem_ld_wait();
+            if (j == kBN1 / kMxBlock - 1) release_acc();
+            float hv[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float uu = __uint_as_float(u[i]);
-            hv[i] = __fdividef(uu, 1.0f + __expf(-uu)) * __uint_as_float(g[i]);
+            for (int i = 0; i < 32; ++i) {
+              const float uu = __uint_as_float(u[i]);
+              hv[i] = __fdividef(uu, 1.0f + __expf(-uu)) * __uint_as_float(g[i]);
+            }
+            uint32_t w8[8];
+            scales |= mx_quantize_block(hv, w8) << (8 * j);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) codes[8 * j + i] = w8[i];
           }
-          uint32_t w8[8];
-          scales |= mx_quantize_block(hv, w8) << (8 * j);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) codes[8 * j + i] = w8[i];
+          // this row's four scales: one 32-bit word of the tile's atom for these 128 columns
+          *reinterpret_cast<uint32_t*>(mx.sf_h + mx_atom_offset(t.tile, t.n0 / kMxBK, ws.ldh) + lane * 16 + q * 4) =
+              scales;
+        } else {
+          release_acc();
         }
-        // this row's four scales: one 32-bit word of the tile's atom for these 128 columns
-        *reinterpret_cast<uint32_t*>(mx.sf_h + mx_atom_offset(t.tile, t.n0 / kMxBK, ws.ldh) + lane * 16 + q * 4) =
-            scales;
-        store_box(&maps.h, codes, t.n0, t.tile * kBM);
-        // publish h: codes (TMA store) and scales (plain stores) must be visible to the async
-        // proxy of other SMs before the tile's counter moves
+        if (!direct) {
+          store_box(&maps.h, codes, t.n0, t.tile * kBM);
+        } else if (valid) {
+          uint4* hrow = reinterpret_cast<uint4*>(mx.h + (size_t)(t.tile * kBM + row) * ws.ldh + t.n0);
+#pragma unroll
+          for (int v = 0; v < 8; ++v) hrow[v] = make_uint4(codes[4 * v], codes[4 * v + 1], codes[4 * v + 2], codes[4 * v + 3]);
+        }
+        // publish h: codes (TMA store or plain stores) and scales (plain stores) must be visible
+        // to the async proxy of other SMs before the tile's counter moves
         fence_proxy_async_global();
         __threadfence();
         named_bar_sync(1, 128);
@@ -370,20 +490,33 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             w = __ldcg(&ws.topk_w[s]);
           }
         }
+        if (has_rows || !direct) {
+          uint16_t* yrow = ws.y + (size_t)(t.tile * kBM + row) * sh.H;
 #pragma unroll 1
-        for (int cc = 0; cc < kBN2 / 64; ++cc) {
-          uint32_t pk[32];
+          for (int cc = 0; cc < kBN2 / 64; ++cc) {
+            uint32_t pk[32];
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            uint32_t v[32];
-            tmem_ld_32x32b_x32(tacc + cc * 64 + half * 32, v);
-            tmem_ld_wait();
+            for (int half = 0; half < 2; ++half) {
+              uint32_t v[32];
+              tmem_ld_32x32b_x32(tacc + cc * 64 + half * 32, v);
+              tmem_ld_wait();
 #pragma unroll
-            for (int j = 0; j < 16; ++j)
-              pk[half * 16 + j] = pack_bf16x2(w * __uint_as_float(v[2 * j]), w * __uint_as_float(v[2 * j + 1]));
+              for (int j = 0; j < 16; ++j)
+                pk[half * 16 + j] = pack_bf16x2(w * __uint_as_float(v[2 * j]), w * __uint_as_float(v[2 * j + 1]));
+            }
+            if (cc == kBN2 / 64 - 1) release_acc();
+            const int col = t.n0 + cc * 64;
+            if (!direct) {
+              store_box(&maps.y, pk, col, t.tile * kBM);
+            } else if (valid && col + 64 <= sh.H) {  // H is a multiple of 128: whole chunks
+#pragma unroll
+              for (int v = 0; v < 8; ++v)
+                *reinterpret_cast<uint4*>(yrow + col + 8 * v) =
+                    make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+            }
           }
-          if (cc == kBN2 / 64 - 1) release_acc();
-          store_box(&maps.y, pk, t.n0 + cc * 64, t.tile * kBM);
+        } else {
+          release_acc();
         }
       }
       if (lane == 0) mbar_arrive(&task_empty[slot]);
@@ -392,7 +525,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       ++use;
       if (++slot == kTaskSlots) { slot = 0; slot_phase ^= 1; }
     }
-    if (leader) bulk_wait_group<0>();
+    if (leader) {
+      bulk_wait_group<0>();
+      add_wait(kWaitEpiLoop, now() - s_ewait[2]);
+      add_wait(kWaitEpiTask, s_ewait[0]);
+      add_wait(kWaitEpiAcc, s_ewait[1]);
+    }
   }
 
   griddep_launch_dependents();

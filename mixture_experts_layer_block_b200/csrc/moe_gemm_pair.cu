@@ -166,12 +166,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int U = __ldcg(&meta->num_units);
     int u_cur = 0;
     uint32_t stage = 0, phase = 0, slot = 0, slot_phase = 0;
+    int next_tau = 0, batch_end = 0;  // a claim takes sh.claim_batch consecutive ids
     while (true) {
       Task t;
       bool ok = true;
       if (rank == 0) {
         int tau = 0;
-        if (lane == 0) tau = aborted(meta, s_abort) ? total : atomicAdd(&meta->task_counter, 1);
+        if (lane == 0) {
+          if (next_tau >= batch_end) {
+            next_tau = atomicAdd(&meta->task_counter, sh.claim_batch);
+            batch_end = next_tau + sh.claim_batch;
+          }
+          tau = aborted(meta, s_abort) ? total : next_tau++;
+        }
         tau = __shfl_sync(0xffffffffu, tau, 0);
         t.id = tau;
         t.kind = kTaskStop;

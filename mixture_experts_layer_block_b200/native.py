@@ -43,7 +43,7 @@ class moe_config(ctypes.Structure):
                 ("top_k", ctypes.c_int32), ("block_m", ctypes.c_int32),
                 ("capacity_factor", ctypes.c_float), ("max_tokens", ctypes.c_int32),
                 ("flags", ctypes.c_uint32), ("device", ctypes.c_int32),
-                ("timeout_ns", ctypes.c_int64)]
+                ("timeout_ns", ctypes.c_int64), ("claim_batch", ctypes.c_int32)]
 
 
 class moe_shared_w(ctypes.Structure):
@@ -149,9 +149,10 @@ class MoELayer:
     fp32, out [T,H] fp32, or bf16 with MOE_FLAG_OUT_BF16)."""
 
     def __init__(self, hidden, inter, num_experts, top_k, block_m, max_tokens, inter_shared=0,
-                 capacity_factor=0.0, flags=0, device=-1, timeout_ns=0):
+                 capacity_factor=0.0, flags=0, device=-1, timeout_ns=0, claim_batch=0):
         self.cfg = moe_config(hidden, inter, inter_shared, num_experts, top_k, block_m,
-                              float(capacity_factor), max_tokens, flags, device, timeout_ns)
+                              float(capacity_factor), max_tokens, flags, device, timeout_ns,
+                              claim_batch)
         h = ctypes.c_void_p()
         check(lib.moe_init(ctypes.byref(self.cfg), ctypes.byref(h)), "moe_init")
         self.h = h

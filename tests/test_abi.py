@@ -40,7 +40,7 @@ def test_library_exports_every_declared_symbol(native):
 
 def _cfg(native, **kw):
     base = dict(hidden=256, inter=128, inter_shared=0, num_experts=8, top_k=2, block_m=16,
-                capacity_factor=0.0, max_tokens=64, flags=0, device=-1, timeout_ns=0)
+                capacity_factor=0.0, max_tokens=64, flags=0, device=-1, timeout_ns=0, claim_batch=0)
     base.update(kw)
     return native.moe_config(**base)
 
@@ -48,7 +48,8 @@ def _cfg(native, **kw):
 @pytest.mark.parametrize("bad", [dict(top_k=9), dict(top_k=0), dict(hidden=100), dict(inter=0),
                                  dict(num_experts=0), dict(num_experts=2048), dict(block_m=0),
                                  dict(max_tokens=0), dict(capacity_factor=-1.0),
-                                 dict(inter_shared=12), dict(top_k=33, num_experts=64)])
+                                 dict(inter_shared=12), dict(top_k=33, num_experts=64),
+                                 dict(claim_batch=-1), dict(claim_batch=65)])
 def test_init_rejects_bad_config_before_cuda(native, bad):
     h = ctypes.c_void_p()
     rc = native.lib.moe_init(ctypes.byref(_cfg(native, **bad)), ctypes.byref(h))
@@ -100,3 +101,15 @@ def test_binding_constants_match_the_header(native):
     assert len(defs) >= 15
     for name, value in defs.items():
         assert getattr(native, name) == int(value), name
+
+
+def test_config_struct_matches_the_header(native):
+    """moe_config's fields, in the header's order, with the C layout (int64 timeout_ns at 40,
+    claim_batch after it, padded to 56 bytes)."""
+    text = open(HEADER).read()
+    body = re.search(r"typedef struct moe_config \{(.*?)\} moe_config;", text, flags=re.S).group(1)
+    names = re.findall(r"^\s*(?:int32_t|uint32_t|int64_t|float)\s+(\w+);", body, flags=re.M)
+    assert names == [f[0] for f in native.moe_config._fields_]
+    assert native.moe_config.timeout_ns.offset == 40
+    assert native.moe_config.claim_batch.offset == 48
+    assert ctypes.sizeof(native.moe_config) == 56

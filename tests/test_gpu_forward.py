@@ -95,18 +95,35 @@ def test_pair_tiles_one_expert(nrows):
 
 def test_tile_shape_selection():
     """Single SMs by default, SM pairs on request (when the device fits 2-CTA clusters), single
-    SMs when both flags are given; batches of at most 16 tokens keep the small-tile shape."""
+    SMs when both flags are given; two-tile task sets by default above 96 slots per expert unless
+    the capacity holds an expert to one tile; the flags that ask for a shape win."""
     w2 = SMALL["skew_small"].replace(E=64, name="skew_small_64")  # 250 slots per expert
     inp2 = {k: (v.cuda() if v is not None else None) for k, v in gen.make_inputs(w2).items()}
     f = _flags()
     layer = _layer(w2)
     check_forward(layer, w2, inp2)
     assert layer.query(6) == 128 and layer.query(1) == layer.query(0)
-    assert layer.query(8) == SHAPE_CODE["tail"]  # 96..384 slots per expert: merged tails
+    assert layer.query(8) == SHAPE_CODE["two"]  # more than 96 slots per expert: two-tile tasks
     wide = w2.replace(E=16, name="skew_small_16")  # 1000 slots per expert
     inp3 = {k: (v.cuda() if v is not None else None) for k, v in gen.make_inputs(wide).items()}
     layer = _layer(wide)
     check_forward(layer, wide, inp3)
+    assert layer.query(8) == SHAPE_CODE["two"]
+    # a capacity of at most one tile per expert, or a light load: the general shape
+    capped = w2.replace(capacity_factor=0.5, name="skew_small_capped")  # 125 slots per expert
+    layer = _layer(capped)
+    check_forward(layer, capped, inp2)
+    assert layer.query(8) == SHAPE_CODE["general"]
+    light = w2.replace(E=256, name="skew_small_256")  # 62.5 slots per expert
+    inp4 = {k: (v.cuda() if v is not None else None) for k, v in gen.make_inputs(light).items()}
+    layer = _layer(light)
+    check_forward(layer, light, inp4)
+    assert layer.query(8) == SHAPE_CODE["general"]
+    layer = _layer(w2, flags=f["tail"])
+    check_forward(layer, w2, inp2)
+    assert layer.query(8) == SHAPE_CODE["tail"]
+    layer = _layer(w2, flags=f["general"])
+    check_forward(layer, w2, inp2)
     assert layer.query(8) == SHAPE_CODE["general"]
     layer = _layer(w2, flags=f["pair"])
     check_forward(layer, w2, inp2)
@@ -219,6 +236,30 @@ def test_single_sm_merged_tails_one_expert(nrows, shape):
     check_forward(layer, w, inp)
     assert layer.query(8) == SHAPE_CODE[shape]
     check_forward(layer, w, inp)  # the same handle again
+
+
+# claim batches: a CTA takes this many consecutive task ids per atomic on the counter
+@pytest.mark.parametrize("batch", [2, 5, 64])
+@pytest.mark.parametrize("name,shape", [("dsv3_small", "general"), ("dsv3_small", "two"), ("skew_small", "tail"),
+                                        ("prefill_small", "pair"), ("small_tokens_shared", None),
+                                        ("small_tokens_ragged", "unfused")])
+def test_forward_claim_batch(name, shape, batch):
+    """Every claim batch gives the oracle's result, and the same bits as one id per claim: the
+    batch changes which CTA runs a task, never what the task computes or the combine order."""
+    from mixture_experts_layer_block_b200 import native
+    w = SMALL[name]
+    inp = {k: (v.cuda() if v is not None else None) for k, v in gen.make_inputs(w).items()}
+    flags = native.MOE_FLAG_UNFUSED_SMALL if shape == "unfused" else _flags().get(shape, 0)
+    outs = []
+    for cb in (0, batch):
+        layer = _layer(w, flags=flags, claim_batch=cb)
+        check_forward(layer, w, inp)
+        o = torch.empty((w.T, w.H), dtype=torch.float32, device="cuda")
+        layer.forward(inp["x"], inp, o)
+        torch.cuda.synchronize()
+        assert layer.status() == (0, 0)
+        outs.append(o)
+    assert torch.equal(outs[0], outs[1])
 
 
 STATIC_CASES = {

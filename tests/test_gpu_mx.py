@@ -164,3 +164,24 @@ def test_forward_mxfp8_is_deterministic():
     assert layer.status() == (0, 0)
     assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
     layer.close()
+
+
+@pytest.mark.parametrize("batch", [3, 64])
+def test_forward_mxfp8_claim_batch(batch):
+    """A claim batch changes which CTA runs a task, not its result: the oracle's result, and the
+    same bits as one id per claim."""
+    native = _native()
+    w = MX_SMALL["dsv3_small"]
+    outs = []
+    for cb in (0, batch):
+        inp = gen.make_inputs(w, device="cuda")
+        layer = native.MoELayer.for_workload(w, flags=native.MOE_FLAG_MXFP8, claim_batch=cb)
+        wq = layer.quantize_experts_mxfp8(inp)
+        check_forward(layer, w, inp, wq=wq)
+        out = torch.empty((w.T, w.H), dtype=torch.float32, device="cuda")
+        layer.forward_mxfp8(inp["x"], inp["W_router"], inp.get("bias"), wq, out)
+        torch.cuda.synchronize()
+        assert layer.status() == (0, 0)
+        outs.append(out)
+        layer.close()
+    assert torch.equal(outs[0], outs[1])

@@ -69,17 +69,21 @@ def test_invalid_arguments_are_rejected():
     assert e.value.code == MOE_ERR_MISALIGNED
 
 
-@pytest.mark.parametrize("name,T", [("dsv3_small", 300), ("small_fused", 12)])
-def test_trace_records_and_wait_accounting(name, T):
+@pytest.mark.parametrize("name,T,mx", [("dsv3_small", 300, False), ("small_fused", 12, False),
+                                       ("dsv3_small_mx", 300, True), ("small_mx", 12, True)])
+def test_trace_records_and_wait_accounting(name, T, mx):
     """MOE_FLAG_TRACE: one record per task (claimed by a CTA of the grid, finished after it was
     claimed), and per-CTA wait totals in which every wait fits inside its role's loop; the
-    traced forward is still correct."""
+    traced forward is still correct (bf16 and MXFP8 experts)."""
     import numpy as np
-    from mixture_experts_layer_block_b200.native import MOE_FLAG_TRACE, MoELayer
+    from mixture_experts_layer_block_b200.native import MOE_FLAG_MXFP8, MOE_FLAG_TRACE, MoELayer
     w = configs.DSV3.replace(name=name, T=T, H=1024, D=256, E=32, D_shared=256)
     inp = {k: (v.cuda() if v is not None else None) for k, v in gen.make_inputs(w).items()}
-    layer = MoELayer.for_workload(w, flags=MOE_FLAG_TRACE)
-    check_forward(layer, w, inp)
+    layer = MoELayer.for_workload(w, flags=MOE_FLAG_TRACE | (MOE_FLAG_MXFP8 if mx else 0))
+    if mx:
+        check_forward(layer, w, inp, wq=layer.quantize_experts_mxfp8(inp))
+    else:
+        check_forward(layer, w, inp)
     rec = layer.trace(1 << 16)
     tasks = layer.query(3)
     assert rec.shape[0] == tasks
