@@ -251,10 +251,14 @@ def front_timeline(w: np.ndarray, names) -> dict:
     last = c["front_last"] == 1
     med = lambda v: float(np.median(v) / 1e3) if v.size else None
     steps = {n[6:]: med(c[n][last]) for n in names if n.startswith("sched_")}
+    comb = c["combine_run"] > 0
     return {"router": med(c["front_router"]), "schedule_compute": med(c["front_schedule"][last]),
             "schedule_steps": steps, "schedule_wait": med(c["front_schedule"][~last]),
             "gather": med(c["front_gather"]), "front_to_end": med(c["front_to_end"]),
-            "max_front_to_end": float(c["front_to_end"].max() / 1e3)}
+            "max_front_to_end": float(c["front_to_end"].max() / 1e3),
+            # per CTA: the column-block counting after its down tasks, and its combines
+            "combine_count": med(c["combine_count"]), "combine_run": med(c["combine_run"][comb]),
+            "combining_ctas": int(comb.sum())}
 
 
 def routing_stats(layer, w, dev):

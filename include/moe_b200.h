@@ -349,7 +349,9 @@ MOE_API int moe_trace_read(moe_handle *h, int64_t *records, int64_t cap, int64_t
  * computed the schedule, 16 from the start of the front to the end of the epilogue loop,
  * and in the CTA that computed the schedule its steps: 17 the arrival count, 18 loading the
  * logits, 19 gating, 20 the count / offset / tile / unit tables, 21 the writes of sorted_ids,
- * the sentinels, expert_ids and the task table, 22 publishing the schedule. (23 per row.) Writes up to `rows` rows (at most one per SM) into the host buffer
+ * the sentinels, expert_ids and the task table, 22 publishing the schedule; 23 the barrier,
+ * fences and column-block counter after each fused down task, 24 the fused combines the CTA ran.
+ * (25 per row.) Writes up to `rows` rows (at most one per SM) into the host buffer
  * `waits` and their number to *n_rows. The SM-pair and MXFP8 kernels leave zeros. */
 MOE_API int moe_trace_waits(moe_handle *h, int64_t *waits, int32_t rows, int32_t *n_rows);
 

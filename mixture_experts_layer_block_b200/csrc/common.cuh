@@ -31,6 +31,7 @@ constexpr int kStagingBytes = 128 * 128;  // one epilogue staging buffer: 128 ro
 constexpr int kNumStaging = 2;            // double-buffered epilogue -> TMA store staging
 constexpr int kAccCols = 256;   // TMEM columns per accumulator buffer (2 buffers)
 constexpr int kGemmThreads = 192;  // warp 0 producer, warp 1 MMA, warps 2-5 epilogue
+constexpr int kMaxTopK = 32;       // largest top_k
 constexpr int kSmallRows = 16;     // A-tile rows of the expert GEMMs' small-tile shape (T <= 16)
 constexpr int kPairBoxRows = 32;   // rows per A load / result store box of the SM-pair shape
 
@@ -118,7 +119,10 @@ enum WaitKind : int {
   kSchedTables = 20,   // counts, offsets, tiles, groups and units (one warp)
   kSchedWrites = 21,   // sorted_ids, sentinels, expert_ids, task table, counter resets
   kSchedPublish = 22,  // memory fence, barrier and the flag
-  kNumWaits = 23,
+  // the fused forward's combine (epilogue leader, summed over this CTA's down tasks)
+  kCombineCount = 23,  // barrier, fences and the column block's counter after each down task
+  kCombineRun = 24,    // the combines this CTA ran (one per column block it completed)
+  kNumWaits = 25,
 };
 
 // Task kinds in the ring.

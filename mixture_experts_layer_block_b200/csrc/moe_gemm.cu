@@ -73,7 +73,9 @@ struct Cfg {
   static constexpr int kNumBars = 2 * kStagesN + 4 + 2 * kTaskSlots + 1;
   static constexpr int kRingOff = kBarOff + ((kNumBars * 8 + 63) & ~63);
   static constexpr int kMiscOff = kRingOff + kTaskSlots * (int)sizeof(Task);
-  static constexpr int kBytes = kMiscOff + 64;
+  // the fused small-batch forward keeps every slot's tile row (row_of_slot) in shared memory
+  static constexpr int kSlotRowsOff = kMiscOff + 64;
+  static constexpr int kBytes = kSlotRowsOff + (kShape == kShapeSmallFused ? kSmallRows * kMaxTopK * 4 : 0);
   static_assert(kStageBytesN % 1024 == 0 && kABytesN % 1024 == 0 && kTailBytesN % 1024 == 0,
                 "1024-byte aligned operand tiles");
   static_assert(kBytes + 1024 <= 227 * 1024, "shared memory budget");
@@ -417,10 +419,10 @@ __device__ bool wait_schedule(const int* flag, int epoch, DeviceMeta* meta, int6
 // This CTA's share of the row gather: the x row of every kept slot s = blockIdx.x + j * gridDim.x
 // into its tile row of xs; each row bumps its tile's gather count (release), which the tile's
 // up tasks wait for before their TMA loads.
-__device__ void front_gather(const FrontArgs& fa, const Workspace& ws, const Shape& sh) {
+__device__ void front_gather(const FrontArgs& fa, const Workspace& ws, const Shape& sh, const int* slot_rows) {
   const int S = sh.T * sh.k, nvec = sh.H / 8;
   for (int s = blockIdx.x; s < S; s += gridDim.x) {
-    const int row = __ldcg(ws.row_of_slot + s);
+    const int row = slot_rows[s];
     if (row < 0) continue;
     const uint4* src = reinterpret_cast<const uint4*>(fa.x + (size_t)(s / sh.k) * sh.H);
     uint4* dst = reinterpret_cast<uint4*>(ws.xs + (size_t)row * sh.H);
@@ -439,8 +441,10 @@ __device__ void front_gather(const FrontArgs& fa, const Workspace& ws, const Sha
 // The combine of columns [n0, n0 + kBN2) for every token, once every down task of that column
 // block is done: out[t] = y[shared row of t] + sum_j y[row of slot t*k + j], in this order, in
 // fp32 (the standalone combine kernel's order, so the result is the same bit for bit). Thread
-// i < 128: token i / 8, 32 columns.
-__device__ void fused_combine(const FrontArgs& fa, const Workspace& ws, const Shape& sh, int n0, int i, int Mr) {
+// i < 128: token i / 8, 32 columns. slot_rows: every slot's tile row (-1: dropped), in shared
+// memory.
+__device__ void fused_combine(const FrontArgs& fa, const Workspace& ws, const Shape& sh, int n0, int i, int Mr,
+                              const int* slot_rows) {
   const int t = i >> 3;
   if (t >= sh.T) return;
   const int c0 = n0 + (i & 7) * 32;
@@ -449,39 +453,29 @@ __device__ void fused_combine(const FrontArgs& fa, const Workspace& ws, const Sh
   for (int v = 0; v < 4; ++v)
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[v][j] = 0.f;
-  // the rows in summation order: the shared expert's, then slots j = 0..k-1 (-1: dropped); every
-  // index is loaded in one round, then the rows' data four rows at a time
-  constexpr int kMaxRows = 33;  // top_k <= 32, plus the shared row
-  int rows[kMaxRows];
+  // the rows in summation order: the shared expert's, then slots j = 0..k-1; their data is
+  // loaded kRound rows at a time (one round trip for top-8 without a shared expert)
+  constexpr int kRound = 8;
   const int nr = (sh.Ds > 0 ? 1 : 0) + sh.k;
+  auto row_of = [&](int j) {
+    const int jj = sh.Ds > 0 ? j - 1 : j;
+    return jj < 0 ? (Mr + t / sh.tile_m) * sh.tile_m + t % sh.tile_m : slot_rows[t * sh.k + jj];
+  };
+  for (int j0 = 0; j0 < nr; j0 += kRound) {
+    uint4 d[kRound][4];
+    int rows[kRound];
 #pragma unroll
-  for (int j = 0; j < kMaxRows; ++j) {
-    if (j < nr) {
-      const int jj = sh.Ds > 0 ? j - 1 : j;
-      rows[j] = jj < 0 ? (Mr + t / sh.tile_m) * sh.tile_m + t % sh.tile_m
-                       : __ldcg(ws.row_of_slot + t * sh.k + jj);
-    } else {
-      rows[j] = -1;
-    }
-  }
-#pragma unroll
-  for (int j0 = 0; j0 < kMaxRows; j0 += 4) {
-    if (j0 >= nr) break;
-    uint4 d[4][4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int row = rows[j0 + q < kMaxRows ? j0 + q : 0];
-      const bool use = j0 + q < nr && row >= 0;
-      const uint16_t* yr = ws.y + (size_t)(use ? row : 0) * sh.H;
+    for (int q = 0; q < kRound; ++q) {
+      rows[q] = j0 + q < nr ? row_of(j0 + q) : -1;
+      const uint16_t* yr = ws.y + (size_t)(rows[q] >= 0 ? rows[q] : 0) * sh.H;
 #pragma unroll
       for (int v = 0; v < 4; ++v)
-        d[q][v] = (use && c0 + 8 * v + 8 <= sh.H) ? __ldcg(reinterpret_cast<const uint4*>(yr + c0 + 8 * v))
-                                                   : make_uint4(0, 0, 0, 0);
+        d[q][v] = (rows[q] >= 0 && c0 + 8 * v + 8 <= sh.H) ? __ldcg(reinterpret_cast<const uint4*>(yr + c0 + 8 * v))
+                                                         : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int row = rows[j0 + q < kMaxRows ? j0 + q : 0];
-      if (j0 + q < nr && row >= 0) {
+    for (int q = 0; q < kRound; ++q) {
+      if (rows[q] >= 0) {
 #pragma unroll
         for (int v = 0; v < 4; ++v) add_bf16x8(acc[v], d[q][v]);
       }
@@ -509,7 +503,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   constexpr int kABytes = C::kABytesN;
   constexpr int kBOff = C::kABytesN + C::kTailBytesN;  // B's offset in a stage
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // aligned by pointer arithmetic on the shared array (not through an integer), so that the
+  // compiler keeps every access through `smem` in the shared address space
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
   uint64_t* full = bars;
   uint64_t* empty = full + kStages;
@@ -524,6 +520,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   volatile int* s_epi_go = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 8);  // [2]
   volatile int* s_front = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 16);  // fused: last / ok
   volatile int* s_comb = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 24);   // fused: combine
+  int* s_slot_rows = reinterpret_cast<int*>(smem + C::kSlotRowsOff);                 // fused: [T*k]
+  int* s_tiles = reinterpret_cast<int*>(smem + C::kMiscOff + 32);  // fused: m-tiles, routed m-tiles
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   DeviceMeta* meta = ws.meta;
@@ -596,7 +594,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncthreads();
     const int64_t t_s = now();
     run_tasks = s_front[1] != 0;
-    if (run_tasks) front_gather(fa, ws, sh);
+    if (run_tasks) {
+      // every slot's tile row, for the gather and the combine
+      for (int i = threadIdx.x; i < sh.T * sh.k; i += blockDim.x) s_slot_rows[i] = __ldcg(ws.row_of_slot + i);
+      if (threadIdx.x == 0) {
+        s_tiles[0] = __ldcg(&meta->num_tiles);
+        s_tiles[1] = __ldcg(&meta->num_routed_tiles);
+      }
+      __syncthreads();
+      front_gather(fa, ws, sh, s_slot_rows);
+    }
     // the ring's generic-proxy writes come before the TMA fills that reuse it
     fence_proxy_async_shared();
     __syncthreads();
@@ -1057,15 +1064,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&acc_empty[next]);
           if constexpr (kFused) {
-            // count this task's column block; the task that completes a block combines it
-            __threadfence();
+            // count this task's column block; the task that completes a block combines it. The
+            // barrier orders every epilogue thread's y stores before the leader's fence (release,
+            // cumulative over the barrier); the last task's leader fences again (acquire) before
+            // the barrier that lets its threads read the other tasks' rows.
+            const int64_t tc0 = now();
             named_bar_sync(1, 128);
-            if (leader)
-              *s_comb = (atomicAdd(&ws.col_done[t.n0 / kBN2], 1) == __ldcg(&meta->num_tiles) - 1) ? 1 : 0;
-            named_bar_sync(1, 128);
-            if (*s_comb) {
+            if (leader) {
               __threadfence();
-              fused_combine(fa, ws, sh, t.n0, (int)threadIdx.x - 64, __ldcg(&meta->num_routed_tiles));
+              const bool last = atomicAdd(&ws.col_done[t.n0 / kBN2], 1) == s_tiles[0] - 1;
+              if (last) __threadfence();
+              *s_comb = last ? 1 : 0;
+            }
+            named_bar_sync(1, 128);
+            const int64_t tc1 = now();
+            wacc[kCombineCount] += tc1 - tc0;
+            if (*s_comb) {
+              fused_combine(fa, ws, sh, t.n0, (int)threadIdx.x - 64, s_tiles[1], s_slot_rows);
+              if (tracing) {
+                named_bar_sync(1, 128);  // the combine of every thread
+                wacc[kCombineRun] += now() - tc1;
+              }
             }
           }
         }

@@ -96,7 +96,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   constexpr int kStages = kPStages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // both CTAs get the same layout: the MMA addresses the two CTAs' operands at equal offsets
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // aligned by pointer arithmetic on the shared array (not through an integer), so that the
+  // compiler keeps every access through `smem` in the shared address space
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kPBarOff);
   uint64_t* full = bars;
   uint64_t* empty = full + kStages;

@@ -21,50 +21,152 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 }
 
 // Top-k with renormalised softmax for NT tokens at once (their dependency chains interleave):
-// v[n][j] holds expert lane + 32 j of token n. Each of the k rounds takes, per token, the
-// largest remaining logit, ties to the lower expert index: every lane's best candidate, the
-// warp's largest key (one redux), then the lowest index among the lanes that hold it (another).
-// Lane r < k returns round r's expert in ids[n] and its weight exp(v_r - v_0) / sum_i
-// exp(v_i - v_0) over the k chosen in w[n].
+// v[n][j] holds expert lane + 32 j of token n. Each lane first sorts its VPL candidates of every
+// token (largest first, ties to the lower expert index; an odd-even merge network). Each of the
+// k rounds then takes, per token, the largest remaining logit, ties to the lower expert index:
+// the warp's largest head key (one redux), then the lowest expert index among the lanes whose
+// head holds it (another); the winning lane drops its head. Lane r < k returns round r's expert
+// in ids[n] and its weight exp(v_r - v_0) / sum_i exp(v_i - v_0) over the k chosen in w[n].
+// Experts >= E and NaN logits are never chosen while another candidate is left.
+template <int VPL>
+__device__ __forceinline__ void lane_sort_desc(uint32_t (&key)[VPL], int (&idx)[VPL], float (&val)[VPL]) {
+  // compare-exchange (a, b): a keeps the larger key, the lower index on equal keys
+  auto cx = [&](int a, int b) {
+    const bool sw = key[a] < key[b] || (key[a] == key[b] && idx[a] > idx[b]);
+    const uint32_t ka = key[a], kb = key[b];
+    const int ia = idx[a], ib = idx[b];
+    const float va = val[a], vb = val[b];
+    key[a] = sw ? kb : ka;
+    key[b] = sw ? ka : kb;
+    idx[a] = sw ? ib : ia;
+    idx[b] = sw ? ia : ib;
+    val[a] = sw ? vb : va;
+    val[b] = sw ? va : vb;
+  };
+  // Batcher's odd-even merge sort, for VPL a power of two
+#pragma unroll
+  for (int p = 1; p < VPL; p <<= 1)
+#pragma unroll
+    for (int q = p; q >= 1; q >>= 1)
+#pragma unroll
+      for (int j = q % p; j + q < VPL; j += 2 * q)
+#pragma unroll
+        for (int i = 0; i < q; ++i)
+          if (i + j + q < VPL && (i + j) / (2 * p) == (i + j + q) / (2 * p)) cx(i + j, i + j + q);
+}
+
+// More than 8 candidates per lane (E > 256): no sort; each round scans the lane's remaining
+// candidates for its best, with the same order.
 template <int VPL, int NT>
-__device__ __forceinline__ void warp_topk_softmax_n(const float (&v)[NT][VPL], int E, int k, int lane,
-                                                    int (&ids)[NT], float (&w)[NT]) {
+__device__ __forceinline__ void warp_topk_scan_n(const float (&v)[NT][VPL], int E, int k, int lane,
+                                                 float (&my_v)[NT], float (&top_v)[NT], int (&ids)[NT]) {
   uint32_t taken[NT];
-  float my_v[NT], top_v[NT];
 #pragma unroll
   for (int n = 0; n < NT; ++n) {
     taken[n] = 0;
 #pragma unroll
     for (int j = 0; j < VPL; ++j)
-      if (lane + 32 * j >= E) taken[n] |= 1u << j;
+      if (lane + 32 * j >= E || v[n][j] != v[n][j]) taken[n] |= 1u << j;
+  }
+  for (int r = 0; r < k; ++r) {
+    float bv[NT];
+    int bi[NT];
+    uint32_t key[NT], best[NT];
+    int win[NT];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      bv[n] = -INFINITY;
+      bi[n] = INT_MAX;
+#pragma unroll
+      for (int j = 0; j < VPL; ++j) {
+        const int e = lane + 32 * j;
+        if (!((taken[n] >> j) & 1u) && (v[n][j] > bv[n] || (v[n][j] == bv[n] && e < bi[n]))) {
+          bv[n] = v[n][j];
+          bi[n] = e;
+        }
+      }
+      key[n] = bi[n] == INT_MAX ? 0u : order_key(bv[n]);
+    }
+#pragma unroll
+    for (int n = 0; n < NT; ++n) best[n] = __reduce_max_sync(0xffffffffu, key[n]);
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+      win[n] = (int)__reduce_min_sync(0xffffffffu, (uint32_t)(key[n] == best[n] ? bi[n] : INT_MAX));
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      if (win[n] != INT_MAX && (win[n] & 31) == lane) taken[n] |= 1u << (win[n] >> 5);
+      const float wv = __shfl_sync(0xffffffffu, bv[n], win[n] & 31);
+      if (lane == r) {
+        my_v[n] = wv;
+        ids[n] = win[n];
+      }
+      if (r == 0) top_v[n] = wv;
+    }
+  }
+}
+
+template <int VPL, int NT>
+__device__ __forceinline__ void warp_topk_softmax_n(const float (&v)[NT][VPL], int E, int k, int lane,
+                                                    int (&ids)[NT], float (&w)[NT]) {
+  static_assert((VPL & (VPL - 1)) == 0, "candidates per lane: a power of two");
+  float my_v[NT], top_v[NT];
+  if constexpr (VPL > 8) {
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      my_v[n] = 0.f;
+      top_v[n] = 0.f;
+      ids[n] = -1;
+    }
+    warp_topk_scan_n<VPL, NT>(v, E, k, lane, my_v, top_v, ids);
+  } else {
+  uint32_t key[NT][VPL];
+  int idx[NT][VPL];
+  float val[NT][VPL];
+#pragma unroll
+  for (int n = 0; n < NT; ++n) {
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) {
+      const int e = lane + 32 * j;
+      const bool ok = e < E && !(v[n][j] != v[n][j]);
+      key[n][j] = ok ? order_key(v[n][j]) : 0u;
+      idx[n][j] = ok ? e : INT_MAX;
+      val[n][j] = v[n][j];
+    }
+    lane_sort_desc<VPL>(key[n], idx[n], val[n]);
     my_v[n] = 0.f;
     top_v[n] = 0.f;
     ids[n] = -1;
   }
   for (int r = 0; r < k; ++r) {
+    uint32_t best[NT];
+    int win[NT];
+    // each step runs for all NT tokens before the next: the warp-wide reductions are not moved
+    // across one another, so token-major code would run the NT chains one after the other
+#pragma unroll
+    for (int n = 0; n < NT; ++n) best[n] = __reduce_max_sync(0xffffffffu, key[n][0]);
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+      win[n] = (int)__reduce_min_sync(0xffffffffu, (uint32_t)(key[n][0] == best[n] ? idx[n][0] : INT_MAX));
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
-      float bv = -INFINITY;
-      int bi = INT_MAX;
-#pragma unroll
-      for (int j = 0; j < VPL; ++j) {
-        const int e = lane + 32 * j;
-        if (!((taken[n] >> j) & 1u) && (v[n][j] > bv || (v[n][j] == bv && e < bi))) {
-          bv = v[n][j];
-          bi = e;
-        }
-      }
-      const uint32_t key = bi == INT_MAX ? 0u : order_key(bv);
-      const uint32_t best = __reduce_max_sync(0xffffffffu, key);
-      const int win = (int)__reduce_min_sync(0xffffffffu, (uint32_t)(key == best ? bi : INT_MAX));
-      if (win != INT_MAX && (win & 31) == lane) taken[n] |= 1u << (win >> 5);
-      const float wv = __shfl_sync(0xffffffffu, bv, win & 31);  // the winner's value
+      const bool mine = win[n] != INT_MAX && idx[n][0] == win[n];
+      const float wv = __shfl_sync(0xffffffffu, val[n][0], win[n] & 31);  // the winner's value
       if (lane == r) {
         my_v[n] = wv;
-        ids[n] = win;
+        ids[n] = win[n];
       }
       if (r == 0) top_v[n] = wv;
+      // the winning lane drops its head
+#pragma unroll
+      for (int j = 0; j + 1 < VPL; ++j) {
+        key[n][j] = mine ? key[n][j + 1] : key[n][j];
+        idx[n][j] = mine ? idx[n][j + 1] : idx[n][j];
+        val[n][j] = mine ? val[n][j + 1] : val[n][j];
+      }
+      key[n][VPL - 1] = mine ? 0u : key[n][VPL - 1];
+      idx[n][VPL - 1] = mine ? INT_MAX : idx[n][VPL - 1];
     }
+  }
   }
 #pragma unroll
   for (int n = 0; n < NT; ++n) {

@@ -52,7 +52,9 @@ __global__ void __launch_bounds__(kRThreads, 1)
                   const float* __restrict__ bias, float* __restrict__ logits, int T, int E, int H,
                   int BN, int kb_per_split, DeviceMeta* meta, int64_t timeout_ns) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // aligned by pointer arithmetic on the shared array (not through an integer), so that the
+  // compiler keeps every access through `smem` in the shared address space
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int b_bytes = BN * kBK * 2;
   const int stage_bytes = kRABytes + ((b_bytes + 1023) & ~1023);
   const int nst = router_stages(BN);

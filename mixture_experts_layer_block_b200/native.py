@@ -330,10 +330,10 @@ class MoELayer:
     WAITS = ("prod_empty", "prod_dep", "prod_ring", "prod_claim", "mma_full", "mma_acc", "mma_task",
              "epi_task", "epi_acc", "prod_loop", "mma_loop", "epi_loop", "front_router", "front_schedule",
              "front_gather", "front_last", "front_to_end", "sched_arrive", "sched_logits", "sched_gating",
-             "sched_tables", "sched_writes", "sched_publish")
+             "sched_tables", "sched_writes", "sched_publish", "combine_count", "combine_run")
 
     def trace_waits(self):
-        """moe_trace_waits: [CTAs, 23] int64 ns (columns named by WAITS)."""
+        """moe_trace_waits: [CTAs, 25] int64 ns (columns named by WAITS)."""
         import numpy as np
         buf = np.zeros((1024, len(self.WAITS)), dtype=np.int64)
         n = ctypes.c_int32(0)

@@ -96,7 +96,7 @@ def test_wait_fractions_and_front_timeline():
     names = ("prod_empty", "prod_dep", "prod_ring", "prod_claim", "mma_full", "mma_acc", "mma_task",
              "epi_task", "epi_acc", "prod_loop", "mma_loop", "epi_loop", "front_router", "front_schedule",
              "front_gather", "front_last", "front_to_end", "sched_arrive", "sched_logits", "sched_gating",
-             "sched_tables", "sched_writes", "sched_publish")
+             "sched_tables", "sched_writes", "sched_publish", "combine_count", "combine_run")
     w = np.zeros((4, len(names)), dtype=np.int64)
     col = {n: i for i, n in enumerate(names)}
     w[:, col["mma_loop"]] = 1000
@@ -109,6 +109,8 @@ def test_wait_fractions_and_front_timeline():
     w[:, col["front_last"]] = [0, 0, 0, 1]
     w[:, col["front_to_end"]] = [80000, 81000, 82000, 90000]
     w[3, col["sched_gating"]] = 4000
+    w[:, col["combine_count"]] = [1000, 2000, 3000, 4000]
+    w[:, col["combine_run"]] = [0, 5000, 7000, 0]
     f = bench.wait_fractions(w, names)
     assert f["mma"]["operands"] == pytest.approx(2000 / 4000)
     assert f["producer"]["free_stage"] == pytest.approx(0.25)
@@ -116,3 +118,5 @@ def test_wait_fractions_and_front_timeline():
     assert fr["schedule_compute"] == pytest.approx(9.0) and fr["schedule_wait"] == pytest.approx(12.0)
     assert fr["router"] == pytest.approx(4.5) and fr["max_front_to_end"] == pytest.approx(90.0)
     assert fr["schedule_steps"]["gating"] == pytest.approx(4.0)
+    assert fr["combine_count"] == pytest.approx(2.5) and fr["combine_run"] == pytest.approx(6.0)
+    assert fr["combining_ctas"] == 2
