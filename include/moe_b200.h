@@ -328,7 +328,8 @@ MOE_API int moe_stage_times(moe_handle *h, float *ms, int32_t n);
  * 8 expert-GEMM shape of the last forward (0 general, 1 small-tile, 2 tail, 3 SM pairs,
  * 4 MXFP8, 5 two-tile), 9 rows of the per-row buffers of moe_debug_expert_rows, 10 their h row stride
  * (elements, max(D, D_shared)), 11 kernels the last forward launched (1 for a fused small
- * batch, else 6), 12 whether batches of at most 16 tokens run fused on this handle (1) or not. */
+ * batch, else 6), 12 whether batches of at most 16 tokens run fused on this handle (1) or not
+ * (for moe_forward_mxfp8 on a handle made with MOE_FLAG_MXFP8, else for moe_forward). */
 MOE_API int moe_query(const moe_handle *h, int32_t which, int64_t *value);
 
 /* Per-task trace of the last forward (needs MOE_FLAG_TRACE; synchronises). Fills up to

@@ -75,6 +75,7 @@ struct moe_handle {
   int last_shape = 0;  // expert-GEMM shape of the last forward: 0 general, 1 small, 2 tail, 3 pair
   int last_kernels = 0;  // kernels launched by the last forward
   bool fused_ok = false;  // batches of <= 16 tokens may run as one fused launch on this device
+  bool mx_fused_ok = false;  // the same for moe_forward_mxfp8
   int32_t epoch = 0;      // fused forwards launched (the schedule flag's value of the last one)
   int parts_rows = 0;  // rows of the K-split partial logits buffer
   std::vector<cudaEvent_t> ev;  // kTimingRing x (kNumStages + 1) events around the kernels
@@ -420,6 +421,8 @@ int moe_init(const moe_config* cfg, moe_handle** out) {
   if (cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, h->device) != cudaSuccess) return fail(MOE_ERR_CUDA);
   h->fused_ok = coop != 0 && E <= kFusedMaxExperts && small_fused_blocks_per_sm() >= 1 &&
                 !(c.flags & MOE_FLAG_UNFUSED_SMALL) && !(c.flags & MOE_FLAG_STATIC_QUOTA);
+  h->mx_fused_ok = coop != 0 && E <= kFusedMaxExperts && (c.flags & MOE_FLAG_MXFP8) &&
+                   mx_small_fused_blocks_per_sm() >= 1 && !(c.flags & MOE_FLAG_UNFUSED_SMALL);
   h->max_pairs = std::min(h->max_pairs, h->num_sms / 2);
   h->last_workers = h->num_sms;
   if (h->timing) {
@@ -739,6 +742,31 @@ int moe_forward_mxfp8(moe_handle* h, const void* x, int32_t T, const void* w_rou
   // tracing: the per-CTA wait accounting of this forward starts from zero
   if (w.waits && cudaMemsetAsync(w.waits, 0, (size_t)h->num_sms * kNumWaits * 8, st) != cudaSuccess)
     return MOE_ERR_CUDA;
+  if (T <= kSmallRows && h->mx_fused_ok) {
+    // one launch, as for bf16 experts: router slices, schedule, quantising gather, GEMMs, combine
+    for (int i = 0; i <= 4; ++i)
+      if ((rc = mark(i))) return rc;
+    FrontArgs fa{};
+    fa.x = static_cast<const uint16_t*>(x);
+    fa.w_router = static_cast<const uint16_t*>(w_router);
+    fa.bias = router_bias;
+    fa.out = out;
+    fa.out_bf16 = (c.flags & MOE_FLAG_OUT_BF16) ? 1 : 0;
+    fa.epoch = h->epoch + 1;
+    const cudaError_t le = launch_moe_mx_small_fused(maps, w, mx, sh, fa, h->num_sms, st);
+    if (le == cudaSuccess) {
+      h->epoch = fa.epoch;
+      h->last_kernels = 1;
+      if ((rc = mark(5))) return rc;
+      return mark(6);
+    }
+    // the device refused the cooperative launch (nothing ran): the separate kernels from now on
+    cudaGetLastError();
+    h->mx_fused_ok = false;
+    if (ev) --h->timed;
+    h->dep_extra_next = sh.dep_extra;
+    return moe_forward_mxfp8(h, x, T, w_router, router_bias, wq, top_k, out, stream);
+  }
   if ((rc = mark(0))) return rc;
   int splits = router_splits(T, E, H, bn, h->num_sms);
   while (splits > 1 && (int64_t)splits * T > h->parts_rows) splits /= 2;
@@ -1003,7 +1031,7 @@ int moe_query(const moe_handle* h, int32_t which, int64_t* value) {
     case 9: *value = h->tile_rows; return MOE_OK;
     case 10: *value = h->ws.ldh; return MOE_OK;
     case 11: *value = h->last_kernels; return MOE_OK;
-    case 12: *value = h->fused_ok ? 1 : 0; return MOE_OK;
+    case 12: *value = ((h->cfg.flags & MOE_FLAG_MXFP8) ? h->mx_fused_ok : h->fused_ok) ? 1 : 0; return MOE_OK;
     default: return MOE_ERR_INVALID_ARG;
   }
 }

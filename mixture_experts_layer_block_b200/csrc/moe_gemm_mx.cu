@@ -22,6 +22,7 @@
 //
 // Warp roles and bounded waits as in the bf16 kernel: warp 0 producer, warp 1 MMA issuer (one
 // lane), warps 2-5 epilogue.
+#include "front.cuh"
 #include "launch.h"
 #include "mx.cuh"
 
@@ -42,7 +43,9 @@ struct MxCfg {
   static constexpr int kNumBars = 2 * kStages + 2 + 2 * kTaskSlots + 1;
   static constexpr int kRingOff = kBarOff + ((kNumBars * 8 + 63) & ~63);
   static constexpr int kMiscOff = kRingOff + kTaskSlots * (int)sizeof(Task);
-  static constexpr int kBytes = kMiscOff + 64;
+  // the fused small-batch forward keeps every slot's tile row (row_of_slot) in shared memory
+  static constexpr int kSlotRowsOff = kMiscOff + 64;
+  static constexpr int kBytes = kSlotRowsOff + kSmallRows * kMaxTopK * 4;
   static constexpr uint32_t kSfCol0 = kAccCols;        // first TMEM column of the scale slots
   static constexpr uint32_t kSfColsPerStage = 16;
   static_assert(kStageBytes % 1024 == 0 && kSfOff % 1024 == 0, "1024-byte aligned operand tiles");
@@ -55,8 +58,12 @@ __device__ __forceinline__ int n1_of(int expert, const Shape& sh) {
   return ceil_div(expert == sh.E ? sh.Ds : sh.D, kBN1);
 }
 
+// kFused: the whole forward of at most 16 tokens in one launch (front.cuh): router slices, the
+// schedule from the last CTA to arrive, the MXFP8 row gather, then the tasks; the down task that
+// completes a 256-column block combines it.
+template <bool kFused>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    moe_gemm_mx_kernel(const __grid_constant__ MxMaps maps, Workspace ws, MxBuffers mx, Shape sh) {
+    moe_gemm_mx_kernel(const __grid_constant__ MxMaps maps, Workspace ws, MxBuffers mx, Shape sh, FrontArgs fa) {
   using C = MxCfg;
   constexpr int kStages = C::kStages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -75,6 +82,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
   volatile int* s_epi_go = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 8);  // [2]
+  // (misc + 16 .. + 39: the epilogue leader's wait sums)
+  volatile int* s_front = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 40);  // fused: last / ok
+  volatile int* s_comb = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 48);   // fused: combine
+  int* s_tiles = reinterpret_cast<int*>(smem + C::kMiscOff + 52);  // fused: m-tiles, routed m-tiles
+  int* s_slot_rows = reinterpret_cast<int*>(smem + C::kSlotRowsOff);                 // fused: [T*k]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   DeviceMeta* meta = ws.meta;
@@ -123,7 +135,63 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 (unsigned long long)v);
   };
 
-  if (warp == 0) {
+  bool run_tasks = true;
+  if constexpr (kFused) {
+    // the front, by all 192 threads, as in the bf16 kernel; the operand ring is free until the
+    // first TMA fill
+    const int64_t t_front = now();
+    int* fsm = reinterpret_cast<int*>(smem);
+    front_router(fa, ws, sh, reinterpret_cast<float*>(fsm));
+    const int64_t t_r = now();
+    if (threadIdx.x == 0) {
+      __threadfence();
+      s_front[0] = (atomicAdd(&ws.front->front_done, 1) == (int)gridDim.x - 1) ? 1 : 0;
+    }
+    __syncthreads();
+    int64_t ts[4] = {0, 0, 0, 0};
+    const int64_t t_arrived = now();
+    if (s_front[0]) {
+      __threadfence();
+      front_schedule(fa, ws, sh, fsm, ts);
+      if (threadIdx.x == 0) s_front[1] = 1;
+    } else if (threadIdx.x == 0) {
+      s_front[1] = wait_schedule(&ws.front->sched_flag, fa.epoch, meta, limit) ? 1 : 0;
+      __threadfence();
+    }
+    __syncthreads();
+    const int64_t t_s = now();
+    run_tasks = s_front[1] != 0;
+    if (run_tasks) {
+      for (int i = threadIdx.x; i < sh.T * sh.k; i += blockDim.x) s_slot_rows[i] = __ldcg(ws.row_of_slot + i);
+      if (threadIdx.x == 0) {
+        s_tiles[0] = __ldcg(&meta->num_tiles);
+        s_tiles[1] = __ldcg(&meta->num_routed_tiles);
+      }
+      __syncthreads();
+      front_gather_mx(fa, ws, mx, sh, s_slot_rows, s_tiles[1]);
+    }
+    // the ring's generic-proxy writes come before the TMA fills that reuse it
+    fence_proxy_async_shared();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      add_wait(kFrontRouter, t_r - t_front);
+      add_wait(kFrontSchedule, t_s - t_r);
+      add_wait(kFrontGather, now() - t_s);
+      add_wait(kFrontLast, tracing ? s_front[0] : 0);
+      if (tracing && s_front[0]) {
+        add_wait(kSchedArrive, t_arrived - t_r);
+        add_wait(kSchedLogits, ts[0] - t_arrived);
+        add_wait(kSchedGating, ts[1] - ts[0]);
+        add_wait(kSchedTables, ts[2] - ts[1]);
+        add_wait(kSchedWrites, ts[3] - ts[2]);
+        add_wait(kSchedPublish, t_s - ts[3]);
+      }
+    }
+  }
+
+  if (!run_tasks) {
+    // the schedule never came (bounded wait ran out): nothing was issued, go to the teardown
+  } else if (warp == 0) {
     // ===================================== producer =====================================
     const int total = __ldcg(&meta->total_tasks);
     const int Mg = __ldcg(&meta->num_groups), Mgr = __ldcg(&meta->num_routed_groups);
@@ -216,6 +284,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       const bool shared = (t.expert == sh.E);
       const bool up = (t.kind == kTaskUp);
+      if (kFused && up) {
+        // the tile's quantised x rows (or, for the shared tile, every token's) are gathered
+        if (lane == 0) {
+          const int64_t t0 = now();
+          ok = wait_count(&ws.gather_done[t.tile], t.nrows, meta, s_abort, limit);
+          if (ok) fence_proxy_async_global();
+          w_dep += now() - t0;
+        }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
+      }
       if (!up) {
         if (lane == 0) {
           const int64_t t0 = now();
@@ -520,6 +599,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         } else {
           release_acc();
         }
+        if constexpr (kFused) {
+          // count this task's column block; the task that completes a block combines it (the
+          // barrier orders every epilogue thread's y stores -- and the leader's TMA stores, once
+          // complete -- before the leader's acquire-release add)
+          const int64_t tc0 = now();
+          if (leader) bulk_wait_group<0>();
+          named_bar_sync(1, 128);
+          if (leader) *s_comb = atom_add_acq_rel_gpu(&ws.col_done[t.n0 / kBN2], 1) == s_tiles[0] - 1 ? 1 : 0;
+          named_bar_sync(1, 128);
+          const int64_t tc1 = now();
+          if (leader) add_wait(kCombineCount, tc1 - tc0);
+          if (*s_comb) {
+            fused_combine(fa, ws, sh, t.n0, (int)threadIdx.x - 64, s_tiles[1], s_slot_rows);
+            if (tracing) {
+              named_bar_sync(1, 128);
+              if (leader) add_wait(kCombineRun, now() - tc1);
+            }
+          }
+        }
       }
       if (lane == 0) mbar_arrive(&task_empty[slot]);
       if (ws.trace_cap > 0 && leader && t.id < ws.trace_cap)
@@ -555,14 +653,45 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 size_t gemm_mx_smem_bytes() { return (size_t)MxCfg::kBytes + 1024; }
 
 cudaError_t configure_gemm_mx_kernel() {
-  return cudaFuncSetAttribute(moe_gemm_mx_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(moe_gemm_mx_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)gemm_mx_smem_bytes());
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(moe_gemm_mx_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               (int)gemm_mx_smem_bytes());
 }
 
 cudaError_t launch_moe_gemm_mx(const MxMaps& maps, const Workspace& ws, const MxBuffers& mx, const Shape& sh,
                                int grid, cudaStream_t stream) {
-  return launch_k(moe_gemm_mx_kernel, dim3(grid), dim3(kGemmThreads), gemm_mx_smem_bytes(), stream, maps, ws, mx,
-                  sh);
+  return launch_k(moe_gemm_mx_kernel<false>, dim3(grid), dim3(kGemmThreads), gemm_mx_smem_bytes(), stream, maps, ws,
+                  mx, sh, FrontArgs{});
+}
+
+cudaError_t launch_moe_mx_small_fused(const MxMaps& maps, const Workspace& ws, const MxBuffers& mx, const Shape& sh,
+                                      const FrontArgs& fa, int grid, cudaStream_t stream) {
+  // every CTA waits for the schedule that one of them publishes: all must be resident at once
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = gemm_mx_smem_bytes();
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, moe_gemm_mx_kernel<true>, maps, ws, mx, sh, fa);
+}
+
+int mx_small_fused_blocks_per_sm() {
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, moe_gemm_mx_kernel<true>, kGemmThreads,
+                                                    gemm_mx_smem_bytes()) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
 }
 
 }  // namespace moe

@@ -39,6 +39,27 @@ __host__ __device__ inline size_t mx_atom_offset(int64_t rb, int64_t kq, int64_t
   return ((size_t)rb * (size_t)(K >> 7) + (size_t)kq) * kSfAtomBytes;
 }
 
+// 32 bf16 values at p (64 bytes, 16-byte aligned) widened to fp32.
+__device__ __forceinline__ void load_bf16x32(const uint16_t* p, float (&v)[32]) {
+  const uint4* p4 = reinterpret_cast<const uint4*>(p);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint4 w = __ldcg(p4 + i);
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      v[8 * i + 2 * j] = __uint_as_float(ws[j] << 16);
+      v[8 * i + 2 * j + 1] = __uint_as_float(ws[j] & 0xffff0000u);
+    }
+  }
+}
+
+__device__ __forceinline__ void store_codes32(uint8_t* p, const uint32_t (&q)[8]) {
+  uint4* p4 = reinterpret_cast<uint4*>(p);
+  p4[0] = make_uint4(q[0], q[1], q[2], q[3]);
+  p4[1] = make_uint4(q[4], q[5], q[6], q[7]);
+}
+
 // Tensor maps of the MXFP8 expert GEMMs (E4M3 operands as 8-bit elements, 128-byte swizzle).
 struct alignas(64) MxMaps {
   CUtensorMap x_tile;  // xq [T][H], box {128, 128} (shared-expert tiles read tokens in order)
@@ -157,5 +178,12 @@ size_t gemm_mx_smem_bytes();
 cudaError_t configure_gemm_mx_kernel();
 cudaError_t launch_moe_gemm_mx(const MxMaps& maps, const Workspace& ws, const MxBuffers& mx, const Shape& sh,
                                int grid, cudaStream_t stream);
+
+// The whole MXFP8 forward of at most 16 tokens (and at most 256 experts) as one cooperative
+// launch of `grid` CTAs, as launch_moe_small_fused does for bf16 experts; the front's row gather
+// quantises the x rows.
+cudaError_t launch_moe_mx_small_fused(const MxMaps& maps, const Workspace& ws, const MxBuffers& mx, const Shape& sh,
+                                      const FrontArgs& fa, int grid, cudaStream_t stream);
+int mx_small_fused_blocks_per_sm();
 
 }  // namespace moe

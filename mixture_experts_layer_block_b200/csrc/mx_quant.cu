@@ -14,27 +14,6 @@ namespace {
 
 constexpr int kMxQuantThreads = 256;
 
-// 32 bf16 values at p (64 bytes, 16-byte aligned) widened to fp32.
-__device__ __forceinline__ void load_bf16x32(const uint16_t* p, float (&v)[32]) {
-  const uint4* p4 = reinterpret_cast<const uint4*>(p);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint4 w = __ldcg(p4 + i);
-    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      v[8 * i + 2 * j] = __uint_as_float(ws[j] << 16);
-      v[8 * i + 2 * j + 1] = __uint_as_float(ws[j] & 0xffff0000u);
-    }
-  }
-}
-
-__device__ __forceinline__ void store_codes32(uint8_t* p, const uint32_t (&q)[8]) {
-  uint4* p4 = reinterpret_cast<uint4*>(p);
-  p4[0] = make_uint4(q[0], q[1], q[2], q[3]);
-  p4[1] = make_uint4(q[4], q[5], q[6], q[7]);
-}
-
 __global__ void __launch_bounds__(kMxQuantThreads)
     mx_quantize_kernel(const uint16_t* __restrict__ src, int64_t R, int K, uint8_t* __restrict__ q,
                        uint8_t* __restrict__ sf) {

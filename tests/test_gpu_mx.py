@@ -185,3 +185,41 @@ def test_forward_mxfp8_claim_batch(batch):
         outs.append(out)
         layer.close()
     assert torch.equal(outs[0], outs[1])
+
+
+MX_FUSED = {
+    "one_token": MX_SMALL["one_token"],
+    "decode": MX_SMALL["decode"],                            # 256 experts top-8, router bias
+    "small_tokens_shared": configs.DSV3.replace(name="small_tokens_shared", T=12, H=512, D=256, E=16, top_k=4,
+                                                D_shared=256),  # the shared tile reads token-order xq
+    "capacity_drops": configs.MoEWorkload("capacity_drops", T=9, H=384, D=256, E=6, top_k=2, block_m=16,
+                                          sigma_w=0.05, capacity_factor=1.0),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MX_FUSED))
+def test_forward_mxfp8_small_batch_fused_and_unfused(name):
+    """At most 16 tokens, MXFP8 experts: one fused launch by default (router slices, schedule,
+    quantising gather, GEMMs, combine by the last down task of each column block) and the six
+    kernels with MOE_FLAG_UNFUSED_SMALL; both match the oracle, and repeated fused forwards agree
+    bit for bit."""
+    native = _native()
+    w = MX_FUSED[name]
+    layer, inp, wq = _setup(w)
+    assert layer.query(12) == 1
+    res = check_forward(layer, w, inp, wq=wq)
+    assert layer.query(11) == 1 and layer.query(8) == 4
+    unfused, _, wq2 = _setup(w, flags=native.MOE_FLAG_UNFUSED_SMALL)
+    check_forward(unfused, w, inp, wq=wq2)
+    assert unfused.query(11) == 6 and unfused.query(12) == 0
+    outs = []
+    for _ in range(3):
+        out = torch.empty((w.T, w.H), dtype=torch.float32, device="cuda")
+        layer.forward_mxfp8(inp["x"], inp["W_router"], inp.get("bias"), wq, out)
+        outs.append(out)
+    torch.cuda.synchronize()
+    assert layer.status() == (0, 0)
+    assert all(torch.equal(o, outs[0]) for o in outs[1:])
+    print(name, res)
+    layer.close()
+    unfused.close()
