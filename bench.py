@@ -48,16 +48,20 @@ L2_BYTES = 126 * 1024 * 1024
 # the ncu captures summarised under profiles/, with the hash of the kernel sources it was taken
 # on. A different hash (the kernel changed since) reports null.
 KERNEL_SOURCES = ["mixture_experts_layer_block_b200/csrc/moe_gemm.cu",
+                  "mixture_experts_layer_block_b200/csrc/front.cuh",
+                  "mixture_experts_layer_block_b200/csrc/route.cuh",
+                  "mixture_experts_layer_block_b200/csrc/mx.cuh",
                   "mixture_experts_layer_block_b200/csrc/common.cuh",
                   "mixture_experts_layer_block_b200/csrc/ptx.cuh",
                   "mixture_experts_layer_block_b200/csrc/launch.h"]
 MEASURED_TRAFFIC = {
-    "flashmoe_prefill": ("8e58c2e2d8dae369", 1.677245e9 + 0.061002e9, "one full-size launch"),
-    "decode": ("8e58c2e2d8dae369", 0.337762e9 + 0.004001e9, "one full-size launch"),
+    "flashmoe_prefill": ("09643c157456f277", 1.679893e9 + 0.059025e9, "one full-size launch"),
+    # at most 16 tokens the forward is one launch: its traffic covers the router, gather and combine
+    "decode": ("09643c157456f277", 0.338446e9 + 0.003994e9, "one full-size launch of the fused forward"),
     # full DSV3 holds 22.6 GB of weights, too large for a multi-pass capture: the T=512, E=32
     # case of the same layer (the same per-expert load, 1/8 of the experts and tokens) scaled
     # by the 8x more units of a full launch
-    "dsv3": ("8e58c2e2d8dae369", 8 * (3.063093e9 + 0.115249e9), "T=512, E=32 capture x 8"),
+    "dsv3": ("09643c157456f277", 8 * (3.033681e9 + 0.113203e9), "T=512, E=32 capture x 8"),
 }
 
 
