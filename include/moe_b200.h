@@ -96,7 +96,8 @@ extern "C" {
  * schedule, every CTA gathers its share of the x rows, then all claim the expert-GEMM tasks, and
  * the CTA that finishes the last down task of a 256-column block combines that block for every
  * token (moe_query 11 reports 1 kernel). MOE_FLAG_UNFUSED_SMALL runs such batches as the six
- * separate kernels instead. The fused router (fp32 on the CUDA cores) sums each logit in
+ * separate kernels instead (for moe_forward and moe_forward_mxfp8). The fused router (fp32 on
+ * the CUDA cores) sums each logit in
  * another order than the separate router kernel (fp32 on the tensor cores): logits and gating
  * weights differ in the last bits, and an exact near-tie may go the other way; both are
  * deterministic. */
@@ -237,9 +238,11 @@ MOE_API int moe_quantize_mxfp8(moe_handle *h, const void *src, int64_t rows, int
  * router-weighted rows are combined as in moe_forward (fp32 sums; `out` fp32 [T][H], or bf16
  * with MOE_FLAG_OUT_BF16). x, w_router, router_bias, top_k, out and stream as in moe_forward.
  * The expert GEMMs run on single SMs with 128-row tiles and the atomic task counter
- * (MOE_FLAG_PAIR_TILES, MOE_FLAG_TAIL_TILES and MOE_FLAG_STATIC_QUOTA do not apply; moe_query
- * 8 reports 4). Needs MOE_FLAG_MXFP8 at moe_init (else MOE_ERR_NOT_READY). Asynchronous, no
- * host synchronisation, no allocation. */
+ * (MOE_FLAG_PAIR_TILES, MOE_FLAG_TAIL_TILES, MOE_FLAG_TWO_TILES and MOE_FLAG_STATIC_QUOTA do not
+ * apply; moe_query 8 reports 4). A batch of at most 16 tokens runs as one fused launch as in
+ * moe_forward (MOE_FLAG_UNFUSED_SMALL: the separate kernels), its row gather quantising the x
+ * rows. Needs MOE_FLAG_MXFP8 at moe_init (else MOE_ERR_NOT_READY). Asynchronous, no host
+ * synchronisation, no allocation. */
 MOE_API int moe_forward_mxfp8(moe_handle *h, const void *x, int32_t T, const void *w_router,
                               const float *router_bias, const moe_mxfp8_experts *w, int32_t top_k,
                               void *out, void *stream);

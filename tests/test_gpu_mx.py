@@ -194,6 +194,9 @@ MX_FUSED = {
                                                 D_shared=256),  # the shared tile reads token-order xq
     "capacity_drops": configs.MoEWorkload("capacity_drops", T=9, H=384, D=256, E=6, top_k=2, block_m=16,
                                           sigma_w=0.05, capacity_factor=1.0),
+    # the router bias moves the hit experts from seed to seed
+    "decode_seed1": MX_SMALL["decode"].replace(name="decode_seed1", seed=1),
+    "decode_seed2": MX_SMALL["decode"].replace(name="decode_seed2", seed=2),
 }
 
 
