@@ -30,9 +30,12 @@ namespace moe {
 
 namespace {
 
+// kSmall (batches of at most 16 tokens: every tile holds at most 16 rows): the A slot holds one
+// 32-row box, so the same shared memory holds a fifth stage (more weight bytes in flight per SM).
+template <bool kSmall>
 struct MxCfg {
-  static constexpr int kStages = 4;
-  static constexpr int kABytes = kBM * kMxBK;          // 16 KB
+  static constexpr int kStages = kSmall ? 5 : 4;
+  static constexpr int kABytes = (kSmall ? kPairBoxRows : kBM) * kMxBK;  // 4 KB or 16 KB
   static constexpr int kBBytes = kUmmaN * kMxBK;       // 32 KB
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kSfStageBytes = 2048;           // SFA atom at 0, SFB atoms at 512 and 1024
@@ -61,10 +64,11 @@ __device__ __forceinline__ int n1_of(int expert, const Shape& sh) {
 // kFused: the whole forward of at most 16 tokens in one launch (front.cuh): router slices, the
 // schedule from the last CTA to arrive, the MXFP8 row gather, then the tasks; the down task that
 // completes a 256-column block combines it.
-template <bool kFused>
+template <bool kFused, bool kSmall>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     moe_gemm_mx_kernel(const __grid_constant__ MxMaps maps, Workspace ws, MxBuffers mx, Shape sh, FrontArgs fa) {
-  using C = MxCfg;
+  static_assert(!kFused || kSmall, "the fused forward is for batches of at most 16 tokens");
+  using C = MxCfg<kSmall>;
   constexpr int kStages = C::kStages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // aligned by pointer arithmetic on the shared array (not through an integer), so that the
@@ -314,7 +318,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // A: one 128-row box, or (tiles of at most 96 rows) only the 32-row boxes that hold the
       // tile's rows; the rest of the A slot keeps stale rows, whose results land in accumulator
       // rows that are never stored
-      const int nbox = (t.nrows <= 3 * kPairBoxRows) ? ceil_div(t.nrows, kPairBoxRows) : 0;
+      // (small: every tile has at most 16 rows, one 32-row box in the 4 KB A slot; the MMA's other
+      // 96 rows read the start of B, and their results are never stored either)
+      const int nbox = kSmall ? 1 : ((t.nrows <= 3 * kPairBoxRows) ? ceil_div(t.nrows, kPairBoxRows) : 0);
       const uint32_t a_bytes = nbox ? (uint32_t)(nbox * kPairBoxRows * kMxBK) : (uint32_t)C::kABytes;
       // scale atoms: A's row block (128-aligned rows), B's row blocks
       const uint8_t* sfa = up ? (shared ? mx.sf_xq + mx_atom_offset(t.row0 >> 7, 0, H)
@@ -650,20 +656,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
 }  // namespace
 
-size_t gemm_mx_smem_bytes() { return (size_t)MxCfg::kBytes + 1024; }
+size_t gemm_mx_smem_bytes(bool small) {
+  return (size_t)(small ? MxCfg<true>::kBytes : MxCfg<false>::kBytes) + 1024;
+}
 
 cudaError_t configure_gemm_mx_kernel() {
-  cudaError_t e = cudaFuncSetAttribute(moe_gemm_mx_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)gemm_mx_smem_bytes());
+  cudaError_t e = cudaFuncSetAttribute(moe_gemm_mx_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)gemm_mx_smem_bytes(false));
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(moe_gemm_mx_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)gemm_mx_smem_bytes());
+  e = cudaFuncSetAttribute(moe_gemm_mx_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)gemm_mx_smem_bytes(true));
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(moe_gemm_mx_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)gemm_mx_smem_bytes(true));
 }
 
 cudaError_t launch_moe_gemm_mx(const MxMaps& maps, const Workspace& ws, const MxBuffers& mx, const Shape& sh,
                                int grid, cudaStream_t stream) {
-  return launch_k(moe_gemm_mx_kernel<false>, dim3(grid), dim3(kGemmThreads), gemm_mx_smem_bytes(), stream, maps, ws,
-                  mx, sh, FrontArgs{});
+  if (sh.T <= kSmallRows)
+    return launch_k(moe_gemm_mx_kernel<false, true>, dim3(grid), dim3(kGemmThreads), gemm_mx_smem_bytes(true),
+                    stream, maps, ws, mx, sh, FrontArgs{});
+  return launch_k(moe_gemm_mx_kernel<false, false>, dim3(grid), dim3(kGemmThreads), gemm_mx_smem_bytes(false),
+                  stream, maps, ws, mx, sh, FrontArgs{});
 }
 
 cudaError_t launch_moe_mx_small_fused(const MxMaps& maps, const Workspace& ws, const MxBuffers& mx, const Shape& sh,
@@ -672,7 +686,7 @@ cudaError_t launch_moe_mx_small_fused(const MxMaps& maps, const Workspace& ws, c
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kGemmThreads);
-  cfg.dynamicSmemBytes = gemm_mx_smem_bytes();
+  cfg.dynamicSmemBytes = gemm_mx_smem_bytes(true);
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeCooperative;
@@ -681,13 +695,13 @@ cudaError_t launch_moe_mx_small_fused(const MxMaps& maps, const Workspace& ws, c
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, moe_gemm_mx_kernel<true>, maps, ws, mx, sh, fa);
+  return cudaLaunchKernelEx(&cfg, moe_gemm_mx_kernel<true, true>, maps, ws, mx, sh, fa);
 }
 
 int mx_small_fused_blocks_per_sm() {
   int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, moe_gemm_mx_kernel<true>, kGemmThreads,
-                                                    gemm_mx_smem_bytes()) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, moe_gemm_mx_kernel<true, true>, kGemmThreads,
+                                                    gemm_mx_smem_bytes(true)) != cudaSuccess) {
     cudaGetLastError();
     return 0;
   }
