@@ -656,27 +656,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
 }  // namespace
 
-size_t gemm_mx_smem_bytes(bool small) {
-  return (size_t)(small ? MxCfg<true>::kBytes : MxCfg<false>::kBytes) + 1024;
-}
+// dynamic shared memory of the general and of the small-batch configuration
+static size_t mx_smem_bytes(bool small) { return (size_t)(small ? MxCfg<true>::kBytes : MxCfg<false>::kBytes) + 1024; }
+
+size_t gemm_mx_smem_bytes() { return mx_smem_bytes(false); }
 
 cudaError_t configure_gemm_mx_kernel() {
   cudaError_t e = cudaFuncSetAttribute(moe_gemm_mx_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)gemm_mx_smem_bytes(false));
+                                       (int)mx_smem_bytes(false));
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(moe_gemm_mx_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)gemm_mx_smem_bytes(true));
+                           (int)mx_smem_bytes(true));
   if (e != cudaSuccess) return e;
   return cudaFuncSetAttribute(moe_gemm_mx_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)gemm_mx_smem_bytes(true));
+                              (int)mx_smem_bytes(true));
 }
 
 cudaError_t launch_moe_gemm_mx(const MxMaps& maps, const Workspace& ws, const MxBuffers& mx, const Shape& sh,
                                int grid, cudaStream_t stream) {
   if (sh.T <= kSmallRows)
-    return launch_k(moe_gemm_mx_kernel<false, true>, dim3(grid), dim3(kGemmThreads), gemm_mx_smem_bytes(true),
+    return launch_k(moe_gemm_mx_kernel<false, true>, dim3(grid), dim3(kGemmThreads), mx_smem_bytes(true),
                     stream, maps, ws, mx, sh, FrontArgs{});
-  return launch_k(moe_gemm_mx_kernel<false, false>, dim3(grid), dim3(kGemmThreads), gemm_mx_smem_bytes(false),
+  return launch_k(moe_gemm_mx_kernel<false, false>, dim3(grid), dim3(kGemmThreads), mx_smem_bytes(false),
                   stream, maps, ws, mx, sh, FrontArgs{});
 }
 
@@ -686,7 +687,7 @@ cudaError_t launch_moe_mx_small_fused(const MxMaps& maps, const Workspace& ws, c
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kGemmThreads);
-  cfg.dynamicSmemBytes = gemm_mx_smem_bytes(true);
+  cfg.dynamicSmemBytes = mx_smem_bytes(true);
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeCooperative;
@@ -701,7 +702,7 @@ cudaError_t launch_moe_mx_small_fused(const MxMaps& maps, const Workspace& ws, c
 int mx_small_fused_blocks_per_sm() {
   int n = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, moe_gemm_mx_kernel<true, true>, kGemmThreads,
-                                                    gemm_mx_smem_bytes(true)) != cudaSuccess) {
+                                                    mx_smem_bytes(true)) != cudaSuccess) {
     cudaGetLastError();
     return 0;
   }

@@ -174,7 +174,7 @@ cudaError_t launch_mx_quantize(const uint16_t* src, int64_t R, int K, uint8_t* q
 cudaError_t launch_mx_gather(const uint16_t* x, const Workspace& ws, const MxBuffers& mx, const Shape& sh,
                              bool token_order, int grid, cudaStream_t stream);
 
-size_t gemm_mx_smem_bytes(bool small);  // small: the ring of batches of at most 16 tokens
+size_t gemm_mx_smem_bytes();
 cudaError_t configure_gemm_mx_kernel();
 cudaError_t launch_moe_gemm_mx(const MxMaps& maps, const Workspace& ws, const MxBuffers& mx, const Shape& sh,
                                int grid, cudaStream_t stream);
