@@ -118,18 +118,70 @@ __device__ __forceinline__ int unit_start_of(int u, int Mr, int Mg, const Shape&
   return n1r * min(ups, Mr) + n1s * max(0, ups - Mr) + n2 * downs;
 }
 
-// Run by the CTA that finished its router slice last, once every slice is in. For a batch of
-// at most 16 tokens every expert receives at most 16 slots, so each hit expert has one m-tile
-// and one scheduling group, and the whole schedule fits one warp's scans:
+// The schedule of a fused forward, kept by every CTA in shared memory beside the operand ring:
+// the tiles (one per hit expert, in expert order, then the shared expert's), each slot's tile row
+// and router weight, and each routed tile row's slot.
+struct FusedSched {
+  int n_tiles, n_routed, n_units, n_tasks;
+  int slot_row[kSmallRows * kMaxTopK];  // tile row of slot s = t*k + j, -1 if dropped
+  float slot_w[kSmallRows * kMaxTopK];  // its router weight
+  int tile_exp[kFusedMaxExperts + 1];   // expert of tile g (E: the shared expert)
+  int tile_row0[kFusedMaxExperts + 1];  // its first sorted row (0 for the shared tile)
+  int tile_nrows[kFusedMaxExperts + 1];
+  int16_t row_slot[kFusedMaxExperts * kSmallRows];  // slot of row r of routed tile g, at g*16 + r
+};
+
+// CTA 0, before it arrives: this forward's counters start from zero. No CTA reads them before
+// every CTA has arrived, and the launch before this one has completed (griddepcontrol.wait).
+__device__ void front_reset(const Workspace& ws, const Shape& sh) {
+  const int mt_max = min(sh.E, sh.T * sh.k) + 1;
+  for (int i = threadIdx.x; i < mt_max; i += blockDim.x) {
+    ws.gather_done[i] = 0;
+    ws.done1[i] = 0;
+  }
+  for (int i = threadIdx.x; i < ceil_div(sh.H, kBN2); i += blockDim.x) ws.col_done[i] = 0;
+  if (threadIdx.x == 0) {
+    ws.meta->task_counter = 0;
+    ws.meta->abort = 0;
+    ws.meta->trace_count = 0;
+  }
+}
+
+// Thread 0: this CTA's router slice (and CTA 0's resets) are in; wait (bounded) until every CTA's
+// are. The counter only grows: forward `epoch` is complete when it reaches gridDim.x * epoch.
+__device__ bool front_arrive(const Workspace& ws, const FrontArgs& fa, DeviceMeta* meta, int64_t limit_ns) {
+  __threadfence();
+  int* cnt = &ws.front->front_done;
+  atomicAdd(cnt, 1);
+  const unsigned target = (unsigned)gridDim.x * (unsigned)fa.epoch;
+  auto done = [&](int v) { return (int)((unsigned)v - target) >= 0; };
+  if (done(ld_acquire_gpu(cnt))) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    __nanosleep(64);
+    if (done(ld_relaxed_gpu(cnt)) && done(ld_acquire_gpu(cnt))) return true;
+    if (static_cast<int64_t>(globaltimer_ns() - t0) > limit_ns) {
+      raise_error(meta, nullptr, kStatusTimeout | kSiteFront);
+      return false;
+    }
+  }
+}
+
+// Run by every CTA once every router slice is in (all threads). For a batch of at most 16 tokens
+// every expert receives at most 16 slots, so each hit expert has one m-tile and one scheduling
+// group, and the whole schedule fits one warp's scans:
 //  - gating (Weave blog section 1.1: top-k, ties to the lower expert index, softmax
-//    renormalised over the selection), from the logits staged in shared memory;
+//    renormalised over the selection);
 //  - the align (vLLM PR #53280 summary, implementation breakdown): per-expert counts, the
-//    capacity cut, padded segment offsets, the stable writes of sorted_ids in ascending slot
-//    order, the padding sentinels and expert_ids;
-//  - the tile and task schedule of the expert GEMMs: the same tables (tiles, groups, units with
-//    the dependency lag) that the align scans write for a larger batch;
-// then the reset of this forward's counters and the schedule flag. sm: shared scratch (ints).
-__device__ void front_schedule(const FrontArgs& fa, const Workspace& ws, const Shape& sh, int* sm, int64_t* ts) {
+//    capacity cut, padded segment offsets, each kept slot's rank (stable: ascending slot order);
+//  - the tile and task schedule of the expert GEMMs: one tile per hit expert, units with the
+//    dependency lag, as the align scans lay them out for a larger batch.
+// The result goes to `fs`. With `write_outputs` (CTA 0) the CTA also writes the layer's outputs
+// that nothing in this launch reads: top-k ids and weights, sorted_ids with its padding,
+// expert_ids, row_of_slot, the tile and group tables, the unit starts and the counts (the tests
+// compare them with the oracle). sm: shared scratch (ints) in the operand ring.
+__device__ void front_schedule(const FrontArgs& fa, const Workspace& ws, const Shape& sh, int* sm,
+                               FusedSched* fs, bool write_outputs, int64_t* ts) {
   // ts (thread 0, tracing): the end times of the steps, for the wait accounting
   const bool tracing = ws.trace_cap > 0;
   auto stamp = [&](int i) {
@@ -172,9 +224,12 @@ __device__ void front_schedule(const FrontArgs& fa, const Workspace& ws, const S
     for (int i = 0; i < kTokPerWarp; ++i) {
       const int t = warp + i * nw;
       if (t < T && lane < k) {
-        ws.topk_ids[t * k + lane] = id[i];
-        ws.topk_w[t * k + lane] = wt[i];
+        if (write_outputs) {
+          ws.topk_ids[t * k + lane] = id[i];
+          ws.topk_w[t * k + lane] = wt[i];
+        }
         ids_s[t * k + lane] = id[i];
+        fs->slot_w[t * k + lane] = wt[i];
         atomicAdd(&cnt[id[i]], 1);
         atomicOr(&tmask[id[i]], 1u << t);
       }
@@ -220,8 +275,39 @@ __device__ void front_schedule(const FrontArgs& fa, const Workspace& ws, const S
   }
   __syncthreads();
   stamp(2);
-  // every write of the schedule, spread over the CTA
+  // the schedule of this CTA: tiles, slot rows and weights, tile rows' slots
   const int P = off[E], Mt = s_mt[0], Mr = s_mt[1], Mg = Mt, U = Mt > 0 ? Mt + sh.lag : 0;
+  for (int e = tid; e < E; e += nthr) {
+    const int kp = kept[e];
+    if (kp > 0) {
+      const int t0 = tile0[e];
+      fs->tile_exp[t0] = e;
+      fs->tile_row0[t0] = off[e];
+      fs->tile_nrows[t0] = kp;
+    }
+  }
+  // slot s = t*k + j: its rank in its expert is the number of earlier tokens that chose it
+  for (int s = tid; s < S; s += nthr) {
+    const int t = s / k, e = ids_s[s];
+    const int r = __popc(tmask[e] & ((1u << t) - 1u));
+    const bool keep = sh.capacity == 0 || r < sh.capacity;
+    fs->slot_row[s] = keep ? tile0[e] * sh.tile_m + r : -1;
+    if (keep) fs->row_slot[tile0[e] * kSmallRows + r] = (int16_t)s;
+  }
+  if (tid == 0) {
+    if (sh.Ds > 0) {
+      fs->tile_exp[Mr] = E;
+      fs->tile_row0[Mr] = 0;
+      fs->tile_nrows[Mr] = T;
+    }
+    fs->n_tiles = Mt;
+    fs->n_routed = Mr;
+    fs->n_units = U;
+    fs->n_tasks = unit_start_of(U, Mr, Mg, sh);
+  }
+  stamp(3);
+  if (!write_outputs) return;
+  // CTA 0: the outputs that the tests and the debug calls read after the launch
   const int bm = sh.block_m;
   for (int e = tid; e < E; e += nthr) {
     const int o = off[e], kp = kept[e], t0 = tile0[e], end = off[e + 1];
@@ -237,8 +323,9 @@ __device__ void front_schedule(const FrontArgs& fa, const Workspace& ws, const S
       ws.group_ntiles[t0] = 1;
       ws.group_tasks[t0] = 1;
     }
+    for (int i = o + kp; i < end; ++i) ws.sorted_ids[i] = S;  // the segment's padding
+    for (int b = o / bm; b < end / bm; ++b) ws.expert_ids[b] = e;
   }
-  // slot s = t*k + j: its rank in its expert is the number of earlier tokens that chose it
   for (int s = tid; s < S; s += nthr) {
     const int t = s / k, e = ids_s[s];
     const int r = __popc(tmask[e] & ((1u << t) - 1u));
@@ -246,6 +333,9 @@ __device__ void front_schedule(const FrontArgs& fa, const Workspace& ws, const S
     if (keep) ws.sorted_ids[off[e] + r] = s;
     ws.row_of_slot[s] = keep ? tile0[e] * sh.tile_m + r : -1;
   }
+  for (int i = P + tid; i < sh.sorted_len; i += nthr) ws.sorted_ids[i] = S;
+  for (int b = P / bm + tid; b < sh.blocks_len; b += nthr) ws.expert_ids[b] = -1;
+  for (int u = tid; u <= U; u += nthr) ws.unit_start[u] = unit_start_of(u, Mr, Mg, sh);
   if (tid == 0) {
     ws.expert_off[E] = P;
     if (sh.Ds > 0) {
@@ -266,80 +356,33 @@ __device__ void front_schedule(const FrontArgs& fa, const Workspace& ws, const S
     m->num_routed_groups = Mr;
     m->num_units = U;
     m->total_tasks = unit_start_of(U, Mr, Mg, sh);
-    m->task_counter = 0;
-    m->abort = 0;
-    m->trace_count = 0;
   }
-  for (int i = tid; i < Mt; i += nthr) {
-    ws.gather_done[i] = 0;
-    ws.done1[i] = 0;
-  }
-  for (int i = tid; i < ceil_div(sh.H, kBN2); i += nthr) ws.col_done[i] = 0;
-  for (int u = tid; u <= U; u += nthr) ws.unit_start[u] = unit_start_of(u, Mr, Mg, sh);
-  // the task table: one m-tile per group here, so unit u's tasks are the up tasks of tile u, then
-  // the down tasks of tile u - lag (as write_unit_tasks lays them out); a tile's expert, first
-  // row and rows come from its expert's entries above (the shared tile: E, 0, T)
-  if (ws.task_tab) {
-    // tile -> expert: the routed tiles are the hit experts in expert order
-    int* t_exp = s_mt + 2;  // [Mt]
-    for (int e = tid; e < E; e += nthr)
-      if (kept[e] > 0) t_exp[tile0[e]] = e;
-    if (tid == 0 && sh.Ds > 0) t_exp[Mr] = E;
-    __syncthreads();
-    auto tile_info = [&](int g, int& ex, int& r0, int& nr) {
-      ex = t_exp[g];
-      r0 = ex == E ? 0 : off[ex];
-      nr = ex == E ? T : kept[ex];
-    };
-    for (int u = tid; u < U; u += nthr) {
-      int tau = unit_start_of(u, Mr, Mg, sh);
-      int ex, r0, nr;
-      if (u < Mt) {
-        tile_info(u, ex, r0, nr);
-        const int n1 = ceil_div(u < Mr ? sh.D : sh.Ds, kBN1);
-        for (int nt = 0; nt < n1; ++nt) ws.task_tab[tau++] = task_entry(kTaskUp, u, nt, 1, ex, r0, nr, 0);
-      }
-      const int g = u - sh.lag;
-      if (g >= 0 && g < Mt) {
-        tile_info(g, ex, r0, nr);
-        for (int nt = 0; nt < ceil_div(sh.H, kBN2); ++nt)
-          ws.task_tab[tau++] = task_entry(kTaskDown, g, nt, 1, ex, r0, nr, 0);
-      }
-    }
-  }
-  stamp(3);
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) {
-    ws.front->front_done = 0;  // every CTA has arrived: ready for the next forward
-    st_release_gpu(&ws.front->sched_flag, fa.epoch);
-  }
-  // the rest of the align outputs (the padding sentinels of sorted_ids and expert_ids), which
-  // nothing in this launch reads: after the schedule is out, before this CTA's own tasks
-  for (int e = tid; e < E; e += nthr) {
-    const int o = off[e], end = off[e + 1];
-    for (int i = o + kept[e]; i < end; ++i) ws.sorted_ids[i] = S;  // the segment's padding
-    for (int b = o / bm; b < end / bm; ++b) ws.expert_ids[b] = e;
-  }
-  for (int i = P + tid; i < sh.sorted_len; i += nthr) ws.sorted_ids[i] = S;
-  for (int b = P / bm + tid; b < sh.blocks_len; b += nthr) ws.expert_ids[b] = -1;
 }
 
-// Bounded wait (one thread) until the schedule of forward `epoch` is published. Only the time
-// limit ends it early: the abort flag may still hold an earlier forward's value until the
-// schedule resets it.
-__device__ bool wait_schedule(const int* flag, int epoch, DeviceMeta* meta, int64_t limit_ns) {
-  // relaxed polls, then one acquire load once the value is there
-  if (ld_acquire_gpu(flag) == epoch) return true;
-  const uint64_t t0 = globaltimer_ns();
-  while (true) {
-    __nanosleep(128);
-    if (ld_relaxed_gpu(flag) == epoch && ld_acquire_gpu(flag) == epoch) return true;
-    if (static_cast<int64_t>(globaltimer_ns() - t0) > limit_ns) {
-      raise_error(meta, nullptr, kStatusTimeout | kSiteFront);
-      return false;
-    }
+// Task `tau` of a fused forward, from the CTA's schedule: unit u (the last unit whose first id
+// is at most tau; empty units share their successor's first id) holds the up tasks of tile u,
+// then the down tasks of tile u - lag, as the align scans number them for a larger batch.
+__device__ __forceinline__ void fused_task(const FusedSched& fs, const Shape& sh, int tau, Task& t) {
+  const int Mt = fs.n_tiles, Mr = fs.n_routed;
+  int lo = 0, hi = fs.n_units - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (unit_start_of(mid, Mr, Mt, sh) <= tau) lo = mid;
+    else hi = mid - 1;
   }
+  const int off = tau - unit_start_of(lo, Mr, Mt, sh);
+  const int nup = lo < Mt ? ceil_div(lo < Mr ? sh.D : sh.Ds, kBN1) : 0;
+  const bool up = off < nup;
+  const int g = up ? lo : lo - sh.lag;
+  const int nt = up ? off : off - nup;
+  t.kind = up ? kTaskUp : kTaskDown;
+  t.tile = g;
+  t.expert = fs.tile_exp[g];
+  t.row0 = fs.tile_row0[g];
+  t.nrows = fs.tile_nrows[g];
+  t.ntiles = 1;
+  t.nrows2 = 0;
+  t.n0 = nt * (up ? kBN1 : kBN2);
 }
 
 // This CTA's share of the row gather: the x row of every kept slot s = blockIdx.x + j * gridDim.x

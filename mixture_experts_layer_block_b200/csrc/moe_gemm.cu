@@ -75,8 +75,9 @@ struct Cfg {
   static constexpr int kRingOff = kBarOff + ((kNumBars * 8 + 63) & ~63);
   static constexpr int kMiscOff = kRingOff + kTaskSlots * (int)sizeof(Task);
   // the fused small-batch forward keeps every slot's tile row (row_of_slot) in shared memory
-  static constexpr int kSlotRowsOff = kMiscOff + 64;
-  static constexpr int kBytes = kSlotRowsOff + (kShape == kShapeSmallFused ? kSmallRows * kMaxTopK * 4 : 0);
+  // the fused small-batch forward keeps its schedule (FusedSched) in shared memory
+  static constexpr int kFusedOff = kMiscOff + 64;
+  static constexpr int kBytes = kFusedOff + (kShape == kShapeSmallFused ? (int)((sizeof(FusedSched) + 15) & ~15) : 0);
   static_assert(kStageBytesN % 1024 == 0 && kABytesN % 1024 == 0 && kTailBytesN % 1024 == 0,
                 "1024-byte aligned operand tiles");
   static_assert(kBytes + 1024 <= 227 * 1024, "shared memory budget");
@@ -115,10 +116,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
   volatile int* s_epi_go = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 8);  // [2]
-  volatile int* s_front = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 16);  // fused: last / ok
+  volatile int* s_front = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 16);  // fused: ok
   volatile int* s_comb = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 24);   // fused: combine
-  int* s_slot_rows = reinterpret_cast<int*>(smem + C::kSlotRowsOff);                 // fused: [T*k]
-  int* s_tiles = reinterpret_cast<int*>(smem + C::kMiscOff + 32);  // fused: m-tiles, routed m-tiles
+  FusedSched* fs = reinterpret_cast<FusedSched*>(smem + C::kFusedOff);  // fused: the schedule
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   DeviceMeta* meta = ws.meta;
@@ -169,38 +169,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   bool run_tasks = true;
   const int64_t t_front = now();
   if constexpr (kFused) {
-    // the front, by all 192 threads; the operand ring is free until the first TMA fill
+    // the front, by all 192 threads; the operand ring is free until the first TMA fill. CTA 0
+    // resets the forward's counters, every CTA computes its router slice, then, once every
+    // slice is in, the whole schedule for itself (no CTA waits for another's tables)
     int* fsm = reinterpret_cast<int*>(smem);
+    if (blockIdx.x == 0) front_reset(ws, sh);
     front_router(fa, ws, sh, reinterpret_cast<float*>(fsm));
+    __syncthreads();
     const int64_t t_r = now();
-    if (threadIdx.x == 0) {
-      __threadfence();
-      s_front[0] = (atomicAdd(&ws.front->front_done, 1) == (int)gridDim.x - 1) ? 1 : 0;
-    }
+    if (threadIdx.x == 0) s_front[0] = front_arrive(ws, fa, meta, limit) ? 1 : 0;
     __syncthreads();
     int64_t ts[4] = {0, 0, 0, 0};
     const int64_t t_arrived = now();
-    if (s_front[0]) {
-      __threadfence();
-      front_schedule(fa, ws, sh, fsm, ts);
-      if (threadIdx.x == 0) s_front[1] = 1;
-    } else if (threadIdx.x == 0) {
-      s_front[1] = wait_schedule(&ws.front->sched_flag, fa.epoch, meta, limit) ? 1 : 0;
-      __threadfence();
-    }
-    __syncthreads();
-    const int64_t t_s = now();
-    run_tasks = s_front[1] != 0;
+    run_tasks = s_front[0] != 0;
     if (run_tasks) {
-      // every slot's tile row, for the gather and the combine
-      for (int i = threadIdx.x; i < sh.T * sh.k; i += blockDim.x) s_slot_rows[i] = __ldcg(ws.row_of_slot + i);
-      if (threadIdx.x == 0) {
-        s_tiles[0] = __ldcg(&meta->num_tiles);
-        s_tiles[1] = __ldcg(&meta->num_routed_tiles);
-      }
+      front_schedule(fa, ws, sh, fsm, fs, blockIdx.x == 0, ts);
       __syncthreads();
-      front_gather(fa, ws, sh, s_slot_rows);
     }
+    const int64_t t_s = now();
+    if (run_tasks) front_gather(fa, ws, sh, fs->slot_row);
     // the ring's generic-proxy writes come before the TMA fills that reuse it
     fence_proxy_async_shared();
     __syncthreads();
@@ -208,8 +195,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       wacc[kFrontRouter] = t_r - t_front;
       wacc[kFrontSchedule] = t_s - t_r;
       wacc[kFrontGather] = now() - t_s;
-      wacc[kFrontLast] = tracing ? s_front[0] : 0;
-      if (tracing && s_front[0]) {
+      wacc[kFrontLast] = tracing && blockIdx.x == 0 ? 1 : 0;
+      if (tracing) {
         wacc[kSchedArrive] = t_arrived - t_r;
         wacc[kSchedLogits] = ts[0] - t_arrived;
         wacc[kSchedGating] = ts[1] - ts[0];
@@ -224,7 +211,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // the schedule never came (bounded wait ran out): nothing was issued, go to the teardown
   } else if (warp == 0) {
     // ===================================== producer =====================================
-    const int total = __ldcg(&meta->total_tasks);
+    const int total = kFused ? fs->n_tasks : __ldcg(&meta->total_tasks);
     const int Mg = __ldcg(&meta->num_groups), Mgr = __ldcg(&meta->num_routed_groups);
     const int U = __ldcg(&meta->num_units);
     const int nk1 = ceil_div(sh.H, kBK);
@@ -255,7 +242,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       batch_end = next_tau + sh.claim_batch;
     }
     // with the task table, the claimed task's entry is loaded one stage after the claim
-    const bool use_tab = ws.task_tab != nullptr && !sh.static_quota;
+    const bool use_tab = ws.task_tab != nullptr && !sh.static_quota && !kFused;
     int4 next_ent = make_int4(0, 0, 0, 0);
     int ent_tau = -1;  // the claim whose entry next_ent holds
     const int64_t t_loop = now();
@@ -292,6 +279,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       t.nrows2 = 0;
       if (tau >= total) {
         t.kind = kTaskStop;
+      } else if (kFused) {
+        if (lane == 0) fused_task(*fs, sh, tau, t);
+        t.kind = __shfl_sync(0xffffffffu, t.kind, 0);
+        t.tile = __shfl_sync(0xffffffffu, t.tile, 0);
+        t.expert = __shfl_sync(0xffffffffu, t.expert, 0);
+        t.row0 = __shfl_sync(0xffffffffu, t.row0, 0);
+        t.nrows = __shfl_sync(0xffffffffu, t.nrows, 0);
+        t.n0 = __shfl_sync(0xffffffffu, t.n0, 0);
+        t.ntiles = 1;
+        t.nrows2 = 0;
+        t.nk = t.kind == kTaskUp ? nk1 : ceil_div(t.expert == sh.E ? sh.Ds : sh.D, kBK);
       } else if (use_tab) {
         int4 ent = next_ent;
         if (lane == 0 && ent_tau != tau) ent = __ldcg(ws.task_tab + tau);
@@ -628,6 +626,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (valid) {
             if (shared) {
               w = 1.f;
+            } else if constexpr (kFused) {
+              w = fs->slot_w[fs->row_slot[t.tile * kSmallRows + row]];
             } else {
               const int s = __ldcg(&ws.sorted_ids[t.row0 + row]);
               w = __ldcg(&ws.topk_w[s]);
@@ -668,14 +668,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const int64_t tc0 = now();
             named_bar_sync(1, 128);
             if (leader) {
-              const bool last = atom_add_acq_rel_gpu(&ws.col_done[t.n0 / kBN2], 1) == s_tiles[0] - 1;
+              const bool last = atom_add_acq_rel_gpu(&ws.col_done[t.n0 / kBN2], 1) == fs->n_tiles - 1;
               *s_comb = last ? 1 : 0;
             }
             named_bar_sync(1, 128);
             const int64_t tc1 = now();
             wacc[kCombineCount] += tc1 - tc0;
             if (*s_comb) {
-              fused_combine(fa, ws, sh, t.n0, (int)threadIdx.x - 64, s_tiles[1], s_slot_rows);
+              fused_combine(fa, ws, sh, t.n0, (int)threadIdx.x - 64, fs->n_routed, fs->slot_row);
               if (tracing) {
                 named_bar_sync(1, 128);  // the combine of every thread
                 wacc[kCombineRun] += now() - tc1;
@@ -835,12 +835,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 }
 
 size_t gemm_smem_bytes(int shape) {
-  const bool small = shape == kShapeSmall || shape == kShapeSmallFused;
-  return (size_t)(small ? Cfg<kShapeSmall>::kBytes
-                        : (shape == kShapeTail ? Cfg<kShapeTail>::kBytes
-                                               : (shape == kShapeTwo ? Cfg<kShapeTwo>::kBytes
-                                                                     : Cfg<kShapeGeneral>::kBytes))) +
-         1024;
+  // (the fused shape's layout is the small shape's plus its schedule)
+  const int bytes = shape == kShapeSmallFused ? Cfg<kShapeSmallFused>::kBytes
+                    : shape == kShapeSmall    ? Cfg<kShapeSmall>::kBytes
+                    : shape == kShapeTail     ? Cfg<kShapeTail>::kBytes
+                    : shape == kShapeTwo      ? Cfg<kShapeTwo>::kBytes
+                                              : Cfg<kShapeGeneral>::kBytes;
+  return (size_t)bytes + 1024;
 }
 
 cudaError_t launch_moe_gemm(const GemmMaps& maps, const Workspace& ws, const Shape& sh, int grid, int shape,

@@ -47,8 +47,9 @@ struct MxCfg {
   static constexpr int kRingOff = kBarOff + ((kNumBars * 8 + 63) & ~63);
   static constexpr int kMiscOff = kRingOff + kTaskSlots * (int)sizeof(Task);
   // the fused small-batch forward keeps every slot's tile row (row_of_slot) in shared memory
-  static constexpr int kSlotRowsOff = kMiscOff + 64;
-  static constexpr int kBytes = kSlotRowsOff + kSmallRows * kMaxTopK * 4;
+  // the fused small-batch forward keeps its schedule (FusedSched) in shared memory
+  static constexpr int kFusedOff = kMiscOff + 64;
+  static constexpr int kBytes = kFusedOff + (kSmall ? (int)((sizeof(FusedSched) + 15) & ~15) : 0);
   static constexpr uint32_t kSfCol0 = kAccCols;        // first TMEM column of the scale slots
   static constexpr uint32_t kSfColsPerStage = 16;
   static_assert(kStageBytes % 1024 == 0 && kSfOff % 1024 == 0, "1024-byte aligned operand tiles");
@@ -87,10 +88,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
   volatile int* s_epi_go = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 8);  // [2]
   // (misc + 16 .. + 39: the epilogue leader's wait sums)
-  volatile int* s_front = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 40);  // fused: last / ok
+  volatile int* s_front = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 40);  // fused: ok
   volatile int* s_comb = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 48);   // fused: combine
-  int* s_tiles = reinterpret_cast<int*>(smem + C::kMiscOff + 52);  // fused: m-tiles, routed m-tiles
-  int* s_slot_rows = reinterpret_cast<int*>(smem + C::kSlotRowsOff);                 // fused: [T*k]
+  FusedSched* fs = reinterpret_cast<FusedSched*>(smem + C::kFusedOff);  // fused: the schedule
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   DeviceMeta* meta = ws.meta;
@@ -145,35 +145,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // first TMA fill
     const int64_t t_front = now();
     int* fsm = reinterpret_cast<int*>(smem);
+    if (blockIdx.x == 0) front_reset(ws, sh);
     front_router(fa, ws, sh, reinterpret_cast<float*>(fsm));
+    __syncthreads();
     const int64_t t_r = now();
-    if (threadIdx.x == 0) {
-      __threadfence();
-      s_front[0] = (atomicAdd(&ws.front->front_done, 1) == (int)gridDim.x - 1) ? 1 : 0;
-    }
+    if (threadIdx.x == 0) s_front[0] = front_arrive(ws, fa, meta, limit) ? 1 : 0;
     __syncthreads();
     int64_t ts[4] = {0, 0, 0, 0};
     const int64_t t_arrived = now();
-    if (s_front[0]) {
-      __threadfence();
-      front_schedule(fa, ws, sh, fsm, ts);
-      if (threadIdx.x == 0) s_front[1] = 1;
-    } else if (threadIdx.x == 0) {
-      s_front[1] = wait_schedule(&ws.front->sched_flag, fa.epoch, meta, limit) ? 1 : 0;
-      __threadfence();
-    }
-    __syncthreads();
-    const int64_t t_s = now();
-    run_tasks = s_front[1] != 0;
+    run_tasks = s_front[0] != 0;
     if (run_tasks) {
-      for (int i = threadIdx.x; i < sh.T * sh.k; i += blockDim.x) s_slot_rows[i] = __ldcg(ws.row_of_slot + i);
-      if (threadIdx.x == 0) {
-        s_tiles[0] = __ldcg(&meta->num_tiles);
-        s_tiles[1] = __ldcg(&meta->num_routed_tiles);
-      }
+      front_schedule(fa, ws, sh, fsm, fs, blockIdx.x == 0, ts);
       __syncthreads();
-      front_gather_mx(fa, ws, mx, sh, s_slot_rows, s_tiles[1]);
     }
+    const int64_t t_s = now();
+    if (run_tasks) front_gather_mx(fa, ws, mx, sh, fs->slot_row, fs->n_routed);
     // the ring's generic-proxy writes come before the TMA fills that reuse it
     fence_proxy_async_shared();
     __syncthreads();
@@ -181,8 +167,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       add_wait(kFrontRouter, t_r - t_front);
       add_wait(kFrontSchedule, t_s - t_r);
       add_wait(kFrontGather, now() - t_s);
-      add_wait(kFrontLast, tracing ? s_front[0] : 0);
-      if (tracing && s_front[0]) {
+      add_wait(kFrontLast, tracing && blockIdx.x == 0 ? 1 : 0);
+      if (tracing) {
         add_wait(kSchedArrive, t_arrived - t_r);
         add_wait(kSchedLogits, ts[0] - t_arrived);
         add_wait(kSchedGating, ts[1] - ts[0]);
@@ -197,7 +183,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // the schedule never came (bounded wait ran out): nothing was issued, go to the teardown
   } else if (warp == 0) {
     // ===================================== producer =====================================
-    const int total = __ldcg(&meta->total_tasks);
+    const int total = kFused ? fs->n_tasks : __ldcg(&meta->total_tasks);
     const int Mg = __ldcg(&meta->num_groups), Mgr = __ldcg(&meta->num_routed_groups);
     const int U = __ldcg(&meta->num_units);
     const int H = sh.H;
@@ -212,7 +198,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       next_tau = atomicAdd(&meta->task_counter, sh.claim_batch);
       batch_end = next_tau + sh.claim_batch;
     }
-    const bool use_tab = ws.task_tab != nullptr;
+    const bool use_tab = ws.task_tab != nullptr && !kFused;
     int4 next_ent = make_int4(0, 0, 0, 0);
     int ent_tau = -1;
     const int64_t t_loop = now();
@@ -228,6 +214,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       t.nrows2 = 0;
       if (tau >= total) {
         t.kind = kTaskStop;
+      } else if (kFused) {
+        if (lane == 0) fused_task(*fs, sh, tau, t);
+        t.kind = __shfl_sync(0xffffffffu, t.kind, 0);
+        t.tile = __shfl_sync(0xffffffffu, t.tile, 0);
+        t.expert = __shfl_sync(0xffffffffu, t.expert, 0);
+        t.row0 = __shfl_sync(0xffffffffu, t.row0, 0);
+        t.nrows = __shfl_sync(0xffffffffu, t.nrows, 0);
+        t.n0 = __shfl_sync(0xffffffffu, t.n0, 0);
+        t.ntiles = 1;
+        t.nrows2 = 0;
+        t.nk = t.kind == kTaskUp ? H / kMxBK : (t.expert == sh.E ? sh.Ds : sh.D) / kMxBK;
       } else if (use_tab) {
         int4 ent = next_ent;
         if (lane == 0 && ent_tau != tau) ent = __ldcg(ws.task_tab + tau);
@@ -572,6 +569,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (row < t.nrows) {
           if (shared) {
             w = 1.f;
+          } else if constexpr (kFused) {
+            w = fs->slot_w[fs->row_slot[t.tile * kSmallRows + row]];
           } else {
             const int s = __ldcg(&ws.sorted_ids[t.row0 + row]);
             w = __ldcg(&ws.topk_w[s]);
@@ -612,12 +611,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const int64_t tc0 = now();
           if (leader) bulk_wait_group<0>();
           named_bar_sync(1, 128);
-          if (leader) *s_comb = atom_add_acq_rel_gpu(&ws.col_done[t.n0 / kBN2], 1) == s_tiles[0] - 1 ? 1 : 0;
+          if (leader) *s_comb = atom_add_acq_rel_gpu(&ws.col_done[t.n0 / kBN2], 1) == fs->n_tiles - 1 ? 1 : 0;
           named_bar_sync(1, 128);
           const int64_t tc1 = now();
           if (leader) add_wait(kCombineCount, tc1 - tc0);
           if (*s_comb) {
-            fused_combine(fa, ws, sh, t.n0, (int)threadIdx.x - 64, s_tiles[1], s_slot_rows);
+            fused_combine(fa, ws, sh, t.n0, (int)threadIdx.x - 64, fs->n_routed, fs->slot_row);
             if (tracing) {
               named_bar_sync(1, 128);
               if (leader) add_wait(kCombineRun, now() - tc1);
