@@ -92,15 +92,15 @@ extern "C" {
 #define MOE_FLAG_MXFP8        512u
 /* Batches of at most 16 tokens normally run as ONE launch (on devices that allow a cooperative
  * launch of one CTA per SM, and with E <= 256): every CTA computes the router logits of a slice
- * of the experts, the last one to finish takes the gating and the align and publishes the
- * schedule, every CTA gathers its share of the x rows, then all claim the expert-GEMM tasks, and
+ * of the experts; once every slice is in, every CTA computes the gating, the align and the task
+ * schedule for itself, gathers its share of the x rows, then all claim the expert-GEMM tasks, and
  * the CTA that finishes the last down task of a 256-column block combines that block for every
- * token (moe_query 11 reports 1 kernel). MOE_FLAG_UNFUSED_SMALL runs such batches as the six
- * separate kernels instead (for moe_forward and moe_forward_mxfp8). The fused router (fp32 on
- * the CUDA cores) sums each logit in
- * another order than the separate router kernel (fp32 on the tensor cores): logits and gating
- * weights differ in the last bits, and an exact near-tie may go the other way; both are
- * deterministic. */
+ * token (moe_query 11 reports 1 kernel). The align outputs (moe_debug_outputs) are written as
+ * for the separate kernels. MOE_FLAG_UNFUSED_SMALL runs such batches as the six separate kernels
+ * instead (for moe_forward and moe_forward_mxfp8). The fused router (fp32 on the CUDA cores) sums
+ * each logit in another order than the separate router kernel (fp32 on the tensor cores): logits
+ * and gating weights differ in the last bits, and an exact near-tie may go the other way; both
+ * are deterministic. */
 #define MOE_FLAG_UNFUSED_SMALL 1024u
 /* The one-SM expert GEMMs of batches of more than 16 tokens run every group of two m-tiles of one
  * expert as one task set: each task computes both tiles from the same weight stages into the two
