@@ -325,6 +325,9 @@ FUSED_CASES = {
                                                    block_m=16, D_shared=128, sigma_w=0.05),
     "many_experts_few_ctas": configs.MoEWorkload("many_experts_few_ctas", T=9, H=512, D=256, E=200, top_k=6,
                                                  block_m=16, sigma_w=0.05),
+    # the largest fused batch: 16 tokens x top-32 = 512 slots, every tile 16 rows, a shared expert
+    "max_slots": configs.MoEWorkload("max_slots", T=16, H=256, D=128, E=32, top_k=32, block_m=16,
+                                     D_shared=128, sigma_w=0.05),
 }
 
 

@@ -194,6 +194,9 @@ MX_FUSED = {
                                                 D_shared=256),  # the shared tile reads token-order xq
     "capacity_drops": configs.MoEWorkload("capacity_drops", T=9, H=384, D=256, E=6, top_k=2, block_m=16,
                                           sigma_w=0.05, capacity_factor=1.0),
+    # the largest fused batch: 16 tokens x top-32 = 512 slots, every tile 16 rows, a shared expert
+    "max_slots": configs.MoEWorkload("max_slots", T=16, H=256, D=128, E=32, top_k=32, block_m=16,
+                                     D_shared=128, sigma_w=0.05),
     # the router bias moves the hit experts from seed to seed
     "decode_seed1": MX_SMALL["decode"].replace(name="decode_seed1", seed=1),
     "decode_seed2": MX_SMALL["decode"].replace(name="decode_seed2", seed=2),
