@@ -66,11 +66,18 @@ MEASURED_TRAFFIC = {
 
 
 def kernel_source_hash() -> str:
+    """SHA-256 (first 16 hex digits) of the kernel sources with their comments and blank lines
+    left out: a comment edit keeps the measured traffic, a code edit drops it."""
     import hashlib
+    import re
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, f), encoding="utf-8") as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        code = "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+        h.update(code.encode("utf-8"))
     return h.hexdigest()[:16]
 
 
@@ -249,8 +256,9 @@ def wait_fractions(w: np.ndarray, names) -> dict:
 
 def front_timeline(w: np.ndarray, names) -> dict:
     """The fused small-batch forward's front in microseconds: the median CTA's router slice and
-    gather, the schedule's computation in the CTA that did it, the median wait for it, and the
-    median time from the front's start to the end of the epilogue loop."""
+    gather; the arrival plus the schedule in CTA 0 (which also writes the align outputs; its steps
+    are `schedule_steps`) and the median over the other CTAs; the median time from the front's
+    start to the end of the epilogue loop; the column-block counting and combines."""
     c = {n: w[:, i] for i, n in enumerate(names)}
     last = c["front_last"] == 1
     med = lambda v: float(np.median(v) / 1e3) if v.size else None

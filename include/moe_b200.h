@@ -348,12 +348,12 @@ MOE_API int moe_trace_read(moe_handle *h, int64_t *records, int64_t cap, int64_t
  *   5 MMA lane waiting for a free accumulator        6 MMA lane waiting for the next task
  *   7 epilogue waiting for the next task             8 epilogue waiting for a finished accumulator
  *   9 / 10 / 11 the producer / MMA / epilogue loop durations;
- * and for a fused small batch: 12 the CTA's router slice, 13 waiting for the schedule (or, in
- * the CTA that computed it, computing it), 14 its share of the row gather, 15 1 for the CTA that
- * computed the schedule, 16 from the start of the front to the end of the epilogue loop,
- * and in the CTA that computed the schedule its steps: 17 the arrival count, 18 loading the
- * logits, 19 gating, 20 the count / offset / tile / unit tables, 21 the writes of sorted_ids,
- * the sentinels, expert_ids and the task table, 22 publishing the schedule; 23 the barrier,
+ * and for a fused small batch: 12 the CTA's router slice, 13 the arrival and the CTA's own
+ * schedule, 14 its share of the row gather, 15 1 for CTA 0 (which also writes the align
+ * outputs), 16 from the start of the front to the end of the epilogue loop, the schedule's
+ * steps: 17 waiting for every CTA's router slice, 18 loading the logits, 19 gating, 20 the
+ * count / offset / tile / unit tables, 21 the CTA's schedule in shared memory, 22 (CTA 0) the
+ * align and tile outputs for the host; 23 the barrier,
  * fences and column-block counter after each fused down task, 24 the fused combines the CTA ran.
  * (25 per row.) Writes up to `rows` rows (at most one per SM) into the host buffer
  * `waits` and their number to *n_rows. The SM-pair and MXFP8 kernels leave zeros. */

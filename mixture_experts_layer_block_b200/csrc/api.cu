@@ -76,7 +76,7 @@ struct moe_handle {
   int last_kernels = 0;  // kernels launched by the last forward
   bool fused_ok = false;  // batches of <= 16 tokens may run as one fused launch on this device
   bool mx_fused_ok = false;  // the same for moe_forward_mxfp8
-  int32_t epoch = 0;      // fused forwards launched (the schedule flag's value of the last one)
+  int32_t epoch = 0;      // fused forwards launched (the arrival counter's target / grid size)
   int parts_rows = 0;  // rows of the K-split partial logits buffer
   std::vector<cudaEvent_t> ev;  // kTimingRing x (kNumStages + 1) events around the kernels
   int timed = 0;                // forwards recorded since the last moe_stage_times

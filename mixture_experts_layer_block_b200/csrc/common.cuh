@@ -61,7 +61,7 @@ enum WaitSite : int {
   kSiteEpiAcc = 8,
   kSiteDrain = 9,
   kSiteRouter = 10,
-  kSiteFront = 11,  // fused small-batch forward: the schedule was not published in time
+  kSiteFront = 11,  // fused small-batch forward: not every CTA arrived in time
 };
 
 // Counters and scalars that live in device memory (one int each).
@@ -81,14 +81,12 @@ struct DeviceMeta {
   int pad[4];
 };
 
-// The fused small-batch forward's two synchronisation words, each on a 128-byte line of its own
-// (the CTAs poll the flag while the scheduling CTA writes the DeviceMeta fields).
+// The fused small-batch forward's arrival counter, on a 128-byte line of its own: each CTA adds
+// 1 once its router slice is in, so forward n is complete when it reaches n times the grid size
+// (it is never reset).
 struct FrontSync {
-  int front_done;      // CTAs that finished their router slice
+  int front_done;
   int pad0[31];
-  int sched_flag;      // number of the last forward whose schedule is published (the CTAs wait
-                       // for their forward's number)
-  int pad1[31];
 };
 
 // Per-CTA wait accounting of the expert-GEMM kernel while tracing (ns of %globaltimer, summed
@@ -108,17 +106,17 @@ enum WaitKind : int {
   kWaitEpiLoop = 11,   // epilogue loop duration
   // the fused small-batch forward's front, per CTA (0 for the other kernels)
   kFrontRouter = 12,   // this CTA's router slice
-  kFrontSchedule = 13, // waiting for the schedule, or (the last CTA) computing it
+  kFrontSchedule = 13, // the arrival and this CTA's schedule
   kFrontGather = 14,   // this CTA's share of the row gather
-  kFrontLast = 15,     // 1 for the CTA that computed the schedule
+  kFrontLast = 15,     // 1 for CTA 0 (which also writes the align outputs)
   kFrontToEnd = 16,    // from the front's start to the end of the epilogue loop
-  // the scheduling CTA's steps (0 elsewhere)
-  kSchedArrive = 17,   // arrival count and CTA barrier
+  // the steps of this CTA's schedule
+  kSchedArrive = 17,   // waiting for every CTA's router slice
   kSchedLogits = 18,   // loading every token's logits
   kSchedGating = 19,   // top-k and softmax of every token
-  kSchedTables = 20,   // counts, offsets, tiles, groups and units (one warp)
-  kSchedWrites = 21,   // sorted_ids, sentinels, expert_ids, task table, counter resets
-  kSchedPublish = 22,  // memory fence, barrier and the flag
+  kSchedTables = 20,   // counts, offsets, tiles and units (one warp)
+  kSchedWrites = 21,   // the CTA's schedule in shared memory (slot rows and weights, tiles)
+  kSchedPublish = 22,  // CTA 0: the align and tile outputs for the host (0 elsewhere)
   // the fused forward's combine (epilogue leader, summed over this CTA's down tasks)
   kCombineCount = 23,  // barrier, fences and the column block's counter after each down task
   kCombineRun = 24,    // the combines this CTA ran (one per column block it completed)
@@ -195,7 +193,7 @@ struct FrontArgs {
   const float* bias;         // [E] fp32, or null
   void* out;                 // [T][H] fp32, or bf16 when out_bf16
   int32_t out_bf16;
-  int32_t epoch;             // this forward's number: the value of the published schedule flag
+  int32_t epoch;             // this forward's number (the arrival counter's target / grid size)
 };
 
 // Shapes and knobs of one forward, passed by value.

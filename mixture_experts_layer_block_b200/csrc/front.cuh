@@ -1,7 +1,7 @@
 // front.cuh -- device code of the fused small-batch forward (at most 16 tokens, one launch):
-// the front (router slices, gating and align by the last CTA to arrive, the schedule flag, the
-// row gather) and the combine that the task completing a column block runs. Used by the bf16
-// and the MXFP8 expert-GEMM kernels.
+// the front (router slices, the grid-wide arrival, every CTA's own gating, align and task
+// schedule, the row gather) and the combine that the task completing a column block runs. Used
+// by the bf16 and the MXFP8 expert-GEMM kernels.
 #pragma once
 
 #include "common.cuh"

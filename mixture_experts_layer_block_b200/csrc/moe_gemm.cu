@@ -859,7 +859,7 @@ cudaError_t launch_moe_gemm(const GemmMaps& maps, const Workspace& ws, const Sha
 
 cudaError_t launch_moe_small_fused(const GemmMaps& maps, const Workspace& ws, const Shape& sh,
                                    const FrontArgs& fa, int grid, cudaStream_t stream) {
-  // every CTA waits for the schedule that one of them publishes: all must be resident at once
+  // every CTA waits at the front's arrival for all the others: all must be resident at once
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kGemmThreads);

@@ -62,9 +62,9 @@ __device__ __forceinline__ int n1_of(int expert, const Shape& sh) {
   return ceil_div(expert == sh.E ? sh.Ds : sh.D, kBN1);
 }
 
-// kFused: the whole forward of at most 16 tokens in one launch (front.cuh): router slices, the
-// schedule from the last CTA to arrive, the MXFP8 row gather, then the tasks; the down task that
-// completes a 256-column block combines it.
+// kFused: the whole forward of at most 16 tokens in one launch (front.cuh): router slices, each
+// CTA's own schedule once every slice is in, the MXFP8 row gather, then the tasks; the down task
+// that completes a 256-column block combines it.
 template <bool kFused, bool kSmall>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     moe_gemm_mx_kernel(const __grid_constant__ MxMaps maps, Workspace ws, MxBuffers mx, Shape sh, FrontArgs fa) {
@@ -682,7 +682,7 @@ cudaError_t launch_moe_gemm_mx(const MxMaps& maps, const Workspace& ws, const Mx
 
 cudaError_t launch_moe_mx_small_fused(const MxMaps& maps, const Workspace& ws, const MxBuffers& mx, const Shape& sh,
                                       const FrontArgs& fa, int grid, cudaStream_t stream) {
-  // every CTA waits for the schedule that one of them publishes: all must be resident at once
+  // every CTA waits at the front's arrival for all the others: all must be resident at once
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kGemmThreads);
