@@ -316,7 +316,7 @@ int moe_init(const moe_config* cfg, moe_handle** out) {
       {(void**)&w.waits, (c.flags & MOE_FLAG_TRACE) ? (size_t)h->num_sms * kNumWaits * 8 : 0},
       {(void**)&w.task_tab, (size_t)h->max_tiles * n_task_max * sizeof(int4)},
       {(void**)&w.front, sizeof(FrontSync)},
-      {(void**)&w.col_done, (size_t)ceil_div(c.hidden, kBN2) * 4},
+      {(void**)&w.tok_done, (size_t)kSmallRows * ceil_div(c.hidden, kBN2) * 4},
       {(void**)&w.gather_done, (size_t)h->max_tiles * 4},
       {(void**)&h->x_stage, (c.flags & MOE_FLAG_HOST_STAGING) ? 2 * T_ * c.hidden * 2 : 0},
       {(void**)&h->out_stage, (c.flags & MOE_FLAG_HOST_STAGING) ? 2 * T_ * c.hidden * 4 : 0},

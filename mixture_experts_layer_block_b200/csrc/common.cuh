@@ -180,8 +180,9 @@ struct Workspace {
   int4* task_tab;        // [task_cap] every task of the forward, decoded (task_entry), or null
   int32_t task_cap;
   int64_t* waits;        // [grid][kNumWaits] per-CTA wait accounting while tracing, or null
-  int32_t* col_done;     // [ceil(H / kBN2)]  fused small-batch forward: down tasks finished per
-                         //                   256-column block (the last one combines the block)
+  int32_t* tok_done;     // [16][ceil(H / kBN2)] fused small-batch forward: a token's rows finished
+                         //   per 256-column block (the down task that finishes the last one
+                         //   combines that token's block)
   int32_t* gather_done;  // [max_tiles]       fused small-batch forward: x rows gathered per tile
 };
 

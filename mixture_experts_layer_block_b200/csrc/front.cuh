@@ -129,6 +129,8 @@ struct FusedSched {
   int tile_row0[kFusedMaxExperts + 1];  // its first sorted row (0 for the shared tile)
   int tile_nrows[kFusedMaxExperts + 1];
   int16_t row_slot[kFusedMaxExperts * kSmallRows];  // slot of row r of routed tile g, at g*16 + r
+  int tok_need[kSmallRows];             // rows of token t in y: its kept slots (+1 shared)
+  int comb_list[1 + kSmallRows];        // a down task's completed tokens (count, tokens)
 };
 
 // CTA 0, before it arrives: this forward's counters start from zero. No CTA reads them before
@@ -139,7 +141,7 @@ __device__ void front_reset(const Workspace& ws, const Shape& sh) {
     ws.gather_done[i] = 0;
     ws.done1[i] = 0;
   }
-  for (int i = threadIdx.x; i < ceil_div(sh.H, kBN2); i += blockDim.x) ws.col_done[i] = 0;
+  for (int i = threadIdx.x; i < sh.T * ceil_div(sh.H, kBN2); i += blockDim.x) ws.tok_done[i] = 0;
   if (threadIdx.x == 0) {
     ws.meta->task_counter = 0;
     ws.meta->abort = 0;
@@ -304,6 +306,25 @@ __device__ void front_schedule(const FrontArgs& fa, const Workspace& ws, const S
     fs->n_routed = Mr;
     fs->n_units = U;
     fs->n_tasks = unit_start_of(U, Mr, Mg, sh);
+    fs->comb_list[0] = 0;
+  }
+  // token t's rows in y: its kept slots, and its shared-expert row
+  for (int t = tid; t < T; t += nthr) {
+    int need = sh.Ds > 0 ? 1 : 0;
+    for (int j = 0; j < k; ++j) {
+      const int e = ids_s[t * k + j];
+      need += (sh.capacity == 0 || __popc(tmask[e] & ((1u << t) - 1u)) < sh.capacity) ? 1 : 0;
+    }
+    fs->tok_need[t] = need;
+    // a token without a row in y (every slot dropped, no shared expert): its output is zero,
+    // written here, since no down task completes it
+    if (need == 0 && write_outputs) {
+      for (int c = 0; c < sh.H; c += 8) {
+        const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (fa.out_bf16) store8<true>(fa.out, (size_t)t * sh.H + c, z);
+        else store8<false>(fa.out, (size_t)t * sh.H + c, z);
+      }
+    }
   }
   stamp(3);
   if (!write_outputs) return;
@@ -443,56 +464,63 @@ __device__ void front_gather_mx(const FrontArgs& fa, const Workspace& ws, const 
   }
 }
 
-// The combine of columns [n0, n0 + kBN2) for every token, once every down task of that column
-// block is done: out[t] = y[shared row of t] + sum_j y[row of slot t*k + j], in this order, in
-// fp32 (the standalone combine kernel's order, so the result is the same bit for bit). Thread
-// i < 128: token i / 8, the 8-column groups n0 + 8 (i % 8) + 64 v, v = 0..3 (the eight threads of
-// a token read 128 contiguous bytes of a row per load). slot_rows: every slot's tile row (-1:
-// dropped), in shared memory.
-__device__ void fused_combine(const FrontArgs& fa, const Workspace& ws, const Shape& sh, int n0, int i, int Mr,
-                              const int* slot_rows) {
-  const int t = i >> 3;
-  if (t >= sh.T) return;
-  const int cl = n0 + (i & 7) * 8;  // column of group v: cl + 64 v
-  float acc[4][8];
-#pragma unroll
-  for (int v = 0; v < 4; ++v)
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc[v][j] = 0.f;
-  // the rows in summation order: the shared expert's, then slots j = 0..k-1; their data is
-  // loaded kRound rows at a time (one round trip for top-8 without a shared expert)
-  constexpr int kRound = 8;
+// One token's combine of columns [c*kBN2, (c+1)*kBN2) by one warp, once all of that token's rows
+// of the block are in y: out[t] = y[shared row of t] + sum_j y[row of slot t*k + j], in this
+// order, in fp32 (the standalone combine kernel's order, so the result is the same bit for bit).
+// Lane l takes the 8 columns c*kBN2 + 8 l (the warp reads 512 contiguous bytes of a row per
+// load); the rows' loads go out 8 at a time.
+__device__ void combine_token_block(const FrontArgs& fa, const Workspace& ws, const Shape& sh, const FusedSched& fs,
+                                    int tok, int c, int lane) {
+  const int col = c * kBN2 + lane * 8;
+  if (col + 8 > sh.H) return;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   const int nr = (sh.Ds > 0 ? 1 : 0) + sh.k;
   auto row_of = [&](int j) {
     const int jj = sh.Ds > 0 ? j - 1 : j;
-    return jj < 0 ? (Mr + t / sh.tile_m) * sh.tile_m + t % sh.tile_m : slot_rows[t * sh.k + jj];
+    return jj < 0 ? (fs.n_routed + tok / sh.tile_m) * sh.tile_m + tok % sh.tile_m : fs.slot_row[tok * sh.k + jj];
   };
+  constexpr int kRound = 8;
   for (int j0 = 0; j0 < nr; j0 += kRound) {
-    uint4 d[kRound][4];
+    uint4 d[kRound];
     int rows[kRound];
 #pragma unroll
     for (int q = 0; q < kRound; ++q) {
       rows[q] = j0 + q < nr ? row_of(j0 + q) : -1;
-      const uint16_t* yr = ws.y + (size_t)(rows[q] >= 0 ? rows[q] : 0) * sh.H;
-#pragma unroll
-      for (int v = 0; v < 4; ++v)
-        d[q][v] = (rows[q] >= 0 && cl + 64 * v + 8 <= sh.H) ? __ldcg(reinterpret_cast<const uint4*>(yr + cl + 64 * v))
-                                                          : make_uint4(0, 0, 0, 0);
+      d[q] = rows[q] >= 0 ? __ldcg(reinterpret_cast<const uint4*>(ws.y + (size_t)rows[q] * sh.H + col))
+                          : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
-    for (int q = 0; q < kRound; ++q) {
-      if (rows[q] >= 0) {
-#pragma unroll
-        for (int v = 0; v < 4; ++v) add_bf16x8(acc[v], d[q][v]);
-      }
+    for (int q = 0; q < kRound; ++q)
+      if (rows[q] >= 0) add_bf16x8(acc, d[q]);
+  }
+  if (fa.out_bf16) store8<true>(fa.out, (size_t)tok * sh.H + col, acc);
+  else store8<false>(fa.out, (size_t)tok * sh.H + col, acc);
+}
+
+// After a fused down task's y stores (the 128 epilogue threads, warps 2-5; `row` is the thread's
+// tile row): each valid row adds 1 to its token's counter for the task's column block with one
+// acquire-release atomic (its release covers the thread's own row of y), and the row that
+// completes a token's block lists the token; then one warp per listed token combines it. A
+// token's block is combined as soon as its last row is in, not after the block's last task.
+// s_list: shared [1 + 16] (count, tokens), zero on entry. Returns the number of tokens combined.
+__device__ int fused_down_done(const FrontArgs& fa, const Workspace& ws, const Shape& sh, const FusedSched& fs,
+                                const Task& t, int row, volatile int* s_list, bool leader) {
+  const int nblk = ceil_div(sh.H, kBN2), c = t.n0 / kBN2;
+  named_bar_sync(1, 128);  // the previous task's list is cleared
+  if (row < t.nrows) {
+    const int tok = (t.expert == sh.E) ? t.row0 + row : fs.row_slot[t.tile * kSmallRows + row] / sh.k;
+    if (atom_add_acq_rel_gpu(&ws.tok_done[tok * nblk + c], 1) == fs.tok_need[tok] - 1) {
+      __threadfence();
+      s_list[1 + atomicAdd(const_cast<int*>(&s_list[0]), 1)] = tok;
     }
   }
-#pragma unroll
-  for (int v = 0; v < 4; ++v) {
-    if (cl + 64 * v + 8 > sh.H) continue;
-    if (fa.out_bf16) store8<true>(fa.out, (size_t)t * sh.H + cl + 64 * v, acc[v]);
-    else store8<false>(fa.out, (size_t)t * sh.H + cl + 64 * v, acc[v]);
-  }
+  named_bar_sync(1, 128);
+  const int n = s_list[0];
+  for (int i = ((int)threadIdx.x >> 5) - 2; i < n; i += 4)
+    combine_token_block(fa, ws, sh, fs, s_list[1 + i], c, (int)threadIdx.x & 31);
+  named_bar_sync(1, 128);
+  if (leader) s_list[0] = 0;
+  return n;
 }
 
 }  // namespace

@@ -117,7 +117,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
   volatile int* s_epi_go = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 8);  // [2]
   volatile int* s_front = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 16);  // fused: ok
-  volatile int* s_comb = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 24);   // fused: combine
   FusedSched* fs = reinterpret_cast<FusedSched*>(smem + C::kFusedOff);  // fused: the schedule
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -661,26 +660,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&acc_empty[next]);
           if constexpr (kFused) {
-            // count this task's column block; the task that completes a block combines it. The
-            // barrier orders every epilogue thread's y stores before the leader's acquire-release
-            // add (its release is cumulative over the barrier; its acquire orders the other tasks'
-            // rows before the barrier that lets this task's threads read them).
+            // count this task's rows per token; the row that completes a token's column block
+            // has that token's block combined by one epilogue warp
             const int64_t tc0 = now();
-            named_bar_sync(1, 128);
-            if (leader) {
-              const bool last = atom_add_acq_rel_gpu(&ws.col_done[t.n0 / kBN2], 1) == fs->n_tiles - 1;
-              *s_comb = last ? 1 : 0;
-            }
-            named_bar_sync(1, 128);
-            const int64_t tc1 = now();
-            wacc[kCombineCount] += tc1 - tc0;
-            if (*s_comb) {
-              fused_combine(fa, ws, sh, t.n0, (int)threadIdx.x - 64, fs->n_routed, fs->slot_row);
-              if (tracing) {
-                named_bar_sync(1, 128);  // the combine of every thread
-                wacc[kCombineRun] += now() - tc1;
-              }
-            }
+            const int n = fused_down_done(fa, ws, sh, *fs, t, row, fs->comb_list, leader);
+            const int64_t dt = now() - tc0;
+            wacc[kCombineCount] += dt;
+            if (n > 0) wacc[kCombineRun] += dt;
           }
         }
         if (lane == 0) mbar_arrive(&task_empty[slot]);

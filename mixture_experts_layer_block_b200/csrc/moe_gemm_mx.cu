@@ -89,7 +89,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   volatile int* s_epi_go = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 8);  // [2]
   // (misc + 16 .. + 39: the epilogue leader's wait sums)
   volatile int* s_front = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 40);  // fused: ok
-  volatile int* s_comb = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 48);   // fused: combine
   FusedSched* fs = reinterpret_cast<FusedSched*>(smem + C::kFusedOff);  // fused: the schedule
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -605,22 +604,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           release_acc();
         }
         if constexpr (kFused) {
-          // count this task's column block; the task that completes a block combines it (the
-          // barrier orders every epilogue thread's y stores -- and the leader's TMA stores, once
-          // complete -- before the leader's acquire-release add)
+          // count this task's rows per token (every fused tile is partial: each thread stored its
+          // own row straight from registers); the row that completes a token's column block has
+          // that token's block combined by one epilogue warp
           const int64_t tc0 = now();
-          if (leader) bulk_wait_group<0>();
-          named_bar_sync(1, 128);
-          if (leader) *s_comb = atom_add_acq_rel_gpu(&ws.col_done[t.n0 / kBN2], 1) == fs->n_tiles - 1 ? 1 : 0;
-          named_bar_sync(1, 128);
-          const int64_t tc1 = now();
-          if (leader) add_wait(kCombineCount, tc1 - tc0);
-          if (*s_comb) {
-            fused_combine(fa, ws, sh, t.n0, (int)threadIdx.x - 64, fs->n_routed, fs->slot_row);
-            if (tracing) {
-              named_bar_sync(1, 128);
-              if (leader) add_wait(kCombineRun, now() - tc1);
-            }
+          const int n = fused_down_done(fa, ws, sh, *fs, t, row, fs->comb_list, leader);
+          const int64_t dt = now() - tc0;
+          if (leader) {
+            add_wait(kCombineCount, dt);
+            if (n > 0) add_wait(kCombineRun, dt);
           }
         }
       }
