@@ -55,13 +55,13 @@ KERNEL_SOURCES = ["mixture_experts_layer_block_b200/csrc/moe_gemm.cu",
                   "mixture_experts_layer_block_b200/csrc/ptx.cuh",
                   "mixture_experts_layer_block_b200/csrc/launch.h"]
 MEASURED_TRAFFIC = {
-    "flashmoe_prefill": ("92f7da763527f0bd", 1.680044e9 + 0.062322e9, "one full-size launch"),
+    "flashmoe_prefill": ("f7bab268de21caa7", 1.679793e9 + 0.059929e9, "one full-size launch"),
     # at most 16 tokens the forward is one launch: its traffic covers the router, gather and combine
-    "decode": ("92f7da763527f0bd", 0.338452e9 + 0.003861e9, "one full-size launch of the fused forward"),
+    "decode": ("f7bab268de21caa7", 0.338417e9 + 0.004369e9, "one full-size launch of the fused forward"),
     # full DSV3 holds 22.6 GB of weights, too large for a multi-pass capture: the T=512, E=32
     # case of the same layer (the same per-expert load, 1/8 of the experts and tokens) scaled
     # by the 8x more units of a full launch
-    "dsv3": ("92f7da763527f0bd", 8 * (3.040076e9 + 0.113133e9), "T=512, E=32 capture x 8"),
+    "dsv3": ("f7bab268de21caa7", 8 * (3.035066e9 + 0.113653e9), "T=512, E=32 capture x 8"),
 }
 
 
