@@ -94,8 +94,8 @@ extern "C" {
  * launch of one CTA per SM, and with E <= 256): every CTA computes the router logits of a slice
  * of the experts; once every slice is in, every CTA computes the gating, the align and the task
  * schedule for itself, gathers its share of the x rows, then all claim the expert-GEMM tasks, and
- * the CTA that finishes the last down task of a 256-column block combines that block for every
- * token (moe_query 11 reports 1 kernel). The align outputs (moe_debug_outputs) are written as
+ * the down task that brings in a token's last row of a 256-column block combines that token's
+ * block (moe_query 11 reports 1 kernel). The align outputs (moe_debug_outputs) are written as
  * for the separate kernels. MOE_FLAG_UNFUSED_SMALL runs such batches as the six separate kernels
  * instead (for moe_forward and moe_forward_mxfp8). The fused router (fp32 on the CUDA cores) sums
  * each logit in another order than the separate router kernel (fp32 on the tensor cores): logits
@@ -354,7 +354,8 @@ MOE_API int moe_trace_read(moe_handle *h, int64_t *records, int64_t cap, int64_t
  * steps: 17 waiting for every CTA's router slice, 18 loading the logits, 19 gating, 20 the
  * count / offset / tile / unit tables, 21 the CTA's schedule in shared memory, 22 (CTA 0) the
  * align and tile outputs for the host; 23 the barrier,
- * fences and column-block counter after each fused down task, 24 the fused combines the CTA ran.
+ * per-token counters and combines after each fused down task, 24 the same for the tasks that
+ * combined at least one token.
  * (25 per row.) Writes up to `rows` rows (at most one per SM) into the host buffer
  * `waits` and their number to *n_rows. The SM-pair and MXFP8 kernels leave zeros. */
 MOE_API int moe_trace_waits(moe_handle *h, int64_t *waits, int32_t rows, int32_t *n_rows);

@@ -118,8 +118,8 @@ enum WaitKind : int {
   kSchedWrites = 21,   // the CTA's schedule in shared memory (slot rows and weights, tiles)
   kSchedPublish = 22,  // CTA 0: the align and tile outputs for the host (0 elsewhere)
   // the fused forward's combine (epilogue leader, summed over this CTA's down tasks)
-  kCombineCount = 23,  // barrier, fences and the column block's counter after each down task
-  kCombineRun = 24,    // the combines this CTA ran (one per column block it completed)
+  kCombineCount = 23,  // the per-token counters and combines after each down task
+  kCombineRun = 24,    // the same, for the down tasks that combined at least one token
   kNumWaits = 25,
 };
 

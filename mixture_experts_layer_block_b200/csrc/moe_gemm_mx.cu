@@ -64,7 +64,7 @@ __device__ __forceinline__ int n1_of(int expert, const Shape& sh) {
 
 // kFused: the whole forward of at most 16 tokens in one launch (front.cuh): router slices, each
 // CTA's own schedule once every slice is in, the MXFP8 row gather, then the tasks; the down task
-// that completes a 256-column block combines it.
+// that brings in a token's last row of a 256-column block combines that token's block.
 template <bool kFused, bool kSmall>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     moe_gemm_mx_kernel(const __grid_constant__ MxMaps maps, Workspace ws, MxBuffers mx, Shape sh, FrontArgs fa) {
