@@ -120,3 +120,23 @@ def test_wait_fractions_and_front_timeline():
     assert fr["schedule_steps"]["gating"] == pytest.approx(4.0)
     assert fr["combine_count"] == pytest.approx(2.5) and fr["combine_run"] == pytest.approx(6.0)
     assert fr["combining_ctas"] == 2
+
+
+def test_kernel_source_hash_ignores_comments_only(tmp_path, monkeypatch):
+    """The traffic figures stay tied to the kernel code: a comment edit keeps the hash, a code edit
+    changes it (and bench.py then reports the traffic as null)."""
+    import shutil
+    for f in bench.KERNEL_SOURCES:
+        dst = tmp_path / f
+        dst.parent.mkdir(parents=True, exist_ok=True)
+        shutil.copy(os.path.join(bench.ROOT, f), dst)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    base = bench.kernel_source_hash()
+    target = tmp_path / bench.KERNEL_SOURCES[0]
+    text = target.read_text()
+    target.write_text(text + "\n// a note\n/* a block\n   comment */\n\n")
+    assert bench.kernel_source_hash() == base
+    target.write_text(text + "\nstatic int moe_extra_symbol = 1;\n")
+    assert bench.kernel_source_hash() != base
+    for w, rec in bench.MEASURED_TRAFFIC.items():
+        assert bench.measured_traffic(w) is None
